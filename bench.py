@@ -1,0 +1,475 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 weight-only quantized linear layer (int4 nested superscale).
+
+Headline: int4 decode GEMV at M=1 in GB/s of algorithmic bytes (packed codes +
+group metadata + step words + x + y) and its fraction of the measured HBM
+peak; alongside it, the int4 prefill GEMM at M=2048 in TFLOP/s against the
+measured dense bf16 peak.
+
+One timed step = one decode token through two layers of the int4 decode
+workload -- (K=5120, N=27648) then (K=27648, N=5120), M=1 -- each a single
+qlinear_gemv launch.  Three packed copies of each layer are rotated so that a
+weight copy is touched only once per 491 MB of traffic (> 3x the 126 MB L2).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Under torchrun (N > 1) every rank runs the same per-GPU workload on its own
+GPU (an independent row partition of a wider layer: no data-path
+collective); time is the max over ranks; rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+METRIC = "int4 qmv GEMV GB/s & % HBM peak (M=1); qmm GEMM TFLOP/s at M=2048"
+LAYERS = [(5120, 27648), (27648, 5120)]  # (K, N) of the two decode layers
+GEMM_M, GEMM_K, GEMM_N = 2048, 5120, 27648
+COPIES = 3
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# DRAM bytes per GEMV launch from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum),
+# valid only while the GEMV source is unchanged (hash of csrc/gemv.cuh at capture time).
+NCU_TRAFFIC = {"gemv_src_sha256": None, "bytes_per_launch": None}
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--gemm-iters", type=int, default=10)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args(argv)
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (also exercised by a 2-rank gloo test on CPU)
+# ---------------------------------------------------------------------------
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def dist_init(backend: str):
+    import torch.distributed as dist
+    rank, world, _ = dist_env()
+    if world > 1 and not dist.is_initialized():
+        import datetime
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return rank, world
+
+
+def reduce_scalar(x: float, op: str, device=None) -> float:
+    """max/sum of a float over ranks (identity when not distributed)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def aggregate(units_this_rank: float, seconds_this_rank: float, device=None):
+    """Whole-job throughput: units summed over ranks / max time over ranks."""
+    total = reduce_scalar(units_this_rank, "sum", device)
+    tmax = reduce_scalar(seconds_this_rank, "max", device)
+    return total, tmax, total / tmax
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled while the GPU is under load
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.windows = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+            return
+        threading.Thread(target=self._read, daemon=True).start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def mark(self, t0: float, t1: float):
+        self.windows.append((t0, t1))
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons, n = [], None, set(), 0
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ts, line in self.lines:
+            if not any(a - 0.05 <= ts <= b + 0.05 for a, b in self.windows):
+                continue
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            n += 1
+            for name, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": n}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return dict(FALLBACK_PEAKS, source="fallback")
+
+
+def gemv_bytes(K: int, N: int, M: int = 1) -> int:
+    """Algorithmic bytes of one int4 GEMV: packed codes + group words + step words + x + y."""
+    return N * K // 2 + N * (K // 32) * 2 + N * (K // 256) * 4 + M * K * 2 + M * N * 2
+
+
+def gemv_src_sha():
+    with open(os.path.join(ROOT, "int6_quantized_linear_b200", "csrc", "gemv.cuh"), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()
+
+
+# ---------------------------------------------------------------------------
+# native (CUDA) arm
+# ---------------------------------------------------------------------------
+
+def build_layers(device, copies=COPIES):
+    import torch
+
+    import int6_quantized_linear_b200 as ql
+    from int6_quantized_linear_b200 import synth
+
+    layers = []
+    for li, (K, N) in enumerate(LAYERS):
+        d = ql.Desc("int4", N, K)
+        w = synth.int4_weights(1, N, K)
+        dev = lambda a: torch.from_numpy(a.view("int16") if a.itemsize == 2 else a).to(device)
+        q, sc, zc, ss, zs = (dev(w[k]) for k in ("q", "sc", "zc", "ss", "zs"))
+        c0, g0, s0 = ql.alloc_packed(d, device)
+        ql.qlinear_pack(d, q, sc, zc, ss, zs, c0, g0, s0)
+        del q, sc, zc, ss, zs
+        reps = [(c0, g0, s0)] + [(c0.clone(), g0.clone(), s0.clone()) for _ in range(copies - 1)]
+        x = torch.from_numpy(synth.activations(1, 1, K).view("int16")).to(device).view(torch.bfloat16)
+        y = torch.empty((1, N), dtype=torch.bfloat16, device=device)
+        layers.append(dict(desc=d, reps=reps, x=x, y=y, K=K, N=N))
+    torch.cuda.synchronize(device)
+    return layers
+
+
+def gemv_step(layers, i: int, ql, events=None):
+    for L in layers:
+        c, g, s = L["reps"][i % len(L["reps"])]
+        if events is not None:
+            events[0].append(_ev())
+            events[0][-1].record()
+        ql.qlinear_gemv(L["desc"], c, g, s, L["x"], 1, L["y"])
+        if events is not None:
+            events[1].append(_ev())
+            events[1][-1].record()
+
+
+def _ev():
+    import torch
+    return torch.cuda.Event(enable_timing=True)
+
+
+def run_native(args):
+    import torch
+
+    import int6_quantized_linear_b200 as ql
+
+    rank, world = dist_init("nccl")
+    _, _, local_rank = dist_env()
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    peaks = load_peaks()
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+
+    layers = build_layers(device)
+    step_bytes = sum(gemv_bytes(L["K"], L["N"]) for L in layers)
+
+    # warm-up, then exactly K timed steps between barrier + synchronize
+    for i in range(args.warmup):
+        gemv_step(layers, i, ql)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    launch_ev = ([], [])
+    t_wall0 = time.time()
+    ev0, ev1 = _ev(), _ev()
+    ev0.record()
+    for i in range(args.steps):
+        gemv_step(layers, i, ql, launch_ev)
+    ev1.record()
+    torch.cuda.synchronize(device)
+    t_wall1 = time.time()
+    barrier(device)
+    sampler.mark(t_wall0, t_wall1)
+    assert ql.qlinear_sync_status() == ql.QL_OK
+    elapsed_s = ev0.elapsed_time(ev1) / 1e3
+    launch_ms = [a.elapsed_time(b) for a, b in zip(*launch_ev)]
+
+    # keep the same load running for ~1.5 s so the clock sampler sees it
+    t_a = time.time()
+    i = 0
+    while time.time() - t_a < 1.5:
+        gemv_step(layers, i, ql)
+        i += 1
+        if i % 200 == 0:
+            torch.cuda.synchronize(device)
+    torch.cuda.synchronize(device)
+    sampler.mark(t_a, time.time())
+
+    total_bytes, tmax, value_bps = aggregate(step_bytes * args.steps, elapsed_s, device)
+    ms_per_step = tmax / args.steps * 1e3
+
+    # roofline of the dominant kernel (the GEMV): algorithmic bytes per launch / mean launch time
+    mean_launch_s = statistics.fmean(launch_ms) / 1e3
+    bytes_per_launch = step_bytes / len(layers)
+    achieved_gbs = bytes_per_launch / mean_launch_s / 1e9
+    traffic = (NCU_TRAFFIC["bytes_per_launch"]
+               if NCU_TRAFFIC["gemv_src_sha256"] == gemv_src_sha() else None)
+
+    gemm = run_gemm(args, device, peaks, sampler)
+    e2e = run_e2e(args, layers, device, step_bytes)
+    for L in layers:
+        L["reps"].clear()
+    clocks = sampler.stop()
+
+    if rank != 0:
+        return None
+    line = {
+        "metric": METRIC,
+        "value": round(value_bps / 1e9, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "int4 weights, bf16 activations, fp32 accumulate",
+        "data": "synthetic (seeded uniform codes/metadata per the workload recipe; x ~ N(0,1) in bf16)",
+        "config": {"workload": "int4 nested-superscale decode GEMV, M=1, layers (K=5120,N=27648) and "
+                               "(K=27648,N=5120)", "M": 1, "layers": LAYERS,
+                   "parallelism": f"{world} independent row partitions" if world > 1 else "single GPU",
+                   "l2": f"{COPIES} rotating packed copies per layer "
+                         f"({COPIES * step_bytes / 1e6:.0f} MB per rotation > 3x 126 MB L2)"},
+        "pct_hbm_peak": round(100 * value_bps / 1e9 / peaks["hbm_gbs"], 2),
+        "roofline": {"bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": round(achieved_gbs / peaks["hbm_gbs"], 4), "traffic": traffic,
+                     "peak_source": f"{peaks['source']} (copy bandwidth)", "kernel": "qlinear_gemv (int4)",
+                     "bytes_per_launch": bytes_per_launch, "mean_launch_us": round(mean_launch_s * 1e6, 3)},
+        "gemm_m2048": gemm,
+        "e2e": e2e,
+        "gpu_launches": len(launch_ms),
+        "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
+        "clock_samples": clocks["samples"],
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline()
+    return line
+
+
+def run_gemm(args, device, peaks, sampler):
+    """qlinear_gemm on the int4 prefill workload at M=2048 (K=5120, N=27648)."""
+    import torch
+
+    import int6_quantized_linear_b200 as ql
+    from int6_quantized_linear_b200 import synth
+
+    d = ql.Desc("int4", GEMM_N, GEMM_K)
+    w = synth.int4_weights(3, GEMM_N, GEMM_K)
+    t16 = lambda a: torch.from_numpy(a.view("int16") if a.itemsize == 2 else a).to(device)
+    c, g, s = ql.alloc_packed(d, device)
+    ql.qlinear_pack(d, t16(w["q"]), t16(w["sc"]), t16(w["zc"]), t16(w["ss"]), t16(w["zs"]), c, g, s)
+    x = t16(synth.activations(3, GEMM_M, GEMM_K)).view(torch.bfloat16)
+    y = torch.empty((GEMM_M, GEMM_N), dtype=torch.bfloat16, device=device)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
+    for _ in range(3):
+        ql.qlinear_gemm(d, c, g, s, x, GEMM_M, y)
+    torch.cuda.synchronize(device)
+    times = []
+    t0 = time.time()
+    for _ in range(args.gemm_iters):
+        flush.fill_(1)  # write > L2 between timed calls
+        a, b = _ev(), _ev()
+        a.record()
+        ql.qlinear_gemm(d, c, g, s, x, GEMM_M, y)
+        b.record()
+        torch.cuda.synchronize(device)
+        times.append(a.elapsed_time(b) / 1e3)
+    sampler.mark(t0, time.time())
+    assert ql.qlinear_sync_status() == ql.QL_OK
+    flops = 2.0 * GEMM_M * GEMM_N * GEMM_K
+    tmed = statistics.median(times)
+    tmax = reduce_scalar(tmed, "max", device)
+    tflops = flops / tmax / 1e12
+    del flush, x, y, c, g, s
+    return {"value": round(tflops, 1), "unit": "TFLOP/s", "ms": round(tmax * 1e3, 4), "M": GEMM_M,
+            "K": GEMM_K, "N": GEMM_N, "iters": args.gemm_iters,
+            "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": peaks["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": round(tflops / peaks["bf16_tflops"], 4),
+                         "peak_source": f"{peaks['source']} dense bf16 (burst)"},
+            "l2": "256 MiB buffer written between timed calls"}
+
+
+def run_e2e(args, layers, device, step_bytes):
+    """Same metric through the public API with host buffers: every step copies x from pinned host
+    memory to the device and reads y back, inside the timed region."""
+    import torch
+
+    import int6_quantized_linear_b200 as ql
+
+    xh = [L["x"].cpu().pin_memory() for L in layers]
+    yh = [torch.empty(L["y"].shape, dtype=torch.bfloat16).pin_memory() for L in layers]
+    h2d = sum(x.numel() * 2 for x in xh)
+    d2h = sum(y.numel() * 2 for y in yh)
+
+    def step(i):
+        for L, xhost, yhost in zip(layers, xh, yh):
+            c, g, s = L["reps"][i % len(L["reps"])]
+            L["x"].copy_(xhost, non_blocking=True)
+            ql.qlinear_gemv(L["desc"], c, g, s, L["x"], 1, L["y"])
+            yhost.copy_(L["y"], non_blocking=True)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    a, b = _ev(), _ev()
+    a.record()
+    for i in range(args.steps):
+        step(i)
+    b.record()
+    torch.cuda.synchronize(device)
+    barrier(device)
+    _, tmax, v = aggregate(step_bytes * args.steps, a.elapsed_time(b) / 1e3, device)
+    return {"value": round(v / 1e9, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": round(tmax / args.steps * 1e3, 5)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle: the baseline leg and the reference arm
+# ---------------------------------------------------------------------------
+
+def _oracle_sample_step(rows_per_layer: int):
+    """One oracle pass: dequantise a sample of rows of each decode layer and multiply in fp64.
+    Returns (algorithmic bytes covered, seconds)."""
+    from int6_quantized_linear_b200 import synth
+    from oracle import oracle_c as OC
+
+    total_bytes, total_s = 0, 0.0
+    for (K, N) in LAYERS:
+        n = min(N, rows_per_layer)
+        w = synth.int4_weights(1, n, K)  # same recipe; a leading block of rows
+        x = synth.activations(1, 1, K)
+        packed = OC.int4_pack(w["q"], w["sc"], w["zc"], w["ss"], w["zs"])
+        t0 = time.perf_counter()
+        wf = OC.int4_dequant(*packed)
+        OC.matmul_f64(x, wf)
+        total_s += time.perf_counter() - t0
+        total_bytes += gemv_bytes(K, n)
+    return total_bytes, total_s
+
+
+def cpu_baseline(rows_per_layer: int = 2048) -> dict:
+    from oracle import oracle_c as OC
+    b, s = _oracle_sample_step(rows_per_layer)
+    return {"value": round(b / s / 1e9, 4), "unit": "GB/s", "cores": OC.num_threads(), "kind": "oracle",
+            "sample": f"first {rows_per_layer} rows of each decode layer, M=1: C oracle fp32 dequant + "
+                      f"fp64 matmul ({b / 1e6:.1f} MB of algorithmic bytes in {s:.2f} s)"}
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:  # the oracle runs once, on rank 0's host cores
+        return None
+    from oracle import oracle_c as OC
+    rows = 1024
+    for _ in range(args.warmup):
+        _oracle_sample_step(rows)
+    tot_b, tot_s = 0, 0.0
+    for _ in range(args.steps):
+        b, s = _oracle_sample_step(rows)
+        tot_b += b
+        tot_s += s
+    v = tot_b / tot_s / 1e9
+    sample = f"first {rows} rows of each decode layer per step (C oracle fp32 dequant + fp64 matmul)"
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(tot_s / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int4 weights, fp64 matmul",
+        "data": "synthetic", "config": {"workload": "int4 nested-superscale decode GEMV, M=1, layers "
+                                                    "(K=5120,N=27648) and (K=27648,N=5120)", "M": 1},
+        "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": OC.num_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    line = run_reference(args) if args.impl == "reference" else run_native(args)
+    if line is not None:
+        print(json.dumps(line), flush=True)
+    try:
+        import torch.distributed as dist
+        if dist.is_initialized():
+            dist.destroy_process_group()
+    except Exception:
+        pass
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,206 @@
+/*
+ * qlinear.h -- C ABI of the B200 (sm_100a) weight-only quantized linear layer
+ *
+ *     y[M][N] = x[M][K] . dequant(Wq)[N][K]^T
+ *
+ * with group-wise dequantisation fused into the contraction.
+ *
+ * Formats (sources are web pages, cited by title and section):
+ *
+ *  QL_INT4_NSS   nested-superscale int4.  ExecuTorch PR "[cuda] Nestest
+ *                Superscale Quantization for CUDA Weights (int4 / int6)",
+ *                section "Quant schema update", int4 bullet: 4-bit codes,
+ *                group 32, super-block 256; scale = uint8 code x per-256 fp16
+ *                step, zero = uint8 code x per-256 fp16 step, both steps in
+ *                one 32-bit word; w = (q - zero) * scale; 4.625 bits/weight.
+ *  QL_INT6_SYM   symmetric int6, same page and section, int6 bullet: no zero,
+ *                group 16, super-block 256, scale = int8 code x per-256 fp16
+ *                step; 6.5625 bits/weight.  Section "Why this design" (b)
+ *                gives the reason the int8 scale code is kept.
+ *  QL_AFFINE_U32 uint32-packed affine.  Hugging Face Transformers docs,
+ *                "Metal" quantization page, introduction: codes packed into
+ *                uint32 words with per-group scales and biases; bit widths
+ *                2, 4, 8; group size configurable, default 64;
+ *                w = q * scale + bias.
+ *
+ * Layout of every weight buffer: W has N rows (output features) and K columns
+ * (input features); each row's data is contiguous and rows follow each other
+ * (row-major).  16-bit floats are raw IEEE binary16 / bfloat16 bit patterns.
+ *
+ *  QL_INT4_NSS  codes u8  [N][K/2]   byte i = q[2i] | q[2i+1] << 4
+ *               gmeta u16 [N][K/32]  scale code | zero code << 8
+ *               steps u32 [N][K/256] fp16 scale step | fp16 zero step << 16
+ *  QL_INT6_SYM  codes u8  [N][3K/4]  every 4 codes form one little-endian
+ *                                    24-bit unit: sum_i (q[4j+i] & 63) << 6i
+ *               gmeta i8  [N][K/16]  scale code
+ *               steps u16 [N][K/256] fp16 step
+ *  QL_AFFINE_U32 codes u32 [N][K*bits/32]  word t = sum_i q[tP+i] << bits*i,
+ *                                          P = 32/bits (first code lowest)
+ *               gmeta u32 [N][K/group] bf16 scale | bf16 bias << 16
+ *               steps (none)
+ *
+ * Dequantisation, exactly (each step one binary32 operation, nearest-even,
+ * no fused multiply-add):
+ *  int4:   S = f32(sc)*f32(ss); Z = f32(zc)*f32(zs); w = (f32(q) - Z) * S
+ *  int6:   S = f32(sc)*f32(st); w = f32(q) * S
+ *  affine: w = f32(q)*f32(scale) + f32(bias)
+ *
+ * Conventions for every entry point:
+ *  - Ownership: the caller allocates and frees every buffer; pointers are
+ *    device pointers unless stated otherwise.  The library allocates no
+ *    device memory in any call.  It keeps one small static device status
+ *    word per device and a host-side cache of kernel attributes.
+ *  - Asynchrony: calls enqueue work on `stream` and return without
+ *    synchronising (qlinear_sync_status excepted).
+ *  - Errors: arguments are validated on the host before anything is
+ *    launched; a non-QL_OK status means nothing was enqueued.  A launch
+ *    failure returns QL_ERR_CUDA.  Kernels never trap: a device-side wait
+ *    that gives up sets the device status word, which qlinear_sync_status
+ *    reports as QL_ERR_TIMEOUT.
+ *  - Alignment: every device pointer must be 16-byte aligned.
+ *  - Values out of range in the data (e.g. an int8 scale code of -128) are
+ *    not checked; they are defined by the formulas above.
+ */
+#ifndef QLINEAR_H
+#define QLINEAR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *ql_stream_t; /* a cudaStream_t; NULL = legacy default stream */
+
+typedef enum {
+  QL_OK = 0,
+  QL_ERR_NULL = 1,        /* a required pointer is NULL                          */
+  QL_ERR_SHAPE = 2,       /* N, K, M, bits or group not allowed for the format   */
+  QL_ERR_ALIGN = 3,       /* a pointer is not 16-byte aligned                    */
+  QL_ERR_RANGE = 4,       /* M outside the range of the entry point              */
+  QL_ERR_UNSUPPORTED = 5, /* unknown format, or the device is not sm_100         */
+  QL_ERR_CUDA = 6,        /* a CUDA runtime call or launch failed                */
+  QL_ERR_TIMEOUT = 7      /* a device-side bounded wait gave up                  */
+} ql_status;
+
+typedef enum { QL_INT4_NSS = 1, QL_INT6_SYM = 2, QL_AFFINE_U32 = 3 } ql_format;
+
+typedef enum { QL_OUT_F32 = 0, QL_OUT_BF16 = 1 } ql_out_dtype;
+
+/* Describes one quantized weight matrix.
+ *  fmt   : a ql_format value
+ *  bits  : QL_AFFINE_U32: 2, 4 or 8.  Ignored (0) for int4 / int6.
+ *  group : QL_AFFINE_U32: 32, 64 or 128.  Ignored (0) for int4 / int6, whose
+ *          groups are fixed at 32 and 16.
+ *  N     : output features, N >= 1.
+ *  K     : input features.  int4 / int6: K % 256 == 0.  affine:
+ *          K % group == 0 and (K * bits) % 128 == 0 (whole 16-byte rows). */
+typedef struct {
+  int32_t fmt;
+  int32_t bits;
+  int32_t group;
+  int32_t reserved;
+  int64_t N;
+  int64_t K;
+} ql_desc;
+
+/* The packed weight buffers (device pointers, caller-owned).  `steps` is
+ * unused (may be NULL) for QL_AFFINE_U32. */
+typedef struct {
+  void *codes;
+  void *gmeta;
+  void *steps;
+} ql_packed;
+
+typedef struct {
+  const void *codes;
+  const void *gmeta;
+  const void *steps;
+} ql_packed_const;
+
+/* The unpacked inputs of qlinear_pack (device pointers, caller-owned):
+ *              q (one code per byte)   meta0          meta1        step0        step1
+ *  int4:       u8 [N][K] 0..15         sc u8 [N][K/32] zc u8 [..]  ss f16 [N][K/256] zs f16 [..]
+ *  int6:       i8 [N][K] -32..31       sc i8 [N][K/16] (unused)    st f16 [N][K/256] (unused)
+ *  affine:     u8 [N][K] 0..2^bits-1   scale bf16 [N][K/group] bias bf16 [..] (unused) (unused)
+ * Codes are reduced to their low `bits` bits (int6: two's complement low
+ * 6 bits) when packed. */
+typedef struct {
+  const void *q;
+  const void *meta0;
+  const void *meta1;
+  const void *step0;
+  const void *step1;
+} ql_unpacked;
+
+/* Byte sizes of the three packed buffers for `desc` (host-only, no CUDA call).
+ * Size closed forms: int4 K/2 + K/16 + K/64 bytes per row (4.625 bits per
+ * weight); int6 3K/4 + K/16 + K/128 (6.5625); affine K*bits/8 + 4K/group
+ * (bits + 32/group).  Errors: QL_ERR_NULL, QL_ERR_SHAPE, QL_ERR_UNSUPPORTED. */
+ql_status qlinear_packed_bytes(const ql_desc *desc, size_t *codes_bytes,
+                               size_t *gmeta_bytes, size_t *steps_bytes);
+
+/* Pack unpacked codes and metadata into the layout above (one kernel).
+ * Same page and section as each format; bit-exact by definition.
+ * Errors: QL_ERR_NULL, QL_ERR_SHAPE, QL_ERR_ALIGN, QL_ERR_UNSUPPORTED,
+ * QL_ERR_CUDA. */
+ql_status qlinear_pack(const ql_desc *desc, const ql_unpacked *in,
+                       const ql_packed *out, ql_stream_t stream);
+
+/* Where qlinear_unpack writes: same element types and shapes as ql_unpacked
+ * (int6 codes come back sign-extended; unused members may be NULL). */
+typedef struct {
+  void *q;
+  void *meta0;
+  void *meta1;
+  void *step0;
+  void *step1;
+} ql_unpacked_out;
+
+/* Inverse of qlinear_pack (one kernel); bit-exact by definition.
+ * Errors: as qlinear_pack. */
+ql_status qlinear_unpack(const ql_desc *desc, const ql_packed_const *in,
+                         const ql_unpacked_out *out, ql_stream_t stream);
+
+/* Standalone dequantisation: out[N][K] = w as defined above, as binary32
+ * (QL_OUT_F32, bit-exact) or as its nearest-even bfloat16 (QL_OUT_BF16).
+ * Errors: as qlinear_pack, plus QL_ERR_SHAPE for an unknown out_dtype. */
+ql_status qlinear_dequant(const ql_desc *desc, const ql_packed_const *w,
+                          void *out, int32_t out_dtype, ql_stream_t stream);
+
+/* Decode-shaped layer, HBM-bound: y[M][N] (bf16) = x[M][K] (bf16) . W^T,
+ * fp32 accumulation, one nearest-even rounding to bf16 at the end.
+ * 1 <= M <= 8 for int4 / int6; 1 <= M <= 32 for affine.
+ * ExecuTorch page above, review section "Things done well" (the decode
+ * kernel's one-shuffle step-word broadcast and full-warp trip counts) and
+ * "Quant schema update" (hoisted int6 codes).
+ * Errors: QL_ERR_NULL, QL_ERR_SHAPE, QL_ERR_ALIGN, QL_ERR_RANGE,
+ * QL_ERR_UNSUPPORTED, QL_ERR_CUDA. */
+ql_status qlinear_gemv(const ql_desc *desc, const ql_packed_const *w,
+                       const void *x, int64_t M, void *y, ql_stream_t stream);
+
+/* Prefill-shaped layer on the tcgen05 tensor cores: same result definition
+ * as qlinear_gemv, any M >= 1 (meant for M >= 128).  Weights are
+ * dequantised once per tile to bf16 (one rounding of the exact binary32
+ * weight) and contracted with x in bf16 with fp32 accumulation in tensor
+ * memory.  Requires an sm_100 device.
+ * Errors: as qlinear_gemv, plus QL_ERR_UNSUPPORTED off sm_100. */
+ql_status qlinear_gemm(const ql_desc *desc, const ql_packed_const *w,
+                       const void *x, int64_t M, void *y, ql_stream_t stream);
+
+/* Synchronise `stream`, then read and clear the current device's status
+ * word: QL_ERR_TIMEOUT if a kernel's bounded wait gave up since the last
+ * call, QL_ERR_CUDA if the synchronisation failed, else QL_OK. */
+ql_status qlinear_sync_status(ql_stream_t stream);
+
+/* Static, never NULL. */
+const char *qlinear_status_string(ql_status status);
+
+/* Library version, e.g. 1 */
+int32_t qlinear_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* QLINEAR_H */

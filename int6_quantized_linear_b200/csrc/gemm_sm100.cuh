@@ -1,0 +1,328 @@
+// gemm_sm100.cuh -- prefill-shaped layer on the 5th-generation tensor core.
+//
+//   y[M][N] = x[M][K] . W^T,  x bf16, W quantized, y bf16, fp32 accumulation
+//
+// Persistent kernel, one CTA per SM, tiles of BM=128 tokens x BN=256 weight
+// rows, K streamed in BK=64 steps through a STAGES-deep shared-memory ring.
+// Warp roles:
+//   warp 0      TMA producer: x tile (128 x 64 bf16, 128-byte swizzle) and the
+//               packed code tile (256 rows x BK codes) per stage
+//   warp 1      TMEM allocator; lane 0 issues tcgen05.mma (M=128, N=256,
+//               K=16, bf16 x bf16 -> f32) into one of two TMEM accumulators
+//   warps 4-7   epilogue: tcgen05.ld the accumulator (warp w reads TMEM lanes
+//               32*(w%4)..), round to bf16, store y
+//   warps 8-15  dequantisers: packed codes (shared) + metadata (global, one
+//               stage ahead) -> exact binary32 weight -> nearest-even bf16,
+//               written in the canonical K-major 128-byte-swizzled layout the
+//               MMA reads as its B operand
+// Every mbarrier wait is bounded; a wait that gives up sets the device status
+// word and makes every role leave its loop.
+#pragma once
+#include "pack_dequant.cuh"
+
+namespace ql {
+namespace gemm {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 64;
+constexpr int STAGES = 3;
+constexpr int NUM_DEQ_WARPS = 8;
+constexpr int WARP_TMA = 0;
+constexpr int WARP_MMA = 1;
+constexpr int WARP_EPI0 = 4;
+constexpr int WARP_DEQ0 = 8;
+constexpr int NUM_THREADS = (WARP_DEQ0 + NUM_DEQ_WARPS) * 32;
+constexpr int A_BYTES = BM * BK * 2;  // 16 KB
+constexpr int B_BYTES = BN * BK * 2;  // 32 KB
+constexpr uint32_t TMEM_COLS = 2 * BN;  // two fp32 accumulators of 256 columns
+
+__host__ __device__ constexpr int code_bits(int fmt, int bits) {
+  return fmt == FMT_INT4 ? 4 : (fmt == FMT_INT6 ? 6 : bits);
+}
+__host__ __device__ constexpr int p_row_bytes(int fmt, int bits) { return BK * code_bits(fmt, bits) / 8; }
+__host__ __device__ constexpr int p_bytes(int fmt, int bits) { return BN * p_row_bytes(fmt, bits); }
+
+// byte offsets inside the dynamic shared memory (base aligned to 1024)
+__host__ __device__ constexpr int off_a(int s) { return s * A_BYTES; }
+__host__ __device__ constexpr int off_b(int s) { return STAGES * A_BYTES + s * B_BYTES; }
+__host__ __device__ constexpr int off_p(int fmt, int bits, int s) {
+  return STAGES * (A_BYTES + B_BYTES) + s * p_bytes(fmt, bits);
+}
+__host__ __device__ constexpr int off_bar(int fmt, int bits) {
+  return STAGES * (A_BYTES + B_BYTES + p_bytes(fmt, bits));
+}
+// barriers: tma_full[S], b_full[S], empty[S], acc_full[2], acc_empty[2], final
+constexpr int NUM_BARS = 3 * STAGES + 5;
+__host__ __device__ constexpr int smem_bytes(int fmt, int bits) {
+  return off_bar(fmt, bits) + NUM_BARS * 8 + 16 /* tmem base + abort flag */ + 1024 /* alignment slack */;
+}
+
+struct Params {
+  int64_t M, N, K;
+  int G;
+  const uint8_t *gmeta;
+  const uint8_t *steps;
+  __nv_bfloat16 *y;
+};
+
+// Metadata of one 32-weight chunk (see formats.cuh): int4 (gm, st); int6
+// (two scale codes, st); affine (gm, unused).
+template <int FMT>
+QL_DEVI void load_meta(const Params &p, int64_t n, int64_t c, uint32_t &gm, uint32_t &st) {
+  if (n >= p.N) {
+    gm = 0;
+    st = 0;
+    return;
+  }
+  if constexpr (FMT == FMT_INT4) {
+    gm = __ldg(reinterpret_cast<const uint16_t *>(p.gmeta) + n * (p.K / 32) + c);
+    st = __ldg(reinterpret_cast<const uint32_t *>(p.steps) + n * (p.K / 256) + (c >> 3));
+  } else if constexpr (FMT == FMT_INT6) {
+    gm = __ldg(reinterpret_cast<const uint16_t *>(p.gmeta + n * (p.K / 16)) + c);
+    st = __ldg(reinterpret_cast<const uint16_t *>(p.steps) + n * (p.K / 256) + (c >> 3));
+  } else {
+    gm = __ldg(reinterpret_cast<const uint32_t *>(p.gmeta) + n * (p.K / p.G) + (32 * c) / p.G);
+    st = 0;
+  }
+}
+
+// Decode one chunk whose codes sit in shared memory at `src`.
+template <int FMT, int BITS>
+QL_DEVI void smem_decode32(const uint8_t *src, uint32_t gm, uint32_t st, float (&w)[32]) {
+  if constexpr (FMT == FMT_INT4) {
+    const uint4 v = *reinterpret_cast<const uint4 *>(src);
+    const uint32_t c[4] = {v.x, v.y, v.z, v.w};
+    int4_decode32(c, gm, st, w);
+  } else if constexpr (FMT == FMT_INT6) {
+    const uint2 *s2 = reinterpret_cast<const uint2 *>(src);
+    const uint2 a = s2[0], b = s2[1], d = s2[2];
+    const uint32_t c[6] = {a.x, a.y, b.x, b.y, d.x, d.y};
+    int6_decode32(c, gm, st, w);
+  } else {
+    uint32_t c[BITS];
+    if constexpr (BITS == 2) {
+      const uint2 v = *reinterpret_cast<const uint2 *>(src);
+      c[0] = v.x;
+      c[1] = v.y;
+    } else {
+#pragma unroll
+      for (int t = 0; t < BITS / 4; ++t) {
+        const uint4 v = reinterpret_cast<const uint4 *>(src)[t];
+        c[4 * t] = v.x; c[4 * t + 1] = v.y; c[4 * t + 2] = v.z; c[4 * t + 3] = v.w;
+      }
+    }
+    affine_decode32<BITS>(c, gm, w);
+  }
+}
+
+template <int FMT, int BITS>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_codes,
+                Params p) {
+  constexpr int PROW = p_row_bytes(FMT, BITS);
+  constexpr uint32_t STAGE_TX = A_BYTES + p_bytes(FMT, BITS);
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + off_bar(FMT, BITS));
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + NUM_BARS);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+  auto bar_tma_full = [&](int s) { return smem_u32(bars + s); };
+  auto bar_b_full = [&](int s) { return smem_u32(bars + STAGES + s); };
+  auto bar_empty = [&](int s) { return smem_u32(bars + 2 * STAGES + s); };
+  auto bar_acc_full = [&](int a) { return smem_u32(bars + 3 * STAGES + a); };
+  auto bar_acc_empty = [&](int a) { return smem_u32(bars + 3 * STAGES + 2 + a); };
+  const uint32_t bar_final = smem_u32(bars + 3 * STAGES + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t m_tiles = (p.M + BM - 1) / BM, n_tiles = (p.N + BN - 1) / BN;
+  const int64_t num_tiles = m_tiles * n_tiles;
+  const int num_kb = (int)(p.K / BK);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(bar_tma_full(s), 1);
+      mbar_init(bar_b_full(s), NUM_DEQ_WARPS);
+      mbar_init(bar_empty(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(bar_acc_full(a), 1);
+      mbar_init(bar_acc_empty(a), 4);
+    }
+    mbar_init(bar_final, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == WARP_MMA) {
+    tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == WARP_TMA) {
+    if (lane == 0) {
+      tma_prefetch_desc(&map_x);
+      tma_prefetch_desc(&map_codes);
+      int64_t it = 0;
+      bool ok = true;
+      for (int64_t tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        const int64_t n_tile = tile / m_tiles, m_tile = tile - n_tile * m_tiles;
+        for (int kb = 0; kb < num_kb; ++kb, ++it) {
+          const int s = (int)(it % STAGES);
+          const uint32_t use = (uint32_t)(it / STAGES);
+          if (!mbar_wait_bounded(bar_empty(s), (use & 1) ^ 1, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(bar_tma_full(s), STAGE_TX);
+          tma_load_2d(sbase + off_a(s), &map_x, bar_tma_full(s), kb * BK, (int32_t)(m_tile * BM));
+          tma_load_2d(sbase + off_p(FMT, BITS, s), &map_codes, bar_tma_full(s), kb * PROW,
+                      (int32_t)(n_tile * BN));
+        }
+      }
+      if (!ok) {  // let copies already issued land before the CTA can exit
+        for (int64_t j = it - 1; j >= 0 && j >= it - STAGES; --j) {
+          const long long t0 = clock64();
+          while (!mbar_try_wait(bar_tma_full((int)(j % STAGES)), (uint32_t)((j / STAGES) & 1)) &&
+                 clock64() - t0 < QL_WAIT_LIMIT_CYCLES) {
+          }
+        }
+      }
+    }
+  } else if (warp == WARP_MMA) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = umma_idesc_bf16_f32(BM, BN);
+      int64_t it = 0, tcount = 0;
+      bool ok = true, issued = false;
+      for (int64_t tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++tcount) {
+        const int a = (int)(tcount & 1);
+        const uint32_t ause = (uint32_t)(tcount >> 1);
+        if (!mbar_wait_bounded(bar_acc_empty(a), (ause & 1) ^ 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(a * BN);
+        for (int kb = 0; kb < num_kb; ++kb, ++it) {
+          const int s = (int)(it % STAGES);
+          const uint32_t par = (uint32_t)((it / STAGES) & 1);
+          if (!mbar_wait_bounded(bar_tma_full(s), par, abort_flag) ||
+              !mbar_wait_bounded(bar_b_full(s), par, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t adesc = umma_desc_k_sw128(sbase + off_a(s));
+          const uint64_t bdesc = umma_desc_k_sw128(sbase + off_b(s));
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)  // advance 16 bf16 = 32 bytes = 2 descriptor units
+            umma_f16(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) != 0);
+          umma_commit(bar_empty(s));
+          issued = true;
+        }
+        if (!ok) break;
+        umma_commit(bar_acc_full(a));
+      }
+      if (issued) {  // all MMAs retired before teardown
+        umma_commit(bar_final);
+        const long long t0 = clock64();
+        while (!mbar_try_wait(bar_final, 0) && clock64() - t0 < QL_WAIT_LIMIT_CYCLES) {
+        }
+      }
+    }
+  } else if (warp >= WARP_EPI0 && warp < WARP_EPI0 + 4) {
+    const int e = warp - WARP_EPI0;  // TMEM lane quarter
+    int64_t tcount = 0;
+    const bool vec_ok = (p.N % 8) == 0;
+    for (int64_t tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tcount) {
+      const int64_t n_tile = tile / m_tiles, m_tile = tile - n_tile * m_tiles;
+      const int a = (int)(tcount & 1);
+      const uint32_t ause = (uint32_t)(tcount >> 1);
+      if (!mbar_wait_bounded(bar_acc_full(a), ause & 1, abort_flag)) break;
+      tc_fence_after();
+      const int64_t m = m_tile * BM + 32 * e + lane;
+#pragma unroll 1
+      for (int cchunk = 0; cchunk < BN / 32; ++cchunk) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(32 * e) << 16) + (uint32_t)(a * BN + 32 * cchunk), r);
+        tmem_ld_wait();
+        const int64_t n0 = n_tile * BN + 32 * cchunk;
+        if (m < p.M) {
+          __nv_bfloat16 *dst = p.y + m * p.N + n0;
+          if (vec_ok && n0 + 32 <= p.N) {
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+              uint4 v;
+              v.x = pack_bf16x2(__uint_as_float(r[8 * t + 0]), __uint_as_float(r[8 * t + 1]));
+              v.y = pack_bf16x2(__uint_as_float(r[8 * t + 2]), __uint_as_float(r[8 * t + 3]));
+              v.z = pack_bf16x2(__uint_as_float(r[8 * t + 4]), __uint_as_float(r[8 * t + 5]));
+              v.w = pack_bf16x2(__uint_as_float(r[8 * t + 6]), __uint_as_float(r[8 * t + 7]));
+              reinterpret_cast<uint4 *>(dst)[t] = v;
+            }
+          } else {
+            for (int i = 0; i < 32; ++i)
+              if (n0 + i < p.N) dst[i] = __float2bfloat16_rn(__uint_as_float(r[i]));
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_acc_empty(a));
+    }
+  } else if (warp >= WARP_DEQ0) {
+    const int t = threadIdx.x - WARP_DEQ0 * 32;  // 0..255
+    const int h = t & 1;                          // which 32-weight half of the 64-k stage
+    const int r0 = t >> 1, r1 = r0 + 128;         // the two tile rows this thread fills
+    int64_t it = 0;
+    const int64_t my_tiles = (num_tiles - blockIdx.x + gridDim.x - 1) / gridDim.x;
+    const int64_t total_it = my_tiles * num_kb;
+    auto tile_of = [&](int64_t i) { return (int64_t)blockIdx.x + (i / num_kb) * gridDim.x; };
+    uint32_t gm0 = 0, st0 = 0, gm1 = 0, st1 = 0;
+    if (total_it > 0) {
+      const int64_t n_tile = tile_of(0) / m_tiles;
+      load_meta<FMT>(p, n_tile * BN + r0, h, gm0, st0);
+      load_meta<FMT>(p, n_tile * BN + r1, h, gm1, st1);
+    }
+    for (; it < total_it; ++it) {
+      uint32_t ngm0 = 0, nst0 = 0, ngm1 = 0, nst1 = 0;
+      if (it + 1 < total_it) {  // prefetch the next stage's metadata
+        const int64_t n_tile = tile_of(it + 1) / m_tiles;
+        const int64_t c = (int64_t)((it + 1) % num_kb) * (BK / 32) + h;
+        load_meta<FMT>(p, n_tile * BN + r0, c, ngm0, nst0);
+        load_meta<FMT>(p, n_tile * BN + r1, c, ngm1, nst1);
+      }
+      const int s = (int)(it % STAGES);
+      if (!mbar_wait_bounded(bar_tma_full(s), (uint32_t)((it / STAGES) & 1), abort_flag)) break;
+      const uint8_t *P = smem + off_p(FMT, BITS, s);
+      uint8_t *B = smem + off_b(s);
+#pragma unroll
+      for (int rr = 0; rr < 2; ++rr) {
+        const int r = rr ? r1 : r0;
+        float w[32];
+        smem_decode32<FMT, BITS>(P + r * PROW + h * (PROW / 2), rr ? gm1 : gm0, rr ? st1 : st0, w);
+        uint8_t *row = B + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int j = 4 * h + q;  // logical 16-byte chunk of the 128-byte row
+          uint4 v;
+          v.x = pack_bf16x2(w[8 * q + 0], w[8 * q + 1]);
+          v.y = pack_bf16x2(w[8 * q + 2], w[8 * q + 3]);
+          v.z = pack_bf16x2(w[8 * q + 4], w[8 * q + 5]);
+          v.w = pack_bf16x2(w[8 * q + 6], w[8 * q + 7]);
+          *reinterpret_cast<uint4 *>(row + ((j ^ (r & 7)) << 4)) = v;
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if ((t & 31) == 0) mbar_arrive(bar_b_full(s));
+      gm0 = ngm0; st0 = nst0; gm1 = ngm1; st1 = nst1;
+    }
+  }
+
+  __syncthreads();
+  if (warp == WARP_MMA) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+}  // namespace gemm
+}  // namespace ql

@@ -1,0 +1,368 @@
+// qlinear.cu -- the C ABI (include/qlinear.h): host-side validation, launch
+// configuration and TMA descriptor encoding.  Single translation unit: the
+// kernels live in the included .cuh files and share one device status word.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "../../include/qlinear.h"
+#include "gemm_sm100.cuh"
+#include "gemv.cuh"
+#include "pack_dequant.cuh"
+
+using namespace ql;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool init = false;
+  int sms = 0;
+  int major = 0, minor = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_mu;
+
+ql_status device_info(DeviceInfo **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return QL_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceInfo &d = g_dev[dev];
+  if (!d.init) {
+    if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return QL_ERR_CUDA;
+    d.init = true;
+  }
+  *out = &d;
+  return QL_OK;
+}
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+ql_status check_desc(const ql_desc *d) {
+  if (!d) return QL_ERR_NULL;
+  if (d->N < 1 || d->K < 1) return QL_ERR_SHAPE;
+  switch (d->fmt) {
+    case QL_INT4_NSS:
+    case QL_INT6_SYM:
+      if (d->K % 256 != 0) return QL_ERR_SHAPE;
+      return QL_OK;
+    case QL_AFFINE_U32:
+      if (d->bits != 2 && d->bits != 4 && d->bits != 8) return QL_ERR_SHAPE;
+      if (d->group != 32 && d->group != 64 && d->group != 128) return QL_ERR_SHAPE;
+      if (d->K % d->group != 0 || (d->K * d->bits) % 128 != 0) return QL_ERR_SHAPE;
+      return QL_OK;
+    default:
+      return QL_ERR_UNSUPPORTED;
+  }
+}
+
+void sizes(const ql_desc *d, size_t *c, size_t *g, size_t *s) {
+  const size_t N = (size_t)d->N, K = (size_t)d->K;
+  switch (d->fmt) {
+    case QL_INT4_NSS: *c = N * K / 2; *g = N * (K / 32) * 2; *s = N * (K / 256) * 4; break;
+    case QL_INT6_SYM: *c = N * 3 * K / 4; *g = N * (K / 16); *s = N * (K / 256) * 2; break;
+    default: *c = N * K * d->bits / 8; *g = N * (K / d->group) * 4; *s = 0; break;
+  }
+}
+
+ql_status check_packed(const ql_desc *d, const void *codes, const void *gmeta, const void *steps) {
+  if (!codes || !gmeta || (d->fmt != QL_AFFINE_U32 && !steps)) return QL_ERR_NULL;
+  if (!aligned16(codes) || !aligned16(gmeta) || (d->fmt != QL_AFFINE_U32 && !aligned16(steps)))
+    return QL_ERR_ALIGN;
+  return QL_OK;
+}
+
+inline int grid_for(int64_t units, int sms, int per_sm = 8) {
+  int64_t g = (units + 255) / 256;
+  const int64_t cap = (int64_t)sms * per_sm;
+  if (g > cap) g = cap;
+  if (g < 1) g = 1;
+  return (int)g;
+}
+
+inline ql_status launched() {
+  return cudaGetLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
+}
+
+WeightPtrs make_ptrs(const ql_desc *d, const ql_packed_const *w) {
+  WeightPtrs p;
+  p.codes = static_cast<const uint8_t *>(w->codes);
+  p.gmeta = static_cast<const uint8_t *>(w->gmeta);
+  p.steps = static_cast<const uint8_t *>(w->steps);
+  p.K = d->K;
+  p.G = d->group;
+  return p;
+}
+
+// ---- TMA descriptors ---------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+bool encode_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64_t inner, uint64_t outer,
+               uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int FMT, int BITS>
+ql_status launch_gemm(const ql_desc *d, const ql_packed_const *w, const void *x, int64_t M, void *y,
+                      cudaStream_t st, int sms) {
+  using namespace ql::gemm;
+  const int64_t N = d->N, K = d->K;
+  const uint64_t row_bytes = (uint64_t)K * code_bits(FMT, BITS) / 8;
+  CUtensorMap mx, mc;
+  if (!encode_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, BK, BM,
+                 CU_TENSOR_MAP_SWIZZLE_128B))
+    return QL_ERR_CUDA;
+  if (!encode_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->codes, row_bytes, (uint64_t)N, row_bytes,
+                 (uint32_t)p_row_bytes(FMT, BITS), BN, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return QL_ERR_CUDA;
+  Params p;
+  p.M = M; p.N = N; p.K = K; p.G = d->group;
+  p.gmeta = static_cast<const uint8_t *>(w->gmeta);
+  p.steps = static_cast<const uint8_t *>(w->steps);
+  p.y = static_cast<__nv_bfloat16 *>(y);
+  const int smem = smem_bytes(FMT, BITS);
+  auto kern = gemm_kernel<FMT, BITS>;
+  static thread_local int configured_dev = -1;  // per (kernel instantiation, thread)
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (configured_dev != dev) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return QL_ERR_CUDA;
+    configured_dev = dev;
+  }
+  const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+  const int grid = (int)(tiles < sms ? tiles : sms);
+  kern<<<grid, NUM_THREADS, smem, st>>>(mx, mc, p);
+  return launched();
+}
+
+template <int FMT, int BITS>
+ql_status launch_gemv(const ql_desc *d, const ql_packed_const *w, const void *x, int64_t M, void *y,
+                      cudaStream_t st, int sms) {
+  const WeightPtrs p = make_ptrs(d, w);
+  const int64_t rows_per_block = 8;
+  int64_t g = (d->N + rows_per_block - 1) / rows_per_block;
+  const int64_t cap = (int64_t)sms * 16;
+  if (g > cap) g = cap;
+  const auto *xb = static_cast<const __nv_bfloat16 *>(x);
+  auto *yb = static_cast<__nv_bfloat16 *>(y);
+  if (M == 1)
+    gemv_simple_kernel<FMT, BITS, 1><<<(int)g, 256, 0, st>>>(p, d->N, xb, (int)M, yb);
+  else if (M == 2)
+    gemv_simple_kernel<FMT, BITS, 2><<<(int)g, 256, 0, st>>>(p, d->N, xb, (int)M, yb);
+  else if (M <= 4)
+    gemv_simple_kernel<FMT, BITS, 4><<<(int)g, 256, 0, st>>>(p, d->N, xb, (int)M, yb);
+  else
+    gemv_simple_kernel<FMT, BITS, 8><<<(int)g, 256, 0, st>>>(p, d->N, xb, (int)M, yb);
+  return launched();
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t qlinear_version(void) { return 1; }
+
+const char *qlinear_status_string(ql_status s) {
+  switch (s) {
+    case QL_OK: return "ok";
+    case QL_ERR_NULL: return "a required pointer is NULL";
+    case QL_ERR_SHAPE: return "shape, bit width or group size not allowed for this format";
+    case QL_ERR_ALIGN: return "a device pointer is not 16-byte aligned";
+    case QL_ERR_RANGE: return "M outside the range of this entry point";
+    case QL_ERR_UNSUPPORTED: return "unknown format or unsupported device";
+    case QL_ERR_CUDA: return "a CUDA call or kernel launch failed";
+    case QL_ERR_TIMEOUT: return "a device-side bounded wait gave up";
+  }
+  return "unknown status";
+}
+
+ql_status qlinear_packed_bytes(const ql_desc *d, size_t *c, size_t *g, size_t *s) {
+  if (!c || !g || !s) return QL_ERR_NULL;
+  const ql_status st = check_desc(d);
+  if (st != QL_OK) return st;
+  sizes(d, c, g, s);
+  return QL_OK;
+}
+
+ql_status qlinear_pack(const ql_desc *d, const ql_unpacked *in, const ql_packed *out, ql_stream_t stream) {
+  ql_status st = check_desc(d);
+  if (st != QL_OK) return st;
+  if (!in || !out || !in->q || !in->meta0) return QL_ERR_NULL;
+  if ((d->fmt == QL_INT4_NSS && (!in->meta1 || !in->step0 || !in->step1)) ||
+      (d->fmt == QL_INT6_SYM && !in->step0) || (d->fmt == QL_AFFINE_U32 && !in->meta1))
+    return QL_ERR_NULL;
+  if ((st = check_packed(d, out->codes, out->gmeta, out->steps)) != QL_OK) return st;
+  const void *ins[5] = {in->q, in->meta0, in->meta1, in->step0, in->step1};
+  for (const void *p : ins)
+    if (p && !aligned16(p)) return QL_ERR_ALIGN;
+  DeviceInfo *di;
+  if ((st = device_info(&di)) != QL_OK) return st;
+  PackArgs a;
+  a.N = d->N; a.K = d->K; a.bits = d->bits; a.G = d->group;
+  a.q = static_cast<const uint8_t *>(in->q);
+  a.meta0 = static_cast<const uint8_t *>(in->meta0);
+  a.meta1 = static_cast<const uint8_t *>(in->meta1);
+  a.step0 = static_cast<const uint16_t *>(in->step0);
+  a.step1 = static_cast<const uint16_t *>(in->step1);
+  a.codes = static_cast<uint8_t *>(out->codes);
+  a.gmeta = static_cast<uint8_t *>(out->gmeta);
+  a.steps = static_cast<uint8_t *>(out->steps);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t NK = d->N * d->K;
+  switch (d->fmt) {
+    case QL_INT4_NSS: pack_int4_kernel<<<grid_for(NK / 32 + NK / 128, di->sms), 256, 0, s>>>(a); break;
+    case QL_INT6_SYM: pack_int6_kernel<<<grid_for(NK / 64 + NK / 128, di->sms), 256, 0, s>>>(a); break;
+    default: {
+      const int g = grid_for(NK * d->bits / 128 + NK / d->group, di->sms);
+      if (d->bits == 2) pack_affine_kernel<2><<<g, 256, 0, s>>>(a);
+      else if (d->bits == 4) pack_affine_kernel<4><<<g, 256, 0, s>>>(a);
+      else pack_affine_kernel<8><<<g, 256, 0, s>>>(a);
+    }
+  }
+  return launched();
+}
+
+ql_status qlinear_unpack(const ql_desc *d, const ql_packed_const *in, const ql_unpacked_out *out,
+                         ql_stream_t stream) {
+  ql_status st = check_desc(d);
+  if (st != QL_OK) return st;
+  if (!in || !out || !out->q) return QL_ERR_NULL;
+  if ((st = check_packed(d, in->codes, in->gmeta, in->steps)) != QL_OK) return st;
+  const void *outs[5] = {out->q, out->meta0, out->meta1, out->step0, out->step1};
+  for (const void *p : outs)
+    if (p && !aligned16(p)) return QL_ERR_ALIGN;
+  DeviceInfo *di;
+  if ((st = device_info(&di)) != QL_OK) return st;
+  UnpackArgs a;
+  a.N = d->N; a.K = d->K; a.bits = d->bits; a.G = d->group;
+  a.codes = static_cast<const uint8_t *>(in->codes);
+  a.gmeta = static_cast<const uint8_t *>(in->gmeta);
+  a.steps = static_cast<const uint8_t *>(in->steps);
+  a.q = static_cast<uint8_t *>(out->q);
+  a.meta0 = static_cast<uint8_t *>(out->meta0);
+  a.meta1 = static_cast<uint8_t *>(out->meta1);
+  a.step0 = static_cast<uint16_t *>(out->step0);
+  a.step1 = static_cast<uint16_t *>(out->step1);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t NK = d->N * d->K;
+  switch (d->fmt) {
+    case QL_INT4_NSS: unpack_int4_kernel<<<grid_for(NK / 32 * 2 + NK / 256, di->sms), 256, 0, s>>>(a); break;
+    case QL_INT6_SYM: unpack_int6_kernel<<<grid_for(NK / 64 + NK / 16, di->sms), 256, 0, s>>>(a); break;
+    default: {
+      const int g = grid_for(NK * d->bits / 32 + NK / d->group, di->sms);
+      if (d->bits == 2) unpack_affine_kernel<2><<<g, 256, 0, s>>>(a);
+      else if (d->bits == 4) unpack_affine_kernel<4><<<g, 256, 0, s>>>(a);
+      else unpack_affine_kernel<8><<<g, 256, 0, s>>>(a);
+    }
+  }
+  return launched();
+}
+
+ql_status qlinear_dequant(const ql_desc *d, const ql_packed_const *w, void *out, int32_t out_dtype,
+                          ql_stream_t stream) {
+  ql_status st = check_desc(d);
+  if (st != QL_OK) return st;
+  if (!w || !out) return QL_ERR_NULL;
+  if ((st = check_packed(d, w->codes, w->gmeta, w->steps)) != QL_OK) return st;
+  if (!aligned16(out)) return QL_ERR_ALIGN;
+  if (out_dtype != QL_OUT_F32 && out_dtype != QL_OUT_BF16) return QL_ERR_SHAPE;
+  DeviceInfo *di;
+  if ((st = device_info(&di)) != QL_OK) return st;
+  const WeightPtrs p = make_ptrs(d, w);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int g = grid_for(d->N * d->K / 32, di->sms);
+  const bool bf = out_dtype == QL_OUT_BF16;
+#define QL_DQ(F, B)                                                        \
+  do {                                                                     \
+    if (bf) dequant_kernel<F, B, true><<<g, 256, 0, s>>>(p, d->N, out);    \
+    else dequant_kernel<F, B, false><<<g, 256, 0, s>>>(p, d->N, out);      \
+  } while (0)
+  switch (d->fmt) {
+    case QL_INT4_NSS: QL_DQ(FMT_INT4, 4); break;
+    case QL_INT6_SYM: QL_DQ(FMT_INT6, 6); break;
+    default:
+      if (d->bits == 2) QL_DQ(FMT_AFFINE, 2);
+      else if (d->bits == 4) QL_DQ(FMT_AFFINE, 4);
+      else QL_DQ(FMT_AFFINE, 8);
+  }
+#undef QL_DQ
+  return launched();
+}
+
+ql_status qlinear_gemv(const ql_desc *d, const ql_packed_const *w, const void *x, int64_t M, void *y,
+                       ql_stream_t stream) {
+  ql_status st = check_desc(d);
+  if (st != QL_OK) return st;
+  if (!w || !x || !y) return QL_ERR_NULL;
+  if ((st = check_packed(d, w->codes, w->gmeta, w->steps)) != QL_OK) return st;
+  if (!aligned16(x) || !aligned16(y)) return QL_ERR_ALIGN;
+  const int64_t mmax = d->fmt == QL_AFFINE_U32 ? 32 : 8;
+  if (M < 1 || M > mmax) return QL_ERR_RANGE;
+  DeviceInfo *di;
+  if ((st = device_info(&di)) != QL_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  switch (d->fmt) {
+    case QL_INT4_NSS: return launch_gemv<FMT_INT4, 4>(d, w, x, M, y, s, di->sms);
+    case QL_INT6_SYM: return launch_gemv<FMT_INT6, 6>(d, w, x, M, y, s, di->sms);
+    default:
+      if (d->bits == 2) return launch_gemv<FMT_AFFINE, 2>(d, w, x, M, y, s, di->sms);
+      if (d->bits == 4) return launch_gemv<FMT_AFFINE, 4>(d, w, x, M, y, s, di->sms);
+      return launch_gemv<FMT_AFFINE, 8>(d, w, x, M, y, s, di->sms);
+  }
+}
+
+ql_status qlinear_gemm(const ql_desc *d, const ql_packed_const *w, const void *x, int64_t M, void *y,
+                       ql_stream_t stream) {
+  ql_status st = check_desc(d);
+  if (st != QL_OK) return st;
+  if (!w || !x || !y) return QL_ERR_NULL;
+  if ((st = check_packed(d, w->codes, w->gmeta, w->steps)) != QL_OK) return st;
+  if (!aligned16(x) || !aligned16(y)) return QL_ERR_ALIGN;
+  if (M < 1 || M > (int64_t)INT32_MAX) return QL_ERR_RANGE;
+  if (d->K % gemm::BK != 0 || d->N > (int64_t)INT32_MAX) return QL_ERR_SHAPE;
+  DeviceInfo *di;
+  if ((st = device_info(&di)) != QL_OK) return st;
+  if (di->major != 10) return QL_ERR_UNSUPPORTED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  switch (d->fmt) {
+    case QL_INT4_NSS: return launch_gemm<FMT_INT4, 4>(d, w, x, M, y, s, di->sms);
+    case QL_INT6_SYM: return launch_gemm<FMT_INT6, 6>(d, w, x, M, y, s, di->sms);
+    default:
+      if (d->bits == 2) return launch_gemm<FMT_AFFINE, 2>(d, w, x, M, y, s, di->sms);
+      if (d->bits == 4) return launch_gemm<FMT_AFFINE, 4>(d, w, x, M, y, s, di->sms);
+      return launch_gemm<FMT_AFFINE, 8>(d, w, x, M, y, s, di->sms);
+  }
+}
+
+ql_status qlinear_sync_status(ql_stream_t stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return QL_ERR_CUDA;
+  unsigned int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_ql_status, sizeof v) != cudaSuccess) return QL_ERR_CUDA;
+  if (v != 0 && cudaMemcpyToSymbol(g_ql_status, &zero, sizeof zero) != cudaSuccess) return QL_ERR_CUDA;
+  return (v & QL_DEV_TIMEOUT) ? QL_ERR_TIMEOUT : QL_OK;
+}
+
+}  // extern "C"

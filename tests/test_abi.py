@@ -1,0 +1,103 @@
+"""The C-ABI library: loads, exports every entry point its header declares, and
+validates arguments on the host (CPU only; no compute call is made)."""
+import ctypes as C
+import os
+import re
+import subprocess
+
+import pytest
+
+import int6_quantized_linear_b200 as ql
+from int6_quantized_linear_b200 import _build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    _build.build()
+    return ql.lib()
+
+
+def declared_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b(qlinear_\w+)\s*\(", src))
+    return sorted(names)
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("qlinear_pack", "qlinear_dequant", "qlinear_gemv", "qlinear_gemm",
+                     "qlinear_packed_bytes", "qlinear_status_string", "qlinear_sync_status"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", ql.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r"\bT (qlinear_\w+)", out))
+    for name in declared_functions():
+        assert name in exported, name
+        assert hasattr(lib, name)
+    assert set(ql._SIGNATURES) == set(declared_functions())
+
+
+def test_no_oracle_in_the_product():
+    """The library neither defines nor links an oracle routine, and no product module imports it."""
+    out = subprocess.run(["nm", "-D", ql.LIB_PATH], capture_output=True, text=True, check=True).stdout
+    assert not re.search(r"\bor_(int4|int6|affine|matmul|f32|bf16)", out)
+    pkg = os.path.join(ROOT, "int6_quantized_linear_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for fn in files:
+            if fn.endswith((".py", ".cu", ".cuh", ".h")):
+                src = open(os.path.join(dirpath, fn)).read()
+                assert not re.search(r"^\s*(import|from)\s+oracle\b", src, flags=re.M), fn
+                assert "liboracle" not in src and "oracle.h" not in src, fn
+
+
+@pytest.mark.parametrize("fmt,N,K,bits,group,bpw", [
+    ("int4", 3, 512, 0, 0, 4.625), ("int6", 3, 512, 0, 0, 6.5625),
+    ("affine", 3, 512, 2, 64, 2.5), ("affine", 3, 512, 4, 64, 4.5), ("affine", 3, 512, 8, 64, 8.5),
+    ("affine", 3, 512, 4, 32, 5.0), ("affine", 3, 512, 4, 128, 4.25)])
+def test_packed_bytes_closed_forms(lib, fmt, N, K, bits, group, bpw):
+    c, g, s = ql.qlinear_packed_bytes(ql.Desc(fmt, N, K, bits, group))
+    assert 8 * (c + g + s) == bpw * N * K
+
+
+@pytest.mark.parametrize("desc", [
+    ql.Desc("int4", 4, 255), ql.Desc("int4", 0, 256), ql.Desc("int6", 4, 384),
+    ql.Desc("affine", 4, 512, 3, 64), ql.Desc("affine", 4, 512, 4, 48), ql.Desc("affine", 4, 96, 2, 32)])
+def test_bad_shapes_rejected(lib, desc):
+    with pytest.raises(ql.QLinearError) as e:
+        ql.qlinear_packed_bytes(desc)
+    assert e.value.status == ql.QL_ERR_SHAPE
+
+
+def _call_gemv(lib, desc, codes, gmeta, steps, x, M, y):
+    d = desc.c()
+    w = ql.ql_packed(codes, gmeta, steps)
+    return lib.qlinear_gemv(C.byref(d), C.byref(w), x, M, y, None)
+
+
+def test_host_validation_before_any_launch(lib):
+    """Errors detected on the host come back before the library touches the device."""
+    d = ql.Desc("int4", 8, 256)
+    A = 0x10000  # an aligned address that is never dereferenced: validation fails first
+    assert _call_gemv(lib, d, None, A, A, A, 1, A) == ql.QL_ERR_NULL
+    assert _call_gemv(lib, d, A + 4, A, A, A, 1, A) == ql.QL_ERR_ALIGN
+    assert _call_gemv(lib, d, A, A, A, A + 2, 1, A) == ql.QL_ERR_ALIGN
+    assert _call_gemv(lib, d, A, A, A, A, 0, A) == ql.QL_ERR_RANGE
+    assert _call_gemv(lib, d, A, A, A, A, 9, A) == ql.QL_ERR_RANGE
+    assert _call_gemv(lib, ql.Desc("int4", 8, 100), A, A, A, A, 1, A) == ql.QL_ERR_SHAPE
+    da = ql.Desc("affine", 8, 256, 4, 64)
+    assert _call_gemv(lib, da, A, A, None, A, 33, A) == ql.QL_ERR_RANGE
+    bad = ql.ql_desc(9, 0, 0, 0, 8, 256)
+    w = ql.ql_packed(A, A, A)
+    assert lib.qlinear_gemm(C.byref(bad), C.byref(w), A, 1, A, None) == ql.QL_ERR_UNSUPPORTED
+    for s in range(8):
+        assert isinstance(ql.status_string(s), str) and ql.status_string(s)
+    assert lib.qlinear_version() >= 1

@@ -1,0 +1,163 @@
+"""CUDA path vs the CPU oracle, through the C ABI (GPU only).
+
+Bit-exact: pack, unpack, fp32 dequant, bf16 dequant.  Within the stated
+tolerance (see gpu_helpers.assert_close): the GEMV and the tcgen05 GEMM.
+Small shapes are compared element by element; the full layer shapes are
+compared on sampled output rows the oracle computes one by one.
+"""
+import numpy as np
+import pytest
+import torch
+
+import int6_quantized_linear_b200 as ql
+from int6_quantized_linear_b200 import synth
+from oracle import oracle_c as OC
+from tests.gpu_helpers import Layer, assert_close, dev, host, run_gemm, run_gemv, x_dev
+
+pytestmark = pytest.mark.gpu
+
+FORMATS = [("int4", 0, 0), ("int6", 0, 0), ("affine", 2, 64), ("affine", 4, 64), ("affine", 8, 64),
+           ("affine", 4, 32), ("affine", 8, 128)]
+FMT_IDS = [f"{f}{b or ''}g{g or ''}" for f, b, g in FORMATS]
+# several tiles plus a ragged tail in N; K of one super-block and several
+SMALL_SHAPES = [(1, 256), (7, 512), (33, 1024), (300, 2048), (513, 768)]
+
+
+@pytest.mark.parametrize("fmt,bits,group", FORMATS, ids=FMT_IDS)
+@pytest.mark.parametrize("N,K", SMALL_SHAPES)
+def test_pack_unpack_dequant_bitexact(cuda, fmt, bits, group, N, K):
+    L = Layer(fmt, N, K, seed=N + K, bits=bits, group=group)
+    got = L.packed_host()
+    want = L.oracle_pack()
+    for a, b in zip(got, want):
+        if b is not None:
+            assert np.array_equal(a, b)
+    # unpack on the GPU recovers the inputs
+    u = L.unpacked_host()
+    outs = [torch.empty_like(dev(a)) if a is not None else None for a in u]
+    ql.qlinear_unpack(L.desc, *L.packed(), *outs)
+    for a, o in zip(u, outs):
+        if a is not None:
+            assert np.array_equal(host(o, a.dtype).reshape(a.shape), a)
+    # dequant, fp32 bit-exact and bf16 = nearest-even of the fp32 value
+    w_ref = L.oracle_w()
+    w32 = torch.empty((N, K), dtype=torch.float32, device="cuda")
+    ql.qlinear_dequant(L.desc, *L.packed(), w32, ql.QL_OUT_F32)
+    assert np.array_equal(host(w32, np.uint32), w_ref.view(np.uint32))
+    w16 = torch.empty((N, K), dtype=torch.bfloat16, device="cuda")
+    ql.qlinear_dequant(L.desc, *L.packed(), w16, ql.QL_OUT_BF16)
+    want16 = np.array([OC.bf16_from_f32(v) for v in w_ref.ravel()[:4096]], np.uint16)
+    assert np.array_equal(host(w16.view(torch.int16), np.uint16).ravel()[:4096], want16)
+    assert ql.qlinear_sync_status() == ql.QL_OK
+
+
+@pytest.mark.parametrize("fmt,bits,group", FORMATS, ids=FMT_IDS)
+@pytest.mark.parametrize("N,K", SMALL_SHAPES)
+def test_gemv_small(cuda, fmt, bits, group, N, K):
+    L = Layer(fmt, N, K, seed=3 * N + K, bits=bits, group=group)
+    w_ref = L.oracle_w()
+    for M in ((1, 2, 3, 5, 8) if fmt != "affine" else (1, 4, 8, 13, 32)):
+        xb, xd = x_dev(K, M, seed=M)
+        y = run_gemv(L, xd, M)
+        assert_close(y, OC.matmul_f64(xb, w_ref), f"gemv {fmt} N={N} K={K} M={M}")
+
+
+@pytest.mark.parametrize("fmt,bits,group", [("int4", 0, 0), ("int6", 0, 0), ("affine", 4, 64),
+                                            ("affine", 2, 32), ("affine", 8, 128)])
+@pytest.mark.parametrize("N,K,Ms", [(256, 256, (1, 127, 128)), (300, 512, (129, 200)),
+                                    (1000, 1024, (64, 256)), (40, 768, (300,))])
+def test_gemm_small(cuda, fmt, bits, group, N, K, Ms):
+    L = Layer(fmt, N, K, seed=N + 5 * K, bits=bits, group=group)
+    w_ref = L.oracle_w()
+    for M in Ms:
+        xb, xd = x_dev(K, M, seed=M + 1)
+        y = run_gemm(L, xd, M)
+        assert_close(y, OC.matmul_f64(xb, w_ref), f"gemm {fmt} N={N} K={K} M={M}")
+
+
+def _sampled_rows(N, count, seed):
+    rng = np.random.default_rng(seed)
+    rows = np.unique(np.concatenate([[0, N - 1], rng.choice(N, size=min(count, N), replace=False)]))
+    return rows
+
+
+@pytest.mark.parametrize("name", ["int4_gemv_2048x2048", "int4_gemv_k5120_n27648", "int4_gemv_k27648_n5120",
+                                  "int6_gemv_k5120_n5120", "int6_gemv_k5120_n27648",
+                                  "affine2_k4096_n14336", "affine4_k4096_n14336", "affine8_k4096_n14336"])
+def test_gemv_full_size_sampled(cuda, name):
+    wl = synth.WORKLOADS[name]
+    L = Layer(wl.fmt, wl.N, wl.K, wl.seed, wl.bits, wl.group)
+    # packed bytes of the full layer are bit-exact
+    got = L.packed_host()
+    want = L.oracle_pack()
+    for a, b in zip(got, want):
+        if b is not None:
+            assert np.array_equal(a, b)
+    rows = _sampled_rows(wl.N, 384, wl.seed)
+    w_ref = L.oracle_w(rows)
+    xb8 = wl.x(max(wl.Ms))
+    for M in wl.Ms:
+        xd = dev(xb8[:M])
+        y = run_gemv(L, xd, M)
+        y_ref = OC.matmul_f64(xb8[:M], w_ref)
+        assert_close(y[:, rows], y_ref, f"gemv {name} M={M}")
+
+
+@pytest.mark.parametrize("M", [512, 2048, 8192])
+def test_gemm_full_size_sampled(cuda, M):
+    wl = synth.WORKLOADS["int4_gemm_k5120_n27648"]
+    L = Layer(wl.fmt, wl.N, wl.K, wl.seed)
+    rows = _sampled_rows(wl.N, 192, M)
+    w_ref = L.oracle_w(rows)
+    xb = wl.x(M)
+    y = run_gemm(L, dev(xb), M)
+    toks = _sampled_rows(M, 96, M + 1)
+    y_ref = OC.matmul_f64(xb[toks], w_ref)
+    assert_close(y[np.ix_(toks, rows)], y_ref, f"gemm full M={M}")
+
+
+def test_gemm_matches_bf16_dequant_matmul(cuda):
+    """The GEMM contracts the bf16-rounded exact weights: compare with a bf16-weight fp64 product."""
+    L = Layer("int4", 512, 1024, seed=77)
+    w16 = torch.empty((512, 1024), dtype=torch.bfloat16, device="cuda")
+    ql.qlinear_dequant(L.desc, *L.packed(), w16, ql.QL_OUT_BF16)
+    wb = host(w16.view(torch.int16), np.uint16)
+    w_bf = (wb.astype(np.uint32) << 16).view(np.float32)
+    xb, xd = x_dev(1024, 256, seed=9)
+    y = run_gemm(L, xd, 256)
+    ref = OC.matmul_f64(xb, w_bf)
+    y64 = (y.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    # only accumulation order and the final rounding differ
+    assert np.all(np.abs(y64 - ref) <= 1e-4 * np.sqrt(np.mean(ref ** 2)) + 2 * 2.0 ** (
+        np.floor(np.log2(np.maximum(np.abs(ref), 1e-30))) - 8))
+
+
+def test_deterministic_and_in_bounds(cuda):
+    """Two runs give identical bits; sentinel bytes around the output are untouched."""
+    L = Layer("int4", 1000, 2048, seed=5)
+    for runner, M in ((run_gemv, 3), (run_gemm, 200)):
+        xb, xd = x_dev(2048, M, seed=2)
+        pad = 4096
+        buf = torch.full((pad + M * 1000 + pad,), 0x7B7B, dtype=torch.int16, device="cuda")
+        y = buf[pad:pad + M * 1000].view(torch.bfloat16).view(M, 1000)
+        fn = ql.qlinear_gemv if runner is run_gemv else ql.qlinear_gemm
+        fn(L.desc, *L.packed(), xd, M, y)
+        first = host(y.view(torch.int16).clone(), np.uint16)
+        fn(L.desc, *L.packed(), xd, M, y)
+        assert ql.qlinear_sync_status() == ql.QL_OK
+        assert np.array_equal(first, host(y.view(torch.int16), np.uint16))
+        b = host(buf, np.uint16)
+        assert np.all(b[:pad] == 0x7B7B) and np.all(b[pad + M * 1000:] == 0x7B7B)
+
+
+def test_device_errors_do_not_launch(cuda):
+    L = Layer("int4", 64, 256, seed=1)
+    xd = x_dev(256, 1, 1)[1]
+    y = torch.empty((1, 64), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(ql.QLinearError) as e:
+        ql.qlinear_gemv(L.desc, *L.packed(), xd, 9, y)
+    assert e.value.status == ql.QL_ERR_RANGE
+    with pytest.raises(ql.QLinearError) as e:
+        ql.qlinear_gemv(L.desc, L.codes[1:], L.gmeta, L.steps, xd, 1, y)
+    assert e.value.status == ql.QL_ERR_ALIGN
+    assert ql.qlinear_sync_status() == ql.QL_OK
