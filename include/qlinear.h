@@ -46,9 +46,9 @@
  *  affine: w = f32(q)*f32(scale) + f32(bias)
  *
  * Conventions for every entry point:
- *  - Ownership: the caller allocates and frees every buffer; pointers are
- *    device pointers unless stated otherwise.  The library allocates no
- *    device memory in any call.  It keeps one small static device status
+ *  - Ownership: the caller allocates and frees every buffer (including the
+ *    GEMM's workspace); pointers are device pointers unless stated
+ *    otherwise.  The library allocates no device memory in any call.  It keeps one small static device status
  *    word per device and a host-side cache of kernel attributes.
  *  - Asynchrony: calls enqueue work on `stream` and return without
  *    synchronising (qlinear_sync_status excepted).
@@ -180,14 +180,34 @@ ql_status qlinear_dequant(const ql_desc *desc, const ql_packed_const *w,
 ql_status qlinear_gemv(const ql_desc *desc, const ql_packed_const *w,
                        const void *x, int64_t M, void *y, ql_stream_t stream);
 
+/* Bytes of caller-provided device workspace qlinear_gemm needs for `desc`
+ * and M (host-only, no CUDA call): 2*M*K for the fp16 copy of x, plus
+ * 4*M + 8*ceil(N/256)*256 for the per-row scales, each part rounded up to
+ * 256 bytes.  Errors: QL_ERR_NULL, QL_ERR_SHAPE, QL_ERR_RANGE,
+ * QL_ERR_UNSUPPORTED. */
+ql_status qlinear_gemm_workspace_bytes(const ql_desc *desc, int64_t M, size_t *bytes);
+
 /* Prefill-shaped layer on the tcgen05 tensor cores: same result definition
- * as qlinear_gemv, any M >= 1 (meant for M >= 128).  Weights are
- * dequantised once per tile to bf16 (one rounding of the exact binary32
- * weight) and contracted with x in bf16 with fp32 accumulation in tensor
- * memory.  Requires an sm_100 device.
- * Errors: as qlinear_gemv, plus QL_ERR_UNSUPPORTED off sm_100. */
+ * as qlinear_gemv, any M >= 1 (meant for M >= 128).  Three launches on
+ * `stream`: (1) x is scaled per token row by a power of two 2^a_m that puts
+ * the row's max |x| in [2^15, 2^16) and stored as fp16 in the workspace
+ * (exact for every value within 2^29 of the row maximum); (2) each weight
+ * row gets a power of two 2^b_n from a metadata bound on its max |w|;
+ * (3) the persistent GEMM dequantises each weight once per tile to its exact
+ * binary32 value, scales it by 2^b_n and rounds it once to fp16, contracts
+ * with fp32 accumulation in tensor memory, and stores
+ * RN_bf16(acc * 2^-a_m * 2^-b_n).  fp16 operands rather than bf16 keep the
+ * weight rounding at ~0.1% of rms(y) instead of ~1%.
+ * `workspace`: device memory of at least qlinear_gemm_workspace_bytes(),
+ * 256-byte aligned, owned by the caller, overwritten; calls sharing one
+ * workspace must not overlap on the GPU.  K % 64 == 0.  Requires an sm_100
+ * device.
+ * Errors: QL_ERR_NULL, QL_ERR_SHAPE (also: workspace too small),
+ * QL_ERR_ALIGN, QL_ERR_RANGE, QL_ERR_UNSUPPORTED (format or device),
+ * QL_ERR_CUDA. */
 ql_status qlinear_gemm(const ql_desc *desc, const ql_packed_const *w,
-                       const void *x, int64_t M, void *y, ql_stream_t stream);
+                       const void *x, int64_t M, void *y, void *workspace,
+                       size_t workspace_bytes, ql_stream_t stream);
 
 /* Synchronise `stream`, then read and clear the current device's status
  * word: QL_ERR_TIMEOUT if a kernel's bounded wait gave up since the last

@@ -117,7 +117,7 @@ QL_DEVI void tmem_dealloc(uint32_t taddr, uint32_t ncols) {  // whole warp
 QL_DEVI void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 QL_DEVI void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-// D[tmem] (+)= A[smem desc] * B[smem desc]^T, kind::f16 (bf16 inputs, f32 accumulate).
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T, kind::f16 (16-bit inputs, f32 accumulate).
 QL_DEVI void umma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
@@ -163,11 +163,12 @@ QL_DEVI uint64_t umma_desc_k_sw128(uint32_t smem_addr) {
   return d;
 }
 
-// Instruction descriptor, kind::f16: D f32, A bf16, B bf16, both K-major.
-__host__ __device__ constexpr uint32_t umma_idesc_bf16_f32(int M, int N) {
+// Instruction descriptor, kind::f16: D f32, A and B both f16 (format 0),
+// both K-major.
+__host__ __device__ constexpr uint32_t umma_idesc_f16_f32(int M, int N) {
   return (1u << 4)                      // D format: f32
-         | (1u << 7)                    // A format: bf16
-         | (1u << 10)                   // B format: bf16
+         | (0u << 7)                    // A format: f16
+         | (0u << 10)                   // B format: f16
          | ((uint32_t)(N >> 3) << 17)   // N / 8
          | ((uint32_t)(M >> 4) << 24);  // M / 16
 }
@@ -177,6 +178,10 @@ __host__ __device__ constexpr uint32_t umma_idesc_bf16_f32(int M, int N) {
 // ---------------------------------------------------------------------------
 QL_DEVI float f16_bits_to_f32(uint32_t h) { return __half2float(__ushort_as_half((unsigned short)(h & 0xffff))); }
 QL_DEVI float bf16_bits_to_f32(uint32_t b) { return __uint_as_float((b & 0xffffu) << 16); }
+QL_DEVI uint32_t pack_f16x2(float lo, float hi) {  // nearest-even, lo in the low half
+  __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&v);
+}
 QL_DEVI uint32_t pack_bf16x2(float lo, float hi) {  // nearest-even, lo in the low half
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t *>(&v);

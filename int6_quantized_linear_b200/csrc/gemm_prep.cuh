@@ -1,0 +1,145 @@
+// gemm_prep.cuh -- the two short passes that let the tensor-core GEMM run on
+// fp16 operands without giving up fp32 range.
+//
+// fp16 keeps 11 significant bits (bf16 keeps 8); rounding each weight to bf16
+// alone puts the layer's error near 1% of rms(y), fp16 brings it to ~0.1%.
+// fp16's range is what needs care, so both operands are scaled by exact
+// powers of two that the epilogue undoes:
+//
+//  x:  a_m per token row, chosen so max_k |x[m][k]| * 2^a_m lies in
+//      [2^15, 2^16).  A bf16 value scaled into that range is exactly an fp16
+//      value unless it is more than 2^29 below the row's maximum.
+//  W:  b_n per weight row, chosen so a bound on max_k |w[n][k]| times 2^b_n
+//      lies in [2^14, 2^15) (headroom for the rounding to fp16).  The bound
+//      comes from the metadata alone:  int4 |S|*max(|Z|, |15-Z|),
+//      int6 32*|S|,  affine max(|bias|, |(2^bits-1)*scale + bias|).
+//
+// Workspace layout (caller-provided, 256-byte aligned sections):
+//   x16   fp16 [M][K]   scaled activations
+//   xinv  f32  [M]      2^-a_m
+//   wsc   f32  [N']     2^b_n   (N' = N rounded up to 256; the tail is unused)
+//   winv  f32  [N']     2^-b_n
+#pragma once
+#include "formats.cuh"
+
+namespace ql {
+
+inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+struct GemmWorkspace {
+  __half *x16;
+  float *xinv;
+  float *wsc;
+  float *winv;
+};
+
+// the per-row weight scales are padded to whole 256-row tiles
+inline size_t padded_rows(int64_t N) { return (size_t)((N + 255) / 256 * 256); }
+
+inline size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  return align256((size_t)M * K * 2) + align256((size_t)M * 4) + 2 * align256(padded_rows(N) * 4);
+}
+
+inline GemmWorkspace gemm_workspace_carve(void *base, int64_t M, int64_t N, int64_t K) {
+  uint8_t *p = static_cast<uint8_t *>(base);
+  GemmWorkspace w;
+  w.x16 = reinterpret_cast<__half *>(p);
+  p += align256((size_t)M * K * 2);
+  w.xinv = reinterpret_cast<float *>(p);
+  p += align256((size_t)M * 4);
+  w.wsc = reinterpret_cast<float *>(p);
+  p += align256(padded_rows(N) * 4);
+  w.winv = reinterpret_cast<float *>(p);
+  return w;
+}
+
+// 2^e as a binary32 for e in [-126, 127]
+QL_DEVI float exp2i(int e) { return __int_as_float((e + 127) << 23); }
+
+// Exponent that puts amax * 2^s into [2^top, 2^(top+1)); 0 for zero or non-finite.
+QL_DEVI int scale_exponent(float amax, int top) {
+  if (!(amax > 0.f) || !isfinite(amax)) return 0;
+  int e = ((__float_as_int(amax) >> 23) & 0xff) - 127;  // floor(log2(amax)) for normal amax
+  if (e == -127) e = -118 - __clz(__float_as_int(amax) & 0x7fffff);  // subnormal: m * 2^-149
+  int s = top - e;
+  return s < -126 ? -126 : (s > 126 ? 126 : s);
+}
+
+// One warp per token row: find max|x|, then write the scaled fp16 row.
+__global__ void __launch_bounds__(256) x_to_f16_kernel(const __nv_bfloat16 *x, int64_t M, int64_t K,
+                                                        GemmWorkspace ws) {
+  const int lane = threadIdx.x & 31;
+  const int64_t m = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+  if (m >= M) return;
+  const uint4 *row = reinterpret_cast<const uint4 *>(x + m * K);
+  const int64_t nv = K / 8;  // 16-byte vectors
+  float amax = 0.f;
+  for (int64_t i = lane; i < nv; i += 32) {
+    const uint4 v = __ldg(row + i);
+    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(u[j] << 16)), fabsf(__uint_as_float(u[j] & 0xffff0000u))));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  const int a = scale_exponent(amax, 15);
+  const float sc = exp2i(a);
+  uint4 *out = reinterpret_cast<uint4 *>(ws.x16 + m * K);
+  for (int64_t i = lane; i < nv; i += 32) {
+    const uint4 v = __ldg(row + i);
+    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const __half2 h = __floats2half2_rn(__uint_as_float(u[j] << 16) * sc, __uint_as_float(u[j] & 0xffff0000u) * sc);
+      o[j] = *reinterpret_cast<const uint32_t *>(&h);
+    }
+    out[i] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+  if (lane == 0) ws.xinv[m] = exp2i(-a);
+}
+
+// One thread per weight row: bound max|w| from the metadata, pick b_n.
+template <int FMT, int BITS>
+__global__ void __launch_bounds__(256) w_scale_kernel(const uint8_t *gmeta, const uint8_t *steps, int64_t N,
+                                                       int64_t K, int G, GemmWorkspace ws) {
+  const int64_t n = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (n >= N) return;
+  float bound = 0.f;
+  if constexpr (FMT == FMT_INT4) {
+    const uint16_t *gm = reinterpret_cast<const uint16_t *>(gmeta) + n * (K / 32);
+    const uint32_t *st = reinterpret_cast<const uint32_t *>(steps) + n * (K / 256);
+    for (int64_t j = 0; j < K / 256; ++j) {
+      const uint32_t s = __ldg(st + j);
+      const float ss = f16_bits_to_f32(s), zs = f16_bits_to_f32(s >> 16);
+      for (int g = 0; g < 8; ++g) {
+        const uint32_t c = __ldg(gm + 8 * j + g);
+        const float S = __fmul_rn((float)(c & 0xffu), ss);
+        const float Z = __fmul_rn((float)(c >> 8), zs);
+        bound = fmaxf(bound, __fmul_rn(fabsf(S), fmaxf(fabsf(Z), fabsf(__fsub_rn(15.f, Z)))));
+      }
+    }
+  } else if constexpr (FMT == FMT_INT6) {
+    const int8_t *gm = reinterpret_cast<const int8_t *>(gmeta) + n * (K / 16);
+    const uint16_t *st = reinterpret_cast<const uint16_t *>(steps) + n * (K / 256);
+    for (int64_t j = 0; j < K / 256; ++j) {
+      const float step = f16_bits_to_f32(__ldg(st + j));
+      for (int g = 0; g < 16; ++g)
+        bound = fmaxf(bound, __fmul_rn(32.f, fabsf(__fmul_rn((float)__ldg(gm + 16 * j + g), step))));
+    }
+  } else {
+    const uint32_t *gm = reinterpret_cast<const uint32_t *>(gmeta) + n * (K / G);
+    const float qmax = (float)((1 << BITS) - 1);
+    for (int64_t g = 0; g < K / G; ++g) {
+      const uint32_t c = __ldg(gm + g);
+      const float s = bf16_bits_to_f32(c), b = bf16_bits_to_f32(c >> 16);
+      bound = fmaxf(bound, fmaxf(fabsf(b), fabsf(__fadd_rn(__fmul_rn(qmax, s), b))));
+    }
+  }
+  const int e = scale_exponent(bound, 14);
+  ws.wsc[n] = exp2i(e);
+  ws.winv[n] = exp2i(-e);
+}
+
+}  // namespace ql

@@ -5,19 +5,24 @@
 // Persistent kernel, one CTA per SM, tiles of BM=128 tokens x BN=256 weight
 // rows, K streamed in BK=64 steps through a STAGES-deep shared-memory ring.
 // Warp roles:
-//   warp 0      TMA producer: x tile (128 x 64 bf16, 128-byte swizzle) and the
-//               packed code tile (256 rows x BK codes) per stage
+//   warp 0      TMA producer: scaled fp16 x tile (128 x 64, 128-byte
+//               swizzle) and the packed code tile (256 rows x BK codes)
 //   warp 1      TMEM allocator; lane 0 issues tcgen05.mma (M=128, N=256,
-//               K=16, bf16 x bf16 -> f32) into one of two TMEM accumulators
+//               K=16, f16 x f16 -> f32) into one of two TMEM accumulators
 //   warps 4-7   epilogue: tcgen05.ld the accumulator (warp w reads TMEM lanes
-//               32*(w%4)..), round to bf16, store y
+//               32*(w%4)..), undo the two power-of-two scales, round to bf16,
+//               store y
 //   warps 8-15  dequantisers: packed codes (shared) + metadata (global, one
-//               stage ahead) -> exact binary32 weight -> nearest-even bf16,
-//               written in the canonical K-major 128-byte-swizzled layout the
-//               MMA reads as its B operand
+//               stage ahead) -> exact binary32 weight -> times 2^b_n (exact)
+//               -> nearest-even fp16, written in the canonical K-major
+//               128-byte-swizzled layout the MMA reads as its B operand
+// The operands are fp16 rather than bf16 because rounding every weight to
+// bf16 costs ~1% of rms(y); fp16 costs ~0.1% (see gemm_prep.cuh for the
+// scaling that keeps fp32 range).
 // Every mbarrier wait is bounded; a wait that gives up sets the device status
 // word and makes every role leave its loop.
 #pragma once
+#include "gemm_prep.cuh"
 #include "pack_dequant.cuh"
 
 namespace ql {
@@ -64,6 +69,7 @@ struct Params {
   const uint8_t *gmeta;
   const uint8_t *steps;
   __nv_bfloat16 *y;
+  GemmWorkspace ws;
 };
 
 // Metadata of one 32-weight chunk (see formats.cuh): int4 (gm, st); int6
@@ -192,7 +198,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else if (warp == WARP_MMA) {
     if (lane == 0) {
-      constexpr uint32_t idesc = umma_idesc_bf16_f32(BM, BN);
+      constexpr uint32_t idesc = umma_idesc_f16_f32(BM, BN);
       int64_t it = 0, tcount = 0;
       bool ok = true, issued = false;
       for (int64_t tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++tcount) {
@@ -239,12 +245,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!mbar_wait_bounded(bar_acc_full(a), ause & 1, abort_flag)) break;
       tc_fence_after();
       const int64_t m = m_tile * BM + 32 * e + lane;
+      const float xs = m < p.M ? p.ws.xinv[m] : 0.f;
 #pragma unroll 1
       for (int cchunk = 0; cchunk < BN / 32; ++cchunk) {
         uint32_t r[32];
         tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(32 * e) << 16) + (uint32_t)(a * BN + 32 * cchunk), r);
         tmem_ld_wait();
         const int64_t n0 = n_tile * BN + 32 * cchunk;
+        {  // y = D * 2^-a_m * 2^-b_n, both exact power-of-two multiplications
+          const float4 *wi = reinterpret_cast<const float4 *>(p.ws.winv + n0);
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            const float4 v = wi[t];
+            r[4 * t + 0] = __float_as_uint(__uint_as_float(r[4 * t + 0]) * xs * v.x);
+            r[4 * t + 1] = __float_as_uint(__uint_as_float(r[4 * t + 1]) * xs * v.y);
+            r[4 * t + 2] = __float_as_uint(__uint_as_float(r[4 * t + 2]) * xs * v.z);
+            r[4 * t + 3] = __float_as_uint(__uint_as_float(r[4 * t + 3]) * xs * v.w);
+          }
+        }
         if (m < p.M) {
           __nv_bfloat16 *dst = p.y + m * p.N + n0;
           if (vec_ok && n0 + 32 <= p.N) {
@@ -275,19 +293,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int64_t my_tiles = (num_tiles - blockIdx.x + gridDim.x - 1) / gridDim.x;
     const int64_t total_it = my_tiles * num_kb;
     auto tile_of = [&](int64_t i) { return (int64_t)blockIdx.x + (i / num_kb) * gridDim.x; };
+    auto row_scale = [&](int64_t n) { return n < p.N ? p.ws.wsc[n] : 0.f; };
     uint32_t gm0 = 0, st0 = 0, gm1 = 0, st1 = 0;
+    float sc0 = 0.f, sc1 = 0.f;
     if (total_it > 0) {
       const int64_t n_tile = tile_of(0) / m_tiles;
       load_meta<FMT>(p, n_tile * BN + r0, h, gm0, st0);
       load_meta<FMT>(p, n_tile * BN + r1, h, gm1, st1);
+      sc0 = row_scale(n_tile * BN + r0);
+      sc1 = row_scale(n_tile * BN + r1);
     }
     for (; it < total_it; ++it) {
       uint32_t ngm0 = 0, nst0 = 0, ngm1 = 0, nst1 = 0;
+      float nsc0 = sc0, nsc1 = sc1;
       if (it + 1 < total_it) {  // prefetch the next stage's metadata
         const int64_t n_tile = tile_of(it + 1) / m_tiles;
         const int64_t c = (int64_t)((it + 1) % num_kb) * (BK / 32) + h;
         load_meta<FMT>(p, n_tile * BN + r0, c, ngm0, nst0);
         load_meta<FMT>(p, n_tile * BN + r1, c, ngm1, nst1);
+        if ((it + 1) % num_kb == 0) {
+          nsc0 = row_scale(n_tile * BN + r0);
+          nsc1 = row_scale(n_tile * BN + r1);
+        }
       }
       const int s = (int)(it % STAGES);
       if (!mbar_wait_bounded(bar_tma_full(s), (uint32_t)((it / STAGES) & 1), abort_flag)) break;
@@ -298,15 +325,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int r = rr ? r1 : r0;
         float w[32];
         smem_decode32<FMT, BITS>(P + r * PROW + h * (PROW / 2), rr ? gm1 : gm0, rr ? st1 : st0, w);
+        const float sc = rr ? sc1 : sc0;
         uint8_t *row = B + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const int j = 4 * h + q;  // logical 16-byte chunk of the 128-byte row
           uint4 v;
-          v.x = pack_bf16x2(w[8 * q + 0], w[8 * q + 1]);
-          v.y = pack_bf16x2(w[8 * q + 2], w[8 * q + 3]);
-          v.z = pack_bf16x2(w[8 * q + 4], w[8 * q + 5]);
-          v.w = pack_bf16x2(w[8 * q + 6], w[8 * q + 7]);
+          v.x = pack_f16x2(w[8 * q + 0] * sc, w[8 * q + 1] * sc);
+          v.y = pack_f16x2(w[8 * q + 2] * sc, w[8 * q + 3] * sc);
+          v.z = pack_f16x2(w[8 * q + 4] * sc, w[8 * q + 5] * sc);
+          v.w = pack_f16x2(w[8 * q + 6] * sc, w[8 * q + 7] * sc);
           *reinterpret_cast<uint4 *>(row + ((j ^ (r & 7)) << 4)) = v;
         }
       }
@@ -314,6 +342,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       __syncwarp();
       if ((t & 31) == 0) mbar_arrive(bar_b_full(s));
       gm0 = ngm0; st0 = nst0; gm1 = ngm1; st1 = nst1;
+      sc0 = nsc0; sc1 = nsc1;
     }
   }
 

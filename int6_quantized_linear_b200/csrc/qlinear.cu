@@ -126,12 +126,17 @@ bool encode_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint6
 
 template <int FMT, int BITS>
 ql_status launch_gemm(const ql_desc *d, const ql_packed_const *w, const void *x, int64_t M, void *y,
-                      cudaStream_t st, int sms) {
+                      void *workspace, cudaStream_t st, int sms) {
   using namespace ql::gemm;
   const int64_t N = d->N, K = d->K;
   const uint64_t row_bytes = (uint64_t)K * code_bits(FMT, BITS) / 8;
+  const GemmWorkspace ws = gemm_workspace_carve(workspace, M, N, K);
+  // pass 1: scaled fp16 activations; pass 2: per-row weight scales
+  x_to_f16_kernel<<<(int)((M * 32 + 255) / 256), 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(x), M, K, ws);
+  w_scale_kernel<FMT, BITS><<<(int)((N + 255) / 256), 256, 0, st>>>(
+      static_cast<const uint8_t *>(w->gmeta), static_cast<const uint8_t *>(w->steps), N, K, d->group, ws);
   CUtensorMap mx, mc;
-  if (!encode_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, BK, BM,
+  if (!encode_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws.x16, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, BK, BM,
                  CU_TENSOR_MAP_SWIZZLE_128B))
     return QL_ERR_CUDA;
   if (!encode_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->codes, row_bytes, (uint64_t)N, row_bytes,
@@ -142,6 +147,7 @@ ql_status launch_gemm(const ql_desc *d, const ql_packed_const *w, const void *x,
   p.gmeta = static_cast<const uint8_t *>(w->gmeta);
   p.steps = static_cast<const uint8_t *>(w->steps);
   p.y = static_cast<__nv_bfloat16 *>(y);
+  p.ws = ws;
   const int smem = smem_bytes(FMT, BITS);
   auto kern = gemm_kernel<FMT, BITS>;
   static thread_local int configured_dev = -1;  // per (kernel instantiation, thread)
@@ -334,26 +340,36 @@ ql_status qlinear_gemv(const ql_desc *d, const ql_packed_const *w, const void *x
   }
 }
 
+ql_status qlinear_gemm_workspace_bytes(const ql_desc *d, int64_t M, size_t *bytes) {
+  const ql_status st = check_desc(d);
+  if (st != QL_OK) return st;
+  if (!bytes) return QL_ERR_NULL;
+  if (M < 1 || M > (int64_t)INT32_MAX) return QL_ERR_RANGE;
+  *bytes = gemm_workspace_bytes(M, d->N, d->K);
+  return QL_OK;
+}
+
 ql_status qlinear_gemm(const ql_desc *d, const ql_packed_const *w, const void *x, int64_t M, void *y,
-                       ql_stream_t stream) {
+                       void *workspace, size_t workspace_bytes, ql_stream_t stream) {
   ql_status st = check_desc(d);
   if (st != QL_OK) return st;
-  if (!w || !x || !y) return QL_ERR_NULL;
+  if (!w || !x || !y || !workspace) return QL_ERR_NULL;
   if ((st = check_packed(d, w->codes, w->gmeta, w->steps)) != QL_OK) return st;
-  if (!aligned16(x) || !aligned16(y)) return QL_ERR_ALIGN;
+  if (!aligned16(x) || !aligned16(y) || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return QL_ERR_ALIGN;
   if (M < 1 || M > (int64_t)INT32_MAX) return QL_ERR_RANGE;
   if (d->K % gemm::BK != 0 || d->N > (int64_t)INT32_MAX) return QL_ERR_SHAPE;
+  if (workspace_bytes < gemm_workspace_bytes(M, d->N, d->K)) return QL_ERR_SHAPE;
   DeviceInfo *di;
   if ((st = device_info(&di)) != QL_OK) return st;
   if (di->major != 10) return QL_ERR_UNSUPPORTED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   switch (d->fmt) {
-    case QL_INT4_NSS: return launch_gemm<FMT_INT4, 4>(d, w, x, M, y, s, di->sms);
-    case QL_INT6_SYM: return launch_gemm<FMT_INT6, 6>(d, w, x, M, y, s, di->sms);
+    case QL_INT4_NSS: return launch_gemm<FMT_INT4, 4>(d, w, x, M, y, workspace, s, di->sms);
+    case QL_INT6_SYM: return launch_gemm<FMT_INT6, 6>(d, w, x, M, y, workspace, s, di->sms);
     default:
-      if (d->bits == 2) return launch_gemm<FMT_AFFINE, 2>(d, w, x, M, y, s, di->sms);
-      if (d->bits == 4) return launch_gemm<FMT_AFFINE, 4>(d, w, x, M, y, s, di->sms);
-      return launch_gemm<FMT_AFFINE, 8>(d, w, x, M, y, s, di->sms);
+      if (d->bits == 2) return launch_gemm<FMT_AFFINE, 2>(d, w, x, M, y, workspace, s, di->sms);
+      if (d->bits == 4) return launch_gemm<FMT_AFFINE, 4>(d, w, x, M, y, workspace, s, di->sms);
+      return launch_gemm<FMT_AFFINE, 8>(d, w, x, M, y, workspace, s, di->sms);
   }
 }
 

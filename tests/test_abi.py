@@ -32,7 +32,8 @@ def declared_functions():
 def test_header_declares_the_boundary():
     names = declared_functions()
     for required in ("qlinear_pack", "qlinear_dequant", "qlinear_gemv", "qlinear_gemm",
-                     "qlinear_packed_bytes", "qlinear_status_string", "qlinear_sync_status"):
+                     "qlinear_packed_bytes", "qlinear_status_string", "qlinear_sync_status",
+                     "qlinear_gemm_workspace_bytes"):
         assert required in names
 
 
@@ -97,7 +98,11 @@ def test_host_validation_before_any_launch(lib):
     assert _call_gemv(lib, da, A, A, None, A, 33, A) == ql.QL_ERR_RANGE
     bad = ql.ql_desc(9, 0, 0, 0, 8, 256)
     w = ql.ql_packed(A, A, A)
-    assert lib.qlinear_gemm(C.byref(bad), C.byref(w), A, 1, A, None) == ql.QL_ERR_UNSUPPORTED
+    assert lib.qlinear_gemm(C.byref(bad), C.byref(w), A, 1, A, A, 1 << 20, None) == ql.QL_ERR_UNSUPPORTED
+    d2 = ql.Desc("int4", 8, 256).c()
+    assert lib.qlinear_gemm(C.byref(d2), C.byref(w), A, 1, A, A, 16, None) == ql.QL_ERR_SHAPE  # workspace too small
+    assert lib.qlinear_gemm(C.byref(d2), C.byref(w), A, 1, A, A + 16, 1 << 20, None) == ql.QL_ERR_ALIGN
+    assert ql.qlinear_gemm_workspace_bytes(ql.Desc("int4", 300, 512), 3) == 3 * 512 * 2 + 256 + 2 * 512 * 4 + (256 - 3 * 512 * 2 % 256) % 256
     for s in range(8):
         assert isinstance(ql.status_string(s), str) and ql.status_string(s)
     assert lib.qlinear_version() >= 1

@@ -116,20 +116,15 @@ def test_gemm_full_size_sampled(cuda, M):
     assert_close(y[np.ix_(toks, rows)], y_ref, f"gemm full M={M}")
 
 
-def test_gemm_matches_bf16_dequant_matmul(cuda):
-    """The GEMM contracts the bf16-rounded exact weights: compare with a bf16-weight fp64 product."""
-    L = Layer("int4", 512, 1024, seed=77)
-    w16 = torch.empty((512, 1024), dtype=torch.bfloat16, device="cuda")
-    ql.qlinear_dequant(L.desc, *L.packed(), w16, ql.QL_OUT_BF16)
-    wb = host(w16.view(torch.int16), np.uint16)
-    w_bf = (wb.astype(np.uint32) << 16).view(np.float32)
-    xb, xd = x_dev(1024, 256, seed=9)
+def test_gemm_error_budget(cuda):
+    """fp16 operands with per-row power-of-two scales: the only rounding beyond fp32 accumulation is
+    one 11-bit rounding per weight, so the error stays far inside the gate (bf16 weights would use ~100%)."""
+    L = Layer("int4", 1024, 2048, seed=77)
+    w_ref = L.oracle_w()
+    xb, xd = x_dev(2048, 256, seed=9)
     y = run_gemm(L, xd, 256)
-    ref = OC.matmul_f64(xb, w_bf)
-    y64 = (y.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
-    # only accumulation order and the final rounding differ
-    assert np.all(np.abs(y64 - ref) <= 1e-4 * np.sqrt(np.mean(ref ** 2)) + 2 * 2.0 ** (
-        np.floor(np.log2(np.maximum(np.abs(ref), 1e-30))) - 8))
+    used = assert_close(y, OC.matmul_f64(xb, w_ref), "gemm budget")
+    assert used < 3e-3, used
 
 
 def test_deterministic_and_in_bounds(cuda):
