@@ -209,6 +209,29 @@ ql_status qlinear_gemm(const ql_desc *desc, const ql_packed_const *w,
                        const void *x, int64_t M, void *y, void *workspace,
                        size_t workspace_bytes, ql_stream_t stream);
 
+/* qlinear_gemm for callers that may not allocate device memory at all --
+ * e.g. an op behind a runtime's plug-in interface, which receives its input
+ * and output pointers but no allocator, or a serving process that has
+ * reserved all of HBM for its own pool, where cudaMalloc would fail or stall
+ * the device.  (The pages describe no such entry point; it serves deployment
+ * only.)  Same arguments, result and errors as qlinear_gemm, minus the
+ * workspace: the library takes it from one fixed 32 MiB array in device
+ * memory that exists on every GPU that loads the library, until the process
+ * exits.  No call allocates or frees anything.
+ *  - Limit: the call is accepted while qlinear_gemm_workspace_bytes(desc, M)
+ *    is at most 33554432 bytes (about M*K <= 16.7 million for small N);
+ *    larger problems return QL_ERR_RANGE before anything is enqueued.
+ *  - The first call on a device looks up that device's address of the array
+ *    (cudaGetSymbolAddress, with the device current) and caches it; make that
+ *    first call before any stream capture.
+ *  - All calls on a device share the one array, which keeps whatever the last
+ *    call left in it; nothing in it needs to start at zero, because each call
+ *    writes every element it later reads.  Calls whose work overlaps on the
+ *    GPU (other streams, or other threads) race on the array: order them. */
+ql_status qlinear_gemm_noalloc(const ql_desc *desc, const ql_packed_const *w,
+                               const void *x, int64_t M, void *y,
+                               ql_stream_t stream);
+
 /* Synchronise `stream`, then read and clear the current device's status
  * word: QL_ERR_TIMEOUT if a kernel's bounded wait gave up since the last
  * call, QL_ERR_CUDA if the synchronisation failed, else QL_OK. */

@@ -62,6 +62,8 @@ _SIGNATURES = {
     "qlinear_gemm_workspace_bytes": ([C.POINTER(ql_desc), C.c_int64, C.POINTER(C.c_size_t)], C.c_int),
     "qlinear_gemm": ([C.POINTER(ql_desc), C.POINTER(ql_packed), C.c_void_p, C.c_int64, C.c_void_p, C.c_void_p,
                       C.c_size_t, C.c_void_p], C.c_int),
+    "qlinear_gemm_noalloc": ([C.POINTER(ql_desc), C.POINTER(ql_packed), C.c_void_p, C.c_int64, C.c_void_p,
+                              C.c_void_p], C.c_int),
     "qlinear_sync_status": ([C.c_void_p], C.c_int),
 }
 
@@ -183,6 +185,16 @@ def qlinear_gemm(desc: Desc, codes, gmeta, steps, x, M: int, y, workspace=None, 
     w = ql_packed(_ptr(codes), _ptr(gmeta), _ptr(steps))
     _check(lib().qlinear_gemm(C.byref(d), C.byref(w), _ptr(x), M, _ptr(y), _ptr(workspace),
                               workspace.numel() * workspace.element_size(), _stream(stream)), "qlinear_gemm")
+
+
+def qlinear_gemm_noalloc(desc: Desc, codes, gmeta, steps, x, M: int, y, stream=None):
+    """qlinear_gemm without a workspace argument, for callers that may not allocate device memory:
+    the library uses its own fixed 32 MiB device array (shared by every call on the device, so calls
+    must not overlap on the GPU).  Raises QLinearError(QL_ERR_RANGE) when the problem needs more."""
+    d = desc.c()
+    w = ql_packed(_ptr(codes), _ptr(gmeta), _ptr(steps))
+    _check(lib().qlinear_gemm_noalloc(C.byref(d), C.byref(w), _ptr(x), M, _ptr(y), _stream(stream)),
+           "qlinear_gemm_noalloc")
 
 
 def qlinear_sync_status(stream=None) -> int:

@@ -187,6 +187,36 @@ ql_status launch_gemv(const ql_desc *d, const ql_packed_const *w, const void *x,
 
 }  // namespace
 
+// ---- the GEMM for callers that cannot allocate -------------------------------
+// Some callers of this library may not allocate device memory at all: plug-in
+// and custom-op interfaces of inference runtimes hand an op its input and
+// output pointers but no allocator, and serving processes that reserve all of
+// HBM up front for their own pool would see cudaMalloc fail (or stall the
+// device while it synchronises).  qlinear_gemm_noalloc serves them with the
+// GEMM's workspace taken from this fixed device array instead.
+#define QL_NOALLOC_SCRATCH_BYTES (32u << 20)  // 32 MiB on every GPU that loads the library
+static __device__ __align__(256) unsigned char g_gemm_noalloc_scratch[QL_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+// Device address of g_gemm_noalloc_scratch per device.  In host code the
+// array's name is only a host-side stand-in, so the address is looked up once
+// per device (with that device current) and cached.
+void *g_noalloc_addr[kMaxDevices] = {};
+
+ql_status noalloc_scratch(void **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return QL_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_gemm_noalloc_scratch) != cudaSuccess || p == nullptr) return QL_ERR_CUDA;
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return QL_OK;
+}
+}  // namespace
+
 extern "C" {
 
 int32_t qlinear_version(void) { return 1; }
@@ -370,6 +400,32 @@ ql_status qlinear_gemm(const ql_desc *d, const ql_packed_const *w, const void *x
       if (d->bits == 2) return launch_gemm<FMT_AFFINE, 2>(d, w, x, M, y, workspace, s, di->sms);
       if (d->bits == 4) return launch_gemm<FMT_AFFINE, 4>(d, w, x, M, y, workspace, s, di->sms);
       return launch_gemm<FMT_AFFINE, 8>(d, w, x, M, y, workspace, s, di->sms);
+  }
+}
+
+ql_status qlinear_gemm_noalloc(const ql_desc *d, const ql_packed_const *w, const void *x, int64_t M, void *y,
+                               ql_stream_t stream) {
+  ql_status st = check_desc(d);
+  if (st != QL_OK) return st;
+  if (!w || !x || !y) return QL_ERR_NULL;
+  if ((st = check_packed(d, w->codes, w->gmeta, w->steps)) != QL_OK) return st;
+  if (!aligned16(x) || !aligned16(y)) return QL_ERR_ALIGN;
+  if (M < 1 || M > (int64_t)INT32_MAX) return QL_ERR_RANGE;
+  if (d->K % gemm::BK != 0 || d->N > (int64_t)INT32_MAX) return QL_ERR_SHAPE;
+  if (gemm_workspace_bytes(M, d->N, d->K) > (size_t)QL_NOALLOC_SCRATCH_BYTES) return QL_ERR_RANGE;
+  DeviceInfo *di;
+  if ((st = device_info(&di)) != QL_OK) return st;
+  if (di->major != 10) return QL_ERR_UNSUPPORTED;
+  void *scratch = nullptr;
+  if ((st = noalloc_scratch(&scratch)) != QL_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  switch (d->fmt) {
+    case QL_INT4_NSS: return launch_gemm<FMT_INT4, 4>(d, w, x, M, y, scratch, s, di->sms);
+    case QL_INT6_SYM: return launch_gemm<FMT_INT6, 6>(d, w, x, M, y, scratch, s, di->sms);
+    default:
+      if (d->bits == 2) return launch_gemm<FMT_AFFINE, 2>(d, w, x, M, y, scratch, s, di->sms);
+      if (d->bits == 4) return launch_gemm<FMT_AFFINE, 4>(d, w, x, M, y, scratch, s, di->sms);
+      return launch_gemm<FMT_AFFINE, 8>(d, w, x, M, y, scratch, s, di->sms);
   }
 }
 
