@@ -200,7 +200,8 @@ def build_layers(device, copies=COPIES):
         reps = [(c0, g0, s0)] + [(c0.clone(), g0.clone(), s0.clone()) for _ in range(copies - 1)]
         x = torch.from_numpy(synth.activations(1, 1, K).view("int16")).to(device).view(torch.bfloat16)
         y = torch.empty((1, N), dtype=torch.bfloat16, device=device)
-        layers.append(dict(desc=d, reps=reps, x=x, y=y, K=K, N=N))
+        ws = ql.alloc_gemv_workspace(d, 1, device)
+        layers.append(dict(desc=d, reps=reps, x=x, y=y, K=K, N=N, ws=ws))
     torch.cuda.synchronize(device)
     return layers
 
@@ -211,7 +212,7 @@ def gemv_step(layers, i: int, ql, events=None):
         if events is not None:
             events[0].append(_ev())
             events[0][-1].record()
-        ql.qlinear_gemv(L["desc"], c, g, s, L["x"], 1, L["y"])
+        ql.qlinear_gemv(L["desc"], c, g, s, L["x"], 1, L["y"], L["ws"])
         if events is not None:
             events[1].append(_ev())
             events[1][-1].record()
@@ -382,7 +383,7 @@ def run_e2e(args, layers, device, step_bytes):
         for L, xhost, yhost in zip(layers, xh, yh):
             c, g, s = L["reps"][i % len(L["reps"])]
             L["x"].copy_(xhost, non_blocking=True)
-            ql.qlinear_gemv(L["desc"], c, g, s, L["x"], 1, L["y"])
+            ql.qlinear_gemv(L["desc"], c, g, s, L["x"], 1, L["y"], L["ws"])
             yhost.copy_(L["y"], non_blocking=True)
 
     for i in range(args.warmup):

@@ -169,16 +169,34 @@ ql_status qlinear_unpack(const ql_desc *desc, const ql_packed_const *in,
 ql_status qlinear_dequant(const ql_desc *desc, const ql_packed_const *w,
                           void *out, int32_t out_dtype, ql_stream_t stream);
 
+/* Bytes of caller-provided device workspace qlinear_gemv needs for `desc`
+ * and M (host-only, no CUDA call): 2*M*K for x in the order the kernel's
+ * tensor-core fragments read it, 8*M*K/32 for two sums per 32-weight group,
+ * 4*M for the per-token scales and 256 for a zero block, each part rounded
+ * up to 256 bytes.  Errors: QL_ERR_NULL, QL_ERR_SHAPE, QL_ERR_RANGE,
+ * QL_ERR_UNSUPPORTED. */
+ql_status qlinear_gemv_workspace_bytes(const ql_desc *desc, int64_t M, size_t *bytes);
+
 /* Decode-shaped layer, HBM-bound: y[M][N] (bf16) = x[M][K] (bf16) . W^T,
  * fp32 accumulation, one nearest-even rounding to bf16 at the end.
  * 1 <= M <= 8 for int4 / int6; 1 <= M <= 32 for affine.
+ * int4 at M = 1 runs two launches: a short pass that scales x per token by a
+ * power of two into fp16 range, reorders it for the tensor-core fragments
+ * and sums it per group into the workspace; then the streaming kernel, in
+ * which mma.sync multiplies the exactly converted codes (1024+q, 64+q in
+ * fp16) by x and the per-group scale and zero are applied in fp32.  Other
+ * formats and M: one launch, exact binary32 weights, fp32 FMA.
  * ExecuTorch page above, review section "Things done well" (the decode
  * kernel's one-shuffle step-word broadcast and full-warp trip counts) and
  * "Quant schema update" (hoisted int6 codes).
- * Errors: QL_ERR_NULL, QL_ERR_SHAPE, QL_ERR_ALIGN, QL_ERR_RANGE,
- * QL_ERR_UNSUPPORTED, QL_ERR_CUDA. */
+ * `workspace`: at least qlinear_gemv_workspace_bytes(), 256-byte aligned,
+ * caller-owned, overwritten; calls sharing one workspace must not overlap on
+ * the GPU.
+ * Errors: QL_ERR_NULL, QL_ERR_SHAPE (also: workspace too small),
+ * QL_ERR_ALIGN, QL_ERR_RANGE, QL_ERR_UNSUPPORTED, QL_ERR_CUDA. */
 ql_status qlinear_gemv(const ql_desc *desc, const ql_packed_const *w,
-                       const void *x, int64_t M, void *y, ql_stream_t stream);
+                       const void *x, int64_t M, void *y, void *workspace,
+                       size_t workspace_bytes, ql_stream_t stream);
 
 /* Bytes of caller-provided device workspace qlinear_gemm needs for `desc`
  * and M (host-only, no CUDA call): 2*M*K for the fp16 copy of x, plus

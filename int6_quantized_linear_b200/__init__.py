@@ -57,8 +57,9 @@ _SIGNATURES = {
     "qlinear_pack": ([C.POINTER(ql_desc), C.POINTER(ql_unpacked), C.POINTER(ql_packed), C.c_void_p], C.c_int),
     "qlinear_unpack": ([C.POINTER(ql_desc), C.POINTER(ql_packed), C.POINTER(ql_unpacked), C.c_void_p], C.c_int),
     "qlinear_dequant": ([C.POINTER(ql_desc), C.POINTER(ql_packed), C.c_void_p, C.c_int32, C.c_void_p], C.c_int),
-    "qlinear_gemv": ([C.POINTER(ql_desc), C.POINTER(ql_packed), C.c_void_p, C.c_int64, C.c_void_p, C.c_void_p],
-                     C.c_int),
+    "qlinear_gemv_workspace_bytes": ([C.POINTER(ql_desc), C.c_int64, C.POINTER(C.c_size_t)], C.c_int),
+    "qlinear_gemv": ([C.POINTER(ql_desc), C.POINTER(ql_packed), C.c_void_p, C.c_int64, C.c_void_p, C.c_void_p,
+                      C.c_size_t, C.c_void_p], C.c_int),
     "qlinear_gemm_workspace_bytes": ([C.POINTER(ql_desc), C.c_int64, C.POINTER(C.c_size_t)], C.c_int),
     "qlinear_gemm": ([C.POINTER(ql_desc), C.POINTER(ql_packed), C.c_void_p, C.c_int64, C.c_void_p, C.c_void_p,
                       C.c_size_t, C.c_void_p], C.c_int),
@@ -157,10 +158,27 @@ def qlinear_dequant(desc: Desc, codes, gmeta, steps, out, out_dtype: int, stream
            "qlinear_dequant")
 
 
-def qlinear_gemv(desc: Desc, codes, gmeta, steps, x, M: int, y, stream=None):
+def qlinear_gemv_workspace_bytes(desc: Desc, M: int) -> int:
+    d = desc.c()
+    n = C.c_size_t()
+    _check(lib().qlinear_gemv_workspace_bytes(C.byref(d), M, C.byref(n)), "qlinear_gemv_workspace_bytes")
+    return n.value
+
+
+def alloc_gemv_workspace(desc: Desc, M: int, device="cuda"):
+    import torch
+    return torch.empty(qlinear_gemv_workspace_bytes(desc, M), dtype=torch.uint8, device=device)
+
+
+def qlinear_gemv(desc: Desc, codes, gmeta, steps, x, M: int, y, workspace=None, stream=None):
+    """``workspace``: a uint8 CUDA tensor of at least qlinear_gemv_workspace_bytes(desc, M) bytes;
+    allocated here when omitted."""
+    if workspace is None:
+        workspace = alloc_gemv_workspace(desc, M, x.device)
     d = desc.c()
     w = ql_packed(_ptr(codes), _ptr(gmeta), _ptr(steps))
-    _check(lib().qlinear_gemv(C.byref(d), C.byref(w), _ptr(x), M, _ptr(y), _stream(stream)), "qlinear_gemv")
+    _check(lib().qlinear_gemv(C.byref(d), C.byref(w), _ptr(x), M, _ptr(y), _ptr(workspace),
+                              workspace.numel() * workspace.element_size(), _stream(stream)), "qlinear_gemv")
 
 
 def qlinear_gemm_workspace_bytes(desc: Desc, M: int) -> int:

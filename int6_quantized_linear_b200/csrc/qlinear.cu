@@ -166,14 +166,60 @@ ql_status launch_gemm(const ql_desc *d, const ql_packed_const *w, const void *x,
 
 template <int FMT, int BITS>
 ql_status launch_gemv(const ql_desc *d, const ql_packed_const *w, const void *x, int64_t M, void *y,
-                      cudaStream_t st, int sms) {
+                      void *workspace, cudaStream_t st, int sms) {
+  const auto *xb = static_cast<const __nv_bfloat16 *>(x);
+  auto *yb = static_cast<__nv_bfloat16 *>(y);
+  if constexpr (FMT == FMT_INT4) {
+    if (M == 1) {  // tensor-core path: preparation pass, then the streaming kernel as its dependent
+      const GemvWorkspace ws = gemv_workspace_carve(workspace, M, d->K);
+      const int64_t ng = M * (d->K / 32);
+      gemv_xprep_kernel<<<(int)((ng + 255) / 256), 256, 0, st>>>(xb, M, d->K, ws);
+      GemvTcParams p;
+      p.gmeta = static_cast<const uint8_t *>(w->gmeta);
+      p.steps = static_cast<const uint8_t *>(w->steps);
+      p.N = d->N;
+      p.K = d->K;
+      p.ws = ws;
+      p.y = yb;
+      CUtensorMap mc;  // codes as [N][K/2] bytes, boxes of 16 rows x 128 bytes, 128-byte swizzle
+      if (!encode_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->codes, (uint64_t)d->K / 2, (uint64_t)d->N,
+                     (uint64_t)d->K / 2, 128, 16, CU_TENSOR_MAP_SWIZZLE_128B))
+        return QL_ERR_CUDA;
+      const int64_t NS = d->K / 256, n_tiles = (d->N + 15) / 16;
+      // split K over more warps per tile while the grid still fits one wave (4 CTAs per SM)
+      const int64_t slots = (int64_t)sms * 4;
+      int P = 1;
+      while (2 * P <= GEMV_WARPS && 2 * P <= NS && (n_tiles * 2 * P + GEMV_WARPS - 1) / GEMV_WARPS <= slots) P *= 2;
+      p.parts = P;
+      const int64_t T = GEMV_WARPS / P;
+      static thread_local int configured_dev = -1;
+      int dev = 0;
+      cudaGetDevice(&dev);
+      if (configured_dev != dev) {
+        if (cudaFuncSetAttribute(gemv_int4_m1_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 gemv_smem_bytes()) != cudaSuccess)
+          return QL_ERR_CUDA;
+        configured_dev = dev;
+      }
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3((unsigned)((n_tiles + T - 1) / T));
+      cfg.blockDim = dim3(32 * GEMV_WARPS);
+      cfg.dynamicSmemBytes = gemv_smem_bytes();
+      cfg.stream = st;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[0].val.programmaticStreamSerializationAllowed = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      if (cudaLaunchKernelEx(&cfg, gemv_int4_m1_tc_kernel, mc, p) != cudaSuccess) return QL_ERR_CUDA;
+      return launched();
+    }
+  }
   const WeightPtrs p = make_ptrs(d, w);
   const int64_t rows_per_block = 8;
   int64_t g = (d->N + rows_per_block - 1) / rows_per_block;
   const int64_t cap = (int64_t)sms * 16;
   if (g > cap) g = cap;
-  const auto *xb = static_cast<const __nv_bfloat16 *>(x);
-  auto *yb = static_cast<__nv_bfloat16 *>(y);
   if (M == 1)
     gemv_simple_kernel<FMT, BITS, 1><<<(int)g, 256, 0, st>>>(p, d->N, xb, (int)M, yb);
   else if (M == 2)
@@ -348,25 +394,36 @@ ql_status qlinear_dequant(const ql_desc *d, const ql_packed_const *w, void *out,
   return launched();
 }
 
-ql_status qlinear_gemv(const ql_desc *d, const ql_packed_const *w, const void *x, int64_t M, void *y,
-                       ql_stream_t stream) {
-  ql_status st = check_desc(d);
+ql_status qlinear_gemv_workspace_bytes(const ql_desc *d, int64_t M, size_t *bytes) {
+  const ql_status st = check_desc(d);
   if (st != QL_OK) return st;
-  if (!w || !x || !y) return QL_ERR_NULL;
-  if ((st = check_packed(d, w->codes, w->gmeta, w->steps)) != QL_OK) return st;
-  if (!aligned16(x) || !aligned16(y)) return QL_ERR_ALIGN;
+  if (!bytes) return QL_ERR_NULL;
   const int64_t mmax = d->fmt == QL_AFFINE_U32 ? 32 : 8;
   if (M < 1 || M > mmax) return QL_ERR_RANGE;
+  *bytes = gemv_workspace_bytes(M, d->K);
+  return QL_OK;
+}
+
+ql_status qlinear_gemv(const ql_desc *d, const ql_packed_const *w, const void *x, int64_t M, void *y,
+                       void *workspace, size_t workspace_bytes, ql_stream_t stream) {
+  ql_status st = check_desc(d);
+  if (st != QL_OK) return st;
+  if (!w || !x || !y || !workspace) return QL_ERR_NULL;
+  if ((st = check_packed(d, w->codes, w->gmeta, w->steps)) != QL_OK) return st;
+  if (!aligned16(x) || !aligned16(y) || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return QL_ERR_ALIGN;
+  const int64_t mmax = d->fmt == QL_AFFINE_U32 ? 32 : 8;
+  if (M < 1 || M > mmax) return QL_ERR_RANGE;
+  if (workspace_bytes < gemv_workspace_bytes(M, d->K)) return QL_ERR_SHAPE;
   DeviceInfo *di;
   if ((st = device_info(&di)) != QL_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   switch (d->fmt) {
-    case QL_INT4_NSS: return launch_gemv<FMT_INT4, 4>(d, w, x, M, y, s, di->sms);
-    case QL_INT6_SYM: return launch_gemv<FMT_INT6, 6>(d, w, x, M, y, s, di->sms);
+    case QL_INT4_NSS: return launch_gemv<FMT_INT4, 4>(d, w, x, M, y, workspace, s, di->sms);
+    case QL_INT6_SYM: return launch_gemv<FMT_INT6, 6>(d, w, x, M, y, workspace, s, di->sms);
     default:
-      if (d->bits == 2) return launch_gemv<FMT_AFFINE, 2>(d, w, x, M, y, s, di->sms);
-      if (d->bits == 4) return launch_gemv<FMT_AFFINE, 4>(d, w, x, M, y, s, di->sms);
-      return launch_gemv<FMT_AFFINE, 8>(d, w, x, M, y, s, di->sms);
+      if (d->bits == 2) return launch_gemv<FMT_AFFINE, 2>(d, w, x, M, y, workspace, s, di->sms);
+      if (d->bits == 4) return launch_gemv<FMT_AFFINE, 4>(d, w, x, M, y, workspace, s, di->sms);
+      return launch_gemv<FMT_AFFINE, 8>(d, w, x, M, y, workspace, s, di->sms);
   }
 }
 

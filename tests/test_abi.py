@@ -33,7 +33,7 @@ def test_header_declares_the_boundary():
     names = declared_functions()
     for required in ("qlinear_pack", "qlinear_dequant", "qlinear_gemv", "qlinear_gemm",
                      "qlinear_packed_bytes", "qlinear_status_string", "qlinear_sync_status",
-                     "qlinear_gemm_workspace_bytes"):
+                     "qlinear_gemm_workspace_bytes", "qlinear_gemv_workspace_bytes"):
         assert required in names
 
 
@@ -78,10 +78,10 @@ def test_bad_shapes_rejected(lib, desc):
     assert e.value.status == ql.QL_ERR_SHAPE
 
 
-def _call_gemv(lib, desc, codes, gmeta, steps, x, M, y):
+def _call_gemv(lib, desc, codes, gmeta, steps, x, M, y, ws=0x20000, ws_bytes=1 << 24):
     d = desc.c()
     w = ql.ql_packed(codes, gmeta, steps)
-    return lib.qlinear_gemv(C.byref(d), C.byref(w), x, M, y, None)
+    return lib.qlinear_gemv(C.byref(d), C.byref(w), x, M, y, ws, ws_bytes, None)
 
 
 def test_host_validation_before_any_launch(lib):
@@ -96,6 +96,9 @@ def test_host_validation_before_any_launch(lib):
     assert _call_gemv(lib, ql.Desc("int4", 8, 100), A, A, A, A, 1, A) == ql.QL_ERR_SHAPE
     da = ql.Desc("affine", 8, 256, 4, 64)
     assert _call_gemv(lib, da, A, A, None, A, 33, A) == ql.QL_ERR_RANGE
+    assert _call_gemv(lib, d, A, A, A, A, 1, A, ws=None) == ql.QL_ERR_NULL
+    assert _call_gemv(lib, d, A, A, A, A, 1, A, ws=A + 128) == ql.QL_ERR_ALIGN
+    assert _call_gemv(lib, d, A, A, A, A, 1, A, ws_bytes=16) == ql.QL_ERR_SHAPE
     bad = ql.ql_desc(9, 0, 0, 0, 8, 256)
     w = ql.ql_packed(A, A, A)
     assert lib.qlinear_gemm(C.byref(bad), C.byref(w), A, 1, A, A, 1 << 20, None) == ql.QL_ERR_UNSUPPORTED
