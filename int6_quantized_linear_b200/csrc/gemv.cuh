@@ -62,58 +62,61 @@ __global__ void __launch_bounds__(256) gemv_simple_kernel(WeightPtrs p, int64_t 
 
 
 // ===========================================================================
-// Tensor-core decode GEMV for int4 at M = 1.
+// Tensor-core decode GEMV for int4 at M = 1 (integer MMA).
 //
 // Each warp owns a tile of 16 weight rows and a range of super-blocks.  The
 // codes of one super-block of the tile (16 rows x 128 bytes) arrive by TMA
 // into a per-warp ring in shared memory.  Lane (g = lane/4, c = lane%4) reads
-// whole 16-byte groups -- groups c and c+4 of two tile rows -- and turns every
-// 32-bit word of 8 nibbles into four f16x2 registers with one bit operation
-// each (after one shift per word): the nibble is OR-ed into the mantissa of
-// 1024.0 (even k) or of 64.0 (odd k), giving 1024+q or 64+q exactly.
+// whole 16-byte groups -- groups c and c+4 of two tile rows -- and turns each
+// 32-bit word of 8 nibbles into two u8x4 registers with one bit operation
+// each: w & 0xF0F0F0F0 holds the odd-k codes times 16, (w << 4) & 0xF0F0F0F0
+// the even-k codes times 16.
 //
-// mma.sync.m16n8k16 then multiplies these 16x16 weight fragments by a
-// "diagonal" x operand: column n of B holds x only in the two k-slots that
-// carry group n's weights and zeros elsewhere, so after the 16 MMAs of a
-// super-block D[row][n] is group n's partial dot product
-//     D = sum_k (bias_k + q_k) * x'_k,     bias_k = 1024 (k even) / 64 (k odd)
-// with x' = x * 2^a_g, x scaled per 32-element group by a power of two that
-// puts the group's max |x| in [2^15, 2^16) (exact in fp16).  The scale and
-// zero are applied once per (row, group):
-//     y += S * 2^-a_g * (D - B'_g - Z * X'_g),  B'_g = sum bias_k x'_k, X'_g = sum x'_k.
-// A short preparation pass writes x' in the order the fragments read it and
-// (B'_g, X'_g, 2^-a_g); lanes that hold no x for an MMA read a zero block,
-// so no per-MMA selects are needed.  The streaming kernel is launched as a
-// programmatic dependent of that pass and starts fetching weights before the
-// pass has finished (griddepcontrol.wait guards the first read of x).
+// mma.sync.m16n8k32 (u8 x s8 / u8 x u8, s32 accumulate) multiplies these
+// 16x32 fragments by a "diagonal" x operand: column n of B holds x only in
+// the k-slots that carry group n's codes and zeros elsewhere, so D[row][n]
+// collects group n's partial dot product.  x enters as 16-bit fixed point per
+// 32-element group, x_int = rint(x * 2^a_g) with the group's max |x| scaled
+// into [2^14, 2^15), split into a signed high byte and an unsigned low byte
+// (x_int = 256 * hi + lo), one MMA for each.  Per (row, group) of a
+// super-block the two integer sums are exact and below 2^22 in magnitude, so
+// the accumulators start at 1.5 * 2^23 (as bits) and read back as floats
+// with one subtraction.  The scale and zero are applied once per (row, group):
+//     T = 16 * sum_k q_k x_int_k = 256 * D_hi + D_lo
+//     y += S * (2^-a_g / 16) * (T - 16 * Z * X_g),   X_g = sum_k x_int_k
+// with S = sc * ss and Z = zc * zs.  A short preparation pass writes the x
+// bytes in the order the fragments read them with (2^-a_g / 16, -16 X_g) per
+// group; the streaming kernel is launched as a programmatic dependent of that
+// pass and starts fetching weights before it has finished (griddepcontrol.wait
+// guards the first read of x).  Lanes that hold no x for an MMA read a zero
+// block, so no per-MMA selects are needed.
 // ===========================================================================
 
 struct GemvWorkspace {
-  uint32_t *xperm;  // [M][K/32 groups][16] f16x2 pairs: pair t = (x'[8(t/4)+t%4], x'[8(t/4)+t%4+4])
-  float4 *gsum;     // [M][K/32] (B'_g, X'_g, 2^-a_g, 0)
-  uint32_t *zero;   // 64 zero bytes
+  uint4 *xq;      // [M][K/32 groups][4 j][16 B]: for j, (even-k hi, even-k lo, odd-k hi, odd-k lo), 4 bytes each
+  float2 *gsum;   // [M][K/32] (2^-a_g / 16, -16 * sum x_int)
+  uint4 *zero;    // 64 zero bytes
 };
 
 inline size_t gemv_workspace_bytes(int64_t M, int64_t K) {
-  return align256((size_t)M * K * 2) + align256((size_t)M * (K / 32) * 16) + 256;
+  return align256((size_t)M * K * 2) + align256((size_t)M * (K / 32) * 8) + 256;
 }
 
 inline GemvWorkspace gemv_workspace_carve(void *base, int64_t M, int64_t K) {
   uint8_t *p = static_cast<uint8_t *>(base);
   GemvWorkspace w;
-  w.xperm = reinterpret_cast<uint32_t *>(p);
+  w.xq = reinterpret_cast<uint4 *>(p);
   p += align256((size_t)M * K * 2);
-  w.gsum = reinterpret_cast<float4 *>(p);
-  p += align256((size_t)M * (K / 32) * 16);
-  w.zero = reinterpret_cast<uint32_t *>(p);
+  w.gsum = reinterpret_cast<float2 *>(p);
+  p += align256((size_t)M * (K / 32) * 8);
+  w.zero = reinterpret_cast<uint4 *>(p);
   return w;
 }
 
 QL_DEVI void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 QL_DEVI void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
-// One thread per 32-element group of x: scale into fp16 range, reorder into
-// fragment pairs, sum.
+// One thread per 32-element group of x: fixed-point conversion, byte split in fragment order, sum.
 __global__ void __launch_bounds__(256) gemv_xprep_kernel(const __nv_bfloat16 *x, int64_t M, int64_t K,
                                                          GemvWorkspace ws) {
   pdl_launch_dependents();
@@ -121,7 +124,7 @@ __global__ void __launch_bounds__(256) gemv_xprep_kernel(const __nv_bfloat16 *x,
   const int64_t gi = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;  // over M * ng
   if (gi == 0) {
 #pragma unroll
-    for (int t = 0; t < 16; ++t) ws.zero[t] = 0u;
+    for (int t = 0; t < 4; ++t) ws.zero[t] = make_uint4(0u, 0u, 0u, 0u);
   }
   if (gi >= M * ng) return;
   const uint4 *src = reinterpret_cast<const uint4 *>(x) + 4 * gi;  // 32 bf16 = 64 bytes
@@ -138,22 +141,35 @@ __global__ void __launch_bounds__(256) gemv_xprep_kernel(const __nv_bfloat16 *x,
       amax = fmaxf(amax, fmaxf(fabsf(xs[8 * t + 2 * j]), fabsf(xs[8 * t + 2 * j + 1])));
     }
   }
-  const int a = scale_exponent(amax, 15);
+  const int a = scale_exponent(amax, 14);  // max |x_int| < 2^15
   const float sc = exp2i(a);
-  uint32_t pr[16];
-  float be = 0.f, bo = 0.f;
+  int xi[32];
+  int sum = 0;
 #pragma unroll
-  for (int t = 0; t < 16; ++t) {
-    const int k0 = 8 * (t >> 2) + (t & 3);
-    const __half2 h = __floats2half2_rn(xs[k0] * sc, xs[k0 + 4] * sc);
-    pr[t] = *reinterpret_cast<const uint32_t *>(&h);
-    const float2 f = __half22float2(h);  // the values the MMA will see
-    if (t & 1) bo += f.x + f.y; else be += f.x + f.y;
+  for (int k = 0; k < 32; ++k) {
+    xi[k] = __float2int_rn(xs[k] * sc);
+    sum += xi[k];
   }
-  uint4 *dst = reinterpret_cast<uint4 *>(ws.xperm + 16 * gi);
+  uint32_t o[16];
 #pragma unroll
-  for (int t = 0; t < 4; ++t) dst[t] = make_uint4(pr[4 * t], pr[4 * t + 1], pr[4 * t + 2], pr[4 * t + 3]);
-  ws.gsum[gi] = make_float4(1024.f * be + 64.f * bo, be + bo, exp2i(-a), 0.f);
+  for (int j = 0; j < 4; ++j) {
+#pragma unroll
+    for (int kind = 0; kind < 2; ++kind) {
+      uint32_t hi = 0, lo = 0;
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const int v = xi[8 * j + 2 * b + kind];
+        hi |= ((uint32_t)(v >> 8) & 0xffu) << (8 * b);
+        lo |= ((uint32_t)v & 0xffu) << (8 * b);
+      }
+      o[4 * j + 2 * kind] = hi;
+      o[4 * j + 2 * kind + 1] = lo;
+    }
+  }
+  uint4 *dst = ws.xq + 4 * gi;
+#pragma unroll
+  for (int t = 0; t < 4; ++t) dst[t] = make_uint4(o[4 * t], o[4 * t + 1], o[4 * t + 2], o[4 * t + 3]);
+  ws.gsum[gi] = make_float2(exp2i(-a) * 0.0625f, -16.f * (float)sum);
 }
 
 // A byte of a metadata word as a float: 2^23 + b, to be fused into an FMA with -2^23 * step.
@@ -190,24 +206,18 @@ QL_DEVI bool mbar_wait_suspend(uint32_t bar, uint32_t parity, volatile int *abor
   }
 }
 
-// One MMA of the GEMV: builds the four f16x2 A registers from the code words in place
-// ((w & mask) | magic: 1024+q for a nibble in bits 0-3 of a half, 64+q for bits 4-7) and
-// multiplies them into acc.
-#define QL_GEMV_MMA(MASK, MAGIC, W0, W1, W2, W3, B0, B1)                                              \
-  asm volatile(                                                                                         \
-      "{\n\t.reg .b32 a0, a1, a2, a3;\n\t"                                                            \
-      "lop3.b32 a0, %4, " MASK ", " MAGIC ", 0xEA;\n\t"                                               \
-      "lop3.b32 a1, %5, " MASK ", " MAGIC ", 0xEA;\n\t"                                               \
-      "lop3.b32 a2, %6, " MASK ", " MAGIC ", 0xEA;\n\t"                                               \
-      "lop3.b32 a3, %7, " MASK ", " MAGIC ", 0xEA;\n\t"                                               \
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {a0,a1,a2,a3}, {%8,%9}, "     \
-      "{%0,%1,%2,%3};\n\t}"                                                                             \
-      : "+f"(acc[0]), "+f"(acc[1]), "+f"(acc[2]), "+f"(acc[3])                                        \
-      : "r"(W0), "r"(W1), "r"(W2), "r"(W3), "r"(B0), "r"(B1))
+// acc += A * B with A = u8 codes x 16 and B = the high (signed) or low (unsigned) x bytes
+#define QL_IMMA(TB, ACC, A0, A1, A2, A3, B0, B1)                                                      \
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.u8." TB ".s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "  \
+      "{%0,%1,%2,%3};"                                                                                  \
+      : "+r"(ACC[0]), "+r"(ACC[1]), "+r"(ACC[2]), "+r"(ACC[3])                                        \
+      : "r"(A0), "r"(A1), "r"(A2), "r"(A3), "r"(B0), "r"(B1))
 
-constexpr int GEMV_RING = 4;   // super-blocks in flight per warp (RING - 1 copies ahead)
+constexpr int GEMV_RING = 4;   // super-blocks in flight per warp
 constexpr int GEMV_WARPS = 4;  // warps per CTA: GEMV_WARPS / parts tiles, each split over `parts` warps
 constexpr int GEMV_STAGE_BYTES = 16 * 128;  // one super-block of a 16-row tile: 16 rows x 128 code bytes
+constexpr int32_t GEMV_ACC0 = 0x4B400000;    // 1.5 * 2^23 as float bits: integer sums below 2^22 read back exactly
+constexpr float GEMV_ACC0_F = 12582912.f;
 
 struct GemvTcParams {
   const uint8_t *gmeta, *steps;
@@ -281,10 +291,10 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS, 4)
   // x operand: lane (g, c) feeds column g from its b0 slots when g == c, from b1 when g == c + 4;
   // other lanes read the zero block
   const bool on0 = (g == c), on1 = (g == c + 4);
-  const uint4 *xb0 = reinterpret_cast<const uint4 *>(on0 ? p.ws.xperm + 16 * c + 128 * sb0 : p.ws.zero);
-  const uint4 *xb1 = reinterpret_cast<const uint4 *>(on1 ? p.ws.xperm + 16 * (c + 4) + 128 * sb0 : p.ws.zero);
+  const uint4 *xb0 = on0 ? p.ws.xq + 4 * (8 * sb0 + c) : p.ws.zero;
+  const uint4 *xb1 = on1 ? p.ws.xq + 4 * (8 * sb0 + c + 4) : p.ws.zero;
   const int xinc0 = on0 ? 32 : 0, xinc1 = on1 ? 32 : 0;  // uint4 per super-block (8 groups x 64 B)
-  const float4 *gs = p.ws.gsum + 8 * sb0 + 2 * c;        // (B', X', 2^-a) of groups 2c, 2c+1; + 8 per sb
+  const float4 *gs = reinterpret_cast<const float4 *>(p.ws.gsum) + 4 * sb0 + c;  // groups 2c, 2c+1; + 4 per sb
   // shared-memory offsets of this lane's four 16-byte chunks inside a stage
   const uint32_t o00 = pg * 128 + ((c ^ pg) << 4), o01 = pg * 128 + (((c + 4) ^ pg) << 4);
   const uint32_t o10 = (pg + 8) * 128 + ((c ^ pg) << 4), o11 = (pg + 8) * 128 + (((c + 4) ^ pg) << 4);
@@ -298,46 +308,50 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS, 4)
       m0 = __ldg(gm0 + 4 * (i + 1)); m1 = __ldg(gm1 + 4 * (i + 1));
       s0 = __ldg(st0 + i + 1); s1 = __ldg(st1 + i + 1);
     }
-    const float4 G0 = __ldg(gs), G1 = __ldg(gs + 1);
-    gs += 8;
+    const float4 G = __ldg(gs);  // (2^-a/16, -16 X) of groups 2c and 2c+1
+    gs += 4;
     const int s = i % GEMV_RING;
     if (!mbar_wait_suspend(bar0 + 8 * s, (uint32_t)((i / GEMV_RING) & 1), &abort_flag)) break;
     const uint32_t stg = ring + s * GEMV_STAGE_BYTES;
     const uint4 a00 = lds128(stg + o00), a10 = lds128(stg + o10);  // (r0 | r1, group c)
     const uint4 a01 = lds128(stg + o01), a11 = lds128(stg + o11);  // (r0 | r1, group c+4)
     __syncwarp();  // every lane has read the stage: the next turn may refill it
-    // two independent accumulator chains (even / odd words) halve the MMA dependency latency
-    float d[4] = {0.f, 0.f, 0.f, 0.f}, e[4] = {0.f, 0.f, 0.f, 0.f};
+    int32_t dh[4] = {GEMV_ACC0, GEMV_ACC0, GEMV_ACC0, GEMV_ACC0};
+    int32_t dl[4] = {GEMV_ACC0, GEMV_ACC0, GEMV_ACC0, GEMV_ACC0};
     const uint32_t w00[4] = {a00.x, a00.y, a00.z, a00.w}, w01[4] = {a01.x, a01.y, a01.z, a01.w};
     const uint32_t w10[4] = {a10.x, a10.y, a10.z, a10.w}, w11[4] = {a11.x, a11.y, a11.z, a11.w};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const uint4 xv0 = __ldg(xb0 + j), xv1 = __ldg(xb1 + j);
-      const uint32_t v00 = w00[j] >> 8, v10 = w10[j] >> 8, v01 = w01[j] >> 8, v11 = w11[j] >> 8;
-      float(&acc)[4] = (j & 1) ? e : d;
-      QL_GEMV_MMA("0x000F000F", "0x64006400", w00[j], w10[j], w01[j], w11[j], xv0.x, xv1.x);  // (n0, n4)
-      QL_GEMV_MMA("0x00F000F0", "0x54005400", w00[j], w10[j], w01[j], w11[j], xv0.y, xv1.y);  // (n1, n5)
-      QL_GEMV_MMA("0x000F000F", "0x64006400", v00, v10, v01, v11, xv0.z, xv1.z);              // (n2, n6)
-      QL_GEMV_MMA("0x00F000F0", "0x54005400", v00, v10, v01, v11, xv0.w, xv1.w);              // (n3, n7)
+      const uint32_t h00 = w00[j] & 0xF0F0F0F0u, h10 = w10[j] & 0xF0F0F0F0u;  // odd k, x16
+      const uint32_t h01 = w01[j] & 0xF0F0F0F0u, h11 = w11[j] & 0xF0F0F0F0u;
+      QL_IMMA("s8", dh, h00, h10, h01, h11, xv0.z, xv1.z);
+      QL_IMMA("u8", dl, h00, h10, h01, h11, xv0.w, xv1.w);
+      const uint32_t e00 = (w00[j] << 4) & 0xF0F0F0F0u, e10 = (w10[j] << 4) & 0xF0F0F0F0u;  // even k, x16
+      const uint32_t e01 = (w01[j] << 4) & 0xF0F0F0F0u, e11 = (w11[j] << 4) & 0xF0F0F0F0u;
+      QL_IMMA("s8", dh, e00, e10, e01, e11, xv0.x, xv1.x);
+      QL_IMMA("u8", dl, e00, e10, e01, e11, xv0.y, xv1.y);
     }
     xb0 += xinc0;
     xb1 += xinc1;
+    // D[q]: q = 0 (r0, group 2c), 1 (r0, 2c+1), 2 (r1, 2c), 3 (r1, 2c+1)
+    float t[4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) d[q] += e[q];
-    // d0: (r0, group 2c)  d1: (r0, 2c+1)  d2: (r1, 2c)  d3: (r1, 2c+1)
+    for (int q = 0; q < 4; ++q)
+      t[q] = fmaf(__int_as_float(dh[q]) - GEMV_ACC0_F, 256.f, __int_as_float(dl[q]) - GEMV_ACC0_F);
     // S = sc * ss and Z = zc * zs, each one FMA from the byte placed in the mantissa of 2^23
     const float ss0 = f16_bits_to_f32(cs0), zs0 = f16_bits_to_f32(cs0 >> 16);
     const float ss1 = f16_bits_to_f32(cs1), zs1 = f16_bits_to_f32(cs1 >> 16);
     const float nss0 = -8388608.f * ss0, nzs0 = -8388608.f * zs0;
     const float nss1 = -8388608.f * ss1, nzs1 = -8388608.f * zs1;
-    const float S00 = fmaf(byte_magic(cm0, 0), ss0, nss0) * G0.z, Z00 = fmaf(byte_magic(cm0, 1), zs0, nzs0);
-    const float S01 = fmaf(byte_magic(cm0, 2), ss0, nss0) * G1.z, Z01 = fmaf(byte_magic(cm0, 3), zs0, nzs0);
-    const float S10 = fmaf(byte_magic(cm1, 0), ss1, nss1) * G0.z, Z10 = fmaf(byte_magic(cm1, 1), zs1, nzs1);
-    const float S11 = fmaf(byte_magic(cm1, 2), ss1, nss1) * G1.z, Z11 = fmaf(byte_magic(cm1, 3), zs1, nzs1);
-    acc0 = fmaf(S00, fmaf(-Z00, G0.y, d[0] - G0.x), acc0);
-    acc0 = fmaf(S01, fmaf(-Z01, G1.y, d[1] - G1.x), acc0);
-    acc1 = fmaf(S10, fmaf(-Z10, G0.y, d[2] - G0.x), acc1);
-    acc1 = fmaf(S11, fmaf(-Z11, G1.y, d[3] - G1.x), acc1);
+    const float S00 = fmaf(byte_magic(cm0, 0), ss0, nss0) * G.x, Z00 = fmaf(byte_magic(cm0, 1), zs0, nzs0);
+    const float S01 = fmaf(byte_magic(cm0, 2), ss0, nss0) * G.z, Z01 = fmaf(byte_magic(cm0, 3), zs0, nzs0);
+    const float S10 = fmaf(byte_magic(cm1, 0), ss1, nss1) * G.x, Z10 = fmaf(byte_magic(cm1, 1), zs1, nzs1);
+    const float S11 = fmaf(byte_magic(cm1, 2), ss1, nss1) * G.z, Z11 = fmaf(byte_magic(cm1, 3), zs1, nzs1);
+    acc0 = fmaf(S00, fmaf(Z00, G.y, t[0]), acc0);
+    acc0 = fmaf(S01, fmaf(Z01, G.w, t[1]), acc0);
+    acc1 = fmaf(S10, fmaf(Z10, G.y, t[2]), acc1);
+    acc1 = fmaf(S11, fmaf(Z11, G.w, t[3]), acc1);
   }
   if (abort_flag && lane == 0) {  // a wait gave up: let this warp's copies in flight land first
     for (int i = issued - GEMV_RING; i < issued; ++i) {
