@@ -89,6 +89,14 @@ QL_DEVI void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint32_t bar, int
       : "memory");
 }
 
+// Untiled bulk copy global -> shared completing on an mbarrier: both addresses 16-byte aligned,
+// size a multiple of 16.
+QL_DEVI void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
 QL_DEVI void tma_prefetch_desc(const CUtensorMap *map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

@@ -93,13 +93,12 @@ __global__ void __launch_bounds__(256) gemv_simple_kernel(WeightPtrs p, int64_t 
 // ===========================================================================
 
 struct GemvWorkspace {
-  uint4 *xq;      // [M][K/32 groups][4 j][16 B]: for j, (even-k hi, even-k lo, odd-k hi, odd-k lo), 4 bytes each
+  uint4 *xq;      // [M][K/256 super-blocks][4 j][8 groups][16 B]: (even-k hi, even-k lo, odd-k hi, odd-k lo) bytes
   float2 *gsum;   // [M][K/32] (2^-a_g / 16, -16 * sum x_int)
-  uint4 *zero;    // 64 zero bytes
 };
 
 inline size_t gemv_workspace_bytes(int64_t M, int64_t K) {
-  return align256((size_t)M * K * 2) + align256((size_t)M * (K / 32) * 8) + 256;
+  return align256((size_t)M * K * 2) + align256((size_t)M * (K / 32) * 8);
 }
 
 inline GemvWorkspace gemv_workspace_carve(void *base, int64_t M, int64_t K) {
@@ -108,8 +107,6 @@ inline GemvWorkspace gemv_workspace_carve(void *base, int64_t M, int64_t K) {
   w.xq = reinterpret_cast<uint4 *>(p);
   p += align256((size_t)M * K * 2);
   w.gsum = reinterpret_cast<float2 *>(p);
-  p += align256((size_t)M * (K / 32) * 8);
-  w.zero = reinterpret_cast<uint4 *>(p);
   return w;
 }
 
@@ -122,10 +119,6 @@ __global__ void __launch_bounds__(256) gemv_xprep_kernel(const __nv_bfloat16 *x,
   pdl_launch_dependents();
   const int64_t ng = K / 32;
   const int64_t gi = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;  // over M * ng
-  if (gi == 0) {
-#pragma unroll
-    for (int t = 0; t < 4; ++t) ws.zero[t] = make_uint4(0u, 0u, 0u, 0u);
-  }
   if (gi >= M * ng) return;
   const uint4 *src = reinterpret_cast<const uint4 *>(x) + 4 * gi;  // 32 bf16 = 64 bytes
   float xs[32];
@@ -150,9 +143,12 @@ __global__ void __launch_bounds__(256) gemv_xprep_kernel(const __nv_bfloat16 *x,
     xi[k] = __float2int_rn(xs[k] * sc);
     sum += xi[k];
   }
-  uint32_t o[16];
+  // group gi = (m, super-block sb, group-in-block grp): chunk j goes to [m][sb][j][grp]
+  const int64_t grp = gi & 7, msb = gi >> 3;
+  uint4 *dst = ws.xq + msb * 32 + grp;
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
+    uint32_t o[4];
 #pragma unroll
     for (int kind = 0; kind < 2; ++kind) {
       uint32_t hi = 0, lo = 0;
@@ -162,13 +158,11 @@ __global__ void __launch_bounds__(256) gemv_xprep_kernel(const __nv_bfloat16 *x,
         hi |= ((uint32_t)(v >> 8) & 0xffu) << (8 * b);
         lo |= ((uint32_t)v & 0xffu) << (8 * b);
       }
-      o[4 * j + 2 * kind] = hi;
-      o[4 * j + 2 * kind + 1] = lo;
+      o[2 * kind] = hi;
+      o[2 * kind + 1] = lo;
     }
+    dst[8 * j] = make_uint4(o[0], o[1], o[2], o[3]);
   }
-  uint4 *dst = ws.xq + 4 * gi;
-#pragma unroll
-  for (int t = 0; t < 4; ++t) dst[t] = make_uint4(o[4 * t], o[4 * t + 1], o[4 * t + 2], o[4 * t + 3]);
   ws.gsum[gi] = make_float2(exp2i(-a) * 0.0625f, -16.f * (float)sum);
 }
 
@@ -180,6 +174,16 @@ QL_DEVI float byte_magic(uint32_t w, int i) {
 QL_DEVI uint4 lds128(uint32_t a) {
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+  return v;
+}
+QL_DEVI float4 lds128f(uint32_t a) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(a));
+  return v;
+}
+QL_DEVI uint32_t lds32(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
   return v;
 }
 
@@ -206,7 +210,13 @@ QL_DEVI bool mbar_wait_suspend(uint32_t bar, uint32_t parity, volatile int *abor
   }
 }
 
-// acc += A * B with A = u8 codes x 16 and B = the high (signed) or low (unsigned) x bytes
+// ACC = C + A * B (first MMA of a chain) and ACC += A * B, with A = u8 codes x 16 and B = the
+// high (signed) or low (unsigned) x bytes
+#define QL_IMMA0(TB, ACC, C, A0, A1, A2, A3, B0, B1)                                                  \
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.u8." TB ".s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "  \
+      "{%10,%10,%10,%10};"                                                                              \
+      : "=r"(ACC[0]), "=r"(ACC[1]), "=r"(ACC[2]), "=r"(ACC[3])                                        \
+      : "r"(A0), "r"(A1), "r"(A2), "r"(A3), "r"(B0), "r"(B1), "r"(C))
 #define QL_IMMA(TB, ACC, A0, A1, A2, A3, B0, B1)                                                      \
   asm("mma.sync.aligned.m16n8k32.row.col.s32.u8." TB ".s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "  \
       "{%0,%1,%2,%3};"                                                                                  \
@@ -215,34 +225,43 @@ QL_DEVI bool mbar_wait_suspend(uint32_t bar, uint32_t parity, volatile int *abor
 
 constexpr int GEMV_RING = 4;   // super-blocks in flight per warp
 constexpr int GEMV_WARPS = 4;  // warps per CTA: GEMV_WARPS / parts tiles, each split over `parts` warps
-constexpr int GEMV_STAGE_BYTES = 16 * 128;  // one super-block of a 16-row tile: 16 rows x 128 code bytes
+// one stage = one super-block of a 16-row tile: codes (16 rows x 128 B, 128-byte swizzle), the
+// tile's group words [16 rows][16 B], the super-block's x bytes [4 j][8 groups][16 B], its 8 group sums
+constexpr int GEMV_ST_CODES = 0, GEMV_ST_GMETA = 2048, GEMV_ST_X = 2304, GEMV_ST_GSUM = 2816;
+constexpr int GEMV_STAGE_BYTES = 3072;      // multiple of 1024 (the swizzle atom)
+constexpr uint32_t GEMV_STAGE_TX = 2048 + 512 + 64 + 256;
+constexpr int GEMV_ZERO_BYTES = 512;        // zero x chunks at a 128-byte stride, for lanes that feed no x
 constexpr int32_t GEMV_ACC0 = 0x4B400000;    // 1.5 * 2^23 as float bits: integer sums below 2^22 read back exactly
 constexpr float GEMV_ACC0_F = 12582912.f;
 
 struct GemvTcParams {
-  const uint8_t *gmeta, *steps;
+  const uint8_t *steps;
   int64_t N, K;
   int parts;  // warps splitting K for one tile (1, 2 or 4)
   GemvWorkspace ws;
   __nv_bfloat16 *y;
 };
 
-// dynamic shared memory: [warp][stage] code tiles (1024-aligned), mbarriers, reduction buffer
+// dynamic shared memory: [warp][stage] (1024-aligned), zero block, mbarriers, reduction buffer
 inline constexpr int gemv_smem_bytes() {
-  return GEMV_WARPS * GEMV_RING * GEMV_STAGE_BYTES + GEMV_WARPS * GEMV_RING * 8 + GEMV_WARPS * 16 * 4 + 1024;
+  return GEMV_WARPS * GEMV_RING * GEMV_STAGE_BYTES + GEMV_ZERO_BYTES + GEMV_WARPS * GEMV_RING * 8 +
+         GEMV_WARPS * 16 * 4 + 1024;
 }
 
-// Codes arrive by TMA: each warp runs its own GEMV_RING-deep ring of 16-row x 128-byte boxes (one
-// super-block of its tile) with one mbarrier per stage.  The box is stored with the 128-byte
-// swizzle (16-byte chunk j of row r at chunk j ^ (r & 7)); MMA row g (and g + 8) reads tile row
-// pg = (g >> 1) | ((g & 1) << 2), so the two rows of one 8-lane shared-load phase differ in bit 2
-// and their chunks never share banks.  Group words, step words, x and the group sums are small
-// and come through the L1 cache, one super-block ahead.
+// Everything a super-block needs except its step words arrives by one stage of a per-warp ring:
+// the codes box (TMA, 128-byte swizzle: 16-byte chunk j of row r at chunk j ^ (r & 7)), the group
+// words box (TMA) and the x bytes and group sums (bulk copies), all completing on the stage's
+// mbarrier.  MMA row g (and g + 8) reads tile row pg = (g >> 1) | ((g & 1) << 2), so the two rows of
+// one 8-lane shared-load phase differ in bit 2 and their chunks never share banks.  The loop runs
+// RING super-blocks per turn so every shared-memory offset is a constant; step words come through
+// the L1 cache RING - 1 super-blocks ahead.
 __global__ void __launch_bounds__(32 * GEMV_WARPS, 4)
-    gemv_int4_m1_tc_kernel(const __grid_constant__ CUtensorMap map_codes, GemvTcParams p) {
+    gemv_int4_m1_tc_kernel(const __grid_constant__ CUtensorMap map_codes,
+                           const __grid_constant__ CUtensorMap map_gmeta, GemvTcParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + GEMV_WARPS * GEMV_RING * GEMV_STAGE_BYTES);
+  uint8_t *zero_blk = smem + GEMV_WARPS * GEMV_RING * GEMV_STAGE_BYTES;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(zero_blk + GEMV_ZERO_BYTES);
   float *red = reinterpret_cast<float *>(bars + GEMV_WARPS * GEMV_RING);  // [GEMV_WARPS][16]
   __shared__ int abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -257,103 +276,140 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS, 4)
   const uint32_t ring = smem_u32(smem + warp * GEMV_RING * GEMV_STAGE_BYTES);
   const uint32_t bar0 = smem_u32(bars + warp * GEMV_RING);
   if (threadIdx.x == 0) abort_flag = 0;
+  for (int t = threadIdx.x; t < GEMV_ZERO_BYTES / 16; t += blockDim.x)
+    reinterpret_cast<uint4 *>(zero_blk)[t] = make_uint4(0u, 0u, 0u, 0u);
   if (lane == 0) {
     for (int s = 0; s < GEMV_RING; ++s) mbar_init(bar0 + 8 * s, 1);
     fence_mbar_init();
   }
   __syncthreads();
-  // i-th super-block of this warp's range goes to stage i % RING; its wait parity is (i / RING) & 1
-  auto issue = [&](int i) {
-    const int s = i % GEMV_RING;
-    mbar_arrive_expect_tx(bar0 + 8 * s, GEMV_STAGE_BYTES);
-    tma_load_2d(ring + s * GEMV_STAGE_BYTES, &map_codes, bar0 + 8 * s, (sb0 + i) * 128, (int32_t)(tile * 16));
+  const uint8_t *xq_sb = reinterpret_cast<const uint8_t *>(p.ws.xq) + (int64_t)sb0 * 512;  // M = 1
+  const uint8_t *gs_sb = reinterpret_cast<const uint8_t *>(p.ws.gsum) + (int64_t)sb0 * 64;
+  // stage s of super-block i: weights (codes, group words) need no x; x and sums come after pdl_wait
+  auto issue_w = [&](int i, int s) {
+    const uint32_t st = ring + s * GEMV_STAGE_BYTES, bar = bar0 + 8 * s;
+    mbar_arrive_expect_tx(bar, GEMV_STAGE_TX);
+    tma_load_2d(st + GEMV_ST_CODES, &map_codes, bar, (sb0 + i) * 128, (int32_t)(tile * 16));
+    tma_load_2d(st + GEMV_ST_GMETA, &map_gmeta, bar, (sb0 + i) * 16, (int32_t)(tile * 16));
   };
-  int issued = 0;
+  auto issue_x = [&](int i, int s) {
+    const uint32_t st = ring + s * GEMV_STAGE_BYTES, bar = bar0 + 8 * s;
+    bulk_load(st + GEMV_ST_X, xq_sb + (int64_t)i * 512, 512, bar);
+    bulk_load(st + GEMV_ST_GSUM, gs_sb + (int64_t)i * 64, 64, bar);
+  };
+  const int pre = nsb < GEMV_RING - 1 ? nsb : GEMV_RING - 1;
+  int issued = pre;  // super-blocks whose stage copies were started (lane 0's count is the one used)
   if (lane == 0) {
     tma_prefetch_desc(&map_codes);
-    for (; issued < GEMV_RING - 1 && issued < nsb; ++issued) issue(issued);  // weights need no x
+    tma_prefetch_desc(&map_gmeta);
+    for (int i = 0; i < pre; ++i) issue_w(i, i);
   }
   const int pg = (g >> 1) | ((g & 1) << 2);
   int64_t r0 = tile * 16 + pg, r1 = r0 + 8;
   if (r0 >= p.N) r0 = p.N - 1;  // rows past the end are computed on a valid row and discarded
   if (r1 >= p.N) r1 = p.N - 1;
-  const uint32_t *gm0 = reinterpret_cast<const uint32_t *>(p.gmeta + r0 * (p.K / 16)) + 4 * sb0 + c;
-  const uint32_t *gm1 = reinterpret_cast<const uint32_t *>(p.gmeta + r1 * (p.K / 16)) + 4 * sb0 + c;
   const uint32_t *st0 = reinterpret_cast<const uint32_t *>(p.steps) + r0 * NS + sb0;
   const uint32_t *st1 = reinterpret_cast<const uint32_t *>(p.steps) + r1 * NS + sb0;
-  uint32_t m0 = 0, m1 = 0, s0 = 0, s1 = 0;
-  if (nsb > 0) {
-    m0 = __ldg(gm0); m1 = __ldg(gm1);
-    s0 = __ldg(st0); s1 = __ldg(st1);
+  uint32_t sr0[GEMV_RING], sr1[GEMV_RING];  // step words of the next RING - 1 super-blocks, by stage
+#pragma unroll
+  for (int s = 0; s < GEMV_RING; ++s) {
+    sr0[s] = 0u;
+    sr1[s] = 0u;
+    if (s < pre) {
+      sr0[s] = __ldg(st0 + s);
+      sr1[s] = __ldg(st1 + s);
+    }
   }
-  pdl_wait();  // x in fragment order and its group sums are ready from here on
+  pdl_wait();  // x bytes and group sums are ready from here on
+  if (lane == 0)
+    for (int i = 0; i < pre; ++i) issue_x(i, i);
 
-  // x operand: lane (g, c) feeds column g from its b0 slots when g == c, from b1 when g == c + 4;
-  // other lanes read the zero block
+  // per-lane shared-memory addresses (offsets inside a stage are added as constants)
   const bool on0 = (g == c), on1 = (g == c + 4);
-  const uint4 *xb0 = on0 ? p.ws.xq + 4 * (8 * sb0 + c) : p.ws.zero;
-  const uint4 *xb1 = on1 ? p.ws.xq + 4 * (8 * sb0 + c + 4) : p.ws.zero;
-  const int xinc0 = on0 ? 32 : 0, xinc1 = on1 ? 32 : 0;  // uint4 per super-block (8 groups x 64 B)
-  const float4 *gs = reinterpret_cast<const float4 *>(p.ws.gsum) + 4 * sb0 + c;  // groups 2c, 2c+1; + 4 per sb
-  // shared-memory offsets of this lane's four 16-byte chunks inside a stage
-  const uint32_t o00 = pg * 128 + ((c ^ pg) << 4), o01 = pg * 128 + (((c + 4) ^ pg) << 4);
-  const uint32_t o10 = (pg + 8) * 128 + ((c ^ pg) << 4), o11 = (pg + 8) * 128 + (((c + 4) ^ pg) << 4);
+  const uint32_t zero_a = smem_u32(zero_blk);
+  uint32_t xa0[GEMV_RING], xa1[GEMV_RING];  // x chunk j of this lane's b0 / b1 at xa + 128 j
+#pragma unroll
+  for (int s = 0; s < GEMV_RING; ++s) {
+    xa0[s] = on0 ? ring + s * GEMV_STAGE_BYTES + GEMV_ST_X + 16 * c : zero_a;
+    xa1[s] = on1 ? ring + s * GEMV_STAGE_BYTES + GEMV_ST_X + 16 * (c + 4) : zero_a;
+  }
+  const uint32_t a00 = ring + pg * 128 + ((c ^ pg) << 4), a01 = ring + pg * 128 + (((c + 4) ^ pg) << 4);
+  const uint32_t a10 = a00 + 1024, a11 = a01 + 1024;  // row pg + 8: same swizzle phase, next atom
+  const uint32_t ag = ring + GEMV_ST_GSUM + 16 * c;
+  const uint32_t am = ring + GEMV_ST_GMETA + pg * 16 + 4 * c;
 
   float acc0 = 0.f, acc1 = 0.f;
-  for (int i = 0; i < nsb; ++i) {
-    // refill the stage released at the end of the previous turn (RING - 1 stages stay in flight)
-    if (lane == 0 && issued < nsb) issue(issued++);
-    const uint32_t cm0 = m0, cm1 = m1, cs0 = s0, cs1 = s1;
-    if (i + 1 < nsb) {
-      m0 = __ldg(gm0 + 4 * (i + 1)); m1 = __ldg(gm1 + 4 * (i + 1));
-      s0 = __ldg(st0 + i + 1); s1 = __ldg(st1 + i + 1);
-    }
-    const float4 G = __ldg(gs);  // (2^-a/16, -16 X) of groups 2c and 2c+1
-    gs += 4;
-    const int s = i % GEMV_RING;
-    if (!mbar_wait_suspend(bar0 + 8 * s, (uint32_t)((i / GEMV_RING) & 1), &abort_flag)) break;
-    const uint32_t stg = ring + s * GEMV_STAGE_BYTES;
-    const uint4 a00 = lds128(stg + o00), a10 = lds128(stg + o10);  // (r0 | r1, group c)
-    const uint4 a01 = lds128(stg + o01), a11 = lds128(stg + o11);  // (r0 | r1, group c+4)
-    __syncwarp();  // every lane has read the stage: the next turn may refill it
-    int32_t dh[4] = {GEMV_ACC0, GEMV_ACC0, GEMV_ACC0, GEMV_ACC0};
-    int32_t dl[4] = {GEMV_ACC0, GEMV_ACC0, GEMV_ACC0, GEMV_ACC0};
-    const uint32_t w00[4] = {a00.x, a00.y, a00.z, a00.w}, w01[4] = {a01.x, a01.y, a01.z, a01.w};
-    const uint32_t w10[4] = {a10.x, a10.y, a10.z, a10.w}, w11[4] = {a11.x, a11.y, a11.z, a11.w};
+  bool ok = true;
+  for (int base = 0; base < nsb && ok; base += GEMV_RING) {
+    const uint32_t par = (uint32_t)((base / GEMV_RING) & 1);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint4 xv0 = __ldg(xb0 + j), xv1 = __ldg(xb1 + j);
-      const uint32_t h00 = w00[j] & 0xF0F0F0F0u, h10 = w10[j] & 0xF0F0F0F0u;  // odd k, x16
-      const uint32_t h01 = w01[j] & 0xF0F0F0F0u, h11 = w11[j] & 0xF0F0F0F0u;
-      QL_IMMA("s8", dh, h00, h10, h01, h11, xv0.z, xv1.z);
-      QL_IMMA("u8", dl, h00, h10, h01, h11, xv0.w, xv1.w);
-      const uint32_t e00 = (w00[j] << 4) & 0xF0F0F0F0u, e10 = (w10[j] << 4) & 0xF0F0F0F0u;  // even k, x16
-      const uint32_t e01 = (w01[j] << 4) & 0xF0F0F0F0u, e11 = (w11[j] << 4) & 0xF0F0F0F0u;
-      QL_IMMA("s8", dh, e00, e10, e01, e11, xv0.x, xv1.x);
-      QL_IMMA("u8", dl, e00, e10, e01, e11, xv0.y, xv1.y);
-    }
-    xb0 += xinc0;
-    xb1 += xinc1;
-    // D[q]: q = 0 (r0, group 2c), 1 (r0, 2c+1), 2 (r1, 2c), 3 (r1, 2c+1)
-    float t[4];
+    for (int s = 0; s < GEMV_RING; ++s) {
+      const int i = base + s;
+      if (i >= nsb) break;
+      // refill the stage released by the previous super-block with super-block i + RING - 1
+      const int nx = i + GEMV_RING - 1;
+      const int sn = (s + GEMV_RING - 1) % GEMV_RING;
+      __syncwarp();  // every lane has read that stage in the previous turn
+      if (nx < nsb) {
+        if (lane == 0) {
+          issue_w(nx, sn);
+          issue_x(nx, sn);
+          issued = nx + 1;
+        }
+        sr0[sn] = __ldg(st0 + nx);
+        sr1[sn] = __ldg(st1 + nx);
+      }
+      if (!mbar_wait_suspend(bar0 + 8 * s, par, &abort_flag)) {
+        ok = false;
+        break;
+      }
+      const uint32_t so = s * GEMV_STAGE_BYTES;
+      const uint4 w00 = lds128(a00 + so), w10 = lds128(a10 + so);  // (r0 | r1, group c)
+      const uint4 w01 = lds128(a01 + so), w11 = lds128(a11 + so);  // (r0 | r1, group c+4)
+      const float4 G = lds128f(ag + so);                           // (2^-a/16, -16 X) of groups 2c, 2c+1
+      const uint32_t cm0 = lds32(am + so), cm1 = lds32(am + so + 128);
+      const uint32_t ww00[4] = {w00.x, w00.y, w00.z, w00.w}, ww01[4] = {w01.x, w01.y, w01.z, w01.w};
+      const uint32_t ww10[4] = {w10.x, w10.y, w10.z, w10.w}, ww11[4] = {w11.x, w11.y, w11.z, w11.w};
+      int32_t dh[4], dl[4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-      t[q] = fmaf(__int_as_float(dh[q]) - GEMV_ACC0_F, 256.f, __int_as_float(dl[q]) - GEMV_ACC0_F);
-    // S = sc * ss and Z = zc * zs, each one FMA from the byte placed in the mantissa of 2^23
-    const float ss0 = f16_bits_to_f32(cs0), zs0 = f16_bits_to_f32(cs0 >> 16);
-    const float ss1 = f16_bits_to_f32(cs1), zs1 = f16_bits_to_f32(cs1 >> 16);
-    const float nss0 = -8388608.f * ss0, nzs0 = -8388608.f * zs0;
-    const float nss1 = -8388608.f * ss1, nzs1 = -8388608.f * zs1;
-    const float S00 = fmaf(byte_magic(cm0, 0), ss0, nss0) * G.x, Z00 = fmaf(byte_magic(cm0, 1), zs0, nzs0);
-    const float S01 = fmaf(byte_magic(cm0, 2), ss0, nss0) * G.z, Z01 = fmaf(byte_magic(cm0, 3), zs0, nzs0);
-    const float S10 = fmaf(byte_magic(cm1, 0), ss1, nss1) * G.x, Z10 = fmaf(byte_magic(cm1, 1), zs1, nzs1);
-    const float S11 = fmaf(byte_magic(cm1, 2), ss1, nss1) * G.z, Z11 = fmaf(byte_magic(cm1, 3), zs1, nzs1);
-    acc0 = fmaf(S00, fmaf(Z00, G.y, t[0]), acc0);
-    acc0 = fmaf(S01, fmaf(Z01, G.w, t[1]), acc0);
-    acc1 = fmaf(S10, fmaf(Z10, G.y, t[2]), acc1);
-    acc1 = fmaf(S11, fmaf(Z11, G.w, t[3]), acc1);
+      for (int j = 0; j < 4; ++j) {
+        const uint4 xv0 = lds128(xa0[s] + 128 * j), xv1 = lds128(xa1[s] + 128 * j);
+        const uint32_t h00 = ww00[j] & 0xF0F0F0F0u, h10 = ww10[j] & 0xF0F0F0F0u;  // odd k, x16
+        const uint32_t h01 = ww01[j] & 0xF0F0F0F0u, h11 = ww11[j] & 0xF0F0F0F0u;
+        if (j == 0) {
+          QL_IMMA0("s8", dh, GEMV_ACC0, h00, h10, h01, h11, xv0.z, xv1.z);
+          QL_IMMA0("u8", dl, GEMV_ACC0, h00, h10, h01, h11, xv0.w, xv1.w);
+        } else {
+          QL_IMMA("s8", dh, h00, h10, h01, h11, xv0.z, xv1.z);
+          QL_IMMA("u8", dl, h00, h10, h01, h11, xv0.w, xv1.w);
+        }
+        const uint32_t e00 = (ww00[j] << 4) & 0xF0F0F0F0u, e10 = (ww10[j] << 4) & 0xF0F0F0F0u;  // even k, x16
+        const uint32_t e01 = (ww01[j] << 4) & 0xF0F0F0F0u, e11 = (ww11[j] << 4) & 0xF0F0F0F0u;
+        QL_IMMA("s8", dh, e00, e10, e01, e11, xv0.x, xv1.x);
+        QL_IMMA("u8", dl, e00, e10, e01, e11, xv0.y, xv1.y);
+      }
+      // D[q]: q = 0 (r0, group 2c), 1 (r0, 2c+1), 2 (r1, 2c), 3 (r1, 2c+1)
+      float t[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        t[q] = fmaf(__int_as_float(dh[q]) - GEMV_ACC0_F, 256.f, __int_as_float(dl[q]) - GEMV_ACC0_F);
+      // S = sc * ss and Z = zc * zs, each one FMA from the byte placed in the mantissa of 2^23
+      const uint32_t cs0 = sr0[s], cs1 = sr1[s];
+      const float ss0 = f16_bits_to_f32(cs0), zs0 = f16_bits_to_f32(cs0 >> 16);
+      const float ss1 = f16_bits_to_f32(cs1), zs1 = f16_bits_to_f32(cs1 >> 16);
+      const float nss0 = -8388608.f * ss0, nzs0 = -8388608.f * zs0;
+      const float nss1 = -8388608.f * ss1, nzs1 = -8388608.f * zs1;
+      const float S00 = fmaf(byte_magic(cm0, 0), ss0, nss0) * G.x, Z00 = fmaf(byte_magic(cm0, 1), zs0, nzs0);
+      const float S01 = fmaf(byte_magic(cm0, 2), ss0, nss0) * G.z, Z01 = fmaf(byte_magic(cm0, 3), zs0, nzs0);
+      const float S10 = fmaf(byte_magic(cm1, 0), ss1, nss1) * G.x, Z10 = fmaf(byte_magic(cm1, 1), zs1, nzs1);
+      const float S11 = fmaf(byte_magic(cm1, 2), ss1, nss1) * G.z, Z11 = fmaf(byte_magic(cm1, 3), zs1, nzs1);
+      acc0 = fmaf(S00, fmaf(Z00, G.y, t[0]), acc0);
+      acc0 = fmaf(S01, fmaf(Z01, G.w, t[1]), acc0);
+      acc1 = fmaf(S10, fmaf(Z10, G.y, t[2]), acc1);
+      acc1 = fmaf(S11, fmaf(Z11, G.w, t[3]), acc1);
+    }
   }
-  if (abort_flag && lane == 0) {  // a wait gave up: let this warp's copies in flight land first
+  if (!ok && lane == 0) {  // a wait gave up: let this warp's copies in flight land first
     for (int i = issued - GEMV_RING; i < issued; ++i) {
       if (i < 0) continue;
       const long long t0 = clock64();

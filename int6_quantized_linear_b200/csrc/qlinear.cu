@@ -175,15 +175,17 @@ ql_status launch_gemv(const ql_desc *d, const ql_packed_const *w, const void *x,
       const int64_t ng = M * (d->K / 32);
       gemv_xprep_kernel<<<(int)((ng + 255) / 256), 256, 0, st>>>(xb, M, d->K, ws);
       GemvTcParams p;
-      p.gmeta = static_cast<const uint8_t *>(w->gmeta);
       p.steps = static_cast<const uint8_t *>(w->steps);
       p.N = d->N;
       p.K = d->K;
       p.ws = ws;
       p.y = yb;
-      CUtensorMap mc;  // codes as [N][K/2] bytes, boxes of 16 rows x 128 bytes, 128-byte swizzle
+      CUtensorMap mc, mg;  // codes as [N][K/2] bytes, boxes of 16 rows x 128 bytes, 128-byte swizzle;
+                           // group words as [N][K/16] bytes, boxes of 16 rows x 16 bytes
       if (!encode_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->codes, (uint64_t)d->K / 2, (uint64_t)d->N,
-                     (uint64_t)d->K / 2, 128, 16, CU_TENSOR_MAP_SWIZZLE_128B))
+                     (uint64_t)d->K / 2, 128, 16, CU_TENSOR_MAP_SWIZZLE_128B) ||
+          !encode_2d(&mg, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->gmeta, (uint64_t)d->K / 16, (uint64_t)d->N,
+                     (uint64_t)d->K / 16, 16, 16, CU_TENSOR_MAP_SWIZZLE_NONE))
         return QL_ERR_CUDA;
       const int64_t NS = d->K / 256, n_tiles = (d->N + 15) / 16;
       // split K over more warps per tile while the grid still fits one wave (4 CTAs per SM)
@@ -211,7 +213,7 @@ ql_status launch_gemv(const ql_desc *d, const ql_packed_const *w, const void *x,
       attr[0].val.programmaticStreamSerializationAllowed = 1;
       cfg.attrs = attr;
       cfg.numAttrs = 1;
-      if (cudaLaunchKernelEx(&cfg, gemv_int4_m1_tc_kernel, mc, p) != cudaSuccess) return QL_ERR_CUDA;
+      if (cudaLaunchKernelEx(&cfg, gemv_int4_m1_tc_kernel, mc, mg, p) != cudaSuccess) return QL_ERR_CUDA;
       return launched();
     }
   }
