@@ -93,19 +93,19 @@ __global__ void __launch_bounds__(256) gemv_simple_kernel(WeightPtrs p, int64_t 
 // ===========================================================================
 
 struct GemvWorkspace {
-  uint4 *xq;      // [M][K/256 super-blocks][4 j][8 groups][16 B]: (even-k hi, even-k lo, odd-k hi, odd-k lo) bytes
+  uint4 *xq;      // [M][K/256 super-blocks][4 j][2 kinds][8 groups][16 B]: B-operand pairs, see gemv_xprep_kernel
   float2 *gsum;   // [M][K/32] (2^-a_g / 16, -16 * sum x_int)
 };
 
 inline size_t gemv_workspace_bytes(int64_t M, int64_t K) {
-  return align256((size_t)M * K * 2) + align256((size_t)M * (K / 32) * 8);
+  return align256((size_t)M * K * 4) + align256((size_t)M * (K / 32) * 8);
 }
 
 inline GemvWorkspace gemv_workspace_carve(void *base, int64_t M, int64_t K) {
   uint8_t *p = static_cast<uint8_t *>(base);
   GemvWorkspace w;
   w.xq = reinterpret_cast<uint4 *>(p);
-  p += align256((size_t)M * K * 2);
+  p += align256((size_t)M * K * 4);
   w.gsum = reinterpret_cast<float2 *>(p);
   return w;
 }
@@ -114,6 +114,9 @@ QL_DEVI void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_depen
 QL_DEVI void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 // One thread per 32-element group of x: fixed-point conversion, byte split in fragment order, sum.
+// Chunk (j, kind) of group grp is the register quad its feeding lane loads: the high-byte and low-byte
+// words of k = 8j + kind + {0, 2, 4, 6}, each paired with a zero word so that one 16-byte load gives
+// the B pairs of two MMAs -- (x, 0) for groups 0-3 (their lanes feed b0), (0, x) for groups 4-7 (b1).
 __global__ void __launch_bounds__(256) gemv_xprep_kernel(const __nv_bfloat16 *x, int64_t M, int64_t K,
                                                          GemvWorkspace ws) {
   pdl_launch_dependents();
@@ -143,12 +146,11 @@ __global__ void __launch_bounds__(256) gemv_xprep_kernel(const __nv_bfloat16 *x,
     xi[k] = __float2int_rn(xs[k] * sc);
     sum += xi[k];
   }
-  // group gi = (m, super-block sb, group-in-block grp): chunk j goes to [m][sb][j][grp]
+  // group gi = (m, super-block sb, group-in-block grp): chunk (j, kind) goes to [m][sb][j][kind][grp]
   const int64_t grp = gi & 7, msb = gi >> 3;
-  uint4 *dst = ws.xq + msb * 32 + grp;
+  uint4 *dst = ws.xq + msb * 64 + grp;
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    uint32_t o[4];
 #pragma unroll
     for (int kind = 0; kind < 2; ++kind) {
       uint32_t hi = 0, lo = 0;
@@ -158,10 +160,8 @@ __global__ void __launch_bounds__(256) gemv_xprep_kernel(const __nv_bfloat16 *x,
         hi |= ((uint32_t)(v >> 8) & 0xffu) << (8 * b);
         lo |= ((uint32_t)v & 0xffu) << (8 * b);
       }
-      o[2 * kind] = hi;
-      o[2 * kind + 1] = lo;
+      dst[8 * (2 * j + kind)] = grp < 4 ? make_uint4(hi, 0u, lo, 0u) : make_uint4(0u, hi, 0u, lo);
     }
-    dst[8 * j] = make_uint4(o[0], o[1], o[2], o[3]);
   }
   ws.gsum[gi] = make_float2(exp2i(-a) * 0.0625f, -16.f * (float)sum);
 }
@@ -214,9 +214,9 @@ QL_DEVI bool mbar_wait_suspend(uint32_t bar, uint32_t parity, volatile int *abor
 // high (signed) or low (unsigned) x bytes
 #define QL_IMMA0(TB, ACC, C, A0, A1, A2, A3, B0, B1)                                                  \
   asm("mma.sync.aligned.m16n8k32.row.col.s32.u8." TB ".s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "  \
-      "{%10,%10,%10,%10};"                                                                              \
+      "{%10,%11,%12,%13};"                                                                              \
       : "=r"(ACC[0]), "=r"(ACC[1]), "=r"(ACC[2]), "=r"(ACC[3])                                        \
-      : "r"(A0), "r"(A1), "r"(A2), "r"(A3), "r"(B0), "r"(B1), "r"(C))
+      : "r"(A0), "r"(A1), "r"(A2), "r"(A3), "r"(B0), "r"(B1), "r"(C[0]), "r"(C[1]), "r"(C[2]), "r"(C[3]))
 #define QL_IMMA(TB, ACC, A0, A1, A2, A3, B0, B1)                                                      \
   asm("mma.sync.aligned.m16n8k32.row.col.s32.u8." TB ".s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "  \
       "{%0,%1,%2,%3};"                                                                                  \
@@ -224,13 +224,14 @@ QL_DEVI bool mbar_wait_suspend(uint32_t bar, uint32_t parity, volatile int *abor
       : "r"(A0), "r"(A1), "r"(A2), "r"(A3), "r"(B0), "r"(B1))
 
 constexpr int GEMV_RING = 4;   // super-blocks in flight per warp
+constexpr int GEMV_CTAS_PER_SM = 3;
 constexpr int GEMV_WARPS = 4;  // warps per CTA: GEMV_WARPS / parts tiles, each split over `parts` warps
 // one stage = one super-block of a 16-row tile: codes (16 rows x 128 B, 128-byte swizzle), the
-// tile's group words [16 rows][16 B], the super-block's x bytes [4 j][8 groups][16 B], its 8 group sums
-constexpr int GEMV_ST_CODES = 0, GEMV_ST_GMETA = 2048, GEMV_ST_X = 2304, GEMV_ST_GSUM = 2816;
-constexpr int GEMV_STAGE_BYTES = 3072;      // multiple of 1024 (the swizzle atom)
-constexpr uint32_t GEMV_STAGE_TX = 2048 + 512 + 64 + 256;
-constexpr int GEMV_ZERO_BYTES = 512;        // zero x chunks at a 128-byte stride, for lanes that feed no x
+// tile's group words [16 rows][16 B], the super-block's 8 group sums, its x pairs [4 j][2 kinds][8 groups][16 B]
+constexpr int GEMV_ST_CODES = 0, GEMV_ST_GMETA = 2048, GEMV_ST_GSUM = 2304, GEMV_ST_X = 2368;
+constexpr int GEMV_STAGE_BYTES = 4096;      // multiple of 1024 (the swizzle atom)
+constexpr uint32_t GEMV_STAGE_TX = 2048 + 256 + 64 + 1024;
+constexpr int GEMV_ZERO_BYTES = 1024;       // zero x chunks at a 128-byte stride, for lanes that feed no x
 constexpr int32_t GEMV_ACC0 = 0x4B400000;    // 1.5 * 2^23 as float bits: integer sums below 2^22 read back exactly
 constexpr float GEMV_ACC0_F = 12582912.f;
 
@@ -255,7 +256,7 @@ inline constexpr int gemv_smem_bytes() {
 // one 8-lane shared-load phase differ in bit 2 and their chunks never share banks.  The loop runs
 // RING super-blocks per turn so every shared-memory offset is a constant; step words come through
 // the L1 cache RING - 1 super-blocks ahead.
-__global__ void __launch_bounds__(32 * GEMV_WARPS, 4)
+__global__ void __launch_bounds__(32 * GEMV_WARPS, GEMV_CTAS_PER_SM)
     gemv_int4_m1_tc_kernel(const __grid_constant__ CUtensorMap map_codes,
                            const __grid_constant__ CUtensorMap map_gmeta, GemvTcParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -283,7 +284,7 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS, 4)
     fence_mbar_init();
   }
   __syncthreads();
-  const uint8_t *xq_sb = reinterpret_cast<const uint8_t *>(p.ws.xq) + (int64_t)sb0 * 512;  // M = 1
+  const uint8_t *xq_sb = reinterpret_cast<const uint8_t *>(p.ws.xq) + (int64_t)sb0 * 1024;  // M = 1
   const uint8_t *gs_sb = reinterpret_cast<const uint8_t *>(p.ws.gsum) + (int64_t)sb0 * 64;
   // stage s of super-block i: weights (codes, group words) need no x; x and sums come after pdl_wait
   auto issue_w = [&](int i, int s) {
@@ -294,7 +295,7 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS, 4)
   };
   auto issue_x = [&](int i, int s) {
     const uint32_t st = ring + s * GEMV_STAGE_BYTES, bar = bar0 + 8 * s;
-    bulk_load(st + GEMV_ST_X, xq_sb + (int64_t)i * 512, 512, bar);
+    bulk_load(st + GEMV_ST_X, xq_sb + (int64_t)i * 1024, 1024, bar);
     bulk_load(st + GEMV_ST_GSUM, gs_sb + (int64_t)i * 64, 64, bar);
   };
   const int pre = nsb < GEMV_RING - 1 ? nsb : GEMV_RING - 1;
@@ -327,17 +328,18 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS, 4)
   // per-lane shared-memory addresses (offsets inside a stage are added as constants)
   const bool on0 = (g == c), on1 = (g == c + 4);
   const uint32_t zero_a = smem_u32(zero_blk);
-  uint32_t xa0[GEMV_RING], xa1[GEMV_RING];  // x chunk j of this lane's b0 / b1 at xa + 128 j
+  uint32_t xa[GEMV_RING];  // this lane's B pairs of MMA step (j, kind) at xa + 128 (2 j + kind)
 #pragma unroll
   for (int s = 0; s < GEMV_RING; ++s) {
-    xa0[s] = on0 ? ring + s * GEMV_STAGE_BYTES + GEMV_ST_X + 16 * c : zero_a;
-    xa1[s] = on1 ? ring + s * GEMV_STAGE_BYTES + GEMV_ST_X + 16 * (c + 4) : zero_a;
+    xa[s] = on0 ? ring + s * GEMV_STAGE_BYTES + GEMV_ST_X + 16 * c
+          : on1 ? ring + s * GEMV_STAGE_BYTES + GEMV_ST_X + 16 * (c + 4) : zero_a;
   }
   const uint32_t a00 = ring + pg * 128 + ((c ^ pg) << 4), a01 = ring + pg * 128 + (((c + 4) ^ pg) << 4);
   const uint32_t a10 = a00 + 1024, a11 = a01 + 1024;  // row pg + 8: same swizzle phase, next atom
   const uint32_t ag = ring + GEMV_ST_GSUM + 16 * c;
   const uint32_t am = ring + GEMV_ST_GMETA + pg * 16 + 4 * c;
 
+  const int32_t acc_init[4] = {GEMV_ACC0, GEMV_ACC0, GEMV_ACC0, GEMV_ACC0};
   float acc0 = 0.f, acc1 = 0.f;
   bool ok = true;
   for (int base = 0; base < nsb && ok; base += GEMV_RING) {
@@ -373,20 +375,20 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS, 4)
       int32_t dh[4], dl[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const uint4 xv0 = lds128(xa0[s] + 128 * j), xv1 = lds128(xa1[s] + 128 * j);
+        const uint4 xe = lds128(xa[s] + 256 * j), xo = lds128(xa[s] + 256 * j + 128);  // even k, odd k
         const uint32_t h00 = ww00[j] & 0xF0F0F0F0u, h10 = ww10[j] & 0xF0F0F0F0u;  // odd k, x16
         const uint32_t h01 = ww01[j] & 0xF0F0F0F0u, h11 = ww11[j] & 0xF0F0F0F0u;
         if (j == 0) {
-          QL_IMMA0("s8", dh, GEMV_ACC0, h00, h10, h01, h11, xv0.z, xv1.z);
-          QL_IMMA0("u8", dl, GEMV_ACC0, h00, h10, h01, h11, xv0.w, xv1.w);
+          QL_IMMA0("s8", dh, acc_init, h00, h10, h01, h11, xo.x, xo.y);
+          QL_IMMA0("u8", dl, acc_init, h00, h10, h01, h11, xo.z, xo.w);
         } else {
-          QL_IMMA("s8", dh, h00, h10, h01, h11, xv0.z, xv1.z);
-          QL_IMMA("u8", dl, h00, h10, h01, h11, xv0.w, xv1.w);
+          QL_IMMA("s8", dh, h00, h10, h01, h11, xo.x, xo.y);
+          QL_IMMA("u8", dl, h00, h10, h01, h11, xo.z, xo.w);
         }
         const uint32_t e00 = (ww00[j] << 4) & 0xF0F0F0F0u, e10 = (ww10[j] << 4) & 0xF0F0F0F0u;  // even k, x16
         const uint32_t e01 = (ww01[j] << 4) & 0xF0F0F0F0u, e11 = (ww11[j] << 4) & 0xF0F0F0F0u;
-        QL_IMMA("s8", dh, e00, e10, e01, e11, xv0.x, xv1.x);
-        QL_IMMA("u8", dl, e00, e10, e01, e11, xv0.y, xv1.y);
+        QL_IMMA("s8", dh, e00, e10, e01, e11, xe.x, xe.y);
+        QL_IMMA("u8", dl, e00, e10, e01, e11, xe.z, xe.w);
       }
       // D[q]: q = 0 (r0, group 2c), 1 (r0, 2c+1), 2 (r1, 2c), 3 (r1, 2c+1)
       float t[4];

@@ -188,8 +188,8 @@ ql_status launch_gemv(const ql_desc *d, const ql_packed_const *w, const void *x,
                      (uint64_t)d->K / 16, 16, 16, CU_TENSOR_MAP_SWIZZLE_NONE))
         return QL_ERR_CUDA;
       const int64_t NS = d->K / 256, n_tiles = (d->N + 15) / 16;
-      // split K over more warps per tile while the grid still fits one wave (4 CTAs per SM)
-      const int64_t slots = (int64_t)sms * 4;
+      // split K over more warps per tile while the grid still fits one wave
+      const int64_t slots = (int64_t)sms * GEMV_CTAS_PER_SM;
       int P = 1;
       while (2 * P <= GEMV_WARPS && 2 * P <= NS && (n_tiles * 2 * P + GEMV_WARPS - 1) / GEMV_WARPS <= slots) P *= 2;
       p.parts = P;
