@@ -119,7 +119,8 @@ QL_DEVI void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 // the B pairs of two MMAs -- (x, 0) for groups 0-3 (their lanes feed b0), (0, x) for groups 4-7 (b1).
 __global__ void __launch_bounds__(256) gemv_xprep_kernel(const __nv_bfloat16 *x, int64_t M, int64_t K,
                                                          GemvWorkspace ws) {
-  pdl_launch_dependents();
+  pdl_launch_dependents();  // the streaming kernel may start fetching weights now
+  pdl_wait();               // x (and this workspace) may belong to the kernel launched before this one
   const int64_t ng = K / 32;
   const int64_t gi = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;  // over M * ng
   if (gi >= M * ng) return;
@@ -284,6 +285,9 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS, GEMV_CTAS_PER_SM)
     fence_mbar_init();
   }
   __syncthreads();
+  // the next call's preparation pass may be scheduled as this grid's CTAs retire; it waits for this
+  // grid to finish before touching x or the workspace
+  pdl_launch_dependents();
   const uint8_t *xq_sb = reinterpret_cast<const uint8_t *>(p.ws.xq) + (int64_t)sb0 * 1024;  // M = 1
   const uint8_t *gs_sb = reinterpret_cast<const uint8_t *>(p.ws.gsum) + (int64_t)sb0 * 64;
   // stage s of super-block i: weights (codes, group words) need no x; x and sums come after pdl_wait

@@ -173,7 +173,18 @@ ql_status launch_gemv(const ql_desc *d, const ql_packed_const *w, const void *x,
     if (M == 1) {  // tensor-core path: preparation pass, then the streaming kernel as its dependent
       const GemvWorkspace ws = gemv_workspace_carve(workspace, M, d->K);
       const int64_t ng = M * (d->K / 32);
-      gemv_xprep_kernel<<<(int)((ng + 255) / 256), 256, 0, st>>>(xb, M, d->K, ws);
+      {  // programmatic dependent of whatever precedes it on the stream (it waits before reading x)
+        cudaLaunchConfig_t pc = {};
+        pc.gridDim = dim3((unsigned)((ng + 255) / 256));
+        pc.blockDim = dim3(256);
+        pc.stream = st;
+        cudaLaunchAttribute pa[1];
+        pa[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        pa[0].val.programmaticStreamSerializationAllowed = 1;
+        pc.attrs = pa;
+        pc.numAttrs = 1;
+        if (cudaLaunchKernelEx(&pc, gemv_xprep_kernel, xb, M, (int64_t)d->K, ws) != cudaSuccess) return QL_ERR_CUDA;
+      }
       GemvTcParams p;
       p.steps = static_cast<const uint8_t *>(w->steps);
       p.N = d->N;
