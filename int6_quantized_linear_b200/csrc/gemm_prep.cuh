@@ -65,7 +65,10 @@ QL_DEVI int scale_exponent(float amax, int top) {
   return s < -126 ? -126 : (s > 126 ? 126 : s);
 }
 
-// One warp per token row: find max|x|, then write the scaled fp16 row.
+// One warp per token row: find max|x|, then write the scaled fp16 row.  Within every 8-element
+// chunk the elements are stored in the order k = 0,4,1,5,2,6,3,7 (pairs (0,4) (1,5) (2,6) (3,7)):
+// the weight operand is written in the same order, which is the order a single bit operation
+// pulls nibble pairs out of a code word (the MMA's sum over k does not depend on it).
 __global__ void __launch_bounds__(256) x_to_f16_kernel(const __nv_bfloat16 *x, int64_t M, int64_t K,
                                                         GemmWorkspace ws) {
   const int lane = threadIdx.x & 31;
@@ -91,8 +94,11 @@ __global__ void __launch_bounds__(256) x_to_f16_kernel(const __nv_bfloat16 *x, i
     const uint32_t u[4] = {v.x, v.y, v.z, v.w};
     uint32_t o[4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const __half2 h = __floats2half2_rn(__uint_as_float(u[j] << 16) * sc, __uint_as_float(u[j] & 0xffff0000u) * sc);
+    for (int j = 0; j < 4; ++j) {  // pair j = (x[j], x[j + 4]): u[j / 2] holds x[j & ~1], x[j | 1]
+      const uint32_t a = u[j >> 1], b = u[2 + (j >> 1)];
+      const float lo = (j & 1) ? __uint_as_float(a & 0xffff0000u) : __uint_as_float(a << 16);
+      const float hi = (j & 1) ? __uint_as_float(b & 0xffff0000u) : __uint_as_float(b << 16);
+      const __half2 h = __floats2half2_rn(lo * sc, hi * sc);
       o[j] = *reinterpret_cast<const uint32_t *>(&h);
     }
     out[i] = make_uint4(o[0], o[1], o[2], o[3]);

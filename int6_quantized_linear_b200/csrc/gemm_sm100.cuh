@@ -323,19 +323,50 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
       for (int rr = 0; rr < 2; ++rr) {
         const int r = rr ? r1 : r0;
-        float w[32];
-        smem_decode32<FMT, BITS>(P + r * PROW + h * (PROW / 2), rr ? gm1 : gm0, rr ? st1 : st0, w);
         const float sc = rr ? sc1 : sc0;
         uint8_t *row = B + (r >> 3) * 1024 + (r & 7) * 128;
+        // each 16-byte chunk holds k = 0,4,1,5,2,6,3,7 of its 8 weights (the order of the x tile)
+        if constexpr (FMT == FMT_INT4) {
+          // packed-half arithmetic: q as 1024+q / 64+q from one bit operation, then
+          // w * 2^b_n = q * S' - Z * S' in fp16 with S' = S * 2^b_n
+          const uint32_t gm = rr ? gm1 : gm0, st = rr ? st1 : st0;
+          const float S = __fmul_rn((float)(gm & 0xffu), f16_bits_to_f32(st)) * sc;
+          const float ZS = __fmul_rn((float)((gm >> 8) & 0xffu), f16_bits_to_f32(st >> 16)) * S;
+          const __half2 s2 = __float2half2_rn(S), nz2 = __float2half2_rn(-ZS);
+          const __half2 m1024 = __float2half2_rn(1024.f), m64 = __float2half2_rn(64.f);
+          const uint4 cv = *reinterpret_cast<const uint4 *>(P + r * PROW + h * (PROW / 2));
+          const uint32_t cw[4] = {cv.x, cv.y, cv.z, cv.w};
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int j = 4 * h + q;  // logical 16-byte chunk of the 128-byte row
-          uint4 v;
-          v.x = pack_f16x2(w[8 * q + 0] * sc, w[8 * q + 1] * sc);
-          v.y = pack_f16x2(w[8 * q + 2] * sc, w[8 * q + 3] * sc);
-          v.z = pack_f16x2(w[8 * q + 4] * sc, w[8 * q + 5] * sc);
-          v.w = pack_f16x2(w[8 * q + 6] * sc, w[8 * q + 7] * sc);
-          *reinterpret_cast<uint4 *>(row + ((j ^ (r & 7)) << 4)) = v;
+          for (int q = 0; q < 4; ++q) {
+            const uint32_t wd = cw[q], w8 = wd >> 8;
+            uint32_t pr[4];
+            pr[0] = (wd & 0x000F000Fu) | 0x64006400u;  // (1024 + n0, 1024 + n4)
+            pr[1] = (wd & 0x00F000F0u) | 0x54005400u;  // (64 + n1, 64 + n5)
+            pr[2] = (w8 & 0x000F000Fu) | 0x64006400u;  // (1024 + n2, 1024 + n6)
+            pr[3] = (w8 & 0x00F000F0u) | 0x54005400u;  // (64 + n3, 64 + n7)
+            uint32_t o[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const __half2 qv = __hsub2(*reinterpret_cast<const __half2 *>(&pr[e]), (e & 1) ? m64 : m1024);
+              const __half2 wv = __hfma2(qv, s2, nz2);
+              o[e] = *reinterpret_cast<const uint32_t *>(&wv);
+            }
+            const int j = 4 * h + q;  // logical 16-byte chunk of the 128-byte row
+            *reinterpret_cast<uint4 *>(row + ((j ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+          }
+        } else {
+          float w[32];
+          smem_decode32<FMT, BITS>(P + r * PROW + h * (PROW / 2), rr ? gm1 : gm0, rr ? st1 : st0, w);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int j = 4 * h + q;  // logical 16-byte chunk of the 128-byte row
+            uint4 v;
+            v.x = pack_f16x2(w[8 * q + 0] * sc, w[8 * q + 4] * sc);
+            v.y = pack_f16x2(w[8 * q + 1] * sc, w[8 * q + 5] * sc);
+            v.z = pack_f16x2(w[8 * q + 2] * sc, w[8 * q + 6] * sc);
+            v.w = pack_f16x2(w[8 * q + 3] * sc, w[8 * q + 7] * sc);
+            *reinterpret_cast<uint4 *>(row + ((j ^ (r & 7)) << 4)) = v;
+          }
         }
       }
       fence_proxy_async_smem();
