@@ -3,7 +3,7 @@
 //   y[M][N] = x[M][K] . W^T,  x bf16, W quantized, y bf16, fp32 accumulation
 //
 // Persistent kernel, one CTA per SM, tiles of BM=128 tokens x BN=256 weight
-// rows, K streamed in BK=64 steps through a STAGES-deep shared-memory ring.
+// rows, K streamed in BK=64 steps through a 3- or 4-deep shared-memory ring.
 // Warp roles:
 //   warp 0      TMA producer: scaled fp16 x tile (128 x 64, 128-byte
 //               swizzle) and the packed code tile (256 rows x BK codes)
@@ -31,7 +31,6 @@ namespace gemm {
 constexpr int BM = 128;
 constexpr int BN = 256;
 constexpr int BK = 64;
-constexpr int STAGES = 3;
 constexpr int NUM_DEQ_WARPS = 8;
 constexpr int WARP_TMA = 0;
 constexpr int WARP_MMA = 1;
@@ -48,20 +47,24 @@ __host__ __device__ constexpr int code_bits(int fmt, int bits) {
 __host__ __device__ constexpr int p_row_bytes(int fmt, int bits) { return BK * code_bits(fmt, bits) / 8; }
 __host__ __device__ constexpr int p_bytes(int fmt, int bits) { return BN * p_row_bytes(fmt, bits); }
 
+// Stages of the ring: four when they fit in the 227 KB a CTA may use, else three.
+constexpr int NUM_BARS_PER_STAGE = 3;  // tma_full, b_full, empty
+constexpr int NUM_BARS_FIXED = 5;      // acc_full[2], acc_empty[2], final
+__host__ __device__ constexpr int stage_bytes(int fmt, int bits) { return A_BYTES + B_BYTES + p_bytes(fmt, bits); }
+__host__ __device__ constexpr int smem_need(int fmt, int bits, int st) {
+  return st * stage_bytes(fmt, bits) + (NUM_BARS_PER_STAGE * st + NUM_BARS_FIXED) * 8 + 16 + 1024;
+}
+__host__ __device__ constexpr int stages(int fmt, int bits) { return smem_need(fmt, bits, 4) <= 232448 ? 4 : 3; }
+
 // byte offsets inside the dynamic shared memory (base aligned to 1024)
 __host__ __device__ constexpr int off_a(int s) { return s * A_BYTES; }
-__host__ __device__ constexpr int off_b(int s) { return STAGES * A_BYTES + s * B_BYTES; }
+__host__ __device__ constexpr int off_b(int fmt, int bits, int s) { return stages(fmt, bits) * A_BYTES + s * B_BYTES; }
 __host__ __device__ constexpr int off_p(int fmt, int bits, int s) {
-  return STAGES * (A_BYTES + B_BYTES) + s * p_bytes(fmt, bits);
+  return stages(fmt, bits) * (A_BYTES + B_BYTES) + s * p_bytes(fmt, bits);
 }
-__host__ __device__ constexpr int off_bar(int fmt, int bits) {
-  return STAGES * (A_BYTES + B_BYTES + p_bytes(fmt, bits));
-}
-// barriers: tma_full[S], b_full[S], empty[S], acc_full[2], acc_empty[2], final
-constexpr int NUM_BARS = 3 * STAGES + 5;
-__host__ __device__ constexpr int smem_bytes(int fmt, int bits) {
-  return off_bar(fmt, bits) + NUM_BARS * 8 + 16 /* tmem base + abort flag */ + 1024 /* alignment slack */;
-}
+__host__ __device__ constexpr int off_bar(int fmt, int bits) { return stages(fmt, bits) * stage_bytes(fmt, bits); }
+// barriers: tma_full[S], b_full[S], empty[S], acc_full[2], acc_empty[2], final (+ tmem base, abort flag)
+__host__ __device__ constexpr int smem_bytes(int fmt, int bits) { return smem_need(fmt, bits, stages(fmt, bits)); }
 
 struct Params {
   int64_t M, N, K;
@@ -127,12 +130,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_codes,
                 Params p) {
   constexpr int PROW = p_row_bytes(FMT, BITS);
+  constexpr int STAGES = stages(FMT, BITS);
   constexpr uint32_t STAGE_TX = A_BYTES + p_bytes(FMT, BITS);
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + off_bar(FMT, BITS));
-  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + NUM_BARS);
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + NUM_BARS_PER_STAGE * STAGES + NUM_BARS_FIXED);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
   auto bar_tma_full = [&](int s) { return smem_u32(bars + s); };
   auto bar_b_full = [&](int s) { return smem_u32(bars + STAGES + s); };
@@ -217,7 +221,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           tc_fence_after();
           const uint64_t adesc = umma_desc_k_sw128(sbase + off_a(s));
-          const uint64_t bdesc = umma_desc_k_sw128(sbase + off_b(s));
+          const uint64_t bdesc = umma_desc_k_sw128(sbase + off_b(FMT, BITS, s));
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)  // advance 16 bf16 = 32 bytes = 2 descriptor units
             umma_f16(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) != 0);
@@ -319,7 +323,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int s = (int)(it % STAGES);
       if (!mbar_wait_bounded(bar_tma_full(s), (uint32_t)((it / STAGES) & 1), abort_flag)) break;
       const uint8_t *P = smem + off_p(FMT, BITS, s);
-      uint8_t *B = smem + off_b(s);
+      uint8_t *B = smem + off_b(FMT, BITS, s);
 #pragma unroll
       for (int rr = 0; rr < 2; ++rr) {
         const int r = rr ? r1 : r0;
