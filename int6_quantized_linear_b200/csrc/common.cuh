@@ -97,6 +97,20 @@ QL_DEVI void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t b
                : "memory");
 }
 
+// 4-byte asynchronous copy global -> shared; with valid == false the 4 bytes are zero-filled and
+// src is not read.
+QL_DEVI void cp_async4(uint32_t dst, const void *src, bool valid) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(reinterpret_cast<uint64_t>(src)),
+               "r"(valid ? 4 : 0)
+               : "memory");
+}
+// The mbarrier receives one arrival once every cp.async this thread issued before has landed
+// (counted in the barrier's expected arrivals).
+QL_DEVI void cp_async_arrive_noinc(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+QL_DEVI void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 QL_DEVI void tma_prefetch_desc(const CUtensorMap *map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

@@ -34,6 +34,10 @@ constexpr int BK = 64;
 constexpr int NUM_DEQ_WARPS = 8;
 constexpr int WARP_TMA = 0;
 constexpr int WARP_MMA = 1;
+constexpr int WARP_META0 = 2;    // int4: two warps copy each stage's group and step words ahead
+constexpr int NUM_META_WARPS = 2;
+constexpr int MSTAGES = 8;       // metadata ring depth (int4)
+constexpr int META_STAGE_BYTES = BN * 8;  // per tile row: the stage's two group words (u32), its step word
 constexpr int WARP_EPI0 = 4;
 constexpr int WARP_DEQ0 = 8;
 constexpr int NUM_THREADS = (WARP_DEQ0 + NUM_DEQ_WARPS) * 32;
@@ -47,12 +51,16 @@ __host__ __device__ constexpr int code_bits(int fmt, int bits) {
 __host__ __device__ constexpr int p_row_bytes(int fmt, int bits) { return BK * code_bits(fmt, bits) / 8; }
 __host__ __device__ constexpr int p_bytes(int fmt, int bits) { return BN * p_row_bytes(fmt, bits); }
 
-// Stages of the ring: four when they fit in the 227 KB a CTA may use, else three.
+// Stages of the ring: four when they fit in the 227 KB a CTA may use, else three.  int4 adds the
+// metadata ring [MSTAGES][BN rows][8 bytes] and its barriers.
 constexpr int NUM_BARS_PER_STAGE = 3;  // tma_full, b_full, empty
 constexpr int NUM_BARS_FIXED = 5;      // acc_full[2], acc_empty[2], final
 __host__ __device__ constexpr int stage_bytes(int fmt, int bits) { return A_BYTES + B_BYTES + p_bytes(fmt, bits); }
+__host__ __device__ constexpr int meta_bytes(int fmt) { return fmt == FMT_INT4 ? MSTAGES * META_STAGE_BYTES : 0; }
+__host__ __device__ constexpr int meta_bars(int fmt) { return fmt == FMT_INT4 ? 2 * MSTAGES : 0; }
 __host__ __device__ constexpr int smem_need(int fmt, int bits, int st) {
-  return st * stage_bytes(fmt, bits) + (NUM_BARS_PER_STAGE * st + NUM_BARS_FIXED) * 8 + 16 + 1024;
+  return st * stage_bytes(fmt, bits) + meta_bytes(fmt) +
+         (NUM_BARS_PER_STAGE * st + NUM_BARS_FIXED + meta_bars(fmt)) * 8 + 16 + 1024;
 }
 __host__ __device__ constexpr int stages(int fmt, int bits) { return smem_need(fmt, bits, 4) <= 232448 ? 4 : 3; }
 
@@ -62,8 +70,14 @@ __host__ __device__ constexpr int off_b(int fmt, int bits, int s) { return stage
 __host__ __device__ constexpr int off_p(int fmt, int bits, int s) {
   return stages(fmt, bits) * (A_BYTES + B_BYTES) + s * p_bytes(fmt, bits);
 }
-__host__ __device__ constexpr int off_bar(int fmt, int bits) { return stages(fmt, bits) * stage_bytes(fmt, bits); }
-// barriers: tma_full[S], b_full[S], empty[S], acc_full[2], acc_empty[2], final (+ tmem base, abort flag)
+__host__ __device__ constexpr int off_meta(int fmt, int bits, int s) {
+  return stages(fmt, bits) * stage_bytes(fmt, bits) + s * META_STAGE_BYTES;
+}
+__host__ __device__ constexpr int off_bar(int fmt, int bits) {
+  return stages(fmt, bits) * stage_bytes(fmt, bits) + meta_bytes(fmt);
+}
+// barriers: tma_full[S], b_full[S], empty[S], acc_full[2], acc_empty[2], final, (int4) meta_full[MS],
+// meta_empty[MS]; then the tmem base and the abort flag
 __host__ __device__ constexpr int smem_bytes(int fmt, int bits) { return smem_need(fmt, bits, stages(fmt, bits)); }
 
 struct Params {
@@ -136,7 +150,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + off_bar(FMT, BITS));
-  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + NUM_BARS_PER_STAGE * STAGES + NUM_BARS_FIXED);
+  uint32_t *tmem_holder =
+      reinterpret_cast<uint32_t *>(bars + NUM_BARS_PER_STAGE * STAGES + NUM_BARS_FIXED + meta_bars(FMT));
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
   auto bar_tma_full = [&](int s) { return smem_u32(bars + s); };
   auto bar_b_full = [&](int s) { return smem_u32(bars + STAGES + s); };
@@ -144,6 +159,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   auto bar_acc_full = [&](int a) { return smem_u32(bars + 3 * STAGES + a); };
   auto bar_acc_empty = [&](int a) { return smem_u32(bars + 3 * STAGES + 2 + a); };
   const uint32_t bar_final = smem_u32(bars + 3 * STAGES + 4);
+  auto bar_meta_full = [&](int s) { return smem_u32(bars + 3 * STAGES + 5 + s); };
+  auto bar_meta_empty = [&](int s) { return smem_u32(bars + 3 * STAGES + 5 + MSTAGES + s); };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t m_tiles = (p.M + BM - 1) / BM, n_tiles = (p.N + BN - 1) / BN;
@@ -161,6 +178,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(bar_acc_empty(a), 4);
     }
     mbar_init(bar_final, 1);
+    if constexpr (FMT == FMT_INT4) {
+      for (int s = 0; s < MSTAGES; ++s) {
+        mbar_init(bar_meta_full(s), NUM_META_WARPS * 32);  // one cp.async arrival per copying thread
+        mbar_init(bar_meta_empty(s), NUM_DEQ_WARPS);
+      }
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -238,6 +261,34 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
     }
+  } else if (FMT == FMT_INT4 && warp >= WARP_META0 && warp < WARP_META0 + NUM_META_WARPS) {
+    // metadata copier: for every stage, each tile row's group words (u32 holding the stage's two
+    // 32-weight groups) and its super-block step word, up to MSTAGES stages ahead of the dequantisers
+    const int t = threadIdx.x - WARP_META0 * 32;  // 0..63: rows t, t+64, t+128, t+192
+    const int64_t my_tiles = (num_tiles - blockIdx.x + gridDim.x - 1) / gridDim.x;
+    const int64_t total_it = my_tiles * num_kb;
+    bool ok = true;
+    for (int64_t it = 0; it < total_it && ok; ++it) {
+      const int ms = (int)(it % MSTAGES);
+      if (!mbar_wait_bounded(bar_meta_empty(ms), (uint32_t)(((it / MSTAGES) & 1) ^ 1), abort_flag)) {
+        ok = false;
+        break;
+      }
+      const int64_t n_tile = ((int64_t)blockIdx.x + (it / num_kb) * gridDim.x) / m_tiles;
+      const int kb = (int)(it % num_kb);
+      const uint32_t dst = sbase + off_meta(FMT, BITS, ms);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = t + 64 * i;
+        const int64_t n = n_tile * BN + r;
+        const bool valid = n < p.N;
+        const int64_t nn = valid ? n : p.N - 1;
+        cp_async4(dst + r * 8, p.gmeta + nn * (p.K / 16) + 4 * kb, valid);
+        cp_async4(dst + r * 8 + 4, p.steps + 4 * (nn * (p.K / 256) + kb / 4), valid);
+      }
+      cp_async_arrive_noinc(bar_meta_full(ms));
+    }
+    cp_async_wait_all();  // no copy may land after the CTA is gone
   } else if (warp >= WARP_EPI0 && warp < WARP_EPI0 + 4) {
     const int e = warp - WARP_EPI0;  // TMEM lane quarter
     int64_t tcount = 0;
@@ -302,8 +353,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     float sc0 = 0.f, sc1 = 0.f;
     if (total_it > 0) {
       const int64_t n_tile = tile_of(0) / m_tiles;
-      load_meta<FMT>(p, n_tile * BN + r0, h, gm0, st0);
-      load_meta<FMT>(p, n_tile * BN + r1, h, gm1, st1);
+      if constexpr (FMT != FMT_INT4) {
+        load_meta<FMT>(p, n_tile * BN + r0, h, gm0, st0);
+        load_meta<FMT>(p, n_tile * BN + r1, h, gm1, st1);
+      }
       sc0 = row_scale(n_tile * BN + r0);
       sc1 = row_scale(n_tile * BN + r1);
     }
@@ -313,14 +366,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (it + 1 < total_it) {  // prefetch the next stage's metadata
         const int64_t n_tile = tile_of(it + 1) / m_tiles;
         const int64_t c = (int64_t)((it + 1) % num_kb) * (BK / 32) + h;
-        load_meta<FMT>(p, n_tile * BN + r0, c, ngm0, nst0);
-        load_meta<FMT>(p, n_tile * BN + r1, c, ngm1, nst1);
+        if constexpr (FMT != FMT_INT4) {
+          load_meta<FMT>(p, n_tile * BN + r0, c, ngm0, nst0);
+          load_meta<FMT>(p, n_tile * BN + r1, c, ngm1, nst1);
+        }
         if ((it + 1) % num_kb == 0) {
           nsc0 = row_scale(n_tile * BN + r0);
           nsc1 = row_scale(n_tile * BN + r1);
         }
       }
       const int s = (int)(it % STAGES);
+      if constexpr (FMT == FMT_INT4) {  // this stage's group and step words, from the metadata ring
+        const int ms = (int)(it % MSTAGES);
+        if (!mbar_wait_bounded(bar_meta_full(ms), (uint32_t)((it / MSTAGES) & 1), abort_flag)) break;
+        const uint8_t *mrow = smem + off_meta(FMT, BITS, ms);
+        const uint2 m0 = *reinterpret_cast<const uint2 *>(mrow + r0 * 8);
+        const uint2 m1 = *reinterpret_cast<const uint2 *>(mrow + r1 * 8);
+        gm0 = (m0.x >> (16 * h)) & 0xffffu;
+        st0 = m0.y;
+        gm1 = (m1.x >> (16 * h)) & 0xffffu;
+        st1 = m1.y;
+        __syncwarp();
+        if ((t & 31) == 0) mbar_arrive(bar_meta_empty(ms));
+      }
       if (!mbar_wait_bounded(bar_tma_full(s), (uint32_t)((it / STAGES) & 1), abort_flag)) break;
       const uint8_t *P = smem + off_p(FMT, BITS, s);
       uint8_t *B = smem + off_b(FMT, BITS, s);
