@@ -2,23 +2,29 @@
 //
 //   y[M][N] = x[M][K] . W^T,  x bf16, W quantized, y bf16, fp32 accumulation
 //
-// Persistent kernel, one CTA per SM, tiles of BM=128 tokens x BN=256 weight
+// Persistent kernel, one CTA per SM, tiles of BM=256 tokens x BN=128 weight
 // rows, K streamed in BK=64 steps through a 3- or 4-deep shared-memory ring.
+// Each k-step is two MMAs of M=128 (the two token halves) against the same
+// dequantised weight tile, so every weight is dequantised once per 256 tokens.
 // Warp roles:
-//   warp 0      TMA producer: scaled fp16 x tile (128 x 64, 128-byte
-//               swizzle) and the packed code tile (256 rows x BK codes)
-//   warp 1      TMEM allocator; lane 0 issues tcgen05.mma (M=128, N=256,
-//               K=16, f16 x f16 -> f32) into one of two TMEM accumulators
-//   warps 4-7   epilogue: tcgen05.ld the accumulator (warp w reads TMEM lanes
-//               32*(w%4)..), undo the two power-of-two scales, round to bf16,
-//               store y
-//   warps 8-15  dequantisers: packed codes (shared) + metadata (global, one
-//               stage ahead) -> exact binary32 weight -> times 2^b_n (exact)
-//               -> nearest-even fp16, written in the canonical K-major
-//               128-byte-swizzled layout the MMA reads as its B operand
+//   warp 0      TMA producer: scaled fp16 x tile (256 x 64, 128-byte
+//               swizzle) and the packed code tile (128 rows x BK codes)
+//   warp 1      TMEM allocator; lane 0 issues tcgen05.mma (M=128, N=128,
+//               K=16, f16 x f16 -> f32), two per 16-k slice, into one of two
+//               TMEM accumulator pairs
+//   warps 2-3   (int4) copy each stage's group and step words into a
+//               metadata ring, MSTAGES ahead
+//   warps 4-7   epilogue: tcgen05.ld the accumulators (warp w reads TMEM
+//               lanes 32*(w%4).. of both halves), undo the two power-of-two
+//               scales, round to bf16, store y
+//   warps 8-15  dequantisers, one tile row and 32 weights each per stage:
+//               packed codes + metadata -> weight times 2^b_n -> fp16, written
+//               in the canonical K-major 128-byte-swizzled layout the MMA reads
+//               as its B operand
 // The operands are fp16 rather than bf16 because rounding every weight to
 // bf16 costs ~1% of rms(y); fp16 costs ~0.1% (see gemm_prep.cuh for the
-// scaling that keeps fp32 range).
+// scaling that keeps fp32 range).  Loop state advances by counters: no
+// division runs per stage.
 // Every mbarrier wait is bounded; a wait that gives up sets the device status
 // word and makes every role leave its loop.
 #pragma once
@@ -28,22 +34,23 @@
 namespace ql {
 namespace gemm {
 
-constexpr int BM = 128;
-constexpr int BN = 256;
+constexpr int BM = 256;  // tokens per tile: two MMA halves of 128
+constexpr int BN = 128;  // weight rows per tile
 constexpr int BK = 64;
 constexpr int NUM_DEQ_WARPS = 8;
 constexpr int WARP_TMA = 0;
 constexpr int WARP_MMA = 1;
 constexpr int WARP_META0 = 2;    // int4: two warps copy each stage's group and step words ahead
 constexpr int NUM_META_WARPS = 2;
-constexpr int MSTAGES = 8;       // metadata ring depth (int4)
-constexpr int META_STAGE_BYTES = BN * 8;  // per tile row: the stage's two group words (u32), its step word
 constexpr int WARP_EPI0 = 4;
 constexpr int WARP_DEQ0 = 8;
 constexpr int NUM_THREADS = (WARP_DEQ0 + NUM_DEQ_WARPS) * 32;
-constexpr int A_BYTES = BM * BK * 2;  // 16 KB
-constexpr int B_BYTES = BN * BK * 2;  // 32 KB
-constexpr uint32_t TMEM_COLS = 2 * BN;  // two fp32 accumulators of 256 columns
+constexpr int A_BYTES = BM * BK * 2;  // 32 KB
+constexpr int B_BYTES = BN * BK * 2;  // 16 KB
+constexpr uint32_t TMEM_COLS = 512;   // two accumulator pairs of 2 x 128 fp32 columns
+constexpr int MSTAGES = 8;            // metadata ring depth (int4)
+constexpr int META_STAGE_BYTES = BN * 8;  // per tile row: the stage's two group words (u32), its step word
+constexpr int SMEM_LIMIT = 232448;        // dynamic shared memory a CTA may use
 
 __host__ __device__ constexpr int code_bits(int fmt, int bits) {
   return fmt == FMT_INT4 ? 4 : (fmt == FMT_INT6 ? 6 : bits);
@@ -51,8 +58,8 @@ __host__ __device__ constexpr int code_bits(int fmt, int bits) {
 __host__ __device__ constexpr int p_row_bytes(int fmt, int bits) { return BK * code_bits(fmt, bits) / 8; }
 __host__ __device__ constexpr int p_bytes(int fmt, int bits) { return BN * p_row_bytes(fmt, bits); }
 
-// Stages of the ring: four when they fit in the 227 KB a CTA may use, else three.  int4 adds the
-// metadata ring [MSTAGES][BN rows][8 bytes] and its barriers.
+// Stages of the ring: four when they fit, else three.  int4 adds the metadata ring
+// [MSTAGES][BN rows][8 bytes] and its barriers.
 constexpr int NUM_BARS_PER_STAGE = 3;  // tma_full, b_full, empty
 constexpr int NUM_BARS_FIXED = 5;      // acc_full[2], acc_empty[2], final
 __host__ __device__ constexpr int stage_bytes(int fmt, int bits) { return A_BYTES + B_BYTES + p_bytes(fmt, bits); }
@@ -62,7 +69,7 @@ __host__ __device__ constexpr int smem_need(int fmt, int bits, int st) {
   return st * stage_bytes(fmt, bits) + meta_bytes(fmt) +
          (NUM_BARS_PER_STAGE * st + NUM_BARS_FIXED + meta_bars(fmt)) * 8 + 16 + 1024;
 }
-__host__ __device__ constexpr int stages(int fmt, int bits) { return smem_need(fmt, bits, 4) <= 232448 ? 4 : 3; }
+__host__ __device__ constexpr int stages(int fmt, int bits) { return smem_need(fmt, bits, 4) <= SMEM_LIMIT ? 4 : 3; }
 
 // byte offsets inside the dynamic shared memory (base aligned to 1024)
 __host__ __device__ constexpr int off_a(int s) { return s * A_BYTES; }
@@ -166,6 +173,37 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int64_t m_tiles = (p.M + BM - 1) / BM, n_tiles = (p.N + BN - 1) / BN;
   const int64_t num_tiles = m_tiles * n_tiles;
   const int num_kb = (int)(p.K / BK);
+  const int64_t my_tiles = (num_tiles - blockIdx.x + gridDim.x - 1) / gridDim.x;
+  const int64_t total_it = my_tiles * num_kb;  // k-stages this CTA runs, in order
+
+  // (k-step, tile) of a stage, advanced one stage at a time
+  struct Cursor {
+    int kb;
+    int64_t tile, n_tile, m_tile;
+  };
+  auto cursor0 = [&]() {
+    Cursor c;
+    c.kb = 0;
+    c.tile = blockIdx.x;
+    c.n_tile = c.tile / m_tiles;
+    c.m_tile = c.tile - c.n_tile * m_tiles;
+    return c;
+  };
+  auto advance = [&](Cursor &c) {
+    if (++c.kb == num_kb) {
+      c.kb = 0;
+      c.tile += gridDim.x;
+      c.n_tile = c.tile / m_tiles;
+      c.m_tile = c.tile - c.n_tile * m_tiles;
+    }
+  };
+  // slot and phase of a ring position, advanced one use at a time
+  auto step_ring = [](int &slot, uint32_t &phase, int depth) {
+    if (++slot == depth) {
+      slot = 0;
+      phase ^= 1u;
+    }
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -201,18 +239,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tma_prefetch_desc(&map_x);
       tma_prefetch_desc(&map_codes);
       int64_t it = 0;
+      int s = 0;
+      uint32_t ph = 0;
+      Cursor cur = cursor0();
       bool ok = true;
-      for (int64_t tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        const int64_t n_tile = tile / m_tiles, m_tile = tile - n_tile * m_tiles;
-        for (int kb = 0; kb < num_kb; ++kb, ++it) {
-          const int s = (int)(it % STAGES);
-          const uint32_t use = (uint32_t)(it / STAGES);
-          if (!mbar_wait_bounded(bar_empty(s), (use & 1) ^ 1, abort_flag)) { ok = false; break; }
-          mbar_arrive_expect_tx(bar_tma_full(s), STAGE_TX);
-          tma_load_2d(sbase + off_a(s), &map_x, bar_tma_full(s), kb * BK, (int32_t)(m_tile * BM));
-          tma_load_2d(sbase + off_p(FMT, BITS, s), &map_codes, bar_tma_full(s), kb * PROW,
-                      (int32_t)(n_tile * BN));
+      for (; it < total_it; ++it) {
+        if (!mbar_wait_bounded(bar_empty(s), ph ^ 1u, abort_flag)) {
+          ok = false;
+          break;
         }
+        mbar_arrive_expect_tx(bar_tma_full(s), STAGE_TX);
+        tma_load_2d(sbase + off_a(s), &map_x, bar_tma_full(s), cur.kb * BK, (int32_t)(cur.m_tile * BM));
+        tma_load_2d(sbase + off_p(FMT, BITS, s), &map_codes, bar_tma_full(s), cur.kb * PROW,
+                    (int32_t)(cur.n_tile * BN));
+        step_ring(s, ph, STAGES);
+        advance(cur);
       }
       if (!ok) {  // let copies already issued land before the CTA can exit
         for (int64_t j = it - 1; j >= 0 && j >= it - STAGES; --j) {
@@ -225,31 +266,34 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else if (warp == WARP_MMA) {
     if (lane == 0) {
-      constexpr uint32_t idesc = umma_idesc_f16_f32(BM, BN);
-      int64_t it = 0, tcount = 0;
+      constexpr uint32_t idesc = umma_idesc_f16_f32(128, BN);
+      int64_t tcount = 0;
+      int s = 0;
+      uint32_t ph = 0;
       bool ok = true, issued = false;
       for (int64_t tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++tcount) {
         const int a = (int)(tcount & 1);
         const uint32_t ause = (uint32_t)(tcount >> 1);
         if (!mbar_wait_bounded(bar_acc_empty(a), (ause & 1) ^ 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + (uint32_t)(a * BN);
-        for (int kb = 0; kb < num_kb; ++kb, ++it) {
-          const int s = (int)(it % STAGES);
-          const uint32_t par = (uint32_t)((it / STAGES) & 1);
-          if (!mbar_wait_bounded(bar_tma_full(s), par, abort_flag) ||
-              !mbar_wait_bounded(bar_b_full(s), par, abort_flag)) {
+        const uint32_t d_tmem = tmem_base + (uint32_t)(a * 2 * BN);  // half hm at + hm * BN columns
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait_bounded(bar_tma_full(s), ph, abort_flag) || !mbar_wait_bounded(bar_b_full(s), ph, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint64_t adesc = umma_desc_k_sw128(sbase + off_a(s));
           const uint64_t bdesc = umma_desc_k_sw128(sbase + off_b(FMT, BITS, s));
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk)  // advance 16 bf16 = 32 bytes = 2 descriptor units
-            umma_f16(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) != 0);
+          for (int hm = 0; hm < 2; ++hm) {  // token half: rows 128*hm.. of the x tile (16 KB in)
+            const uint64_t adesc = umma_desc_k_sw128(sbase + off_a(s) + hm * (A_BYTES / 2));
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk)  // advance 16 fp16 = 32 bytes = 2 descriptor units
+              umma_f16(d_tmem + (uint32_t)(hm * BN), adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) != 0);
+          }
           umma_commit(bar_empty(s));
           issued = true;
+          step_ring(s, ph, STAGES);
         }
         if (!ok) break;
         umma_commit(bar_acc_full(a));
@@ -261,34 +305,32 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
     }
-  } else if (FMT == FMT_INT4 && warp >= WARP_META0 && warp < WARP_META0 + NUM_META_WARPS) {
-    // metadata copier: for every stage, each tile row's group words (u32 holding the stage's two
-    // 32-weight groups) and its super-block step word, up to MSTAGES stages ahead of the dequantisers
-    const int t = threadIdx.x - WARP_META0 * 32;  // 0..63: rows t, t+64, t+128, t+192
-    const int64_t my_tiles = (num_tiles - blockIdx.x + gridDim.x - 1) / gridDim.x;
-    const int64_t total_it = my_tiles * num_kb;
-    bool ok = true;
-    for (int64_t it = 0; it < total_it && ok; ++it) {
-      const int ms = (int)(it % MSTAGES);
-      if (!mbar_wait_bounded(bar_meta_empty(ms), (uint32_t)(((it / MSTAGES) & 1) ^ 1), abort_flag)) {
-        ok = false;
-        break;
-      }
-      const int64_t n_tile = ((int64_t)blockIdx.x + (it / num_kb) * gridDim.x) / m_tiles;
-      const int kb = (int)(it % num_kb);
-      const uint32_t dst = sbase + off_meta(FMT, BITS, ms);
+  } else if (warp >= WARP_META0 && warp < WARP_META0 + NUM_META_WARPS) {
+    if constexpr (FMT == FMT_INT4) {
+      // for every stage, each tile row's group words (u32 holding the stage's two 32-weight groups)
+      // and its super-block step word, up to MSTAGES stages ahead of the dequantisers
+      const int t = threadIdx.x - WARP_META0 * 32;  // 0..63: rows t and t + 64
+      int ms = 0;
+      uint32_t phm = 0;
+      Cursor cur = cursor0();
+      for (int64_t it = 0; it < total_it; ++it) {
+        if (!mbar_wait_bounded(bar_meta_empty(ms), phm ^ 1u, abort_flag)) break;
+        const uint32_t dst = sbase + off_meta(FMT, BITS, ms);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int r = t + 64 * i;
-        const int64_t n = n_tile * BN + r;
-        const bool valid = n < p.N;
-        const int64_t nn = valid ? n : p.N - 1;
-        cp_async4(dst + r * 8, p.gmeta + nn * (p.K / 16) + 4 * kb, valid);
-        cp_async4(dst + r * 8 + 4, p.steps + 4 * (nn * (p.K / 256) + kb / 4), valid);
+        for (int i = 0; i < BN / 64; ++i) {
+          const int r = t + 64 * i;
+          const int64_t n = cur.n_tile * BN + r;
+          const bool valid = n < p.N;
+          const int64_t nn = valid ? n : p.N - 1;
+          cp_async4(dst + r * 8, p.gmeta + nn * (p.K / 16) + 4 * cur.kb, valid);
+          cp_async4(dst + r * 8 + 4, p.steps + 4 * (nn * (p.K / 256) + cur.kb / 4), valid);
+        }
+        cp_async_arrive_noinc(bar_meta_full(ms));
+        step_ring(ms, phm, MSTAGES);
+        advance(cur);
       }
-      cp_async_arrive_noinc(bar_meta_full(ms));
+      cp_async_wait_all();  // no copy may land after the CTA is gone
     }
-    cp_async_wait_all();  // no copy may land after the CTA is gone
   } else if (warp >= WARP_EPI0 && warp < WARP_EPI0 + 4) {
     const int e = warp - WARP_EPI0;  // TMEM lane quarter
     int64_t tcount = 0;
@@ -299,40 +341,44 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint32_t ause = (uint32_t)(tcount >> 1);
       if (!mbar_wait_bounded(bar_acc_full(a), ause & 1, abort_flag)) break;
       tc_fence_after();
-      const int64_t m = m_tile * BM + 32 * e + lane;
-      const float xs = m < p.M ? p.ws.xinv[m] : 0.f;
 #pragma unroll 1
-      for (int cchunk = 0; cchunk < BN / 32; ++cchunk) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(32 * e) << 16) + (uint32_t)(a * BN + 32 * cchunk), r);
-        tmem_ld_wait();
-        const int64_t n0 = n_tile * BN + 32 * cchunk;
-        {  // y = D * 2^-a_m * 2^-b_n, both exact power-of-two multiplications
-          const float4 *wi = reinterpret_cast<const float4 *>(p.ws.winv + n0);
+      for (int hm = 0; hm < 2; ++hm) {
+        const int64_t m = m_tile * BM + 128 * hm + 32 * e + lane;
+        const float xs = m < p.M ? p.ws.xinv[m] : 0.f;
+#pragma unroll 1
+        for (int cchunk = 0; cchunk < BN / 32; ++cchunk) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(32 * e) << 16) + (uint32_t)(a * 2 * BN + hm * BN + 32 * cchunk),
+                             r);
+          tmem_ld_wait();
+          const int64_t n0 = n_tile * BN + 32 * cchunk;
+          {  // y = D * 2^-a_m * 2^-b_n, both exact power-of-two multiplications
+            const float4 *wi = reinterpret_cast<const float4 *>(p.ws.winv + n0);
 #pragma unroll
-          for (int t = 0; t < 8; ++t) {
-            const float4 v = wi[t];
-            r[4 * t + 0] = __float_as_uint(__uint_as_float(r[4 * t + 0]) * xs * v.x);
-            r[4 * t + 1] = __float_as_uint(__uint_as_float(r[4 * t + 1]) * xs * v.y);
-            r[4 * t + 2] = __float_as_uint(__uint_as_float(r[4 * t + 2]) * xs * v.z);
-            r[4 * t + 3] = __float_as_uint(__uint_as_float(r[4 * t + 3]) * xs * v.w);
-          }
-        }
-        if (m < p.M) {
-          __nv_bfloat16 *dst = p.y + m * p.N + n0;
-          if (vec_ok && n0 + 32 <= p.N) {
-#pragma unroll
-            for (int t = 0; t < 4; ++t) {
-              uint4 v;
-              v.x = pack_bf16x2(__uint_as_float(r[8 * t + 0]), __uint_as_float(r[8 * t + 1]));
-              v.y = pack_bf16x2(__uint_as_float(r[8 * t + 2]), __uint_as_float(r[8 * t + 3]));
-              v.z = pack_bf16x2(__uint_as_float(r[8 * t + 4]), __uint_as_float(r[8 * t + 5]));
-              v.w = pack_bf16x2(__uint_as_float(r[8 * t + 6]), __uint_as_float(r[8 * t + 7]));
-              reinterpret_cast<uint4 *>(dst)[t] = v;
+            for (int t = 0; t < 8; ++t) {
+              const float4 v = wi[t];
+              r[4 * t + 0] = __float_as_uint(__uint_as_float(r[4 * t + 0]) * xs * v.x);
+              r[4 * t + 1] = __float_as_uint(__uint_as_float(r[4 * t + 1]) * xs * v.y);
+              r[4 * t + 2] = __float_as_uint(__uint_as_float(r[4 * t + 2]) * xs * v.z);
+              r[4 * t + 3] = __float_as_uint(__uint_as_float(r[4 * t + 3]) * xs * v.w);
             }
-          } else {
-            for (int i = 0; i < 32; ++i)
-              if (n0 + i < p.N) dst[i] = __float2bfloat16_rn(__uint_as_float(r[i]));
+          }
+          if (m < p.M) {
+            __nv_bfloat16 *dst = p.y + m * p.N + n0;
+            if (vec_ok && n0 + 32 <= p.N) {
+#pragma unroll
+              for (int t = 0; t < 4; ++t) {
+                uint4 v;
+                v.x = pack_bf16x2(__uint_as_float(r[8 * t + 0]), __uint_as_float(r[8 * t + 1]));
+                v.y = pack_bf16x2(__uint_as_float(r[8 * t + 2]), __uint_as_float(r[8 * t + 3]));
+                v.z = pack_bf16x2(__uint_as_float(r[8 * t + 4]), __uint_as_float(r[8 * t + 5]));
+                v.w = pack_bf16x2(__uint_as_float(r[8 * t + 6]), __uint_as_float(r[8 * t + 7]));
+                reinterpret_cast<uint4 *>(dst)[t] = v;
+              }
+            } else {
+              for (int i = 0; i < 32; ++i)
+                if (n0 + i < p.N) dst[i] = __float2bfloat16_rn(__uint_as_float(r[i]));
+            }
           }
         }
       }
@@ -343,109 +389,93 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else if (warp >= WARP_DEQ0) {
     const int t = threadIdx.x - WARP_DEQ0 * 32;  // 0..255
     const int h = t & 1;                          // which 32-weight half of the 64-k stage
-    const int r0 = t >> 1, r1 = r0 + 128;         // the two tile rows this thread fills
-    int64_t it = 0;
-    const int64_t my_tiles = (num_tiles - blockIdx.x + gridDim.x - 1) / gridDim.x;
-    const int64_t total_it = my_tiles * num_kb;
-    auto tile_of = [&](int64_t i) { return (int64_t)blockIdx.x + (i / num_kb) * gridDim.x; };
+    const int r = t >> 1;                         // the tile row this thread fills
     auto row_scale = [&](int64_t n) { return n < p.N ? p.ws.wsc[n] : 0.f; };
-    uint32_t gm0 = 0, st0 = 0, gm1 = 0, st1 = 0;
-    float sc0 = 0.f, sc1 = 0.f;
+    Cursor nxt = cursor0();  // the stage after the current one
+    advance(nxt);
+    int s = 0, ms = 0;
+    uint32_t ph = 0, phm = 0;
+    uint32_t gm = 0, st = 0;
+    float sc = 0.f;
     if (total_it > 0) {
-      const int64_t n_tile = tile_of(0) / m_tiles;
-      if constexpr (FMT != FMT_INT4) {
-        load_meta<FMT>(p, n_tile * BN + r0, h, gm0, st0);
-        load_meta<FMT>(p, n_tile * BN + r1, h, gm1, st1);
-      }
-      sc0 = row_scale(n_tile * BN + r0);
-      sc1 = row_scale(n_tile * BN + r1);
+      const int64_t n_tile = cursor0().n_tile;
+      if constexpr (FMT != FMT_INT4) load_meta<FMT>(p, n_tile * BN + r, h, gm, st);
+      sc = row_scale(n_tile * BN + r);
     }
-    for (; it < total_it; ++it) {
-      uint32_t ngm0 = 0, nst0 = 0, ngm1 = 0, nst1 = 0;
-      float nsc0 = sc0, nsc1 = sc1;
-      if (it + 1 < total_it) {  // prefetch the next stage's metadata
-        const int64_t n_tile = tile_of(it + 1) / m_tiles;
-        const int64_t c = (int64_t)((it + 1) % num_kb) * (BK / 32) + h;
-        if constexpr (FMT != FMT_INT4) {
-          load_meta<FMT>(p, n_tile * BN + r0, c, ngm0, nst0);
-          load_meta<FMT>(p, n_tile * BN + r1, c, ngm1, nst1);
-        }
-        if ((it + 1) % num_kb == 0) {
-          nsc0 = row_scale(n_tile * BN + r0);
-          nsc1 = row_scale(n_tile * BN + r1);
-        }
+    uint8_t *row = smem + (r >> 3) * 1024 + (r & 7) * 128;  // + off_b(stage)
+    for (int64_t it = 0; it < total_it; ++it) {
+      uint32_t ngm = 0, nst = 0;
+      float nsc = sc;
+      if (it + 1 < total_it) {  // the next stage's metadata (int6, affine) and row scale
+        const int64_t n = nxt.n_tile * BN + r;
+        if constexpr (FMT != FMT_INT4) load_meta<FMT>(p, n, (int64_t)nxt.kb * (BK / 32) + h, ngm, nst);
+        if (nxt.kb == 0) nsc = row_scale(n);
       }
-      const int s = (int)(it % STAGES);
+      advance(nxt);
       if constexpr (FMT == FMT_INT4) {  // this stage's group and step words, from the metadata ring
-        const int ms = (int)(it % MSTAGES);
-        if (!mbar_wait_bounded(bar_meta_full(ms), (uint32_t)((it / MSTAGES) & 1), abort_flag)) break;
-        const uint8_t *mrow = smem + off_meta(FMT, BITS, ms);
-        const uint2 m0 = *reinterpret_cast<const uint2 *>(mrow + r0 * 8);
-        const uint2 m1 = *reinterpret_cast<const uint2 *>(mrow + r1 * 8);
-        gm0 = (m0.x >> (16 * h)) & 0xffffu;
-        st0 = m0.y;
-        gm1 = (m1.x >> (16 * h)) & 0xffffu;
-        st1 = m1.y;
+        if (!mbar_wait_bounded(bar_meta_full(ms), phm, abort_flag)) break;
+        const uint2 mv = *reinterpret_cast<const uint2 *>(smem + off_meta(FMT, BITS, ms) + r * 8);
+        gm = (mv.x >> (16 * h)) & 0xffffu;
+        st = mv.y;
         __syncwarp();
         if ((t & 31) == 0) mbar_arrive(bar_meta_empty(ms));
+        step_ring(ms, phm, MSTAGES);
       }
-      if (!mbar_wait_bounded(bar_tma_full(s), (uint32_t)((it / STAGES) & 1), abort_flag)) break;
-      const uint8_t *P = smem + off_p(FMT, BITS, s);
-      uint8_t *B = smem + off_b(FMT, BITS, s);
+      if (!mbar_wait_bounded(bar_tma_full(s), ph, abort_flag)) break;
+      const uint8_t *src = smem + off_p(FMT, BITS, s) + r * PROW + h * (PROW / 2);
+      uint8_t *dst_row = row + off_b(FMT, BITS, s);
+      // each 16-byte chunk holds k = 0,4,1,5,2,6,3,7 of its 8 weights (the order of the x tile)
+      if constexpr (FMT == FMT_INT4) {
+        // packed-half arithmetic: q as 1024+q / 64+q from one bit operation, then
+        // w * 2^b_n = q * S' - Z * S' in fp16 with S' = S * 2^b_n; the codes sc, zc become floats
+        // by placing the byte in the mantissa of 2^23 and subtracting 2^23 (exact)
+        const float scf = __uint_as_float(0x4B000000u | (gm & 0xffu)) - 8388608.f;
+        const float zcf = __uint_as_float(0x4B000000u | ((gm >> 8) & 0xffu)) - 8388608.f;
+        const float S = __fmul_rn(scf, f16_bits_to_f32(st)) * sc;
+        const float ZS = __fmul_rn(zcf, f16_bits_to_f32(st >> 16)) * S;
+        const __half2 s2 = __float2half2_rn(S), nz2 = __float2half2_rn(-ZS);
+        const __half2 m1024 = __float2half2_rn(1024.f), m64 = __float2half2_rn(64.f);
+        const uint4 cv = *reinterpret_cast<const uint4 *>(src);
+        const uint32_t cw[4] = {cv.x, cv.y, cv.z, cv.w};
 #pragma unroll
-      for (int rr = 0; rr < 2; ++rr) {
-        const int r = rr ? r1 : r0;
-        const float sc = rr ? sc1 : sc0;
-        uint8_t *row = B + (r >> 3) * 1024 + (r & 7) * 128;
-        // each 16-byte chunk holds k = 0,4,1,5,2,6,3,7 of its 8 weights (the order of the x tile)
-        if constexpr (FMT == FMT_INT4) {
-          // packed-half arithmetic: q as 1024+q / 64+q from one bit operation, then
-          // w * 2^b_n = q * S' - Z * S' in fp16 with S' = S * 2^b_n
-          const uint32_t gm = rr ? gm1 : gm0, st = rr ? st1 : st0;
-          const float S = __fmul_rn((float)(gm & 0xffu), f16_bits_to_f32(st)) * sc;
-          const float ZS = __fmul_rn((float)((gm >> 8) & 0xffu), f16_bits_to_f32(st >> 16)) * S;
-          const __half2 s2 = __float2half2_rn(S), nz2 = __float2half2_rn(-ZS);
-          const __half2 m1024 = __float2half2_rn(1024.f), m64 = __float2half2_rn(64.f);
-          const uint4 cv = *reinterpret_cast<const uint4 *>(P + r * PROW + h * (PROW / 2));
-          const uint32_t cw[4] = {cv.x, cv.y, cv.z, cv.w};
+        for (int q = 0; q < 4; ++q) {
+          const uint32_t wd = cw[q], w8 = wd >> 8;
+          uint32_t pr[4];
+          pr[0] = (wd & 0x000F000Fu) | 0x64006400u;  // (1024 + n0, 1024 + n4)
+          pr[1] = (wd & 0x00F000F0u) | 0x54005400u;  // (64 + n1, 64 + n5)
+          pr[2] = (w8 & 0x000F000Fu) | 0x64006400u;  // (1024 + n2, 1024 + n6)
+          pr[3] = (w8 & 0x00F000F0u) | 0x54005400u;  // (64 + n3, 64 + n7)
+          uint32_t o[4];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const uint32_t wd = cw[q], w8 = wd >> 8;
-            uint32_t pr[4];
-            pr[0] = (wd & 0x000F000Fu) | 0x64006400u;  // (1024 + n0, 1024 + n4)
-            pr[1] = (wd & 0x00F000F0u) | 0x54005400u;  // (64 + n1, 64 + n5)
-            pr[2] = (w8 & 0x000F000Fu) | 0x64006400u;  // (1024 + n2, 1024 + n6)
-            pr[3] = (w8 & 0x00F000F0u) | 0x54005400u;  // (64 + n3, 64 + n7)
-            uint32_t o[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const __half2 qv = __hsub2(*reinterpret_cast<const __half2 *>(&pr[e]), (e & 1) ? m64 : m1024);
-              const __half2 wv = __hfma2(qv, s2, nz2);
-              o[e] = *reinterpret_cast<const uint32_t *>(&wv);
-            }
-            const int j = 4 * h + q;  // logical 16-byte chunk of the 128-byte row
-            *reinterpret_cast<uint4 *>(row + ((j ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+          for (int e = 0; e < 4; ++e) {
+            const __half2 qv = __hsub2(*reinterpret_cast<const __half2 *>(&pr[e]), (e & 1) ? m64 : m1024);
+            const __half2 wv = __hfma2(qv, s2, nz2);
+            o[e] = *reinterpret_cast<const uint32_t *>(&wv);
           }
-        } else {
-          float w[32];
-          smem_decode32<FMT, BITS>(P + r * PROW + h * (PROW / 2), rr ? gm1 : gm0, rr ? st1 : st0, w);
+          const int j = 4 * h + q;  // logical 16-byte chunk of the 128-byte row
+          *reinterpret_cast<uint4 *>(dst_row + ((j ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+      } else {
+        float w[32];
+        smem_decode32<FMT, BITS>(src, gm, st, w);
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int j = 4 * h + q;  // logical 16-byte chunk of the 128-byte row
-            uint4 v;
-            v.x = pack_f16x2(w[8 * q + 0] * sc, w[8 * q + 4] * sc);
-            v.y = pack_f16x2(w[8 * q + 1] * sc, w[8 * q + 5] * sc);
-            v.z = pack_f16x2(w[8 * q + 2] * sc, w[8 * q + 6] * sc);
-            v.w = pack_f16x2(w[8 * q + 3] * sc, w[8 * q + 7] * sc);
-            *reinterpret_cast<uint4 *>(row + ((j ^ (r & 7)) << 4)) = v;
-          }
+        for (int q = 0; q < 4; ++q) {
+          const int j = 4 * h + q;  // logical 16-byte chunk of the 128-byte row
+          uint4 v;
+          v.x = pack_f16x2(w[8 * q + 0] * sc, w[8 * q + 4] * sc);
+          v.y = pack_f16x2(w[8 * q + 1] * sc, w[8 * q + 5] * sc);
+          v.z = pack_f16x2(w[8 * q + 2] * sc, w[8 * q + 6] * sc);
+          v.w = pack_f16x2(w[8 * q + 3] * sc, w[8 * q + 7] * sc);
+          *reinterpret_cast<uint4 *>(dst_row + ((j ^ (r & 7)) << 4)) = v;
         }
       }
       fence_proxy_async_smem();
       __syncwarp();
       if ((t & 31) == 0) mbar_arrive(bar_b_full(s));
-      gm0 = ngm0; st0 = nst0; gm1 = ngm1; st1 = nst1;
-      sc0 = nsc0; sc1 = nsc1;
+      step_ring(s, ph, STAGES);
+      gm = ngm;
+      st = nst;
+      sc = nsc;
     }
   }
 
