@@ -49,6 +49,9 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--gemm-iters", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-other-configs", action="store_true")
+    ap.add_argument("--load-window", type=float, default=1.5,
+                    help="seconds of extra steps run after the timed region so the clock sampler sees load")
     return ap.parse_args(argv)
 
 
@@ -302,7 +305,7 @@ def run_native(args):
 
     # keep the same load running for ~1.5 s so the clock sampler sees it
     t_a = time.time()
-    while time.time() - t_a < 1.5:
+    while time.time() - t_a < args.load_window:
         g_timed.replay()
         torch.cuda.synchronize(device)
     sampler.mark(t_a, time.time())
@@ -320,6 +323,7 @@ def run_native(args):
 
     gemm = run_gemm(args, device, peaks, sampler)
     e2e = run_e2e(args, layers, device, step_bytes)
+    others = None if args.no_other_configs else run_other_configs(device, peaks)
     for L in layers:
         L["reps"].clear()
     clocks = sampler.stop()
@@ -351,6 +355,7 @@ def run_native(args):
                      "peak_source": f"{peaks['source']} (copy bandwidth)", "kernel": "qlinear_gemv (int4, M=1)",
                      "bytes_per_call": bytes_per_call, "mean_call_us": [round(u, 3) for u in launch_us]},
         "gemm_m2048": gemm,
+        "other_configs": others,
         "e2e": e2e,
         "gpu_launches": args.steps * len(layers) * KERNELS_PER_GEMV,
         "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
@@ -404,6 +409,99 @@ def run_gemm(args, device, peaks, sampler):
                          "peak_source": f"{peaks['source']} dense bf16 (burst)"},
             "l2": "256 MiB buffer written between timed calls",
             "launches_per_call": 3, "note": "each call = x->fp16 pass + weight-scale pass + tcgen05 GEMM"}
+
+
+def packed_layer(wl, device):
+    """Pack one synthetic workload layer on the device; returns (desc, (codes, gmeta, steps), bytes)."""
+    import numpy as np
+    import torch
+
+    import int6_quantized_linear_b200 as ql
+
+    d = ql.Desc(wl.fmt, wl.N, wl.K, wl.bits, wl.group)
+    w = wl.weights()
+    t16 = lambda a: torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a).to(device)
+    if wl.fmt == "int4":
+        u = (w["q"], w["sc"], w["zc"], w["ss"], w["zs"])
+    elif wl.fmt == "int6":
+        u = (w["q"], w["sc"], None, w["st"], None)
+    else:
+        u = (w["q"], w["s"], w["b"], None, None)
+    packed = ql.alloc_packed(d, device)
+    ql.qlinear_pack(d, *[t16(a) if a is not None else None for a in u], *packed)
+    return d, packed, sum(ql.qlinear_packed_bytes(d))
+
+
+def run_other_configs(device, peaks):
+    """The remaining workload configurations, each at its batch sizes: GB/s of algorithmic bytes for
+    the GEMVs (CUDA-graph replays of 30 calls over 3 rotating weight copies), TFLOP/s for the GEMM
+    (CUDA events around single calls, 256 MiB written between calls)."""
+    import torch
+
+    import int6_quantized_linear_b200 as ql
+    from int6_quantized_linear_b200 import synth
+
+    out = {}
+    for name in ("int4_gemv_k5120_n27648", "int4_gemv_k27648_n5120", "int6_gemv_k5120_n5120",
+                 "int6_gemv_k5120_n27648", "affine2_k4096_n14336", "affine4_k4096_n14336",
+                 "affine8_k4096_n14336"):
+        wl = synth.WORKLOADS[name]
+        d, p0, wbytes = packed_layer(wl, device)
+        reps = [p0] + [tuple(t.clone() for t in p0) for _ in range(2)]
+        xb = torch.from_numpy(wl.x(max(wl.Ms)).view("int16")).to(device).view(torch.bfloat16)
+        res = {}
+        for M in wl.Ms:
+            if name.startswith("int4") and M == 1:
+                continue  # the headline line above
+            x = xb[:M].contiguous()
+            y = torch.empty((M, wl.N), dtype=torch.bfloat16, device=device)
+            ws = ql.alloc_gemv_workspace(d, M, device)
+            for i in range(3):
+                ql.qlinear_gemv(d, *reps[i], x, M, y, ws)
+            calls = 30
+            g = capture(lambda: [ql.qlinear_gemv(d, *reps[i % 3], x, M, y, ws) for i in range(calls)], device)
+            g.replay()
+            torch.cuda.synchronize(device)
+            a, b = _ev(), _ev()
+            a.record()
+            g.replay()
+            g.replay()
+            b.record()
+            torch.cuda.synchronize(device)
+            us = a.elapsed_time(b) * 1e3 / (2 * calls)
+            nbytes = wbytes + M * wl.K * 2 + M * wl.N * 2
+            res[f"M{M}"] = {"us": round(us, 3), "GB/s": round(nbytes / us / 1e3, 1),
+                            "frac_hbm": round(nbytes / us / 1e3 / peaks["hbm_gbs"], 4)}
+            del g
+        out[name] = res
+        del reps
+    wl = synth.WORKLOADS["int4_gemm_k5120_n27648"]
+    d, (c, g_, s), _ = packed_layer(wl, device)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
+    res = {}
+    for M in (512, 8192):
+        x = torch.from_numpy(wl.x(M).view("int16")).to(device).view(torch.bfloat16)
+        y = torch.empty((M, wl.N), dtype=torch.bfloat16, device=device)
+        ws = ql.alloc_gemm_workspace(d, M, device)
+        for _ in range(2):
+            ql.qlinear_gemm(d, c, g_, s, x, M, y, ws)
+        times = []
+        for _ in range(5):
+            flush.fill_(1)
+            a, b = _ev(), _ev()
+            a.record()
+            ql.qlinear_gemm(d, c, g_, s, x, M, y, ws)
+            b.record()
+            torch.cuda.synchronize(device)
+            times.append(a.elapsed_time(b) / 1e3)
+        t = statistics.median(times)
+        tf = 2.0 * M * wl.N * wl.K / t / 1e12
+        res[f"M{M}"] = {"ms": round(t * 1e3, 4), "TFLOP/s": round(tf, 1),
+                        "frac_bf16_peak": round(tf / peaks["bf16_tflops"], 4)}
+        del x, y, ws
+    out["int4_gemm_k5120_n27648"] = res
+    assert ql.qlinear_sync_status() == ql.QL_OK
+    return out
 
 
 def run_e2e(args, layers, device, step_bytes):
