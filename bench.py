@@ -39,7 +39,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes per GEMV launch from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum),
 # valid only while the GEMV source is unchanged (hash of csrc/gemv.cuh at capture time).
 NCU_TRAFFIC = {"gemv_src_sha256": "2afddf42e467fc10e0f205c81da84f9875f1874a7bd3a70dcea1d47e6ba1b05e",
-               "bytes_per_launch": 83168768}  # mean of the two decode layers (profiles/gemv_int4_m1_*.md)
+               "bytes_per_launch": 83168768}  # mean over the two decode layers
 
 
 def parse_args(argv=None):
