@@ -92,13 +92,19 @@ __global__ void __launch_bounds__(256) gemv_simple_kernel(WeightPtrs p, int64_t 
 // block, so no per-MMA selects are needed.
 // ===========================================================================
 
+constexpr int GEMV_MT_MAX_CTAS = 4096;  // bound on the CTAs of one multi-token launch (sizes its partial sums)
+
 struct GemvWorkspace {
-  uint4 *xq;      // [M][K/256 super-blocks][4 j][2 kinds][8 groups][16 B]: B-operand pairs, see gemv_xprep_kernel
-  float2 *gsum;   // [M][K/32] (2^-a_g / 16, -16 * sum x_int)
+  uint4 *xq;        // M = 1: [K/256 super-blocks][4 j][2 kinds][8 groups][16 B] B-operand pairs (gemv_xprep_kernel)
+                    // M > 1: [K/32 groups][M tokens][4][16 B] B-operand words (gemv_xprep_mt_kernel)
+  float2 *gsum;     // M = 1: [K/32]; M > 1: [K/32][M]: (2^-a_g / 16, -16 * sum x_int)
+  float *partial;   // M > 1: [CTA][M][64 rows] sums of a CTA's K range
+  int *counters;    // M > 1: [N/64 row groups] parts finished so far
 };
 
-inline size_t gemv_workspace_bytes(int64_t M, int64_t K) {
-  return align256((size_t)M * K * 4) + align256((size_t)M * (K / 32) * 8);
+inline size_t gemv_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  return align256((size_t)M * K * 4) + align256((size_t)M * (K / 32) * 8) +
+         align256((size_t)GEMV_MT_MAX_CTAS * 64 * M * 4) + align256((size_t)((N + 63) / 64) * 4);
 }
 
 inline GemvWorkspace gemv_workspace_carve(void *base, int64_t M, int64_t K) {
@@ -107,6 +113,10 @@ inline GemvWorkspace gemv_workspace_carve(void *base, int64_t M, int64_t K) {
   w.xq = reinterpret_cast<uint4 *>(p);
   p += align256((size_t)M * K * 4);
   w.gsum = reinterpret_cast<float2 *>(p);
+  p += align256((size_t)M * (K / 32) * 8);
+  w.partial = reinterpret_cast<float *>(p);
+  p += align256((size_t)GEMV_MT_MAX_CTAS * 64 * M * 4);
+  w.counters = reinterpret_cast<int *>(p);
   return w;
 }
 
@@ -180,6 +190,11 @@ QL_DEVI uint4 lds128(uint32_t a) {
 QL_DEVI float4 lds128f(uint32_t a) {
   float4 v;
   asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(a));
+  return v;
+}
+QL_DEVI float2 lds64f(uint32_t a) {
+  float2 v;
+  asm volatile("ld.shared.v2.f32 {%0,%1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(a));
   return v;
 }
 QL_DEVI uint32_t lds32(uint32_t a) {
@@ -439,6 +454,288 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS, GEMV_CTAS_PER_SM)
     for (int q = 0; q < P; ++q) sum += red[(warp + q) * 16 + lane];
     const int64_t r = tile * 16 + lane;
     if (r < p.N) p.y[r] = __float2bfloat16_rn(sum);
+  }
+}
+
+
+// ===========================================================================
+// Tensor-core decode GEMV for int4 at 2 <= M <= 8 tokens.
+//
+// The same integer MMA (m16n8k32, u8 codes x16 against the high / low bytes of
+// 16-bit fixed-point x) with the 8 MMA columns as the tokens (a dense B):
+// one MMA pair per (16 rows, 32-weight group) covers every token, so D is the
+// group partial of 16 rows x 8 tokens and the scale and zero are applied per
+// (row, token, group).  Lane (g, c) supplies code word c of the group for tile
+// rows g and g + 8 (even-k codes to slots 4c.., odd-k codes to slots 4c+16..)
+// and, as column g, token g's x bytes of those slots; it ends with the sums of
+// rows g, g + 8 for tokens 2c, 2c + 1.
+//
+// A CTA is one producer warp and four consumer warps on 64 weight rows (four
+// 16-row tiles) and a range of super-blocks: each stage (codes box, group-word
+// box, every token's x words and group sums) is fetched once and read by all
+// four.  When the row groups alone do not fill one wave of GEMV_MT_CTAS_PER_SM
+// CTAs per SM, K is split over P CTAs per row group; each writes its sums to the
+// workspace and the CTA that finds the others done (a counter per row group,
+// cleared by the preparation pass) adds the P parts in part order and writes y.
+// ===========================================================================
+
+// x preparation for M > 1: 4 lanes per (token, 32-element group); lane c owns k = 8c .. 8c + 7 and
+// writes its MMA word quad (even-k high bytes, odd-k high bytes, even-k low bytes, odd-k low bytes).
+__global__ void __launch_bounds__(256) gemv_xprep_mt_kernel(const __nv_bfloat16 *x, int64_t M, int64_t K,
+                                                            int64_t n_counters, GemvWorkspace ws) {
+  pdl_launch_dependents();  // the streaming kernel may start fetching weights now
+  pdl_wait();               // x (and this workspace) may belong to the kernel launched before this one
+  const int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (t < n_counters) ws.counters[t] = 0;
+  const int64_t ng = K / 32;
+  const int64_t gq = t >> 2;  // (token, group), token-major
+  const int c = (int)(t & 3);
+  const bool live = gq < M * ng;  // every lane takes part in the shuffles
+  const int64_t m = live ? gq / ng : 0, g = live ? gq - m * ng : 0;
+  uint4 v = make_uint4(0u, 0u, 0u, 0u);
+  if (live) v = __ldg(reinterpret_cast<const uint4 *>(x + m * K + 32 * g + 8 * c));
+  const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+  float xs[8];
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    xs[2 * i] = bf16_bits_to_f32(u[i]);
+    xs[2 * i + 1] = bf16_bits_to_f32(u[i] >> 16);
+    amax = fmaxf(amax, fmaxf(fabsf(xs[2 * i]), fabsf(xs[2 * i + 1])));
+  }
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+  const int a = scale_exponent(amax, 14);  // max |x_int| < 2^15
+  const float sc = exp2i(a);
+  uint32_t eh = 0, oh = 0, el = 0, ol = 0;
+  int sum = 0;
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    const int xe = __float2int_rn(xs[2 * b] * sc), xo = __float2int_rn(xs[2 * b + 1] * sc);
+    sum += xe + xo;
+    eh |= ((uint32_t)(xe >> 8) & 0xffu) << (8 * b);
+    el |= ((uint32_t)xe & 0xffu) << (8 * b);
+    oh |= ((uint32_t)(xo >> 8) & 0xffu) << (8 * b);
+    ol |= ((uint32_t)xo & 0xffu) << (8 * b);
+  }
+  sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+  sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+  if (!live) return;
+  ws.xq[(g * M + m) * 4 + c] = make_uint4(eh, oh, el, ol);
+  if (c == 0) ws.gsum[g * M + m] = make_float2(exp2i(-a) * 0.0625f, -16.f * (float)sum);
+}
+
+constexpr int GEMV_MT_WARPS = 4;  // consumer warps per CTA; warp 4 produces
+constexpr int GEMV_MT_THREADS = 32 * (GEMV_MT_WARPS + 1);
+constexpr int GEMV_MT_RING = 4;
+constexpr int GEMV_MT_CTAS_PER_SM = 3;
+// stage: codes [64 rows][128 B] (128-byte swizzle), group words [64][16 B], group sums [8][M][8 B],
+// x words [8 groups][M][4][16 B]
+constexpr int GEMV_MT_ST_CODES = 0, GEMV_MT_ST_GMETA = 8192, GEMV_MT_ST_GSUM = 9216, GEMV_MT_ST_X = 9728;
+constexpr int GEMV_MT_STAGE_BYTES = 14336;
+
+struct GemvMtParams {
+  const uint8_t *steps;
+  int64_t N, K;
+  int M;  // 2 .. 8 tokens
+  int P;  // CTAs per 64-row group (K split)
+  GemvWorkspace ws;
+  __nv_bfloat16 *y;
+};
+
+inline constexpr int gemv_mt_smem_bytes() { return GEMV_MT_RING * GEMV_MT_STAGE_BYTES + GEMV_MT_RING * 16 + 16 + 1024; }
+
+__global__ void __launch_bounds__(GEMV_MT_THREADS, GEMV_MT_CTAS_PER_SM)
+    gemv_int4_mt_kernel(const __grid_constant__ CUtensorMap map_codes,
+                        const __grid_constant__ CUtensorMap map_gmeta, GemvMtParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + GEMV_MT_RING * GEMV_MT_STAGE_BYTES);  // full[R], empty[R]
+  int *flags = reinterpret_cast<int *>(bars + 2 * GEMV_MT_RING);  // abort, last-part
+  volatile int *abort_flag = flags;
+  const uint32_t sbase = smem_u32(smem);
+  auto bar_full = [&](int s) { return smem_u32(bars + s); };
+  auto bar_empty = [&](int s) { return smem_u32(bars + GEMV_MT_RING + s); };
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int P = p.P, M = p.M;
+  const int NS = (int)(p.K / 256);
+  const int64_t rg = blockIdx.x / P;  // 64-row group
+  const int part = (int)(blockIdx.x - rg * P);
+  const int sb0 = part * NS / P, nsb = (part + 1) * NS / P - sb0;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < GEMV_MT_RING; ++s) {
+      mbar_init(bar_full(s), 1);
+      mbar_init(bar_empty(s), GEMV_MT_WARPS);
+    }
+    flags[0] = 0;
+    flags[1] = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  pdl_launch_dependents();  // the next call's preparation pass waits for this grid before touching anything
+
+  if (warp == GEMV_MT_WARPS) {  // producer
+    if (lane == 0) {
+      tma_prefetch_desc(&map_codes);
+      tma_prefetch_desc(&map_gmeta);
+      const uint32_t tx = 8192 + 1024 + (uint32_t)M * 64 + (uint32_t)M * 512;
+      auto issue_w = [&](int i, int s) {
+        const uint32_t st = sbase + s * GEMV_MT_STAGE_BYTES;
+        mbar_arrive_expect_tx(bar_full(s), tx);
+        tma_load_2d(st + GEMV_MT_ST_CODES, &map_codes, bar_full(s), (sb0 + i) * 128, (int32_t)(rg * 64));
+        tma_load_2d(st + GEMV_MT_ST_GMETA, &map_gmeta, bar_full(s), (sb0 + i) * 16, (int32_t)(rg * 64));
+      };
+      auto issue_x = [&](int i, int s) {
+        const uint32_t st = sbase + s * GEMV_MT_STAGE_BYTES;
+        const int64_t g0 = (int64_t)(sb0 + i) * 8;  // first group of the super-block
+        bulk_load(st + GEMV_MT_ST_GSUM, p.ws.gsum + g0 * M, (uint32_t)M * 64, bar_full(s));
+        bulk_load(st + GEMV_MT_ST_X, p.ws.xq + g0 * M * 4, (uint32_t)M * 512, bar_full(s));
+      };
+      const int pre = nsb < GEMV_MT_RING ? nsb : GEMV_MT_RING;
+      for (int i = 0; i < pre; ++i) issue_w(i, i);  // weights need no x
+      pdl_wait();
+      for (int i = 0; i < pre; ++i) issue_x(i, i);
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      int i = pre;
+      for (; i < nsb; ++i) {  // unit i reuses the stage of unit i - RING
+        if (!mbar_wait_bounded(bar_empty(s), ph, abort_flag)) {
+          ok = false;
+          break;
+        }
+        issue_w(i, s);
+        issue_x(i, s);
+        if (++s == GEMV_MT_RING) {
+          s = 0;
+          ph ^= 1u;
+        }
+      }
+      if (!ok) {  // let the copies in flight land before the CTA can exit
+        for (int j = i - 1; j >= 0 && j >= i - GEMV_MT_RING; --j) {
+          const long long t0 = clock64();
+          while (!mbar_try_wait(bar_full(j % GEMV_MT_RING), (uint32_t)((j / GEMV_MT_RING) & 1)) &&
+                 clock64() - t0 < QL_WAIT_LIMIT_CYCLES) {
+          }
+        }
+      }
+    }
+  } else {  // consumers: warp w owns box rows 16w + g and 16w + g + 8
+    const int g = lane >> 2, c = lane & 3;
+    const int r0 = 16 * warp + g, r1 = r0 + 8;
+    int64_t n0 = rg * 64 + r0, n1 = n0 + 8;
+    const int64_t c0 = n0 < p.N ? n0 : p.N - 1, c1 = n1 < p.N ? n1 : p.N - 1;
+    const uint32_t *st0 = reinterpret_cast<const uint32_t *>(p.steps) + c0 * NS + sb0;
+    const uint32_t *st1 = reinterpret_cast<const uint32_t *>(p.steps) + c1 * NS + sb0;
+    uint32_t sr0[GEMV_MT_RING], sr1[GEMV_MT_RING];  // step words by stage, RING - 1 super-blocks ahead
+#pragma unroll
+    for (int s = 0; s < GEMV_MT_RING; ++s) {
+      sr0[s] = 0u;
+      sr1[s] = 0u;
+      if (s < GEMV_MT_RING - 1 && s < nsb) {
+        sr0[s] = __ldg(st0 + s);
+        sr1[s] = __ldg(st1 + s);
+      }
+    }
+    const int32_t acc_init[4] = {GEMV_ACC0, GEMV_ACC0, GEMV_ACC0, GEMV_ACC0};
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};  // (row g | g + 8) x (token 2c | 2c + 1)
+    const uint32_t sw = (uint32_t)(r0 & 7);
+    bool ok = true;
+    for (int base = 0; base < nsb && ok; base += GEMV_MT_RING) {
+      const uint32_t par = (uint32_t)((base / GEMV_MT_RING) & 1);
+#pragma unroll
+      for (int s = 0; s < GEMV_MT_RING; ++s) {
+        const int i = base + s;
+        if (i >= nsb) break;
+        const int nx = i + GEMV_MT_RING - 1, sn = (s + GEMV_MT_RING - 1) % GEMV_MT_RING;
+        if (nx < nsb) {
+          sr0[sn] = __ldg(st0 + nx);
+          sr1[sn] = __ldg(st1 + nx);
+        }
+        if (!mbar_wait_bounded(bar_full(s), par, abort_flag)) {
+          ok = false;
+          break;
+        }
+        const uint32_t stg = sbase + s * GEMV_MT_STAGE_BYTES;
+        const uint4 gm0 = lds128(stg + GEMV_MT_ST_GMETA + r0 * 16), gm1 = lds128(stg + GEMV_MT_ST_GMETA + r1 * 16);
+        const uint32_t gw0[4] = {gm0.x, gm0.y, gm0.z, gm0.w}, gw1[4] = {gm1.x, gm1.y, gm1.z, gm1.w};
+        const uint32_t cs0 = sr0[s], cs1 = sr1[s];
+        const float ss0 = f16_bits_to_f32(cs0), zs0 = f16_bits_to_f32(cs0 >> 16);
+        const float ss1 = f16_bits_to_f32(cs1), zs1 = f16_bits_to_f32(cs1 >> 16);
+        const float nss0 = -8388608.f * ss0, nzs0 = -8388608.f * zs0;
+        const float nss1 = -8388608.f * ss1, nzs1 = -8388608.f * zs1;
+#pragma unroll
+        for (int gg = 0; gg < 8; ++gg) {
+          const uint32_t coff = (((uint32_t)gg ^ sw) << 4) + 4 * c;
+          const uint32_t w0 = lds32(stg + r0 * 128 + coff), w1 = lds32(stg + r1 * 128 + coff);
+          const uint4 xv = lds128(stg + GEMV_MT_ST_X + ((gg * M + g) * 4 + c) * 16);
+          // (2^-a/16, -16 X) of tokens 2c and 2c + 1: 8-byte records, so two 8-byte loads (odd M)
+          const float2 Ga = lds64f(stg + GEMV_MT_ST_GSUM + (gg * M + 2 * c) * 8);
+          const float2 Gb = lds64f(stg + GEMV_MT_ST_GSUM + (gg * M + 2 * c + 1) * 8);
+          const float4 G = make_float4(Ga.x, Ga.y, Gb.x, Gb.y);
+          const uint32_t e0 = (w0 << 4) & 0xF0F0F0F0u, e1 = (w1 << 4) & 0xF0F0F0F0u;  // even k, x16
+          const uint32_t o0 = w0 & 0xF0F0F0F0u, o1 = w1 & 0xF0F0F0F0u;                  // odd k, x16
+          int32_t dh[4], dl[4];
+          QL_IMMA0("s8", dh, acc_init, e0, e1, o0, o1, xv.x, xv.y);
+          QL_IMMA0("u8", dl, acc_init, e0, e1, o0, o1, xv.z, xv.w);
+          float t[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            t[q] = fmaf(__int_as_float(dh[q]) - GEMV_ACC0_F, 256.f, __int_as_float(dl[q]) - GEMV_ACC0_F);
+          const uint32_t gw0g = gw0[gg >> 1], gw1g = gw1[gg >> 1];
+          const int bsc = 2 * (gg & 1);
+          const float S0 = fmaf(byte_magic(gw0g, bsc), ss0, nss0), Z0 = fmaf(byte_magic(gw0g, bsc + 1), zs0, nzs0);
+          const float S1 = fmaf(byte_magic(gw1g, bsc), ss1, nss1), Z1 = fmaf(byte_magic(gw1g, bsc + 1), zs1, nzs1);
+          acc[0] = fmaf(S0 * G.x, fmaf(Z0, G.y, t[0]), acc[0]);
+          acc[1] = fmaf(S0 * G.z, fmaf(Z0, G.w, t[1]), acc[1]);
+          acc[2] = fmaf(S1 * G.x, fmaf(Z1, G.y, t[2]), acc[2]);
+          acc[3] = fmaf(S1 * G.z, fmaf(Z1, G.w, t[3]), acc[3]);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_empty(s));
+      }
+    }
+    // publish: rows n0, n1 x tokens 2c, 2c + 1
+    const int tk0 = 2 * c, tk1 = 2 * c + 1;
+    if (ok) {
+      if (P == 1) {
+        if (n0 < p.N) {
+          if (tk0 < M) p.y[(int64_t)tk0 * p.N + n0] = __float2bfloat16_rn(acc[0]);
+          if (tk1 < M) p.y[(int64_t)tk1 * p.N + n0] = __float2bfloat16_rn(acc[1]);
+        }
+        if (n1 < p.N) {
+          if (tk0 < M) p.y[(int64_t)tk0 * p.N + n1] = __float2bfloat16_rn(acc[2]);
+          if (tk1 < M) p.y[(int64_t)tk1 * p.N + n1] = __float2bfloat16_rn(acc[3]);
+        }
+      } else {
+        float *mine = p.ws.partial + (int64_t)blockIdx.x * M * 64;
+        if (tk0 < M) {
+          mine[tk0 * 64 + r0] = acc[0];
+          mine[tk0 * 64 + r1] = acc[2];
+        }
+        if (tk1 < M) {
+          mine[tk1 * 64 + r0] = acc[1];
+          mine[tk1 * 64 + r1] = acc[3];
+        }
+        __threadfence();
+      }
+    }
+  }
+  if (P > 1) {  // the CTA that completes a row group adds its P parts in part order
+    __syncthreads();
+    if (threadIdx.x == 0 && !*abort_flag) flags[1] = atomicAdd(p.ws.counters + rg, 1) == P - 1;
+    __syncthreads();
+    if (flags[1] && warp < GEMV_MT_WARPS) {
+      __threadfence();
+      const float *base = p.ws.partial + (int64_t)rg * P * M * 64;
+      for (int e = threadIdx.x; e < M * 64; e += GEMV_MT_WARPS * 32) {
+        const int tk = e >> 6, r = e & 63;
+        float sum = 0.f;
+        for (int q = 0; q < P; ++q) sum += __ldcg(base + (int64_t)q * M * 64 + e);
+        const int64_t n = rg * 64 + r;
+        if (n < p.N) p.y[(int64_t)tk * p.N + n] = __float2bfloat16_rn(sum);
+      }
+    }
   }
 }
 

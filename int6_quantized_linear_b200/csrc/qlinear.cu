@@ -227,6 +227,60 @@ ql_status launch_gemv(const ql_desc *d, const ql_packed_const *w, const void *x,
       if (cudaLaunchKernelEx(&cfg, gemv_int4_m1_tc_kernel, mc, mg, p) != cudaSuccess) return QL_ERR_CUDA;
       return launched();
     }
+    if (M >= 2 && M <= 8) {  // multi-token tensor-core path
+      const int64_t N = d->N, K = d->K, NS = K / 256, TG = (N + 63) / 64;
+      const GemvWorkspace ws = gemv_workspace_carve(workspace, M, K);
+      cudaLaunchAttribute pa[1];
+      pa[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      pa[0].val.programmaticStreamSerializationAllowed = 1;
+      {
+        const int64_t threads = std::max<int64_t>(4 * M * (K / 32), TG);
+        cudaLaunchConfig_t pc = {};
+        pc.gridDim = dim3((unsigned)((threads + 255) / 256));
+        pc.blockDim = dim3(256);
+        pc.stream = st;
+        pc.attrs = pa;
+        pc.numAttrs = 1;
+        if (cudaLaunchKernelEx(&pc, gemv_xprep_mt_kernel, xb, M, K, TG, ws) != cudaSuccess) return QL_ERR_CUDA;
+      }
+      GemvMtParams p;
+      p.steps = static_cast<const uint8_t *>(w->steps);
+      p.N = N;
+      p.K = K;
+      p.M = (int)M;
+      // split K over P CTAs per 64-row group while the row groups alone leave a wave unfilled
+      int64_t P = std::max<int64_t>(1, std::min<int64_t>(NS, (int64_t)sms * GEMV_MT_CTAS_PER_SM / TG));
+      P = std::min<int64_t>(P, std::max<int64_t>(1, GEMV_MT_MAX_CTAS / TG));
+      if (TG * P > GEMV_MT_MAX_CTAS) return QL_ERR_RANGE;
+      p.P = (int)P;
+      p.ws = ws;
+      p.y = yb;
+      CUtensorMap mc, mg;  // codes as [N][K/2] bytes, boxes of 64 rows x 128 bytes, 128-byte swizzle;
+                           // group words as [N][K/16] bytes, boxes of 64 rows x 16 bytes
+      if (!encode_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->codes, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2,
+                     128, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+          !encode_2d(&mg, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->gmeta, (uint64_t)K / 16, (uint64_t)N, (uint64_t)K / 16,
+                     16, 64, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return QL_ERR_CUDA;
+      static thread_local int configured_dev = -1;
+      int dev = 0;
+      cudaGetDevice(&dev);
+      if (configured_dev != dev) {
+        if (cudaFuncSetAttribute(gemv_int4_mt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 gemv_mt_smem_bytes()) != cudaSuccess)
+          return QL_ERR_CUDA;
+        configured_dev = dev;
+      }
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3((unsigned)(TG * P));
+      cfg.blockDim = dim3(GEMV_MT_THREADS);
+      cfg.dynamicSmemBytes = gemv_mt_smem_bytes();
+      cfg.stream = st;
+      cfg.attrs = pa;
+      cfg.numAttrs = 1;
+      if (cudaLaunchKernelEx(&cfg, gemv_int4_mt_kernel, mc, mg, p) != cudaSuccess) return QL_ERR_CUDA;
+      return launched();
+    }
   }
   const WeightPtrs p = make_ptrs(d, w);
   const int64_t rows_per_block = 8;
@@ -413,7 +467,7 @@ ql_status qlinear_gemv_workspace_bytes(const ql_desc *d, int64_t M, size_t *byte
   if (!bytes) return QL_ERR_NULL;
   const int64_t mmax = d->fmt == QL_AFFINE_U32 ? 32 : 8;
   if (M < 1 || M > mmax) return QL_ERR_RANGE;
-  *bytes = gemv_workspace_bytes(M, d->K);
+  *bytes = gemv_workspace_bytes(M, d->N, d->K);
   return QL_OK;
 }
 
@@ -426,7 +480,7 @@ ql_status qlinear_gemv(const ql_desc *d, const ql_packed_const *w, const void *x
   if (!aligned16(x) || !aligned16(y) || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return QL_ERR_ALIGN;
   const int64_t mmax = d->fmt == QL_AFFINE_U32 ? 32 : 8;
   if (M < 1 || M > mmax) return QL_ERR_RANGE;
-  if (workspace_bytes < gemv_workspace_bytes(M, d->K)) return QL_ERR_SHAPE;
+  if (workspace_bytes < gemv_workspace_bytes(M, d->N, d->K)) return QL_ERR_SHAPE;
   DeviceInfo *di;
   if ((st = device_info(&di)) != QL_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
