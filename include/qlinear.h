@@ -170,28 +170,38 @@ ql_status qlinear_dequant(const ql_desc *desc, const ql_packed_const *w,
                           void *out, int32_t out_dtype, ql_stream_t stream);
 
 /* Bytes of caller-provided device workspace qlinear_gemv needs for `desc`
- * and M (host-only, no CUDA call): 2*M*K for x in the order the kernel's
- * tensor-core fragments read it, 8*M*K/32 for two sums per 32-weight group,
- * 4*M for the per-token scales and 256 for a zero block, each part rounded
- * up to 256 bytes.  Errors: QL_ERR_NULL, QL_ERR_SHAPE, QL_ERR_RANGE,
- * QL_ERR_UNSUPPORTED. */
+ * and M (host-only, no CUDA call): 4*M*K for x in the order the tensor-core
+ * fragments read it, 8*M*K/32 for two sums per 32-weight group,
+ * 4*4096*64*M for the partial sums of a K split and 4*ceil(N/64) for its
+ * counters, each part rounded up to 256 bytes; for int6 / affine at M >= 8
+ * (those calls run on the GEMM) at least qlinear_gemm_workspace_bytes().
+ * Errors: QL_ERR_NULL, QL_ERR_SHAPE, QL_ERR_RANGE, QL_ERR_UNSUPPORTED. */
 ql_status qlinear_gemv_workspace_bytes(const ql_desc *desc, int64_t M, size_t *bytes);
 
 /* Decode-shaped layer, HBM-bound: y[M][N] (bf16) = x[M][K] (bf16) . W^T,
- * fp32 accumulation, one nearest-even rounding to bf16 at the end.
+ * fp32 scales and accumulation, one nearest-even rounding to bf16 at the end.
  * 1 <= M <= 8 for int4 / int6; 1 <= M <= 32 for affine.
- * int4 at M = 1 runs two launches: a short pass that scales x per token by a
- * power of two into fp16 range, reorders it for the tensor-core fragments
- * and sums it per group into the workspace; then the streaming kernel, in
- * which mma.sync multiplies the exactly converted codes (1024+q, 64+q in
- * fp16) by x and the per-group scale and zero are applied in fp32.  Other
- * formats and M: one launch, exact binary32 weights, fp32 FMA.
- * ExecuTorch page above, review section "Things done well" (the decode
- * kernel's one-shuffle step-word broadcast and full-warp trip counts) and
- * "Quant schema update" (hoisted int6 codes).
+ *  - int4, 1 <= M <= 8: two launches.  A short pass turns each 32-element
+ *    group of x into 16-bit fixed point (x_int = rint(x * 2^a), the group's
+ *    max |x| scaled into [2^14, 2^15)), split into high and low bytes in the
+ *    order the tensor-core fragments read them, with the group's sum; then
+ *    the streaming kernel multiplies the codes (as u8 times 16) by those bytes
+ *    on the integer tensor core (mma.sync m16n8k32, exact s32 sums) and
+ *    applies scale and zero once per (row, group[, token]) in fp32.  M = 1
+ *    uses a diagonal x operand (one MMA column per group); M >= 2 uses the
+ *    tokens as MMA columns and may split K over CTAs, adding the parts in a
+ *    fixed order through the workspace.
+ *  - int6 / affine, M < 8: one launch, exact binary32 weights, fp32 FMA.
+ *  - int6 / affine, M >= 8: runs as qlinear_gemm (faster there).
+ * ExecuTorch page above, "Quant schema update" (the int4 / int6 formats)
+ * and the review's "Things done well" (the decode kernel's per-super-block
+ * step word and full-warp trip counts).
  * `workspace`: at least qlinear_gemv_workspace_bytes(), 256-byte aligned,
  * caller-owned, overwritten; calls sharing one workspace must not overlap on
- * the GPU.
+ * the GPU.  Consecutive int4 calls on one stream chain by programmatic
+ * dependent launch: a call's weight stream may start while the previous
+ * kernel on the stream drains, and its preparation pass waits for that
+ * kernel before it reads x or writes the workspace.
  * Errors: QL_ERR_NULL, QL_ERR_SHAPE (also: workspace too small),
  * QL_ERR_ALIGN, QL_ERR_RANGE, QL_ERR_UNSUPPORTED, QL_ERR_CUDA. */
 ql_status qlinear_gemv(const ql_desc *desc, const ql_packed_const *w,
@@ -211,11 +221,12 @@ ql_status qlinear_gemm_workspace_bytes(const ql_desc *desc, int64_t M, size_t *b
  * the row's max |x| in [2^15, 2^16) and stored as fp16 in the workspace
  * (exact for every value within 2^29 of the row maximum); (2) each weight
  * row gets a power of two 2^b_n from a metadata bound on its max |w|;
- * (3) the persistent GEMM dequantises each weight once per tile to its exact
- * binary32 value, scales it by 2^b_n and rounds it once to fp16, contracts
- * with fp32 accumulation in tensor memory, and stores
- * RN_bf16(acc * 2^-a_m * 2^-b_n).  fp16 operands rather than bf16 keep the
- * weight rounding at ~0.1% of rms(y) instead of ~1%.
+ * (3) the persistent GEMM (tiles of 256 tokens x 128 weight rows) dequantises
+ * each weight once per tile into fp16 -- int4 as q * S' - Z * S' in packed
+ * halves with S' = S * 2^b_n, int6 / affine as the exact binary32 value times
+ * 2^b_n rounded once -- contracts with fp32 accumulation in tensor memory,
+ * and stores RN_bf16(acc * 2^-a_m * 2^-b_n).  fp16 operands rather than
+ * bf16 keep the weight rounding at ~0.1% of rms(y) instead of ~1%.
  * `workspace`: device memory of at least qlinear_gemm_workspace_bytes(),
  * 256-byte aligned, owned by the caller, overwritten; calls sharing one
  * workspace must not overlap on the GPU.  K % 64 == 0.  Requires an sm_100

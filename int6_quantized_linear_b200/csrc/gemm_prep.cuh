@@ -106,46 +106,49 @@ __global__ void __launch_bounds__(256) x_to_f16_kernel(const __nv_bfloat16 *x, i
   if (lane == 0) ws.xinv[m] = exp2i(-a);
 }
 
-// One thread per weight row: bound max|w| from the metadata, pick b_n.
+// One warp per weight row: bound max|w| from the metadata (lanes stride over the groups, then a
+// max-reduction), pick b_n.
 template <int FMT, int BITS>
 __global__ void __launch_bounds__(256) w_scale_kernel(const uint8_t *gmeta, const uint8_t *steps, int64_t N,
                                                        int64_t K, int G, GemmWorkspace ws) {
-  const int64_t n = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-  if (n >= N) return;
+  const int lane = threadIdx.x & 31;
+  const int64_t n = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+  if (n >= N) return;  // whole warps leave together
   float bound = 0.f;
   if constexpr (FMT == FMT_INT4) {
     const uint16_t *gm = reinterpret_cast<const uint16_t *>(gmeta) + n * (K / 32);
     const uint32_t *st = reinterpret_cast<const uint32_t *>(steps) + n * (K / 256);
-    for (int64_t j = 0; j < K / 256; ++j) {
-      const uint32_t s = __ldg(st + j);
+    for (int64_t g = lane; g < K / 32; g += 32) {
+      const uint32_t s = __ldg(st + (g >> 3));
       const float ss = f16_bits_to_f32(s), zs = f16_bits_to_f32(s >> 16);
-      for (int g = 0; g < 8; ++g) {
-        const uint32_t c = __ldg(gm + 8 * j + g);
-        const float S = __fmul_rn((float)(c & 0xffu), ss);
-        const float Z = __fmul_rn((float)(c >> 8), zs);
-        bound = fmaxf(bound, __fmul_rn(fabsf(S), fmaxf(fabsf(Z), fabsf(__fsub_rn(15.f, Z)))));
-      }
+      const uint32_t c = __ldg(gm + g);
+      const float S = __fmul_rn((float)(c & 0xffu), ss);
+      const float Z = __fmul_rn((float)(c >> 8), zs);
+      bound = fmaxf(bound, __fmul_rn(fabsf(S), fmaxf(fabsf(Z), fabsf(__fsub_rn(15.f, Z)))));
     }
   } else if constexpr (FMT == FMT_INT6) {
     const int8_t *gm = reinterpret_cast<const int8_t *>(gmeta) + n * (K / 16);
     const uint16_t *st = reinterpret_cast<const uint16_t *>(steps) + n * (K / 256);
-    for (int64_t j = 0; j < K / 256; ++j) {
-      const float step = f16_bits_to_f32(__ldg(st + j));
-      for (int g = 0; g < 16; ++g)
-        bound = fmaxf(bound, __fmul_rn(32.f, fabsf(__fmul_rn((float)__ldg(gm + 16 * j + g), step))));
+    for (int64_t g = lane; g < K / 16; g += 32) {
+      const float step = f16_bits_to_f32(__ldg(st + (g >> 4)));
+      bound = fmaxf(bound, __fmul_rn(32.f, fabsf(__fmul_rn((float)__ldg(gm + g), step))));
     }
   } else {
     const uint32_t *gm = reinterpret_cast<const uint32_t *>(gmeta) + n * (K / G);
     const float qmax = (float)((1 << BITS) - 1);
-    for (int64_t g = 0; g < K / G; ++g) {
+    for (int64_t g = lane; g < K / G; g += 32) {
       const uint32_t c = __ldg(gm + g);
       const float s = bf16_bits_to_f32(c), b = bf16_bits_to_f32(c >> 16);
       bound = fmaxf(bound, fmaxf(fabsf(b), fabsf(__fadd_rn(__fmul_rn(qmax, s), b))));
     }
   }
-  const int e = scale_exponent(bound, 14);
-  ws.wsc[n] = exp2i(e);
-  ws.winv[n] = exp2i(-e);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) bound = fmaxf(bound, __shfl_xor_sync(0xffffffffu, bound, o));
+  if (lane == 0) {
+    const int e = scale_exponent(bound, 14);
+    ws.wsc[n] = exp2i(e);
+    ws.winv[n] = exp2i(-e);
+  }
 }
 
 }  // namespace ql

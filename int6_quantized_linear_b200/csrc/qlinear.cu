@@ -133,7 +133,7 @@ ql_status launch_gemm(const ql_desc *d, const ql_packed_const *w, const void *x,
   const GemmWorkspace ws = gemm_workspace_carve(workspace, M, N, K);
   // pass 1: scaled fp16 activations; pass 2: per-row weight scales
   x_to_f16_kernel<<<(int)((M * 32 + 255) / 256), 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(x), M, K, ws);
-  w_scale_kernel<FMT, BITS><<<(int)((N + 255) / 256), 256, 0, st>>>(
+  w_scale_kernel<FMT, BITS><<<(int)((N * 32 + 255) / 256), 256, 0, st>>>(
       static_cast<const uint8_t *>(w->gmeta), static_cast<const uint8_t *>(w->steps), N, K, d->group, ws);
   CUtensorMap mx, mc;
   if (!encode_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws.x16, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, BK, BM,
@@ -164,11 +164,28 @@ ql_status launch_gemm(const ql_desc *d, const ql_packed_const *w, const void *x,
   return launched();
 }
 
+// int6 and affine GEMV calls with M >= 8 tokens run on the tensor-core GEMM (measured faster there:
+// affine M=32 70-74 us vs 537-551 us, int6 M=8 198 us vs 284 us on the benchmark layers); int4 has
+// its own tensor-core GEMV up to M = 8.
+inline bool gemv_runs_on_gemm(const ql_desc *d, int64_t M) { return d->fmt != QL_INT4_NSS && M >= 8; }
+
+inline size_t gemv_call_workspace_bytes(const ql_desc *d, int64_t M) {
+  const size_t own = gemv_workspace_bytes(M, d->N, d->K);
+  if (!gemv_runs_on_gemm(d, M)) return own;
+  const size_t gemm = gemm_workspace_bytes(M, d->N, d->K);
+  return own > gemm ? own : gemm;
+}
+
+template <int FMT, int BITS>
+ql_status launch_gemm(const ql_desc *d, const ql_packed_const *w, const void *x, int64_t M, void *y,
+                      void *workspace, cudaStream_t st, int sms);
+
 template <int FMT, int BITS>
 ql_status launch_gemv(const ql_desc *d, const ql_packed_const *w, const void *x, int64_t M, void *y,
                       void *workspace, cudaStream_t st, int sms) {
   const auto *xb = static_cast<const __nv_bfloat16 *>(x);
   auto *yb = static_cast<__nv_bfloat16 *>(y);
+  if (gemv_runs_on_gemm(d, M)) return launch_gemm<FMT, BITS>(d, w, x, M, y, workspace, st, sms);
   if constexpr (FMT == FMT_INT4) {
     if (M == 1) {  // tensor-core path: preparation pass, then the streaming kernel as its dependent
       const GemvWorkspace ws = gemv_workspace_carve(workspace, M, d->K);
@@ -467,7 +484,7 @@ ql_status qlinear_gemv_workspace_bytes(const ql_desc *d, int64_t M, size_t *byte
   if (!bytes) return QL_ERR_NULL;
   const int64_t mmax = d->fmt == QL_AFFINE_U32 ? 32 : 8;
   if (M < 1 || M > mmax) return QL_ERR_RANGE;
-  *bytes = gemv_workspace_bytes(M, d->N, d->K);
+  *bytes = gemv_call_workspace_bytes(d, M);
   return QL_OK;
 }
 
@@ -480,7 +497,7 @@ ql_status qlinear_gemv(const ql_desc *d, const ql_packed_const *w, const void *x
   if (!aligned16(x) || !aligned16(y) || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return QL_ERR_ALIGN;
   const int64_t mmax = d->fmt == QL_AFFINE_U32 ? 32 : 8;
   if (M < 1 || M > mmax) return QL_ERR_RANGE;
-  if (workspace_bytes < gemv_workspace_bytes(M, d->N, d->K)) return QL_ERR_SHAPE;
+  if (workspace_bytes < gemv_call_workspace_bytes(d, M)) return QL_ERR_SHAPE;
   DeviceInfo *di;
   if ((st = device_info(&di)) != QL_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
