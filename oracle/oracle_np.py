@@ -10,6 +10,9 @@ Sources, cited by page title and section:
   [NSS] ExecuTorch PR "[cuda] Nestest Superscale Quantization for CUDA Weights
         (int4 / int6)", section "Quant schema update".
   [MTL] Hugging Face Transformers docs, "Metal" quantization page.
+  [REV] the same ExecuTorch PR, the review ("PR Review: Superscale
+        Quantization for CUDA Weights"), "Correctness" note 1 and "Things
+        done well" (encode/decode agreement); "Ablation study" (SNR).
 """
 from __future__ import annotations
 
@@ -131,3 +134,57 @@ def matmul_f64(x_bf16, w):
     """y = x . w^T with x given as bf16 bit patterns, in binary64."""
     x = f32_from_bf16_bits(x_bf16).astype(np.float64)
     return x @ np.asarray(w, np.float32).astype(np.float64).T
+
+
+# ---- metadata encoder ([NSS] "Quant schema update"; [REV] "Correctness" 1) ----------
+# Per 256-weight super-block, each per-group float field becomes a code times one fp16 step.
+
+def encode_u8_per_super(v, groups_per_super: int):
+    """int4 scale or zero field -> (u8 codes [N][G], fp16 step bits [N][G/groups_per_super]).
+
+    Steps, as the review describes the encoder: block_max = the super-block's max (a max, not an
+    absmax; the field must be non-negative, checked here), step = fp16(block_max / 255) with the
+    division in float32, code = clamp(round_half_even(v / step_f), 0, 255) where step_f is the
+    fp16-rounded step (so encoder and decoder reconstruct with the same step).  A super-block
+    whose max is 0 gets step 0 and codes 0 (the pages do not say; the plainest reading)."""
+    v = np.asarray(v, np.float32)
+    if not np.isfinite(v).all() or (v < 0).any():
+        raise ValueError("int4 metadata fields must be finite and non-negative")
+    N, G = v.shape
+    vb = v.reshape(N, G // groups_per_super, groups_per_super)
+    block_max = vb.max(axis=2)
+    step16 = (block_max / f32(255)).astype(np.float16)
+    step_f = step16.astype(np.float32)[..., None]
+    with np.errstate(divide="ignore", invalid="ignore"):
+        q = np.rint(vb / step_f)
+    q = np.where(step_f > 0, q, 0)
+    codes = np.clip(q, 0, 255).astype(np.uint8)
+    return codes.reshape(N, G), step16.view(np.uint16)
+
+
+def encode_i8_per_super(v, groups_per_super: int):
+    """int6 scale field -> (i8 codes [N][G], fp16 step bits [N][G/groups_per_super]).
+
+    The pages give no int6 encoder; the symmetric counterpart of the int4 one is taken:
+    step = fp16(max|v| / 127), code = clamp(round_half_even(v / step_f), -127, 127)."""
+    v = np.asarray(v, np.float32)
+    if not np.isfinite(v).all():
+        raise ValueError("int6 scale field must be finite")
+    N, G = v.shape
+    vb = v.reshape(N, G // groups_per_super, groups_per_super)
+    block_max = np.abs(vb).max(axis=2)
+    step16 = (block_max / f32(127)).astype(np.float16)
+    step_f = step16.astype(np.float32)[..., None]
+    with np.errstate(divide="ignore", invalid="ignore"):
+        q = np.rint(vb / step_f)
+    q = np.where(step_f > 0, q, 0)
+    codes = np.clip(q, -127, 127).astype(np.int8)
+    return codes.reshape(N, G), step16.view(np.uint16)
+
+
+def snr_db(w, w_hat) -> float:
+    """Whole-tensor signal-to-noise ratio in dB, 10 log10(sum w^2 / sum (w - w_hat)^2), as the
+    ablation study reports it (formula not printed there; the standard definition)."""
+    w = np.asarray(w, np.float64)
+    e = w - np.asarray(w_hat, np.float64)
+    return float(10.0 * np.log10((w * w).sum() / (e * e).sum()))

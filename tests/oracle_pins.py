@@ -276,3 +276,102 @@ def pin_matmul(impl):
     xa = x.copy(); xa[:, K // 2:] = 0
     xb = x.copy(); xb[:, :K // 2] = 0
     assert np.allclose(impl.matmul_f64(xa, w) + impl.matmul_f64(xb, w), y, rtol=1e-12, atol=1e-12)
+
+
+# ---- metadata encoder ([NSS] 'Quant schema update'; [REV] 'Correctness' 1, 'Things done well') --
+
+def fr_round_f32(fr: Fraction) -> Fraction:
+    """Nearest-even binary32 of an exact positive rational in the normal range, computed exactly."""
+    assert fr > 0
+    e = fr.numerator.bit_length() - fr.denominator.bit_length()
+    while Fraction(2) ** e > fr:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= fr:
+        e += 1
+    assert -126 <= e <= 127, "outside the binary32 normal range"
+    ulp = Fraction(2) ** (e - 23)
+    m = fr / ulp  # in [2^23, 2^24)
+    lo = m.numerator // m.denominator
+    rem = m - lo
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and lo % 2 == 1):
+        lo += 1
+    return lo * ulp
+
+
+def fr_round_f16_bits(fr: Fraction) -> int:
+    """Binary16 bit pattern nearest (ties to even) to a value that binary64 holds exactly."""
+    d = float(fr)
+    assert Fraction(d) == fr
+    return struct.unpack("<H", struct.pack("<e", d))[0]
+
+
+def _encode_expected(v: np.ndarray, per: int, top: int, signed: bool):
+    """Codes and step bits of one field, derived with exact rationals from the encoder's definition."""
+    N, G = v.shape
+    codes = np.zeros((N, G), np.int64)
+    steps = np.zeros((N, G // per), np.int64)
+    for r in range(N):
+        for b in range(G // per):
+            block = [Fraction(float(x)) for x in v[r, b * per:(b + 1) * per]]
+            m = max(abs(x) for x in block) if signed else max(block)
+            step_bits = fr_round_f16_bits(fr_round_f32(m / top)) if m > 0 else 0
+            steps[r, b] = step_bits
+            sf = fr_f16(step_bits)
+            for i, x in enumerate(block):
+                if sf == 0 or x == 0:
+                    c = 0
+                else:
+                    qv = fr_round_f32(abs(x) / sf) * (1 if x > 0 else -1)
+                    c = round(qv)  # Fraction rounds half to even
+                codes[r, b * per + i] = max(-top, min(top, c)) if signed else max(0, min(255, c))
+    return codes, steps
+
+
+def pin_encoder_golden(impl):
+    g = golden("meta_encoder_worked_example.json")
+    codes, steps = impl.encode_u8_per_super(np.array([g["values"]], np.float32), 8)
+    assert codes.ravel().tolist() == g["codes"], codes
+    assert int(steps[0, 0]) == g["step_bits"], hex(int(steps[0, 0]))
+
+
+def pin_encoder_exact(impl, seed=31):
+    rng = np.random.default_rng(seed)
+    # int4 fields: scales ~ 1e-4..1e-2 and zero points 0..15 (code units), 4 super-blocks per row,
+    # one all-zero super-block
+    sc = rng.uniform(1e-4, 1e-2, (3, 32)).astype(np.float32)
+    zp = (rng.uniform(0, 15, (3, 32)) * (rng.random((3, 32)) > 0.1)).astype(np.float32)
+    zp[1, 8:16] = 0.0
+    for v in (sc, zp):
+        c, s = impl.encode_u8_per_super(v, 8)
+        ce, se = _encode_expected(v, 8, 255, False)
+        assert np.array_equal(np.asarray(c, np.int64), ce)
+        assert np.array_equal(np.asarray(s, np.int64), se)
+    # int6 field: signed scales, 16 groups per super-block
+    s6 = (rng.uniform(1e-4, 1e-2, (2, 32)) * rng.choice([-1, 1], (2, 32))).astype(np.float32)
+    c, s = impl.encode_i8_per_super(s6, 16)
+    ce, se = _encode_expected(s6, 16, 127, True)
+    assert np.array_equal(np.asarray(c, np.int64), ce)
+    assert np.array_equal(np.asarray(s, np.int64), se)
+
+
+def pin_encoder_agreement(impl, seed=32):
+    """Encode/decode agreement: every value lies within half a step (plus the binary32 rounding of
+    the quotient) of code * step_f, the block max encodes to 254 or 255, and int6 codes are odd in v."""
+    rng = np.random.default_rng(seed)
+    v = rng.uniform(0, 3, (4, 64)).astype(np.float32)
+    c, s = impl.encode_u8_per_super(v, 8)
+    sf = np.repeat(np.asarray(s, np.uint16).view(np.float16).astype(np.float64), 8, 1)
+    err = np.abs(v.astype(np.float64) - np.asarray(c, np.float64) * sf)
+    assert np.all(err <= sf * (0.5 + 2.0 ** -15)), err.max()
+    vb = v.reshape(4, 8, 8)
+    cb = np.asarray(c).reshape(4, 8, 8)
+    assert np.all(cb[np.arange(4)[:, None], np.arange(8)[None, :], vb.argmax(2)] >= 254)
+    c6, _ = impl.encode_i8_per_super(v - 1.5, 16)
+    c6n, _ = impl.encode_i8_per_super(-(v - 1.5), 16)
+    assert np.array_equal(np.asarray(c6, np.int64), -np.asarray(c6n, np.int64))
+
+
+def pin_snr(impl):
+    w = np.ones(1000)
+    assert abs(impl.snr_db(w, 0.9 * w) - 20.0) < 1e-9  # 10 log10(1 / 0.01)
+    assert abs(impl.snr_db(w, w + 1e-3) - 60.0) < 1e-6
