@@ -476,6 +476,29 @@ def run_other_configs(device, peaks):
             del g
         out[name] = res
         del reps
+    # metadata encoder on the int4 decode layer's metadata: float scale and zero per group -> codes + steps
+    wl = synth.WORKLOADS["int4_gemv_k5120_n27648"]
+    G = wl.K // 32
+    gen = torch.Generator(device=device).manual_seed(wl.seed)
+    scale = torch.rand((wl.N, G), generator=gen, device=device) * 1e-2 + 1e-4
+    zero = torch.rand((wl.N, G), generator=gen, device=device) * 15
+    sc, zc = (torch.empty((wl.N, G), dtype=torch.uint8, device=device) for _ in range(2))
+    ss, zs = (torch.empty((wl.N, G // 8), dtype=torch.int16, device=device) for _ in range(2))
+    de = ql.Desc("int4", wl.N, wl.K)
+    calls = 20
+    g = capture(lambda: [ql.qlinear_quantize_meta(de, scale, zero, sc, zc, ss, zs) for _ in range(calls)], device)
+    g.replay()
+    torch.cuda.synchronize(device)
+    a, b = _ev(), _ev()
+    a.record()
+    g.replay()
+    b.record()
+    torch.cuda.synchronize(device)
+    us = a.elapsed_time(b) * 1e3 / calls
+    nbytes = 2 * wl.N * G * 4 + 2 * wl.N * G + 2 * wl.N * (G // 8) * 2
+    out["metadata_encoder_int4_k5120_n27648"] = {"us": round(us, 3), "GB/s": round(nbytes / us / 1e3, 1),
+                                                 "frac_hbm": round(nbytes / us / 1e3 / peaks["hbm_gbs"], 4)}
+    del g, scale, zero, sc, zc, ss, zs
     wl = synth.WORKLOADS["int4_gemm_k5120_n27648"]
     d, (c, g_, s), _ = packed_layer(wl, device)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)

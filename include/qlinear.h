@@ -78,7 +78,8 @@ typedef enum {
   QL_ERR_NULL = 1,        /* a required pointer is NULL                          */
   QL_ERR_SHAPE = 2,       /* N, K, M, bits or group not allowed for the format   */
   QL_ERR_ALIGN = 3,       /* a pointer is not 16-byte aligned                    */
-  QL_ERR_RANGE = 4,       /* M outside the range of the entry point              */
+  QL_ERR_RANGE = 4,       /* M outside the range of the entry point, or (from    */
+                          /* qlinear_sync_status) an encoder input out of domain */
   QL_ERR_UNSUPPORTED = 5, /* unknown format, or the device is not sm_100         */
   QL_ERR_CUDA = 6,        /* a CUDA runtime call or launch failed                */
   QL_ERR_TIMEOUT = 7      /* a device-side bounded wait gave up                  */
@@ -168,6 +169,31 @@ ql_status qlinear_unpack(const ql_desc *desc, const ql_packed_const *in,
  * Errors: as qlinear_pack, plus QL_ERR_SHAPE for an unknown out_dtype. */
 ql_status qlinear_dequant(const ql_desc *desc, const ql_packed_const *w,
                           void *out, int32_t out_dtype, ql_stream_t stream);
+
+/* Metadata encoder: float per-group metadata -> the codes and per-256 fp16
+ * steps that qlinear_pack takes (ExecuTorch PR above, "Quant schema update";
+ * its review, "Correctness" note 1 and "Things done well").  One field at a
+ * time, per 256-weight super-block of a row:
+ *   int4: scale and zero, float32 [N][K/32] each, finite and >= 0 (zero in
+ *         code units: w = (q - zero) * scale):
+ *         step = RN_fp16(block max / 255)  (binary32 division, then fp16),
+ *         code = clamp(round_half_even(v / f32(step)), 0, 255)  -> u8;
+ *         out->meta0 = sc [N][K/32], out->meta1 = zc, out->step0 = ss
+ *         [N][K/256] fp16 bits, out->step1 = zs.
+ *   int6: scale float32 [N][K/16], finite, either sign; `zero` unused:
+ *         step = RN_fp16(block max|v| / 127),
+ *         code = clamp(round_half_even(v / f32(step)), -127, 127) -> i8;
+ *         out->meta0 = sc [N][K/16], out->step0 = st [N][K/256].
+ * Codes are rounded against the fp16-rounded step, so qlinear_pack +
+ * qlinear_dequant reconstruct code * step exactly as the encoder saw it.  A
+ * super-block whose max is 0 gets step 0 and codes 0.  A negative (int4) or
+ * non-finite input is not rejected on the host (it is device data): the
+ * kernel records it and the next qlinear_sync_status returns QL_ERR_RANGE.
+ * Device pointers, caller-owned, 16-byte aligned.  affine: QL_ERR_UNSUPPORTED.
+ * Errors: QL_ERR_NULL, QL_ERR_SHAPE, QL_ERR_ALIGN, QL_ERR_UNSUPPORTED,
+ * QL_ERR_CUDA. */
+ql_status qlinear_quantize_meta(const ql_desc *desc, const float *scale, const float *zero,
+                                const ql_unpacked_out *out, ql_stream_t stream);
 
 /* Bytes of caller-provided device workspace qlinear_gemv needs for `desc`
  * and M (host-only, no CUDA call): 4*M*K for x in the order the tensor-core

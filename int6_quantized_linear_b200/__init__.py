@@ -66,6 +66,8 @@ _SIGNATURES = {
     "qlinear_gemm_noalloc": ([C.POINTER(ql_desc), C.POINTER(ql_packed), C.c_void_p, C.c_int64, C.c_void_p,
                               C.c_void_p], C.c_int),
     "qlinear_sync_status": ([C.c_void_p], C.c_int),
+    "qlinear_quantize_meta": ([C.POINTER(ql_desc), C.c_void_p, C.c_void_p, C.POINTER(ql_unpacked), C.c_void_p],
+                              C.c_int),
 }
 
 
@@ -156,6 +158,17 @@ def qlinear_dequant(desc: Desc, codes, gmeta, steps, out, out_dtype: int, stream
     w = ql_packed(_ptr(codes), _ptr(gmeta), _ptr(steps))
     _check(lib().qlinear_dequant(C.byref(d), C.byref(w), _ptr(out), out_dtype, _stream(stream)),
            "qlinear_dequant")
+
+
+def qlinear_quantize_meta(desc: Desc, scale, zero, meta0, meta1, step0, step1, stream=None):
+    """Float per-group metadata (float32 CUDA tensors) -> codes and fp16 step bits in the given
+    output tensors (int4: sc, zc u8 [N][K/32], ss, zs [N][K/256] 16-bit; int6: sc i8 [N][K/16],
+    st [N][K/256]; pass None for the unused ones).  Out-of-domain inputs show up as QL_ERR_RANGE
+    from qlinear_sync_status()."""
+    d = desc.c()
+    o = ql_unpacked(None, _ptr(meta0), _ptr(meta1), _ptr(step0), _ptr(step1))
+    _check(lib().qlinear_quantize_meta(C.byref(d), _ptr(scale), _ptr(zero), C.byref(o), _stream(stream)),
+           "qlinear_quantize_meta")
 
 
 def qlinear_gemv_workspace_bytes(desc: Desc, M: int) -> int:

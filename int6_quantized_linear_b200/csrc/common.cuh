@@ -19,6 +19,7 @@
 // ---------------------------------------------------------------------------
 __device__ unsigned int g_ql_status;
 #define QL_DEV_TIMEOUT 1u
+#define QL_DEV_RANGE 2u  // an input outside the domain of the operation (reported as QL_ERR_RANGE)
 
 // ~1 s at the B200's 1.9 GHz SM clock: far longer than any legitimate wait.
 #define QL_WAIT_LIMIT_CYCLES 2000000000LL

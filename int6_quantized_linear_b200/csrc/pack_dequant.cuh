@@ -296,4 +296,38 @@ __global__ void __launch_bounds__(256) dequant_kernel(WeightPtrs p, int64_t N, v
   }
 }
 
+
+// Metadata encoder (the int4 / int6 metadata of the ExecuTorch PR "[cuda] Nestest Superscale
+// Quantization for CUDA Weights", "Quant schema update"; its review, "Correctness" note 1 and
+// "Things done well"): one thread per (row, super-block) of one per-group float field.
+// int4 (SIGNED false): step = fp16(max / 255), code = clamp(rint(v / step_f), 0, 255);
+// int6 (SIGNED true):  step = fp16(max|v| / 127), code = clamp(rint(v / step_f), -127, 127);
+// step_f is the fp16-rounded step, so encoder and decoder reconstruct with the same value; the
+// divisions are IEEE binary32, rint rounds half to even, a zero max gives step 0 and codes 0.
+// A non-finite value (or a negative one for int4) sets QL_DEV_RANGE.
+template <bool SIGNED>
+__global__ void __launch_bounds__(256) quantize_meta_kernel(const float *v, int64_t rows, int64_t G, int per,
+                                                            uint8_t *codes, uint16_t *steps) {
+  const int64_t S = G / per;
+  const int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (t >= rows * S) return;
+  const int64_t r = t / S, b = t - r * S;
+  const float *src = v + r * G + b * per;
+  float m = 0.f;
+  bool bad = false;
+  for (int i = 0; i < per; ++i) {
+    const float x = src[i];
+    bad |= !isfinite(x) || (!SIGNED && x < 0.f);
+    m = fmaxf(m, SIGNED ? fabsf(x) : x);
+  }
+  if (bad) atomicOr(&g_ql_status, QL_DEV_RANGE);
+  const __half st = __float2half_rn(__fdiv_rn(m, SIGNED ? 127.f : 255.f));
+  const float sf = __half2float(st);
+  const float lo = SIGNED ? -127.f : 0.f, hi = SIGNED ? 127.f : 255.f;
+  for (int i = 0; i < per; ++i) {
+    const float q = sf > 0.f ? fminf(hi, fmaxf(lo, rintf(__fdiv_rn(src[i], sf)))) : 0.f;
+    codes[r * G + b * per + i] = SIGNED ? (uint8_t)(int8_t)(int)q : (uint8_t)(int)q;
+  }
+  steps[r * S + b] = __half_as_ushort(st);
+}
 }  // namespace ql

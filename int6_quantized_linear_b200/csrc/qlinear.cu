@@ -570,12 +570,42 @@ ql_status qlinear_gemm_noalloc(const ql_desc *d, const ql_packed_const *w, const
   }
 }
 
+ql_status qlinear_quantize_meta(const ql_desc *d, const float *scale, const float *zero, const ql_unpacked_out *out,
+                                ql_stream_t stream) {
+  ql_status st = check_desc(d);
+  if (st != QL_OK) return st;
+  if (d->fmt == QL_AFFINE_U32) return QL_ERR_UNSUPPORTED;
+  const bool i4 = d->fmt == QL_INT4_NSS;
+  if (!scale || !out || !out->meta0 || !out->step0) return QL_ERR_NULL;
+  if (i4 && (!zero || !out->meta1 || !out->step1)) return QL_ERR_NULL;
+  if (!aligned16(scale) || !aligned16(out->meta0) || !aligned16(out->step0)) return QL_ERR_ALIGN;
+  if (i4 && (!aligned16(zero) || !aligned16(out->meta1) || !aligned16(out->step1))) return QL_ERR_ALIGN;
+  DeviceInfo *di;
+  if ((st = device_info(&di)) != QL_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t N = d->N, K = d->K;
+  const int per = i4 ? 8 : 16;                  // groups per 256-weight super-block
+  const int64_t G = K / (i4 ? 32 : 16);         // groups per row
+  const int64_t threads = N * (G / per);
+  const int blocks = (int)((threads + 255) / 256);
+  if (i4) {
+    quantize_meta_kernel<false><<<blocks, 256, 0, s>>>(scale, N, G, per, static_cast<uint8_t *>(out->meta0),
+                                                       static_cast<uint16_t *>(out->step0));
+    quantize_meta_kernel<false><<<blocks, 256, 0, s>>>(zero, N, G, per, static_cast<uint8_t *>(out->meta1),
+                                                       static_cast<uint16_t *>(out->step1));
+  } else {
+    quantize_meta_kernel<true><<<blocks, 256, 0, s>>>(scale, N, G, per, static_cast<uint8_t *>(out->meta0),
+                                                      static_cast<uint16_t *>(out->step0));
+  }
+  return launched();
+}
+
 ql_status qlinear_sync_status(ql_stream_t stream) {
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return QL_ERR_CUDA;
   unsigned int v = 0, zero = 0;
   if (cudaMemcpyFromSymbol(&v, g_ql_status, sizeof v) != cudaSuccess) return QL_ERR_CUDA;
   if (v != 0 && cudaMemcpyToSymbol(g_ql_status, &zero, sizeof zero) != cudaSuccess) return QL_ERR_CUDA;
-  return (v & QL_DEV_TIMEOUT) ? QL_ERR_TIMEOUT : QL_OK;
+  return (v & QL_DEV_TIMEOUT) ? QL_ERR_TIMEOUT : (v & QL_DEV_RANGE) ? QL_ERR_RANGE : QL_OK;
 }
 
 }  // extern "C"
