@@ -476,6 +476,30 @@ def run_other_configs(device, peaks):
             del g
         out[name] = res
         del reps
+    # the int4 decode GEMV with a bias epilogue (M=1, first decode layer)
+    wl = synth.WORKLOADS["int4_gemv_k5120_n27648"]
+    d, p0, wbytes = packed_layer(wl, device)
+    reps = [p0] + [tuple(t.clone() for t in p0) for _ in range(2)]
+    x = torch.from_numpy(wl.x(1).view("int16")).to(device).view(torch.bfloat16)
+    y = torch.empty((1, wl.N), dtype=torch.bfloat16, device=device)
+    bias = torch.zeros(wl.N, dtype=torch.bfloat16, device=device)
+    ws = ql.alloc_gemv_workspace(d, 1, device)
+    for i in range(3):
+        ql.qlinear_gemv_bias(d, *reps[i], x, 1, bias, y, ws)
+    calls = 30
+    g = capture(lambda: [ql.qlinear_gemv_bias(d, *reps[i % 3], x, 1, bias, y, ws) for i in range(calls)], device)
+    g.replay()
+    torch.cuda.synchronize(device)
+    a, b = _ev(), _ev()
+    a.record()
+    g.replay()
+    b.record()
+    torch.cuda.synchronize(device)
+    us = a.elapsed_time(b) * 1e3 / calls
+    nbytes = wbytes + wl.K * 2 + wl.N * 4
+    out["int4_gemv_bias_k5120_n27648"] = {"M1": {"us": round(us, 3), "GB/s": round(nbytes / us / 1e3, 1),
+                                                 "frac_hbm": round(nbytes / us / 1e3 / peaks["hbm_gbs"], 4)}}
+    del g, reps
     # metadata encoder on the int4 decode layer's metadata: float scale and zero per group -> codes + steps
     wl = synth.WORKLOADS["int4_gemv_k5120_n27648"]
     G = wl.K // 32

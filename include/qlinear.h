@@ -234,6 +234,15 @@ ql_status qlinear_gemv(const ql_desc *desc, const ql_packed_const *w,
                        const void *x, int64_t M, void *y, void *workspace,
                        size_t workspace_bytes, ql_stream_t stream);
 
+/* qlinear_gemv plus a per-output-row bias: y[m][n] = RN_bf16(acc[m][n] +
+ * f32(bias[n])), the bias added in fp32 before the one rounding.  `bias`:
+ * bf16 [N] on the device, 16-byte aligned, not NULL.  Otherwise as
+ * qlinear_gemv (Metal backend notes on the ExecuTorch page: "linear with
+ * bias", "4-bit linear with bias").  Errors: as qlinear_gemv. */
+ql_status qlinear_gemv_bias(const ql_desc *desc, const ql_packed_const *w,
+                            const void *x, int64_t M, const void *bias, void *y,
+                            void *workspace, size_t workspace_bytes, ql_stream_t stream);
+
 /* Bytes of caller-provided device workspace qlinear_gemm needs for `desc`
  * and M (host-only, no CUDA call): 2*M*K for the fp16 copy of x, plus
  * 4*M + 8*ceil(N/256)*256 for the per-row scales, each part rounded up to
@@ -263,6 +272,26 @@ ql_status qlinear_gemm_workspace_bytes(const ql_desc *desc, int64_t M, size_t *b
 ql_status qlinear_gemm(const ql_desc *desc, const ql_packed_const *w,
                        const void *x, int64_t M, void *y, void *workspace,
                        size_t workspace_bytes, ql_stream_t stream);
+
+/* qlinear_gemm plus a per-output-row bias (bf16 [N], added in fp32 before
+ * the rounding to bf16), as qlinear_gemv_bias.  Errors: as qlinear_gemm. */
+ql_status qlinear_gemm_bias(const ql_desc *desc, const ql_packed_const *w,
+                            const void *x, int64_t M, const void *bias, void *y,
+                            void *workspace, size_t workspace_bytes, ql_stream_t stream);
+
+/* Two packed layers with the same format, bits, group and K, stacked along
+ * N (fused projections such as QKV or gate/up; the ExecuTorch PR's
+ * "_concat_coalesced_int4_along_n", review "Correctness" note 3): `out` is
+ * the packed layer with N = a.N + b.N whose rows are a's rows then b's.
+ * Every packed buffer is row-major per weight row with per-row metadata, so
+ * each output buffer is a's buffer followed by b's (six device-to-device
+ * copies on `stream`).  `out` buffers sized by qlinear_packed_bytes for the
+ * stacked desc, caller-owned, 16-byte aligned.
+ * Errors: QL_ERR_NULL, QL_ERR_SHAPE (formats or K differ), QL_ERR_ALIGN,
+ * QL_ERR_UNSUPPORTED, QL_ERR_CUDA. */
+ql_status qlinear_concat_n(const ql_desc *a, const ql_packed_const *wa,
+                           const ql_desc *b, const ql_packed_const *wb,
+                           const ql_packed *out, ql_stream_t stream);
 
 /* qlinear_gemm for callers that may not allocate device memory at all --
  * e.g. an op behind a runtime's plug-in interface, which receives its input

@@ -66,6 +66,12 @@ _SIGNATURES = {
     "qlinear_gemm_noalloc": ([C.POINTER(ql_desc), C.POINTER(ql_packed), C.c_void_p, C.c_int64, C.c_void_p,
                               C.c_void_p], C.c_int),
     "qlinear_sync_status": ([C.c_void_p], C.c_int),
+    "qlinear_gemv_bias": ([C.POINTER(ql_desc), C.POINTER(ql_packed), C.c_void_p, C.c_int64, C.c_void_p,
+                           C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p], C.c_int),
+    "qlinear_gemm_bias": ([C.POINTER(ql_desc), C.POINTER(ql_packed), C.c_void_p, C.c_int64, C.c_void_p,
+                           C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p], C.c_int),
+    "qlinear_concat_n": ([C.POINTER(ql_desc), C.POINTER(ql_packed), C.POINTER(ql_desc), C.POINTER(ql_packed),
+                          C.POINTER(ql_packed), C.c_void_p], C.c_int),
     "qlinear_quantize_meta": ([C.POINTER(ql_desc), C.c_void_p, C.c_void_p, C.POINTER(ql_unpacked), C.c_void_p],
                               C.c_int),
 }
@@ -194,6 +200,27 @@ def qlinear_gemv(desc: Desc, codes, gmeta, steps, x, M: int, y, workspace=None, 
                               workspace.numel() * workspace.element_size(), _stream(stream)), "qlinear_gemv")
 
 
+def qlinear_gemv_bias(desc: Desc, codes, gmeta, steps, x, M: int, bias, y, workspace=None, stream=None):
+    """qlinear_gemv with a bf16 [N] bias added before the rounding to bf16."""
+    if workspace is None:
+        workspace = alloc_gemv_workspace(desc, M, x.device)
+    d = desc.c()
+    w = ql_packed(_ptr(codes), _ptr(gmeta), _ptr(steps))
+    _check(lib().qlinear_gemv_bias(C.byref(d), C.byref(w), _ptr(x), M, _ptr(bias), _ptr(y), _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(), _stream(stream)),
+           "qlinear_gemv_bias")
+
+
+def qlinear_concat_n(desc_a: Desc, packed_a, desc_b: Desc, packed_b, out, stream=None):
+    """Stack two packed layers along N into ``out`` = (codes, gmeta, steps) of the stacked layer."""
+    da, db = desc_a.c(), desc_b.c()
+    wa = ql_packed(*[_ptr(t) for t in packed_a])
+    wb = ql_packed(*[_ptr(t) for t in packed_b])
+    o = ql_packed(*[_ptr(t) for t in out])
+    _check(lib().qlinear_concat_n(C.byref(da), C.byref(wa), C.byref(db), C.byref(wb), C.byref(o), _stream(stream)),
+           "qlinear_concat_n")
+
+
 def qlinear_gemm_workspace_bytes(desc: Desc, M: int) -> int:
     d = desc.c()
     n = C.c_size_t()
@@ -216,6 +243,17 @@ def qlinear_gemm(desc: Desc, codes, gmeta, steps, x, M: int, y, workspace=None, 
     w = ql_packed(_ptr(codes), _ptr(gmeta), _ptr(steps))
     _check(lib().qlinear_gemm(C.byref(d), C.byref(w), _ptr(x), M, _ptr(y), _ptr(workspace),
                               workspace.numel() * workspace.element_size(), _stream(stream)), "qlinear_gemm")
+
+
+def qlinear_gemm_bias(desc: Desc, codes, gmeta, steps, x, M: int, bias, y, workspace=None, stream=None):
+    """qlinear_gemm with a bf16 [N] bias added before the rounding to bf16."""
+    if workspace is None:
+        workspace = alloc_gemm_workspace(desc, M, x.device)
+    d = desc.c()
+    w = ql_packed(_ptr(codes), _ptr(gmeta), _ptr(steps))
+    _check(lib().qlinear_gemm_bias(C.byref(d), C.byref(w), _ptr(x), M, _ptr(bias), _ptr(y), _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(), _stream(stream)),
+           "qlinear_gemm_bias")
 
 
 def qlinear_gemm_noalloc(desc: Desc, codes, gmeta, steps, x, M: int, y, stream=None):

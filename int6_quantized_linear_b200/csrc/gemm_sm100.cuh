@@ -90,6 +90,7 @@ __host__ __device__ constexpr int smem_bytes(int fmt, int bits) { return smem_ne
 struct Params {
   int64_t M, N, K;
   int G;
+  const __nv_bfloat16 *bias;  // [N] or NULL: added in fp32 before the rounding to bf16
   const uint8_t *gmeta;
   const uint8_t *steps;
   __nv_bfloat16 *y;
@@ -362,6 +363,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               r[4 * t + 2] = __float_as_uint(__uint_as_float(r[4 * t + 2]) * xs * v.z);
               r[4 * t + 3] = __float_as_uint(__uint_as_float(r[4 * t + 3]) * xs * v.w);
             }
+          }
+          if (p.bias) {  // + bias[n], still in fp32
+#pragma unroll 4
+            for (int i = 0; i < 32; ++i)
+              if (n0 + i < p.N) r[i] = __float_as_uint(__uint_as_float(r[i]) + __bfloat162float(p.bias[n0 + i]));
           }
           if (m < p.M) {
             __nv_bfloat16 *dst = p.y + m * p.N + n0;

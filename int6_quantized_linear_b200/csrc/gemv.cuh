@@ -11,9 +11,12 @@
 
 namespace ql {
 
+// Optional per-output-row bias (bf16 [N], may be NULL), added in fp32 before the one rounding.
+QL_DEVI float bias_at(const __nv_bfloat16 *bias, int64_t n) { return bias ? __bfloat162float(bias[n]) : 0.f; }
+
 template <int FMT, int BITS, int MT>
 __global__ void __launch_bounds__(256) gemv_simple_kernel(WeightPtrs p, int64_t N, const __nv_bfloat16 *x,
-                                                          int M, __nv_bfloat16 *y) {
+                                                          int M, const __nv_bfloat16 *bias, __nv_bfloat16 *y) {
   const int lane = threadIdx.x & 31;
   const int64_t warp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
@@ -54,7 +57,7 @@ __global__ void __launch_bounds__(256) gemv_simple_kernel(WeightPtrs p, int64_t 
       if (lane == 0) {
 #pragma unroll
         for (int m = 0; m < MT; ++m)
-          if (m0 + m < M) y[(int64_t)(m0 + m) * N + n] = __float2bfloat16_rn(acc[m]);
+          if (m0 + m < M) y[(int64_t)(m0 + m) * N + n] = __float2bfloat16_rn(acc[m] + bias_at(bias, n));
       }
     }
   }
@@ -253,6 +256,7 @@ constexpr float GEMV_ACC0_F = 12582912.f;
 
 struct GemvTcParams {
   const uint8_t *steps;
+  const __nv_bfloat16 *bias;  // [N] or NULL
   int64_t N, K;
   int parts;  // warps splitting K for one tile (1, 2 or 4)
   GemvWorkspace ws;
@@ -453,7 +457,7 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS, GEMV_CTAS_PER_SM)
     float sum = 0.f;
     for (int q = 0; q < P; ++q) sum += red[(warp + q) * 16 + lane];
     const int64_t r = tile * 16 + lane;
-    if (r < p.N) p.y[r] = __float2bfloat16_rn(sum);
+    if (r < p.N) p.y[r] = __float2bfloat16_rn(sum + bias_at(p.bias, r));
   }
 }
 
@@ -536,6 +540,7 @@ constexpr int GEMV_MT_STAGE_BYTES = 14336;
 
 struct GemvMtParams {
   const uint8_t *steps;
+  const __nv_bfloat16 *bias;  // [N] or NULL
   int64_t N, K;
   int M;  // 2 .. 8 tokens
   int P;  // CTAs per 64-row group (K split)
@@ -700,12 +705,14 @@ __global__ void __launch_bounds__(GEMV_MT_THREADS, GEMV_MT_CTAS_PER_SM)
     if (ok) {
       if (P == 1) {
         if (n0 < p.N) {
-          if (tk0 < M) p.y[(int64_t)tk0 * p.N + n0] = __float2bfloat16_rn(acc[0]);
-          if (tk1 < M) p.y[(int64_t)tk1 * p.N + n0] = __float2bfloat16_rn(acc[1]);
+          const float b0 = bias_at(p.bias, n0);
+          if (tk0 < M) p.y[(int64_t)tk0 * p.N + n0] = __float2bfloat16_rn(acc[0] + b0);
+          if (tk1 < M) p.y[(int64_t)tk1 * p.N + n0] = __float2bfloat16_rn(acc[1] + b0);
         }
         if (n1 < p.N) {
-          if (tk0 < M) p.y[(int64_t)tk0 * p.N + n1] = __float2bfloat16_rn(acc[2]);
-          if (tk1 < M) p.y[(int64_t)tk1 * p.N + n1] = __float2bfloat16_rn(acc[3]);
+          const float b1 = bias_at(p.bias, n1);
+          if (tk0 < M) p.y[(int64_t)tk0 * p.N + n1] = __float2bfloat16_rn(acc[2] + b1);
+          if (tk1 < M) p.y[(int64_t)tk1 * p.N + n1] = __float2bfloat16_rn(acc[3] + b1);
         }
       } else {
         float *mine = p.ws.partial + (int64_t)blockIdx.x * M * 64;
@@ -733,7 +740,7 @@ __global__ void __launch_bounds__(GEMV_MT_THREADS, GEMV_MT_CTAS_PER_SM)
         float sum = 0.f;
         for (int q = 0; q < P; ++q) sum += __ldcg(base + (int64_t)q * M * 64 + e);
         const int64_t n = rg * 64 + r;
-        if (n < p.N) p.y[(int64_t)tk * p.N + n] = __float2bfloat16_rn(sum);
+        if (n < p.N) p.y[(int64_t)tk * p.N + n] = __float2bfloat16_rn(sum + bias_at(p.bias, n));
       }
     }
   }

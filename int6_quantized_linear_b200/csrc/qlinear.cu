@@ -125,8 +125,8 @@ bool encode_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint6
 }
 
 template <int FMT, int BITS>
-ql_status launch_gemm(const ql_desc *d, const ql_packed_const *w, const void *x, int64_t M, void *y,
-                      void *workspace, cudaStream_t st, int sms) {
+ql_status launch_gemm(const ql_desc *d, const ql_packed_const *w, const void *x, int64_t M, const void *bias,
+                      void *y, void *workspace, cudaStream_t st, int sms) {
   using namespace ql::gemm;
   const int64_t N = d->N, K = d->K;
   const uint64_t row_bytes = (uint64_t)K * code_bits(FMT, BITS) / 8;
@@ -144,6 +144,7 @@ ql_status launch_gemm(const ql_desc *d, const ql_packed_const *w, const void *x,
     return QL_ERR_CUDA;
   Params p;
   p.M = M; p.N = N; p.K = K; p.G = d->group;
+  p.bias = static_cast<const __nv_bfloat16 *>(bias);
   p.gmeta = static_cast<const uint8_t *>(w->gmeta);
   p.steps = static_cast<const uint8_t *>(w->steps);
   p.y = static_cast<__nv_bfloat16 *>(y);
@@ -177,15 +178,16 @@ inline size_t gemv_call_workspace_bytes(const ql_desc *d, int64_t M) {
 }
 
 template <int FMT, int BITS>
-ql_status launch_gemm(const ql_desc *d, const ql_packed_const *w, const void *x, int64_t M, void *y,
-                      void *workspace, cudaStream_t st, int sms);
+ql_status launch_gemm(const ql_desc *d, const ql_packed_const *w, const void *x, int64_t M, const void *bias,
+                      void *y, void *workspace, cudaStream_t st, int sms);
 
 template <int FMT, int BITS>
-ql_status launch_gemv(const ql_desc *d, const ql_packed_const *w, const void *x, int64_t M, void *y,
-                      void *workspace, cudaStream_t st, int sms) {
+ql_status launch_gemv(const ql_desc *d, const ql_packed_const *w, const void *x, int64_t M, const void *bias,
+                      void *y, void *workspace, cudaStream_t st, int sms) {
   const auto *xb = static_cast<const __nv_bfloat16 *>(x);
   auto *yb = static_cast<__nv_bfloat16 *>(y);
-  if (gemv_runs_on_gemm(d, M)) return launch_gemm<FMT, BITS>(d, w, x, M, y, workspace, st, sms);
+  const auto *bb = static_cast<const __nv_bfloat16 *>(bias);
+  if (gemv_runs_on_gemm(d, M)) return launch_gemm<FMT, BITS>(d, w, x, M, bias, y, workspace, st, sms);
   if constexpr (FMT == FMT_INT4) {
     if (M == 1) {  // tensor-core path: preparation pass, then the streaming kernel as its dependent
       const GemvWorkspace ws = gemv_workspace_carve(workspace, M, d->K);
@@ -204,6 +206,7 @@ ql_status launch_gemv(const ql_desc *d, const ql_packed_const *w, const void *x,
       }
       GemvTcParams p;
       p.steps = static_cast<const uint8_t *>(w->steps);
+      p.bias = bb;
       p.N = d->N;
       p.K = d->K;
       p.ws = ws;
@@ -262,6 +265,7 @@ ql_status launch_gemv(const ql_desc *d, const ql_packed_const *w, const void *x,
       }
       GemvMtParams p;
       p.steps = static_cast<const uint8_t *>(w->steps);
+      p.bias = bb;
       p.N = N;
       p.K = K;
       p.M = (int)M;
@@ -305,13 +309,13 @@ ql_status launch_gemv(const ql_desc *d, const ql_packed_const *w, const void *x,
   const int64_t cap = (int64_t)sms * 16;
   if (g > cap) g = cap;
   if (M == 1)
-    gemv_simple_kernel<FMT, BITS, 1><<<(int)g, 256, 0, st>>>(p, d->N, xb, (int)M, yb);
+    gemv_simple_kernel<FMT, BITS, 1><<<(int)g, 256, 0, st>>>(p, d->N, xb, (int)M, bb, yb);
   else if (M == 2)
-    gemv_simple_kernel<FMT, BITS, 2><<<(int)g, 256, 0, st>>>(p, d->N, xb, (int)M, yb);
+    gemv_simple_kernel<FMT, BITS, 2><<<(int)g, 256, 0, st>>>(p, d->N, xb, (int)M, bb, yb);
   else if (M <= 4)
-    gemv_simple_kernel<FMT, BITS, 4><<<(int)g, 256, 0, st>>>(p, d->N, xb, (int)M, yb);
+    gemv_simple_kernel<FMT, BITS, 4><<<(int)g, 256, 0, st>>>(p, d->N, xb, (int)M, bb, yb);
   else
-    gemv_simple_kernel<FMT, BITS, 8><<<(int)g, 256, 0, st>>>(p, d->N, xb, (int)M, yb);
+    gemv_simple_kernel<FMT, BITS, 8><<<(int)g, 256, 0, st>>>(p, d->N, xb, (int)M, bb, yb);
   return launched();
 }
 
@@ -488,13 +492,14 @@ ql_status qlinear_gemv_workspace_bytes(const ql_desc *d, int64_t M, size_t *byte
   return QL_OK;
 }
 
-ql_status qlinear_gemv(const ql_desc *d, const ql_packed_const *w, const void *x, int64_t M, void *y,
-                       void *workspace, size_t workspace_bytes, ql_stream_t stream) {
+static ql_status gemv_call(const ql_desc *d, const ql_packed_const *w, const void *x, int64_t M, const void *bias,
+                           void *y, void *workspace, size_t workspace_bytes, ql_stream_t stream) {
   ql_status st = check_desc(d);
   if (st != QL_OK) return st;
   if (!w || !x || !y || !workspace) return QL_ERR_NULL;
   if ((st = check_packed(d, w->codes, w->gmeta, w->steps)) != QL_OK) return st;
   if (!aligned16(x) || !aligned16(y) || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return QL_ERR_ALIGN;
+  if (bias && !aligned16(bias)) return QL_ERR_ALIGN;
   const int64_t mmax = d->fmt == QL_AFFINE_U32 ? 32 : 8;
   if (M < 1 || M > mmax) return QL_ERR_RANGE;
   if (workspace_bytes < gemv_call_workspace_bytes(d, M)) return QL_ERR_SHAPE;
@@ -502,13 +507,25 @@ ql_status qlinear_gemv(const ql_desc *d, const ql_packed_const *w, const void *x
   if ((st = device_info(&di)) != QL_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   switch (d->fmt) {
-    case QL_INT4_NSS: return launch_gemv<FMT_INT4, 4>(d, w, x, M, y, workspace, s, di->sms);
-    case QL_INT6_SYM: return launch_gemv<FMT_INT6, 6>(d, w, x, M, y, workspace, s, di->sms);
+    case QL_INT4_NSS: return launch_gemv<FMT_INT4, 4>(d, w, x, M, bias, y, workspace, s, di->sms);
+    case QL_INT6_SYM: return launch_gemv<FMT_INT6, 6>(d, w, x, M, bias, y, workspace, s, di->sms);
     default:
-      if (d->bits == 2) return launch_gemv<FMT_AFFINE, 2>(d, w, x, M, y, workspace, s, di->sms);
-      if (d->bits == 4) return launch_gemv<FMT_AFFINE, 4>(d, w, x, M, y, workspace, s, di->sms);
-      return launch_gemv<FMT_AFFINE, 8>(d, w, x, M, y, workspace, s, di->sms);
+      if (d->bits == 2) return launch_gemv<FMT_AFFINE, 2>(d, w, x, M, bias, y, workspace, s, di->sms);
+      if (d->bits == 4) return launch_gemv<FMT_AFFINE, 4>(d, w, x, M, bias, y, workspace, s, di->sms);
+      return launch_gemv<FMT_AFFINE, 8>(d, w, x, M, bias, y, workspace, s, di->sms);
   }
+}
+
+ql_status qlinear_gemv(const ql_desc *d, const ql_packed_const *w, const void *x, int64_t M, void *y,
+                       void *workspace, size_t workspace_bytes, ql_stream_t stream) {
+  return gemv_call(d, w, x, M, nullptr, y, workspace, workspace_bytes, stream);
+}
+
+ql_status qlinear_gemv_bias(const ql_desc *d, const ql_packed_const *w, const void *x, int64_t M,
+                            const void *bias, void *y, void *workspace, size_t workspace_bytes,
+                            ql_stream_t stream) {
+  if (!bias) return QL_ERR_NULL;
+  return gemv_call(d, w, x, M, bias, y, workspace, workspace_bytes, stream);
 }
 
 ql_status qlinear_gemm_workspace_bytes(const ql_desc *d, int64_t M, size_t *bytes) {
@@ -520,13 +537,14 @@ ql_status qlinear_gemm_workspace_bytes(const ql_desc *d, int64_t M, size_t *byte
   return QL_OK;
 }
 
-ql_status qlinear_gemm(const ql_desc *d, const ql_packed_const *w, const void *x, int64_t M, void *y,
-                       void *workspace, size_t workspace_bytes, ql_stream_t stream) {
+static ql_status gemm_call(const ql_desc *d, const ql_packed_const *w, const void *x, int64_t M, const void *bias,
+                           void *y, void *workspace, size_t workspace_bytes, ql_stream_t stream) {
   ql_status st = check_desc(d);
   if (st != QL_OK) return st;
   if (!w || !x || !y || !workspace) return QL_ERR_NULL;
   if ((st = check_packed(d, w->codes, w->gmeta, w->steps)) != QL_OK) return st;
   if (!aligned16(x) || !aligned16(y) || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return QL_ERR_ALIGN;
+  if (bias && !aligned16(bias)) return QL_ERR_ALIGN;
   if (M < 1 || M > (int64_t)INT32_MAX) return QL_ERR_RANGE;
   if (d->K % gemm::BK != 0 || d->N > (int64_t)INT32_MAX) return QL_ERR_SHAPE;
   if (workspace_bytes < gemm_workspace_bytes(M, d->N, d->K)) return QL_ERR_SHAPE;
@@ -535,13 +553,56 @@ ql_status qlinear_gemm(const ql_desc *d, const ql_packed_const *w, const void *x
   if (di->major != 10) return QL_ERR_UNSUPPORTED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   switch (d->fmt) {
-    case QL_INT4_NSS: return launch_gemm<FMT_INT4, 4>(d, w, x, M, y, workspace, s, di->sms);
-    case QL_INT6_SYM: return launch_gemm<FMT_INT6, 6>(d, w, x, M, y, workspace, s, di->sms);
+    case QL_INT4_NSS: return launch_gemm<FMT_INT4, 4>(d, w, x, M, bias, y, workspace, s, di->sms);
+    case QL_INT6_SYM: return launch_gemm<FMT_INT6, 6>(d, w, x, M, bias, y, workspace, s, di->sms);
     default:
-      if (d->bits == 2) return launch_gemm<FMT_AFFINE, 2>(d, w, x, M, y, workspace, s, di->sms);
-      if (d->bits == 4) return launch_gemm<FMT_AFFINE, 4>(d, w, x, M, y, workspace, s, di->sms);
-      return launch_gemm<FMT_AFFINE, 8>(d, w, x, M, y, workspace, s, di->sms);
+      if (d->bits == 2) return launch_gemm<FMT_AFFINE, 2>(d, w, x, M, bias, y, workspace, s, di->sms);
+      if (d->bits == 4) return launch_gemm<FMT_AFFINE, 4>(d, w, x, M, bias, y, workspace, s, di->sms);
+      return launch_gemm<FMT_AFFINE, 8>(d, w, x, M, bias, y, workspace, s, di->sms);
   }
+}
+
+ql_status qlinear_gemm(const ql_desc *d, const ql_packed_const *w, const void *x, int64_t M, void *y,
+                       void *workspace, size_t workspace_bytes, ql_stream_t stream) {
+  return gemm_call(d, w, x, M, nullptr, y, workspace, workspace_bytes, stream);
+}
+
+ql_status qlinear_gemm_bias(const ql_desc *d, const ql_packed_const *w, const void *x, int64_t M,
+                            const void *bias, void *y, void *workspace, size_t workspace_bytes,
+                            ql_stream_t stream) {
+  if (!bias) return QL_ERR_NULL;
+  return gemm_call(d, w, x, M, bias, y, workspace, workspace_bytes, stream);
+}
+
+// Two packed layers with the same format and K side by side along N: every packed buffer is
+// row-major per weight row with per-row metadata, so the result is each buffer of `a` followed by
+// the same buffer of `b` (six device-to-device copies on the stream).
+ql_status qlinear_concat_n(const ql_desc *da, const ql_packed_const *wa, const ql_desc *db,
+                           const ql_packed_const *wb, const ql_packed *out, ql_stream_t stream) {
+  ql_status st;
+  if (!da || !db || !wa || !wb || !out) return QL_ERR_NULL;
+  if ((st = check_desc(da)) != QL_OK || (st = check_desc(db)) != QL_OK) return st;
+  if (da->fmt != db->fmt || da->bits != db->bits || da->group != db->group || da->K != db->K) return QL_ERR_SHAPE;
+  if ((st = check_packed(da, wa->codes, wa->gmeta, wa->steps)) != QL_OK) return st;
+  if ((st = check_packed(db, wb->codes, wb->gmeta, wb->steps)) != QL_OK) return st;
+  ql_desc dc = *da;
+  dc.N = da->N + db->N;
+  if ((st = check_packed(&dc, out->codes, out->gmeta, out->steps)) != QL_OK) return st;
+  size_t ca, ga, sa, cb, gb, sb;
+  if ((st = qlinear_packed_bytes(da, &ca, &ga, &sa)) != QL_OK) return st;
+  if ((st = qlinear_packed_bytes(db, &cb, &gb, &sb)) != QL_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const void *srcs[3][2] = {{wa->codes, wb->codes}, {wa->gmeta, wb->gmeta}, {wa->steps, wb->steps}};
+  void *dsts[3] = {out->codes, out->gmeta, out->steps};
+  const size_t na[3] = {ca, ga, sa}, nb[3] = {cb, gb, sb};
+  for (int i = 0; i < 3; ++i) {
+    if (na[i] + nb[i] == 0) continue;  // affine: no step buffer
+    uint8_t *dst = static_cast<uint8_t *>(dsts[i]);
+    if (cudaMemcpyAsync(dst, srcs[i][0], na[i], cudaMemcpyDeviceToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(dst + na[i], srcs[i][1], nb[i], cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+      return QL_ERR_CUDA;
+  }
+  return QL_OK;
 }
 
 ql_status qlinear_gemm_noalloc(const ql_desc *d, const ql_packed_const *w, const void *x, int64_t M, void *y,
@@ -561,12 +622,12 @@ ql_status qlinear_gemm_noalloc(const ql_desc *d, const ql_packed_const *w, const
   if ((st = noalloc_scratch(&scratch)) != QL_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   switch (d->fmt) {
-    case QL_INT4_NSS: return launch_gemm<FMT_INT4, 4>(d, w, x, M, y, scratch, s, di->sms);
-    case QL_INT6_SYM: return launch_gemm<FMT_INT6, 6>(d, w, x, M, y, scratch, s, di->sms);
+    case QL_INT4_NSS: return launch_gemm<FMT_INT4, 4>(d, w, x, M, nullptr, y, scratch, s, di->sms);
+    case QL_INT6_SYM: return launch_gemm<FMT_INT6, 6>(d, w, x, M, nullptr, y, scratch, s, di->sms);
     default:
-      if (d->bits == 2) return launch_gemm<FMT_AFFINE, 2>(d, w, x, M, y, scratch, s, di->sms);
-      if (d->bits == 4) return launch_gemm<FMT_AFFINE, 4>(d, w, x, M, y, scratch, s, di->sms);
-      return launch_gemm<FMT_AFFINE, 8>(d, w, x, M, y, scratch, s, di->sms);
+      if (d->bits == 2) return launch_gemm<FMT_AFFINE, 2>(d, w, x, M, nullptr, y, scratch, s, di->sms);
+      if (d->bits == 4) return launch_gemm<FMT_AFFINE, 4>(d, w, x, M, nullptr, y, scratch, s, di->sms);
+      return launch_gemm<FMT_AFFINE, 8>(d, w, x, M, nullptr, y, scratch, s, di->sms);
   }
 }
 
