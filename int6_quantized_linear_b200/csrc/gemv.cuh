@@ -200,6 +200,11 @@ QL_DEVI float2 lds64f(uint32_t a) {
   asm volatile("ld.shared.v2.f32 {%0,%1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(a));
   return v;
 }
+QL_DEVI uint2 lds64(uint32_t a) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+  return v;
+}
 QL_DEVI uint32_t lds32(uint32_t a) {
   uint32_t v;
   asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
@@ -531,36 +536,57 @@ __global__ void __launch_bounds__(256) gemv_xprep_mt_kernel(const __nv_bfloat16 
 
 constexpr int GEMV_MT_WARPS = 4;  // consumer warps per CTA; warp 4 produces
 constexpr int GEMV_MT_THREADS = 32 * (GEMV_MT_WARPS + 1);
-constexpr int GEMV_MT_RING = 4;
 constexpr int GEMV_MT_CTAS_PER_SM = 3;
-// stage: codes [64 rows][128 B] (128-byte swizzle), group words [64][16 B], group sums [8][M][8 B],
-// x words [8 groups][M][4][16 B]
-constexpr int GEMV_MT_ST_CODES = 0, GEMV_MT_ST_GMETA = 8192, GEMV_MT_ST_GSUM = 9216, GEMV_MT_ST_X = 9728;
-constexpr int GEMV_MT_STAGE_BYTES = 14336;
+
+// Stage layout of the multi-token kernel per format, for one 256-weight super-block of 64 rows:
+// codes [64 rows][CODE_ROW B] as 128-byte-swizzled boxes of 128 B, group words [64][META_ROW B],
+// group sums [8][M][8 B], x words [8 groups][M][4][16 B].  int4 and 4-bit affine codes share one
+// layout (a nibble per weight, low nibble first); 8-bit affine codes are bytes.
+template <int FMT, int BITS, int G>
+struct MtLayout {
+  static constexpr int CODE_ROW = FMT == FMT_INT4 ? 128 : 256 * BITS / 8;
+  static constexpr int CODE_BOXES = CODE_ROW / 128;
+  static constexpr int META_ROW = FMT == FMT_INT4 ? 16 : 4 * (256 / G);  // int4: 8 x u16; affine: 256/G x u32
+  static constexpr int ST_GMETA = CODE_BOXES * 64 * 128;
+  static constexpr int ST_GSUM = ST_GMETA + 64 * META_ROW;
+  static constexpr int ST_X = ST_GSUM + 512;
+  static constexpr int STAGE = (ST_X + 4096 + 1023) / 1024 * 1024;
+  static constexpr int RING = 3 * (4 * STAGE + 1024) <= 227 * 1024 ? 4 : 3;
+  static constexpr int SMEM = RING * STAGE + RING * 16 + 16 + 1024;
+};
 
 struct GemvMtParams {
-  const uint8_t *steps;
+  const uint8_t *steps;       // int4 step words; unused for affine
   const __nv_bfloat16 *bias;  // [N] or NULL
   int64_t N, K;
-  int M;  // 2 .. 8 tokens
+  int M;  // 1 .. 8 tokens (int4: 2 .. 8)
   int P;  // CTAs per 64-row group (K split)
   GemvWorkspace ws;
   __nv_bfloat16 *y;
 };
 
-inline constexpr int gemv_mt_smem_bytes() { return GEMV_MT_RING * GEMV_MT_STAGE_BYTES + GEMV_MT_RING * 16 + 16 + 1024; }
+template <int FMT, int BITS, int G>
+inline constexpr int gemv_mt_smem_bytes() { return MtLayout<FMT, BITS, G>::SMEM; }
 
+// int4: w = (q - zc zs)(sc ss) with the step word per super-block; affine (4 / 8 bits, group 32 or
+// 64): w = q s + b with (s, b) bf16 per group.  Per (row, token, 32-weight slice) the integer MMA
+// gives T = sum_k A_k x_int_k with A = 16 q (nibbles) or q (bytes); then
+//   int4:   y += S (2^-a / 16) (T - 16 Z X)
+//   affine: y += s' (2^-a / 16) T + b 2^-a X      (s' = s, or 16 s for bytes)
+template <int FMT, int BITS, int G>
 __global__ void __launch_bounds__(GEMV_MT_THREADS, GEMV_MT_CTAS_PER_SM)
-    gemv_int4_mt_kernel(const __grid_constant__ CUtensorMap map_codes,
-                        const __grid_constant__ CUtensorMap map_gmeta, GemvMtParams p) {
+    gemv_mt_kernel(const __grid_constant__ CUtensorMap map_codes, const __grid_constant__ CUtensorMap map_gmeta,
+                   GemvMtParams p) {
+  using L = MtLayout<FMT, BITS, G>;
+  constexpr int RING = L::RING;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + GEMV_MT_RING * GEMV_MT_STAGE_BYTES);  // full[R], empty[R]
-  int *flags = reinterpret_cast<int *>(bars + 2 * GEMV_MT_RING);  // abort, last-part
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + RING * L::STAGE);  // full[R], empty[R]
+  int *flags = reinterpret_cast<int *>(bars + 2 * RING);                   // abort, last-part
   volatile int *abort_flag = flags;
   const uint32_t sbase = smem_u32(smem);
   auto bar_full = [&](int s) { return smem_u32(bars + s); };
-  auto bar_empty = [&](int s) { return smem_u32(bars + GEMV_MT_RING + s); };
+  auto bar_empty = [&](int s) { return smem_u32(bars + RING + s); };
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int P = p.P, M = p.M;
   const int NS = (int)(p.K / 256);
@@ -568,7 +594,7 @@ __global__ void __launch_bounds__(GEMV_MT_THREADS, GEMV_MT_CTAS_PER_SM)
   const int part = (int)(blockIdx.x - rg * P);
   const int sb0 = part * NS / P, nsb = (part + 1) * NS / P - sb0;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < GEMV_MT_RING; ++s) {
+    for (int s = 0; s < RING; ++s) {
       mbar_init(bar_full(s), 1);
       mbar_init(bar_empty(s), GEMV_MT_WARPS);
     }
@@ -583,20 +609,23 @@ __global__ void __launch_bounds__(GEMV_MT_THREADS, GEMV_MT_CTAS_PER_SM)
     if (lane == 0) {
       tma_prefetch_desc(&map_codes);
       tma_prefetch_desc(&map_gmeta);
-      const uint32_t tx = 8192 + 1024 + (uint32_t)M * 64 + (uint32_t)M * 512;
+      const uint32_t tx = L::ST_GSUM + (uint32_t)M * 64 + (uint32_t)M * 512;  // codes + group words + sums + x
       auto issue_w = [&](int i, int s) {
-        const uint32_t st = sbase + s * GEMV_MT_STAGE_BYTES;
+        const uint32_t st = sbase + s * L::STAGE;
         mbar_arrive_expect_tx(bar_full(s), tx);
-        tma_load_2d(st + GEMV_MT_ST_CODES, &map_codes, bar_full(s), (sb0 + i) * 128, (int32_t)(rg * 64));
-        tma_load_2d(st + GEMV_MT_ST_GMETA, &map_gmeta, bar_full(s), (sb0 + i) * 16, (int32_t)(rg * 64));
+#pragma unroll
+        for (int bx = 0; bx < L::CODE_BOXES; ++bx)
+          tma_load_2d(st + bx * 8192, &map_codes, bar_full(s), (sb0 + i) * L::CODE_ROW + bx * 128,
+                      (int32_t)(rg * 64));
+        tma_load_2d(st + L::ST_GMETA, &map_gmeta, bar_full(s), (sb0 + i) * L::META_ROW, (int32_t)(rg * 64));
       };
       auto issue_x = [&](int i, int s) {
-        const uint32_t st = sbase + s * GEMV_MT_STAGE_BYTES;
-        const int64_t g0 = (int64_t)(sb0 + i) * 8;  // first group of the super-block
-        bulk_load(st + GEMV_MT_ST_GSUM, p.ws.gsum + g0 * M, (uint32_t)M * 64, bar_full(s));
-        bulk_load(st + GEMV_MT_ST_X, p.ws.xq + g0 * M * 4, (uint32_t)M * 512, bar_full(s));
+        const uint32_t st = sbase + s * L::STAGE;
+        const int64_t g0 = (int64_t)(sb0 + i) * 8;  // first 32-element group of the super-block
+        bulk_load(st + L::ST_GSUM, p.ws.gsum + g0 * M, (uint32_t)M * 64, bar_full(s));
+        bulk_load(st + L::ST_X, p.ws.xq + g0 * M * 4, (uint32_t)M * 512, bar_full(s));
       };
-      const int pre = nsb < GEMV_MT_RING ? nsb : GEMV_MT_RING;
+      const int pre = nsb < RING ? nsb : RING;
       for (int i = 0; i < pre; ++i) issue_w(i, i);  // weights need no x
       pdl_wait();
       for (int i = 0; i < pre; ++i) issue_x(i, i);
@@ -611,15 +640,15 @@ __global__ void __launch_bounds__(GEMV_MT_THREADS, GEMV_MT_CTAS_PER_SM)
         }
         issue_w(i, s);
         issue_x(i, s);
-        if (++s == GEMV_MT_RING) {
+        if (++s == RING) {
           s = 0;
           ph ^= 1u;
         }
       }
       if (!ok) {  // let the copies in flight land before the CTA can exit
-        for (int j = i - 1; j >= 0 && j >= i - GEMV_MT_RING; --j) {
+        for (int j = i - 1; j >= 0 && j >= i - RING; --j) {
           const long long t0 = clock64();
-          while (!mbar_try_wait(bar_full(j % GEMV_MT_RING), (uint32_t)((j / GEMV_MT_RING) & 1)) &&
+          while (!mbar_try_wait(bar_full(j % RING), (uint32_t)((j / RING) & 1)) &&
                  clock64() - t0 < QL_WAIT_LIMIT_CYCLES) {
           }
         }
@@ -632,54 +661,76 @@ __global__ void __launch_bounds__(GEMV_MT_THREADS, GEMV_MT_CTAS_PER_SM)
     const int64_t c0 = n0 < p.N ? n0 : p.N - 1, c1 = n1 < p.N ? n1 : p.N - 1;
     const uint32_t *st0 = reinterpret_cast<const uint32_t *>(p.steps) + c0 * NS + sb0;
     const uint32_t *st1 = reinterpret_cast<const uint32_t *>(p.steps) + c1 * NS + sb0;
-    uint32_t sr0[GEMV_MT_RING], sr1[GEMV_MT_RING];  // step words by stage, RING - 1 super-blocks ahead
+    uint32_t sr0[RING], sr1[RING];  // int4 step words by stage, RING - 1 super-blocks ahead
 #pragma unroll
-    for (int s = 0; s < GEMV_MT_RING; ++s) {
+    for (int s = 0; s < RING; ++s) {
       sr0[s] = 0u;
       sr1[s] = 0u;
-      if (s < GEMV_MT_RING - 1 && s < nsb) {
-        sr0[s] = __ldg(st0 + s);
-        sr1[s] = __ldg(st1 + s);
+      if constexpr (FMT == FMT_INT4) {
+        if (s < RING - 1 && s < nsb) {
+          sr0[s] = __ldg(st0 + s);
+          sr1[s] = __ldg(st1 + s);
+        }
       }
     }
     const int32_t acc_init[4] = {GEMV_ACC0, GEMV_ACC0, GEMV_ACC0, GEMV_ACC0};
     float acc[4] = {0.f, 0.f, 0.f, 0.f};  // (row g | g + 8) x (token 2c | 2c + 1)
     const uint32_t sw = (uint32_t)(r0 & 7);
     bool ok = true;
-    for (int base = 0; base < nsb && ok; base += GEMV_MT_RING) {
-      const uint32_t par = (uint32_t)((base / GEMV_MT_RING) & 1);
+    for (int base = 0; base < nsb && ok; base += RING) {
+      const uint32_t par = (uint32_t)((base / RING) & 1);
 #pragma unroll
-      for (int s = 0; s < GEMV_MT_RING; ++s) {
+      for (int s = 0; s < RING; ++s) {
         const int i = base + s;
         if (i >= nsb) break;
-        const int nx = i + GEMV_MT_RING - 1, sn = (s + GEMV_MT_RING - 1) % GEMV_MT_RING;
-        if (nx < nsb) {
-          sr0[sn] = __ldg(st0 + nx);
-          sr1[sn] = __ldg(st1 + nx);
+        if constexpr (FMT == FMT_INT4) {
+          const int nx = i + RING - 1, sn = (s + RING - 1) % RING;
+          if (nx < nsb) {
+            sr0[sn] = __ldg(st0 + nx);
+            sr1[sn] = __ldg(st1 + nx);
+          }
         }
         if (!mbar_wait_bounded(bar_full(s), par, abort_flag)) {
           ok = false;
           break;
         }
-        const uint32_t stg = sbase + s * GEMV_MT_STAGE_BYTES;
-        const uint4 gm0 = lds128(stg + GEMV_MT_ST_GMETA + r0 * 16), gm1 = lds128(stg + GEMV_MT_ST_GMETA + r1 * 16);
-        const uint32_t gw0[4] = {gm0.x, gm0.y, gm0.z, gm0.w}, gw1[4] = {gm1.x, gm1.y, gm1.z, gm1.w};
-        const uint32_t cs0 = sr0[s], cs1 = sr1[s];
-        const float ss0 = f16_bits_to_f32(cs0), zs0 = f16_bits_to_f32(cs0 >> 16);
-        const float ss1 = f16_bits_to_f32(cs1), zs1 = f16_bits_to_f32(cs1 >> 16);
-        const float nss0 = -8388608.f * ss0, nzs0 = -8388608.f * zs0;
-        const float nss1 = -8388608.f * ss1, nzs1 = -8388608.f * zs1;
+        const uint32_t stg = sbase + s * L::STAGE;
+        // group words of rows r0, r1 (int4: 8 x u16 sc|zc; affine: 256/G x u32 s|b)
+        uint32_t gw0[L::META_ROW / 4], gw1[L::META_ROW / 4];
+#pragma unroll
+        for (int q = 0; q < L::META_ROW / 16; ++q) {
+          const uint4 a = lds128(stg + L::ST_GMETA + r0 * L::META_ROW + 16 * q);
+          const uint4 b = lds128(stg + L::ST_GMETA + r1 * L::META_ROW + 16 * q);
+          gw0[4 * q] = a.x; gw0[4 * q + 1] = a.y; gw0[4 * q + 2] = a.z; gw0[4 * q + 3] = a.w;
+          gw1[4 * q] = b.x; gw1[4 * q + 1] = b.y; gw1[4 * q + 2] = b.z; gw1[4 * q + 3] = b.w;
+        }
+        float ss0 = 0.f, zs0 = 0.f, ss1 = 0.f, zs1 = 0.f, nss0 = 0.f, nzs0 = 0.f, nss1 = 0.f, nzs1 = 0.f;
+        if constexpr (FMT == FMT_INT4) {
+          const uint32_t cs0 = sr0[s], cs1 = sr1[s];
+          ss0 = f16_bits_to_f32(cs0); zs0 = f16_bits_to_f32(cs0 >> 16);
+          ss1 = f16_bits_to_f32(cs1); zs1 = f16_bits_to_f32(cs1 >> 16);
+          nss0 = -8388608.f * ss0; nzs0 = -8388608.f * zs0;
+          nss1 = -8388608.f * ss1; nzs1 = -8388608.f * zs1;
+        }
 #pragma unroll
         for (int gg = 0; gg < 8; ++gg) {
-          const uint32_t coff = (((uint32_t)gg ^ sw) << 4) + 4 * c;
-          const uint32_t w0 = lds32(stg + r0 * 128 + coff), w1 = lds32(stg + r1 * 128 + coff);
-          const uint4 xv = lds128(stg + GEMV_MT_ST_X + ((gg * M + g) * 4 + c) * 16);
+          uint32_t e0, e1, o0, o1;  // A: even-k and odd-k codes of rows r0, r1 (x16 for nibbles)
+          if constexpr (FMT == FMT_INT4 || BITS == 4) {
+            const uint32_t coff = (((uint32_t)gg ^ sw) << 4) + 4 * c;
+            const uint32_t w0 = lds32(stg + r0 * 128 + coff), w1 = lds32(stg + r1 * 128 + coff);
+            e0 = (w0 << 4) & 0xF0F0F0F0u; e1 = (w1 << 4) & 0xF0F0F0F0u;
+            o0 = w0 & 0xF0F0F0F0u; o1 = w1 & 0xF0F0F0F0u;
+          } else {  // bytes: slice gg is 32 B of box gg / 4; lane c takes bytes 8c .. 8c + 7
+            const uint32_t ch = (uint32_t)(2 * (gg & 3) + (c >> 1));
+            const uint32_t off = (uint32_t)(gg >> 2) * 8192 + ((ch ^ sw) << 4) + 8 * (c & 1);
+            const uint2 w0 = lds64(stg + r0 * 128 + off), w1 = lds64(stg + r1 * 128 + off);
+            e0 = __byte_perm(w0.x, w0.y, 0x6420); e1 = __byte_perm(w1.x, w1.y, 0x6420);
+            o0 = __byte_perm(w0.x, w0.y, 0x7531); o1 = __byte_perm(w1.x, w1.y, 0x7531);
+          }
+          const uint4 xv = lds128(stg + L::ST_X + ((gg * M + g) * 4 + c) * 16);
           // (2^-a/16, -16 X) of tokens 2c and 2c + 1: 8-byte records, so two 8-byte loads (odd M)
-          const float2 Ga = lds64f(stg + GEMV_MT_ST_GSUM + (gg * M + 2 * c) * 8);
-          const float2 Gb = lds64f(stg + GEMV_MT_ST_GSUM + (gg * M + 2 * c + 1) * 8);
-          const float4 G = make_float4(Ga.x, Ga.y, Gb.x, Gb.y);
-          const uint32_t e0 = (w0 << 4) & 0xF0F0F0F0u, e1 = (w1 << 4) & 0xF0F0F0F0u;  // even k, x16
-          const uint32_t o0 = w0 & 0xF0F0F0F0u, o1 = w1 & 0xF0F0F0F0u;                  // odd k, x16
+          const float2 Ga = lds64f(stg + L::ST_GSUM + (gg * M + 2 * c) * 8);
+          const float2 Gb = lds64f(stg + L::ST_GSUM + (gg * M + 2 * c + 1) * 8);
           int32_t dh[4], dl[4];
           QL_IMMA0("s8", dh, acc_init, e0, e1, o0, o1, xv.x, xv.y);
           QL_IMMA0("u8", dl, acc_init, e0, e1, o0, o1, xv.z, xv.w);
@@ -687,14 +738,27 @@ __global__ void __launch_bounds__(GEMV_MT_THREADS, GEMV_MT_CTAS_PER_SM)
 #pragma unroll
           for (int q = 0; q < 4; ++q)
             t[q] = fmaf(__int_as_float(dh[q]) - GEMV_ACC0_F, 256.f, __int_as_float(dl[q]) - GEMV_ACC0_F);
-          const uint32_t gw0g = gw0[gg >> 1], gw1g = gw1[gg >> 1];
-          const int bsc = 2 * (gg & 1);
-          const float S0 = fmaf(byte_magic(gw0g, bsc), ss0, nss0), Z0 = fmaf(byte_magic(gw0g, bsc + 1), zs0, nzs0);
-          const float S1 = fmaf(byte_magic(gw1g, bsc), ss1, nss1), Z1 = fmaf(byte_magic(gw1g, bsc + 1), zs1, nzs1);
-          acc[0] = fmaf(S0 * G.x, fmaf(Z0, G.y, t[0]), acc[0]);
-          acc[1] = fmaf(S0 * G.z, fmaf(Z0, G.w, t[1]), acc[1]);
-          acc[2] = fmaf(S1 * G.x, fmaf(Z1, G.y, t[2]), acc[2]);
-          acc[3] = fmaf(S1 * G.z, fmaf(Z1, G.w, t[3]), acc[3]);
+          if constexpr (FMT == FMT_INT4) {
+            const uint32_t gw0g = gw0[gg >> 1], gw1g = gw1[gg >> 1];
+            const int bsc = 2 * (gg & 1);
+            const float S0 = fmaf(byte_magic(gw0g, bsc), ss0, nss0), Z0 = fmaf(byte_magic(gw0g, bsc + 1), zs0, nzs0);
+            const float S1 = fmaf(byte_magic(gw1g, bsc), ss1, nss1), Z1 = fmaf(byte_magic(gw1g, bsc + 1), zs1, nzs1);
+            acc[0] = fmaf(S0 * Ga.x, fmaf(Z0, Ga.y, t[0]), acc[0]);
+            acc[1] = fmaf(S0 * Gb.x, fmaf(Z0, Gb.y, t[1]), acc[1]);
+            acc[2] = fmaf(S1 * Ga.x, fmaf(Z1, Ga.y, t[2]), acc[2]);
+            acc[3] = fmaf(S1 * Gb.x, fmaf(Z1, Gb.y, t[3]), acc[3]);
+          } else {
+            // slice gg lies in affine group gg * 32 / G of the super-block; its word holds (s, b) bf16
+            const uint32_t gw0g = gw0[gg * 32 / G], gw1g = gw1[gg * 32 / G];
+            constexpr float SF = BITS == 8 ? 16.f : 1.f;  // bytes carry q, nibbles 16 q
+            const float s0 = bf16_bits_to_f32(gw0g) * SF, b0 = bf16_bits_to_f32(gw0g >> 16);
+            const float s1 = bf16_bits_to_f32(gw1g) * SF, b1 = bf16_bits_to_f32(gw1g >> 16);
+            // b 2^-a X = -b (2^-a/16)(-16 X)
+            acc[0] = fmaf(s0 * Ga.x, t[0], fmaf(-b0 * Ga.x, Ga.y, acc[0]));
+            acc[1] = fmaf(s0 * Gb.x, t[1], fmaf(-b0 * Gb.x, Gb.y, acc[1]));
+            acc[2] = fmaf(s1 * Ga.x, t[2], fmaf(-b1 * Ga.x, Ga.y, acc[2]));
+            acc[3] = fmaf(s1 * Gb.x, t[3], fmaf(-b1 * Gb.x, Gb.y, acc[3]));
+          }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(bar_empty(s));

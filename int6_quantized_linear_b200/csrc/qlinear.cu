@@ -165,10 +165,18 @@ ql_status launch_gemm(const ql_desc *d, const ql_packed_const *w, const void *x,
   return launched();
 }
 
-// int6 and affine GEMV calls with M >= 8 tokens run on the tensor-core GEMM (measured faster there:
-// affine M=32 70-74 us vs 537-551 us, int6 M=8 198 us vs 284 us on the benchmark layers); int4 has
-// its own tensor-core GEMV up to M = 8.
-inline bool gemv_runs_on_gemm(const ql_desc *d, int64_t M) { return d->fmt != QL_INT4_NSS && M >= 8; }
+// Which GEMV calls run on the tensor-core GEMM (measured faster there on the benchmark layers:
+// affine M=32 70-74 us vs 537-551 us, int6 M=8 198 us vs 284 us on the CUDA-core kernel): int6 from
+// M = 8; affine from M = 9 when a multi-token tensor-core GEMV exists for it (4 / 8 bits, group 32 /
+// 64), else from M = 8.  int4 has tensor-core GEMVs up to M = 8.
+inline bool gemv_runs_on_gemm(const ql_desc *d, int64_t M) {
+  if (d->fmt == QL_INT6_SYM) return M >= 8;
+  if (d->fmt == QL_AFFINE_U32) {  // 4- and 8-bit affine with group 32 / 64 have the multi-token kernel up to M = 8
+    const bool mt = (d->bits == 4 || d->bits == 8) && (d->group == 32 || d->group == 64) && d->K % 256 == 0;
+    return M >= (mt ? 9 : 8);
+  }
+  return false;
+}
 
 inline size_t gemv_call_workspace_bytes(const ql_desc *d, int64_t M) {
   const size_t own = gemv_workspace_bytes(M, d->N, d->K);
@@ -181,6 +189,68 @@ template <int FMT, int BITS>
 ql_status launch_gemm(const ql_desc *d, const ql_packed_const *w, const void *x, int64_t M, const void *bias,
                       void *y, void *workspace, cudaStream_t st, int sms);
 
+// Multi-token tensor-core GEMV (int4 at 2..8 tokens; 4- and 8-bit affine with group 32 or 64 at
+// 1..8 tokens): x preparation, then the streaming kernel as its programmatic dependent.
+template <int FMT, int BITS, int G>
+ql_status launch_gemv_mt(const ql_desc *d, const ql_packed_const *w, const __nv_bfloat16 *xb, int64_t M,
+                         const __nv_bfloat16 *bb, __nv_bfloat16 *yb, void *workspace, cudaStream_t st, int sms) {
+  using L = MtLayout<FMT, BITS, G>;
+  const int64_t N = d->N, K = d->K, NS = K / 256, TG = (N + 63) / 64;
+  const GemvWorkspace ws = gemv_workspace_carve(workspace, M, K);
+  cudaLaunchAttribute pa[1];
+  pa[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pa[0].val.programmaticStreamSerializationAllowed = 1;
+  {
+    const int64_t threads = std::max<int64_t>(4 * M * (K / 32), TG);
+    cudaLaunchConfig_t pc = {};
+    pc.gridDim = dim3((unsigned)((threads + 255) / 256));
+    pc.blockDim = dim3(256);
+    pc.stream = st;
+    pc.attrs = pa;
+    pc.numAttrs = 1;
+    if (cudaLaunchKernelEx(&pc, gemv_xprep_mt_kernel, xb, M, K, TG, ws) != cudaSuccess) return QL_ERR_CUDA;
+  }
+  GemvMtParams p;
+  p.steps = static_cast<const uint8_t *>(w->steps);
+  p.bias = bb;
+  p.N = N;
+  p.K = K;
+  p.M = (int)M;
+  // split K over P CTAs per 64-row group while the row groups alone leave a wave unfilled
+  int64_t P = std::max<int64_t>(1, std::min<int64_t>(NS, (int64_t)sms * GEMV_MT_CTAS_PER_SM / TG));
+  P = std::min<int64_t>(P, std::max<int64_t>(1, GEMV_MT_MAX_CTAS / TG));
+  if (TG * P > GEMV_MT_MAX_CTAS) return QL_ERR_RANGE;
+  p.P = (int)P;
+  p.ws = ws;
+  p.y = yb;
+  const uint64_t code_row = FMT == FMT_INT4 ? (uint64_t)K / 2 : (uint64_t)K * BITS / 8;
+  const uint64_t meta_row = FMT == FMT_INT4 ? (uint64_t)K / 16 : (uint64_t)K / G * 4;
+  CUtensorMap mc, mg;  // codes: boxes of 64 rows x 128 bytes, 128-byte swizzle; group words: 64 rows x META_ROW
+  if (!encode_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->codes, code_row, (uint64_t)N, code_row, 128, 64,
+                 CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_2d(&mg, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->gmeta, meta_row, (uint64_t)N, meta_row, L::META_ROW, 64,
+                 CU_TENSOR_MAP_SWIZZLE_NONE))
+    return QL_ERR_CUDA;
+  auto kern = gemv_mt_kernel<FMT, BITS, G>;
+  static thread_local int configured_dev = -1;  // per instantiation and thread
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (configured_dev != dev) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM) != cudaSuccess)
+      return QL_ERR_CUDA;
+    configured_dev = dev;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(TG * P));
+  cfg.blockDim = dim3(GEMV_MT_THREADS);
+  cfg.dynamicSmemBytes = L::SMEM;
+  cfg.stream = st;
+  cfg.attrs = pa;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, mc, mg, p) != cudaSuccess) return QL_ERR_CUDA;
+  return launched();
+}
+
 template <int FMT, int BITS>
 ql_status launch_gemv(const ql_desc *d, const ql_packed_const *w, const void *x, int64_t M, const void *bias,
                       void *y, void *workspace, cudaStream_t st, int sms) {
@@ -188,6 +258,13 @@ ql_status launch_gemv(const ql_desc *d, const ql_packed_const *w, const void *x,
   auto *yb = static_cast<__nv_bfloat16 *>(y);
   const auto *bb = static_cast<const __nv_bfloat16 *>(bias);
   if (gemv_runs_on_gemm(d, M)) return launch_gemm<FMT, BITS>(d, w, x, M, bias, y, workspace, st, sms);
+  if constexpr (FMT == FMT_INT4) {
+    if (M >= 2) return launch_gemv_mt<FMT_INT4, 4, 32>(d, w, xb, M, bb, yb, workspace, st, sms);
+  }
+  if constexpr (FMT == FMT_AFFINE && (BITS == 4 || BITS == 8)) {
+    if (d->K % 256 == 0 && d->group == 64) return launch_gemv_mt<FMT_AFFINE, BITS, 64>(d, w, xb, M, bb, yb, workspace, st, sms);
+    if (d->K % 256 == 0 && d->group == 32) return launch_gemv_mt<FMT_AFFINE, BITS, 32>(d, w, xb, M, bb, yb, workspace, st, sms);
+  }
   if constexpr (FMT == FMT_INT4) {
     if (M == 1) {  // tensor-core path: preparation pass, then the streaming kernel as its dependent
       const GemvWorkspace ws = gemv_workspace_carve(workspace, M, d->K);
@@ -245,61 +322,6 @@ ql_status launch_gemv(const ql_desc *d, const ql_packed_const *w, const void *x,
       cfg.attrs = attr;
       cfg.numAttrs = 1;
       if (cudaLaunchKernelEx(&cfg, gemv_int4_m1_tc_kernel, mc, mg, p) != cudaSuccess) return QL_ERR_CUDA;
-      return launched();
-    }
-    if (M >= 2 && M <= 8) {  // multi-token tensor-core path
-      const int64_t N = d->N, K = d->K, NS = K / 256, TG = (N + 63) / 64;
-      const GemvWorkspace ws = gemv_workspace_carve(workspace, M, K);
-      cudaLaunchAttribute pa[1];
-      pa[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-      pa[0].val.programmaticStreamSerializationAllowed = 1;
-      {
-        const int64_t threads = std::max<int64_t>(4 * M * (K / 32), TG);
-        cudaLaunchConfig_t pc = {};
-        pc.gridDim = dim3((unsigned)((threads + 255) / 256));
-        pc.blockDim = dim3(256);
-        pc.stream = st;
-        pc.attrs = pa;
-        pc.numAttrs = 1;
-        if (cudaLaunchKernelEx(&pc, gemv_xprep_mt_kernel, xb, M, K, TG, ws) != cudaSuccess) return QL_ERR_CUDA;
-      }
-      GemvMtParams p;
-      p.steps = static_cast<const uint8_t *>(w->steps);
-      p.bias = bb;
-      p.N = N;
-      p.K = K;
-      p.M = (int)M;
-      // split K over P CTAs per 64-row group while the row groups alone leave a wave unfilled
-      int64_t P = std::max<int64_t>(1, std::min<int64_t>(NS, (int64_t)sms * GEMV_MT_CTAS_PER_SM / TG));
-      P = std::min<int64_t>(P, std::max<int64_t>(1, GEMV_MT_MAX_CTAS / TG));
-      if (TG * P > GEMV_MT_MAX_CTAS) return QL_ERR_RANGE;
-      p.P = (int)P;
-      p.ws = ws;
-      p.y = yb;
-      CUtensorMap mc, mg;  // codes as [N][K/2] bytes, boxes of 64 rows x 128 bytes, 128-byte swizzle;
-                           // group words as [N][K/16] bytes, boxes of 64 rows x 16 bytes
-      if (!encode_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->codes, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2,
-                     128, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-          !encode_2d(&mg, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->gmeta, (uint64_t)K / 16, (uint64_t)N, (uint64_t)K / 16,
-                     16, 64, CU_TENSOR_MAP_SWIZZLE_NONE))
-        return QL_ERR_CUDA;
-      static thread_local int configured_dev = -1;
-      int dev = 0;
-      cudaGetDevice(&dev);
-      if (configured_dev != dev) {
-        if (cudaFuncSetAttribute(gemv_int4_mt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 gemv_mt_smem_bytes()) != cudaSuccess)
-          return QL_ERR_CUDA;
-        configured_dev = dev;
-      }
-      cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3((unsigned)(TG * P));
-      cfg.blockDim = dim3(GEMV_MT_THREADS);
-      cfg.dynamicSmemBytes = gemv_mt_smem_bytes();
-      cfg.stream = st;
-      cfg.attrs = pa;
-      cfg.numAttrs = 1;
-      if (cudaLaunchKernelEx(&cfg, gemv_int4_mt_kernel, mc, mg, p) != cudaSuccess) return QL_ERR_CUDA;
       return launched();
     }
   }
