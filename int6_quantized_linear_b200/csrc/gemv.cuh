@@ -101,13 +101,13 @@ struct GemvWorkspace {
   uint4 *xq;        // M = 1: [K/256 super-blocks][4 j][2 kinds][8 groups][16 B] B-operand pairs (gemv_xprep_kernel)
                     // M > 1: [K/32 groups][M tokens][4][16 B] B-operand words (gemv_xprep_mt_kernel)
   float2 *gsum;     // M = 1: [K/32]; M > 1: [K/32][M]: (2^-a_g / 16, -16 * sum x_int)
-  float *partial;   // M > 1: [CTA][M][64 rows] sums of a CTA's K range
-  int *counters;    // M > 1: [N/64 row groups] parts finished so far
+  float *partial;   // M = 1: [16-row tile][part][16 rows]; M > 1: [CTA][M][64 rows]: sums of one K range
+  int *counters;    // parts finished so far: M = 1 per 16-row tile, M > 1 per 64-row group
 };
 
 inline size_t gemv_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   return align256((size_t)M * K * 4) + align256((size_t)M * (K / 32) * 8) +
-         align256((size_t)GEMV_MT_MAX_CTAS * 64 * M * 4) + align256((size_t)((N + 63) / 64) * 4);
+         align256((size_t)GEMV_MT_MAX_CTAS * 64 * M * 4) + align256((size_t)((N + 15) / 16) * 4);
 }
 
 inline GemvWorkspace gemv_workspace_carve(void *base, int64_t M, int64_t K) {
@@ -123,6 +123,13 @@ inline GemvWorkspace gemv_workspace_carve(void *base, int64_t M, int64_t K) {
   return w;
 }
 
+// Counter bump with acquire-release semantics at GPU scope; returns the old value.
+QL_DEVI int atomic_add_acq_rel_gpu(int *addr, int v) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(addr), "r"(v) : "memory");
+  return old;
+}
+
 QL_DEVI void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 QL_DEVI void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
@@ -130,12 +137,14 @@ QL_DEVI void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 // Chunk (j, kind) of group grp is the register quad its feeding lane loads: the high-byte and low-byte
 // words of k = 8j + kind + {0, 2, 4, 6}, each paired with a zero word so that one 16-byte load gives
 // the B pairs of two MMAs -- (x, 0) for groups 0-3 (their lanes feed b0), (0, x) for groups 4-7 (b1).
+// It also zeroes the first n_counters tile counters of the K split.
 __global__ void __launch_bounds__(256) gemv_xprep_kernel(const __nv_bfloat16 *x, int64_t M, int64_t K,
-                                                         GemvWorkspace ws) {
+                                                         int64_t n_counters, GemvWorkspace ws) {
   pdl_launch_dependents();  // the streaming kernel may start fetching weights now
   pdl_wait();               // x (and this workspace) may belong to the kernel launched before this one
   const int64_t ng = K / 32;
-  const int64_t gi = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;  // over M * ng
+  const int64_t gi = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;  // over max(M * ng, n_counters)
+  if (gi < n_counters) ws.counters[gi] = 0;
   if (gi >= M * ng) return;
   const uint4 *src = reinterpret_cast<const uint4 *>(x) + 4 * gi;  // 32 bf16 = 64 bytes
   float xs[32];
@@ -263,15 +272,14 @@ struct GemvTcParams {
   const uint8_t *steps;
   const __nv_bfloat16 *bias;  // [N] or NULL
   int64_t N, K;
-  int parts;  // warps splitting K for one tile (1, 2 or 4)
+  int parts;  // warps splitting K for one tile (1 .. K/256); warp w of the grid takes part w % parts of tile w / parts
   GemvWorkspace ws;
   __nv_bfloat16 *y;
 };
 
-// dynamic shared memory: [warp][stage] (1024-aligned), zero block, mbarriers, reduction buffer
+// dynamic shared memory: [warp][stage] (1024-aligned), zero block, mbarriers
 inline constexpr int gemv_smem_bytes() {
-  return GEMV_WARPS * GEMV_RING * GEMV_STAGE_BYTES + GEMV_ZERO_BYTES + GEMV_WARPS * GEMV_RING * 8 +
-         GEMV_WARPS * 16 * 4 + 1024;
+  return GEMV_WARPS * GEMV_RING * GEMV_STAGE_BYTES + GEMV_ZERO_BYTES + GEMV_WARPS * GEMV_RING * 8 + 1024;
 }
 
 // Everything a super-block needs except its step words arrives by one stage of a per-warp ring:
@@ -288,13 +296,13 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS, GEMV_CTAS_PER_SM)
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *zero_blk = smem + GEMV_WARPS * GEMV_RING * GEMV_STAGE_BYTES;
   uint64_t *bars = reinterpret_cast<uint64_t *>(zero_blk + GEMV_ZERO_BYTES);
-  float *red = reinterpret_cast<float *>(bars + GEMV_WARPS * GEMV_RING);  // [GEMV_WARPS][16]
   __shared__ int abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int P = p.parts, T = GEMV_WARPS / P;
-  const int tl = warp / P, part = warp - tl * P;
+  const int P = p.parts;
   const int64_t n_tiles = (p.N + 15) / 16;
-  const int64_t tile = (int64_t)blockIdx.x * T + tl;
+  const int64_t wid = (int64_t)blockIdx.x * GEMV_WARPS + warp;
+  const int64_t tile = wid / P;
+  const int part = (int)(wid - tile * P);
   const int g = lane >> 2, c = lane & 3;
   const bool active = tile < n_tiles;
   const int NS = (int)(p.K / 256);
@@ -453,14 +461,33 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS, GEMV_CTAS_PER_SM)
   acc0 += __shfl_xor_sync(0xffffffffu, acc0, 2);
   acc1 += __shfl_xor_sync(0xffffffffu, acc1, 1);
   acc1 += __shfl_xor_sync(0xffffffffu, acc1, 2);
-  if (c == 0) {
-    red[warp * 16 + pg] = acc0;
-    red[warp * 16 + pg + 8] = acc1;
+  if (!active) return;
+  if (P == 1) {
+    if (c == 0) {
+      const int64_t ra = tile * 16 + pg, rb = ra + 8;
+      if (ra < p.N) p.y[ra] = __float2bfloat16_rn(acc0 + bias_at(p.bias, ra));
+      if (rb < p.N) p.y[rb] = __float2bfloat16_rn(acc1 + bias_at(p.bias, rb));
+    }
+    return;
   }
-  __syncthreads();
-  if (part == 0 && lane < 16 && active) {
+  // K split over warps of (possibly) different CTAs: publish this part's sums; the warp that
+  // finishes the tile last adds the P parts in part order, so the result does not depend on timing
+  float *part_sums = p.ws.partial + tile * P * 16;
+  {  // lane r < 16 stores the sum of tile row r (held by lane 4g with pg(g) = r mod 8)
+    const int rr = lane & 15, prow = rr & 7;
+    const int src = 4 * (((prow & 3) << 1) | (prow >> 2));
+    const float v0 = __shfl_sync(0xffffffffu, acc0, src), v1 = __shfl_sync(0xffffffffu, acc1, src);
+    if (lane < 16) part_sums[part * 16 + rr] = rr < 8 ? v0 : v1;
+  }
+  __syncwarp();  // the stores above precede lane 0's release
+  int last = 0;
+  if (lane == 0) last = atomic_add_acq_rel_gpu(p.ws.counters + tile, 1) == P - 1;
+  last = __shfl_sync(0xffffffffu, last, 0);
+  if (!last) return;
+  __syncwarp();  // lane 0's acquire precedes every lane's reads of the other parts
+  if (lane < 16) {
     float sum = 0.f;
-    for (int q = 0; q < P; ++q) sum += red[(warp + q) * 16 + lane];
+    for (int q = 0; q < P; ++q) sum += __ldcg(part_sums + q * 16 + lane);
     const int64_t r = tile * 16 + lane;
     if (r < p.N) p.y[r] = __float2bfloat16_rn(sum + bias_at(p.bias, r));
   }
@@ -788,16 +815,14 @@ __global__ void __launch_bounds__(GEMV_MT_THREADS, GEMV_MT_CTAS_PER_SM)
           mine[tk1 * 64 + r0] = acc[1];
           mine[tk1 * 64 + r1] = acc[3];
         }
-        __threadfence();
       }
     }
   }
   if (P > 1) {  // the CTA that completes a row group adds its P parts in part order
-    __syncthreads();
-    if (threadIdx.x == 0 && !*abort_flag) flags[1] = atomicAdd(p.ws.counters + rg, 1) == P - 1;
-    __syncthreads();
+    __syncthreads();  // every partial store precedes thread 0's release
+    if (threadIdx.x == 0 && !*abort_flag) flags[1] = atomic_add_acq_rel_gpu(p.ws.counters + rg, 1) == P - 1;
+    __syncthreads();  // thread 0's acquire precedes the reads of the other parts
     if (flags[1] && warp < GEMV_MT_WARPS) {
-      __threadfence();
       const float *base = p.ws.partial + (int64_t)rg * P * M * 64;
       for (int e = threadIdx.x; e < M * 64; e += GEMV_MT_WARPS * 32) {
         const int tk = e >> 6, r = e & 63;

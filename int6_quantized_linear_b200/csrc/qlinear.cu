@@ -269,9 +269,17 @@ ql_status launch_gemv(const ql_desc *d, const ql_packed_const *w, const void *x,
     if (M == 1) {  // tensor-core path: preparation pass, then the streaming kernel as its dependent
       const GemvWorkspace ws = gemv_workspace_carve(workspace, M, d->K);
       const int64_t ng = M * (d->K / 32);
+      const int64_t NS = d->K / 256, n_tiles = (d->N + 15) / 16;
+      // split K over P warps per 16-row tile while the tiles alone leave the resident warp slots
+      // unfilled; the parts' sums go through the workspace (at most GEMV_MT_MAX_CTAS * 64 floats)
+      const int64_t warp_slots = (int64_t)sms * GEMV_CTAS_PER_SM * GEMV_WARPS;
+      int64_t P = std::max<int64_t>(1, std::min<int64_t>(NS, warp_slots / n_tiles));
+      P = std::min<int64_t>(P, std::max<int64_t>(1, (int64_t)GEMV_MT_MAX_CTAS * 64 / 16 / n_tiles));
+      const int64_t n_counters = P > 1 ? n_tiles : 0;
       {  // programmatic dependent of whatever precedes it on the stream (it waits before reading x)
+        const int64_t threads = std::max<int64_t>(ng, n_counters);
         cudaLaunchConfig_t pc = {};
-        pc.gridDim = dim3((unsigned)((ng + 255) / 256));
+        pc.gridDim = dim3((unsigned)((threads + 255) / 256));
         pc.blockDim = dim3(256);
         pc.stream = st;
         cudaLaunchAttribute pa[1];
@@ -279,7 +287,8 @@ ql_status launch_gemv(const ql_desc *d, const ql_packed_const *w, const void *x,
         pa[0].val.programmaticStreamSerializationAllowed = 1;
         pc.attrs = pa;
         pc.numAttrs = 1;
-        if (cudaLaunchKernelEx(&pc, gemv_xprep_kernel, xb, M, (int64_t)d->K, ws) != cudaSuccess) return QL_ERR_CUDA;
+        if (cudaLaunchKernelEx(&pc, gemv_xprep_kernel, xb, M, (int64_t)d->K, n_counters, ws) != cudaSuccess)
+          return QL_ERR_CUDA;
       }
       GemvTcParams p;
       p.steps = static_cast<const uint8_t *>(w->steps);
@@ -295,13 +304,7 @@ ql_status launch_gemv(const ql_desc *d, const ql_packed_const *w, const void *x,
           !encode_2d(&mg, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->gmeta, (uint64_t)d->K / 16, (uint64_t)d->N,
                      (uint64_t)d->K / 16, 16, 16, CU_TENSOR_MAP_SWIZZLE_NONE))
         return QL_ERR_CUDA;
-      const int64_t NS = d->K / 256, n_tiles = (d->N + 15) / 16;
-      // split K over more warps per tile while the grid still fits one wave
-      const int64_t slots = (int64_t)sms * GEMV_CTAS_PER_SM;
-      int P = 1;
-      while (2 * P <= GEMV_WARPS && 2 * P <= NS && (n_tiles * 2 * P + GEMV_WARPS - 1) / GEMV_WARPS <= slots) P *= 2;
-      p.parts = P;
-      const int64_t T = GEMV_WARPS / P;
+      p.parts = (int)P;
       static thread_local int configured_dev = -1;
       int dev = 0;
       cudaGetDevice(&dev);
@@ -312,7 +315,7 @@ ql_status launch_gemv(const ql_desc *d, const ql_packed_const *w, const void *x,
         configured_dev = dev;
       }
       cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3((unsigned)((n_tiles + T - 1) / T));
+      cfg.gridDim = dim3((unsigned)((n_tiles * P + GEMV_WARPS - 1) / GEMV_WARPS));
       cfg.blockDim = dim3(32 * GEMV_WARPS);
       cfg.dynamicSmemBytes = gemv_smem_bytes();
       cfg.stream = st;
