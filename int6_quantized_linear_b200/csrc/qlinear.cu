@@ -8,6 +8,7 @@
 #include "../../include/qlinear.h"
 #include "gemm_sm100.cuh"
 #include "gemv.cuh"
+#include "gemv_int6.cuh"
 #include "pack_dequant.cuh"
 
 using namespace ql;
@@ -251,6 +252,67 @@ ql_status launch_gemv_mt(const ql_desc *d, const ql_packed_const *w, const __nv_
   return launched();
 }
 
+// Tensor-core int6 GEMV at 1..TM tokens: x preparation, then the streaming kernel as its dependent.
+template <int TM>
+ql_status launch_gemv_int6(const ql_desc *d, const ql_packed_const *w, const __nv_bfloat16 *xb, int64_t M,
+                           const __nv_bfloat16 *bb, __nv_bfloat16 *yb, void *workspace, cudaStream_t st, int sms) {
+  using L = Int6Layout<TM>;
+  const int64_t N = d->N, K = d->K, NS = K / 256, TG = (N + 63) / 64;
+  const GemvWorkspace ws = gemv_workspace_carve(workspace, M, K);
+  // split K over P CTAs per 64-row group while the row groups alone leave a wave unfilled
+  int64_t P = std::max<int64_t>(1, std::min<int64_t>(NS, (int64_t)sms * GEMV6_CTAS_PER_SM / TG));
+  P = std::min<int64_t>(P, std::max<int64_t>(1, GEMV_MT_MAX_CTAS / TG));
+  if (TG * P > GEMV_MT_MAX_CTAS) return QL_ERR_RANGE;
+  cudaLaunchAttribute pa[1];
+  pa[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pa[0].val.programmaticStreamSerializationAllowed = 1;
+  {
+    const int64_t threads = std::max<int64_t>(M * (K / 16), P > 1 ? TG : 0);
+    cudaLaunchConfig_t pc = {};
+    pc.gridDim = dim3((unsigned)((threads + 255) / 256));
+    pc.blockDim = dim3(256);
+    pc.stream = st;
+    pc.attrs = pa;
+    pc.numAttrs = 1;
+    if (cudaLaunchKernelEx(&pc, gemv_xprep_int6_kernel, xb, M, K, P > 1 ? TG : (int64_t)0, ws) != cudaSuccess)
+      return QL_ERR_CUDA;
+  }
+  Gemv6Params p;
+  p.steps = static_cast<const uint16_t *>(w->steps);
+  p.bias = bb;
+  p.N = N;
+  p.K = K;
+  p.M = (int)M;
+  p.P = (int)P;
+  p.ws = ws;
+  p.y = yb;
+  const uint64_t code_row = (uint64_t)K * 3 / 4, sc_row = (uint64_t)K / 16;
+  CUtensorMap mc, ms;  // codes: 64 rows x 208 bytes (a super-block and 16 bytes more); scale codes: 64 x 16 B
+  if (!encode_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->codes, code_row, (uint64_t)N, code_row, GEMV6_CODE_ROW, 64,
+                 CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !encode_2d(&ms, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->gmeta, sc_row, (uint64_t)N, sc_row, 16, 64,
+                 CU_TENSOR_MAP_SWIZZLE_NONE))
+    return QL_ERR_CUDA;
+  auto kern = gemv_int6_kernel<TM>;
+  static thread_local int configured_dev = -1;  // per instantiation and thread
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (configured_dev != dev) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM) != cudaSuccess)
+      return QL_ERR_CUDA;
+    configured_dev = dev;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(TG * P));
+  cfg.blockDim = dim3(GEMV6_THREADS);
+  cfg.dynamicSmemBytes = L::SMEM;
+  cfg.stream = st;
+  cfg.attrs = pa;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, mc, ms, p) != cudaSuccess) return QL_ERR_CUDA;
+  return launched();
+}
+
 template <int FMT, int BITS>
 ql_status launch_gemv(const ql_desc *d, const ql_packed_const *w, const void *x, int64_t M, const void *bias,
                       void *y, void *workspace, cudaStream_t st, int sms) {
@@ -260,6 +322,12 @@ ql_status launch_gemv(const ql_desc *d, const ql_packed_const *w, const void *x,
   if (gemv_runs_on_gemm(d, M)) return launch_gemm<FMT, BITS>(d, w, x, M, bias, y, workspace, st, sms);
   if constexpr (FMT == FMT_INT4) {
     if (M >= 2) return launch_gemv_mt<FMT_INT4, 4, 32>(d, w, xb, M, bb, yb, workspace, st, sms);
+  }
+  if constexpr (FMT == FMT_INT6) {  // M <= 7 here
+    if (M == 1) return launch_gemv_int6<1>(d, w, xb, M, bb, yb, workspace, st, sms);
+    if (M == 2) return launch_gemv_int6<2>(d, w, xb, M, bb, yb, workspace, st, sms);
+    if (M <= 4) return launch_gemv_int6<4>(d, w, xb, M, bb, yb, workspace, st, sms);
+    return launch_gemv_int6<8>(d, w, xb, M, bb, yb, workspace, st, sms);
   }
   if constexpr (FMT == FMT_AFFINE && (BITS == 4 || BITS == 8)) {
     if (d->K % 256 == 0 && d->group == 64) return launch_gemv_mt<FMT_AFFINE, BITS, 64>(d, w, xb, M, bb, yb, workspace, st, sms);

@@ -12,7 +12,7 @@ import torch
 import int6_quantized_linear_b200 as ql
 from int6_quantized_linear_b200 import synth
 from oracle import oracle_c as OC
-from tests.gpu_helpers import Layer, assert_close, dev, host, run_gemm, run_gemv, x_dev
+from tests.gpu_helpers import Layer, assert_close, bf16_to_f64, dev, host, run_gemm, run_gemv, x_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -144,6 +144,26 @@ def test_deterministic_and_in_bounds(cuda):
         assert np.array_equal(first, host(y.view(torch.int16), np.uint16))
         b = host(buf, np.uint16)
         assert np.all(b[:pad] == 0x7B7B) and np.all(b[pad + M * 1000:] == 0x7B7B)
+
+
+@pytest.mark.parametrize("N,K", [(200, 1536), (64, 256), (1000, 5120)])
+def test_gemv_int6_every_token_count(cuda, N, K):
+    """int6 tensor-core GEMV at each M it serves (1..7: four token buckets), with and without the
+    split of K over CTAs; repeated runs give identical bits; the bias variant adds bias[n]."""
+    L = Layer("int6", N, K, seed=11 * N + K)
+    w_ref = L.oracle_w()
+    bias_b = synth.activations(N + K, 1, N)[0]
+    for M in range(1, 8):
+        xb, xd = x_dev(K, M, seed=100 + M)
+        y = run_gemv(L, xd, M)
+        y_ref = OC.matmul_f64(xb, w_ref)
+        assert_close(y, y_ref, f"int6 gemv N={N} K={K} M={M}")
+        assert np.array_equal(y, run_gemv(L, xd, M))
+        yb = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        ql.qlinear_gemv_bias(L.desc, *L.packed(), xd, M, dev(bias_b).view(torch.bfloat16), yb)
+        assert ql.qlinear_sync_status() == ql.QL_OK
+        assert_close(host(yb.view(torch.int16), np.uint16), y_ref + bf16_to_f64(bias_b)[None, :],
+                     f"int6 gemv+bias M={M}")
 
 
 def test_device_errors_do_not_launch(cuda):
