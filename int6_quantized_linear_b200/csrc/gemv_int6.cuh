@@ -150,6 +150,7 @@ __global__ void __launch_bounds__(GEMV6_THREADS, GEMV6_CTAS_PER_SM)
                      Gemv6Params p) {
   using L = Int6Layout<TM>;
   constexpr int RING = L::RING;
+  constexpr int MP = TM < 4 ? TM : 4;  // tokens per MMA group
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
   uint8_t *zero16 = smem + RING * L::STAGE;
@@ -292,32 +293,41 @@ __global__ void __launch_bounds__(GEMV6_THREADS, GEMV6_CTAS_PER_SM)
             int6_a_words(lds32(a1), lds32(a1 + 4), lds32(a1 + 8), A10);
             int6_a_words(lds32(a1 + 48), lds32(a1 + 52), lds32(a1 + 56), A11);
           }
+          // up to four tokens at a time: eight independent accumulator chains (hi / lo) per k-step
 #pragma unroll
-          for (int m = 0; m < TM; ++m) {
-            if (m < M) {
-              const uint32_t xrow = stg + L::ST_X + ((m * 2 + set) * 4) * 128 + 16 * g;
-              int32_t dh[4], dl[4];
+          for (int m0 = 0; m0 < TM; m0 += MP) {
+            if (m0 < M) {
+              int32_t dh[MP][4], dl[MP][4];
 #pragma unroll
               for (int j = 0; j < 4; ++j) {
-                const uint4 xv = lds128(on ? xrow + 128 * j : zero_a);
-                if (j == 0) {
-                  QL_IMMA6_0("s8", dh, acc_init, A00[0], A10[0], A01[0], A11[0], xv.x, xv.y);
-                  QL_IMMA6_0("u8", dl, acc_init, A00[0], A10[0], A01[0], A11[0], xv.z, xv.w);
-                } else {
-                  QL_IMMA6("s8", dh, A00[j], A10[j], A01[j], A11[j], xv.x, xv.y);
-                  QL_IMMA6("u8", dl, A00[j], A10[j], A01[j], A11[j], xv.z, xv.w);
+#pragma unroll
+                for (int mm = 0; mm < MP; ++mm) {
+                  const int m = m0 + mm;  // a token past M (odd M) reads stale stage words; its sums are never stored
+                  const uint32_t xrow = stg + L::ST_X + ((m * 2 + set) * 4 + j) * 128 + 16 * g;
+                  const uint4 xv = lds128(on ? xrow : zero_a);
+                  if (j == 0) {
+                    QL_IMMA6_0("s8", dh[mm], acc_init, A00[0], A10[0], A01[0], A11[0], xv.x, xv.y);
+                    QL_IMMA6_0("u8", dl[mm], acc_init, A00[0], A10[0], A01[0], A11[0], xv.z, xv.w);
+                  } else {
+                    QL_IMMA6("s8", dh[mm], A00[j], A10[j], A01[j], A11[j], xv.x, xv.y);
+                    QL_IMMA6("u8", dl[mm], A00[j], A10[j], A01[j], A11[j], xv.z, xv.w);
+                  }
                 }
               }
-              // D[q]: q = 0 (r0, group 8 set + 2c), 1 (r0, + 1), 2 (r1, 2c), 3 (r1, + 1)
-              const float2 G = lds64f(stg + L::ST_G + (m * 16 + 8 * set + 2 * c) * 4);
-              float t[4];
 #pragma unroll
-              for (int q = 0; q < 4; ++q)
-                t[q] = fmaf(__int_as_float(dh[q]) - GEMV_ACC0_F, 256.f, __int_as_float(dl[q]) - GEMV_ACC0_F);
-              acc[m][0] = fmaf(S[set][0][0] * G.x, t[0], acc[m][0]);
-              acc[m][0] = fmaf(S[set][0][1] * G.y, t[1], acc[m][0]);
-              acc[m][1] = fmaf(S[set][1][0] * G.x, t[2], acc[m][1]);
-              acc[m][1] = fmaf(S[set][1][1] * G.y, t[3], acc[m][1]);
+              for (int mm = 0; mm < MP; ++mm) {
+                const int m = m0 + mm;
+                // D[q]: q = 0 (r0, group 8 set + 2c), 1 (r0, + 1), 2 (r1, 2c), 3 (r1, + 1)
+                const float2 G = lds64f(stg + L::ST_G + (m * 16 + 8 * set + 2 * c) * 4);
+                float t[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                  t[q] = fmaf(__int_as_float(dh[mm][q]) - GEMV_ACC0_F, 256.f, __int_as_float(dl[mm][q]) - GEMV_ACC0_F);
+                acc[m][0] = fmaf(S[set][0][0] * G.x, t[0], acc[m][0]);
+                acc[m][0] = fmaf(S[set][0][1] * G.y, t[1], acc[m][0]);
+                acc[m][1] = fmaf(S[set][1][0] * G.x, t[2], acc[m][1]);
+                acc[m][1] = fmaf(S[set][1][1] * G.y, t[3], acc[m][1]);
+              }
             }
           }
         }
