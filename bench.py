@@ -38,8 +38,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM bytes per GEMV launch from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum),
 # valid only while the GEMV source is unchanged (hash of csrc/gemv.cuh at capture time).
-NCU_TRAFFIC = {"gemv_src_sha256": "2afddf42e467fc10e0f205c81da84f9875f1874a7bd3a70dcea1d47e6ba1b05e",
-               "bytes_per_launch": 83168768}  # mean over the two decode layers
+NCU_TRAFFIC = {"gemv_src_sha256": "91123622891a0731e5f78e1fdb4ee29dddddc305294d3fe144a00c509d1625db",
+               "bytes_per_launch": 83054464}  # mean over the two decode layers
 
 
 def parse_args(argv=None):
