@@ -566,15 +566,17 @@ constexpr int GEMV_MT_THREADS = 32 * (GEMV_MT_WARPS + 1);
 constexpr int GEMV_MT_CTAS_PER_SM = 3;
 
 // Stage layout of the multi-token kernel per format, for one 256-weight super-block of 64 rows:
-// codes [64 rows][CODE_ROW B] as 128-byte-swizzled boxes of 128 B, group words [64][META_ROW B],
-// group sums [8][M][8 B], x words [8 groups][M][4][16 B].  int4 and 4-bit affine codes share one
-// layout (a nibble per weight, low nibble first); 8-bit affine codes are bytes.
+// codes [64 rows][CODE_ROW B] as swizzled boxes of CODE_BOX B (128-byte swizzle; 64-byte swizzle for
+// the 64-byte rows of 2-bit codes), group words [64][META_ROW B], group sums [8][M][8 B], x words
+// [8 groups][M][4][16 B].  int4 and 4-bit affine codes share one layout (a nibble per weight, low
+// nibble first); 8-bit affine codes are bytes; 2-bit codes are 16 per word, lowest bits first.
 template <int FMT, int BITS, int G>
 struct MtLayout {
   static constexpr int CODE_ROW = FMT == FMT_INT4 ? 128 : 256 * BITS / 8;
-  static constexpr int CODE_BOXES = CODE_ROW / 128;
+  static constexpr int CODE_BOX = CODE_ROW < 128 ? CODE_ROW : 128;
+  static constexpr int CODE_BOXES = CODE_ROW / CODE_BOX;
   static constexpr int META_ROW = FMT == FMT_INT4 ? 16 : 4 * (256 / G);  // int4: 8 x u16; affine: 256/G x u32
-  static constexpr int ST_GMETA = CODE_BOXES * 64 * 128;
+  static constexpr int ST_GMETA = CODE_BOXES * 64 * CODE_BOX;
   static constexpr int ST_GSUM = ST_GMETA + 64 * META_ROW;
   static constexpr int ST_X = ST_GSUM + 512;
   static constexpr int STAGE = (ST_X + 4096 + 1023) / 1024 * 1024;
@@ -595,11 +597,11 @@ struct GemvMtParams {
 template <int FMT, int BITS, int G>
 inline constexpr int gemv_mt_smem_bytes() { return MtLayout<FMT, BITS, G>::SMEM; }
 
-// int4: w = (q - zc zs)(sc ss) with the step word per super-block; affine (4 / 8 bits, group 32 or
-// 64): w = q s + b with (s, b) bf16 per group.  Per (row, token, 32-weight slice) the integer MMA
-// gives T = sum_k A_k x_int_k with A = 16 q (nibbles) or q (bytes); then
+// int4: w = (q - zc zs)(sc ss) with the step word per super-block; affine (2 / 4 / 8 bits, group 32
+// or 64): w = q s + b with (s, b) bf16 per group.  Per (row, token, 32-weight slice) the integer MMA
+// gives T = sum_k A_k x_int_k with A = 16 q (nibbles) or q (2-bit fields, bytes); then
 //   int4:   y += S (2^-a / 16) (T - 16 Z X)
-//   affine: y += s' (2^-a / 16) T + b 2^-a X      (s' = s, or 16 s for bytes)
+//   affine: y += s' (2^-a / 16) T + b 2^-a X      (s' = s for nibbles, 16 s otherwise)
 template <int FMT, int BITS, int G>
 __global__ void __launch_bounds__(GEMV_MT_THREADS, GEMV_MT_CTAS_PER_SM)
     gemv_mt_kernel(const __grid_constant__ CUtensorMap map_codes, const __grid_constant__ CUtensorMap map_gmeta,
@@ -642,7 +644,7 @@ __global__ void __launch_bounds__(GEMV_MT_THREADS, GEMV_MT_CTAS_PER_SM)
         mbar_arrive_expect_tx(bar_full(s), tx);
 #pragma unroll
         for (int bx = 0; bx < L::CODE_BOXES; ++bx)
-          tma_load_2d(st + bx * 8192, &map_codes, bar_full(s), (sb0 + i) * L::CODE_ROW + bx * 128,
+          tma_load_2d(st + bx * 64 * L::CODE_BOX, &map_codes, bar_full(s), (sb0 + i) * L::CODE_ROW + bx * L::CODE_BOX,
                       (int32_t)(rg * 64));
         tma_load_2d(st + L::ST_GMETA, &map_gmeta, bar_full(s), (sb0 + i) * L::META_ROW, (int32_t)(rg * 64));
       };
@@ -747,6 +749,17 @@ __global__ void __launch_bounds__(GEMV_MT_THREADS, GEMV_MT_CTAS_PER_SM)
             const uint32_t w0 = lds32(stg + r0 * 128 + coff), w1 = lds32(stg + r1 * 128 + coff);
             e0 = (w0 << 4) & 0xF0F0F0F0u; e1 = (w1 << 4) & 0xF0F0F0F0u;
             o0 = w0 & 0xF0F0F0F0u; o1 = w1 & 0xF0F0F0F0u;
+          } else if constexpr (BITS == 2) {
+            // 2-bit: slice gg is 8 B of the 64-byte row (64-byte swizzle: 16-byte chunk ^ (row / 2) % 4);
+            // lane c takes the half-word of k = 8c .. 8c + 7, spreads its nibbles to bytes (one byte
+            // permute, one shift-or) and splits even and odd k with two masks
+            const uint32_t off = ((((uint32_t)gg >> 1) ^ (((uint32_t)r0 >> 1) & 3u)) << 4) + 8 * (gg & 1) + 4 * (c >> 1);
+            const uint32_t sel = (c & 1) ? 0x4342u : 0x4140u;
+            const uint32_t t0 = __byte_perm(lds32(stg + r0 * 64 + off), 0u, sel);
+            const uint32_t t1 = __byte_perm(lds32(stg + r1 * 64 + off), 0u, sel);
+            const uint32_t u0 = (t0 | (t0 << 4)) & 0x0F0F0F0Fu, u1 = (t1 | (t1 << 4)) & 0x0F0F0F0Fu;
+            e0 = u0 & 0x03030303u; e1 = u1 & 0x03030303u;
+            o0 = (u0 >> 2) & 0x03030303u; o1 = (u1 >> 2) & 0x03030303u;
           } else {  // bytes: slice gg is 32 B of box gg / 4; lane c takes bytes 8c .. 8c + 7
             const uint32_t ch = (uint32_t)(2 * (gg & 3) + (c >> 1));
             const uint32_t off = (uint32_t)(gg >> 2) * 8192 + ((ch ^ sw) << 4) + 8 * (c & 1);
@@ -777,7 +790,7 @@ __global__ void __launch_bounds__(GEMV_MT_THREADS, GEMV_MT_CTAS_PER_SM)
           } else {
             // slice gg lies in affine group gg * 32 / G of the super-block; its word holds (s, b) bf16
             const uint32_t gw0g = gw0[gg * 32 / G], gw1g = gw1[gg * 32 / G];
-            constexpr float SF = BITS == 8 ? 16.f : 1.f;  // bytes carry q, nibbles 16 q
+            constexpr float SF = BITS == 4 ? 1.f : 16.f;  // nibbles carry 16 q, 2-bit fields and bytes q
             const float s0 = bf16_bits_to_f32(gw0g) * SF, b0 = bf16_bits_to_f32(gw0g >> 16);
             const float s1 = bf16_bits_to_f32(gw1g) * SF, b1 = bf16_bits_to_f32(gw1g >> 16);
             // b 2^-a X = -b (2^-a/16)(-16 X)

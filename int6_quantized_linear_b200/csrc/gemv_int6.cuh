@@ -1,4 +1,4 @@
-// Tensor-core decode GEMV for the symmetric int6 format at 1 <= M <= 7 tokens.
+// Tensor-core decode GEMV for the symmetric int6 format at 1 <= M <= 8 tokens.
 //
 // Format (int6 sibling of the nested-superscale int4 layout; "Nested superscale
 // quantization", int6 paragraph): 6-bit two's-complement codes, four per three

@@ -167,13 +167,12 @@ ql_status launch_gemm(const ql_desc *d, const ql_packed_const *w, const void *x,
 }
 
 // Which GEMV calls run on the tensor-core GEMM (measured faster there on the benchmark layers:
-// affine M=32 70-74 us vs 537-551 us, int6 M=8 198 us vs 284 us on the CUDA-core kernel): int6 from
-// M = 8; affine from M = 9 when a multi-token tensor-core GEMV exists for it (4 / 8 bits, group 32 /
-// 64), else from M = 8.  int4 has tensor-core GEMVs up to M = 8.
+// affine M=32 70-74 us vs 537-551 us on the CUDA-core kernel): affine from M = 9 when a multi-token
+// tensor-core GEMV exists for it (group 32 / 64, K a multiple of 256), else from M = 8.  int4 and int6
+// have tensor-core GEMVs over their whole GEMV range (M <= 8).
 inline bool gemv_runs_on_gemm(const ql_desc *d, int64_t M) {
-  if (d->fmt == QL_INT6_SYM) return M >= 8;
-  if (d->fmt == QL_AFFINE_U32) {  // 4- and 8-bit affine with group 32 / 64 have the multi-token kernel up to M = 8
-    const bool mt = (d->bits == 4 || d->bits == 8) && (d->group == 32 || d->group == 64) && d->K % 256 == 0;
+  if (d->fmt == QL_AFFINE_U32) {  // 2-, 4- and 8-bit affine with group 32 / 64: multi-token kernel up to M = 8
+    const bool mt = (d->group == 32 || d->group == 64) && d->K % 256 == 0;
     return M >= (mt ? 9 : 8);
   }
   return false;
@@ -190,7 +189,7 @@ template <int FMT, int BITS>
 ql_status launch_gemm(const ql_desc *d, const ql_packed_const *w, const void *x, int64_t M, const void *bias,
                       void *y, void *workspace, cudaStream_t st, int sms);
 
-// Multi-token tensor-core GEMV (int4 at 2..8 tokens; 4- and 8-bit affine with group 32 or 64 at
+// Multi-token tensor-core GEMV (int4 at 2..8 tokens; 2-, 4- and 8-bit affine with group 32 or 64 at
 // 1..8 tokens): x preparation, then the streaming kernel as its programmatic dependent.
 template <int FMT, int BITS, int G>
 ql_status launch_gemv_mt(const ql_desc *d, const ql_packed_const *w, const __nv_bfloat16 *xb, int64_t M,
@@ -226,9 +225,9 @@ ql_status launch_gemv_mt(const ql_desc *d, const ql_packed_const *w, const __nv_
   p.y = yb;
   const uint64_t code_row = FMT == FMT_INT4 ? (uint64_t)K / 2 : (uint64_t)K * BITS / 8;
   const uint64_t meta_row = FMT == FMT_INT4 ? (uint64_t)K / 16 : (uint64_t)K / G * 4;
-  CUtensorMap mc, mg;  // codes: boxes of 64 rows x 128 bytes, 128-byte swizzle; group words: 64 rows x META_ROW
-  if (!encode_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->codes, code_row, (uint64_t)N, code_row, 128, 64,
-                 CU_TENSOR_MAP_SWIZZLE_128B) ||
+  CUtensorMap mc, mg;  // codes: boxes of 64 rows x CODE_BOX bytes, swizzled; group words: 64 rows x META_ROW
+  if (!encode_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->codes, code_row, (uint64_t)N, code_row, L::CODE_BOX, 64,
+                 L::CODE_BOX == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B) ||
       !encode_2d(&mg, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->gmeta, meta_row, (uint64_t)N, meta_row, L::META_ROW, 64,
                  CU_TENSOR_MAP_SWIZZLE_NONE))
     return QL_ERR_CUDA;
@@ -323,13 +322,13 @@ ql_status launch_gemv(const ql_desc *d, const ql_packed_const *w, const void *x,
   if constexpr (FMT == FMT_INT4) {
     if (M >= 2) return launch_gemv_mt<FMT_INT4, 4, 32>(d, w, xb, M, bb, yb, workspace, st, sms);
   }
-  if constexpr (FMT == FMT_INT6) {  // M <= 7 here
+  if constexpr (FMT == FMT_INT6) {  // M <= 8
     if (M == 1) return launch_gemv_int6<1>(d, w, xb, M, bb, yb, workspace, st, sms);
     if (M == 2) return launch_gemv_int6<2>(d, w, xb, M, bb, yb, workspace, st, sms);
     if (M <= 4) return launch_gemv_int6<4>(d, w, xb, M, bb, yb, workspace, st, sms);
     return launch_gemv_int6<8>(d, w, xb, M, bb, yb, workspace, st, sms);
   }
-  if constexpr (FMT == FMT_AFFINE && (BITS == 4 || BITS == 8)) {
+  if constexpr (FMT == FMT_AFFINE) {  // bits 2, 4, 8
     if (d->K % 256 == 0 && d->group == 64) return launch_gemv_mt<FMT_AFFINE, BITS, 64>(d, w, xb, M, bb, yb, workspace, st, sms);
     if (d->K % 256 == 0 && d->group == 32) return launch_gemv_mt<FMT_AFFINE, BITS, 32>(d, w, xb, M, bb, yb, workspace, st, sms);
   }

@@ -146,14 +146,28 @@ def test_deterministic_and_in_bounds(cuda):
         assert np.all(b[:pad] == 0x7B7B) and np.all(b[pad + M * 1000:] == 0x7B7B)
 
 
+@pytest.mark.parametrize("bits,group", [(2, 64), (2, 32)])
+@pytest.mark.parametrize("N,K", [(200, 1536), (64, 256), (700, 4096)])
+def test_gemv_affine2_multi_token(cuda, bits, group, N, K):
+    """2-bit affine on the multi-token tensor-core GEMV (64-byte swizzled code rows) at M = 1..8,
+    with and without the K split; repeated runs give identical bits."""
+    L = Layer("affine", N, K, seed=13 * N + K + group, bits=bits, group=group)
+    w_ref = L.oracle_w()
+    for M in range(1, 9):
+        xb, xd = x_dev(K, M, seed=200 + M)
+        y = run_gemv(L, xd, M)
+        assert_close(y, OC.matmul_f64(xb, w_ref), f"affine{bits} g{group} gemv N={N} K={K} M={M}")
+        assert np.array_equal(y, run_gemv(L, xd, M))
+
+
 @pytest.mark.parametrize("N,K", [(200, 1536), (64, 256), (1000, 5120)])
 def test_gemv_int6_every_token_count(cuda, N, K):
-    """int6 tensor-core GEMV at each M it serves (1..7: four token buckets), with and without the
+    """int6 tensor-core GEMV at each M it serves (1..8: four token buckets), with and without the
     split of K over CTAs; repeated runs give identical bits; the bias variant adds bias[n]."""
     L = Layer("int6", N, K, seed=11 * N + K)
     w_ref = L.oracle_w()
     bias_b = synth.activations(N + K, 1, N)[0]
-    for M in range(1, 8):
+    for M in range(1, 9):
         xb, xd = x_dev(K, M, seed=100 + M)
         y = run_gemv(L, xd, M)
         y_ref = OC.matmul_f64(xb, w_ref)
