@@ -197,37 +197,41 @@ ql_status qlinear_quantize_meta(const ql_desc *desc, const float *scale, const f
 
 /* Bytes of caller-provided device workspace qlinear_gemv needs for `desc`
  * and M (host-only, no CUDA call): 4*M*K for x in the order the tensor-core
- * fragments read it, 8*M*K/32 for two sums per 32-weight group,
- * 4*4096*64*M for the partial sums of a K split and 4*ceil(N/64) for its
- * counters, each part rounded up to 256 bytes; for int6 / affine at M >= 8
- * (those calls run on the GEMM) at least qlinear_gemm_workspace_bytes().
+ * fragments read it, 8*M*K/32 for the per-group x scales and sums,
+ * 4*4096*64*M for the partial sums of a K split and 4*ceil(N/16) for its
+ * counters, each part rounded up to 256 bytes; for affine calls that run on
+ * the GEMM (below) at least qlinear_gemm_workspace_bytes().
  * Errors: QL_ERR_NULL, QL_ERR_SHAPE, QL_ERR_RANGE, QL_ERR_UNSUPPORTED. */
 ql_status qlinear_gemv_workspace_bytes(const ql_desc *desc, int64_t M, size_t *bytes);
 
 /* Decode-shaped layer, HBM-bound: y[M][N] (bf16) = x[M][K] (bf16) . W^T,
  * fp32 scales and accumulation, one nearest-even rounding to bf16 at the end.
  * 1 <= M <= 8 for int4 / int6; 1 <= M <= 32 for affine.
- *  - int4, 1 <= M <= 8: two launches.  A short pass turns each 32-element
- *    group of x into 16-bit fixed point (x_int = rint(x * 2^a), the group's
- *    max |x| scaled into [2^14, 2^15)), split into high and low bytes in the
- *    order the tensor-core fragments read them, with the group's sum; then
- *    the streaming kernel multiplies the codes (as u8 times 16) by those bytes
- *    on the integer tensor core (mma.sync m16n8k32, exact s32 sums) and
- *    applies scale and zero once per (row, group[, token]) in fp32.  M = 1
- *    uses a diagonal x operand (one MMA column per group); M >= 2 uses the
- *    tokens as MMA columns and may split K over CTAs, adding the parts in a
- *    fixed order through the workspace.
- *  - int6 / affine, M < 8: one launch, exact binary32 weights, fp32 FMA.
- *  - int6 / affine, M >= 8: runs as qlinear_gemm (faster there).
+ *  - Tensor-core path (int4 and int6 at every M; affine with group 32 or 64
+ *    and K % 256 == 0 at M <= 8): two launches.  A short pass turns each x
+ *    group (32 elements; 16 for int6) into 16-bit fixed point (x_int =
+ *    rint(x * 2^a), the group's max |x| scaled into [2^14, 2^15)), split
+ *    into high and low bytes in the order the tensor-core fragments read
+ *    them, with the group's scale (and sum); then the streaming kernel
+ *    multiplies the codes (as u8 or s8 bytes: 16q for nibbles, 4q for int6,
+ *    q for 2- and 8-bit fields) by those bytes on the integer tensor core
+ *    (mma.sync m16n8k32, exact s32 sums) and applies scale (and zero or
+ *    bias) once per (row, group[, token]) in fp32.  int4 at M = 1 and int6
+ *    use a diagonal x operand (one MMA column per weight group); int4 at
+ *    M >= 2 and affine use the tokens as MMA columns.  K may be split over
+ *    warps or CTAs, the parts added in a fixed order through the workspace.
+ *  - Affine with other groups, or K % 256 != 0, at M < 8: one launch, exact
+ *    binary32 weights, fp32 FMA.
+ *  - Affine at M >= 9 (M >= 8 on the path above): runs as qlinear_gemm.
  * ExecuTorch page above, "Quant schema update" (the int4 / int6 formats)
  * and the review's "Things done well" (the decode kernel's per-super-block
  * step word and full-warp trip counts).
  * `workspace`: at least qlinear_gemv_workspace_bytes(), 256-byte aligned,
  * caller-owned, overwritten; calls sharing one workspace must not overlap on
- * the GPU.  Consecutive int4 calls on one stream chain by programmatic
- * dependent launch: a call's weight stream may start while the previous
- * kernel on the stream drains, and its preparation pass waits for that
- * kernel before it reads x or writes the workspace.
+ * the GPU.  Consecutive tensor-core calls on one stream chain by
+ * programmatic dependent launch: a call's weight stream may start while the
+ * previous kernel on the stream drains, and its preparation pass waits for
+ * that kernel before it reads x or writes the workspace.
  * Errors: QL_ERR_NULL, QL_ERR_SHAPE (also: workspace too small),
  * QL_ERR_ALIGN, QL_ERR_RANGE, QL_ERR_UNSUPPORTED, QL_ERR_CUDA. */
 ql_status qlinear_gemv(const ql_desc *desc, const ql_packed_const *w,
