@@ -1,10 +1,11 @@
 // gemv.cuh -- decode-shaped layer y[M][N] = x[M][K] . W^T for small M.
 //
-// Simple form: one warp per output row; lane l takes chunks l, l+32, ... of
-// the row (32 weights each: one int4 group, 16-byte coalesced loads), decodes
-// the exact binary32 weights and accumulates x*w in fp32; a warp-shuffle
-// reduction finishes the row.  The trip count over chunks is the same for
-// every lane of a warp, so full-mask shuffles are always reached.
+// Simple form (affine weights whose group size has no tensor-core kernel):
+// one warp per output row; lane l takes chunks l, l+32, ... of the row (32
+// weights each, coalesced loads), decodes the exact binary32 weights and
+// accumulates x*w in fp32; a warp-shuffle reduction finishes the row.  The
+// trip count over chunks is the same for every lane of a warp, so full-mask
+// shuffles are always reached.
 #pragma once
 #include "gemm_prep.cuh"
 #include "pack_dequant.cuh"

@@ -395,20 +395,24 @@ ql_status launch_gemv(const ql_desc *d, const ql_packed_const *w, const void *x,
       return launched();
     }
   }
-  const WeightPtrs p = make_ptrs(d, w);
-  const int64_t rows_per_block = 8;
-  int64_t g = (d->N + rows_per_block - 1) / rows_per_block;
-  const int64_t cap = (int64_t)sms * 16;
-  if (g > cap) g = cap;
-  if (M == 1)
-    gemv_simple_kernel<FMT, BITS, 1><<<(int)g, 256, 0, st>>>(p, d->N, xb, (int)M, bb, yb);
-  else if (M == 2)
-    gemv_simple_kernel<FMT, BITS, 2><<<(int)g, 256, 0, st>>>(p, d->N, xb, (int)M, bb, yb);
-  else if (M <= 4)
-    gemv_simple_kernel<FMT, BITS, 4><<<(int)g, 256, 0, st>>>(p, d->N, xb, (int)M, bb, yb);
-  else
-    gemv_simple_kernel<FMT, BITS, 8><<<(int)g, 256, 0, st>>>(p, d->N, xb, (int)M, bb, yb);
-  return launched();
+  if constexpr (FMT == FMT_AFFINE) {  // groups without the multi-token kernel, M < 8: CUDA cores
+    const WeightPtrs p = make_ptrs(d, w);
+    const int64_t rows_per_block = 8;
+    int64_t g = (d->N + rows_per_block - 1) / rows_per_block;
+    const int64_t cap = (int64_t)sms * 16;
+    if (g > cap) g = cap;
+    if (M == 1)
+      gemv_simple_kernel<FMT, BITS, 1><<<(int)g, 256, 0, st>>>(p, d->N, xb, (int)M, bb, yb);
+    else if (M == 2)
+      gemv_simple_kernel<FMT, BITS, 2><<<(int)g, 256, 0, st>>>(p, d->N, xb, (int)M, bb, yb);
+    else if (M <= 4)
+      gemv_simple_kernel<FMT, BITS, 4><<<(int)g, 256, 0, st>>>(p, d->N, xb, (int)M, bb, yb);
+    else
+      gemv_simple_kernel<FMT, BITS, 8><<<(int)g, 256, 0, st>>>(p, d->N, xb, (int)M, bb, yb);
+    return launched();
+  } else {
+    return QL_ERR_UNSUPPORTED;  // int4 and int6 returned above for every M in range
+  }
 }
 
 }  // namespace
