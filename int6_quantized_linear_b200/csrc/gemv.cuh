@@ -134,60 +134,63 @@ QL_DEVI int atomic_add_acq_rel_gpu(int *addr, int v) {
 QL_DEVI void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 QL_DEVI void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
-// One thread per 32-element group of x: fixed-point conversion, byte split in fragment order, sum.
-// Chunk (j, kind) of group grp is the register quad its feeding lane loads: the high-byte and low-byte
-// words of k = 8j + kind + {0, 2, 4, 6}, each paired with a zero word so that one 16-byte load gives
-// the B pairs of two MMAs -- (x, 0) for groups 0-3 (their lanes feed b0), (0, x) for groups 4-7 (b1).
-// It also zeroes the first n_counters tile counters of the K split.
+// Four lanes per 32-element group of x (lane c holds k = 8c .. 8c + 7): fixed-point conversion with
+// the group's max and sum by shuffles, byte split in fragment order.  Chunk (j, kind) of group grp
+// is the register quad its feeding lane loads: the high-byte and low-byte words of
+// k = 8j + kind + {0, 2, 4, 6}, each paired with a zero word so that one 16-byte load gives the B
+// pairs of two MMAs -- (x, 0) for groups 0-3 (their lanes feed b0), (0, x) for groups 4-7 (b1).
+// Lane c writes the two chunks (j = c, kind = 0 / 1).  It also zeroes the first n_counters tile
+// counters of the K split.
 __global__ void __launch_bounds__(256) gemv_xprep_kernel(const __nv_bfloat16 *x, int64_t M, int64_t K,
                                                          int64_t n_counters, GemvWorkspace ws) {
   pdl_launch_dependents();  // the streaming kernel may start fetching weights now
   pdl_wait();               // x (and this workspace) may belong to the kernel launched before this one
+  const int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (t < n_counters) ws.counters[t] = 0;
   const int64_t ng = K / 32;
-  const int64_t gi = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;  // over max(M * ng, n_counters)
-  if (gi < n_counters) ws.counters[gi] = 0;
-  if (gi >= M * ng) return;
-  const uint4 *src = reinterpret_cast<const uint4 *>(x) + 4 * gi;  // 32 bf16 = 64 bytes
-  float xs[32];
+  const int64_t gi = t >> 2;  // over M * ng groups
+  const int c = (int)(t & 3);
+  const bool live = gi < M * ng;  // every lane takes part in the shuffles
+  uint4 v = make_uint4(0u, 0u, 0u, 0u);
+  if (live) v = __ldg(reinterpret_cast<const uint4 *>(x) + 4 * gi + c);  // 8 bf16 = 16 bytes
+  const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+  float xs[8];
   float amax = 0.f;
 #pragma unroll
-  for (int t = 0; t < 4; ++t) {
-    const uint4 v = __ldg(src + t);
-    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      xs[8 * t + 2 * j] = bf16_bits_to_f32(u[j]);
-      xs[8 * t + 2 * j + 1] = bf16_bits_to_f32(u[j] >> 16);
-      amax = fmaxf(amax, fmaxf(fabsf(xs[8 * t + 2 * j]), fabsf(xs[8 * t + 2 * j + 1])));
-    }
+  for (int i = 0; i < 4; ++i) {
+    xs[2 * i] = bf16_bits_to_f32(u[i]);
+    xs[2 * i + 1] = bf16_bits_to_f32(u[i] >> 16);
+    amax = fmaxf(amax, fmaxf(fabsf(xs[2 * i]), fabsf(xs[2 * i + 1])));
   }
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
   const int a = scale_exponent(amax, 14);  // max |x_int| < 2^15
   const float sc = exp2i(a);
-  int xi[32];
+  int xi[8];
   int sum = 0;
 #pragma unroll
-  for (int k = 0; k < 32; ++k) {
+  for (int k = 0; k < 8; ++k) {
     xi[k] = __float2int_rn(xs[k] * sc);
     sum += xi[k];
   }
+  sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+  sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+  if (!live) return;
   // group gi = (m, super-block sb, group-in-block grp): chunk (j, kind) goes to [m][sb][j][kind][grp]
   const int64_t grp = gi & 7, msb = gi >> 3;
   uint4 *dst = ws.xq + msb * 64 + grp;
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
+  for (int kind = 0; kind < 2; ++kind) {
+    uint32_t hi = 0, lo = 0;
 #pragma unroll
-    for (int kind = 0; kind < 2; ++kind) {
-      uint32_t hi = 0, lo = 0;
-#pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        const int v = xi[8 * j + 2 * b + kind];
-        hi |= ((uint32_t)(v >> 8) & 0xffu) << (8 * b);
-        lo |= ((uint32_t)v & 0xffu) << (8 * b);
-      }
-      dst[8 * (2 * j + kind)] = grp < 4 ? make_uint4(hi, 0u, lo, 0u) : make_uint4(0u, hi, 0u, lo);
+    for (int b = 0; b < 4; ++b) {
+      const int val = xi[2 * b + kind];
+      hi |= ((uint32_t)(val >> 8) & 0xffu) << (8 * b);
+      lo |= ((uint32_t)val & 0xffu) << (8 * b);
     }
+    dst[8 * (2 * c + kind)] = grp < 4 ? make_uint4(hi, 0u, lo, 0u) : make_uint4(0u, hi, 0u, lo);
   }
-  ws.gsum[gi] = make_float2(exp2i(-a) * 0.0625f, -16.f * (float)sum);
+  if (c == 0) ws.gsum[gi] = make_float2(exp2i(-a) * 0.0625f, -16.f * (float)sum);
 }
 
 // A byte of a metadata word as a float: 2^23 + b, to be fused into an FMA with -2^23 * step.

@@ -305,29 +305,49 @@ __global__ void __launch_bounds__(256) dequant_kernel(WeightPtrs p, int64_t N, v
 // step_f is the fp16-rounded step, so encoder and decoder reconstruct with the same value; the
 // divisions are IEEE binary32, rint rounds half to even, a zero max gives step 0 and codes 0.
 // A non-finite value (or a negative one for int4) sets QL_DEV_RANGE.
-template <bool SIGNED>
-__global__ void __launch_bounds__(256) quantize_meta_kernel(const float *v, int64_t rows, int64_t G, int per,
-                                                            uint8_t *codes, uint16_t *steps) {
-  const int64_t S = G / per;
+template <bool SIGNED, int PER>
+__global__ void __launch_bounds__(256) quantize_meta_kernel(const float *v0, const float *v1, int64_t rows, int64_t G,
+                                                            uint8_t *codes0, uint8_t *codes1, uint16_t *steps0,
+                                                            uint16_t *steps1) {
+  // blockIdx.y picks the array (int4: scale, zero); thread t = (row, super-block) owns elements
+  // t * PER .. t * PER + PER - 1, read as 16-byte vectors, and writes its PER codes in one store
+  const float *v = blockIdx.y ? v1 : v0;
+  uint8_t *codes = blockIdx.y ? codes1 : codes0;
+  uint16_t *steps = blockIdx.y ? steps1 : steps0;
   const int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-  if (t >= rows * S) return;
-  const int64_t r = t / S, b = t - r * S;
-  const float *src = v + r * G + b * per;
+  if (t >= rows * (G / PER)) return;
+  const float4 *src = reinterpret_cast<const float4 *>(v) + t * (PER / 4);
+  float x[PER];
+#pragma unroll
+  for (int i = 0; i < PER / 4; ++i) {
+    const float4 f = __ldg(src + i);
+    x[4 * i] = f.x; x[4 * i + 1] = f.y; x[4 * i + 2] = f.z; x[4 * i + 3] = f.w;
+  }
   float m = 0.f;
   bool bad = false;
-  for (int i = 0; i < per; ++i) {
-    const float x = src[i];
-    bad |= !isfinite(x) || (!SIGNED && x < 0.f);
-    m = fmaxf(m, SIGNED ? fabsf(x) : x);
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    bad |= !isfinite(x[i]) || (!SIGNED && x[i] < 0.f);
+    m = fmaxf(m, SIGNED ? fabsf(x[i]) : x[i]);
   }
   if (bad) atomicOr(&g_ql_status, QL_DEV_RANGE);
   const __half st = __float2half_rn(__fdiv_rn(m, SIGNED ? 127.f : 255.f));
   const float sf = __half2float(st);
   const float lo = SIGNED ? -127.f : 0.f, hi = SIGNED ? 127.f : 255.f;
-  for (int i = 0; i < per; ++i) {
-    const float q = sf > 0.f ? fminf(hi, fmaxf(lo, rintf(__fdiv_rn(src[i], sf)))) : 0.f;
-    codes[r * G + b * per + i] = SIGNED ? (uint8_t)(int8_t)(int)q : (uint8_t)(int)q;
+  uint32_t w[PER / 4];
+#pragma unroll
+  for (int i = 0; i < PER / 4; ++i) w[i] = 0u;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const float q = sf > 0.f ? fminf(hi, fmaxf(lo, rintf(__fdiv_rn(x[i], sf)))) : 0.f;
+    const uint32_t b = SIGNED ? (uint32_t)(uint8_t)(int8_t)(int)q : (uint32_t)(uint8_t)(int)q;
+    w[i / 4] |= b << (8 * (i % 4));
   }
-  steps[r * S + b] = __half_as_ushort(st);
+  if constexpr (PER == 8) {
+    reinterpret_cast<uint2 *>(codes)[t] = make_uint2(w[0], w[1]);
+  } else {
+    reinterpret_cast<uint4 *>(codes)[t] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+  steps[t] = __half_as_ushort(st);
 }
 }  // namespace ql

@@ -344,7 +344,7 @@ ql_status launch_gemv(const ql_desc *d, const ql_packed_const *w, const void *x,
       P = std::min<int64_t>(P, std::max<int64_t>(1, (int64_t)GEMV_MT_MAX_CTAS * 64 / 16 / n_tiles));
       const int64_t n_counters = P > 1 ? n_tiles : 0;
       {  // programmatic dependent of whatever precedes it on the stream (it waits before reading x)
-        const int64_t threads = std::max<int64_t>(ng, n_counters);
+        const int64_t threads = std::max<int64_t>(4 * ng, n_counters);  // four lanes per group
         cudaLaunchConfig_t pc = {};
         pc.gridDim = dim3((unsigned)((threads + 255) / 256));
         pc.blockDim = dim3(256);
@@ -743,17 +743,16 @@ ql_status qlinear_quantize_meta(const ql_desc *d, const float *scale, const floa
   const int64_t N = d->N, K = d->K;
   const int per = i4 ? 8 : 16;                  // groups per 256-weight super-block
   const int64_t G = K / (i4 ? 32 : 16);         // groups per row
-  const int64_t threads = N * (G / per);
-  const int blocks = (int)((threads + 255) / 256);
-  if (i4) {
-    quantize_meta_kernel<false><<<blocks, 256, 0, s>>>(scale, N, G, per, static_cast<uint8_t *>(out->meta0),
-                                                       static_cast<uint16_t *>(out->step0));
-    quantize_meta_kernel<false><<<blocks, 256, 0, s>>>(zero, N, G, per, static_cast<uint8_t *>(out->meta1),
-                                                       static_cast<uint16_t *>(out->step1));
-  } else {
-    quantize_meta_kernel<true><<<blocks, 256, 0, s>>>(scale, N, G, per, static_cast<uint8_t *>(out->meta0),
-                                                      static_cast<uint16_t *>(out->step0));
-  }
+  const int64_t threads = N * (G / per);        // one per (row, super-block)
+  const unsigned blocks = (unsigned)((threads + 255) / 256);
+  auto *c0 = static_cast<uint8_t *>(out->meta0);
+  auto *s0 = static_cast<uint16_t *>(out->step0);
+  if (i4)  // scale and zero fields in one launch (grid y)
+    quantize_meta_kernel<false, 8><<<dim3(blocks, 2), 256, 0, s>>>(scale, zero, N, G, c0,
+                                                                  static_cast<uint8_t *>(out->meta1), s0,
+                                                                  static_cast<uint16_t *>(out->step1));
+  else
+    quantize_meta_kernel<true, 16><<<dim3(blocks, 1), 256, 0, s>>>(scale, scale, N, G, c0, c0, s0, s0);
   return launched();
 }
 
