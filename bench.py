@@ -38,7 +38,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM bytes per GEMV launch from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum),
 # valid only while the GEMV source is unchanged (hash of csrc/gemv.cuh at capture time).
-NCU_TRAFFIC = {"gemv_src_sha256": "ed86696bf3f45c13fe0d9d832962cfa919e19faafcd5097c547ac44c6795405d",
+NCU_TRAFFIC = {"gemv_src_sha256": "41625de9a5f893f03e99271b35e9db4bc62ce5cad92590c496b21927c81056ee",
                "bytes_per_launch": 83054464}  # mean over the two decode layers
 
 
