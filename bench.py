@@ -21,6 +21,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import os
 import statistics
@@ -38,7 +39,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM bytes per GEMV launch from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum),
 # valid only while the GEMV source is unchanged (hash of csrc/gemv.cuh at capture time).
-NCU_TRAFFIC = {"gemv_src_sha256": "41625de9a5f893f03e99271b35e9db4bc62ce5cad92590c496b21927c81056ee",
+NCU_TRAFFIC = {"gemv_src_sha256": "ae072c352b994a98ad5c91b47f7f268d7cab37c4c3f7e62bffbb3aed4b0a0f9c",
                "bytes_per_launch": 83054464}  # mean over the two decode layers
 
 
@@ -178,8 +179,12 @@ def gemv_bytes(K: int, N: int, M: int = 1) -> int:
 
 
 def gemv_src_sha():
-    with open(os.path.join(ROOT, "int6_quantized_linear_b200", "csrc", "gemv.cuh"), "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()
+    """Hash of the GEMV source with its // comments removed: any code change invalidates the ncu
+    traffic figure, a comment edit does not."""
+    with open(os.path.join(ROOT, "int6_quantized_linear_b200", "csrc", "gemv.cuh")) as f:
+        lines = (re.sub(r"//.*", "", line).rstrip() for line in f)
+        code = "\n".join(line for line in lines if line)
+    return hashlib.sha256(code.encode()).hexdigest()
 
 
 # ---------------------------------------------------------------------------

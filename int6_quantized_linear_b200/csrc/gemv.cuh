@@ -499,7 +499,8 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS, GEMV_CTAS_PER_SM)
 
 
 // ===========================================================================
-// Tensor-core decode GEMV for int4 at 2 <= M <= 8 tokens.
+// Tensor-core decode GEMV with the tokens as MMA columns: int4 at 2 <= M <= 8, and 2-, 4- and 8-bit
+// affine (group 32 or 64) at 1 <= M <= 8.
 //
 // The same integer MMA (m16n8k32, u8 codes x16 against the high / low bytes of
 // 16-bit fixed-point x) with the 8 MMA columns as the tokens (a dense B):
