@@ -97,11 +97,14 @@ __global__ void __launch_bounds__(256) gemv_simple_kernel(WeightPtrs p, int64_t 
 // ===========================================================================
 
 constexpr int GEMV_MT_MAX_CTAS = 4096;  // bound on the CTAs of one multi-token launch (sizes its partial sums)
+constexpr int GEMV_XBLOB = 1088;         // M = 1 x block per super-block: 8 group sums (64 B) + x words (1 KB)
 
 struct GemvWorkspace {
-  uint4 *xq;        // M = 1: [K/256 super-blocks][4 j][2 kinds][8 groups][16 B] B-operand pairs (gemv_xprep_kernel)
+  uint4 *xq;        // M = 1: [K/256 super-blocks] blocks of GEMV_XBLOB bytes: 8 x (2^-a/16, -16 X) float2, then
+                    //        [4 j][2 kinds][8 groups][16 B] B-operand pairs (gemv_xprep_kernel); the blocks run
+                    //        on into the gsum region, which directly follows (4K is a multiple of 256)
                     // M > 1: [K/32 groups][M tokens][4][16 B] B-operand words (gemv_xprep_mt_kernel)
-  float2 *gsum;     // M = 1: [K/32]; M > 1: [K/32][M]: (2^-a_g / 16, -16 * sum x_int)
+  float2 *gsum;     // M > 1: [K/32][M]: (2^-a_g / 16, -16 * sum x_int); M = 1: the tail of the xq blocks
   float *partial;   // M = 1: [16-row tile][part][16 rows]; M > 1: [CTA][M][64 rows]: sums of one K range
   int *counters;    // parts finished so far: M = 1 per 16-row tile, M > 1 per 64-row group
 };
@@ -176,9 +179,10 @@ __global__ void __launch_bounds__(256) gemv_xprep_kernel(const __nv_bfloat16 *x,
   sum += __shfl_xor_sync(0xffffffffu, sum, 1);
   sum += __shfl_xor_sync(0xffffffffu, sum, 2);
   if (!live) return;
-  // group gi = (m, super-block sb, group-in-block grp): chunk (j, kind) goes to [m][sb][j][kind][grp]
+  // group gi = (m, super-block sb, group-in-block grp): per (m, sb) one block of GEMV_XBLOB bytes,
+  // the eight groups' sums then chunk (j, kind) at [j][kind][grp], so one bulk copy fetches both
   const int64_t grp = gi & 7, msb = gi >> 3;
-  uint4 *dst = ws.xq + msb * 64 + grp;
+  uint4 *dst = ws.xq + msb * (GEMV_XBLOB / 16) + 4 + grp;
 #pragma unroll
   for (int kind = 0; kind < 2; ++kind) {
     uint32_t hi = 0, lo = 0;
@@ -190,7 +194,7 @@ __global__ void __launch_bounds__(256) gemv_xprep_kernel(const __nv_bfloat16 *x,
     }
     dst[8 * (2 * c + kind)] = grp < 4 ? make_uint4(hi, 0u, lo, 0u) : make_uint4(0u, hi, 0u, lo);
   }
-  if (c == 0) ws.gsum[gi] = make_float2(exp2i(-a) * 0.0625f, -16.f * (float)sum);
+  if (c == 0) reinterpret_cast<float2 *>(ws.xq)[msb * (GEMV_XBLOB / 8) + grp] = make_float2(exp2i(-a) * 0.0625f, -16.f * (float)sum);
 }
 
 // A byte of a metadata word as a float: 2^23 + b, to be fused into an FMA with -2^23 * step.
@@ -266,6 +270,7 @@ constexpr int GEMV_WARPS = 4;  // warps per CTA: GEMV_WARPS / parts tiles, each 
 // one stage = one super-block of a 16-row tile: codes (16 rows x 128 B, 128-byte swizzle), the
 // tile's group words [16 rows][16 B], the super-block's 8 group sums, its x pairs [4 j][2 kinds][8 groups][16 B]
 constexpr int GEMV_ST_CODES = 0, GEMV_ST_GMETA = 2048, GEMV_ST_GSUM = 2304, GEMV_ST_X = 2368;
+static_assert(GEMV_ST_X - GEMV_ST_GSUM == 64 && GEMV_XBLOB == 64 + 1024, "one copy fills sums and x");
 constexpr int GEMV_STAGE_BYTES = 4096;      // multiple of 1024 (the swizzle atom)
 constexpr uint32_t GEMV_STAGE_TX = 2048 + 256 + 64 + 1024;
 constexpr int GEMV_ZERO_BYTES = 1024;       // zero x chunks at a 128-byte stride, for lanes that feed no x
@@ -324,8 +329,7 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS, GEMV_CTAS_PER_SM)
   // the next call's preparation pass may be scheduled as this grid's CTAs retire; it waits for this
   // grid to finish before touching x or the workspace
   pdl_launch_dependents();
-  const uint8_t *xq_sb = reinterpret_cast<const uint8_t *>(p.ws.xq) + (int64_t)sb0 * 1024;  // M = 1
-  const uint8_t *gs_sb = reinterpret_cast<const uint8_t *>(p.ws.gsum) + (int64_t)sb0 * 64;
+  const uint8_t *xb_sb = reinterpret_cast<const uint8_t *>(p.ws.xq) + (int64_t)sb0 * GEMV_XBLOB;  // M = 1
   // stage s of super-block i: weights (codes, group words) need no x; x and sums come after pdl_wait
   auto issue_w = [&](int i, int s) {
     const uint32_t st = ring + s * GEMV_STAGE_BYTES, bar = bar0 + 8 * s;
@@ -335,8 +339,7 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS, GEMV_CTAS_PER_SM)
   };
   auto issue_x = [&](int i, int s) {
     const uint32_t st = ring + s * GEMV_STAGE_BYTES, bar = bar0 + 8 * s;
-    bulk_load(st + GEMV_ST_X, xq_sb + (int64_t)i * 1024, 1024, bar);
-    bulk_load(st + GEMV_ST_GSUM, gs_sb + (int64_t)i * 64, 64, bar);
+    bulk_load(st + GEMV_ST_GSUM, xb_sb + (int64_t)i * GEMV_XBLOB, GEMV_XBLOB, bar);  // sums, then x
   };
   const int pre = nsb < GEMV_RING - 1 ? nsb : GEMV_RING - 1;
   int issued = pre;  // super-blocks whose stage copies were started (lane 0's count is the one used)
