@@ -219,7 +219,7 @@ ql_status launch_gemv_mt(const ql_desc *d, const ql_packed_const *w, const __nv_
   // split K over P CTAs per 64-row group while the row groups alone leave a wave unfilled
   int64_t P = std::max<int64_t>(1, std::min<int64_t>(NS, (int64_t)sms * GEMV_MT_CTAS_PER_SM / TG));
   P = std::min<int64_t>(P, std::max<int64_t>(1, GEMV_MT_MAX_CTAS / TG));
-  if (TG * P > GEMV_MT_MAX_CTAS) return QL_ERR_RANGE;
+  if (P > 1 && TG * P > GEMV_MT_MAX_CTAS) return QL_ERR_RANGE;  // partial sums only exist for P > 1
   p.P = (int)P;
   p.ws = ws;
   p.y = yb;
@@ -261,7 +261,7 @@ ql_status launch_gemv_int6(const ql_desc *d, const ql_packed_const *w, const __n
   // split K over P CTAs per 64-row group while the row groups alone leave a wave unfilled
   int64_t P = std::max<int64_t>(1, std::min<int64_t>(NS, (int64_t)sms * GEMV6_CTAS_PER_SM / TG));
   P = std::min<int64_t>(P, std::max<int64_t>(1, GEMV_MT_MAX_CTAS / TG));
-  if (TG * P > GEMV_MT_MAX_CTAS) return QL_ERR_RANGE;
+  if (P > 1 && TG * P > GEMV_MT_MAX_CTAS) return QL_ERR_RANGE;  // partial sums only exist for P > 1
   cudaLaunchAttribute pa[1];
   pa[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   pa[0].val.programmaticStreamSerializationAllowed = 1;
