@@ -96,6 +96,10 @@ def test_host_validation_before_any_launch(lib):
     assert _call_gemv(lib, ql.Desc("int4", 8, 100), A, A, A, A, 1, A) == ql.QL_ERR_SHAPE
     da = ql.Desc("affine", 8, 256, 4, 64)
     assert _call_gemv(lib, da, A, A, None, A, 33, A) == ql.QL_ERR_RANGE
+    d6 = ql.Desc("int6", 8, 256)
+    assert _call_gemv(lib, d6, A, A, A, A, 9, A) == ql.QL_ERR_RANGE  # int6 GEMV serves M <= 8
+    assert _call_gemv(lib, d6, A, A, A, A, 0, A) == ql.QL_ERR_RANGE
+    assert _call_gemv(lib, ql.Desc("int6", 8, 320), A, A, A, A, 1, A) == ql.QL_ERR_SHAPE  # K % 256
     assert _call_gemv(lib, d, A, A, A, A, 1, A, ws=None) == ql.QL_ERR_NULL
     assert _call_gemv(lib, d, A, A, A, A, 1, A, ws=A + 128) == ql.QL_ERR_ALIGN
     assert _call_gemv(lib, d, A, A, A, A, 1, A, ws_bytes=16) == ql.QL_ERR_SHAPE
