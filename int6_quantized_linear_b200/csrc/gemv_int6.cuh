@@ -1,10 +1,10 @@
 // Tensor-core decode GEMV for the symmetric int6 format at 1 <= M <= 8 tokens.
 //
-// Format (int6 sibling of the nested-superscale int4 layout; "Nested superscale
-// quantization", int6 paragraph): 6-bit two's-complement codes, four per three
-// bytes along K (code i of a 16-weight group at bits 6i .. 6i+5 of its 12
-// little-endian bytes), one int8 scale code per 16 weights and one fp16 step
-// per 256: w = q * (code * step), no zero point.
+// Format (ExecuTorch PR "[cuda] Nestest Superscale Quantization for CUDA Weights
+// (int4 / int6)", "Quant schema update", int6 bullet): 6-bit two's-complement
+// codes, four per three bytes along K (code i of a 16-weight group at bits
+// 6i .. 6i+5 of its 12 little-endian bytes), one int8 scale code per 16 weights
+// and one fp16 step per 256: w = q * (code * step), no zero point.
 //
 // The integer MMA (mma.sync m16n8k32, s8 x s8 / s8 x u8, s32 accumulate) runs
 // with a "diagonal" B operand, as in the int4 M = 1 kernel: within a set of 8
