@@ -122,14 +122,14 @@ def _a256(n):
 @pytest.mark.parametrize("fmt,bits,group,N,K,M", [("int4", 0, 0, 300, 512, 1), ("int4", 0, 0, 27648, 5120, 8),
                                                   ("int6", 0, 0, 5120, 5120, 1), ("int6", 0, 0, 1000, 768, 8),
                                                   ("affine", 2, 64, 14336, 4096, 8), ("affine", 4, 128, 64, 256, 3)])
-def test_gemv_workspace_formula(fmt, bits, group, N, K, M):
+def test_gemv_workspace_formula(lib, fmt, bits, group, N, K, M):
     """The GEMV workspace size is the documented sum: x words, per-group scales and sums, the partial
     sums of a K split, one counter per 16 rows, each part rounded up to 256 bytes."""
     want = _a256(4 * M * K) + _a256(8 * M * (K // 32)) + _a256(4 * 4096 * 64 * M) + _a256(4 * ((N + 15) // 16))
     assert ql.qlinear_gemv_workspace_bytes(ql.Desc(fmt, N, K, bits, group), M) == want
 
 
-def test_gemv_workspace_covers_the_gemm_route():
+def test_gemv_workspace_covers_the_gemm_route(lib):
     """Affine calls past the multi-token range run on the GEMM: the GEMV workspace covers the GEMM's."""
     for d, M in ((ql.Desc("affine", 14336, 4096, 2, 64), 32), (ql.Desc("affine", 640, 1024, 8, 128), 8)):
         assert ql.qlinear_gemv_workspace_bytes(d, M) >= ql.qlinear_gemm_workspace_bytes(d, M)
