@@ -104,6 +104,14 @@ int or_num_threads(void) {
 #endif
 }
 
+void or_set_num_threads(int n) {
+#ifdef _OPENMP
+  if (n >= 1) omp_set_num_threads(n);
+#else
+  (void)n;
+#endif
+}
+
 /* ------------------------------------------------------------------------ */
 /* int4 nested superscale: group 32, super-block 256 (8 groups).            */
 /* [NSS] "Quant schema update": scale = uint8 code x per-256 fp16 step,     */
@@ -223,6 +231,71 @@ void or_int6_dequant(int64_t N, int64_t K, const uint8_t *codes,
   for (int64_t n = 0; n < N; ++n) {
     for (int64_t k = 0; k < K; ++k) {
       int q = int6_code_at(codes + n * rb, k);
+      float step = or_f32_from_f16(steps[n * nsb + k / 256]);
+      float S = (float)gmeta[n * ng + k / 16] * step; /* scale = code x step */
+      w[n * K + k] = (float)q * S;                     /* q * scale          */
+    }
+  }
+}
+
+/* ------------------------------------------------------------------------ */
+/* int6, planar storage.  [REV] "Correctness" note 2 describes the reference */
+/* int6 decode kernel's 16-byte load as spanning one 32-weight group at 4    */
+/* bits, i.e. the 6-bit codes are held as a 4-bit plane plus a 2-bit plane.  */
+/* Reading: per 256-weight super-block of a row, 128 bytes of low nibbles    */
+/* (weight i of the super-block at byte i/2, even i in the low nibble), then */
+/* 64 bytes of the codes' bits 4-5 (weight i at byte 128 + i/4, bits         */
+/* 2*(i%4)); the codes are the same two's-complement 6-bit values as the     */
+/* dense layout, and so are the metadata and the dequantisation.             */
+/* ------------------------------------------------------------------------ */
+
+void or_int6p_pack(int64_t N, int64_t K, const int8_t *q, const int8_t *sc,
+                   const uint16_t *st, uint8_t *codes, int8_t *gmeta,
+                   uint16_t *steps) {
+  const int64_t ng = K / 16, nsb = K / 256, rb = 3 * K / 4;
+  for (int64_t n = 0; n < N; ++n) {
+    for (int64_t j = 0; j < nsb; ++j) {
+      uint8_t *blk = codes + n * rb + 192 * j;
+      for (int b = 0; b < 192; ++b) blk[b] = 0;
+      for (int i = 0; i < 256; ++i) {
+        uint32_t f = (uint32_t)(uint8_t)q[n * K + 256 * j + i] & 0x3f; /* 6-bit field */
+        blk[i / 2] |= (uint8_t)((f & 0xf) << (4 * (i % 2)));          /* low plane   */
+        blk[128 + i / 4] |= (uint8_t)((f >> 4) << (2 * (i % 4)));     /* high plane  */
+      }
+    }
+    for (int64_t g = 0; g < ng; ++g) gmeta[n * ng + g] = sc[n * ng + g];
+    for (int64_t j = 0; j < nsb; ++j) steps[n * nsb + j] = st[n * nsb + j];
+  }
+}
+
+static int int6p_code_at(const uint8_t *row, int64_t k) {
+  const uint8_t *blk = row + 192 * (k / 256);
+  int i = (int)(k % 256);
+  int lo = (blk[i / 2] >> (4 * (i % 2))) & 0xf;
+  int hi = (blk[128 + i / 4] >> (2 * (i % 4))) & 0x3;
+  int field = lo | (hi << 4);
+  return field >= 32 ? field - 64 : field; /* two's complement, 6 bits */
+}
+
+void or_int6p_unpack(int64_t N, int64_t K, const uint8_t *codes,
+                     const int8_t *gmeta, const uint16_t *steps, int8_t *q,
+                     int8_t *sc, uint16_t *st) {
+  const int64_t ng = K / 16, nsb = K / 256, rb = 3 * K / 4;
+  for (int64_t n = 0; n < N; ++n) {
+    for (int64_t k = 0; k < K; ++k)
+      q[n * K + k] = (int8_t)int6p_code_at(codes + n * rb, k);
+    for (int64_t g = 0; g < ng; ++g) sc[n * ng + g] = gmeta[n * ng + g];
+    for (int64_t j = 0; j < nsb; ++j) st[n * nsb + j] = steps[n * nsb + j];
+  }
+}
+
+void or_int6p_dequant(int64_t N, int64_t K, const uint8_t *codes,
+                      const int8_t *gmeta, const uint16_t *steps, float *w) {
+  const int64_t ng = K / 16, nsb = K / 256, rb = 3 * K / 4;
+#pragma omp parallel for schedule(static)
+  for (int64_t n = 0; n < N; ++n) {
+    for (int64_t k = 0; k < K; ++k) {
+      int q = int6p_code_at(codes + n * rb, k);
       float step = or_f32_from_f16(steps[n * nsb + k / 256]);
       float S = (float)gmeta[n * ng + k / 16] * step; /* scale = code x step */
       w[n * K + k] = (float)q * S;                     /* q * scale          */

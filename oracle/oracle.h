@@ -112,8 +112,26 @@ void or_matmul_f64(int64_t M, int64_t N, int64_t K, const uint16_t *x_bf16,
  * value directly, nearest-even). */
 void or_bf16_from_f64_array(int64_t n, const double *y, uint16_t *out);
 
+/* int6, planar storage: the codes of each 256-weight super-block of a row as
+ * 128 bytes of low nibbles (weight i at byte i/2, even i low) followed by 64
+ * bytes of bits 4-5 (weight i at byte 128 + i/4, bits 2*(i%4)); codes
+ * [N][3K/4] bytes.  Same q, sc, st, gmeta, steps and dequantisation as the
+ * dense int6 functions. */
+void or_int6p_pack(int64_t N, int64_t K, const int8_t *q, const int8_t *sc,
+                   const uint16_t *st, uint8_t *codes, int8_t *gmeta,
+                   uint16_t *steps);
+void or_int6p_unpack(int64_t N, int64_t K, const uint8_t *codes,
+                     const int8_t *gmeta, const uint16_t *steps, int8_t *q,
+                     int8_t *sc, uint16_t *st);
+void or_int6p_dequant(int64_t N, int64_t K, const uint8_t *codes,
+                      const int8_t *gmeta, const uint16_t *steps, float *w);
+
 /* number of OpenMP threads the oracle's loops use (1 without OpenMP) */
 int or_num_threads(void);
+
+/* set the number of OpenMP threads of the following calls (timing only; the
+ * results do not depend on it) */
+void or_set_num_threads(int n);
 
 #ifdef __cplusplus
 }

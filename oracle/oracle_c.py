@@ -30,8 +30,10 @@ def lib():
         L.or_bf16_from_f32.argtypes = [C.c_float]
         L.or_bf16_from_f64_array.argtypes = [I64, P, P]
         L.or_num_threads.restype = C.c_int
+        L.or_set_num_threads.argtypes = [C.c_int]
         for name, n in (("or_int4_pack", 10), ("or_int4_unpack", 10), ("or_int4_dequant", 6),
                         ("or_int6_pack", 8), ("or_int6_unpack", 8), ("or_int6_dequant", 6),
+                        ("or_int6p_pack", 8), ("or_int6p_unpack", 8), ("or_int6p_dequant", 6),
                         ("or_matmul_f64", 6)):
             getattr(L, name).argtypes = [I64, I64] + [P] * (n - 2)
         for name, n in (("or_affine_pack", 9), ("or_affine_unpack", 9), ("or_affine_dequant", 7)):
@@ -51,6 +53,11 @@ def _c(a, dtype):
 
 def num_threads() -> int:
     return lib().or_num_threads()
+
+
+def set_num_threads(n: int) -> None:
+    """Thread count of the following oracle calls (for timing; results do not depend on it)."""
+    lib().or_set_num_threads(int(n))
 
 
 # ---- scalar conversions -------------------------------------------------------
@@ -140,6 +147,39 @@ def int6_dequant(codes, gmeta, steps):
     w = np.empty((N, K), np.float32)
     lib().or_int6_dequant(N, K, _p(codes), _p(_c(gmeta, np.int8)), _p(_c(steps, np.uint16)),
                           _p(w))
+    return w
+
+
+# ---- int6 planar (low-nibble plane + 2-bit plane per super-block) -------------
+
+def int6p_pack(q, sc, st):
+    q = _c(q, np.int8)
+    N, K = q.shape
+    codes = np.empty((N, 3 * K // 4), np.uint8)
+    gmeta = np.empty((N, K // 16), np.int8)
+    steps = np.empty((N, K // 256), np.uint16)
+    lib().or_int6p_pack(N, K, _p(q), _p(_c(sc, np.int8)), _p(_c(st, np.uint16)),
+                        _p(codes), _p(gmeta), _p(steps))
+    return codes, gmeta, steps
+
+
+def int6p_unpack(codes, gmeta, steps):
+    codes = _c(codes, np.uint8)
+    N, K = codes.shape[0], codes.shape[1] * 4 // 3
+    q = np.empty((N, K), np.int8)
+    sc = np.empty((N, K // 16), np.int8)
+    st = np.empty((N, K // 256), np.uint16)
+    lib().or_int6p_unpack(N, K, _p(codes), _p(_c(gmeta, np.int8)), _p(_c(steps, np.uint16)),
+                          _p(q), _p(sc), _p(st))
+    return q, sc, st
+
+
+def int6p_dequant(codes, gmeta, steps):
+    codes = _c(codes, np.uint8)
+    N, K = codes.shape[0], codes.shape[1] * 4 // 3
+    w = np.empty((N, K), np.float32)
+    lib().or_int6p_dequant(N, K, _p(codes), _p(_c(gmeta, np.int8)), _p(_c(steps, np.uint16)),
+                           _p(w))
     return w
 
 

@@ -96,6 +96,39 @@ def int6_dequant(codes, gmeta, steps):
     return (q.astype(f32) * np.repeat(S, 16, axis=1)).astype(f32)
 
 
+# ---- int6 planar ([REV] "Correctness" note 2: a 4-bit plane and a 2-bit plane) -------
+# Per 256-weight super-block of a row: 128 bytes of low nibbles (even weight in the low nibble),
+# then 64 bytes of the codes' bits 4-5 (weight i at bits 2*(i%4) of byte 128 + i/4).
+
+def int6p_pack(q, sc, st):
+    q = np.asarray(q, np.int8)
+    N, K = q.shape
+    f = (q.view(np.uint8) & 0x3F).reshape(N, K // 256, 256)
+    lo, hi = f & 0xF, f >> 4
+    lo_plane = lo[..., 0::2] | (lo[..., 1::2] << 4)
+    hi_plane = hi[..., 0::4] | (hi[..., 1::4] << 2) | (hi[..., 2::4] << 4) | (hi[..., 3::4] << 6)
+    codes = np.concatenate([lo_plane, hi_plane], axis=-1).reshape(N, 3 * K // 4).astype(np.uint8)
+    return codes, np.asarray(sc, np.int8).copy(), np.asarray(st, np.uint16).copy()
+
+
+def int6p_unpack(codes, gmeta, steps):
+    codes = np.asarray(codes, np.uint8)
+    N = codes.shape[0]
+    blk = codes.reshape(N, -1, 192)
+    lo = np.stack([blk[..., :128] & 0xF, blk[..., :128] >> 4], axis=-1).reshape(N, -1, 256)
+    hi = np.stack([(blk[..., 128:] >> (2 * i)) & 0x3 for i in range(4)], axis=-1).reshape(N, -1, 256)
+    f = (lo | (hi << 4)).reshape(N, -1)
+    q = (f.astype(np.int16) - 64 * (f >= 32)).astype(np.int8)
+    return q, np.asarray(gmeta, np.int8).copy(), np.asarray(steps, np.uint16).copy()
+
+
+def int6p_dequant(codes, gmeta, steps):
+    q, sc, st = int6p_unpack(codes, gmeta, steps)
+    step = np.repeat(f32_from_f16_bits(st), 16, axis=1)       # per group of 16
+    S = sc.astype(f32) * step                                  # scale = code x step
+    return (q.astype(f32) * np.repeat(S, 16, axis=1)).astype(f32)
+
+
 # ---- uint32 affine ([MTL]) -------------------------------------------------------
 
 def affine_pack(q, s, b, bits: int, G: int):

@@ -60,6 +60,8 @@ def pin_bpw(impl):
     w = synth.int6_weights(12, N, K)
     parts = impl.int6_pack(w["q"], w["sc"], w["st"])
     assert Fraction(8 * sum(p.nbytes for p in parts), N * K) == Fraction(65625, 10000)
+    parts = impl.int6p_pack(w["q"], w["sc"], w["st"])  # the planar layout stores the same bits
+    assert Fraction(8 * sum(p.nbytes for p in parts), N * K) == Fraction(65625, 10000)
     for bits in (2, 4, 8):
         w = synth.affine_weights(13, N, K, bits, 64)
         parts = impl.affine_pack(w["q"], w["s"], w["b"], bits, 64)
@@ -90,6 +92,16 @@ def pin_golden_layouts(impl):
         q6[0, :4] = case["q"]
         codes, _, _ = impl.int6_pack(q6, np.ones((1, K // 16), np.int8), np.zeros((1, 1), np.uint16))
         assert list(codes[0, :3]) == case["bytes"], case
+    # int6 planar codes: every byte not named in a case is zero
+    for case in g["int6_planar_codes"]["cases"]:
+        q6 = np.zeros((1, 2 * K), np.int8)
+        for k, v in case["q_at"].items():
+            q6[0, int(k)] = v
+        codes, _, _ = impl.int6p_pack(q6, np.ones((1, K // 8), np.int8), np.zeros((1, 2), np.uint16))
+        want = np.zeros(3 * 2 * K // 4, np.uint8)
+        for i, v in case["bytes_at"].items():
+            want[int(i)] = v
+        assert np.array_equal(codes[0], want), case
     # affine words
     for case in g["affine_words"]["cases"]:
         b = case["bits"]
@@ -150,6 +162,10 @@ def pin_roundtrip(impl):
     out = impl.int6_unpack(*impl.int6_pack(q6, sc6, st6))
     for x, y in zip((q6, sc6, st6), out):
         assert np.array_equal(np.asarray(x), np.asarray(y))
+    # int6 planar: the same rows put each value at each position of a nibble pair and a 2-bit quad
+    out = impl.int6p_unpack(*impl.int6p_pack(q6, sc6, st6))
+    for x, y in zip((q6, sc6, st6), out):
+        assert np.array_equal(np.asarray(x), np.asarray(y))
     # affine: each value at each of the P positions of a word
     for bits in (2, 4, 8):
         P, V = 32 // bits, 1 << bits
@@ -185,16 +201,17 @@ def pin_int4_exact(impl, N=3, K=512, seed=21):
 
 
 def pin_int6_exact(impl, N=3, K=512, seed=22):
-    """int6 needs no rounding at all: w equals the exact q * sc * st."""
+    """int6 needs no rounding at all: w equals the exact q * sc * st (dense and planar storage)."""
     w = synth.int6_weights(seed, N, K)
     w["q"][0, :4] = [-32, 31, 0, -1]
     w["sc"][0, :2] = [-128, 127]
-    got = impl.int6_dequant(*impl.int6_pack(w["q"], w["sc"], w["st"]))
     rng = np.random.default_rng(seed)
     idx = [(0, k) for k in range(64)] + [(int(rng.integers(N)), int(rng.integers(K))) for _ in range(300)]
-    for n, k in idx:
-        exact = int(w["q"][n, k]) * int(w["sc"][n, k // 16]) * fr_f16(w["st"][n, k // 256])
-        assert Fraction(float(got[n, k])) == exact, (n, k)
+    for pack, dequant in ((impl.int6_pack, impl.int6_dequant), (impl.int6p_pack, impl.int6p_dequant)):
+        got = dequant(*pack(w["q"], w["sc"], w["st"]))
+        for n, k in idx:
+            exact = int(w["q"][n, k]) * int(w["sc"][n, k // 16]) * fr_f16(w["st"][n, k // 256])
+            assert Fraction(float(got[n, k])) == exact, (n, k)
 
 
 def pin_affine_exact(impl, N=3, K=512, seed=23):
@@ -222,6 +239,13 @@ def pin_special_cases(impl):
     w_neg = impl.int6_dequant(*impl.int6_pack(-q, sc, st))
     assert np.array_equal(w_neg, -w_pos)
     assert np.all((w_pos == 0) == ((q == 0) | (np.repeat(sc, 16, 1) == 0)))
+    # the planar storage holds the same codes: its weights equal the dense layout's, and its
+    # low plane is byte for byte the int4 nibble packing of the codes' low 4 bits
+    assert np.array_equal(impl.int6p_dequant(*impl.int6p_pack(q, sc, st)), w_pos)
+    lo4 = (q.view(np.uint8) & 0xF).astype(np.uint8)
+    nib = impl.int4_pack(lo4, np.zeros((2, 8), np.uint8), np.zeros((2, 8), np.uint8),
+                         np.zeros((2, 1), np.uint16), np.zeros((2, 1), np.uint16))[0]
+    assert np.array_equal(impl.int6p_pack(q, sc, st)[0][:, :128], nib)
     # int4 with zero code 0 reduces to q * scale
     q4 = rng.integers(0, 16, size=(2, K)).astype(np.uint8)
     sc4 = rng.integers(0, 256, size=(2, 8)).astype(np.uint8)

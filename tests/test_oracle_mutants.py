@@ -77,6 +77,32 @@ def int6_dequant_group32(codes, gmeta, steps):
     return (q.astype(f32) * np.repeat(S, 32, 1)[:, :K]).astype(f32)
 
 
+def int6p_pack_planes_swapped(q, sc, st):
+    codes, gmeta, steps = O.int6p_pack(q, sc, st)
+    N = codes.shape[0]
+    blk = codes.reshape(N, -1, 192)
+    return np.concatenate([blk[..., 128:], blk[..., :128]], -1).reshape(N, -1), gmeta, steps
+
+
+def int6p_unpack_planes_swapped(codes, gmeta, steps):
+    N = codes.shape[0]
+    blk = np.asarray(codes, np.uint8).reshape(N, -1, 192)
+    return O.int6p_unpack(np.concatenate([blk[..., 64:], blk[..., :64]], -1).reshape(N, -1), gmeta, steps)
+
+
+def int6p_dequant_planes_swapped(codes, gmeta, steps):
+    q, sc, st = int6p_unpack_planes_swapped(codes, gmeta, steps)
+    return O.int6_dequant(*O.int6_pack(q, sc, st))
+
+
+def int6p_pack_high_nibble_first(q, sc, st):
+    codes, gmeta, steps = O.int6p_pack(q, sc, st)
+    N = codes.shape[0]
+    blk = codes.reshape(N, -1, 192).copy()
+    blk[..., :128] = (blk[..., :128] >> 4) | (blk[..., :128] << 4)
+    return blk.reshape(N, -1), gmeta, steps
+
+
 def affine_bias_first(codes, gmeta, bits, G):
     q, s, b = O.affine_unpack(codes, gmeta, bits, G)
     sc, bi = np.repeat(O.f32_from_bf16_bits(s), G, 1), np.repeat(O.f32_from_bf16_bits(b), G, 1)
@@ -109,6 +135,10 @@ MUTANTS = {
     "int4 metadata too wide": mutant(int4_pack=int4_pack_wide_meta),
     "int6 no sign extension": mutant(int6_unpack=int6_unpack_no_sign, int6_dequant=int6_dequant_no_sign),
     "int6 group of 32": mutant(int6_dequant=int6_dequant_group32),
+    "int6 planar: 2-bit plane first": mutant(int6p_pack=int6p_pack_planes_swapped,
+                                             int6p_unpack=int6p_unpack_planes_swapped,
+                                             int6p_dequant=int6p_dequant_planes_swapped),
+    "int6 planar: high nibble first": mutant(int6p_pack=int6p_pack_high_nibble_first),
     "affine (q+b)*s": mutant(affine_dequant=affine_bias_first),
     "affine msb first": mutant(affine_pack=affine_pack_msb_first),
     "matmul drops a term": mutant(matmul_f64=matmul_drops_last_k),
