@@ -17,6 +17,10 @@
  *                group 16, super-block 256, scale = int8 code x per-256 fp16
  *                step; 6.5625 bits/weight.  Section "Why this design" (b)
  *                gives the reason the int8 scale code is kept.
+ *  QL_INT6_PLANAR the same int6 codes and metadata with the codes held as a
+ *                4-bit plane and a 2-bit plane: the ExecuTorch PR's review,
+ *                "Correctness" note 2, describes the reference int6 decode
+ *                kernel's 16-byte load as one 32-weight group at 4 bits.
  *  QL_AFFINE_U32 uint32-packed affine.  Hugging Face Transformers docs,
  *                "Metal" quantization page, introduction: codes packed into
  *                uint32 words with per-group scales and biases; bit widths
@@ -34,6 +38,12 @@
  *                                    24-bit unit: sum_i (q[4j+i] & 63) << 6i
  *               gmeta i8  [N][K/16]  scale code
  *               steps u16 [N][K/256] fp16 step
+ *  QL_INT6_PLANAR codes u8 [N][3K/4]  per 256-weight super-block j of a row,
+ *                                    192 bytes at 192j: bytes 0..127 hold
+ *                                    the low 4 bits of code 256j+i at byte
+ *                                    i/2 (even i in the low nibble), bytes
+ *                                    128..191 its bits 4-5 at byte 128+i/4,
+ *                                    bits 2*(i%4); gmeta, steps as QL_INT6_SYM
  *  QL_AFFINE_U32 codes u32 [N][K*bits/32]  word t = sum_i q[tP+i] << bits*i,
  *                                          P = 32/bits (first code lowest)
  *               gmeta u32 [N][K/group] bf16 scale | bf16 bias << 16
@@ -42,7 +52,7 @@
  * Dequantisation, exactly (each step one binary32 operation, nearest-even,
  * no fused multiply-add):
  *  int4:   S = f32(sc)*f32(ss); Z = f32(zc)*f32(zs); w = (f32(q) - Z) * S
- *  int6:   S = f32(sc)*f32(st); w = f32(q) * S
+ *  int6 (either storage):   S = f32(sc)*f32(st); w = f32(q) * S
  *  affine: w = f32(q)*f32(scale) + f32(bias)
  *
  * Conventions for every entry point:
@@ -78,14 +88,16 @@ typedef enum {
   QL_ERR_NULL = 1,        /* a required pointer is NULL                          */
   QL_ERR_SHAPE = 2,       /* N, K, M, bits or group not allowed for the format   */
   QL_ERR_ALIGN = 3,       /* a pointer is not 16-byte aligned                    */
-  QL_ERR_RANGE = 4,       /* M outside the range of the entry point, or (from    */
-                          /* qlinear_sync_status) an encoder input out of domain */
+  QL_ERR_RANGE = 4,       /* a value out of range: M for the entry point, a      */
+                          /* problem larger than qlinear_gemm_noalloc's fixed    */
+                          /* scratch array, or (from qlinear_sync_status) an     */
+                          /* encoder input outside its domain                    */
   QL_ERR_UNSUPPORTED = 5, /* unknown format, or the device is not sm_100         */
   QL_ERR_CUDA = 6,        /* a CUDA runtime call or launch failed                */
   QL_ERR_TIMEOUT = 7      /* a device-side bounded wait gave up                  */
 } ql_status;
 
-typedef enum { QL_INT4_NSS = 1, QL_INT6_SYM = 2, QL_AFFINE_U32 = 3 } ql_format;
+typedef enum { QL_INT4_NSS = 1, QL_INT6_SYM = 2, QL_AFFINE_U32 = 3, QL_INT6_PLANAR = 4 } ql_format;
 
 typedef enum { QL_OUT_F32 = 0, QL_OUT_BF16 = 1 } ql_out_dtype;
 
@@ -93,7 +105,7 @@ typedef enum { QL_OUT_F32 = 0, QL_OUT_BF16 = 1 } ql_out_dtype;
  *  fmt   : a ql_format value
  *  bits  : QL_AFFINE_U32: 2, 4 or 8.  Ignored (0) for int4 / int6.
  *  group : QL_AFFINE_U32: 32, 64 or 128.  Ignored (0) for int4 / int6, whose
- *          groups are fixed at 32 and 16.
+ *          groups are fixed at 32 and 16 (int6 in either storage).
  *  N     : output features, N >= 1.
  *  K     : input features.  int4 / int6: K % 256 == 0.  affine:
  *          K % group == 0 and (K * bits) % 128 == 0 (whole 16-byte rows). */
@@ -123,7 +135,7 @@ typedef struct {
 /* The unpacked inputs of qlinear_pack (device pointers, caller-owned):
  *              q (one code per byte)   meta0          meta1        step0        step1
  *  int4:       u8 [N][K] 0..15         sc u8 [N][K/32] zc u8 [..]  ss f16 [N][K/256] zs f16 [..]
- *  int6:       i8 [N][K] -32..31       sc i8 [N][K/16] (unused)    st f16 [N][K/256] (unused)
+ *  int6 (both): i8 [N][K] -32..31      sc i8 [N][K/16] (unused)    st f16 [N][K/256] (unused)
  *  affine:     u8 [N][K] 0..2^bits-1   scale bf16 [N][K/group] bias bf16 [..] (unused) (unused)
  * Codes are reduced to their low `bits` bits (int6: two's complement low
  * 6 bits) when packed. */
@@ -137,7 +149,7 @@ typedef struct {
 
 /* Byte sizes of the three packed buffers for `desc` (host-only, no CUDA call).
  * Size closed forms: int4 K/2 + K/16 + K/64 bytes per row (4.625 bits per
- * weight); int6 3K/4 + K/16 + K/128 (6.5625); affine K*bits/8 + 4K/group
+ * weight); int6 (either storage) 3K/4 + K/16 + K/128 (6.5625); affine K*bits/8 + 4K/group
  * (bits + 32/group).  Errors: QL_ERR_NULL, QL_ERR_SHAPE, QL_ERR_UNSUPPORTED. */
 ql_status qlinear_packed_bytes(const ql_desc *desc, size_t *codes_bytes,
                                size_t *gmeta_bytes, size_t *steps_bytes);
@@ -166,6 +178,12 @@ ql_status qlinear_unpack(const ql_desc *desc, const ql_packed_const *in,
 
 /* Standalone dequantisation: out[N][K] = w as defined above, as binary32
  * (QL_OUT_F32, bit-exact) or as its nearest-even bfloat16 (QL_OUT_BF16).
+ * The formulas are those of the ExecuTorch page's "Quant schema update"
+ * (int4 / int6) and of the Transformers "Metal" page's introduction
+ * (affine); that page's section on dequantisation describes the same
+ * operation as turning a pre-quantized checkpoint back into float weights
+ * where the fused kernels are not used.  `out`: device, [N][K] row-major,
+ * 4 or 2 bytes per element, caller-owned, 16-byte aligned.
  * Errors: as qlinear_pack, plus QL_ERR_SHAPE for an unknown out_dtype. */
 ql_status qlinear_dequant(const ql_desc *desc, const ql_packed_const *w,
                           void *out, int32_t out_dtype, ql_stream_t stream);
@@ -180,7 +198,7 @@ ql_status qlinear_dequant(const ql_desc *desc, const ql_packed_const *w,
  *         code = clamp(round_half_even(v / f32(step)), 0, 255)  -> u8;
  *         out->meta0 = sc [N][K/32], out->meta1 = zc, out->step0 = ss
  *         [N][K/256] fp16 bits, out->step1 = zs.
- *   int6: scale float32 [N][K/16], finite, either sign; `zero` unused:
+ *   int6 (either storage): scale float32 [N][K/16], finite, either sign; `zero` unused:
  *         step = RN_fp16(block max|v| / 127),
  *         code = clamp(round_half_even(v / f32(step)), -127, 127) -> i8;
  *         out->meta0 = sc [N][K/16], out->step0 = st [N][K/256].
@@ -196,10 +214,13 @@ ql_status qlinear_quantize_meta(const ql_desc *desc, const float *scale, const f
                                 const ql_unpacked_out *out, ql_stream_t stream);
 
 /* Bytes of caller-provided device workspace qlinear_gemv needs for `desc`
- * and M (host-only, no CUDA call): 4*M*K for x in the order the tensor-core
- * fragments read it, 8*M*K/32 for the per-group x scales and sums,
- * 4*4096*64*M for the partial sums of a K split and 4*ceil(N/16) for its
- * counters, each part rounded up to 256 bytes; for affine calls that run on
+ * and M (host-only, no CUDA call): 7*M*K for x (24-bit fixed point, three
+ * bytes per element plus the zero padding of the diagonal operands) in the
+ * order the tensor-core fragments read it, 8*M*K/32 for the per-group x
+ * scales and sums,
+ * 4*4096*64*M for the partial sums of a K split, 4*ceil(N/16) for its
+ * counters and 16*K/256 for the per-super-block precision flags, each part
+ * rounded up to 256 bytes; for affine calls that run on
  * the GEMM (below) at least qlinear_gemm_workspace_bytes().
  * Errors: QL_ERR_NULL, QL_ERR_SHAPE, QL_ERR_RANGE, QL_ERR_UNSUPPORTED. */
 ql_status qlinear_gemv_workspace_bytes(const ql_desc *desc, int64_t M, size_t *bytes);
@@ -209,17 +230,22 @@ ql_status qlinear_gemv_workspace_bytes(const ql_desc *desc, int64_t M, size_t *b
  * 1 <= M <= 8 for int4 / int6; 1 <= M <= 32 for affine.
  *  - Tensor-core path (int4 and int6 at every M; affine with group 32 or 64
  *    and K % 256 == 0 at M <= 8): two launches.  A short pass turns each x
- *    group (32 elements; 16 for int6) into 16-bit fixed point (x_int =
- *    rint(x * 2^a), the group's max |x| scaled into [2^14, 2^15)), split
- *    into high and low bytes in the order the tensor-core fragments read
- *    them, with the group's scale (and sum); then the streaming kernel
+ *    group (32 elements; 16 for int6) into fixed point, x_int = rint(x *
+ *    2^a): 16-bit (the group's max |x| scaled into [2^14, 2^15): exact for
+ *    every bf16 element within 2^7 of the group's largest magnitude), or
+ *    24-bit (max in [2^22, 2^23): exact within 2^15) for every group of a
+ *    super-block (per token) in which some group's 16-bit rounding error
+ *    exceeds 2^-12 of its mass outside its largest element; split into high,
+ *    middle and (24-bit) low bytes in the order the tensor-core fragments
+ *    read them, with the group's scale (and sum); then the streaming kernel
  *    multiplies the codes (as u8 or s8 bytes: 16q for nibbles, 4q for int6,
  *    q for 2- and 8-bit fields) by those bytes on the integer tensor core
- *    (mma.sync m16n8k32, exact s32 sums) and applies scale (and zero or
- *    bias) once per (row, group[, token]) in fp32.  int4 at M = 1 and int6
- *    use a diagonal x operand (one MMA column per weight group); int4 at
- *    M >= 2 and affine use the tokens as MMA columns.  K may be split over
- *    warps or CTAs, the parts added in a fixed order through the workspace.
+ *    (mma.sync m16n8k32, exact s32 sums, one MMA per byte) and applies scale
+ *    (and zero or bias) once per (row, group[, token]) in fp32.  int4 at M =
+ *    1 and int6 use a diagonal x operand (one MMA column per weight group);
+ *    int4 at M >= 2 and affine use the tokens as MMA columns.  K may be split
+ *    over warps or CTAs, the parts added in a fixed order through the
+ *    workspace.
  *  - Affine with other groups, or K % 256 != 0, at M < 8: one launch, exact
  *    binary32 weights, fp32 FMA.
  *  - Affine at M >= 9 (M >= 8 on the path above): runs as qlinear_gemm.
@@ -255,7 +281,10 @@ ql_status qlinear_gemv_bias(const ql_desc *desc, const ql_packed_const *w,
 ql_status qlinear_gemm_workspace_bytes(const ql_desc *desc, int64_t M, size_t *bytes);
 
 /* Prefill-shaped layer on the tcgen05 tensor cores: same result definition
- * as qlinear_gemv, any M >= 1 (meant for M >= 128).  Three launches on
+ * as qlinear_gemv, any M >= 1 (meant for M >= 128).  The dequantisation is
+ * fused into the contraction, as the Transformers "Metal" page's
+ * introduction describes for its fused dequantize + matmul kernel; the
+ * ExecuTorch page's "e2e results" measure this shape as prefill.  Three launches on
  * `stream`: (1) x is scaled per token row by a power of two 2^a_m that puts
  * the row's max |x| in [2^15, 2^16) and stored as fp16 in the workspace
  * (exact for every value within 2^29 of the row maximum); (2) each weight
@@ -311,19 +340,43 @@ ql_status qlinear_concat_n(const ql_desc *a, const ql_packed_const *wa,
  *    larger problems return QL_ERR_RANGE before anything is enqueued.
  *  - The first call on a device looks up that device's address of the array
  *    (cudaGetSymbolAddress, with the device current) and caches it; make that
- *    first call before any stream capture.
+ *    first call before any stream capture.  With lazy module loading (the
+ *    default of recent CUDA releases) the array and the library's kernels
+ *    are only placed on a device when the library is first used there, so a
+ *    process that reserves nearly all of HBM should make this first call on
+ *    each device before it reserves its pool.
  *  - All calls on a device share the one array, which keeps whatever the last
  *    call left in it; nothing in it needs to start at zero, because each call
- *    writes every element it later reads.  Calls whose work overlaps on the
- *    GPU (other streams, or other threads) race on the array: order them. */
+ *    writes every element of it that its kernels read.  Calls whose work
+ *    overlaps on the GPU (other streams, or other threads) race on the array:
+ *    order them. */
 ql_status qlinear_gemm_noalloc(const ql_desc *desc, const ql_packed_const *w,
                                const void *x, int64_t M, void *y,
                                ql_stream_t stream);
 
 /* Synchronise `stream`, then read and clear the current device's status
  * word: QL_ERR_TIMEOUT if a kernel's bounded wait gave up since the last
- * call, QL_ERR_CUDA if the synchronisation failed, else QL_OK. */
+ * call, QL_ERR_RANGE if qlinear_quantize_meta met an input outside its
+ * domain (the loud failure the ExecuTorch review's "Correctness" note 1 asks
+ * of the metadata encoder, instead of a silent clamp), QL_ERR_CUDA if the
+ * synchronisation failed, else QL_OK.  The word is per device and shared by
+ * every stream: a status may come from work enqueued on another stream. */
 ql_status qlinear_sync_status(ql_stream_t stream);
+
+/* Bound, in SM clock cycles, of every device-side wait of the current
+ * device's kernels for another role or for data (default 2e9, about 1 s at
+ * the B200's clock); cycles <= 0 restores the default.  A kernel whose wait
+ * runs out sets the device status word (qlinear_sync_status then returns
+ * QL_ERR_TIMEOUT), makes its other roles leave their loops, waits for the
+ * copies and MMAs it has in flight -- those drains always keep the default
+ * bound -- frees its tensor memory and returns.  withhold_copies != 0 makes
+ * the kernels' producers start no copies at all, so the first wait for data
+ * is certain to run out (a wait can otherwise still be met by data arriving
+ * within the bound); 0 restores normal operation.  Both exist so that tests
+ * can drive that give-up path; callers normally never change them.  (The
+ * pages have no counterpart.)  Synchronous; do not call it while this
+ * library's kernels run.  Errors: QL_ERR_CUDA. */
+ql_status qlinear_set_wait_limit(int64_t cycles, int32_t withhold_copies);
 
 /* Static, never NULL. */
 const char *qlinear_status_string(ql_status status);

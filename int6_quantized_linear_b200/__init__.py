@@ -17,7 +17,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libqlinear.
 
 QL_OK, QL_ERR_NULL, QL_ERR_SHAPE, QL_ERR_ALIGN, QL_ERR_RANGE, QL_ERR_UNSUPPORTED, QL_ERR_CUDA, \
     QL_ERR_TIMEOUT = range(8)
-FORMATS = {"int4": 1, "int6": 2, "affine": 3}
+FORMATS = {"int4": 1, "int6": 2, "affine": 3, "int6p": 4}  # int6p: int6 codes in planar storage
 QL_OUT_F32, QL_OUT_BF16 = 0, 1
 
 
@@ -66,6 +66,7 @@ _SIGNATURES = {
     "qlinear_gemm_noalloc": ([C.POINTER(ql_desc), C.POINTER(ql_packed), C.c_void_p, C.c_int64, C.c_void_p,
                               C.c_void_p], C.c_int),
     "qlinear_sync_status": ([C.c_void_p], C.c_int),
+    "qlinear_set_wait_limit": ([C.c_int64, C.c_int32], C.c_int),
     "qlinear_gemv_bias": ([C.POINTER(ql_desc), C.POINTER(ql_packed), C.c_void_p, C.c_int64, C.c_void_p,
                            C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p], C.c_int),
     "qlinear_gemm_bias": ([C.POINTER(ql_desc), C.POINTER(ql_packed), C.c_void_p, C.c_int64, C.c_void_p,
@@ -264,6 +265,12 @@ def qlinear_gemm_noalloc(desc: Desc, codes, gmeta, steps, x, M: int, y, stream=N
     w = ql_packed(_ptr(codes), _ptr(gmeta), _ptr(steps))
     _check(lib().qlinear_gemm_noalloc(C.byref(d), C.byref(w), _ptr(x), M, _ptr(y), _stream(stream)),
            "qlinear_gemm_noalloc")
+
+
+def qlinear_set_wait_limit(cycles: int, withhold_copies: bool = False) -> None:
+    """Bound (SM clock cycles) of the kernels' waits on the current device (<= 0: the default), and
+    whether their producers withhold every copy.  For tests of the give-up path (QL_ERR_TIMEOUT)."""
+    _check(lib().qlinear_set_wait_limit(int(cycles), 1 if withhold_copies else 0), "qlinear_set_wait_limit")
 
 
 def qlinear_sync_status(stream=None) -> int:

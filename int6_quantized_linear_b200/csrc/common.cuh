@@ -11,6 +11,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <type_traits>
+
 #define QL_DEVI __device__ __forceinline__
 
 // ---------------------------------------------------------------------------
@@ -23,6 +25,16 @@ __device__ unsigned int g_ql_status;
 
 // ~1 s at the B200's 1.9 GHz SM clock: far longer than any legitimate wait.
 #define QL_WAIT_LIMIT_CYCLES 2000000000LL
+
+// Bound of the waits for another role or for data (qlinear_set_wait_limit changes it, to exercise
+// the give-up path in tests).  Waits that drain copies or MMAs already in flight before a CTA exits
+// always use QL_WAIT_LIMIT_CYCLES, so nothing lands in the shared memory of a CTA that has left.
+__constant__ long long g_ql_wait_limit = QL_WAIT_LIMIT_CYCLES;
+
+// Test switch (qlinear_set_wait_limit): when set, the kernels' producers start no copies, so the
+// first wait for data runs out.  Nothing is then in flight when a CTA gives up.
+__constant__ int g_ql_withhold;
+QL_DEVI bool copies_withheld() { return g_ql_withhold != 0; }
 
 QL_DEVI uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -71,7 +83,7 @@ QL_DEVI bool mbar_wait_bounded(uint32_t bar, uint32_t parity, volatile int *abor
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (clock64() - t0 > QL_WAIT_LIMIT_CYCLES) {
+    if (clock64() - t0 > g_ql_wait_limit) {
       atomicOr(&g_ql_status, QL_DEV_TIMEOUT);
       *abort = 1;
       return false;

@@ -17,7 +17,7 @@
 
 namespace ql {
 
-enum : int { FMT_INT4 = 1, FMT_INT6 = 2, FMT_AFFINE = 3 };
+enum : int { FMT_INT4 = 1, FMT_INT6 = 2, FMT_AFFINE = 3, FMT_INT6P = 4 };
 
 // ---- int4 -----------------------------------------------------------------
 // c: the chunk's 16 code bytes as 4 little-endian words (low nibble = even k)
@@ -58,6 +58,27 @@ QL_DEVI void int6_decode32(const uint32_t (&c)[6], uint32_t sc2, uint32_t st, fl
       const int q = (f ^ 32) - 32;  // sign-extend 6 bits
       w[4 * j + i] = __fmul_rn((float)q, (4 * j + i) < 16 ? S0 : S1);
     }
+  }
+}
+
+// ---- int6, planar storage -------------------------------------------------
+// The review of the ExecuTorch PR ("Correctness" note 2) describes the
+// reference int6 decode kernel's 16-byte load as one 32-weight group at 4
+// bits: the codes sit in a 4-bit plane and a 2-bit plane.  Per 256-weight
+// super-block: 128 bytes of low nibbles (even weight low), then 64 bytes of
+// bits 4-5 (weight i at bits 2*(i%4) of byte 128 + i/4).
+// lo: the chunk's 16 low-plane bytes as 4 words; hi: its 8 high-plane bytes
+// as 2 words; sc2, st as int6_decode32.
+QL_DEVI void int6p_decode32(const uint32_t (&lo)[4], const uint32_t (&hi)[2], uint32_t sc2, uint32_t st,
+                            float (&w)[32]) {
+  const float step = f16_bits_to_f32(st);
+  const float S0 = __fmul_rn((float)(int8_t)(sc2 & 0xffu), step);
+  const float S1 = __fmul_rn((float)(int8_t)((sc2 >> 8) & 0xffu), step);
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const int f = (int)(((lo[i >> 3] >> (4 * (i & 7))) & 0xfu) | (((hi[i >> 4] >> (2 * (i & 15))) & 0x3u) << 4));
+    const int q = (f ^ 32) - 32;  // sign-extend 6 bits
+    w[i] = __fmul_rn((float)q, i < 16 ? S0 : S1);
   }
 }
 

@@ -12,13 +12,16 @@
 //  W:  b_n per weight row, chosen so a bound on max_k |w[n][k]| times 2^b_n
 //      lies in [2^14, 2^15) (headroom for the rounding to fp16).  The bound
 //      comes from the metadata alone:  int4 |S|*max(|Z|, |15-Z|),
-//      int6 32*|S|,  affine max(|bias|, |(2^bits-1)*scale + bias|).
+//      int6 (either storage) 32*|S|,  affine max(|bias|, |(2^bits-1)*scale + bias|).
+//
+// The epilogue undoes both scales with the combined exponent -(a_m + b_n), so
+// no intermediate product can overflow or underflow where the result does not.
 //
 // Workspace layout (caller-provided, 256-byte aligned sections):
 //   x16   fp16 [M][K]   scaled activations
-//   xinv  f32  [M]      2^-a_m
-//   wsc   f32  [N']     2^b_n   (N' = N rounded up to 256; the tail is unused)
-//   winv  f32  [N']     2^-b_n
+//   xexp  s32  [M]      -a_m
+//   wsc   f32  [N']     2^b_n   (N' = N rounded up to 256; rows N.. hold 0)
+//   wexp  s32  [N']     -b_n    (rows N.. hold 0)
 #pragma once
 #include "formats.cuh"
 
@@ -28,13 +31,13 @@ inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 struct GemmWorkspace {
   __half *x16;
-  float *xinv;
+  int *xexp;
   float *wsc;
-  float *winv;
+  int *wexp;
 };
 
 // the per-row weight scales are padded to whole 256-row tiles
-inline size_t padded_rows(int64_t N) { return (size_t)((N + 255) / 256 * 256); }
+__host__ __device__ inline size_t padded_rows(int64_t N) { return (size_t)((N + 255) / 256 * 256); }
 
 inline size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   return align256((size_t)M * K * 2) + align256((size_t)M * 4) + 2 * align256(padded_rows(N) * 4);
@@ -45,16 +48,23 @@ inline GemmWorkspace gemm_workspace_carve(void *base, int64_t M, int64_t N, int6
   GemmWorkspace w;
   w.x16 = reinterpret_cast<__half *>(p);
   p += align256((size_t)M * K * 2);
-  w.xinv = reinterpret_cast<float *>(p);
+  w.xexp = reinterpret_cast<int *>(p);
   p += align256((size_t)M * 4);
   w.wsc = reinterpret_cast<float *>(p);
   p += align256(padded_rows(N) * 4);
-  w.winv = reinterpret_cast<float *>(p);
+  w.wexp = reinterpret_cast<int *>(p);
   return w;
 }
 
 // 2^e as a binary32 for e in [-126, 127]
 QL_DEVI float exp2i(int e) { return __int_as_float((e + 127) << 23); }
+
+// d * 2^e for any e in [-252, 253] as two exact power-of-two multiplications: the result is the
+// nearest binary32 of the exact product whenever that product is a normal float.
+QL_DEVI float mul_pow2(float d, int e) {
+  const int e1 = max(-126, min(127, e));
+  return (d * exp2i(e1)) * exp2i(max(-126, min(127, e - e1)));
+}
 
 // Exponent that puts amax * 2^s into [2^top, 2^(top+1)); 0 for zero or non-finite.
 QL_DEVI int scale_exponent(float amax, int top) {
@@ -103,17 +113,25 @@ __global__ void __launch_bounds__(256) x_to_f16_kernel(const __nv_bfloat16 *x, i
     }
     out[i] = make_uint4(o[0], o[1], o[2], o[3]);
   }
-  if (lane == 0) ws.xinv[m] = exp2i(-a);
+  if (lane == 0) ws.xexp[m] = -a;
 }
 
 // One warp per weight row: bound max|w| from the metadata (lanes stride over the groups, then a
-// max-reduction), pick b_n.
+// max-reduction), pick b_n.  The grid covers the rows up to N rounded to 256: rows past N get
+// scale 0 and exponent 0, so the padded columns of a tile are defined (and never stored).
 template <int FMT, int BITS>
 __global__ void __launch_bounds__(256) w_scale_kernel(const uint8_t *gmeta, const uint8_t *steps, int64_t N,
                                                        int64_t K, int G, GemmWorkspace ws) {
   const int lane = threadIdx.x & 31;
   const int64_t n = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
-  if (n >= N) return;  // whole warps leave together
+  if (n >= (int64_t)padded_rows(N)) return;  // whole warps leave together
+  if (n >= N) {
+    if (lane == 0) {
+      ws.wsc[n] = 0.f;
+      ws.wexp[n] = 0;
+    }
+    return;
+  }
   float bound = 0.f;
   if constexpr (FMT == FMT_INT4) {
     const uint16_t *gm = reinterpret_cast<const uint16_t *>(gmeta) + n * (K / 32);
@@ -126,7 +144,7 @@ __global__ void __launch_bounds__(256) w_scale_kernel(const uint8_t *gmeta, cons
       const float Z = __fmul_rn((float)(c >> 8), zs);
       bound = fmaxf(bound, __fmul_rn(fabsf(S), fmaxf(fabsf(Z), fabsf(__fsub_rn(15.f, Z)))));
     }
-  } else if constexpr (FMT == FMT_INT6) {
+  } else if constexpr (FMT == FMT_INT6 || FMT == FMT_INT6P) {
     const int8_t *gm = reinterpret_cast<const int8_t *>(gmeta) + n * (K / 16);
     const uint16_t *st = reinterpret_cast<const uint16_t *>(steps) + n * (K / 256);
     for (int64_t g = lane; g < K / 16; g += 32) {
@@ -147,7 +165,7 @@ __global__ void __launch_bounds__(256) w_scale_kernel(const uint8_t *gmeta, cons
   if (lane == 0) {
     const int e = scale_exponent(bound, 14);
     ws.wsc[n] = exp2i(e);
-    ws.winv[n] = exp2i(-e);
+    ws.wexp[n] = -e;
   }
 }
 

@@ -16,7 +16,7 @@
 //               metadata ring, MSTAGES ahead
 //   warps 4-7   epilogue: tcgen05.ld the accumulators (warp w reads TMEM
 //               lanes 32*(w%4).. of both halves), undo the two power-of-two
-//               scales, round to bf16, store y
+//               scales (exponents added first), round to bf16, store y
 //   warps 8-15  dequantisers, one tile row and 32 weights each per stage:
 //               packed codes + metadata -> weight times 2^b_n -> fp16, written
 //               in the canonical K-major 128-byte-swizzled layout the MMA reads
@@ -45,47 +45,60 @@ constexpr int NUM_META_WARPS = 2;
 constexpr int WARP_EPI0 = 4;
 constexpr int WARP_DEQ0 = 8;
 constexpr int NUM_THREADS = (WARP_DEQ0 + NUM_DEQ_WARPS) * 32;
-constexpr int A_BYTES = BM * BK * 2;  // 32 KB
-constexpr int B_BYTES = BN * BK * 2;  // 16 KB
-constexpr uint32_t TMEM_COLS = 512;   // two accumulator pairs of 2 x 128 fp32 columns
+constexpr int B_BYTES = BN * BK * 2;  // 16 KB: the dequantised weight tile
+constexpr int TT_SWAP = 32;           // token tile of the swapped form (weights as the M = 128 operand)
 constexpr int MSTAGES = 8;            // metadata ring depth (int4)
 constexpr int META_STAGE_BYTES = BN * 8;  // per tile row: the stage's two group words (u32), its step word
 constexpr int SMEM_LIMIT = 232448;        // dynamic shared memory a CTA may use
 
 __host__ __device__ constexpr int code_bits(int fmt, int bits) {
-  return fmt == FMT_INT4 ? 4 : (fmt == FMT_INT6 ? 6 : bits);
+  return fmt == FMT_INT4 ? 4 : ((fmt == FMT_INT6 || fmt == FMT_INT6P) ? 6 : bits);
 }
 __host__ __device__ constexpr int p_row_bytes(int fmt, int bits) { return BK * code_bits(fmt, bits) / 8; }
 __host__ __device__ constexpr int p_bytes(int fmt, int bits) { return BN * p_row_bytes(fmt, bits); }
 
-// Stages of the ring: four when they fit, else three.  int4 adds the metadata ring
-// [MSTAGES][BN rows][8 bytes] and its barriers.
+// TT is the token tile: BM = 256 (two M = 128 MMAs per 16-k slice with the x tile as A, the weight
+// tile as B, N = 128) or TT_SWAP = 32 for small batches (one M = 128, N = 32 MMA per slice with the
+// weight tile as A and the x tile as B), whose accumulators are 32 TMEM columns.
+__host__ __device__ constexpr int a_bytes(int tt) { return tt * BK * 2; }  // the fp16 x tile
+__host__ __device__ constexpr uint32_t tmem_cols(int tt) { return tt == BM ? 512u : 64u; }  // two accumulators
+
+// Stages of the ring: as many as fit, up to four (six for the small x tile of the swapped form).
+// int4 adds the metadata ring [MSTAGES][BN rows][8 bytes] and its barriers.
 constexpr int NUM_BARS_PER_STAGE = 3;  // tma_full, b_full, empty
 constexpr int NUM_BARS_FIXED = 5;      // acc_full[2], acc_empty[2], final
-__host__ __device__ constexpr int stage_bytes(int fmt, int bits) { return A_BYTES + B_BYTES + p_bytes(fmt, bits); }
+__host__ __device__ constexpr int stage_bytes(int fmt, int bits, int tt) { return a_bytes(tt) + B_BYTES + p_bytes(fmt, bits); }
 __host__ __device__ constexpr int meta_bytes(int fmt) { return fmt == FMT_INT4 ? MSTAGES * META_STAGE_BYTES : 0; }
 __host__ __device__ constexpr int meta_bars(int fmt) { return fmt == FMT_INT4 ? 2 * MSTAGES : 0; }
-__host__ __device__ constexpr int smem_need(int fmt, int bits, int st) {
-  return st * stage_bytes(fmt, bits) + meta_bytes(fmt) +
+__host__ __device__ constexpr int smem_need(int fmt, int bits, int tt, int st) {
+  return st * stage_bytes(fmt, bits, tt) + meta_bytes(fmt) +
          (NUM_BARS_PER_STAGE * st + NUM_BARS_FIXED + meta_bars(fmt)) * 8 + 16 + 1024;
 }
-__host__ __device__ constexpr int stages(int fmt, int bits) { return smem_need(fmt, bits, 4) <= SMEM_LIMIT ? 4 : 3; }
+__host__ __device__ constexpr int stages(int fmt, int bits, int tt) {
+  return (tt != BM && smem_need(fmt, bits, tt, 6) <= SMEM_LIMIT) ? 6
+       : (tt != BM && smem_need(fmt, bits, tt, 5) <= SMEM_LIMIT) ? 5
+       : smem_need(fmt, bits, tt, 4) <= SMEM_LIMIT ? 4 : 3;
+}
 
 // byte offsets inside the dynamic shared memory (base aligned to 1024)
-__host__ __device__ constexpr int off_a(int s) { return s * A_BYTES; }
-__host__ __device__ constexpr int off_b(int fmt, int bits, int s) { return stages(fmt, bits) * A_BYTES + s * B_BYTES; }
-__host__ __device__ constexpr int off_p(int fmt, int bits, int s) {
-  return stages(fmt, bits) * (A_BYTES + B_BYTES) + s * p_bytes(fmt, bits);
+__host__ __device__ constexpr int off_a(int tt, int s) { return s * a_bytes(tt); }
+__host__ __device__ constexpr int off_b(int fmt, int bits, int tt, int s) {
+  return stages(fmt, bits, tt) * a_bytes(tt) + s * B_BYTES;
 }
-__host__ __device__ constexpr int off_meta(int fmt, int bits, int s) {
-  return stages(fmt, bits) * stage_bytes(fmt, bits) + s * META_STAGE_BYTES;
+__host__ __device__ constexpr int off_p(int fmt, int bits, int tt, int s) {
+  return stages(fmt, bits, tt) * (a_bytes(tt) + B_BYTES) + s * p_bytes(fmt, bits);
 }
-__host__ __device__ constexpr int off_bar(int fmt, int bits) {
-  return stages(fmt, bits) * stage_bytes(fmt, bits) + meta_bytes(fmt);
+__host__ __device__ constexpr int off_meta(int fmt, int bits, int tt, int s) {
+  return stages(fmt, bits, tt) * stage_bytes(fmt, bits, tt) + s * META_STAGE_BYTES;
+}
+__host__ __device__ constexpr int off_bar(int fmt, int bits, int tt) {
+  return stages(fmt, bits, tt) * stage_bytes(fmt, bits, tt) + meta_bytes(fmt);
 }
 // barriers: tma_full[S], b_full[S], empty[S], acc_full[2], acc_empty[2], final, (int4) meta_full[MS],
 // meta_empty[MS]; then the tmem base and the abort flag
-__host__ __device__ constexpr int smem_bytes(int fmt, int bits) { return smem_need(fmt, bits, stages(fmt, bits)); }
+__host__ __device__ constexpr int smem_bytes(int fmt, int bits, int tt) {
+  return smem_need(fmt, bits, tt, stages(fmt, bits, tt));
+}
 
 struct Params {
   int64_t M, N, K;
@@ -109,7 +122,7 @@ QL_DEVI void load_meta(const Params &p, int64_t n, int64_t c, uint32_t &gm, uint
   if constexpr (FMT == FMT_INT4) {
     gm = __ldg(reinterpret_cast<const uint16_t *>(p.gmeta) + n * (p.K / 32) + c);
     st = __ldg(reinterpret_cast<const uint32_t *>(p.steps) + n * (p.K / 256) + (c >> 3));
-  } else if constexpr (FMT == FMT_INT6) {
+  } else if constexpr (FMT == FMT_INT6 || FMT == FMT_INT6P) {
     gm = __ldg(reinterpret_cast<const uint16_t *>(p.gmeta + n * (p.K / 16)) + c);
     st = __ldg(reinterpret_cast<const uint16_t *>(p.steps) + n * (p.K / 256) + (c >> 3));
   } else {
@@ -118,10 +131,16 @@ QL_DEVI void load_meta(const Params &p, int64_t n, int64_t c, uint32_t &gm, uint
   }
 }
 
-// Decode one chunk whose codes sit in shared memory at `src`.
+// Decode one chunk whose codes sit in shared memory at `src` (int6 planar: the chunk's 16 low-plane
+// bytes at `src`, its 8 high-plane bytes at `src_hi`).
 template <int FMT, int BITS>
-QL_DEVI void smem_decode32(const uint8_t *src, uint32_t gm, uint32_t st, float (&w)[32]) {
-  if constexpr (FMT == FMT_INT4) {
+QL_DEVI void smem_decode32(const uint8_t *src, const uint8_t *src_hi, uint32_t gm, uint32_t st, float (&w)[32]) {
+  if constexpr (FMT == FMT_INT6P) {
+    const uint4 l = *reinterpret_cast<const uint4 *>(src);
+    const uint2 h = *reinterpret_cast<const uint2 *>(src_hi);
+    const uint32_t lo[4] = {l.x, l.y, l.z, l.w}, hi[2] = {h.x, h.y};
+    int6p_decode32(lo, hi, gm, st, w);
+  } else if constexpr (FMT == FMT_INT4) {
     const uint4 v = *reinterpret_cast<const uint4 *>(src);
     const uint32_t c[4] = {v.x, v.y, v.z, v.w};
     int4_decode32(c, gm, st, w);
@@ -147,17 +166,19 @@ QL_DEVI void smem_decode32(const uint8_t *src, uint32_t gm, uint32_t st, float (
   }
 }
 
-template <int FMT, int BITS>
+template <int FMT, int BITS, int TT>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_codes,
                 Params p) {
+  constexpr bool SWAP = TT != BM;
   constexpr int PROW = p_row_bytes(FMT, BITS);
-  constexpr int STAGES = stages(FMT, BITS);
-  constexpr uint32_t STAGE_TX = A_BYTES + p_bytes(FMT, BITS);
+  constexpr int STAGES = stages(FMT, BITS, TT);
+  constexpr uint32_t STAGE_TX = a_bytes(TT) + p_bytes(FMT, BITS);
+  constexpr uint32_t TMEM_COLS = tmem_cols(TT);
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + off_bar(FMT, BITS));
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + off_bar(FMT, BITS, TT));
   uint32_t *tmem_holder =
       reinterpret_cast<uint32_t *>(bars + NUM_BARS_PER_STAGE * STAGES + NUM_BARS_FIXED + meta_bars(FMT));
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
@@ -171,7 +192,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   auto bar_meta_empty = [&](int s) { return smem_u32(bars + 3 * STAGES + 5 + MSTAGES + s); };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t m_tiles = (p.M + BM - 1) / BM, n_tiles = (p.N + BN - 1) / BN;
+  const int64_t m_tiles = (p.M + TT - 1) / TT, n_tiles = (p.N + BN - 1) / BN;
   const int64_t num_tiles = m_tiles * n_tiles;
   const int num_kb = (int)(p.K / BK);
   const int64_t my_tiles = (num_tiles - blockIdx.x + gridDim.x - 1) / gridDim.x;
@@ -244,15 +265,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t ph = 0;
       Cursor cur = cursor0();
       bool ok = true;
-      for (; it < total_it; ++it) {
+      const bool hold = copies_withheld();
+      for (; it < total_it && !hold; ++it) {
         if (!mbar_wait_bounded(bar_empty(s), ph ^ 1u, abort_flag)) {
           ok = false;
           break;
         }
         mbar_arrive_expect_tx(bar_tma_full(s), STAGE_TX);
-        tma_load_2d(sbase + off_a(s), &map_x, bar_tma_full(s), cur.kb * BK, (int32_t)(cur.m_tile * BM));
-        tma_load_2d(sbase + off_p(FMT, BITS, s), &map_codes, bar_tma_full(s), cur.kb * PROW,
-                    (int32_t)(cur.n_tile * BN));
+        tma_load_2d(sbase + off_a(TT, s), &map_x, bar_tma_full(s), cur.kb * BK, (int32_t)(cur.m_tile * TT));
+        if constexpr (FMT == FMT_INT6P) {  // k-step kb: low-plane bytes 32 (kb % 4) .. and high-plane
+                                           // bytes 128 + 16 (kb % 4) .. of super-block kb / 4, by 16-byte boxes
+          const int32_t x0 = 192 * (cur.kb >> 2) + 32 * (cur.kb & 3), xh = 192 * (cur.kb >> 2) + 128 + 16 * (cur.kb & 3);
+          tma_load_2d(sbase + off_p(FMT, BITS, TT, s), &map_codes, bar_tma_full(s), x0, (int32_t)(cur.n_tile * BN));
+          tma_load_2d(sbase + off_p(FMT, BITS, TT, s) + 16 * BN, &map_codes, bar_tma_full(s), x0 + 16,
+                      (int32_t)(cur.n_tile * BN));
+          tma_load_2d(sbase + off_p(FMT, BITS, TT, s) + 32 * BN, &map_codes, bar_tma_full(s), xh,
+                      (int32_t)(cur.n_tile * BN));
+        } else {
+          tma_load_2d(sbase + off_p(FMT, BITS, TT, s), &map_codes, bar_tma_full(s), cur.kb * PROW,
+                      (int32_t)(cur.n_tile * BN));
+        }
         step_ring(s, ph, STAGES);
         advance(cur);
       }
@@ -267,7 +299,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else if (warp == WARP_MMA) {
     if (lane == 0) {
-      constexpr uint32_t idesc = umma_idesc_f16_f32(128, BN);
+      constexpr uint32_t idesc = SWAP ? umma_idesc_f16_f32(BN, TT) : umma_idesc_f16_f32(128, BN);
       int64_t tcount = 0;
       int s = 0;
       uint32_t ph = 0;
@@ -277,20 +309,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint32_t ause = (uint32_t)(tcount >> 1);
         if (!mbar_wait_bounded(bar_acc_empty(a), (ause & 1) ^ 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + (uint32_t)(a * 2 * BN);  // half hm at + hm * BN columns
+        // accumulator a: columns a * 2 * BN .. (two token halves of BN columns) or, swapped, a * TT ..
+        const uint32_t d_tmem = tmem_base + (uint32_t)(SWAP ? a * TT : a * 2 * BN);
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait_bounded(bar_tma_full(s), ph, abort_flag) || !mbar_wait_bounded(bar_b_full(s), ph, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint64_t bdesc = umma_desc_k_sw128(sbase + off_b(FMT, BITS, s));
-#pragma unroll
-          for (int hm = 0; hm < 2; ++hm) {  // token half: rows 128*hm.. of the x tile (16 KB in)
-            const uint64_t adesc = umma_desc_k_sw128(sbase + off_a(s) + hm * (A_BYTES / 2));
+          const uint64_t wdesc = umma_desc_k_sw128(sbase + off_b(FMT, BITS, TT, s));
+          if constexpr (SWAP) {  // D[weight row][token] += W tile (A, M = 128) x x tile (B, N = TT)
+            const uint64_t xdesc = umma_desc_k_sw128(sbase + off_a(TT, s));
 #pragma unroll
             for (int kk = 0; kk < BK / 16; ++kk)  // advance 16 fp16 = 32 bytes = 2 descriptor units
-              umma_f16(d_tmem + (uint32_t)(hm * BN), adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) != 0);
+              umma_f16(d_tmem, wdesc + 2 * kk, xdesc + 2 * kk, idesc, (kb | kk) != 0);
+          } else {
+#pragma unroll
+            for (int hm = 0; hm < 2; ++hm) {  // token half: rows 128*hm.. of the x tile (16 KB in)
+              const uint64_t adesc = umma_desc_k_sw128(sbase + off_a(TT, s) + hm * (a_bytes(TT) / 2));
+#pragma unroll
+              for (int kk = 0; kk < BK / 16; ++kk)  // advance 16 fp16 = 32 bytes = 2 descriptor units
+                umma_f16(d_tmem + (uint32_t)(hm * BN), adesc + 2 * kk, wdesc + 2 * kk, idesc, (kb | kk) != 0);
+            }
           }
           umma_commit(bar_empty(s));
           issued = true;
@@ -316,7 +356,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       Cursor cur = cursor0();
       for (int64_t it = 0; it < total_it; ++it) {
         if (!mbar_wait_bounded(bar_meta_empty(ms), phm ^ 1u, abort_flag)) break;
-        const uint32_t dst = sbase + off_meta(FMT, BITS, ms);
+        const uint32_t dst = sbase + off_meta(FMT, BITS, TT, ms);
 #pragma unroll
         for (int i = 0; i < BN / 64; ++i) {
           const int r = t + 64 * i;
@@ -342,10 +382,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint32_t ause = (uint32_t)(tcount >> 1);
       if (!mbar_wait_bounded(bar_acc_full(a), ause & 1, abort_flag)) break;
       tc_fence_after();
+      if constexpr (SWAP) {
+        // lane = weight row n of the tile (TMEM lane 32 e + lane), its TT columns = the tile's tokens
+        uint32_t r[32];
+        static_assert(TT == 32, "one 32-column TMEM load per row");
+        tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(32 * e) << 16) + (uint32_t)(a * TT), r);
+        tmem_ld_wait();
+        const int64_t n = n_tile * BN + 32 * e + lane, m0 = m_tile * TT;
+        const int we = n < p.N ? p.ws.wexp[n] : 0;
+        const float bn = (p.bias && n < p.N) ? __bfloat162float(p.bias[n]) : 0.f;
+        const int xe_lane = m0 + lane < p.M ? p.ws.xexp[m0 + lane] : 0;
+#pragma unroll
+        for (int t = 0; t < TT; ++t) {  // y = D * 2^-(a_m + b_n) (exponents added first), + bias, one rounding
+          const int xe = __shfl_sync(0xffffffffu, xe_lane, t);
+          const float v = mul_pow2(__uint_as_float(r[t]), xe + we) + bn;
+          if (m0 + t < p.M && n < p.N) p.y[(m0 + t) * p.N + n] = __float2bfloat16_rn(v);
+        }
+      } else {
 #pragma unroll 1
       for (int hm = 0; hm < 2; ++hm) {
         const int64_t m = m_tile * BM + 128 * hm + 32 * e + lane;
-        const float xs = m < p.M ? p.ws.xinv[m] : 0.f;
+        const int xe = m < p.M ? p.ws.xexp[m] : 0;
 #pragma unroll 1
         for (int cchunk = 0; cchunk < BN / 32; ++cchunk) {
           uint32_t r[32];
@@ -353,19 +410,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                              r);
           tmem_ld_wait();
           const int64_t n0 = n_tile * BN + 32 * cchunk;
-          {  // y = D * 2^-a_m * 2^-b_n, both exact power-of-two multiplications
-            const float4 *wi = reinterpret_cast<const float4 *>(p.ws.winv + n0);
+          {  // y = D * 2^-(a_m + b_n): the two exponents are added first, then D is scaled exactly
+            const int4 *we = reinterpret_cast<const int4 *>(p.ws.wexp + n0);
 #pragma unroll
             for (int t = 0; t < 8; ++t) {
-              const float4 v = wi[t];
-              r[4 * t + 0] = __float_as_uint(__uint_as_float(r[4 * t + 0]) * xs * v.x);
-              r[4 * t + 1] = __float_as_uint(__uint_as_float(r[4 * t + 1]) * xs * v.y);
-              r[4 * t + 2] = __float_as_uint(__uint_as_float(r[4 * t + 2]) * xs * v.z);
-              r[4 * t + 3] = __float_as_uint(__uint_as_float(r[4 * t + 3]) * xs * v.w);
+              const int4 v = we[t];
+              r[4 * t + 0] = __float_as_uint(mul_pow2(__uint_as_float(r[4 * t + 0]), xe + v.x));
+              r[4 * t + 1] = __float_as_uint(mul_pow2(__uint_as_float(r[4 * t + 1]), xe + v.y));
+              r[4 * t + 2] = __float_as_uint(mul_pow2(__uint_as_float(r[4 * t + 2]), xe + v.z));
+              r[4 * t + 3] = __float_as_uint(mul_pow2(__uint_as_float(r[4 * t + 3]), xe + v.w));
             }
           }
-          if (p.bias) {  // + bias[n], still in fp32
-#pragma unroll 4
+          if (p.bias) {  // + bias[n], still in fp32 (fully unrolled: r stays in registers)
+#pragma unroll
             for (int i = 0; i < 32; ++i)
               if (n0 + i < p.N) r[i] = __float_as_uint(__uint_as_float(r[i]) + __bfloat162float(p.bias[n0 + i]));
           }
@@ -382,11 +439,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 reinterpret_cast<uint4 *>(dst)[t] = v;
               }
             } else {
+#pragma unroll
               for (int i = 0; i < 32; ++i)
                 if (n0 + i < p.N) dst[i] = __float2bfloat16_rn(__uint_as_float(r[i]));
             }
           }
         }
+      }
       }
       tc_fence_before();
       __syncwarp();
@@ -420,7 +479,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       advance(nxt);
       if constexpr (FMT == FMT_INT4) {  // this stage's group and step words, from the metadata ring
         if (!mbar_wait_bounded(bar_meta_full(ms), phm, abort_flag)) break;
-        const uint2 mv = *reinterpret_cast<const uint2 *>(smem + off_meta(FMT, BITS, ms) + r * 8);
+        const uint2 mv = *reinterpret_cast<const uint2 *>(smem + off_meta(FMT, BITS, TT, ms) + r * 8);
         gm = (mv.x >> (16 * h)) & 0xffffu;
         st = mv.y;
         __syncwarp();
@@ -428,8 +487,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         step_ring(ms, phm, MSTAGES);
       }
       if (!mbar_wait_bounded(bar_tma_full(s), ph, abort_flag)) break;
-      const uint8_t *src = smem + off_p(FMT, BITS, s) + r * PROW + h * (PROW / 2);
-      uint8_t *dst_row = row + off_b(FMT, BITS, s);
+      const uint8_t *src = smem + off_p(FMT, BITS, TT, s) + r * PROW + h * (PROW / 2);
+      uint8_t *dst_row = row + off_b(FMT, BITS, TT, s);
       // each 16-byte chunk holds k = 0,4,1,5,2,6,3,7 of its 8 weights (the order of the x tile)
       if constexpr (FMT == FMT_INT4) {
         // packed-half arithmetic: q as 1024+q / 64+q from one bit operation, then
@@ -461,9 +520,54 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const int j = 4 * h + q;  // logical 16-byte chunk of the 128-byte row
           *reinterpret_cast<uint4 *>(dst_row + ((j ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
         }
+      } else if constexpr (FMT == FMT_AFFINE) {
+        // packed-half arithmetic: the codes become 1024 + q halves by bit operations (q exact after
+        // one subtraction), then w * 2^b_n = q * s' + b' in one fused multiply-add with s' = s * 2^b_n
+        // and b' = b * 2^b_n, which are exact in fp16 (bf16 values scaled into fp16's range), so each
+        // weight is rounded once
+        const __half2 s2 = __float2half2_rn(bf16_bits_to_f32(gm) * sc);
+        const __half2 b2 = __float2half2_rn(bf16_bits_to_f32(gm >> 16) * sc);
+        const __half2 m1024 = __float2half2_rn(1024.f);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {  // output chunk q: weights 8q .. 8q+7 of the thread's 32, as (k, k+4) pairs
+          uint32_t pr[4];
+          if constexpr (BITS == 4) {
+            const uint32_t wd = reinterpret_cast<const uint32_t *>(src)[q], w8 = wd >> 8;
+            pr[0] = (wd & 0x000F000Fu) | 0x64006400u;  // (1024 + n0, 1024 + n4)
+            pr[1] = ((wd >> 4) & 0x000F000Fu) | 0x64006400u;
+            pr[2] = (w8 & 0x000F000Fu) | 0x64006400u;
+            pr[3] = ((w8 >> 4) & 0x000F000Fu) | 0x64006400u;
+          } else if constexpr (BITS == 8) {
+            const uint32_t w0 = reinterpret_cast<const uint32_t *>(src)[2 * q];      // k 0..3
+            const uint32_t w1 = reinterpret_cast<const uint32_t *>(src)[2 * q + 1];  // k 4..7
+            const uint32_t t0 = __byte_perm(w0, w1, 0x5140), t1 = __byte_perm(w0, w1, 0x7362);  // (0 4 1 5) (2 6 3 7)
+            pr[0] = __byte_perm(t0, 0x64646464u, 0x4140);
+            pr[1] = __byte_perm(t0, 0x64646464u, 0x4342);
+            pr[2] = __byte_perm(t1, 0x64646464u, 0x4140);
+            pr[3] = __byte_perm(t1, 0x64646464u, 0x4342);
+          } else {  // 2-bit: codes 8q .. 8q+7 are bits 16 (q & 1) .. of word q / 2
+            const uint32_t wd = reinterpret_cast<const uint32_t *>(src)[q >> 1] >> (16 * (q & 1));
+            const uint32_t u = __byte_perm(wd, 0u, 0x4140);  // codes 0-3 in byte 0, codes 4-7 in byte 2
+#pragma unroll
+            for (int e = 0; e < 4; ++e) pr[e] = ((u >> (2 * e)) & 0x00030003u) | 0x64006400u;
+          }
+          uint32_t o[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const __half2 qv = __hsub2(*reinterpret_cast<const __half2 *>(&pr[e]), m1024);
+            const __half2 wv = __hfma2(qv, s2, b2);
+            o[e] = *reinterpret_cast<const uint32_t *>(&wv);
+          }
+          const int j = 4 * h + q;  // logical 16-byte chunk of the 128-byte row
+          *reinterpret_cast<uint4 *>(dst_row + ((j ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
       } else {
         float w[32];
-        smem_decode32<FMT, BITS>(src, gm, st, w);
+        if constexpr (FMT == FMT_INT6P)  // boxes [2 low halves][BN rows][16 B], then [BN rows][16 B] high
+          smem_decode32<FMT, BITS>(smem + off_p(FMT, BITS, TT, s) + h * 16 * BN + r * 16,
+                                   smem + off_p(FMT, BITS, TT, s) + 32 * BN + r * 16 + 8 * h, gm, st, w);
+        else
+          smem_decode32<FMT, BITS>(src, nullptr, gm, st, w);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const int j = 4 * h + q;  // logical 16-byte chunk of the 128-byte row

@@ -79,51 +79,69 @@ __global__ void __launch_bounds__(256) gemv_simple_kernel(WeightPtrs p, int64_t 
 // mma.sync.m16n8k32 (u8 x s8 / u8 x u8, s32 accumulate) multiplies these
 // 16x32 fragments by a "diagonal" x operand: column n of B holds x only in
 // the k-slots that carry group n's codes and zeros elsewhere, so D[row][n]
-// collects group n's partial dot product.  x enters as 16-bit fixed point per
-// 32-element group, x_int = rint(x * 2^a_g) with the group's max |x| scaled
-// into [2^14, 2^15), split into a signed high byte and an unsigned low byte
-// (x_int = 256 * hi + lo), one MMA for each.  Per (row, group) of a
-// super-block the two integer sums are exact and below 2^22 in magnitude, so
-// the accumulators start at 1.5 * 2^23 (as bits) and read back as floats
-// with one subtraction.  The scale and zero are applied once per (row, group):
-//     T = 16 * sum_k q_k x_int_k = 256 * D_hi + D_lo
-//     y += S * (2^-a_g / 16) * (T - 16 * Z * X_g),   X_g = sum_k x_int_k
-// with S = sc * ss and Z = zc * zs.  A short preparation pass writes the x
-// bytes in the order the fragments read them with (2^-a_g / 16, -16 X_g) per
-// group; the streaming kernel is launched as a programmatic dependent of that
-// pass and starts fetching weights before it has finished (griddepcontrol.wait
-// guards the first read of x).  Lanes that hold no x for an MMA read a zero
-// block, so no per-MMA selects are needed.
+// collects group n's partial dot product.  x enters as fixed point per
+// 32-element group, x_int = rint(x * 2^a_g), as up to three bytes x_int =
+// 65536 * hi + 256 * mid + lo (a signed high byte, unsigned middle and low
+// bytes), one MMA each:
+//   - 16-bit (the group's max |x| scaled into [2^14, 2^15), lo = 0: no third
+//     MMA), exact for every bf16 element within 2^7 of the group's largest
+//     magnitude, the rest rounded to 2^-15 of it;
+//   - 24-bit (max |x| in [2^22, 2^23)), exact within 2^15, for every group of
+//     a super-block in which some group's 16-bit rounding error exceeds 2^-12
+//     of that group's mass outside its largest element (a dominant outlier,
+//     where the 16-bit form would lose the other elements); the preparation
+//     pass flags such super-blocks and the kernel adds the third MMA there.
+// Per (row, group) of a super-block the integer sums are exact and below 2^22
+// in magnitude, so the accumulators start at 1.5 * 2^23 (as bits) and read
+// back as floats with one subtraction.  The scale and zero are applied once
+// per (row, group):
+//     T = 65536 * D_hi + 256 * D_mid + D_lo = 16 * 2^u * sum_k q_k x_int_k
+//     y += S * G_x * (T + Z * G_y)
+// with S = sc * ss, Z = zc * zs, u = 0 (24-bit) or 8 (16-bit), G_x = 2^-a_g /
+// (16 * 2^u) and G_y = -16 * 2^u * X_g, X_g = sum_k x_int_k.  A short
+// preparation pass writes the x bytes in the order the fragments read them
+// with (G_x, G_y) per group and the flag per super-block; the streaming kernel
+// is launched as a programmatic dependent of that pass and starts fetching
+// weights before it has finished (griddepcontrol.wait guards the first read of
+// x).  Lanes that hold no x for an MMA read a zero block, so no per-MMA
+// selects are needed.
 // ===========================================================================
 
 constexpr int GEMV_MT_MAX_CTAS = 4096;  // bound on the CTAs of one multi-token launch (sizes its partial sums)
-constexpr int GEMV_XBLOB = 1088;         // M = 1 x block per super-block: 8 group sums (64 B) + x words (1 KB)
+
+// M = 1 x block per super-block: 8 x (G_x, G_y) (64 B), the super-block's 24-bit flag (16 B), the
+// (hi, mid) x words (1 KB) -- the part a stage copies -- then the lo x words (512 B), read from global
+// memory by the kernel only for a 24-bit super-block
+constexpr int GEMV_XBLOB = 1616, GEMV_XCOPY = 1104, GEMV_XB_FLAG = 64, GEMV_XB_Q = 80, GEMV_XB_L = 1104;
 
 struct GemvWorkspace {
-  uint4 *xq;        // M = 1: [K/256 super-blocks] blocks of GEMV_XBLOB bytes: 8 x (2^-a/16, -16 X) float2, then
-                    //        [4 j][2 kinds][8 groups][16 B] B-operand pairs (gemv_xprep_kernel); the blocks run
-                    //        on into the gsum region, which directly follows (4K is a multiple of 256)
-                    // M > 1: [K/32 groups][M tokens][4][16 B] B-operand words (gemv_xprep_mt_kernel)
-  float2 *gsum;     // M > 1: [K/32][M]: (2^-a_g / 16, -16 * sum x_int); M = 1: the tail of the xq blocks
+  uint4 *xq;        // int4 M = 1: [K/256 super-blocks] blocks of GEMV_XBLOB bytes (gemv_xprep_kernel)
+                    // int4 M > 1 / affine: [K/32 groups][M tokens][4][16 B] (hi, mid) B-operand words, then
+                    //   [K/32][M][4][8 B] lo words (gemv_xprep_mt_kernel); int6: see gemv_xprep_int6_kernel
+  float2 *gsum;     // M > 1: [K/32][M]: (G_x, G_y); int6: per 16-element group scales
   float *partial;   // M = 1: [16-row tile][part][16 rows]; M > 1: [CTA][M][64 rows]: sums of one K range
   int *counters;    // parts finished so far: M = 1 per 16-row tile, M > 1 per 64-row group
+  uint8_t *flags;   // M > 1, int6: [K/256][16]: byte m non-zero when token m's x of that super-block is 24-bit
 };
 
 inline size_t gemv_workspace_bytes(int64_t M, int64_t N, int64_t K) {
-  return align256((size_t)M * K * 4) + align256((size_t)M * (K / 32) * 8) +
-         align256((size_t)GEMV_MT_MAX_CTAS * 64 * M * 4) + align256((size_t)((N + 15) / 16) * 4);
+  return align256((size_t)M * K * 7) + align256((size_t)M * (K / 32) * 8) +
+         align256((size_t)GEMV_MT_MAX_CTAS * 64 * M * 4) + align256((size_t)((N + 15) / 16) * 4) +
+         align256((size_t)(K / 256) * 16);
 }
 
-inline GemvWorkspace gemv_workspace_carve(void *base, int64_t M, int64_t K) {
+inline GemvWorkspace gemv_workspace_carve(void *base, int64_t M, int64_t N, int64_t K) {
   uint8_t *p = static_cast<uint8_t *>(base);
   GemvWorkspace w;
   w.xq = reinterpret_cast<uint4 *>(p);
-  p += align256((size_t)M * K * 4);
+  p += align256((size_t)M * K * 7);
   w.gsum = reinterpret_cast<float2 *>(p);
   p += align256((size_t)M * (K / 32) * 8);
   w.partial = reinterpret_cast<float *>(p);
   p += align256((size_t)GEMV_MT_MAX_CTAS * 64 * M * 4);
   w.counters = reinterpret_cast<int *>(p);
+  p += align256((size_t)((N + 15) / 16) * 4);
+  w.flags = p;
   return w;
 }
 
@@ -137,13 +155,27 @@ QL_DEVI int atomic_add_acq_rel_gpu(int *addr, int v) {
 QL_DEVI void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 QL_DEVI void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
-// Four lanes per 32-element group of x (lane c holds k = 8c .. 8c + 7): fixed-point conversion with
-// the group's max and sum by shuffles, byte split in fragment order.  Chunk (j, kind) of group grp
-// is the register quad its feeding lane loads: the high-byte and low-byte words of
+// Whether a group's 16-bit fixed point loses too much: the summed rounding error of its elements,
+// x * 2^a - rint(x * 2^a) with a the 16-bit exponent, above 2^-12 of the group's mass outside its
+// largest element (all in units of 2^-a).  err and mass are a lane's partial sums; the four lanes
+// of a group combine them.
+QL_DEVI bool group_needs_24bit(float err, float mass, float amax_scaled) {
+  err += __shfl_xor_sync(0xffffffffu, err, 1);
+  err += __shfl_xor_sync(0xffffffffu, err, 2);
+  mass += __shfl_xor_sync(0xffffffffu, mass, 1);
+  mass += __shfl_xor_sync(0xffffffffu, mass, 2);
+  return err > (mass - amax_scaled) * (1.f / 4096.f);
+}
+
+// x preparation for the int4 M = 1 kernel: four lanes per 32-element group (lane c holds k = 8c ..
+// 8c + 7), so one warp holds one super-block's eight groups.  Fixed-point conversion with the
+// group's max and sum by shuffles, 16-bit unless some group of the super-block needs 24 bits (then
+// the whole super-block is 24-bit and flagged), byte split in fragment order.  Chunk (j, kind) of
+// group grp is what its feeding lane loads: the high-byte and middle-byte words of
 // k = 8j + kind + {0, 2, 4, 6}, each paired with a zero word so that one 16-byte load gives the B
-// pairs of two MMAs -- (x, 0) for groups 0-3 (their lanes feed b0), (0, x) for groups 4-7 (b1).
-// Lane c writes the two chunks (j = c, kind = 0 / 1).  It also zeroes the first n_counters tile
-// counters of the K split.
+// pairs of two MMAs -- (x, 0) for groups 0-3 (their lanes feed b0), (0, x) for groups 4-7 (b1) --
+// and the low-byte word paired the same way (8 bytes).  Lane c writes the chunks (j = c, kind = 0 / 1).
+// It also zeroes the first n_counters tile counters of the K split.
 __global__ void __launch_bounds__(256) gemv_xprep_kernel(const __nv_bfloat16 *x, int64_t M, int64_t K,
                                                          int64_t n_counters, GemvWorkspace ws) {
   pdl_launch_dependents();  // the streaming kernel may start fetching weights now
@@ -167,10 +199,21 @@ __global__ void __launch_bounds__(256) gemv_xprep_kernel(const __nv_bfloat16 *x,
   }
   amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
   amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-  const int a = scale_exponent(amax, 14);  // max |x_int| < 2^15
+  const int a16 = scale_exponent(amax, 14);  // max |x_int| < 2^15
+  const float s16 = exp2i(a16);
+  float err = 0.f, mass = 0.f;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const float sv = xs[k] * s16;
+    err += fabsf(sv - rintf(sv));
+    mass += fabsf(sv);
+  }
+  const bool wide = group_needs_24bit(err, mass, amax * s16);
+  const bool sb24 = __any_sync(0xffffffffu, wide && live);  // the warp holds one super-block
+  const int a = sb24 ? scale_exponent(amax, 22) : a16;     // 24-bit: max |x_int| < 2^23
   const float sc = exp2i(a);
   int xi[8];
-  int sum = 0;
+  int sum = 0;  // |sum| < 32 * 2^23
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
     xi[k] = __float2int_rn(xs[k] * sc);
@@ -180,21 +223,30 @@ __global__ void __launch_bounds__(256) gemv_xprep_kernel(const __nv_bfloat16 *x,
   sum += __shfl_xor_sync(0xffffffffu, sum, 2);
   if (!live) return;
   // group gi = (m, super-block sb, group-in-block grp): per (m, sb) one block of GEMV_XBLOB bytes,
-  // the eight groups' sums then chunk (j, kind) at [j][kind][grp], so one bulk copy fetches both
+  // the eight groups' (G_x, G_y), the flag, then chunk (j, kind) at [j][kind][grp] of the (hi, mid)
+  // region and of the lo region
   const int64_t grp = gi & 7, msb = gi >> 3;
-  uint4 *dst = ws.xq + msb * (GEMV_XBLOB / 16) + 4 + grp;
+  uint8_t *blk = reinterpret_cast<uint8_t *>(ws.xq) + msb * GEMV_XBLOB;
+  const int hs = sb24 ? 16 : 8;  // the value's top byte: bits 16.. (24-bit) or 8.. (16-bit, lo = 0)
 #pragma unroll
   for (int kind = 0; kind < 2; ++kind) {
-    uint32_t hi = 0, lo = 0;
+    uint32_t hi = 0, mid = 0, lo = 0;
 #pragma unroll
     for (int b = 0; b < 4; ++b) {
       const int val = xi[2 * b + kind];
-      hi |= ((uint32_t)(val >> 8) & 0xffu) << (8 * b);
-      lo |= ((uint32_t)val & 0xffu) << (8 * b);
+      hi |= ((uint32_t)(val >> hs) & 0xffu) << (8 * b);
+      mid |= ((uint32_t)(val >> (hs - 8)) & 0xffu) << (8 * b);
+      lo |= (sb24 ? ((uint32_t)val & 0xffu) : 0u) << (8 * b);
     }
-    dst[8 * (2 * c + kind)] = grp < 4 ? make_uint4(hi, 0u, lo, 0u) : make_uint4(0u, hi, 0u, lo);
+    const int ch = 8 * (2 * c + kind) + (int)grp;  // chunk (j = c, kind) of group grp
+    reinterpret_cast<uint4 *>(blk + GEMV_XB_Q)[ch] = grp < 4 ? make_uint4(hi, 0u, mid, 0u) : make_uint4(0u, hi, 0u, mid);
+    reinterpret_cast<uint2 *>(blk + GEMV_XB_L)[ch] = grp < 4 ? make_uint2(lo, 0u) : make_uint2(0u, lo);
   }
-  if (c == 0) reinterpret_cast<float2 *>(ws.xq)[msb * (GEMV_XBLOB / 8) + grp] = make_float2(exp2i(-a) * 0.0625f, -16.f * (float)sum);
+  if (c == 0) {  // (G_x, G_y) = (2^-a / (16 * 2^u), -16 * 2^u * X) with u = 0 (24-bit) or 8 (16-bit)
+    const float w = sb24 ? 16.f : 4096.f;
+    reinterpret_cast<float2 *>(blk)[grp] = make_float2(exp2i(-a) / w, -w * (float)sum);
+  }
+  if ((t & 31) == 0) reinterpret_cast<uint32_t *>(blk + GEMV_XB_FLAG)[0] = sb24 ? 1u : 0u;
 }
 
 // A byte of a metadata word as a float: 2^23 + b, to be fused into an FMA with -2^23 * step.
@@ -228,10 +280,11 @@ QL_DEVI uint32_t lds32(uint32_t a) {
   return v;
 }
 
-// Wait for an mbarrier phase, letting the hardware suspend the thread (up to the hint, in ns)
-// instead of spinning; bounded like mbar_wait_bounded.
+// Wait for an mbarrier phase, letting the hardware suspend the thread (up to a hint, in ns) instead
+// of spinning; bounded like mbar_wait_bounded (the bound is read only once a try has failed).
 QL_DEVI bool mbar_wait_suspend(uint32_t bar, uint32_t parity, volatile int *abort) {
   const long long t0 = clock64();
+  const uint32_t hint = 1000000u;
   while (true) {
     uint32_t ok;
     asm volatile(
@@ -239,11 +292,11 @@ QL_DEVI bool mbar_wait_suspend(uint32_t bar, uint32_t parity, volatile int *abor
         "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(bar), "r"(parity), "r"(1000000u)
+        : "r"(bar), "r"(parity), "r"(hint)
         : "memory");
     if (ok) return true;
     if (*abort) return false;
-    if (clock64() - t0 > QL_WAIT_LIMIT_CYCLES) {
+    if (clock64() - t0 > g_ql_wait_limit) {
       atomicOr(&g_ql_status, QL_DEV_TIMEOUT);
       *abort = 1;
       return false;
@@ -264,18 +317,21 @@ QL_DEVI bool mbar_wait_suspend(uint32_t bar, uint32_t parity, volatile int *abor
       : "+r"(ACC[0]), "+r"(ACC[1]), "+r"(ACC[2]), "+r"(ACC[3])                                        \
       : "r"(A0), "r"(A1), "r"(A2), "r"(A3), "r"(B0), "r"(B1))
 
+constexpr int32_t GEMV_ACC0 = 0x4B400000;    // 1.5 * 2^23 as float bits: integer sums below 2^22 read back exactly
+constexpr float GEMV_ACC0_F = 12582912.f;
+
 constexpr int GEMV_RING = 4;   // super-blocks in flight per warp
 constexpr int GEMV_CTAS_PER_SM = 3;
 constexpr int GEMV_WARPS = 4;  // warps per CTA: GEMV_WARPS / parts tiles, each split over `parts` warps
 // one stage = one super-block of a 16-row tile: codes (16 rows x 128 B, 128-byte swizzle), the
-// tile's group words [16 rows][16 B], the super-block's 8 group sums, its x pairs [4 j][2 kinds][8 groups][16 B]
-constexpr int GEMV_ST_CODES = 0, GEMV_ST_GMETA = 2048, GEMV_ST_GSUM = 2304, GEMV_ST_X = 2368;
-static_assert(GEMV_ST_X - GEMV_ST_GSUM == 64 && GEMV_XBLOB == 64 + 1024, "one copy fills sums and x");
+// tile's group words [16 rows][16 B], then the first GEMV_XCOPY bytes of the super-block's x block:
+// 8 x (G_x, G_y), its 24-bit flag and its (hi, mid) x pairs [4 j][2 kinds][8 groups][16 B]
+constexpr int GEMV_ST_CODES = 0, GEMV_ST_GMETA = 2048, GEMV_ST_GSUM = 2304, GEMV_ST_FLAG = 2304 + GEMV_XB_FLAG,
+              GEMV_ST_X = 2304 + GEMV_XB_Q;
 constexpr int GEMV_STAGE_BYTES = 4096;      // multiple of 1024 (the swizzle atom)
-constexpr uint32_t GEMV_STAGE_TX = 2048 + 256 + 64 + 1024;
+constexpr uint32_t GEMV_STAGE_TX = 2048 + 256 + GEMV_XCOPY;
+static_assert(GEMV_ST_GSUM + GEMV_XCOPY <= GEMV_STAGE_BYTES && GEMV_XB_Q + 1024 == GEMV_XCOPY, "stage layout");
 constexpr int GEMV_ZERO_BYTES = 1024;       // zero x chunks at a 128-byte stride, for lanes that feed no x
-constexpr int32_t GEMV_ACC0 = 0x4B400000;    // 1.5 * 2^23 as float bits: integer sums below 2^22 read back exactly
-constexpr float GEMV_ACC0_F = 12582912.f;
 
 struct GemvTcParams {
   const uint8_t *steps;
@@ -339,9 +395,10 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS, GEMV_CTAS_PER_SM)
   };
   auto issue_x = [&](int i, int s) {
     const uint32_t st = ring + s * GEMV_STAGE_BYTES, bar = bar0 + 8 * s;
-    bulk_load(st + GEMV_ST_GSUM, xb_sb + (int64_t)i * GEMV_XBLOB, GEMV_XBLOB, bar);  // sums, then x
+    bulk_load(st + GEMV_ST_GSUM, xb_sb + (int64_t)i * GEMV_XBLOB, GEMV_XCOPY, bar);  // sums, flag, then x
   };
-  const int pre = nsb < GEMV_RING - 1 ? nsb : GEMV_RING - 1;
+  const bool hold = copies_withheld();
+  const int pre = hold ? 0 : (nsb < GEMV_RING - 1 ? nsb : GEMV_RING - 1);
   int issued = pre;  // super-blocks whose stage copies were started (lane 0's count is the one used)
   if (lane == 0) {
     tma_prefetch_desc(&map_codes);
@@ -371,12 +428,16 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS, GEMV_CTAS_PER_SM)
   // per-lane shared-memory addresses (offsets inside a stage are added as constants)
   const bool on0 = (g == c), on1 = (g == c + 4);
   const uint32_t zero_a = smem_u32(zero_blk);
-  uint32_t xa[GEMV_RING];  // this lane's B pairs of MMA step (j, kind) at xa + 128 (2 j + kind)
+  // this lane's B pairs of MMA step (j, kind): (hi, mid) at xa + 128 (2 j + kind); for a 24-bit
+  // super-block its lo pairs in global memory at xlg + 8 (2 j + kind) (feeding lanes only)
+  uint32_t xa[GEMV_RING];
 #pragma unroll
   for (int s = 0; s < GEMV_RING; ++s) {
     xa[s] = on0 ? ring + s * GEMV_STAGE_BYTES + GEMV_ST_X + 16 * c
           : on1 ? ring + s * GEMV_STAGE_BYTES + GEMV_ST_X + 16 * (c + 4) : zero_a;
   }
+  const bool feed = on0 || on1;
+  const uint2 *xlg = reinterpret_cast<const uint2 *>(xb_sb + GEMV_XB_L) + (on0 ? c : c + 4);
   const uint32_t a00 = ring + pg * 128 + ((c ^ pg) << 4), a01 = ring + pg * 128 + (((c + 4) ^ pg) << 4);
   const uint32_t a10 = a00 + 1024, a11 = a01 + 1024;  // row pg + 8: same swizzle phase, next atom
   const uint32_t ag = ring + GEMV_ST_GSUM + 16 * c;
@@ -395,7 +456,7 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS, GEMV_CTAS_PER_SM)
       const int nx = i + GEMV_RING - 1;
       const int sn = (s + GEMV_RING - 1) % GEMV_RING;
       __syncwarp();  // every lane has read that stage in the previous turn
-      if (nx < nsb) {
+      if (nx < nsb && !hold) {
         if (lane == 0) {
           issue_w(nx, sn);
           issue_x(nx, sn);
@@ -411,33 +472,49 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS, GEMV_CTAS_PER_SM)
       const uint32_t so = s * GEMV_STAGE_BYTES;
       const uint4 w00 = lds128(a00 + so), w10 = lds128(a10 + so);  // (r0 | r1, group c)
       const uint4 w01 = lds128(a01 + so), w11 = lds128(a11 + so);  // (r0 | r1, group c+4)
-      const float4 G = lds128f(ag + so);                           // (2^-a/16, -16 X) of groups 2c, 2c+1
+      const float4 G = lds128f(ag + so);                           // (G_x, G_y) of groups 2c, 2c+1
       const uint32_t cm0 = lds32(am + so), cm1 = lds32(am + so + 128);
       const uint32_t ww00[4] = {w00.x, w00.y, w00.z, w00.w}, ww01[4] = {w01.x, w01.y, w01.z, w01.w};
       const uint32_t ww10[4] = {w10.x, w10.y, w10.z, w10.w}, ww11[4] = {w11.x, w11.y, w11.z, w11.w};
-      int32_t dh[4], dl[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const uint4 xe = lds128(xa[s] + 256 * j), xo = lds128(xa[s] + 256 * j + 128);  // even k, odd k
-        const uint32_t h00 = ww00[j] & 0xF0F0F0F0u, h10 = ww10[j] & 0xF0F0F0F0u;  // odd k, x16
-        const uint32_t h01 = ww01[j] & 0xF0F0F0F0u, h11 = ww11[j] & 0xF0F0F0F0u;
-        if (j == 0) {
-          QL_IMMA0("s8", dh, acc_init, h00, h10, h01, h11, xo.x, xo.y);
-          QL_IMMA0("u8", dl, acc_init, h00, h10, h01, h11, xo.z, xo.w);
-        } else {
-          QL_IMMA("s8", dh, h00, h10, h01, h11, xo.x, xo.y);
-          QL_IMMA("u8", dl, h00, h10, h01, h11, xo.z, xo.w);
-        }
-        const uint32_t e00 = (ww00[j] << 4) & 0xF0F0F0F0u, e10 = (ww10[j] << 4) & 0xF0F0F0F0u;  // even k, x16
-        const uint32_t e01 = (ww01[j] << 4) & 0xF0F0F0F0u, e11 = (ww11[j] << 4) & 0xF0F0F0F0u;
-        QL_IMMA("s8", dh, e00, e10, e01, e11, xe.x, xe.y);
-        QL_IMMA("u8", dl, e00, e10, e01, e11, xe.z, xe.w);
-      }
-      // D[q]: q = 0 (r0, group 2c), 1 (r0, 2c+1), 2 (r1, 2c), 3 (r1, 2c+1)
+      // D[q]: q = 0 (r0, group 2c), 1 (r0, 2c+1), 2 (r1, 2c), 3 (r1, 2c+1); T = 65536 D_hi + 256 D_mid (+ D_lo)
       float t[4];
+      auto contract = [&](auto x24c) {  // the super-block's MMAs: two bytes of x, or three for 24-bit x
+        constexpr bool X24 = decltype(x24c)::value;
+        const uint2 *lg = xlg + (int64_t)i * (GEMV_XBLOB / 8);
+        int32_t dh[4], dm[4], dl[4];
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
-        t[q] = fmaf(__int_as_float(dh[q]) - GEMV_ACC0_F, 256.f, __int_as_float(dl[q]) - GEMV_ACC0_F);
+        for (int j = 0; j < 4; ++j) {
+          const uint4 xe = lds128(xa[s] + 256 * j), xo = lds128(xa[s] + 256 * j + 128);  // even k, odd k: hi, mid
+          const uint32_t h00 = ww00[j] & 0xF0F0F0F0u, h10 = ww10[j] & 0xF0F0F0F0u;  // odd k, x16
+          const uint32_t h01 = ww01[j] & 0xF0F0F0F0u, h11 = ww11[j] & 0xF0F0F0F0u;
+          const uint32_t e00 = (ww00[j] << 4) & 0xF0F0F0F0u, e10 = (ww10[j] << 4) & 0xF0F0F0F0u;  // even k, x16
+          const uint32_t e01 = (ww01[j] << 4) & 0xF0F0F0F0u, e11 = (ww11[j] << 4) & 0xF0F0F0F0u;
+          if (j == 0) {
+            QL_IMMA0("s8", dh, acc_init, h00, h10, h01, h11, xo.x, xo.y);
+            QL_IMMA0("u8", dm, acc_init, h00, h10, h01, h11, xo.z, xo.w);
+          } else {
+            QL_IMMA("s8", dh, h00, h10, h01, h11, xo.x, xo.y);
+            QL_IMMA("u8", dm, h00, h10, h01, h11, xo.z, xo.w);
+          }
+          QL_IMMA("s8", dh, e00, e10, e01, e11, xe.x, xe.y);
+          QL_IMMA("u8", dm, e00, e10, e01, e11, xe.z, xe.w);
+          if constexpr (X24) {  // the low byte, from global memory (L2): only feeding lanes hold any
+            const uint2 le = feed ? __ldg(lg + 16 * j) : make_uint2(0u, 0u);
+            const uint2 lo = feed ? __ldg(lg + 16 * j + 8) : make_uint2(0u, 0u);
+            if (j == 0) QL_IMMA0("u8", dl, acc_init, h00, h10, h01, h11, lo.x, lo.y);
+            else QL_IMMA("u8", dl, h00, h10, h01, h11, lo.x, lo.y);
+            QL_IMMA("u8", dl, e00, e10, e01, e11, le.x, le.y);
+          }
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          t[q] = fmaf(__int_as_float(dh[q]) - GEMV_ACC0_F, 256.f, __int_as_float(dm[q]) - GEMV_ACC0_F);
+          if constexpr (X24) t[q] = fmaf(t[q], 256.f, __int_as_float(dl[q]) - GEMV_ACC0_F);
+          else t[q] *= 256.f;
+        }
+      };
+      if (lds32(ring + so + GEMV_ST_FLAG) != 0u) contract(std::true_type{});  // the same for the whole warp
+      else contract(std::false_type{});
       // S = sc * ss and Z = zc * zs, each one FMA from the byte placed in the mantissa of 2^23
       const uint32_t cs0 = sr0[s], cs1 = sr1[s];
       const float ss0 = f16_bits_to_f32(cs0), zs0 = f16_bits_to_f32(cs0 >> 16);
@@ -514,7 +591,8 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS, GEMV_CTAS_PER_SM)
 // and, as column g, token g's x bytes of those slots; it ends with the sums of
 // rows g, g + 8 for tokens 2c, 2c + 1.
 //
-// A CTA is one producer warp and four consumer warps on 64 weight rows (four
+// x is 16- or 24-bit fixed point per (token, group) as in the M = 1 kernel
+// (high, middle and, for 24-bit super-blocks, low byte: one MMA each).  A CTA is one producer warp and four consumer warps on 64 weight rows (four
 // 16-row tiles) and a range of super-blocks: each stage (codes box, group-word
 // box, every token's x words and group sums) is fetched once and read by all
 // four.  When the row groups alone do not fill one wave of GEMV_MT_CTAS_PER_SM
@@ -523,8 +601,11 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS, GEMV_CTAS_PER_SM)
 // cleared by the preparation pass) adds the P parts in part order and writes y.
 // ===========================================================================
 
-// x preparation for M > 1: 4 lanes per (token, 32-element group); lane c owns k = 8c .. 8c + 7 and
-// writes its MMA word quad (even-k high bytes, odd-k high bytes, even-k low bytes, odd-k low bytes).
+// x preparation for M > 1: 4 lanes per (token, 32-element group), so one warp holds one token's
+// eight groups of a super-block; 16-bit fixed point unless some group of them needs 24 bits (then
+// all eight are 24-bit and the token's flag byte of the super-block is set).  Lane c owns
+// k = 8c .. 8c + 7 and writes its MMA word quad (even-k high bytes, odd-k high bytes, even-k middle
+// bytes, odd-k middle bytes) and word pair (even-k low bytes, odd-k low bytes; zero for 16-bit).
 __global__ void __launch_bounds__(256) gemv_xprep_mt_kernel(const __nv_bfloat16 *x, int64_t M, int64_t K,
                                                             int64_t n_counters, GemvWorkspace ws) {
   pdl_launch_dependents();  // the streaming kernel may start fetching weights now
@@ -549,24 +630,43 @@ __global__ void __launch_bounds__(256) gemv_xprep_mt_kernel(const __nv_bfloat16 
   }
   amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
   amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-  const int a = scale_exponent(amax, 14);  // max |x_int| < 2^15
+  const int a16 = scale_exponent(amax, 14);  // max |x_int| < 2^15
+  const float s16 = exp2i(a16);
+  float err = 0.f, mass = 0.f;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const float sv = xs[k] * s16;
+    err += fabsf(sv - rintf(sv));
+    mass += fabsf(sv);
+  }
+  const bool wide = group_needs_24bit(err, mass, amax * s16);
+  const bool sb24 = __any_sync(0xffffffffu, wide && live);  // the warp holds one (token, super-block)
+  const int a = sb24 ? scale_exponent(amax, 22) : a16;     // 24-bit: max |x_int| < 2^23
   const float sc = exp2i(a);
-  uint32_t eh = 0, oh = 0, el = 0, ol = 0;
+  const int hs = sb24 ? 16 : 8;  // the value's top byte: bits 16.. (24-bit) or 8.. (16-bit, lo = 0)
+  uint32_t eh = 0, oh = 0, em = 0, om = 0, el = 0, ol = 0;
   int sum = 0;
 #pragma unroll
   for (int b = 0; b < 4; ++b) {
     const int xe = __float2int_rn(xs[2 * b] * sc), xo = __float2int_rn(xs[2 * b + 1] * sc);
     sum += xe + xo;
-    eh |= ((uint32_t)(xe >> 8) & 0xffu) << (8 * b);
-    el |= ((uint32_t)xe & 0xffu) << (8 * b);
-    oh |= ((uint32_t)(xo >> 8) & 0xffu) << (8 * b);
-    ol |= ((uint32_t)xo & 0xffu) << (8 * b);
+    eh |= ((uint32_t)(xe >> hs) & 0xffu) << (8 * b);
+    em |= ((uint32_t)(xe >> (hs - 8)) & 0xffu) << (8 * b);
+    el |= (sb24 ? ((uint32_t)xe & 0xffu) : 0u) << (8 * b);
+    oh |= ((uint32_t)(xo >> hs) & 0xffu) << (8 * b);
+    om |= ((uint32_t)(xo >> (hs - 8)) & 0xffu) << (8 * b);
+    ol |= (sb24 ? ((uint32_t)xo & 0xffu) : 0u) << (8 * b);
   }
   sum += __shfl_xor_sync(0xffffffffu, sum, 1);
   sum += __shfl_xor_sync(0xffffffffu, sum, 2);
   if (!live) return;
-  ws.xq[(g * M + m) * 4 + c] = make_uint4(eh, oh, el, ol);
-  if (c == 0) ws.gsum[g * M + m] = make_float2(exp2i(-a) * 0.0625f, -16.f * (float)sum);
+  ws.xq[(g * M + m) * 4 + c] = make_uint4(eh, oh, em, om);
+  reinterpret_cast<uint2 *>(ws.xq + M * K / 8)[(g * M + m) * 4 + c] = make_uint2(el, ol);
+  if (c == 0) {  // (G_x, G_y) = (2^-a / (16 * 2^u), -16 * 2^u * X), u = 0 (24-bit) or 8 (16-bit)
+    const float w = sb24 ? 16.f : 4096.f;
+    ws.gsum[g * M + m] = make_float2(exp2i(-a) / w, -w * (float)sum);
+  }
+  if ((threadIdx.x & 31) == 0) ws.flags[(g >> 3) * 16 + m] = sb24 ? 1 : 0;
 }
 
 constexpr int GEMV_MT_WARPS = 4;  // consumer warps per CTA; warp 4 produces
@@ -575,8 +675,9 @@ constexpr int GEMV_MT_CTAS_PER_SM = 3;
 
 // Stage layout of the multi-token kernel per format, for one 256-weight super-block of 64 rows:
 // codes [64 rows][CODE_ROW B] as swizzled boxes of CODE_BOX B (128-byte swizzle; 64-byte swizzle for
-// the 64-byte rows of 2-bit codes), group words [64][META_ROW B], group sums [8][M][8 B], x words
-// [8 groups][M][4][16 B].  int4 and 4-bit affine codes share one layout (a nibble per weight, low
+// the 64-byte rows of 2-bit codes), group words [64][META_ROW B], group sums [8][M][8 B], (hi, mid) x
+// words [8 groups][M][4][16 B] and the 24-bit flags [16 B]; a 24-bit super-block's lo x words are read
+// from global memory.  int4 and 4-bit affine codes share one layout (a nibble per weight, low
 // nibble first); 8-bit affine codes are bytes; 2-bit codes are 16 per word, lowest bits first.
 template <int FMT, int BITS, int G>
 struct MtLayout {
@@ -587,7 +688,8 @@ struct MtLayout {
   static constexpr int ST_GMETA = CODE_BOXES * 64 * CODE_BOX;
   static constexpr int ST_GSUM = ST_GMETA + 64 * META_ROW;
   static constexpr int ST_X = ST_GSUM + 512;
-  static constexpr int STAGE = (ST_X + 4096 + 1023) / 1024 * 1024;
+  static constexpr int ST_FL = ST_X + 4096;  // 16 B: a byte per token, non-zero when its x is 24-bit
+  static constexpr int STAGE = (ST_FL + 16 + 1023) / 1024 * 1024;
   static constexpr int RING = 3 * (4 * STAGE + 1024) <= 227 * 1024 ? 4 : 3;
   static constexpr int SMEM = RING * STAGE + RING * 16 + 16 + 1024;
 };
@@ -646,7 +748,7 @@ __global__ void __launch_bounds__(GEMV_MT_THREADS, GEMV_MT_CTAS_PER_SM)
     if (lane == 0) {
       tma_prefetch_desc(&map_codes);
       tma_prefetch_desc(&map_gmeta);
-      const uint32_t tx = L::ST_GSUM + (uint32_t)M * 64 + (uint32_t)M * 512;  // codes + group words + sums + x
+      const uint32_t tx = L::ST_GSUM + (uint32_t)M * (64 + 512) + 16;  // codes, group words, sums, x, flags
       auto issue_w = [&](int i, int s) {
         const uint32_t st = sbase + s * L::STAGE;
         mbar_arrive_expect_tx(bar_full(s), tx);
@@ -661,8 +763,10 @@ __global__ void __launch_bounds__(GEMV_MT_THREADS, GEMV_MT_CTAS_PER_SM)
         const int64_t g0 = (int64_t)(sb0 + i) * 8;  // first 32-element group of the super-block
         bulk_load(st + L::ST_GSUM, p.ws.gsum + g0 * M, (uint32_t)M * 64, bar_full(s));
         bulk_load(st + L::ST_X, p.ws.xq + g0 * M * 4, (uint32_t)M * 512, bar_full(s));
+        bulk_load(st + L::ST_FL, p.ws.flags + (sb0 + i) * 16, 16, bar_full(s));
       };
-      const int pre = nsb < RING ? nsb : RING;
+      const bool hold = copies_withheld();
+      const int pre = hold ? 0 : (nsb < RING ? nsb : RING);
       for (int i = 0; i < pre; ++i) issue_w(i, i);  // weights need no x
       pdl_wait();
       for (int i = 0; i < pre; ++i) issue_x(i, i);
@@ -670,7 +774,7 @@ __global__ void __launch_bounds__(GEMV_MT_THREADS, GEMV_MT_CTAS_PER_SM)
       uint32_t ph = 0;
       bool ok = true;
       int i = pre;
-      for (; i < nsb; ++i) {  // unit i reuses the stage of unit i - RING
+      for (; i < nsb && !hold; ++i) {  // unit i reuses the stage of unit i - RING
         if (!mbar_wait_bounded(bar_empty(s), ph, abort_flag)) {
           ok = false;
           break;
@@ -711,6 +815,7 @@ __global__ void __launch_bounds__(GEMV_MT_THREADS, GEMV_MT_CTAS_PER_SM)
       }
     }
     const int32_t acc_init[4] = {GEMV_ACC0, GEMV_ACC0, GEMV_ACC0, GEMV_ACC0};
+    const uint2 *xlg = reinterpret_cast<const uint2 *>(p.ws.xq + (int64_t)M * p.K / 8);  // lo x words
     float acc[4] = {0.f, 0.f, 0.f, 0.f};  // (row g | g + 8) x (token 2c | 2c + 1)
     const uint32_t sw = (uint32_t)(r0 & 7);
     bool ok = true;
@@ -732,6 +837,12 @@ __global__ void __launch_bounds__(GEMV_MT_THREADS, GEMV_MT_CTAS_PER_SM)
           break;
         }
         const uint32_t stg = sbase + s * L::STAGE;
+        bool x24;  // some token's x of this super-block is 24-bit: the low-byte MMA runs (the same for the warp)
+        {
+          const uint2 fw = lds64(stg + L::ST_FL);
+          const uint64_t f = ((uint64_t)fw.y << 32 | fw.x) & (M >= 8 ? ~0ull : ((1ull << (8 * M)) - 1));
+          x24 = f != 0;
+        }
         // group words of rows r0, r1 (int4: 8 x u16 sc|zc; affine: 256/G x u32 s|b)
         uint32_t gw0[L::META_ROW / 4], gw1[L::META_ROW / 4];
 #pragma unroll
@@ -749,65 +860,79 @@ __global__ void __launch_bounds__(GEMV_MT_THREADS, GEMV_MT_CTAS_PER_SM)
           nss0 = -8388608.f * ss0; nzs0 = -8388608.f * zs0;
           nss1 = -8388608.f * ss1; nzs1 = -8388608.f * zs1;
         }
-#pragma unroll
-        for (int gg = 0; gg < 8; ++gg) {
-          uint32_t e0, e1, o0, o1;  // A: even-k and odd-k codes of rows r0, r1 (x16 for nibbles)
-          if constexpr (FMT == FMT_INT4 || BITS == 4) {
-            const uint32_t coff = (((uint32_t)gg ^ sw) << 4) + 4 * c;
-            const uint32_t w0 = lds32(stg + r0 * 128 + coff), w1 = lds32(stg + r1 * 128 + coff);
-            e0 = (w0 << 4) & 0xF0F0F0F0u; e1 = (w1 << 4) & 0xF0F0F0F0u;
-            o0 = w0 & 0xF0F0F0F0u; o1 = w1 & 0xF0F0F0F0u;
-          } else if constexpr (BITS == 2) {
-            // 2-bit: slice gg is 8 B of the 64-byte row (64-byte swizzle: 16-byte chunk ^ (row / 2) % 4);
-            // lane c takes the half-word of k = 8c .. 8c + 7, spreads its nibbles to bytes (one byte
-            // permute, one shift-or) and splits even and odd k with two masks
-            const uint32_t off = ((((uint32_t)gg >> 1) ^ (((uint32_t)r0 >> 1) & 3u)) << 4) + 8 * (gg & 1) + 4 * (c >> 1);
-            const uint32_t sel = (c & 1) ? 0x4342u : 0x4140u;
-            const uint32_t t0 = __byte_perm(lds32(stg + r0 * 64 + off), 0u, sel);
-            const uint32_t t1 = __byte_perm(lds32(stg + r1 * 64 + off), 0u, sel);
-            const uint32_t u0 = (t0 | (t0 << 4)) & 0x0F0F0F0Fu, u1 = (t1 | (t1 << 4)) & 0x0F0F0F0Fu;
-            e0 = u0 & 0x03030303u; e1 = u1 & 0x03030303u;
-            o0 = (u0 >> 2) & 0x03030303u; o1 = (u1 >> 2) & 0x03030303u;
-          } else {  // bytes: slice gg is 32 B of box gg / 4; lane c takes bytes 8c .. 8c + 7
-            const uint32_t ch = (uint32_t)(2 * (gg & 3) + (c >> 1));
-            const uint32_t off = (uint32_t)(gg >> 2) * 8192 + ((ch ^ sw) << 4) + 8 * (c & 1);
-            const uint2 w0 = lds64(stg + r0 * 128 + off), w1 = lds64(stg + r1 * 128 + off);
-            e0 = __byte_perm(w0.x, w0.y, 0x6420); e1 = __byte_perm(w1.x, w1.y, 0x6420);
-            o0 = __byte_perm(w0.x, w0.y, 0x7531); o1 = __byte_perm(w1.x, w1.y, 0x7531);
+        const int64_t g0s = (int64_t)(sb0 + i) * 8;  // the super-block's first 32-element group
+        auto groups = [&](auto x24c) {  // the stage's eight groups: two bytes of x, or three for 24-bit x
+          constexpr bool X24 = decltype(x24c)::value;
+  #pragma unroll
+          for (int gg = 0; gg < 8; ++gg) {
+            uint32_t e0, e1, o0, o1;  // A: even-k and odd-k codes of rows r0, r1 (x16 for nibbles)
+            if constexpr (FMT == FMT_INT4 || BITS == 4) {
+              const uint32_t coff = (((uint32_t)gg ^ sw) << 4) + 4 * c;
+              const uint32_t w0 = lds32(stg + r0 * 128 + coff), w1 = lds32(stg + r1 * 128 + coff);
+              e0 = (w0 << 4) & 0xF0F0F0F0u; e1 = (w1 << 4) & 0xF0F0F0F0u;
+              o0 = w0 & 0xF0F0F0F0u; o1 = w1 & 0xF0F0F0F0u;
+            } else if constexpr (BITS == 2) {
+              // 2-bit: slice gg is 8 B of the 64-byte row (64-byte swizzle: 16-byte chunk ^ (row / 2) % 4);
+              // lane c takes the half-word of k = 8c .. 8c + 7, spreads its nibbles to bytes (one byte
+              // permute, one shift-or) and splits even and odd k with two masks
+              const uint32_t off = ((((uint32_t)gg >> 1) ^ (((uint32_t)r0 >> 1) & 3u)) << 4) + 8 * (gg & 1) + 4 * (c >> 1);
+              const uint32_t sel = (c & 1) ? 0x4342u : 0x4140u;
+              const uint32_t t0 = __byte_perm(lds32(stg + r0 * 64 + off), 0u, sel);
+              const uint32_t t1 = __byte_perm(lds32(stg + r1 * 64 + off), 0u, sel);
+              const uint32_t u0 = (t0 | (t0 << 4)) & 0x0F0F0F0Fu, u1 = (t1 | (t1 << 4)) & 0x0F0F0F0Fu;
+              e0 = u0 & 0x03030303u; e1 = u1 & 0x03030303u;
+              o0 = (u0 >> 2) & 0x03030303u; o1 = (u1 >> 2) & 0x03030303u;
+            } else {  // bytes: slice gg is 32 B of box gg / 4; lane c takes bytes 8c .. 8c + 7
+              const uint32_t ch = (uint32_t)(2 * (gg & 3) + (c >> 1));
+              const uint32_t off = (uint32_t)(gg >> 2) * 8192 + ((ch ^ sw) << 4) + 8 * (c & 1);
+              const uint2 w0 = lds64(stg + r0 * 128 + off), w1 = lds64(stg + r1 * 128 + off);
+              e0 = __byte_perm(w0.x, w0.y, 0x6420); e1 = __byte_perm(w1.x, w1.y, 0x6420);
+              o0 = __byte_perm(w0.x, w0.y, 0x7531); o1 = __byte_perm(w1.x, w1.y, 0x7531);
+            }
+            const uint4 xv = lds128(stg + L::ST_X + ((gg * M + g) * 4 + c) * 16);
+            // (2^-a/16, -16 X) of tokens 2c and 2c + 1: 8-byte records, so two 8-byte loads (odd M)
+            const float2 Ga = lds64f(stg + L::ST_GSUM + (gg * M + 2 * c) * 8);
+            const float2 Gb = lds64f(stg + L::ST_GSUM + (gg * M + 2 * c + 1) * 8);
+            int32_t dh[4], dm[4], dl[4];
+            QL_IMMA0("s8", dh, acc_init, e0, e1, o0, o1, xv.x, xv.y);
+            QL_IMMA0("u8", dm, acc_init, e0, e1, o0, o1, xv.z, xv.w);
+            if constexpr (X24) {  // the low byte of 24-bit x, from global memory (L2); token g's column
+              const uint2 xl = g < M ? __ldg(xlg + ((int64_t)(g0s + gg) * M + g) * 4 + c) : make_uint2(0u, 0u);
+              QL_IMMA0("u8", dl, acc_init, e0, e1, o0, o1, xl.x, xl.y);
+            }
+            float t[4];  // T = 65536 D_hi + 256 D_mid + D_lo
+  #pragma unroll
+            for (int q = 0; q < 4; ++q)
+            {
+              t[q] = fmaf(__int_as_float(dh[q]) - GEMV_ACC0_F, 256.f, __int_as_float(dm[q]) - GEMV_ACC0_F);
+              if constexpr (X24) t[q] = fmaf(t[q], 256.f, __int_as_float(dl[q]) - GEMV_ACC0_F);
+              else t[q] *= 256.f;
+            }
+            if constexpr (FMT == FMT_INT4) {
+              const uint32_t gw0g = gw0[gg >> 1], gw1g = gw1[gg >> 1];
+              const int bsc = 2 * (gg & 1);
+              const float S0 = fmaf(byte_magic(gw0g, bsc), ss0, nss0), Z0 = fmaf(byte_magic(gw0g, bsc + 1), zs0, nzs0);
+              const float S1 = fmaf(byte_magic(gw1g, bsc), ss1, nss1), Z1 = fmaf(byte_magic(gw1g, bsc + 1), zs1, nzs1);
+              acc[0] = fmaf(S0 * Ga.x, fmaf(Z0, Ga.y, t[0]), acc[0]);
+              acc[1] = fmaf(S0 * Gb.x, fmaf(Z0, Gb.y, t[1]), acc[1]);
+              acc[2] = fmaf(S1 * Ga.x, fmaf(Z1, Ga.y, t[2]), acc[2]);
+              acc[3] = fmaf(S1 * Gb.x, fmaf(Z1, Gb.y, t[3]), acc[3]);
+            } else {
+              // slice gg lies in affine group gg * 32 / G of the super-block; its word holds (s, b) bf16
+              const uint32_t gw0g = gw0[gg * 32 / G], gw1g = gw1[gg * 32 / G];
+              constexpr float SF = BITS == 4 ? 1.f : 16.f;  // nibbles carry 16 q, 2-bit fields and bytes q
+              const float s0 = bf16_bits_to_f32(gw0g) * SF, b0 = bf16_bits_to_f32(gw0g >> 16);
+              const float s1 = bf16_bits_to_f32(gw1g) * SF, b1 = bf16_bits_to_f32(gw1g >> 16);
+              // b 2^-a X = -b (2^-a/16)(-16 X)
+              acc[0] = fmaf(s0 * Ga.x, t[0], fmaf(-b0 * Ga.x, Ga.y, acc[0]));
+              acc[1] = fmaf(s0 * Gb.x, t[1], fmaf(-b0 * Gb.x, Gb.y, acc[1]));
+              acc[2] = fmaf(s1 * Ga.x, t[2], fmaf(-b1 * Ga.x, Ga.y, acc[2]));
+              acc[3] = fmaf(s1 * Gb.x, t[3], fmaf(-b1 * Gb.x, Gb.y, acc[3]));
+            }
           }
-          const uint4 xv = lds128(stg + L::ST_X + ((gg * M + g) * 4 + c) * 16);
-          // (2^-a/16, -16 X) of tokens 2c and 2c + 1: 8-byte records, so two 8-byte loads (odd M)
-          const float2 Ga = lds64f(stg + L::ST_GSUM + (gg * M + 2 * c) * 8);
-          const float2 Gb = lds64f(stg + L::ST_GSUM + (gg * M + 2 * c + 1) * 8);
-          int32_t dh[4], dl[4];
-          QL_IMMA0("s8", dh, acc_init, e0, e1, o0, o1, xv.x, xv.y);
-          QL_IMMA0("u8", dl, acc_init, e0, e1, o0, o1, xv.z, xv.w);
-          float t[4];
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            t[q] = fmaf(__int_as_float(dh[q]) - GEMV_ACC0_F, 256.f, __int_as_float(dl[q]) - GEMV_ACC0_F);
-          if constexpr (FMT == FMT_INT4) {
-            const uint32_t gw0g = gw0[gg >> 1], gw1g = gw1[gg >> 1];
-            const int bsc = 2 * (gg & 1);
-            const float S0 = fmaf(byte_magic(gw0g, bsc), ss0, nss0), Z0 = fmaf(byte_magic(gw0g, bsc + 1), zs0, nzs0);
-            const float S1 = fmaf(byte_magic(gw1g, bsc), ss1, nss1), Z1 = fmaf(byte_magic(gw1g, bsc + 1), zs1, nzs1);
-            acc[0] = fmaf(S0 * Ga.x, fmaf(Z0, Ga.y, t[0]), acc[0]);
-            acc[1] = fmaf(S0 * Gb.x, fmaf(Z0, Gb.y, t[1]), acc[1]);
-            acc[2] = fmaf(S1 * Ga.x, fmaf(Z1, Ga.y, t[2]), acc[2]);
-            acc[3] = fmaf(S1 * Gb.x, fmaf(Z1, Gb.y, t[3]), acc[3]);
-          } else {
-            // slice gg lies in affine group gg * 32 / G of the super-block; its word holds (s, b) bf16
-            const uint32_t gw0g = gw0[gg * 32 / G], gw1g = gw1[gg * 32 / G];
-            constexpr float SF = BITS == 4 ? 1.f : 16.f;  // nibbles carry 16 q, 2-bit fields and bytes q
-            const float s0 = bf16_bits_to_f32(gw0g) * SF, b0 = bf16_bits_to_f32(gw0g >> 16);
-            const float s1 = bf16_bits_to_f32(gw1g) * SF, b1 = bf16_bits_to_f32(gw1g >> 16);
-            // b 2^-a X = -b (2^-a/16)(-16 X)
-            acc[0] = fmaf(s0 * Ga.x, t[0], fmaf(-b0 * Ga.x, Ga.y, acc[0]));
-            acc[1] = fmaf(s0 * Gb.x, t[1], fmaf(-b0 * Gb.x, Gb.y, acc[1]));
-            acc[2] = fmaf(s1 * Ga.x, t[2], fmaf(-b1 * Ga.x, Ga.y, acc[2]));
-            acc[3] = fmaf(s1 * Gb.x, t[3], fmaf(-b1 * Gb.x, Gb.y, acc[3]));
-          }
-        }
+        };
+        if (x24) groups(std::true_type{});
+        else groups(std::false_type{});
         __syncwarp();
         if (lane == 0) mbar_arrive(bar_empty(s));
       }

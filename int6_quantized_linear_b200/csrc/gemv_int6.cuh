@@ -1,4 +1,5 @@
-// Tensor-core decode GEMV for the symmetric int6 format at 1 <= M <= 8 tokens.
+// Tensor-core decode GEMV for the symmetric int6 format at 1 <= M <= 8 tokens, for both storages
+// of its codes (dense, and planar: see int6p_a_words).
 //
 // Format (ExecuTorch PR "[cuda] Nestest Superscale Quantization for CUDA Weights
 // (int4 / int6)", "Quant schema update", int6 bullet): 6-bit two's-complement
@@ -15,12 +16,16 @@
 // A registers (4 q as s8, the codes in the top six bits of each byte) with two
 // byte permutes, at most two shifts and one or two masks each; the k-step j
 // register holds codes int6_kperm(j, 0..3), and the x bytes are written in the
-// same order by the preparation pass.  x enters as 16-bit fixed point per
-// 16-element group, x_int = rint(x * 2^a) with max |x_int| in [2^14, 2^15),
-// split into a signed high and an unsigned low byte, one MMA each; per (row,
-// group) both sums are exact below 2^19, so the accumulators start at the bits
-// of 1.5 * 2^23 and read back with one subtraction:
-//     T = sum_k 4 q_k x_int_k = 256 D_hi + D_lo,    y += S (2^-a / 4) T
+// same order by the preparation pass.  x enters as fixed point per 16-element
+// group, x_int = rint(x * 2^a): 16-bit (max |x_int| in [2^14, 2^15)) or, for a
+// super-block whose 16-bit form would lose too much (as in the int4 kernels),
+// 24-bit (max |x_int| in [2^22, 2^23): exact for every bf16 element within 2^15
+// of the group's largest magnitude), split into a signed high and unsigned
+// middle and low bytes, one MMA each (the low byte only for 24-bit); per (row,
+// group) the sums are exact below 2^19, so the accumulators start at the bits of
+// 1.5 * 2^23 and read back with one subtraction:
+//     T = 65536 D_hi + 256 D_mid + D_lo = 4 * 2^u * sum_k q_k x_int_k,
+//     y += S (2^-a / (4 * 2^u)) T,   u = 0 (24-bit) or 8 (16-bit)
 // with S = code * step (exact in fp32).
 //
 // A CTA is a producer warp and four consumer warps on 64 weight rows and a
@@ -37,9 +42,12 @@
 
 namespace ql {
 
-// Byte b of the k-step j A register holds code int6_kperm(j, b) of the group (times 4).
+// Byte b of the k-step j A register holds code int6_kperm(j, b) of the group (times 4).  Dense
+// storage: the order two byte permutes per register give; planar storage: code 4b + j.
+template <bool PLANAR>
 __host__ __device__ constexpr int int6_kperm(int j, int b) {
-  return j == 0 ? 4 * b
+  return PLANAR ? 4 * b + j
+       : j == 0 ? 4 * b
        : j == 1 ? (b == 0 ? 9 : b == 1 ? 1 : b == 2 ? 13 : 5)
        : j == 2 ? (b == 0 ? 2 : b == 1 ? 10 : b == 2 ? 6 : 14)
                 : 4 * b + 3;
@@ -59,10 +67,28 @@ QL_DEVI void int6_a_words(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t (&a)[4
   a[3] = t3 & 0xFCFCFCFCu;
 }
 
-// x preparation: one thread per (token, 16-element group).  Entry (sb, m, set, j, gi) of the x words
-// is the B pair of k-step j for group 8 set + gi: (hi, 0, lo, 0) for gi < 4 (its lane feeds b0),
-// (0, hi, 0, lo) for gi >= 4 (b1); the group scale 2^-a / 4 goes to gscale[sb][m][16].
+// Planar storage (a 4-bit and a 2-bit plane per super-block, as the review of the ExecuTorch PR
+// describes the reference int6 kernel's loads): the four A registers of one group from its two
+// low-plane words l0, l1 (nibble i = code i, i < 8 in l0) and its high-plane word h (bits 2i, 2i+1 =
+// bits 4-5 of code i).  Register j takes codes j, 4 + j, 8 + j, 12 + j: their nibbles are the low (j
+// even) or high (j odd) halves of bytes j/2 and 2 + j/2 of l0 and of l1 (one byte permute per pair of
+// registers), and their high fields sit at bits 2j of each byte of h.
+QL_DEVI void int6p_a_words(uint32_t l0, uint32_t l1, uint32_t h, uint32_t (&a)[4]) {
+  const uint32_t t01 = __byte_perm(l0, l1, 0x6420), t23 = __byte_perm(l0, l1, 0x7531);
+  a[0] = ((t01 << 2) & 0x3C3C3C3Cu) | ((h << 6) & 0xC0C0C0C0u);
+  a[1] = ((t01 >> 2) & 0x3C3C3C3Cu) | ((h << 4) & 0xC0C0C0C0u);
+  a[2] = ((t23 << 2) & 0x3C3C3C3Cu) | ((h << 2) & 0xC0C0C0C0u);
+  a[3] = ((t23 >> 2) & 0x3C3C3C3Cu) | (h & 0xC0C0C0C0u);
+}
+
+// x preparation: one thread per (token, 16-element group), so a half-warp holds one token's 16 groups
+// of a super-block (16- or 24-bit as in the int4 kernels; the flag byte [sb][m] says which).  Entry
+// (sb, m, set, j, gi) of the x words
+// is the B pairs of k-step j for group 8 set + gi: (hi, 0, mid, 0) for gi < 4 (its lane feeds b0),
+// (0, hi, 0, mid) for gi >= 4 (b1), and (lo, 0) or (0, lo) in the low-byte region that follows the
+// K/256 * M * 1024 bytes of the first; the group scale 2^-a / 4 goes to gscale[sb][m][16].
 // Also zeroes the first n_counters row-group counters.
+template <bool PLANAR>
 __global__ void __launch_bounds__(256) gemv_xprep_int6_kernel(const __nv_bfloat16 *x, int64_t M, int64_t K,
                                                               int64_t n_counters, GemvWorkspace ws) {
   pdl_launch_dependents();  // the streaming kernel may start fetching weights now
@@ -70,10 +96,14 @@ __global__ void __launch_bounds__(256) gemv_xprep_int6_kernel(const __nv_bfloat1
   const int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
   if (t < n_counters) ws.counters[t] = 0;
   const int64_t ng = K / 16;
-  if (t >= M * ng) return;
-  const int64_t m = t / ng, gg = t - m * ng;
+  const bool live = t < M * ng;  // every lane takes part in the ballot below
+  const int64_t m = live ? t / ng : 0, gg = live ? t - m * ng : 0;
   const uint4 *src = reinterpret_cast<const uint4 *>(x + m * K + 16 * gg);
-  const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
+  uint4 v0 = make_uint4(0u, 0u, 0u, 0u), v1 = v0;
+  if (live) {
+    v0 = __ldg(src);
+    v1 = __ldg(src + 1);
+  }
   const uint32_t u[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
   float xs[16];
   float amax = 0.f;
@@ -83,26 +113,48 @@ __global__ void __launch_bounds__(256) gemv_xprep_int6_kernel(const __nv_bfloat1
     xs[2 * i + 1] = bf16_bits_to_f32(u[i] >> 16);
     amax = fmaxf(amax, fmaxf(fabsf(xs[2 * i]), fabsf(xs[2 * i + 1])));
   }
-  const int a = scale_exponent(amax, 14);  // bf16 inputs: max |x_int| <= (2 - 2^-7) 2^14 < 2^15
+  // 16-bit fixed point unless some group of this (token, super-block) -- the 16 threads of a
+  // half-warp -- would lose too much (see group_needs_24bit): then all 16 groups are 24-bit
+  const int a16 = scale_exponent(amax, 14);
+  const float s16 = exp2i(a16);
+  float err = 0.f, mass = 0.f;
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    const float sv = xs[k] * s16;
+    err += fabsf(sv - rintf(sv));
+    mass += fabsf(sv);
+  }
+  const bool wide = live && err > (mass - amax * s16) * (1.f / 4096.f);
+  const uint32_t ballot = __ballot_sync(0xffffffffu, wide);
+  const bool sb24 = ((ballot >> (threadIdx.x & 16)) & 0xffffu) != 0u;
+  const int a = sb24 ? scale_exponent(amax, 22) : a16;  // bf16 inputs: max |x_int| < 2^23 (2^15 for 16-bit)
   const float sc = exp2i(a);
+  const int hs = sb24 ? 16 : 8;  // the value's top byte: bits 16.. (24-bit) or 8.. (16-bit, lo = 0)
   int xi[16];
 #pragma unroll
   for (int k = 0; k < 16; ++k) xi[k] = __float2int_rn(xs[k] * sc);
+  if (!live) return;
   const int64_t sb = gg >> 4;
   const int gl = (int)(gg & 15), set = gl >> 3, gi = gl & 7;
-  uint4 *dst = ws.xq + (((sb * M + m) * 2 + set) * 4) * 8 + gi;
+  const int64_t ent = (((sb * M + m) * 2 + set) * 4) * 8 + gi;
+  uint4 *dst = ws.xq + ent;
+  uint2 *dst8 = reinterpret_cast<uint2 *>(ws.xq + (K / 256) * M * 64) + ent;
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    uint32_t hi = 0, lo = 0;
+    uint32_t hi = 0, mid = 0, lo = 0;
 #pragma unroll
     for (int b = 0; b < 4; ++b) {
-      const int v = xi[int6_kperm(j, b)];
-      hi |= ((uint32_t)(v >> 8) & 0xffu) << (8 * b);
-      lo |= ((uint32_t)v & 0xffu) << (8 * b);
+      const int v = xi[int6_kperm<PLANAR>(j, b)];
+      hi |= ((uint32_t)(v >> hs) & 0xffu) << (8 * b);
+      mid |= ((uint32_t)(v >> (hs - 8)) & 0xffu) << (8 * b);
+      lo |= (sb24 ? ((uint32_t)v & 0xffu) : 0u) << (8 * b);
     }
-    dst[8 * j] = gi < 4 ? make_uint4(hi, 0u, lo, 0u) : make_uint4(0u, hi, 0u, lo);
+    dst[8 * j] = gi < 4 ? make_uint4(hi, 0u, mid, 0u) : make_uint4(0u, hi, 0u, mid);
+    dst8[8 * j] = gi < 4 ? make_uint2(lo, 0u) : make_uint2(0u, lo);
   }
-  reinterpret_cast<float *>(ws.gsum)[(sb * M + m) * 16 + gl] = exp2i(-a) * 0.25f;
+  // the group scale 2^-a / (4 * 2^u), u = 0 (24-bit) or 8 (16-bit): T below is 4 * 2^u * sum q x_int
+  reinterpret_cast<float *>(ws.gsum)[(sb * M + m) * 16 + gl] = exp2i(-a) * (sb24 ? 0.25f : 0.25f / 256.f);
+  if (gl == 0) ws.flags[sb * 16 + m] = sb24 ? 1 : 0;
 }
 
 #define QL_IMMA6_0(TB, ACC, C, A0, A1, A2, A3, B0, B1)                                                \
@@ -122,15 +174,20 @@ constexpr int GEMV6_CTAS_PER_SM = 3;
 constexpr int GEMV6_CODE_ROW = 208;  // bytes per row in a stage: 192 of the super-block + 16 of the next
 
 // Stage layout for up to TM tokens: codes [64][208], scale codes [64][16], group scales [TM][16] f32,
-// x words [TM][2 sets][4 k-steps][8 groups][16 B].
+// (hi, mid) x words [TM][2 sets][4 k-steps][8 groups][16 B] and the 24-bit flags [16 B] (a 24-bit
+// super-block's lo x words are read from global memory).  The ring is as deep (4, 3 or 2 stages) as
+// three CTAs per SM allow.
 template <int TM>
 struct Int6Layout {
   static constexpr int ST_SC = 64 * GEMV6_CODE_ROW;
   static constexpr int ST_G = ST_SC + 64 * 16;
   static constexpr int ST_X = ST_G + TM * 64;
-  static constexpr int STAGE = (ST_X + TM * 1024 + 127) / 128 * 128;
+  static constexpr int ST_FL = ST_X + TM * 1024;  // 16 B: a byte per token, non-zero when its x is 24-bit
+  static constexpr int STAGE = (ST_FL + 16 + 127) / 128 * 128;
   static constexpr int EXTRA = 16 + 2 * 4 * 8 + 16 + 128;  // zero slot, barriers, flags, alignment
-  static constexpr int RING = GEMV6_CTAS_PER_SM * (4 * STAGE + EXTRA + 1024) <= 233472 ? 4 : 3;
+  static constexpr int RING = GEMV6_CTAS_PER_SM * (4 * STAGE + EXTRA + 1024) <= 233472   ? 4
+                            : GEMV6_CTAS_PER_SM * (3 * STAGE + EXTRA + 1024) <= 233472 ? 3
+                                                                                        : 2;
   static constexpr int SMEM = RING * STAGE + EXTRA;
 };
 
@@ -144,7 +201,7 @@ struct Gemv6Params {
   __nv_bfloat16 *y;
 };
 
-template <int TM>
+template <int TM, bool PLANAR>
 __global__ void __launch_bounds__(GEMV6_THREADS, GEMV6_CTAS_PER_SM)
     gemv_int6_kernel(const __grid_constant__ CUtensorMap map_codes, const __grid_constant__ CUtensorMap map_sc,
                      Gemv6Params p) {
@@ -183,7 +240,7 @@ __global__ void __launch_bounds__(GEMV6_THREADS, GEMV6_CTAS_PER_SM)
     if (lane == 0) {
       tma_prefetch_desc(&map_codes);
       tma_prefetch_desc(&map_sc);
-      const uint32_t tx = (uint32_t)L::ST_G + (uint32_t)M * (64 + 1024);
+      const uint32_t tx = (uint32_t)L::ST_G + (uint32_t)M * (64 + 1024) + 16;
       const float *gscale = reinterpret_cast<const float *>(p.ws.gsum);
       auto issue_w = [&](int i, int s) {
         const uint32_t st = sbase + s * L::STAGE;
@@ -196,8 +253,10 @@ __global__ void __launch_bounds__(GEMV6_THREADS, GEMV6_CTAS_PER_SM)
         const int64_t sb = sb0 + i;
         bulk_load(st + L::ST_G, gscale + sb * M * 16, (uint32_t)M * 64, bar_full(s));
         bulk_load(st + L::ST_X, p.ws.xq + sb * M * 64, (uint32_t)M * 1024, bar_full(s));
+        bulk_load(st + L::ST_FL, p.ws.flags + sb * 16, 16, bar_full(s));
       };
-      const int pre = nsb < RING ? nsb : RING;
+      const bool hold = copies_withheld();
+      const int pre = hold ? 0 : (nsb < RING ? nsb : RING);
       for (int i = 0; i < pre; ++i) issue_w(i, i);  // weights need no x
       pdl_wait();
       for (int i = 0; i < pre; ++i) issue_x(i, i);
@@ -205,7 +264,7 @@ __global__ void __launch_bounds__(GEMV6_THREADS, GEMV6_CTAS_PER_SM)
       uint32_t ph = 0;
       bool ok = true;
       int i = pre;
-      for (; i < nsb; ++i) {  // unit i reuses the stage of unit i - RING
+      for (; i < nsb && !hold; ++i) {  // unit i reuses the stage of unit i - RING
         if (!mbar_wait_bounded(bar_empty(s), ph, abort_flag)) {
           ok = false;
           break;
@@ -246,6 +305,7 @@ __global__ void __launch_bounds__(GEMV6_THREADS, GEMV6_CTAS_PER_SM)
     const bool on = (g & 3) == c;
     const uint32_t zero_a = smem_u32(zero16);
     const int32_t acc_init[4] = {GEMV_ACC0, GEMV_ACC0, GEMV_ACC0, GEMV_ACC0};
+    const uint2 *xlg = reinterpret_cast<const uint2 *>(p.ws.xq + (p.K / 256) * M * 64);  // lo x words
     float acc[TM][2];  // (token) x (row r0 | r1)
 #pragma unroll
     for (int m = 0; m < TM; ++m) acc[m][0] = acc[m][1] = 0.f;
@@ -266,6 +326,12 @@ __global__ void __launch_bounds__(GEMV6_THREADS, GEMV6_CTAS_PER_SM)
           break;
         }
         const uint32_t stg = sbase + s * L::STAGE;
+        bool x24;  // some token's x of this super-block is 24-bit: the low-byte MMA runs (the same for the warp)
+        {
+          const uint2 fw = lds64(stg + L::ST_FL);
+          const uint64_t f = ((uint64_t)fw.y << 32 | fw.x) & (M >= 8 ? ~0ull : ((1ull << (8 * M)) - 1));
+          x24 = f != 0;
+        }
         const float stp0 = f16_bits_to_f32(sr0[s]), stp1 = f16_bits_to_f32(sr1[s]);
         // scale codes of the D columns: groups 8 set + 2c, 8 set + 2c + 1 of rows r0, r1
         const uint32_t scw00 = lds32(stg + L::ST_SC + r0 * 16 + 4 * (c >> 1));
@@ -281,56 +347,83 @@ __global__ void __launch_bounds__(GEMV6_THREADS, GEMV6_CTAS_PER_SM)
           S[0][1][h] = __fmul_rn((float)(int8_t)(scw10 >> (bo + 8 * h)), stp1);
           S[1][1][h] = __fmul_rn((float)(int8_t)(scw11 >> (bo + 8 * h)), stp1);
         }
-#pragma unroll
-        for (int set = 0; set < 2; ++set) {
-          // A: groups 8 set + c (slots 4c ..) and 8 set + c + 4 (slots 16 + 4c ..) of rows r0, r1
-          uint32_t A00[4], A01[4], A10[4], A11[4];  // [row][group half]
-          {
-            const uint32_t o = stg + 12 * (8 * set + c);
-            const uint32_t a0 = o + r0 * GEMV6_CODE_ROW, a1 = o + r1 * GEMV6_CODE_ROW;
-            int6_a_words(lds32(a0), lds32(a0 + 4), lds32(a0 + 8), A00);
-            int6_a_words(lds32(a0 + 48), lds32(a0 + 52), lds32(a0 + 56), A01);
-            int6_a_words(lds32(a1), lds32(a1 + 4), lds32(a1 + 8), A10);
-            int6_a_words(lds32(a1 + 48), lds32(a1 + 52), lds32(a1 + 56), A11);
-          }
-          // up to four tokens at a time: eight independent accumulator chains (hi / lo) per k-step
-#pragma unroll
-          for (int m0 = 0; m0 < TM; m0 += MP) {
-            if (m0 < M) {
-              int32_t dh[MP][4], dl[MP][4];
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-#pragma unroll
-                for (int mm = 0; mm < MP; ++mm) {
-                  const int m = m0 + mm;  // a token past M (odd M) reads stale stage words; its sums are never stored
-                  const uint32_t xrow = stg + L::ST_X + ((m * 2 + set) * 4 + j) * 128 + 16 * g;
-                  const uint4 xv = lds128(on ? xrow : zero_a);
-                  if (j == 0) {
-                    QL_IMMA6_0("s8", dh[mm], acc_init, A00[0], A10[0], A01[0], A11[0], xv.x, xv.y);
-                    QL_IMMA6_0("u8", dl[mm], acc_init, A00[0], A10[0], A01[0], A11[0], xv.z, xv.w);
-                  } else {
-                    QL_IMMA6("s8", dh[mm], A00[j], A10[j], A01[j], A11[j], xv.x, xv.y);
-                    QL_IMMA6("u8", dl[mm], A00[j], A10[j], A01[j], A11[j], xv.z, xv.w);
+        const int64_t sbw = (int64_t)(sb0 + i) * M * 64;  // the super-block's lo x words, in uint2
+        auto sets = [&](auto x24c) {  // the stage's two 8-group sets: two bytes of x, or three for 24-bit x
+          constexpr bool X24 = decltype(x24c)::value;
+  #pragma unroll
+          for (int set = 0; set < 2; ++set) {
+            // A: groups 8 set + c (slots 4c ..) and 8 set + c + 4 (slots 16 + 4c ..) of rows r0, r1
+            uint32_t A00[4], A01[4], A10[4], A11[4];  // [row][group half]
+            if constexpr (PLANAR) {  // group gg: low plane bytes 8 gg .., high plane bytes 128 + 4 gg ..
+              const uint32_t gl = 8 * set + c;
+              const uint32_t a0 = stg + r0 * GEMV6_CODE_ROW, a1 = stg + r1 * GEMV6_CODE_ROW;
+              const uint2 l00 = lds64(a0 + 8 * gl), l01 = lds64(a0 + 8 * gl + 32);
+              const uint2 l10 = lds64(a1 + 8 * gl), l11 = lds64(a1 + 8 * gl + 32);
+              int6p_a_words(l00.x, l00.y, lds32(a0 + 128 + 4 * gl), A00);
+              int6p_a_words(l01.x, l01.y, lds32(a0 + 144 + 4 * gl), A01);
+              int6p_a_words(l10.x, l10.y, lds32(a1 + 128 + 4 * gl), A10);
+              int6p_a_words(l11.x, l11.y, lds32(a1 + 144 + 4 * gl), A11);
+            } else {
+              const uint32_t o = stg + 12 * (8 * set + c);
+              const uint32_t a0 = o + r0 * GEMV6_CODE_ROW, a1 = o + r1 * GEMV6_CODE_ROW;
+              int6_a_words(lds32(a0), lds32(a0 + 4), lds32(a0 + 8), A00);
+              int6_a_words(lds32(a0 + 48), lds32(a0 + 52), lds32(a0 + 56), A01);
+              int6_a_words(lds32(a1), lds32(a1 + 4), lds32(a1 + 8), A10);
+              int6_a_words(lds32(a1 + 48), lds32(a1 + 52), lds32(a1 + 56), A11);
+            }
+            // up to four tokens at a time: eight independent accumulator chains (hi / lo) per k-step
+  #pragma unroll
+            for (int m0 = 0; m0 < TM; m0 += MP) {
+              if (m0 < M) {
+                int32_t dh[MP][4], dm[MP][4], dl[MP][4];
+  #pragma unroll
+                for (int mm = 0; mm < MP; ++mm)
+  #pragma unroll
+                  for (int q = 0; q < 4; ++q) dl[mm][q] = GEMV_ACC0;
+  #pragma unroll
+                for (int j = 0; j < 4; ++j) {
+  #pragma unroll
+                  for (int mm = 0; mm < MP; ++mm) {
+                    const int m = m0 + mm;  // a token past M (odd M) reads stale stage words; its sums are never stored
+                    const uint32_t xrow = stg + L::ST_X + ((m * 2 + set) * 4 + j) * 128 + 16 * g;
+                    const uint4 xv = lds128(on ? xrow : zero_a);
+                    if (j == 0) {
+                      QL_IMMA6_0("s8", dh[mm], acc_init, A00[0], A10[0], A01[0], A11[0], xv.x, xv.y);
+                      QL_IMMA6_0("u8", dm[mm], acc_init, A00[0], A10[0], A01[0], A11[0], xv.z, xv.w);
+                    } else {
+                      QL_IMMA6("s8", dh[mm], A00[j], A10[j], A01[j], A11[j], xv.x, xv.y);
+                      QL_IMMA6("u8", dm[mm], A00[j], A10[j], A01[j], A11[j], xv.z, xv.w);
+                    }
+                    if constexpr (X24) {  // the low byte of 24-bit x, from global memory (L2); feeding lanes only
+                      const uint2 xl = (on && m < M) ? __ldg(xlg + sbw + ((m * 2 + set) * 4 + j) * 8 + g)
+                                                     : make_uint2(0u, 0u);
+                      QL_IMMA6("u8", dl[mm], A00[j], A10[j], A01[j], A11[j], xl.x, xl.y);
+                    }
                   }
                 }
-              }
-#pragma unroll
-              for (int mm = 0; mm < MP; ++mm) {
-                const int m = m0 + mm;
-                // D[q]: q = 0 (r0, group 8 set + 2c), 1 (r0, + 1), 2 (r1, 2c), 3 (r1, + 1)
-                const float2 G = lds64f(stg + L::ST_G + (m * 16 + 8 * set + 2 * c) * 4);
-                float t[4];
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-                  t[q] = fmaf(__int_as_float(dh[mm][q]) - GEMV_ACC0_F, 256.f, __int_as_float(dl[mm][q]) - GEMV_ACC0_F);
-                acc[m][0] = fmaf(S[set][0][0] * G.x, t[0], acc[m][0]);
-                acc[m][0] = fmaf(S[set][0][1] * G.y, t[1], acc[m][0]);
-                acc[m][1] = fmaf(S[set][1][0] * G.x, t[2], acc[m][1]);
-                acc[m][1] = fmaf(S[set][1][1] * G.y, t[3], acc[m][1]);
+  #pragma unroll
+                for (int mm = 0; mm < MP; ++mm) {
+                  const int m = m0 + mm;
+                  // D[q]: q = 0 (r0, group 8 set + 2c), 1 (r0, + 1), 2 (r1, 2c), 3 (r1, + 1)
+                  const float2 G = lds64f(stg + L::ST_G + (m * 16 + 8 * set + 2 * c) * 4);
+                  float t[4];  // T = 65536 D_hi + 256 D_mid + D_lo
+  #pragma unroll
+                  for (int q = 0; q < 4; ++q) {
+                    t[q] = fmaf(__int_as_float(dh[mm][q]) - GEMV_ACC0_F, 256.f, __int_as_float(dm[mm][q]) - GEMV_ACC0_F);
+                    if constexpr (X24) t[q] = fmaf(t[q], 256.f, __int_as_float(dl[mm][q]) - GEMV_ACC0_F);
+                    else t[q] *= 256.f;
+                  }
+                  acc[m][0] = fmaf(S[set][0][0] * G.x, t[0], acc[m][0]);
+                  acc[m][0] = fmaf(S[set][0][1] * G.y, t[1], acc[m][0]);
+                  acc[m][1] = fmaf(S[set][1][0] * G.x, t[2], acc[m][1]);
+                  acc[m][1] = fmaf(S[set][1][1] * G.y, t[3], acc[m][1]);
+                }
               }
             }
           }
-        }
+        };
+        if (x24) sets(std::true_type{});
+        else sets(std::false_type{});
         __syncwarp();
         if (lane == 0) mbar_arrive(bar_empty(s));
       }

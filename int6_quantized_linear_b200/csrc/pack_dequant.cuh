@@ -95,6 +95,37 @@ __global__ void __launch_bounds__(256) pack_int6_kernel(PackArgs a) {
   }
 }
 
+// int6 planar: unit = 32 codes -> 16 low-plane bytes (at 192 j + 16 t of the row's super-block j,
+// chunk t) and 8 high-plane bytes (at 192 j + 128 + 8 t); metadata as dense int6.
+__global__ void __launch_bounds__(256) pack_int6p_kernel(PackArgs a) {
+  const int64_t nA = a.N * a.K / 32, nB = a.N * a.K / 256, nC = a.N * a.K / 256;
+  const int64_t total = nA + nB + nC;
+  for (int64_t u = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; u < total; u += (int64_t)gridDim.x * blockDim.x) {
+    if (u < nA) {
+      const uint4 *src = reinterpret_cast<const uint4 *>(a.q + 32 * u);
+      uint4 in[2] = {src[0], src[1]};
+      const uint32_t *iw = reinterpret_cast<const uint32_t *>(in);  // code i in byte i % 4 of word i / 4
+      uint32_t lo[4] = {0u, 0u, 0u, 0u}, hi[2] = {0u, 0u};
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const uint32_t f = (iw[i >> 2] >> (8 * (i & 3))) & 0x3fu;
+        lo[i >> 3] |= (f & 0xfu) << (4 * (i & 7));
+        hi[i >> 4] |= (f >> 4) << (2 * (i & 15));
+      }
+      const int64_t sb = u >> 3, t = u & 7;  // super-block (over all rows: K is a multiple of 256) and chunk
+      uint8_t *blk = a.codes + 192 * sb;
+      *reinterpret_cast<uint4 *>(blk + 16 * t) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      *reinterpret_cast<uint2 *>(blk + 128 + 8 * t) = make_uint2(hi[0], hi[1]);
+    } else if (u < nA + nB) {  // scale codes: 16-byte copy
+      const int64_t v = u - nA;
+      reinterpret_cast<uint4 *>(a.gmeta)[v] = reinterpret_cast<const uint4 *>(a.meta0)[v];
+    } else {
+      const int64_t v = u - nA - nB;
+      reinterpret_cast<uint16_t *>(a.steps)[v] = a.step0[v];
+    }
+  }
+}
+
 template <int BITS>
 __global__ void __launch_bounds__(256) pack_affine_kernel(PackArgs a) {
   constexpr int P = 32 / BITS;
@@ -205,6 +236,41 @@ __global__ void __launch_bounds__(256) unpack_int6_kernel(UnpackArgs a) {
   }
 }
 
+__global__ void __launch_bounds__(256) unpack_int6p_kernel(UnpackArgs a) {
+  const int64_t nA = a.N * a.K / 32, nB = a.N * a.K / 16, nC = a.N * a.K / 256;
+  const int64_t total = nA + nB + nC;
+  for (int64_t u = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; u < total; u += (int64_t)gridDim.x * blockDim.x) {
+    if (u < nA) {
+      const int64_t sb = u >> 3, t = u & 7;
+      const uint8_t *blk = a.codes + 192 * sb;
+      const uint4 l = *reinterpret_cast<const uint4 *>(blk + 16 * t);
+      const uint2 h = *reinterpret_cast<const uint2 *>(blk + 128 + 8 * t);
+      const uint32_t lo[4] = {l.x, l.y, l.z, l.w}, hi[2] = {h.x, h.y};
+      uint32_t o[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        uint32_t r = 0;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          const int i = 4 * j + b;
+          const uint32_t f = ((lo[i >> 3] >> (4 * (i & 7))) & 0xfu) | (((hi[i >> 4] >> (2 * (i & 15))) & 0x3u) << 4);
+          r |= ((f & 0x20u) ? (f | 0xc0u) : f) << (8 * b);  // sign-extend into the byte
+        }
+        o[j] = r;
+      }
+      uint4 *dst = reinterpret_cast<uint4 *>(a.q + 32 * u);
+      dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+      dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+    } else if (u < nA + nB) {
+      const int64_t v = u - nA;
+      if (a.meta0) a.meta0[v] = a.gmeta[v];
+    } else {
+      const int64_t v = u - nA - nB;
+      if (a.step0) a.step0[v] = reinterpret_cast<const uint16_t *>(a.steps)[v];
+    }
+  }
+}
+
 template <int BITS>
 __global__ void __launch_bounds__(256) unpack_affine_kernel(UnpackArgs a) {
   constexpr int P = 32 / BITS;
@@ -256,6 +322,14 @@ QL_DEVI void load_decode32(const WeightPtrs &p, int64_t n, int64_t c, float (&w)
     const uint32_t sc2 = __ldg(reinterpret_cast<const uint16_t *>(p.gmeta + n * (p.K / 16)) + c);
     const uint32_t st = __ldg(reinterpret_cast<const uint16_t *>(p.steps) + n * (p.K / 256) + (c >> 3));
     int6_decode32(cw, sc2, st, w);
+  } else if constexpr (FMT == FMT_INT6P) {
+    const uint8_t *blk = p.codes + n * (3 * p.K / 4) + 192 * (c >> 3);
+    const uint4 l = __ldg(reinterpret_cast<const uint4 *>(blk + 16 * (c & 7)));
+    const uint2 h = __ldg(reinterpret_cast<const uint2 *>(blk + 128 + 8 * (c & 7)));
+    const uint32_t lo[4] = {l.x, l.y, l.z, l.w}, hi[2] = {h.x, h.y};
+    const uint32_t sc2 = __ldg(reinterpret_cast<const uint16_t *>(p.gmeta + n * (p.K / 16)) + c);
+    const uint32_t st = __ldg(reinterpret_cast<const uint16_t *>(p.steps) + n * (p.K / 256) + (c >> 3));
+    int6p_decode32(lo, hi, sc2, st, w);
   } else {
     const uint32_t *src = reinterpret_cast<const uint32_t *>(p.codes + n * (p.K * BITS / 8)) + BITS * c;
     uint32_t cw[BITS];

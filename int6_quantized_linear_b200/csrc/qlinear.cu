@@ -25,23 +25,30 @@ struct DeviceInfo {
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
 
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// A CUDA call on the host failed: clear the runtime's last-error slot (a non-sticky error would
+// otherwise make the next call's launch check report this failure as its own) and say so.
+inline ql_status cuda_failed() {
+  (void)cudaGetLastError();
+  return QL_ERR_CUDA;
+}
+
 ql_status device_info(DeviceInfo **out) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return QL_ERR_CUDA;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return cuda_failed();
   std::lock_guard<std::mutex> lk(g_mu);
   DeviceInfo &d = g_dev[dev];
   if (!d.init) {
     if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&d.minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
-      return QL_ERR_CUDA;
+      return cuda_failed();
     d.init = true;
   }
   *out = &d;
   return QL_OK;
 }
-
-inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 ql_status check_desc(const ql_desc *d) {
   if (!d) return QL_ERR_NULL;
@@ -49,6 +56,7 @@ ql_status check_desc(const ql_desc *d) {
   switch (d->fmt) {
     case QL_INT4_NSS:
     case QL_INT6_SYM:
+    case QL_INT6_PLANAR:
       if (d->K % 256 != 0) return QL_ERR_SHAPE;
       return QL_OK;
     case QL_AFFINE_U32:
@@ -65,7 +73,8 @@ void sizes(const ql_desc *d, size_t *c, size_t *g, size_t *s) {
   const size_t N = (size_t)d->N, K = (size_t)d->K;
   switch (d->fmt) {
     case QL_INT4_NSS: *c = N * K / 2; *g = N * (K / 32) * 2; *s = N * (K / 256) * 4; break;
-    case QL_INT6_SYM: *c = N * 3 * K / 4; *g = N * (K / 16); *s = N * (K / 256) * 2; break;
+    case QL_INT6_SYM:
+    case QL_INT6_PLANAR: *c = N * 3 * K / 4; *g = N * (K / 16); *s = N * (K / 256) * 2; break;
     default: *c = N * K * d->bits / 8; *g = N * (K / d->group) * 4; *s = 0; break;
   }
 }
@@ -125,24 +134,26 @@ bool encode_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint6
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int FMT, int BITS>
-ql_status launch_gemm(const ql_desc *d, const ql_packed_const *w, const void *x, int64_t M, const void *bias,
-                      void *y, void *workspace, cudaStream_t st, int sms) {
+template <int FMT, int BITS, int TT>
+ql_status launch_gemm_tt(const ql_desc *d, const ql_packed_const *w, const void *x, int64_t M, const void *bias,
+                         void *y, void *workspace, cudaStream_t st, int sms) {
   using namespace ql::gemm;
   const int64_t N = d->N, K = d->K;
   const uint64_t row_bytes = (uint64_t)K * code_bits(FMT, BITS) / 8;
   const GemmWorkspace ws = gemm_workspace_carve(workspace, M, N, K);
   // pass 1: scaled fp16 activations; pass 2: per-row weight scales
   x_to_f16_kernel<<<(int)((M * 32 + 255) / 256), 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(x), M, K, ws);
-  w_scale_kernel<FMT, BITS><<<(int)((N * 32 + 255) / 256), 256, 0, st>>>(
+  w_scale_kernel<FMT, BITS><<<(int)(((int64_t)padded_rows(N) * 32 + 255) / 256), 256, 0, st>>>(
       static_cast<const uint8_t *>(w->gmeta), static_cast<const uint8_t *>(w->steps), N, K, d->group, ws);
   CUtensorMap mx, mc;
-  if (!encode_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws.x16, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, BK, BM,
+  if (!encode_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws.x16, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, BK, TT,
                  CU_TENSOR_MAP_SWIZZLE_128B))
-    return QL_ERR_CUDA;
+    return cuda_failed();
+  // int6 planar: a k-step's codes are three 16-byte pieces of its super-block (two of the low plane,
+  // one of the high plane), loaded as three boxes of 16 bytes x BN rows
   if (!encode_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->codes, row_bytes, (uint64_t)N, row_bytes,
-                 (uint32_t)p_row_bytes(FMT, BITS), BN, CU_TENSOR_MAP_SWIZZLE_NONE))
-    return QL_ERR_CUDA;
+                 FMT == FMT_INT6P ? 16u : (uint32_t)p_row_bytes(FMT, BITS), BN, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cuda_failed();
   Params p;
   p.M = M; p.N = N; p.K = K; p.G = d->group;
   p.bias = static_cast<const __nv_bfloat16 *>(bias);
@@ -150,20 +161,29 @@ ql_status launch_gemm(const ql_desc *d, const ql_packed_const *w, const void *x,
   p.steps = static_cast<const uint8_t *>(w->steps);
   p.y = static_cast<__nv_bfloat16 *>(y);
   p.ws = ws;
-  const int smem = smem_bytes(FMT, BITS);
-  auto kern = gemm_kernel<FMT, BITS>;
+  const int smem = smem_bytes(FMT, BITS, TT);
+  auto kern = gemm_kernel<FMT, BITS, TT>;
   static thread_local int configured_dev = -1;  // per (kernel instantiation, thread)
   int dev = 0;
   cudaGetDevice(&dev);
   if (configured_dev != dev) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-      return QL_ERR_CUDA;
+      return cuda_failed();
     configured_dev = dev;
   }
-  const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+  const int64_t tiles = ((M + TT - 1) / TT) * ((N + BN - 1) / BN);
   const int grid = (int)(tiles < sms ? tiles : sms);
   kern<<<grid, NUM_THREADS, smem, st>>>(mx, mc, p);
   return launched();
+}
+
+// Up to 32 tokens: the swapped form (weights as the M = 128 operand, the tokens as N = 32), so no MMA
+// runs on padding rows; from 33 tokens: tiles of 256 tokens x 128 weight rows.
+template <int FMT, int BITS>
+ql_status launch_gemm(const ql_desc *d, const ql_packed_const *w, const void *x, int64_t M, const void *bias,
+                      void *y, void *workspace, cudaStream_t st, int sms) {
+  if (M <= gemm::TT_SWAP) return launch_gemm_tt<FMT, BITS, gemm::TT_SWAP>(d, w, x, M, bias, y, workspace, st, sms);
+  return launch_gemm_tt<FMT, BITS, gemm::BM>(d, w, x, M, bias, y, workspace, st, sms);
 }
 
 // Which GEMV calls run on the tensor-core GEMM (measured faster there on the benchmark layers:
@@ -196,7 +216,7 @@ ql_status launch_gemv_mt(const ql_desc *d, const ql_packed_const *w, const __nv_
                          const __nv_bfloat16 *bb, __nv_bfloat16 *yb, void *workspace, cudaStream_t st, int sms) {
   using L = MtLayout<FMT, BITS, G>;
   const int64_t N = d->N, K = d->K, NS = K / 256, TG = (N + 63) / 64;
-  const GemvWorkspace ws = gemv_workspace_carve(workspace, M, K);
+  const GemvWorkspace ws = gemv_workspace_carve(workspace, M, N, K);
   cudaLaunchAttribute pa[1];
   pa[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   pa[0].val.programmaticStreamSerializationAllowed = 1;
@@ -208,7 +228,7 @@ ql_status launch_gemv_mt(const ql_desc *d, const ql_packed_const *w, const __nv_
     pc.stream = st;
     pc.attrs = pa;
     pc.numAttrs = 1;
-    if (cudaLaunchKernelEx(&pc, gemv_xprep_mt_kernel, xb, M, K, TG, ws) != cudaSuccess) return QL_ERR_CUDA;
+    if (cudaLaunchKernelEx(&pc, gemv_xprep_mt_kernel, xb, M, K, TG, ws) != cudaSuccess) return cuda_failed();
   }
   GemvMtParams p;
   p.steps = static_cast<const uint8_t *>(w->steps);
@@ -230,14 +250,14 @@ ql_status launch_gemv_mt(const ql_desc *d, const ql_packed_const *w, const __nv_
                  L::CODE_BOX == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B) ||
       !encode_2d(&mg, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->gmeta, meta_row, (uint64_t)N, meta_row, L::META_ROW, 64,
                  CU_TENSOR_MAP_SWIZZLE_NONE))
-    return QL_ERR_CUDA;
+    return cuda_failed();
   auto kern = gemv_mt_kernel<FMT, BITS, G>;
   static thread_local int configured_dev = -1;  // per instantiation and thread
   int dev = 0;
   cudaGetDevice(&dev);
   if (configured_dev != dev) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM) != cudaSuccess)
-      return QL_ERR_CUDA;
+      return cuda_failed();
     configured_dev = dev;
   }
   cudaLaunchConfig_t cfg = {};
@@ -247,17 +267,17 @@ ql_status launch_gemv_mt(const ql_desc *d, const ql_packed_const *w, const __nv_
   cfg.stream = st;
   cfg.attrs = pa;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kern, mc, mg, p) != cudaSuccess) return QL_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, kern, mc, mg, p) != cudaSuccess) return cuda_failed();
   return launched();
 }
 
 // Tensor-core int6 GEMV at 1..TM tokens: x preparation, then the streaming kernel as its dependent.
-template <int TM>
+template <int TM, bool PLANAR>
 ql_status launch_gemv_int6(const ql_desc *d, const ql_packed_const *w, const __nv_bfloat16 *xb, int64_t M,
                            const __nv_bfloat16 *bb, __nv_bfloat16 *yb, void *workspace, cudaStream_t st, int sms) {
   using L = Int6Layout<TM>;
   const int64_t N = d->N, K = d->K, NS = K / 256, TG = (N + 63) / 64;
-  const GemvWorkspace ws = gemv_workspace_carve(workspace, M, K);
+  const GemvWorkspace ws = gemv_workspace_carve(workspace, M, N, K);
   // split K over P CTAs per 64-row group while the row groups alone leave a wave unfilled
   int64_t P = std::max<int64_t>(1, std::min<int64_t>(NS, (int64_t)sms * GEMV6_CTAS_PER_SM / TG));
   P = std::min<int64_t>(P, std::max<int64_t>(1, GEMV_MT_MAX_CTAS / TG));
@@ -273,8 +293,9 @@ ql_status launch_gemv_int6(const ql_desc *d, const ql_packed_const *w, const __n
     pc.stream = st;
     pc.attrs = pa;
     pc.numAttrs = 1;
-    if (cudaLaunchKernelEx(&pc, gemv_xprep_int6_kernel, xb, M, K, P > 1 ? TG : (int64_t)0, ws) != cudaSuccess)
-      return QL_ERR_CUDA;
+    if (cudaLaunchKernelEx(&pc, gemv_xprep_int6_kernel<PLANAR>, xb, M, K, P > 1 ? TG : (int64_t)0, ws) !=
+        cudaSuccess)
+      return cuda_failed();
   }
   Gemv6Params p;
   p.steps = static_cast<const uint16_t *>(w->steps);
@@ -291,14 +312,14 @@ ql_status launch_gemv_int6(const ql_desc *d, const ql_packed_const *w, const __n
                  CU_TENSOR_MAP_SWIZZLE_NONE) ||
       !encode_2d(&ms, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->gmeta, sc_row, (uint64_t)N, sc_row, 16, 64,
                  CU_TENSOR_MAP_SWIZZLE_NONE))
-    return QL_ERR_CUDA;
-  auto kern = gemv_int6_kernel<TM>;
+    return cuda_failed();
+  auto kern = gemv_int6_kernel<TM, PLANAR>;
   static thread_local int configured_dev = -1;  // per instantiation and thread
   int dev = 0;
   cudaGetDevice(&dev);
   if (configured_dev != dev) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM) != cudaSuccess)
-      return QL_ERR_CUDA;
+      return cuda_failed();
     configured_dev = dev;
   }
   cudaLaunchConfig_t cfg = {};
@@ -308,7 +329,7 @@ ql_status launch_gemv_int6(const ql_desc *d, const ql_packed_const *w, const __n
   cfg.stream = st;
   cfg.attrs = pa;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kern, mc, ms, p) != cudaSuccess) return QL_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, kern, mc, ms, p) != cudaSuccess) return cuda_failed();
   return launched();
 }
 
@@ -322,11 +343,12 @@ ql_status launch_gemv(const ql_desc *d, const ql_packed_const *w, const void *x,
   if constexpr (FMT == FMT_INT4) {
     if (M >= 2) return launch_gemv_mt<FMT_INT4, 4, 32>(d, w, xb, M, bb, yb, workspace, st, sms);
   }
-  if constexpr (FMT == FMT_INT6) {  // M <= 8
-    if (M == 1) return launch_gemv_int6<1>(d, w, xb, M, bb, yb, workspace, st, sms);
-    if (M == 2) return launch_gemv_int6<2>(d, w, xb, M, bb, yb, workspace, st, sms);
-    if (M <= 4) return launch_gemv_int6<4>(d, w, xb, M, bb, yb, workspace, st, sms);
-    return launch_gemv_int6<8>(d, w, xb, M, bb, yb, workspace, st, sms);
+  if constexpr (FMT == FMT_INT6 || FMT == FMT_INT6P) {  // M <= 8; dense or planar code storage
+    constexpr bool PL = FMT == FMT_INT6P;
+    if (M == 1) return launch_gemv_int6<1, PL>(d, w, xb, M, bb, yb, workspace, st, sms);
+    if (M == 2) return launch_gemv_int6<2, PL>(d, w, xb, M, bb, yb, workspace, st, sms);
+    if (M <= 4) return launch_gemv_int6<4, PL>(d, w, xb, M, bb, yb, workspace, st, sms);
+    return launch_gemv_int6<8, PL>(d, w, xb, M, bb, yb, workspace, st, sms);
   }
   if constexpr (FMT == FMT_AFFINE) {  // bits 2, 4, 8
     if (d->K % 256 == 0 && d->group == 64) return launch_gemv_mt<FMT_AFFINE, BITS, 64>(d, w, xb, M, bb, yb, workspace, st, sms);
@@ -334,7 +356,7 @@ ql_status launch_gemv(const ql_desc *d, const ql_packed_const *w, const void *x,
   }
   if constexpr (FMT == FMT_INT4) {
     if (M == 1) {  // tensor-core path: preparation pass, then the streaming kernel as its dependent
-      const GemvWorkspace ws = gemv_workspace_carve(workspace, M, d->K);
+      const GemvWorkspace ws = gemv_workspace_carve(workspace, M, d->N, d->K);
       const int64_t ng = M * (d->K / 32);
       const int64_t NS = d->K / 256, n_tiles = (d->N + 15) / 16;
       // split K over P warps per 16-row tile while the tiles alone leave the resident warp slots
@@ -355,7 +377,7 @@ ql_status launch_gemv(const ql_desc *d, const ql_packed_const *w, const void *x,
         pc.attrs = pa;
         pc.numAttrs = 1;
         if (cudaLaunchKernelEx(&pc, gemv_xprep_kernel, xb, M, (int64_t)d->K, n_counters, ws) != cudaSuccess)
-          return QL_ERR_CUDA;
+          return cuda_failed();
       }
       GemvTcParams p;
       p.steps = static_cast<const uint8_t *>(w->steps);
@@ -370,7 +392,7 @@ ql_status launch_gemv(const ql_desc *d, const ql_packed_const *w, const void *x,
                      (uint64_t)d->K / 2, 128, 16, CU_TENSOR_MAP_SWIZZLE_128B) ||
           !encode_2d(&mg, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->gmeta, (uint64_t)d->K / 16, (uint64_t)d->N,
                      (uint64_t)d->K / 16, 16, 16, CU_TENSOR_MAP_SWIZZLE_NONE))
-        return QL_ERR_CUDA;
+        return cuda_failed();
       p.parts = (int)P;
       static thread_local int configured_dev = -1;
       int dev = 0;
@@ -378,7 +400,7 @@ ql_status launch_gemv(const ql_desc *d, const ql_packed_const *w, const void *x,
       if (configured_dev != dev) {
         if (cudaFuncSetAttribute(gemv_int4_m1_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  gemv_smem_bytes()) != cudaSuccess)
-          return QL_ERR_CUDA;
+          return cuda_failed();
         configured_dev = dev;
       }
       cudaLaunchConfig_t cfg = {};
@@ -391,7 +413,7 @@ ql_status launch_gemv(const ql_desc *d, const ql_packed_const *w, const void *x,
       attr[0].val.programmaticStreamSerializationAllowed = 1;
       cfg.attrs = attr;
       cfg.numAttrs = 1;
-      if (cudaLaunchKernelEx(&cfg, gemv_int4_m1_tc_kernel, mc, mg, p) != cudaSuccess) return QL_ERR_CUDA;
+      if (cudaLaunchKernelEx(&cfg, gemv_int4_m1_tc_kernel, mc, mg, p) != cudaSuccess) return cuda_failed();
       return launched();
     }
   }
@@ -435,11 +457,11 @@ void *g_noalloc_addr[kMaxDevices] = {};
 
 ql_status noalloc_scratch(void **out) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return QL_ERR_CUDA;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return cuda_failed();
   std::lock_guard<std::mutex> lk(g_mu);
   if (g_noalloc_addr[dev] == nullptr) {
     void *p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_gemm_noalloc_scratch) != cudaSuccess || p == nullptr) return QL_ERR_CUDA;
+    if (cudaGetSymbolAddress(&p, g_gemm_noalloc_scratch) != cudaSuccess || p == nullptr) return cuda_failed();
     g_noalloc_addr[dev] = p;
   }
   *out = g_noalloc_addr[dev];
@@ -457,7 +479,9 @@ const char *qlinear_status_string(ql_status s) {
     case QL_ERR_NULL: return "a required pointer is NULL";
     case QL_ERR_SHAPE: return "shape, bit width or group size not allowed for this format";
     case QL_ERR_ALIGN: return "a device pointer is not 16-byte aligned";
-    case QL_ERR_RANGE: return "M outside the range of this entry point";
+    case QL_ERR_RANGE:
+      return "value out of range: M for this entry point, a problem larger than the fixed scratch array, "
+             "or (from qlinear_sync_status) an encoder input outside its domain";
     case QL_ERR_UNSUPPORTED: return "unknown format or unsupported device";
     case QL_ERR_CUDA: return "a CUDA call or kernel launch failed";
     case QL_ERR_TIMEOUT: return "a device-side bounded wait gave up";
@@ -478,7 +502,8 @@ ql_status qlinear_pack(const ql_desc *d, const ql_unpacked *in, const ql_packed 
   if (st != QL_OK) return st;
   if (!in || !out || !in->q || !in->meta0) return QL_ERR_NULL;
   if ((d->fmt == QL_INT4_NSS && (!in->meta1 || !in->step0 || !in->step1)) ||
-      (d->fmt == QL_INT6_SYM && !in->step0) || (d->fmt == QL_AFFINE_U32 && !in->meta1))
+      ((d->fmt == QL_INT6_SYM || d->fmt == QL_INT6_PLANAR) && !in->step0) ||
+      (d->fmt == QL_AFFINE_U32 && !in->meta1))
     return QL_ERR_NULL;
   if ((st = check_packed(d, out->codes, out->gmeta, out->steps)) != QL_OK) return st;
   const void *ins[5] = {in->q, in->meta0, in->meta1, in->step0, in->step1};
@@ -501,6 +526,7 @@ ql_status qlinear_pack(const ql_desc *d, const ql_unpacked *in, const ql_packed 
   switch (d->fmt) {
     case QL_INT4_NSS: pack_int4_kernel<<<grid_for(NK / 32 + NK / 128, di->sms), 256, 0, s>>>(a); break;
     case QL_INT6_SYM: pack_int6_kernel<<<grid_for(NK / 64 + NK / 128, di->sms), 256, 0, s>>>(a); break;
+    case QL_INT6_PLANAR: pack_int6p_kernel<<<grid_for(NK / 32 + NK / 128, di->sms), 256, 0, s>>>(a); break;
     default: {
       const int g = grid_for(NK * d->bits / 128 + NK / d->group, di->sms);
       if (d->bits == 2) pack_affine_kernel<2><<<g, 256, 0, s>>>(a);
@@ -537,6 +563,7 @@ ql_status qlinear_unpack(const ql_desc *d, const ql_packed_const *in, const ql_u
   switch (d->fmt) {
     case QL_INT4_NSS: unpack_int4_kernel<<<grid_for(NK / 32 * 2 + NK / 256, di->sms), 256, 0, s>>>(a); break;
     case QL_INT6_SYM: unpack_int6_kernel<<<grid_for(NK / 64 + NK / 16, di->sms), 256, 0, s>>>(a); break;
+    case QL_INT6_PLANAR: unpack_int6p_kernel<<<grid_for(NK / 32 + NK / 16, di->sms), 256, 0, s>>>(a); break;
     default: {
       const int g = grid_for(NK * d->bits / 32 + NK / d->group, di->sms);
       if (d->bits == 2) unpack_affine_kernel<2><<<g, 256, 0, s>>>(a);
@@ -569,6 +596,7 @@ ql_status qlinear_dequant(const ql_desc *d, const ql_packed_const *w, void *out,
   switch (d->fmt) {
     case QL_INT4_NSS: QL_DQ(FMT_INT4, 4); break;
     case QL_INT6_SYM: QL_DQ(FMT_INT6, 6); break;
+    case QL_INT6_PLANAR: QL_DQ(FMT_INT6P, 6); break;
     default:
       if (d->bits == 2) QL_DQ(FMT_AFFINE, 2);
       else if (d->bits == 4) QL_DQ(FMT_AFFINE, 4);
@@ -605,6 +633,7 @@ static ql_status gemv_call(const ql_desc *d, const ql_packed_const *w, const voi
   switch (d->fmt) {
     case QL_INT4_NSS: return launch_gemv<FMT_INT4, 4>(d, w, x, M, bias, y, workspace, s, di->sms);
     case QL_INT6_SYM: return launch_gemv<FMT_INT6, 6>(d, w, x, M, bias, y, workspace, s, di->sms);
+    case QL_INT6_PLANAR: return launch_gemv<FMT_INT6P, 6>(d, w, x, M, bias, y, workspace, s, di->sms);
     default:
       if (d->bits == 2) return launch_gemv<FMT_AFFINE, 2>(d, w, x, M, bias, y, workspace, s, di->sms);
       if (d->bits == 4) return launch_gemv<FMT_AFFINE, 4>(d, w, x, M, bias, y, workspace, s, di->sms);
@@ -651,6 +680,7 @@ static ql_status gemm_call(const ql_desc *d, const ql_packed_const *w, const voi
   switch (d->fmt) {
     case QL_INT4_NSS: return launch_gemm<FMT_INT4, 4>(d, w, x, M, bias, y, workspace, s, di->sms);
     case QL_INT6_SYM: return launch_gemm<FMT_INT6, 6>(d, w, x, M, bias, y, workspace, s, di->sms);
+    case QL_INT6_PLANAR: return launch_gemm<FMT_INT6P, 6>(d, w, x, M, bias, y, workspace, s, di->sms);
     default:
       if (d->bits == 2) return launch_gemm<FMT_AFFINE, 2>(d, w, x, M, bias, y, workspace, s, di->sms);
       if (d->bits == 4) return launch_gemm<FMT_AFFINE, 4>(d, w, x, M, bias, y, workspace, s, di->sms);
@@ -696,7 +726,7 @@ ql_status qlinear_concat_n(const ql_desc *da, const ql_packed_const *wa, const q
     uint8_t *dst = static_cast<uint8_t *>(dsts[i]);
     if (cudaMemcpyAsync(dst, srcs[i][0], na[i], cudaMemcpyDeviceToDevice, s) != cudaSuccess ||
         cudaMemcpyAsync(dst + na[i], srcs[i][1], nb[i], cudaMemcpyDeviceToDevice, s) != cudaSuccess)
-      return QL_ERR_CUDA;
+      return cuda_failed();
   }
   return QL_OK;
 }
@@ -720,6 +750,7 @@ ql_status qlinear_gemm_noalloc(const ql_desc *d, const ql_packed_const *w, const
   switch (d->fmt) {
     case QL_INT4_NSS: return launch_gemm<FMT_INT4, 4>(d, w, x, M, nullptr, y, scratch, s, di->sms);
     case QL_INT6_SYM: return launch_gemm<FMT_INT6, 6>(d, w, x, M, nullptr, y, scratch, s, di->sms);
+    case QL_INT6_PLANAR: return launch_gemm<FMT_INT6P, 6>(d, w, x, M, nullptr, y, scratch, s, di->sms);
     default:
       if (d->bits == 2) return launch_gemm<FMT_AFFINE, 2>(d, w, x, M, nullptr, y, scratch, s, di->sms);
       if (d->bits == 4) return launch_gemm<FMT_AFFINE, 4>(d, w, x, M, nullptr, y, scratch, s, di->sms);
@@ -756,11 +787,20 @@ ql_status qlinear_quantize_meta(const ql_desc *d, const float *scale, const floa
   return launched();
 }
 
+ql_status qlinear_set_wait_limit(int64_t cycles, int32_t withhold_copies) {
+  const long long v = cycles > 0 ? (long long)cycles : QL_WAIT_LIMIT_CYCLES;
+  const int h = withhold_copies ? 1 : 0;
+  if (cudaMemcpyToSymbol(g_ql_wait_limit, &v, sizeof v) != cudaSuccess ||
+      cudaMemcpyToSymbol(g_ql_withhold, &h, sizeof h) != cudaSuccess)
+    return cuda_failed();
+  return QL_OK;
+}
+
 ql_status qlinear_sync_status(ql_stream_t stream) {
-  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return QL_ERR_CUDA;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return cuda_failed();
   unsigned int v = 0, zero = 0;
-  if (cudaMemcpyFromSymbol(&v, g_ql_status, sizeof v) != cudaSuccess) return QL_ERR_CUDA;
-  if (v != 0 && cudaMemcpyToSymbol(g_ql_status, &zero, sizeof zero) != cudaSuccess) return QL_ERR_CUDA;
+  if (cudaMemcpyFromSymbol(&v, g_ql_status, sizeof v) != cudaSuccess) return cuda_failed();
+  if (v != 0 && cudaMemcpyToSymbol(g_ql_status, &zero, sizeof zero) != cudaSuccess) return cuda_failed();
   return (v & QL_DEV_TIMEOUT) ? QL_ERR_TIMEOUT : (v & QL_DEV_RANGE) ? QL_ERR_RANGE : QL_OK;
 }
 

@@ -80,7 +80,7 @@ def activations(seed: int, M: int, K: int) -> np.ndarray:
 class Workload:
     """One synthetic layer: format, shape, batch sizes and seed."""
     name: str
-    fmt: str            # "int4" | "int6" | "affine"
+    fmt: str            # "int4" | "int6" | "int6p" (int6 codes, planar storage) | "affine"
     N: int
     K: int
     Ms: tuple
@@ -92,7 +92,7 @@ class Workload:
         n = self.N if N is None else N
         if self.fmt == "int4":
             return int4_weights(self.seed, n, self.K)
-        if self.fmt == "int6":
+        if self.fmt in ("int6", "int6p"):
             return int6_weights(self.seed, n, self.K)
         return affine_weights(self.seed, n, self.K, self.bits, self.group)
 
@@ -110,6 +110,9 @@ WORKLOADS = {
     "int4_gemv_k27648_n5120": Workload("int4_gemv_k27648_n5120", "int4", 5120, 27648, (1, 4, 8), 1),
     "int6_gemv_k5120_n5120": Workload("int6_gemv_k5120_n5120", "int6", 5120, 5120, (1, 4), 2),
     "int6_gemv_k5120_n27648": Workload("int6_gemv_k5120_n27648", "int6", 27648, 5120, (1, 4), 2),
+    # the same int6 layers with their codes in planar storage (a 4-bit and a 2-bit plane)
+    "int6p_gemv_k5120_n5120": Workload("int6p_gemv_k5120_n5120", "int6p", 5120, 5120, (1, 4), 2),
+    "int6p_gemv_k5120_n27648": Workload("int6p_gemv_k5120_n27648", "int6p", 27648, 5120, (1, 4), 2),
     "int4_gemm_k5120_n27648": Workload("int4_gemm_k5120_n27648", "int4", 27648, 5120,
                                        (512, 2048, 8192), 3),
     "affine2_k4096_n14336": Workload("affine2_k4096_n14336", "affine", 14336, 4096, (1, 32), 4, 2, 64),
