@@ -36,7 +36,7 @@ class Layer:
         if weights is None:
             if fmt == "int4":
                 weights = synth.int4_weights(seed, N, K)
-            elif fmt == "int6":
+            elif fmt in ("int6", "int6p"):
                 weights = synth.int6_weights(seed, N, K)
             else:
                 weights = synth.affine_weights(seed, N, K, bits, group)
@@ -51,7 +51,7 @@ class Layer:
         w = self.w
         if self.fmt == "int4":
             return w["q"], w["sc"], w["zc"], w["ss"], w["zs"]
-        if self.fmt == "int6":
+        if self.fmt in ("int6", "int6p"):
             return w["q"], w["sc"], None, w["st"], None
         return w["q"], w["s"], w["b"], None, None
 
@@ -66,6 +66,8 @@ class Layer:
             return OC.int4_pack(sel(w["q"]), sel(w["sc"]), sel(w["zc"]), sel(w["ss"]), sel(w["zs"]))
         if self.fmt == "int6":
             return OC.int6_pack(sel(w["q"]), sel(w["sc"]), sel(w["st"]))
+        if self.fmt == "int6p":
+            return OC.int6p_pack(sel(w["q"]), sel(w["sc"]), sel(w["st"]))
         return OC.affine_pack(sel(w["q"]), sel(w["s"]), sel(w["b"]), self.bits, self.group)
 
     def oracle_w(self, rows=None) -> np.ndarray:
@@ -74,12 +76,14 @@ class Layer:
             return OC.int4_dequant(*p)
         if self.fmt == "int6":
             return OC.int6_dequant(*p)
+        if self.fmt == "int6p":
+            return OC.int6p_dequant(*p)
         return OC.affine_dequant(*p, self.bits, self.group)
 
     def packed_host(self):
         c, g, s = self.packed()
-        gt = {"int4": np.uint16, "int6": np.int8, "affine": np.uint32}[self.fmt]
-        st = {"int4": np.uint32, "int6": np.uint16, "affine": np.uint8}[self.fmt]
+        gt = {"int4": np.uint16, "int6": np.int8, "int6p": np.int8, "affine": np.uint32}[self.fmt]
+        st = {"int4": np.uint32, "int6": np.uint16, "int6p": np.uint16, "affine": np.uint8}[self.fmt]
         ct = np.uint32 if self.fmt == "affine" else np.uint8
         nc, ng, ns = ql.qlinear_packed_bytes(self.desc)
         return (host(c, np.uint8)[:nc].view(ct).reshape(self.N, -1),

@@ -61,7 +61,7 @@ def test_no_oracle_in_the_product():
 
 
 @pytest.mark.parametrize("fmt,N,K,bits,group,bpw", [
-    ("int4", 3, 512, 0, 0, 4.625), ("int6", 3, 512, 0, 0, 6.5625),
+    ("int4", 3, 512, 0, 0, 4.625), ("int6", 3, 512, 0, 0, 6.5625), ("int6p", 3, 512, 0, 0, 6.5625),
     ("affine", 3, 512, 2, 64, 2.5), ("affine", 3, 512, 4, 64, 4.5), ("affine", 3, 512, 8, 64, 8.5),
     ("affine", 3, 512, 4, 32, 5.0), ("affine", 3, 512, 4, 128, 4.25)])
 def test_packed_bytes_closed_forms(lib, fmt, N, K, bits, group, bpw):
@@ -70,7 +70,7 @@ def test_packed_bytes_closed_forms(lib, fmt, N, K, bits, group, bpw):
 
 
 @pytest.mark.parametrize("desc", [
-    ql.Desc("int4", 4, 255), ql.Desc("int4", 0, 256), ql.Desc("int6", 4, 384),
+    ql.Desc("int4", 4, 255), ql.Desc("int4", 0, 256), ql.Desc("int6", 4, 384), ql.Desc("int6p", 4, 384),
     ql.Desc("affine", 4, 512, 3, 64), ql.Desc("affine", 4, 512, 4, 48), ql.Desc("affine", 4, 96, 2, 32)])
 def test_bad_shapes_rejected(lib, desc):
     with pytest.raises(ql.QLinearError) as e:
@@ -123,9 +123,12 @@ def _a256(n):
                                                   ("int6", 0, 0, 5120, 5120, 1), ("int6", 0, 0, 1000, 768, 8),
                                                   ("affine", 2, 64, 14336, 4096, 8), ("affine", 4, 128, 64, 256, 3)])
 def test_gemv_workspace_formula(lib, fmt, bits, group, N, K, M):
-    """The GEMV workspace size is the documented sum: x words, per-group scales and sums, the partial
-    sums of a K split, one counter per 16 rows, each part rounded up to 256 bytes."""
-    want = _a256(4 * M * K) + _a256(8 * M * (K // 32)) + _a256(4 * 4096 * 64 * M) + _a256(4 * ((N + 15) // 16))
+    """The GEMV workspace size is the documented sum: x words (three bytes of 24-bit fixed point per
+    element, laid out for the tensor-core fragments), per-group scales and sums, the partial sums of a K
+    split, one counter per 16 rows, a 16-byte flag record per super-block, each part rounded up to 256
+    bytes."""
+    want = (_a256(7 * M * K) + _a256(8 * M * (K // 32)) + _a256(4 * 4096 * 64 * M) + _a256(4 * ((N + 15) // 16))
+            + _a256(16 * (K // 256)))
     assert ql.qlinear_gemv_workspace_bytes(ql.Desc(fmt, N, K, bits, group), M) == want
 
 

@@ -12,12 +12,13 @@ import torch
 import int6_quantized_linear_b200 as ql
 from int6_quantized_linear_b200 import synth
 from oracle import oracle_c as OC
+from oracle import oracle_np as ON
 from tests.gpu_helpers import Layer, assert_close, bf16_to_f64, dev, host, run_gemm, run_gemv, x_dev
 
 pytestmark = pytest.mark.gpu
 
-FORMATS = [("int4", 0, 0), ("int6", 0, 0), ("affine", 2, 64), ("affine", 4, 64), ("affine", 8, 64),
-           ("affine", 4, 32), ("affine", 8, 128)]
+FORMATS = [("int4", 0, 0), ("int6", 0, 0), ("int6p", 0, 0), ("affine", 2, 64), ("affine", 4, 64),
+           ("affine", 8, 64), ("affine", 4, 32), ("affine", 8, 128)]
 FMT_IDS = [f"{f}{b or ''}g{g or ''}" for f, b, g in FORMATS]
 # several tiles plus a ragged tail in N; K of one super-block and several
 SMALL_SHAPES = [(1, 256), (7, 512), (33, 1024), (300, 2048), (513, 768)]
@@ -46,8 +47,10 @@ def test_pack_unpack_dequant_bitexact(cuda, fmt, bits, group, N, K):
     assert np.array_equal(host(w32, np.uint32), w_ref.view(np.uint32))
     w16 = torch.empty((N, K), dtype=torch.bfloat16, device="cuda")
     ql.qlinear_dequant(L.desc, *L.packed(), w16, ql.QL_OUT_BF16)
-    want16 = np.array([OC.bf16_from_f32(v) for v in w_ref.ravel()[:4096]], np.uint16)
-    assert np.array_equal(host(w16.view(torch.int16), np.uint16).ravel()[:4096], want16)
+    got16 = host(w16.view(torch.int16), np.uint16).reshape(N, K)
+    assert np.array_equal(got16, ON.bf16_bits_from_f32(w_ref))  # every element
+    want16 = np.array([OC.bf16_from_f32(v) for v in w_ref.ravel()[:4096]], np.uint16)  # C oracle's rounding
+    assert np.array_equal(got16.ravel()[:4096], want16)
     assert ql.qlinear_sync_status() == ql.QL_OK
 
 
@@ -62,7 +65,7 @@ def test_gemv_small(cuda, fmt, bits, group, N, K):
         assert_close(y, OC.matmul_f64(xb, w_ref), f"gemv {fmt} N={N} K={K} M={M}")
 
 
-@pytest.mark.parametrize("fmt,bits,group", [("int4", 0, 0), ("int6", 0, 0), ("affine", 4, 64),
+@pytest.mark.parametrize("fmt,bits,group", [("int4", 0, 0), ("int6", 0, 0), ("int6p", 0, 0), ("affine", 4, 64),
                                             ("affine", 2, 32), ("affine", 8, 128)])
 @pytest.mark.parametrize("N,K,Ms", [(256, 256, (1, 127, 128)), (300, 512, (129, 200)),
                                     (1000, 1024, (64, 256)), (40, 768, (300,))])
@@ -83,6 +86,7 @@ def _sampled_rows(N, count, seed):
 
 @pytest.mark.parametrize("name", ["int4_gemv_2048x2048", "int4_gemv_k5120_n27648", "int4_gemv_k27648_n5120",
                                   "int6_gemv_k5120_n5120", "int6_gemv_k5120_n27648",
+                                  "int6p_gemv_k5120_n5120", "int6p_gemv_k5120_n27648",
                                   "affine2_k4096_n14336", "affine4_k4096_n14336", "affine8_k4096_n14336"])
 def test_gemv_full_size_sampled(cuda, name):
     wl = synth.WORKLOADS[name]
@@ -160,18 +164,20 @@ def test_gemv_affine2_multi_token(cuda, bits, group, N, K):
         assert np.array_equal(y, run_gemv(L, xd, M))
 
 
+@pytest.mark.parametrize("fmt", ["int6", "int6p"])
 @pytest.mark.parametrize("N,K", [(200, 1536), (64, 256), (1000, 5120)])
-def test_gemv_int6_every_token_count(cuda, N, K):
-    """int6 tensor-core GEMV at each M it serves (1..8: four token buckets), with and without the
-    split of K over CTAs; repeated runs give identical bits; the bias variant adds bias[n]."""
-    L = Layer("int6", N, K, seed=11 * N + K)
+def test_gemv_int6_every_token_count(cuda, fmt, N, K):
+    """int6 tensor-core GEMV (dense and planar storage) at each M it serves (1..8: four token
+    buckets), with and without the split of K over CTAs; repeated runs give identical bits; the bias
+    variant adds bias[n]."""
+    L = Layer(fmt, N, K, seed=11 * N + K)
     w_ref = L.oracle_w()
     bias_b = synth.activations(N + K, 1, N)[0]
     for M in range(1, 9):
         xb, xd = x_dev(K, M, seed=100 + M)
         y = run_gemv(L, xd, M)
         y_ref = OC.matmul_f64(xb, w_ref)
-        assert_close(y, y_ref, f"int6 gemv N={N} K={K} M={M}")
+        assert_close(y, y_ref, f"{fmt} gemv N={N} K={K} M={M}")
         assert np.array_equal(y, run_gemv(L, xd, M))
         yb = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
         ql.qlinear_gemv_bias(L.desc, *L.packed(), xd, M, dev(bias_b).view(torch.bfloat16), yb)
