@@ -14,8 +14,8 @@ weight copy is touched only once per 491 MB of traffic (> 3x the 126 MB L2).
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
 Under torchrun (N > 1) every rank runs the same per-GPU workload on its own
-GPU (an independent row partition of a wider layer: no data-path
-collective); time is the max over ranks; rank 0 prints one JSON line.
+GPU (replicas: the layer has no data-path exchange, so no collective runs);
+time is the max over ranks; rank 0 prints one JSON line.
 """
 from __future__ import annotations
 
@@ -161,6 +161,19 @@ class ClockSampler:
                     reasons.add(name)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
                 "reasons": sorted(reasons), "samples": n}
+
+
+DATA = "synthetic (seeded uniform codes/metadata per the workload recipe; x ~ N(0,1) in bf16)"
+
+
+def workload_config(world: int) -> dict:
+    return {"workload": "int4 nested-superscale decode GEMV, M=1, layers (K=5120,N=27648) and (K=27648,N=5120)",
+            "M": 1, "layers": LAYERS,
+            "parallelism": (f"{world} replicas: every rank runs the same two layers on its own GPU, no "
+                            f"collective" if world > 1 else "single GPU"),
+            "launch": "the K timed steps are one CUDA graph of 2K qlinear_gemv calls",
+            "l2": f"{COPIES} rotating packed copies per layer "
+                  f"({COPIES * sum(gemv_bytes(K, N) for K, N in LAYERS) / 1e6:.0f} MB per rotation > 3x 126 MB L2)"}
 
 
 def load_peaks():
@@ -348,13 +361,8 @@ def run_native(args):
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "int4 weights, bf16 activations, fp32 accumulate",
-        "data": "synthetic (seeded uniform codes/metadata per the workload recipe; x ~ N(0,1) in bf16)",
-        "config": {"workload": "int4 nested-superscale decode GEMV, M=1, layers (K=5120,N=27648) and "
-                               "(K=27648,N=5120)", "M": 1, "layers": LAYERS,
-                   "parallelism": f"{world} independent row partitions" if world > 1 else "single GPU",
-                   "launch": "the K timed steps are one CUDA graph of 2K qlinear_gemv calls",
-                   "l2": f"{COPIES} rotating packed copies per layer "
-                         f"({COPIES * step_bytes / 1e6:.0f} MB per rotation > 3x 126 MB L2)"},
+        "data": DATA,
+        "config": workload_config(world),
         "pct_hbm_peak": round(100 * value_bps / 1e9 / peaks["hbm_gbs"], 2),
         "roofline": {"bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": round(achieved_gbs / peaks["hbm_gbs"], 4), "traffic": traffic,
@@ -429,7 +437,7 @@ def packed_layer(wl, device):
     t16 = lambda a: torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a).to(device)
     if wl.fmt == "int4":
         u = (w["q"], w["sc"], w["zc"], w["ss"], w["zs"])
-    elif wl.fmt == "int6":
+    elif wl.fmt in ("int6", "int6p"):
         u = (w["q"], w["sc"], None, w["st"], None)
     else:
         u = (w["q"], w["s"], w["b"], None, None)
@@ -440,32 +448,37 @@ def packed_layer(wl, device):
 
 def run_other_configs(device, peaks):
     """The remaining workload configurations, each at its batch sizes: GB/s of algorithmic bytes for
-    the GEMVs (CUDA-graph replays of 30 calls over 3 rotating weight copies), TFLOP/s for the GEMM
-    (CUDA events around single calls, 256 MiB written between calls)."""
+    the GEMVs (CUDA-graph replays of at least 30 calls over enough rotating weight copies to move 3x
+    the L2 per pass), TFLOP/s for the GEMM (CUDA events around single calls, 256 MiB written between
+    calls)."""
     import torch
 
     import int6_quantized_linear_b200 as ql
     from int6_quantized_linear_b200 import synth
 
     out = {}
-    for name in ("int4_gemv_k5120_n27648", "int4_gemv_k27648_n5120", "int6_gemv_k5120_n5120",
-                 "int6_gemv_k5120_n27648", "affine2_k4096_n14336", "affine4_k4096_n14336",
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    for name in ("int4_gemv_2048x2048", "int4_gemv_k5120_n27648", "int4_gemv_k27648_n5120",
+                 "int6_gemv_k5120_n5120", "int6_gemv_k5120_n27648", "int6p_gemv_k5120_n5120",
+                 "int6p_gemv_k5120_n27648", "affine2_k4096_n14336", "affine4_k4096_n14336",
                  "affine8_k4096_n14336"):
         wl = synth.WORKLOADS[name]
         d, p0, wbytes = packed_layer(wl, device)
-        reps = [p0] + [tuple(t.clone() for t in p0) for _ in range(2)]
+        # enough rotating copies that one pass over them moves over 3x the L2 (every call reads HBM)
+        copies = max(3, -(-3 * l2 // wbytes))
+        reps = [p0] + [tuple(t.clone() for t in p0) for _ in range(copies - 1)]
         xb = torch.from_numpy(wl.x(max(wl.Ms)).view("int16")).to(device).view(torch.bfloat16)
         res = {}
         for M in wl.Ms:
-            if name.startswith("int4") and M == 1:
+            if name.startswith("int4") and name != "int4_gemv_2048x2048" and M == 1:
                 continue  # the headline line above
             x = xb[:M].contiguous()
             y = torch.empty((M, wl.N), dtype=torch.bfloat16, device=device)
             ws = ql.alloc_gemv_workspace(d, M, device)
             for i in range(3):
                 ql.qlinear_gemv(d, *reps[i], x, M, y, ws)
-            calls = 30
-            g = capture(lambda: [ql.qlinear_gemv(d, *reps[i % 3], x, M, y, ws) for i in range(calls)], device)
+            calls = max(30, copies)
+            g = capture(lambda: [ql.qlinear_gemv(d, *reps[i % copies], x, M, y, ws) for i in range(calls)], device)
             g.replay()
             torch.cuda.synchronize(device)
             a, b = _ev(), _ev()
@@ -477,7 +490,10 @@ def run_other_configs(device, peaks):
             us = a.elapsed_time(b) * 1e3 / (2 * calls)
             nbytes = wbytes + M * wl.K * 2 + M * wl.N * 2
             res[f"M{M}"] = {"us": round(us, 3), "GB/s": round(nbytes / us / 1e3, 1),
-                            "frac_hbm": round(nbytes / us / 1e3 / peaks["hbm_gbs"], 4)}
+                            "frac_hbm": round(nbytes / us / 1e3 / peaks["hbm_gbs"], 4), "copies": copies}
+            if nbytes < 16e6:
+                res[f"M{M}"]["note"] = (f"{nbytes / 1e6:.1f} MB per call: launch- and latency-dominated "
+                                        f"(the weights alone take {nbytes / peaks['hbm_gbs'] / 1e3:.2f} us at peak)")
             del g
         out[name] = res
         del reps
@@ -553,6 +569,32 @@ def run_other_configs(device, peaks):
                         "frac_bf16_peak": round(tf / peaks["bf16_tflops"], 4)}
         del x, y, ws
     out["int4_gemm_k5120_n27648"] = res
+    # the tcgen05 GEMM on the other formats at M=2048: int6 (dense and planar) on the int6 layer's
+    # shape, affine on the affine layer's shape
+    for name in ("int6_gemv_k5120_n27648", "int6p_gemv_k5120_n27648", "affine2_k4096_n14336",
+                 "affine4_k4096_n14336", "affine8_k4096_n14336"):
+        wl = synth.WORKLOADS[name]
+        d, (c, g_, s), _ = packed_layer(wl, device)
+        M = 2048
+        x = torch.from_numpy(wl.x(M).view("int16")).to(device).view(torch.bfloat16)
+        y = torch.empty((M, wl.N), dtype=torch.bfloat16, device=device)
+        ws = ql.alloc_gemm_workspace(d, M, device)
+        for _ in range(2):
+            ql.qlinear_gemm(d, c, g_, s, x, M, y, ws)
+        times = []
+        for _ in range(5):
+            flush.fill_(1)
+            a, b = _ev(), _ev()
+            a.record()
+            ql.qlinear_gemm(d, c, g_, s, x, M, y, ws)
+            b.record()
+            torch.cuda.synchronize(device)
+            times.append(a.elapsed_time(b) / 1e3)
+        t = statistics.median(times)
+        tf = 2.0 * M * wl.N * wl.K / t / 1e12
+        out["gemm_M2048_" + name.split("_")[0] + f"_k{wl.K}_n{wl.N}"] = {
+            "ms": round(t * 1e3, 4), "TFLOP/s": round(tf, 1), "frac_bf16_peak": round(tf / peaks["bf16_tflops"], 4)}
+        del x, y, ws, c, g_, s
     assert ql.qlinear_sync_status() == ql.QL_OK
     return out
 
@@ -596,32 +638,77 @@ def run_e2e(args, layers, device, step_bytes):
 # CPU oracle: the baseline leg and the reference arm
 # ---------------------------------------------------------------------------
 
-def _oracle_sample_step(rows_per_layer: int):
-    """One oracle pass: dequantise a sample of rows of each decode layer and multiply in fp64.
-    Returns (algorithmic bytes covered, seconds)."""
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def oracle_layers(rows=None):
+    """Both decode layers packed by the C oracle (the first `rows` rows of each when given), with
+    their activation row: the same seeded inputs as the CUDA arm."""
     from int6_quantized_linear_b200 import synth
     from oracle import oracle_c as OC
 
-    total_bytes, total_s = 0, 0.0
+    out = []
     for (K, N) in LAYERS:
-        n = min(N, rows_per_layer)
-        w = synth.int4_weights(1, n, K)  # same recipe; a leading block of rows
-        x = synth.activations(1, 1, K)
-        packed = OC.int4_pack(w["q"], w["sc"], w["zc"], w["ss"], w["zs"])
-        t0 = time.perf_counter()
-        wf = OC.int4_dequant(*packed)
-        OC.matmul_f64(x, wf)
-        total_s += time.perf_counter() - t0
-        total_bytes += gemv_bytes(K, n)
-    return total_bytes, total_s
+        n = N if rows is None else min(N, rows)
+        w = synth.int4_weights(1, N, K)  # the full layer's draw (a leading block of rows of it)
+        packed = OC.int4_pack(w["q"][:n], w["sc"][:n], w["zc"][:n], w["ss"][:n], w["zs"][:n])
+        del w
+        out.append(dict(K=K, N=n, packed=packed, x=synth.activations(1, 1, K)))
+    return out
 
 
-def cpu_baseline(rows_per_layer: int = 2048) -> dict:
+def oracle_step(layers, block_weights: int = 1 << 24):
+    """One pass of the C oracle over the given layers (fp32 dequant + fp64 matmul), in blocks of rows
+    of about `block_weights` weights so host memory stays bounded.  Returns (algorithmic bytes, s)."""
     from oracle import oracle_c as OC
-    b, s = _oracle_sample_step(rows_per_layer)
-    return {"value": round(b / s / 1e9, 4), "unit": "GB/s", "cores": OC.num_threads(), "kind": "oracle",
-            "sample": f"first {rows_per_layer} rows of each decode layer, M=1: C oracle fp32 dequant + "
-                      f"fp64 matmul ({b / 1e6:.1f} MB of algorithmic bytes in {s:.2f} s)"}
+
+    total_b, total_s = 0, 0.0
+    for L in layers:
+        codes, gmeta, steps = L["packed"]
+        rb = max(1, block_weights // L["K"])
+        for r0 in range(0, L["N"], rb):
+            sl = slice(r0, min(L["N"], r0 + rb))
+            t0 = time.perf_counter()
+            wf = OC.int4_dequant(codes[sl], gmeta[sl], steps[sl])
+            OC.matmul_f64(L["x"], wf)
+            total_s += time.perf_counter() - t0
+        total_b += gemv_bytes(L["K"], L["N"])
+    return total_b, total_s
+
+
+def cpu_baseline(min_seconds: float = 10.0, one_core_rows: int = 1024) -> dict:
+    """The C oracle on this host: whole decode steps (both layers, every row) on all cores, repeated
+    until about `min_seconds` of CPU work; then one core on the first rows of each layer."""
+    from oracle import oracle_c as OC
+
+    cores = OC.num_threads()
+    layers = oracle_layers()
+    b_all, s_all, steps = 0, 0.0, 0
+    while s_all < min_seconds:
+        b, s = oracle_step(layers)
+        b_all, s_all, steps = b_all + b, s_all + s, steps + 1
+    del layers
+    small = oracle_layers(one_core_rows)
+    OC.set_num_threads(1)
+    try:
+        b1, s1 = oracle_step(small)
+    finally:
+        OC.set_num_threads(cores)
+    return {"value": round(b_all / s_all / 1e9, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "cpu_model": cpu_model(),
+            "sample": f"{steps} whole decode steps (both layers, all rows, M=1): C oracle fp32 dequant + fp64 "
+                      f"matmul, {b_all / 1e6:.0f} MB of algorithmic bytes in {s_all:.1f} s on {cores} threads",
+            "one_core": {"value": round(b1 / s1 / 1e9, 5), "unit": "GB/s", "cores": 1,
+                         "sample": f"first {one_core_rows} rows of each decode layer ({b1 / 1e6:.1f} MB in "
+                                   f"{s1:.2f} s)"}}
 
 
 def run_reference(args):
@@ -629,23 +716,24 @@ def run_reference(args):
     if rank != 0:  # the oracle runs once, on rank 0's host cores
         return None
     from oracle import oracle_c as OC
-    rows = 1024
+    layers = oracle_layers()
     for _ in range(args.warmup):
-        _oracle_sample_step(rows)
+        oracle_step(layers)
     tot_b, tot_s = 0, 0.0
     for _ in range(args.steps):
-        b, s = _oracle_sample_step(rows)
+        b, s = oracle_step(layers)
         tot_b += b
         tot_s += s
     v = tot_b / tot_s / 1e9
-    sample = f"first {rows} rows of each decode layer per step (C oracle fp32 dequant + fp64 matmul)"
+    cores = OC.num_threads()
+    sample = (f"whole decode steps: both layers, every row, M=1 (C oracle fp32 dequant + fp64 matmul on "
+              f"{cores} threads of {cpu_model()})")
     return {
         "impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(tot_s / args.steps * 1e3, 3),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int4 weights, fp64 matmul",
-        "data": "synthetic", "config": {"workload": "int4 nested-superscale decode GEMV, M=1, layers "
-                                                    "(K=5120,N=27648) and (K=27648,N=5120)", "M": 1},
-        "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": OC.num_threads(), "kind": "oracle",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int4 weights, bf16 activations, fp64 accumulate", "data": DATA, "config": workload_config(world),
+        "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
