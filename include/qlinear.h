@@ -240,8 +240,10 @@ ql_status qlinear_gemv_workspace_bytes(const ql_desc *desc, int64_t M, size_t *b
  *    read them, with the group's scale (and sum); then the streaming kernel
  *    multiplies the codes (as u8 or s8 bytes: 16q for nibbles, 4q for int6,
  *    q for 2- and 8-bit fields) by those bytes on the integer tensor core
- *    (mma.sync m16n8k32, exact s32 sums, one MMA per byte) and applies scale
- *    (and zero or bias) once per (row, group[, token]) in fp32.  int4 at M =
+ *    (mma.sync m16n8k32, exact s32 sums, one MMA per byte: high and middle
+ *    in the streaming loop, the low bytes of 24-bit super-blocks in a pass
+ *    after it that reads their weights again) and applies scale (and zero
+ *    or bias) once per (row, group[, token]) in fp32.  int4 at M =
  *    1 and int6 use a diagonal x operand (one MMA column per weight group);
  *    int4 at M >= 2 and affine use the tokens as MMA columns.  K may be split
  *    over warps or CTAs, the parts added in a fixed order through the
@@ -363,20 +365,18 @@ ql_status qlinear_gemm_noalloc(const ql_desc *desc, const ql_packed_const *w,
  * every stream: a status may come from work enqueued on another stream. */
 ql_status qlinear_sync_status(ql_stream_t stream);
 
-/* Bound, in SM clock cycles, of every device-side wait of the current
- * device's kernels for another role or for data (default 2e9, about 1 s at
- * the B200's clock); cycles <= 0 restores the default.  A kernel whose wait
- * runs out sets the device status word (qlinear_sync_status then returns
- * QL_ERR_TIMEOUT), makes its other roles leave their loops, waits for the
- * copies and MMAs it has in flight -- those drains always keep the default
- * bound -- frees its tensor memory and returns.  withhold_copies != 0 makes
- * the kernels' producers start no copies at all, so the first wait for data
- * is certain to run out (a wait can otherwise still be met by data arriving
- * within the bound); 0 restores normal operation.  Both exist so that tests
- * can drive that give-up path; callers normally never change them.  (The
- * pages have no counterpart.)  Synchronous; do not call it while this
- * library's kernels run.  Errors: QL_ERR_CUDA. */
-ql_status qlinear_set_wait_limit(int64_t cycles, int32_t withhold_copies);
+/* Every device-side wait of this library's kernels for another role or for
+ * data is bounded (2e9 SM clock cycles, about 1 s at the B200's clock).  A
+ * kernel whose wait runs out sets the device status word (qlinear_sync_status
+ * then returns QL_ERR_TIMEOUT), makes its other roles leave their loops, waits
+ * (bounded) for the copies and MMAs it has in flight, frees its tensor memory
+ * and returns.  on != 0 makes the current device's kernels start no copies at
+ * all, so their first wait for data is certain to run out (after about 1 s);
+ * 0 restores normal operation.  It exists so that tests can drive that
+ * give-up path; callers normally never change it.  (The pages have no
+ * counterpart.)  Synchronous; do not call it while this library's kernels
+ * run.  Errors: QL_ERR_CUDA. */
+ql_status qlinear_set_withhold_copies(int32_t on);
 
 /* Static, never NULL. */
 const char *qlinear_status_string(ql_status status);

@@ -66,7 +66,7 @@ _SIGNATURES = {
     "qlinear_gemm_noalloc": ([C.POINTER(ql_desc), C.POINTER(ql_packed), C.c_void_p, C.c_int64, C.c_void_p,
                               C.c_void_p], C.c_int),
     "qlinear_sync_status": ([C.c_void_p], C.c_int),
-    "qlinear_set_wait_limit": ([C.c_int64, C.c_int32], C.c_int),
+    "qlinear_set_withhold_copies": ([C.c_int32], C.c_int),
     "qlinear_gemv_bias": ([C.POINTER(ql_desc), C.POINTER(ql_packed), C.c_void_p, C.c_int64, C.c_void_p,
                            C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p], C.c_int),
     "qlinear_gemm_bias": ([C.POINTER(ql_desc), C.POINTER(ql_packed), C.c_void_p, C.c_int64, C.c_void_p,
@@ -267,10 +267,10 @@ def qlinear_gemm_noalloc(desc: Desc, codes, gmeta, steps, x, M: int, y, stream=N
            "qlinear_gemm_noalloc")
 
 
-def qlinear_set_wait_limit(cycles: int, withhold_copies: bool = False) -> None:
-    """Bound (SM clock cycles) of the kernels' waits on the current device (<= 0: the default), and
-    whether their producers withhold every copy.  For tests of the give-up path (QL_ERR_TIMEOUT)."""
-    _check(lib().qlinear_set_wait_limit(int(cycles), 1 if withhold_copies else 0), "qlinear_set_wait_limit")
+def qlinear_set_withhold_copies(on: bool) -> None:
+    """Whether the current device's kernels start no copies, so that their first wait for data runs
+    out (after about 1 s).  For tests of the give-up path (QL_ERR_TIMEOUT)."""
+    _check(lib().qlinear_set_withhold_copies(1 if on else 0), "qlinear_set_withhold_copies")
 
 
 def qlinear_sync_status(stream=None) -> int:

@@ -23,16 +23,13 @@ __device__ unsigned int g_ql_status;
 #define QL_DEV_TIMEOUT 1u
 #define QL_DEV_RANGE 2u  // an input outside the domain of the operation (reported as QL_ERR_RANGE)
 
-// ~1 s at the B200's 1.9 GHz SM clock: far longer than any legitimate wait.
+// Bound of every device-side wait: ~1 s at the B200's 1.9 GHz SM clock, far longer than any
+// legitimate wait.
 #define QL_WAIT_LIMIT_CYCLES 2000000000LL
 
-// Bound of the waits for another role or for data (qlinear_set_wait_limit changes it, to exercise
-// the give-up path in tests).  Waits that drain copies or MMAs already in flight before a CTA exits
-// always use QL_WAIT_LIMIT_CYCLES, so nothing lands in the shared memory of a CTA that has left.
-__constant__ long long g_ql_wait_limit = QL_WAIT_LIMIT_CYCLES;
-
-// Test switch (qlinear_set_wait_limit): when set, the kernels' producers start no copies, so the
-// first wait for data runs out.  Nothing is then in flight when a CTA gives up.
+// Test switch (qlinear_set_withhold_copies): when set, the kernels' producers start no copies, so the
+// first wait for data runs out.  Nothing is then in flight when a CTA gives up.  Kernels read it once,
+// as the bound of their copy loops (0 when set), so it costs the loops nothing.
 __constant__ int g_ql_withhold;
 QL_DEVI bool copies_withheld() { return g_ql_withhold != 0; }
 
@@ -83,7 +80,7 @@ QL_DEVI bool mbar_wait_bounded(uint32_t bar, uint32_t parity, volatile int *abor
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (clock64() - t0 > g_ql_wait_limit) {
+    if (clock64() - t0 > QL_WAIT_LIMIT_CYCLES) {
       atomicOr(&g_ql_status, QL_DEV_TIMEOUT);
       *abort = 1;
       return false;

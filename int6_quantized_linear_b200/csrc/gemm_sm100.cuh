@@ -265,8 +265,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t ph = 0;
       Cursor cur = cursor0();
       bool ok = true;
-      const bool hold = copies_withheld();
-      for (; it < total_it && !hold; ++it) {
+      const int64_t n_it = copies_withheld() ? 0 : total_it;  // steps whose copies are started
+      for (; it < n_it; ++it) {
         if (!mbar_wait_bounded(bar_empty(s), ph ^ 1u, abort_flag)) {
           ok = false;
           break;

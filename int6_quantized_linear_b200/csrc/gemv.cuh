@@ -89,30 +89,31 @@ __global__ void __launch_bounds__(256) gemv_simple_kernel(WeightPtrs p, int64_t 
 //   - 24-bit (max |x| in [2^22, 2^23)), exact within 2^15, for every group of
 //     a super-block in which some group's 16-bit rounding error exceeds 2^-12
 //     of that group's mass outside its largest element (a dominant outlier,
-//     where the 16-bit form would lose the other elements); the preparation
-//     pass flags such super-blocks and the kernel adds the third MMA there.
+//     where the 16-bit form would lose the other elements).
 // Per (row, group) of a super-block the integer sums are exact and below 2^22
 // in magnitude, so the accumulators start at 1.5 * 2^23 (as bits) and read
-// back as floats with one subtraction.  The scale and zero are applied once
-// per (row, group):
-//     T = 65536 * D_hi + 256 * D_mid + D_lo = 16 * 2^u * sum_k q_k x_int_k
-//     y += S * G_x * (T + Z * G_y)
-// with S = sc * ss, Z = zc * zs, u = 0 (24-bit) or 8 (16-bit), G_x = 2^-a_g /
-// (16 * 2^u) and G_y = -16 * 2^u * X_g, X_g = sum_k x_int_k.  A short
-// preparation pass writes the x bytes in the order the fragments read them
-// with (G_x, G_y) per group and the flag per super-block; the streaming kernel
-// is launched as a programmatic dependent of that pass and starts fetching
-// weights before it has finished (griddepcontrol.wait guards the first read of
-// x).  Lanes that hold no x for an MMA read a zero block, so no per-MMA
-// selects are needed.
+// back as floats with one subtraction.  The streaming loop runs the high and
+// middle bytes only and applies the scale and zero once per (row, group):
+//     T = 256 * D_hi + D_mid,   y += S * G_x * (T + Z * G_y)
+// with S = sc * ss, Z = zc * zs, X_g = sum_k x_int_k and (G_x, G_y) =
+// (2^-a_g / 16, -16 X_g), which for 16-bit x is the whole product.  For 24-bit
+// x, T is 2^-8 of 16 sum_k q_k x_int_k less the low bytes' share, so (G_x, G_y)
+// = (2^8 * 2^-a_g / 16, -16 X_g / 2^8), G_x carries the 24-bit marker
+// (mark_24bit), and after the loop an out-of-line pass adds S G_x 2^-8 D_lo for
+// the marked super-blocks, reading their weights again (gemv_m1_low_bytes).  A
+// short preparation pass writes the x bytes in the order the fragments read
+// them, (G_x, G_y) per group and a 24-bit flag per super-block; the streaming
+// kernel is launched as a programmatic dependent of that pass and starts
+// fetching weights before it has finished (griddepcontrol.wait guards the
+// first read of x).  Lanes that hold no x for an MMA read a zero block, so no
+// per-MMA selects are needed.
 // ===========================================================================
 
 constexpr int GEMV_MT_MAX_CTAS = 4096;  // bound on the CTAs of one multi-token launch (sizes its partial sums)
 
-// M = 1 x block per super-block: 8 x (G_x, G_y) (64 B), the super-block's 24-bit flag (16 B), the
-// (hi, mid) x words (1 KB) -- the part a stage copies -- then the lo x words (512 B), read from global
-// memory by the kernel only for a 24-bit super-block
-constexpr int GEMV_XBLOB = 1616, GEMV_XCOPY = 1104, GEMV_XB_FLAG = 64, GEMV_XB_Q = 80, GEMV_XB_L = 1104;
+// M = 1 x block per super-block: 8 x (G_x, G_y) (64 B) and the (hi, mid) x words (1 KB) -- the part
+// a stage copies -- then the lo x words (512 B), written and read only for a 24-bit super-block
+constexpr int GEMV_XBLOB = 1600, GEMV_XCOPY = 1088, GEMV_XB_Q = 64, GEMV_XB_L = 1088;
 
 struct GemvWorkspace {
   uint4 *xq;        // int4 M = 1: [K/256 super-blocks] blocks of GEMV_XBLOB bytes (gemv_xprep_kernel)
@@ -121,7 +122,7 @@ struct GemvWorkspace {
   float2 *gsum;     // M > 1: [K/32][M]: (G_x, G_y); int6: per 16-element group scales
   float *partial;   // M = 1: [16-row tile][part][16 rows]; M > 1: [CTA][M][64 rows]: sums of one K range
   int *counters;    // parts finished so far: M = 1 per 16-row tile, M > 1 per 64-row group
-  uint8_t *flags;   // M > 1, int6: [K/256][16]: byte m non-zero when token m's x of that super-block is 24-bit
+  uint8_t *flags;   // [K/256][16]: byte m non-zero when token m's x of that super-block is 24-bit
 };
 
 inline size_t gemv_workspace_bytes(int64_t M, int64_t N, int64_t K) {
@@ -154,6 +155,17 @@ QL_DEVI int atomic_add_acq_rel_gpu(int *addr, int v) {
 
 QL_DEVI void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 QL_DEVI void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Bring a line into L2 ahead of a dependent read: L2 is where the previous kernel's stores land, so a
+// load after griddepcontrol.wait still sees them, only sooner.
+QL_DEVI void prefetch_l2(const void *p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
+
+// The 24-bit marker: the lowest mantissa bit of a group's x scale G_x.  For 16-bit x, G_x is a power of
+// two (that bit is 0); for 24-bit x it is a normal power of two with the bit set, which changes it by
+// 2^-23 relative -- below the fp32 rounding of the sums it scales -- so the streaming loops use G_x as
+// stored, OR its bits together once per super-block and add the low bytes' share after the loop only
+// when the bit turned up.
+QL_DEVI float mark_24bit(float gx) { return __uint_as_float(__float_as_uint(gx) | 1u); }
+QL_DEVI float unmark(float gx) { return __uint_as_float(__float_as_uint(gx) & ~1u); }
 
 // Whether a group's 16-bit fixed point loses too much: the summed rounding error of its elements,
 // x * 2^a - rint(x * 2^a) with a the 16-bit exponent, above 2^-12 of the group's mass outside its
@@ -179,13 +191,14 @@ QL_DEVI bool group_needs_24bit(float err, float mass, float amax_scaled) {
 __global__ void __launch_bounds__(256) gemv_xprep_kernel(const __nv_bfloat16 *x, int64_t M, int64_t K,
                                                          int64_t n_counters, GemvWorkspace ws) {
   pdl_launch_dependents();  // the streaming kernel may start fetching weights now
-  pdl_wait();               // x (and this workspace) may belong to the kernel launched before this one
   const int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-  if (t < n_counters) ws.counters[t] = 0;
   const int64_t ng = K / 32;
   const int64_t gi = t >> 2;  // over M * ng groups
   const int c = (int)(t & 3);
   const bool live = gi < M * ng;  // every lane takes part in the shuffles
+  if (live) prefetch_l2(reinterpret_cast<const uint4 *>(x) + 4 * gi + c);
+  pdl_wait();               // x (and this workspace) may belong to the kernel launched before this one
+  if (t < n_counters) ws.counters[t] = 0;
   uint4 v = make_uint4(0u, 0u, 0u, 0u);
   if (live) v = __ldg(reinterpret_cast<const uint4 *>(x) + 4 * gi + c);  // 8 bf16 = 16 bytes
   const uint32_t u[4] = {v.x, v.y, v.z, v.w};
@@ -223,8 +236,8 @@ __global__ void __launch_bounds__(256) gemv_xprep_kernel(const __nv_bfloat16 *x,
   sum += __shfl_xor_sync(0xffffffffu, sum, 2);
   if (!live) return;
   // group gi = (m, super-block sb, group-in-block grp): per (m, sb) one block of GEMV_XBLOB bytes,
-  // the eight groups' (G_x, G_y), the flag, then chunk (j, kind) at [j][kind][grp] of the (hi, mid)
-  // region and of the lo region
+  // the eight groups' (G_x, G_y), then chunk (j, kind) at [j][kind][grp] of the (hi, mid) region
+  // and, for 24-bit x only, of the lo region
   const int64_t grp = gi & 7, msb = gi >> 3;
   uint8_t *blk = reinterpret_cast<uint8_t *>(ws.xq) + msb * GEMV_XBLOB;
   const int hs = sb24 ? 16 : 8;  // the value's top byte: bits 16.. (24-bit) or 8.. (16-bit, lo = 0)
@@ -236,17 +249,17 @@ __global__ void __launch_bounds__(256) gemv_xprep_kernel(const __nv_bfloat16 *x,
       const int val = xi[2 * b + kind];
       hi |= ((uint32_t)(val >> hs) & 0xffu) << (8 * b);
       mid |= ((uint32_t)(val >> (hs - 8)) & 0xffu) << (8 * b);
-      lo |= (sb24 ? ((uint32_t)val & 0xffu) : 0u) << (8 * b);
+      lo |= ((uint32_t)val & 0xffu) << (8 * b);
     }
     const int ch = 8 * (2 * c + kind) + (int)grp;  // chunk (j = c, kind) of group grp
     reinterpret_cast<uint4 *>(blk + GEMV_XB_Q)[ch] = grp < 4 ? make_uint4(hi, 0u, mid, 0u) : make_uint4(0u, hi, 0u, mid);
-    reinterpret_cast<uint2 *>(blk + GEMV_XB_L)[ch] = grp < 4 ? make_uint2(lo, 0u) : make_uint2(0u, lo);
+    if (sb24) reinterpret_cast<uint2 *>(blk + GEMV_XB_L)[ch] = grp < 4 ? make_uint2(lo, 0u) : make_uint2(0u, lo);
   }
-  if (c == 0) {  // (G_x, G_y) = (2^-a / (16 * 2^u), -16 * 2^u * X) with u = 0 (24-bit) or 8 (16-bit)
-    const float w = sb24 ? 16.f : 4096.f;
-    reinterpret_cast<float2 *>(blk)[grp] = make_float2(exp2i(-a) / w, -w * (float)sum);
+  if (c == 0) {  // (G_x, G_y) = (2^-a / 16, -16 X) scaled by (2^v, 2^-v), v = 8 (24-bit) or 0 (16-bit)
+    const float v = sb24 ? 256.f : 1.f, vi = sb24 ? 1.f / 256.f : 1.f, gx = exp2i(-a) * 0.0625f * v;
+    reinterpret_cast<float2 *>(blk)[grp] = make_float2(sb24 ? mark_24bit(gx) : gx, -16.f * (float)sum * vi);
   }
-  if ((t & 31) == 0) reinterpret_cast<uint32_t *>(blk + GEMV_XB_FLAG)[0] = sb24 ? 1u : 0u;
+  if ((t & 31) == 0) ws.flags[msb * 16] = sb24 ? 1 : 0;  // M = 1: msb is the super-block
 }
 
 // A byte of a metadata word as a float: 2^23 + b, to be fused into an FMA with -2^23 * step.
@@ -281,7 +294,7 @@ QL_DEVI uint32_t lds32(uint32_t a) {
 }
 
 // Wait for an mbarrier phase, letting the hardware suspend the thread (up to a hint, in ns) instead
-// of spinning; bounded like mbar_wait_bounded (the bound is read only once a try has failed).
+// of spinning; bounded like mbar_wait_bounded.
 QL_DEVI bool mbar_wait_suspend(uint32_t bar, uint32_t parity, volatile int *abort) {
   const long long t0 = clock64();
   const uint32_t hint = 1000000u;
@@ -296,7 +309,7 @@ QL_DEVI bool mbar_wait_suspend(uint32_t bar, uint32_t parity, volatile int *abor
         : "memory");
     if (ok) return true;
     if (*abort) return false;
-    if (clock64() - t0 > g_ql_wait_limit) {
+    if (clock64() - t0 > QL_WAIT_LIMIT_CYCLES) {
       atomicOr(&g_ql_status, QL_DEV_TIMEOUT);
       *abort = 1;
       return false;
@@ -325,15 +338,16 @@ constexpr int GEMV_CTAS_PER_SM = 3;
 constexpr int GEMV_WARPS = 4;  // warps per CTA: GEMV_WARPS / parts tiles, each split over `parts` warps
 // one stage = one super-block of a 16-row tile: codes (16 rows x 128 B, 128-byte swizzle), the
 // tile's group words [16 rows][16 B], then the first GEMV_XCOPY bytes of the super-block's x block:
-// 8 x (G_x, G_y), its 24-bit flag and its (hi, mid) x pairs [4 j][2 kinds][8 groups][16 B]
-constexpr int GEMV_ST_CODES = 0, GEMV_ST_GMETA = 2048, GEMV_ST_GSUM = 2304, GEMV_ST_FLAG = 2304 + GEMV_XB_FLAG,
-              GEMV_ST_X = 2304 + GEMV_XB_Q;
+// 8 x (G_x, G_y) and its (hi, mid) x pairs [4 j][2 kinds][8 groups][16 B]
+constexpr int GEMV_ST_CODES = 0, GEMV_ST_GMETA = 2048, GEMV_ST_GSUM = 2304, GEMV_ST_X = 2304 + GEMV_XB_Q;
 constexpr int GEMV_STAGE_BYTES = 4096;      // multiple of 1024 (the swizzle atom)
 constexpr uint32_t GEMV_STAGE_TX = 2048 + 256 + GEMV_XCOPY;
-static_assert(GEMV_ST_GSUM + GEMV_XCOPY <= GEMV_STAGE_BYTES && GEMV_XB_Q + 1024 == GEMV_XCOPY, "stage layout");
+static_assert(GEMV_ST_GSUM + GEMV_XCOPY <= GEMV_STAGE_BYTES && GEMV_XB_Q + 1024 == GEMV_XCOPY &&
+              GEMV_XB_L + 512 == GEMV_XBLOB && GEMV_XBLOB % 16 == 0, "stage layout");
 constexpr int GEMV_ZERO_BYTES = 1024;       // zero x chunks at a 128-byte stride, for lanes that feed no x
 
 struct GemvTcParams {
+  const uint8_t *codes, *gmeta;  // [N][K/2], [N][K/16]: read directly only by the 24-bit tail
   const uint8_t *steps;
   const __nv_bfloat16 *bias;  // [N] or NULL
   int64_t N, K;
@@ -345,6 +359,55 @@ struct GemvTcParams {
 // dynamic shared memory: [warp][stage] (1024-aligned), zero block, mbarriers
 inline constexpr int gemv_smem_bytes() {
   return GEMV_WARPS * GEMV_RING * GEMV_STAGE_BYTES + GEMV_ZERO_BYTES + GEMV_WARPS * GEMV_RING * 8 + 1024;
+}
+
+// The low bytes of 24-bit x for one warp of the M = 1 kernel: S G_x 2^-8 D_lo per (row, group) of every
+// flagged super-block of its range, the weights read again from global memory (q0, q1: the code rows of
+// rows r0, r1 at the range's first super-block; m0, m1: their group words; st0, st1: their step words;
+// fl: the range's flags).  Flagged super-blocks are rare, so this runs out of line and leaves the
+// streaming loop's registers alone.  Returns the sums to add for rows r0 and r1 (the lane's groups 2c,
+// 2c + 1).
+__device__ __noinline__ float2 gemv_m1_low_bytes(const uint8_t *q0, const uint8_t *q1, const uint8_t *m0,
+                                                 const uint8_t *m1, const uint32_t *st0, const uint32_t *st1,
+                                                 const uint8_t *xb_sb, const uint8_t *fl, int nsb) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
+  const bool on0 = (g == c), feed = on0 || (g == c + 4);
+  const uint2 *xlg = reinterpret_cast<const uint2 *>(xb_sb + GEMV_XB_L) + (on0 ? c : c + 4);
+  const int32_t acc_init[4] = {GEMV_ACC0, GEMV_ACC0, GEMV_ACC0, GEMV_ACC0};
+  float a0 = 0.f, a1 = 0.f;
+  for (int i = 0; i < nsb; ++i) {
+    if (__ldg(fl + (int64_t)i * 16) == 0) continue;  // the same for the whole warp
+    const uint4 *c0 = reinterpret_cast<const uint4 *>(q0 + (int64_t)i * 128);
+    const uint4 *c1 = reinterpret_cast<const uint4 *>(q1 + (int64_t)i * 128);
+    const uint4 v00 = __ldg(c0 + c), v01 = __ldg(c0 + c + 4), v10 = __ldg(c1 + c), v11 = __ldg(c1 + c + 4);
+    const uint32_t u00[4] = {v00.x, v00.y, v00.z, v00.w}, u01[4] = {v01.x, v01.y, v01.z, v01.w};
+    const uint32_t u10[4] = {v10.x, v10.y, v10.z, v10.w}, u11[4] = {v11.x, v11.y, v11.z, v11.w};
+    const uint2 *lg = xlg + (int64_t)i * (GEMV_XBLOB / 8);
+    int32_t dl[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint2 le = feed ? __ldg(lg + 16 * j) : make_uint2(0u, 0u);      // even k
+      const uint2 lo = feed ? __ldg(lg + 16 * j + 8) : make_uint2(0u, 0u);  // odd k
+      const uint32_t h00 = u00[j] & 0xF0F0F0F0u, h10 = u10[j] & 0xF0F0F0F0u;
+      const uint32_t h01 = u01[j] & 0xF0F0F0F0u, h11 = u11[j] & 0xF0F0F0F0u;
+      const uint32_t e00 = (u00[j] << 4) & 0xF0F0F0F0u, e10 = (u10[j] << 4) & 0xF0F0F0F0u;
+      const uint32_t e01 = (u01[j] << 4) & 0xF0F0F0F0u, e11 = (u11[j] << 4) & 0xF0F0F0F0u;
+      if (j == 0) QL_IMMA0("u8", dl, acc_init, h00, h10, h01, h11, lo.x, lo.y);
+      else QL_IMMA("u8", dl, h00, h10, h01, h11, lo.x, lo.y);
+      QL_IMMA("u8", dl, e00, e10, e01, e11, le.x, le.y);
+    }
+    // (G_x, G_y) of groups 2c, 2c + 1; S = sc * ss per row and group
+    const float4 G = __ldg(reinterpret_cast<const float4 *>(xb_sb + (int64_t)i * GEMV_XBLOB) + c);
+    const uint32_t cm0 = __ldg(reinterpret_cast<const uint32_t *>(m0 + (int64_t)i * 16) + c);
+    const uint32_t cm1 = __ldg(reinterpret_cast<const uint32_t *>(m1 + (int64_t)i * 16) + c);
+    const float ss0 = f16_bits_to_f32(__ldg(st0 + i)), ss1 = f16_bits_to_f32(__ldg(st1 + i));
+    const float gx0 = unmark(G.x) * (1.f / 256.f), gx1 = unmark(G.z) * (1.f / 256.f);
+    a0 = fmaf(fmaf(byte_magic(cm0, 0), ss0, -8388608.f * ss0) * gx0, __int_as_float(dl[0]) - GEMV_ACC0_F, a0);
+    a0 = fmaf(fmaf(byte_magic(cm0, 2), ss0, -8388608.f * ss0) * gx1, __int_as_float(dl[1]) - GEMV_ACC0_F, a0);
+    a1 = fmaf(fmaf(byte_magic(cm1, 0), ss1, -8388608.f * ss1) * gx0, __int_as_float(dl[2]) - GEMV_ACC0_F, a1);
+    a1 = fmaf(fmaf(byte_magic(cm1, 2), ss1, -8388608.f * ss1) * gx1, __int_as_float(dl[3]) - GEMV_ACC0_F, a1);
+  }
+  return make_float2(a0, a1);
 }
 
 // Everything a super-block needs except its step words arrives by one stage of a per-warp ring:
@@ -395,10 +458,10 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS, GEMV_CTAS_PER_SM)
   };
   auto issue_x = [&](int i, int s) {
     const uint32_t st = ring + s * GEMV_STAGE_BYTES, bar = bar0 + 8 * s;
-    bulk_load(st + GEMV_ST_GSUM, xb_sb + (int64_t)i * GEMV_XBLOB, GEMV_XCOPY, bar);  // sums, flag, then x
+    bulk_load(st + GEMV_ST_GSUM, xb_sb + (int64_t)i * GEMV_XBLOB, GEMV_XCOPY, bar);  // sums, then x
   };
-  const bool hold = copies_withheld();
-  const int pre = hold ? 0 : (nsb < GEMV_RING - 1 ? nsb : GEMV_RING - 1);
+  const int nis = copies_withheld() ? 0 : nsb;  // super-blocks whose copies this warp starts
+  const int pre = nis < GEMV_RING - 1 ? nis : GEMV_RING - 1;
   int issued = pre;  // super-blocks whose stage copies were started (lane 0's count is the one used)
   if (lane == 0) {
     tma_prefetch_desc(&map_codes);
@@ -428,16 +491,12 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS, GEMV_CTAS_PER_SM)
   // per-lane shared-memory addresses (offsets inside a stage are added as constants)
   const bool on0 = (g == c), on1 = (g == c + 4);
   const uint32_t zero_a = smem_u32(zero_blk);
-  // this lane's B pairs of MMA step (j, kind): (hi, mid) at xa + 128 (2 j + kind); for a 24-bit
-  // super-block its lo pairs in global memory at xlg + 8 (2 j + kind) (feeding lanes only)
-  uint32_t xa[GEMV_RING];
+  uint32_t xa[GEMV_RING];  // this lane's B pairs of MMA step (j, kind): (hi, mid) at xa + 128 (2 j + kind)
 #pragma unroll
   for (int s = 0; s < GEMV_RING; ++s) {
     xa[s] = on0 ? ring + s * GEMV_STAGE_BYTES + GEMV_ST_X + 16 * c
           : on1 ? ring + s * GEMV_STAGE_BYTES + GEMV_ST_X + 16 * (c + 4) : zero_a;
   }
-  const bool feed = on0 || on1;
-  const uint2 *xlg = reinterpret_cast<const uint2 *>(xb_sb + GEMV_XB_L) + (on0 ? c : c + 4);
   const uint32_t a00 = ring + pg * 128 + ((c ^ pg) << 4), a01 = ring + pg * 128 + (((c + 4) ^ pg) << 4);
   const uint32_t a10 = a00 + 1024, a11 = a01 + 1024;  // row pg + 8: same swizzle phase, next atom
   const uint32_t ag = ring + GEMV_ST_GSUM + 16 * c;
@@ -445,6 +504,7 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS, GEMV_CTAS_PER_SM)
 
   const int32_t acc_init[4] = {GEMV_ACC0, GEMV_ACC0, GEMV_ACC0, GEMV_ACC0};
   float acc0 = 0.f, acc1 = 0.f;
+  uint32_t x24s = 0u;  // bit 0: some super-block's G_x carries the 24-bit marker
   bool ok = true;
   for (int base = 0; base < nsb && ok; base += GEMV_RING) {
     const uint32_t par = (uint32_t)((base / GEMV_RING) & 1);
@@ -456,7 +516,7 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS, GEMV_CTAS_PER_SM)
       const int nx = i + GEMV_RING - 1;
       const int sn = (s + GEMV_RING - 1) % GEMV_RING;
       __syncwarp();  // every lane has read that stage in the previous turn
-      if (nx < nsb && !hold) {
+      if (nx < nis) {
         if (lane == 0) {
           issue_w(nx, sn);
           issue_x(nx, sn);
@@ -476,51 +536,36 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS, GEMV_CTAS_PER_SM)
       const uint32_t cm0 = lds32(am + so), cm1 = lds32(am + so + 128);
       const uint32_t ww00[4] = {w00.x, w00.y, w00.z, w00.w}, ww01[4] = {w01.x, w01.y, w01.z, w01.w};
       const uint32_t ww10[4] = {w10.x, w10.y, w10.z, w10.w}, ww11[4] = {w11.x, w11.y, w11.z, w11.w};
-      // D[q]: q = 0 (r0, group 2c), 1 (r0, 2c+1), 2 (r1, 2c), 3 (r1, 2c+1); T = 65536 D_hi + 256 D_mid (+ D_lo)
+      // D[q]: q = 0 (r0, group 2c), 1 (r0, 2c+1), 2 (r1, 2c), 3 (r1, 2c+1); T = 256 D_hi + D_mid
+      int32_t dh[4], dm[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint4 xe = lds128(xa[s] + 256 * j), xo = lds128(xa[s] + 256 * j + 128);  // even k, odd k
+        const uint32_t h00 = ww00[j] & 0xF0F0F0F0u, h10 = ww10[j] & 0xF0F0F0F0u;  // odd k, x16
+        const uint32_t h01 = ww01[j] & 0xF0F0F0F0u, h11 = ww11[j] & 0xF0F0F0F0u;
+        if (j == 0) {
+          QL_IMMA0("s8", dh, acc_init, h00, h10, h01, h11, xo.x, xo.y);
+          QL_IMMA0("u8", dm, acc_init, h00, h10, h01, h11, xo.z, xo.w);
+        } else {
+          QL_IMMA("s8", dh, h00, h10, h01, h11, xo.x, xo.y);
+          QL_IMMA("u8", dm, h00, h10, h01, h11, xo.z, xo.w);
+        }
+        const uint32_t e00 = (ww00[j] << 4) & 0xF0F0F0F0u, e10 = (ww10[j] << 4) & 0xF0F0F0F0u;  // even k, x16
+        const uint32_t e01 = (ww01[j] << 4) & 0xF0F0F0F0u, e11 = (ww11[j] << 4) & 0xF0F0F0F0u;
+        QL_IMMA("s8", dh, e00, e10, e01, e11, xe.x, xe.y);
+        QL_IMMA("u8", dm, e00, e10, e01, e11, xe.z, xe.w);
+      }
       float t[4];
-      auto contract = [&](auto x24c) {  // the super-block's MMAs: two bytes of x, or three for 24-bit x
-        constexpr bool X24 = decltype(x24c)::value;
-        const uint2 *lg = xlg + (int64_t)i * (GEMV_XBLOB / 8);
-        int32_t dh[4], dm[4], dl[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint4 xe = lds128(xa[s] + 256 * j), xo = lds128(xa[s] + 256 * j + 128);  // even k, odd k: hi, mid
-          const uint32_t h00 = ww00[j] & 0xF0F0F0F0u, h10 = ww10[j] & 0xF0F0F0F0u;  // odd k, x16
-          const uint32_t h01 = ww01[j] & 0xF0F0F0F0u, h11 = ww11[j] & 0xF0F0F0F0u;
-          const uint32_t e00 = (ww00[j] << 4) & 0xF0F0F0F0u, e10 = (ww10[j] << 4) & 0xF0F0F0F0u;  // even k, x16
-          const uint32_t e01 = (ww01[j] << 4) & 0xF0F0F0F0u, e11 = (ww11[j] << 4) & 0xF0F0F0F0u;
-          if (j == 0) {
-            QL_IMMA0("s8", dh, acc_init, h00, h10, h01, h11, xo.x, xo.y);
-            QL_IMMA0("u8", dm, acc_init, h00, h10, h01, h11, xo.z, xo.w);
-          } else {
-            QL_IMMA("s8", dh, h00, h10, h01, h11, xo.x, xo.y);
-            QL_IMMA("u8", dm, h00, h10, h01, h11, xo.z, xo.w);
-          }
-          QL_IMMA("s8", dh, e00, e10, e01, e11, xe.x, xe.y);
-          QL_IMMA("u8", dm, e00, e10, e01, e11, xe.z, xe.w);
-          if constexpr (X24) {  // the low byte, from global memory (L2): only feeding lanes hold any
-            const uint2 le = feed ? __ldg(lg + 16 * j) : make_uint2(0u, 0u);
-            const uint2 lo = feed ? __ldg(lg + 16 * j + 8) : make_uint2(0u, 0u);
-            if (j == 0) QL_IMMA0("u8", dl, acc_init, h00, h10, h01, h11, lo.x, lo.y);
-            else QL_IMMA("u8", dl, h00, h10, h01, h11, lo.x, lo.y);
-            QL_IMMA("u8", dl, e00, e10, e01, e11, le.x, le.y);
-          }
-        }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          t[q] = fmaf(__int_as_float(dh[q]) - GEMV_ACC0_F, 256.f, __int_as_float(dm[q]) - GEMV_ACC0_F);
-          if constexpr (X24) t[q] = fmaf(t[q], 256.f, __int_as_float(dl[q]) - GEMV_ACC0_F);
-          else t[q] *= 256.f;
-        }
-      };
-      if (lds32(ring + so + GEMV_ST_FLAG) != 0u) contract(std::true_type{});  // the same for the whole warp
-      else contract(std::false_type{});
+      for (int q = 0; q < 4; ++q)
+        t[q] = fmaf(__int_as_float(dh[q]) - GEMV_ACC0_F, 256.f, __int_as_float(dm[q]) - GEMV_ACC0_F);
       // S = sc * ss and Z = zc * zs, each one FMA from the byte placed in the mantissa of 2^23
       const uint32_t cs0 = sr0[s], cs1 = sr1[s];
       const float ss0 = f16_bits_to_f32(cs0), zs0 = f16_bits_to_f32(cs0 >> 16);
       const float ss1 = f16_bits_to_f32(cs1), zs1 = f16_bits_to_f32(cs1 >> 16);
       const float nss0 = -8388608.f * ss0, nzs0 = -8388608.f * zs0;
       const float nss1 = -8388608.f * ss1, nzs1 = -8388608.f * zs1;
+      x24s |= __float_as_uint(G.x);
       const float S00 = fmaf(byte_magic(cm0, 0), ss0, nss0) * G.x, Z00 = fmaf(byte_magic(cm0, 1), zs0, nzs0);
       const float S01 = fmaf(byte_magic(cm0, 2), ss0, nss0) * G.z, Z01 = fmaf(byte_magic(cm0, 3), zs0, nzs0);
       const float S10 = fmaf(byte_magic(cm1, 0), ss1, nss1) * G.x, Z10 = fmaf(byte_magic(cm1, 1), zs1, nzs1);
@@ -539,6 +584,15 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS, GEMV_CTAS_PER_SM)
              clock64() - t0 < QL_WAIT_LIMIT_CYCLES) {
       }
     }
+  }
+  if (__any_sync(0xffffffffu, (x24s & 1u) != 0u) && ok) {  // rare
+    const float2 lb = gemv_m1_low_bytes(p.codes + r0 * (p.K / 2) + (int64_t)sb0 * 128,
+                                        p.codes + r1 * (p.K / 2) + (int64_t)sb0 * 128,
+                                        p.gmeta + r0 * (p.K / 16) + (int64_t)sb0 * 16,
+                                        p.gmeta + r1 * (p.K / 16) + (int64_t)sb0 * 16, st0, st1, xb_sb,
+                                        p.ws.flags + (int64_t)sb0 * 16, nsb);
+    acc0 += lb.x;
+    acc1 += lb.y;
   }
   // the four lanes of a row hold its groups 2c, 2c+1: sum them
   acc0 += __shfl_xor_sync(0xffffffffu, acc0, 1);
@@ -609,14 +663,15 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS, GEMV_CTAS_PER_SM)
 __global__ void __launch_bounds__(256) gemv_xprep_mt_kernel(const __nv_bfloat16 *x, int64_t M, int64_t K,
                                                             int64_t n_counters, GemvWorkspace ws) {
   pdl_launch_dependents();  // the streaming kernel may start fetching weights now
-  pdl_wait();               // x (and this workspace) may belong to the kernel launched before this one
   const int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-  if (t < n_counters) ws.counters[t] = 0;
   const int64_t ng = K / 32;
   const int64_t gq = t >> 2;  // (token, group), token-major
   const int c = (int)(t & 3);
   const bool live = gq < M * ng;  // every lane takes part in the shuffles
   const int64_t m = live ? gq / ng : 0, g = live ? gq - m * ng : 0;
+  if (live) prefetch_l2(x + m * K + 32 * g + 8 * c);
+  pdl_wait();               // x (and this workspace) may belong to the kernel launched before this one
+  if (t < n_counters) ws.counters[t] = 0;
   uint4 v = make_uint4(0u, 0u, 0u, 0u);
   if (live) v = __ldg(reinterpret_cast<const uint4 *>(x + m * K + 32 * g + 8 * c));
   const uint32_t u[4] = {v.x, v.y, v.z, v.w};
@@ -652,32 +707,43 @@ __global__ void __launch_bounds__(256) gemv_xprep_mt_kernel(const __nv_bfloat16 
     sum += xe + xo;
     eh |= ((uint32_t)(xe >> hs) & 0xffu) << (8 * b);
     em |= ((uint32_t)(xe >> (hs - 8)) & 0xffu) << (8 * b);
-    el |= (sb24 ? ((uint32_t)xe & 0xffu) : 0u) << (8 * b);
+    el |= ((uint32_t)xe & 0xffu) << (8 * b);
     oh |= ((uint32_t)(xo >> hs) & 0xffu) << (8 * b);
     om |= ((uint32_t)(xo >> (hs - 8)) & 0xffu) << (8 * b);
-    ol |= (sb24 ? ((uint32_t)xo & 0xffu) : 0u) << (8 * b);
+    ol |= ((uint32_t)xo & 0xffu) << (8 * b);
   }
   sum += __shfl_xor_sync(0xffffffffu, sum, 1);
   sum += __shfl_xor_sync(0xffffffffu, sum, 2);
   if (!live) return;
   ws.xq[(g * M + m) * 4 + c] = make_uint4(eh, oh, em, om);
-  reinterpret_cast<uint2 *>(ws.xq + M * K / 8)[(g * M + m) * 4 + c] = make_uint2(el, ol);
-  if (c == 0) {  // (G_x, G_y) = (2^-a / (16 * 2^u), -16 * 2^u * X), u = 0 (24-bit) or 8 (16-bit)
-    const float w = sb24 ? 16.f : 4096.f;
-    ws.gsum[g * M + m] = make_float2(exp2i(-a) / w, -w * (float)sum);
+  if (sb24) reinterpret_cast<uint2 *>(ws.xq + M * K / 8)[(g * M + m) * 4 + c] = make_uint2(el, ol);
+  if (c == 0) {  // (G_x, G_y) = (2^-a / 16, -16 X) scaled by (2^v, 2^-v), v = 8 (24-bit) or 0 (16-bit)
+    const float v = sb24 ? 256.f : 1.f, vi = sb24 ? 1.f / 256.f : 1.f, gx = exp2i(-a) * 0.0625f * v;
+    ws.gsum[g * M + m] = make_float2(sb24 ? mark_24bit(gx) : gx, -16.f * (float)sum * vi);
   }
   if ((threadIdx.x & 31) == 0) ws.flags[(g >> 3) * 16 + m] = sb24 ? 1 : 0;
 }
 
 constexpr int GEMV_MT_WARPS = 4;  // consumer warps per CTA; warp 4 produces
 constexpr int GEMV_MT_THREADS = 32 * (GEMV_MT_WARPS + 1);
+// int4: three CTAs an SM, so at most 128 registers a thread (an SM partition's 16K registers hold four
+// of their warps).  Affine: two CTAs an SM with up to GEMV_MT_AFFINE_NREG registers a thread (three
+// warps a partition) -- at the row counts it serves its per-CTA rate, not the CTA count, bounds it,
+// and the extra registers raise that rate.
 constexpr int GEMV_MT_CTAS_PER_SM = 3;
+constexpr int GEMV_MT_AFFINE_CTAS_PER_SM = 2;
+#define GEMV_MT_AFFINE_NREG 168
+// the warps of the resident CTAs spread over an SM's four partitions of 16K registers each
+static_assert(((GEMV_MT_AFFINE_CTAS_PER_SM * GEMV_MT_THREADS / 32 + 3) / 4) * 32 * GEMV_MT_AFFINE_NREG <= 16384 &&
+                  ((GEMV_MT_CTAS_PER_SM * GEMV_MT_THREADS / 32 + 3) / 4) * 32 * 128 <= 16384,
+              "register budgets of the multi-token kernels");
+template <int FMT>
+constexpr int gemv_mt_ctas_per_sm() { return FMT == FMT_INT4 ? GEMV_MT_CTAS_PER_SM : GEMV_MT_AFFINE_CTAS_PER_SM; }
 
 // Stage layout of the multi-token kernel per format, for one 256-weight super-block of 64 rows:
 // codes [64 rows][CODE_ROW B] as swizzled boxes of CODE_BOX B (128-byte swizzle; 64-byte swizzle for
 // the 64-byte rows of 2-bit codes), group words [64][META_ROW B], group sums [8][M][8 B], (hi, mid) x
-// words [8 groups][M][4][16 B] and the 24-bit flags [16 B]; a 24-bit super-block's lo x words are read
-// from global memory.  int4 and 4-bit affine codes share one layout (a nibble per weight, low
+// words [8 groups][M][4][16 B].  A 24-bit super-block's lo x words are read from global memory.  int4 and 4-bit affine codes share one layout (a nibble per weight, low
 // nibble first); 8-bit affine codes are bytes; 2-bit codes are 16 per word, lowest bits first.
 template <int FMT, int BITS, int G>
 struct MtLayout {
@@ -688,13 +754,22 @@ struct MtLayout {
   static constexpr int ST_GMETA = CODE_BOXES * 64 * CODE_BOX;
   static constexpr int ST_GSUM = ST_GMETA + 64 * META_ROW;
   static constexpr int ST_X = ST_GSUM + 512;
-  static constexpr int ST_FL = ST_X + 4096;  // 16 B: a byte per token, non-zero when its x is 24-bit
-  static constexpr int STAGE = (ST_FL + 16 + 1023) / 1024 * 1024;
-  static constexpr int RING = 3 * (4 * STAGE + 1024) <= 227 * 1024 ? 4 : 3;
-  static constexpr int SMEM = RING * STAGE + RING * 16 + 16 + 1024;
+  static constexpr int STAGE = (ST_X + 4096 + 1023) / 1024 * 1024;
+  // CTAs an SM holds (gemv_mt_ctas_per_sm) and the deepest ring (up to 4 stages for int4, 6 for affine)
+  // with which they share its 228 KB of shared memory (1 KB of it reserved per CTA)
+  static constexpr int CTAS = FMT == FMT_INT4 ? GEMV_MT_CTAS_PER_SM : GEMV_MT_AFFINE_CTAS_PER_SM;
+  static constexpr int PER_CTA = 233472 / CTAS - 1024 - (1024 + 6 * 16 + 16);
+  static constexpr int RING = (FMT == FMT_INT4 ? 4 : 6) < PER_CTA / STAGE ? (FMT == FMT_INT4 ? 4 : 6) : PER_CTA / STAGE;
+  static constexpr int USED = RING * STAGE + RING * 16 + 16 + 1024;  // stages, barriers, flags, alignment
+  // affine: the request also keeps a CTAS + 1-th CTA off the SM, so the row groups spread over more SMs
+  static constexpr int FLOOR = FMT == FMT_INT4 ? 0 : 233472 / (CTAS + 1);
+  static constexpr int SMEM = USED > FLOOR ? USED : FLOOR;
+  static_assert(RING >= 3 && CTAS * (SMEM + 1024) <= 233472 && (CTAS + 1) * (SMEM + 1024) > 233472 || FMT == FMT_INT4,
+                "affine ring and occupancy");
 };
 
 struct GemvMtParams {
+  const uint8_t *codes, *gmeta;  // read directly only by the 24-bit tail
   const uint8_t *steps;       // int4 step words; unused for affine
   const __nv_bfloat16 *bias;  // [N] or NULL
   int64_t N, K;
@@ -707,15 +782,92 @@ struct GemvMtParams {
 template <int FMT, int BITS, int G>
 inline constexpr int gemv_mt_smem_bytes() { return MtLayout<FMT, BITS, G>::SMEM; }
 
+// The low bytes of 24-bit x for one consumer warp of the multi-token kernel: S G_x 2^-8 D_lo per (row,
+// token, 32-weight group) of every super-block of the range [sb0, sb0 + nsb) in which some token's x
+// is 24-bit, the weights read again from global memory (rows c0, c1; rows past N read row N - 1 and
+// their sums are never stored).  Flagged super-blocks are rare, so this runs out of line and leaves
+// the streaming loop's registers alone.  Returns the sums to add for (row g | g + 8) x (token 2c |
+// 2c + 1).
+template <int FMT, int BITS, int G>
+__device__ __noinline__ float4 gemv_mt_low_bytes(const uint8_t *codes, const uint8_t *gmeta, int64_t c0, int64_t c1,
+                                                 const uint32_t *st0, const uint32_t *st1, const uint8_t *flags,
+                                                 const float2 *gsum, const uint2 *xlg, int64_t K, int M, int sb0,
+                                                 int nsb) {
+  using L = MtLayout<FMT, BITS, G>;
+  const int lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
+  const int tk0 = 2 * c, tk1 = 2 * c + 1;
+  const uint64_t fmask = M >= 8 ? ~0ull : ((1ull << (8 * M)) - 1);  // the flag bytes of tokens < M
+  const int32_t acc_init[4] = {GEMV_ACC0, GEMV_ACC0, GEMV_ACC0, GEMV_ACC0};
+  constexpr int64_t CB = FMT == FMT_INT4 ? 128 : 32 * BITS;  // code bytes per row and super-block
+  constexpr int64_t MB = L::META_ROW;                         // group-word bytes per row and super-block
+  constexpr float SF = (FMT == FMT_INT4 || BITS == 4) ? 1.f : 16.f;
+  const uint8_t *q0 = codes + c0 * (K / 256) * CB, *q1 = codes + c1 * (K / 256) * CB;
+  const uint8_t *g0 = gmeta + c0 * (K / 256) * MB, *g1 = gmeta + c1 * (K / 256) * MB;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int i = 0; i < nsb; ++i) {
+    const int64_t sb = sb0 + i;
+    const uint2 fw = __ldg(reinterpret_cast<const uint2 *>(flags + sb * 16));
+    const uint64_t f24 = ((uint64_t)fw.y << 32 | fw.x) & fmask;
+    if (f24 == 0) continue;  // the same for the whole warp
+    const bool mine24 = g < M && ((f24 >> (8 * g)) & 0xffu) != 0;  // token g: this lane's column
+    float ss0 = 0.f, ss1 = 0.f;
+    if constexpr (FMT == FMT_INT4) {
+      ss0 = f16_bits_to_f32(__ldg(st0 + i));
+      ss1 = f16_bits_to_f32(__ldg(st1 + i));
+    }
+#pragma unroll 1
+    for (int gg = 0; gg < 8; ++gg) {
+      uint32_t e0, e1, o0, o1;  // as in the streaming loop, from the unswizzled rows
+      if constexpr (FMT == FMT_INT4 || BITS == 4) {
+        const uint32_t w0 = __ldg(reinterpret_cast<const uint32_t *>(q0 + sb * CB + 16 * gg + 4 * c));
+        const uint32_t w1 = __ldg(reinterpret_cast<const uint32_t *>(q1 + sb * CB + 16 * gg + 4 * c));
+        e0 = (w0 << 4) & 0xF0F0F0F0u; e1 = (w1 << 4) & 0xF0F0F0F0u;
+        o0 = w0 & 0xF0F0F0F0u; o1 = w1 & 0xF0F0F0F0u;
+      } else if constexpr (BITS == 2) {
+        const uint32_t sel = (c & 1) ? 0x4342u : 0x4140u;
+        const uint32_t t0 = __byte_perm(__ldg(reinterpret_cast<const uint32_t *>(q0 + sb * CB + 8 * gg + 4 * (c >> 1))), 0u, sel);
+        const uint32_t t1 = __byte_perm(__ldg(reinterpret_cast<const uint32_t *>(q1 + sb * CB + 8 * gg + 4 * (c >> 1))), 0u, sel);
+        const uint32_t u0 = (t0 | (t0 << 4)) & 0x0F0F0F0Fu, u1 = (t1 | (t1 << 4)) & 0x0F0F0F0Fu;
+        e0 = u0 & 0x03030303u; e1 = u1 & 0x03030303u;
+        o0 = (u0 >> 2) & 0x03030303u; o1 = (u1 >> 2) & 0x03030303u;
+      } else {
+        const uint2 w0 = __ldg(reinterpret_cast<const uint2 *>(q0 + sb * CB + 32 * gg + 8 * c));
+        const uint2 w1 = __ldg(reinterpret_cast<const uint2 *>(q1 + sb * CB + 32 * gg + 8 * c));
+        e0 = __byte_perm(w0.x, w0.y, 0x6420); e1 = __byte_perm(w1.x, w1.y, 0x6420);
+        o0 = __byte_perm(w0.x, w0.y, 0x7531); o1 = __byte_perm(w1.x, w1.y, 0x7531);
+      }
+      const int64_t grp = sb * 8 + gg;
+      const uint2 xl = mine24 ? __ldg(xlg + (grp * M + g) * 4 + c) : make_uint2(0u, 0u);
+      int32_t dl[4];
+      QL_IMMA0("u8", dl, acc_init, e0, e1, o0, o1, xl.x, xl.y);
+      const float ga = tk0 < M ? unmark(__ldg(&gsum[grp * M + tk0].x)) * (1.f / 256.f) : 0.f;
+      const float gb = tk1 < M ? unmark(__ldg(&gsum[grp * M + tk1].x)) * (1.f / 256.f) : 0.f;
+      float S0, S1;
+      if constexpr (FMT == FMT_INT4) {
+        const int bsc = 2 * (gg & 1);
+        S0 = fmaf(byte_magic(__ldg(reinterpret_cast<const uint32_t *>(g0 + sb * MB) + (gg >> 1)), bsc), ss0, -8388608.f * ss0);
+        S1 = fmaf(byte_magic(__ldg(reinterpret_cast<const uint32_t *>(g1 + sb * MB) + (gg >> 1)), bsc), ss1, -8388608.f * ss1);
+      } else {
+        S0 = bf16_bits_to_f32(__ldg(reinterpret_cast<const uint32_t *>(g0 + sb * MB) + gg * 32 / G)) * SF;
+        S1 = bf16_bits_to_f32(__ldg(reinterpret_cast<const uint32_t *>(g1 + sb * MB) + gg * 32 / G)) * SF;
+      }
+      acc.x = fmaf(S0 * ga, __int_as_float(dl[0]) - GEMV_ACC0_F, acc.x);
+      acc.y = fmaf(S0 * gb, __int_as_float(dl[1]) - GEMV_ACC0_F, acc.y);
+      acc.z = fmaf(S1 * ga, __int_as_float(dl[2]) - GEMV_ACC0_F, acc.z);
+      acc.w = fmaf(S1 * gb, __int_as_float(dl[3]) - GEMV_ACC0_F, acc.w);
+    }
+  }
+  return acc;
+}
+
 // int4: w = (q - zc zs)(sc ss) with the step word per super-block; affine (2 / 4 / 8 bits, group 32
 // or 64): w = q s + b with (s, b) bf16 per group.  Per (row, token, 32-weight slice) the integer MMA
 // gives T = sum_k A_k x_int_k with A = 16 q (nibbles) or q (2-bit fields, bytes); then
 //   int4:   y += S (2^-a / 16) (T - 16 Z X)
 //   affine: y += s' (2^-a / 16) T + b 2^-a X      (s' = s for nibbles, 16 s otherwise)
 template <int FMT, int BITS, int G>
-__global__ void __launch_bounds__(GEMV_MT_THREADS, GEMV_MT_CTAS_PER_SM)
-    gemv_mt_kernel(const __grid_constant__ CUtensorMap map_codes, const __grid_constant__ CUtensorMap map_gmeta,
-                   GemvMtParams p) {
+__device__ __forceinline__ void gemv_mt_body(const CUtensorMap &map_codes, const CUtensorMap &map_gmeta,
+                                             const GemvMtParams &p) {
   using L = MtLayout<FMT, BITS, G>;
   constexpr int RING = L::RING;
   extern __shared__ uint8_t smem_raw[];
@@ -741,6 +893,12 @@ __global__ void __launch_bounds__(GEMV_MT_THREADS, GEMV_MT_CTAS_PER_SM)
     flags[1] = 0;
     fence_mbar_init();
   }
+  // the (G_x, G_y) slots of tokens M..7 in every stage: never written by the copies, read (and their
+  // sums dropped) by lanes whose tokens are past M; zero, so they carry no 24-bit marker
+  if (threadIdx.x < (8 - M) * 16) {
+#pragma unroll
+    for (int s = 0; s < RING; ++s) reinterpret_cast<uint32_t *>(smem + s * L::STAGE + L::ST_GSUM + M * 64)[threadIdx.x] = 0u;
+  }
   __syncthreads();
   pdl_launch_dependents();  // the next call's preparation pass waits for this grid before touching anything
 
@@ -748,7 +906,7 @@ __global__ void __launch_bounds__(GEMV_MT_THREADS, GEMV_MT_CTAS_PER_SM)
     if (lane == 0) {
       tma_prefetch_desc(&map_codes);
       tma_prefetch_desc(&map_gmeta);
-      const uint32_t tx = L::ST_GSUM + (uint32_t)M * (64 + 512) + 16;  // codes, group words, sums, x, flags
+      const uint32_t tx = L::ST_GSUM + (uint32_t)M * (64 + 512);  // codes, group words, sums, x
       auto issue_w = [&](int i, int s) {
         const uint32_t st = sbase + s * L::STAGE;
         mbar_arrive_expect_tx(bar_full(s), tx);
@@ -763,10 +921,9 @@ __global__ void __launch_bounds__(GEMV_MT_THREADS, GEMV_MT_CTAS_PER_SM)
         const int64_t g0 = (int64_t)(sb0 + i) * 8;  // first 32-element group of the super-block
         bulk_load(st + L::ST_GSUM, p.ws.gsum + g0 * M, (uint32_t)M * 64, bar_full(s));
         bulk_load(st + L::ST_X, p.ws.xq + g0 * M * 4, (uint32_t)M * 512, bar_full(s));
-        bulk_load(st + L::ST_FL, p.ws.flags + (sb0 + i) * 16, 16, bar_full(s));
       };
-      const bool hold = copies_withheld();
-      const int pre = hold ? 0 : (nsb < RING ? nsb : RING);
+      const int nis = copies_withheld() ? 0 : nsb;  // super-blocks whose copies are started
+      const int pre = nis < RING ? nis : RING;
       for (int i = 0; i < pre; ++i) issue_w(i, i);  // weights need no x
       pdl_wait();
       for (int i = 0; i < pre; ++i) issue_x(i, i);
@@ -774,7 +931,7 @@ __global__ void __launch_bounds__(GEMV_MT_THREADS, GEMV_MT_CTAS_PER_SM)
       uint32_t ph = 0;
       bool ok = true;
       int i = pre;
-      for (; i < nsb && !hold; ++i) {  // unit i reuses the stage of unit i - RING
+      for (; i < nis; ++i) {  // unit i reuses the stage of unit i - RING
         if (!mbar_wait_bounded(bar_empty(s), ph, abort_flag)) {
           ok = false;
           break;
@@ -818,6 +975,7 @@ __global__ void __launch_bounds__(GEMV_MT_THREADS, GEMV_MT_CTAS_PER_SM)
     const uint2 *xlg = reinterpret_cast<const uint2 *>(p.ws.xq + (int64_t)M * p.K / 8);  // lo x words
     float acc[4] = {0.f, 0.f, 0.f, 0.f};  // (row g | g + 8) x (token 2c | 2c + 1)
     const uint32_t sw = (uint32_t)(r0 & 7);
+    uint32_t x24s = 0u;  // bit 0: some super-block's G_x of token 2c or 2c + 1 carries the 24-bit marker
     bool ok = true;
     for (int base = 0; base < nsb && ok; base += RING) {
       const uint32_t par = (uint32_t)((base / RING) & 1);
@@ -837,12 +995,6 @@ __global__ void __launch_bounds__(GEMV_MT_THREADS, GEMV_MT_CTAS_PER_SM)
           break;
         }
         const uint32_t stg = sbase + s * L::STAGE;
-        bool x24;  // some token's x of this super-block is 24-bit: the low-byte MMA runs (the same for the warp)
-        {
-          const uint2 fw = lds64(stg + L::ST_FL);
-          const uint64_t f = ((uint64_t)fw.y << 32 | fw.x) & (M >= 8 ? ~0ull : ((1ull << (8 * M)) - 1));
-          x24 = f != 0;
-        }
         // group words of rows r0, r1 (int4: 8 x u16 sc|zc; affine: 256/G x u32 s|b)
         uint32_t gw0[L::META_ROW / 4], gw1[L::META_ROW / 4];
 #pragma unroll
@@ -860,85 +1012,87 @@ __global__ void __launch_bounds__(GEMV_MT_THREADS, GEMV_MT_CTAS_PER_SM)
           nss0 = -8388608.f * ss0; nzs0 = -8388608.f * zs0;
           nss1 = -8388608.f * ss1; nzs1 = -8388608.f * zs1;
         }
-        const int64_t g0s = (int64_t)(sb0 + i) * 8;  // the super-block's first 32-element group
-        auto groups = [&](auto x24c) {  // the stage's eight groups: two bytes of x, or three for 24-bit x
-          constexpr bool X24 = decltype(x24c)::value;
-  #pragma unroll
-          for (int gg = 0; gg < 8; ++gg) {
-            uint32_t e0, e1, o0, o1;  // A: even-k and odd-k codes of rows r0, r1 (x16 for nibbles)
-            if constexpr (FMT == FMT_INT4 || BITS == 4) {
-              const uint32_t coff = (((uint32_t)gg ^ sw) << 4) + 4 * c;
-              const uint32_t w0 = lds32(stg + r0 * 128 + coff), w1 = lds32(stg + r1 * 128 + coff);
-              e0 = (w0 << 4) & 0xF0F0F0F0u; e1 = (w1 << 4) & 0xF0F0F0F0u;
-              o0 = w0 & 0xF0F0F0F0u; o1 = w1 & 0xF0F0F0F0u;
-            } else if constexpr (BITS == 2) {
-              // 2-bit: slice gg is 8 B of the 64-byte row (64-byte swizzle: 16-byte chunk ^ (row / 2) % 4);
-              // lane c takes the half-word of k = 8c .. 8c + 7, spreads its nibbles to bytes (one byte
-              // permute, one shift-or) and splits even and odd k with two masks
-              const uint32_t off = ((((uint32_t)gg >> 1) ^ (((uint32_t)r0 >> 1) & 3u)) << 4) + 8 * (gg & 1) + 4 * (c >> 1);
-              const uint32_t sel = (c & 1) ? 0x4342u : 0x4140u;
-              const uint32_t t0 = __byte_perm(lds32(stg + r0 * 64 + off), 0u, sel);
-              const uint32_t t1 = __byte_perm(lds32(stg + r1 * 64 + off), 0u, sel);
-              const uint32_t u0 = (t0 | (t0 << 4)) & 0x0F0F0F0Fu, u1 = (t1 | (t1 << 4)) & 0x0F0F0F0Fu;
-              e0 = u0 & 0x03030303u; e1 = u1 & 0x03030303u;
-              o0 = (u0 >> 2) & 0x03030303u; o1 = (u1 >> 2) & 0x03030303u;
-            } else {  // bytes: slice gg is 32 B of box gg / 4; lane c takes bytes 8c .. 8c + 7
-              const uint32_t ch = (uint32_t)(2 * (gg & 3) + (c >> 1));
-              const uint32_t off = (uint32_t)(gg >> 2) * 8192 + ((ch ^ sw) << 4) + 8 * (c & 1);
-              const uint2 w0 = lds64(stg + r0 * 128 + off), w1 = lds64(stg + r1 * 128 + off);
-              e0 = __byte_perm(w0.x, w0.y, 0x6420); e1 = __byte_perm(w1.x, w1.y, 0x6420);
-              o0 = __byte_perm(w0.x, w0.y, 0x7531); o1 = __byte_perm(w1.x, w1.y, 0x7531);
-            }
-            const uint4 xv = lds128(stg + L::ST_X + ((gg * M + g) * 4 + c) * 16);
-            // (2^-a/16, -16 X) of tokens 2c and 2c + 1: 8-byte records, so two 8-byte loads (odd M)
-            const float2 Ga = lds64f(stg + L::ST_GSUM + (gg * M + 2 * c) * 8);
-            const float2 Gb = lds64f(stg + L::ST_GSUM + (gg * M + 2 * c + 1) * 8);
-            int32_t dh[4], dm[4], dl[4];
-            QL_IMMA0("s8", dh, acc_init, e0, e1, o0, o1, xv.x, xv.y);
-            QL_IMMA0("u8", dm, acc_init, e0, e1, o0, o1, xv.z, xv.w);
-            if constexpr (X24) {  // the low byte of 24-bit x, from global memory (L2); token g's column
-              const uint2 xl = g < M ? __ldg(xlg + ((int64_t)(g0s + gg) * M + g) * 4 + c) : make_uint2(0u, 0u);
-              QL_IMMA0("u8", dl, acc_init, e0, e1, o0, o1, xl.x, xl.y);
-            }
-            float t[4];  // T = 65536 D_hi + 256 D_mid + D_lo
-  #pragma unroll
-            for (int q = 0; q < 4; ++q)
-            {
-              t[q] = fmaf(__int_as_float(dh[q]) - GEMV_ACC0_F, 256.f, __int_as_float(dm[q]) - GEMV_ACC0_F);
-              if constexpr (X24) t[q] = fmaf(t[q], 256.f, __int_as_float(dl[q]) - GEMV_ACC0_F);
-              else t[q] *= 256.f;
-            }
-            if constexpr (FMT == FMT_INT4) {
-              const uint32_t gw0g = gw0[gg >> 1], gw1g = gw1[gg >> 1];
-              const int bsc = 2 * (gg & 1);
-              const float S0 = fmaf(byte_magic(gw0g, bsc), ss0, nss0), Z0 = fmaf(byte_magic(gw0g, bsc + 1), zs0, nzs0);
-              const float S1 = fmaf(byte_magic(gw1g, bsc), ss1, nss1), Z1 = fmaf(byte_magic(gw1g, bsc + 1), zs1, nzs1);
-              acc[0] = fmaf(S0 * Ga.x, fmaf(Z0, Ga.y, t[0]), acc[0]);
-              acc[1] = fmaf(S0 * Gb.x, fmaf(Z0, Gb.y, t[1]), acc[1]);
-              acc[2] = fmaf(S1 * Ga.x, fmaf(Z1, Ga.y, t[2]), acc[2]);
-              acc[3] = fmaf(S1 * Gb.x, fmaf(Z1, Gb.y, t[3]), acc[3]);
-            } else {
-              // slice gg lies in affine group gg * 32 / G of the super-block; its word holds (s, b) bf16
-              const uint32_t gw0g = gw0[gg * 32 / G], gw1g = gw1[gg * 32 / G];
-              constexpr float SF = BITS == 4 ? 1.f : 16.f;  // nibbles carry 16 q, 2-bit fields and bytes q
-              const float s0 = bf16_bits_to_f32(gw0g) * SF, b0 = bf16_bits_to_f32(gw0g >> 16);
-              const float s1 = bf16_bits_to_f32(gw1g) * SF, b1 = bf16_bits_to_f32(gw1g >> 16);
-              // b 2^-a X = -b (2^-a/16)(-16 X)
-              acc[0] = fmaf(s0 * Ga.x, t[0], fmaf(-b0 * Ga.x, Ga.y, acc[0]));
-              acc[1] = fmaf(s0 * Gb.x, t[1], fmaf(-b0 * Gb.x, Gb.y, acc[1]));
-              acc[2] = fmaf(s1 * Ga.x, t[2], fmaf(-b1 * Ga.x, Ga.y, acc[2]));
-              acc[3] = fmaf(s1 * Gb.x, t[3], fmaf(-b1 * Gb.x, Gb.y, acc[3]));
-            }
+        // A operand of group gg: even-k and odd-k codes of rows r0, r1 (x16 for nibbles)
+        auto codes = [&](int gg, uint32_t &e0, uint32_t &e1, uint32_t &o0, uint32_t &o1) {
+          if constexpr (FMT == FMT_INT4 || BITS == 4) {
+            const uint32_t coff = (((uint32_t)gg ^ sw) << 4) + 4 * c;
+            const uint32_t w0 = lds32(stg + r0 * 128 + coff), w1 = lds32(stg + r1 * 128 + coff);
+            e0 = (w0 << 4) & 0xF0F0F0F0u; e1 = (w1 << 4) & 0xF0F0F0F0u;
+            o0 = w0 & 0xF0F0F0F0u; o1 = w1 & 0xF0F0F0F0u;
+          } else if constexpr (BITS == 2) {
+            // 2-bit: slice gg is 8 B of the 64-byte row (64-byte swizzle: 16-byte chunk ^ (row / 2) % 4);
+            // lane c takes the half-word of k = 8c .. 8c + 7, spreads its nibbles to bytes (one byte
+            // permute, one shift-or) and splits even and odd k with two masks
+            const uint32_t off = ((((uint32_t)gg >> 1) ^ (((uint32_t)r0 >> 1) & 3u)) << 4) + 8 * (gg & 1) + 4 * (c >> 1);
+            const uint32_t sel = (c & 1) ? 0x4342u : 0x4140u;
+            const uint32_t t0 = __byte_perm(lds32(stg + r0 * 64 + off), 0u, sel);
+            const uint32_t t1 = __byte_perm(lds32(stg + r1 * 64 + off), 0u, sel);
+            const uint32_t u0 = (t0 | (t0 << 4)) & 0x0F0F0F0Fu, u1 = (t1 | (t1 << 4)) & 0x0F0F0F0Fu;
+            e0 = u0 & 0x03030303u; e1 = u1 & 0x03030303u;
+            o0 = (u0 >> 2) & 0x03030303u; o1 = (u1 >> 2) & 0x03030303u;
+          } else {  // bytes: slice gg is 32 B of box gg / 4; lane c takes bytes 8c .. 8c + 7
+            const uint32_t ch = (uint32_t)(2 * (gg & 3) + (c >> 1));
+            const uint32_t off = (uint32_t)(gg >> 2) * 8192 + ((ch ^ sw) << 4) + 8 * (c & 1);
+            const uint2 w0 = lds64(stg + r0 * 128 + off), w1 = lds64(stg + r1 * 128 + off);
+            e0 = __byte_perm(w0.x, w0.y, 0x6420); e1 = __byte_perm(w1.x, w1.y, 0x6420);
+            o0 = __byte_perm(w0.x, w0.y, 0x7531); o1 = __byte_perm(w1.x, w1.y, 0x7531);
           }
         };
-        if (x24) groups(std::true_type{});
-        else groups(std::false_type{});
+        // the weight scale of group gg for rows r0, r1 (int4: S = sc * ss; affine: s, times 16 when the
+        // codes enter the MMA as q rather than 16 q)
+        constexpr float SF = (FMT == FMT_INT4 || BITS == 4) ? 1.f : 16.f;
+#pragma unroll
+        for (int gg = 0; gg < 8; ++gg) {
+          uint32_t e0, e1, o0, o1;
+          codes(gg, e0, e1, o0, o1);
+          const uint4 xv = lds128(stg + L::ST_X + ((gg * M + g) * 4 + c) * 16);
+          // (G_x, G_y) of tokens 2c and 2c + 1: 8-byte records, so two 8-byte loads (odd M)
+          const float2 Ga = lds64f(stg + L::ST_GSUM + (gg * M + 2 * c) * 8);
+          const float2 Gb = lds64f(stg + L::ST_GSUM + (gg * M + 2 * c + 1) * 8);
+          if (gg == 0) x24s |= __float_as_uint(Ga.x) | __float_as_uint(Gb.x);  // zero for tokens past M
+          const float gax = Ga.x, gbx = Gb.x;
+          int32_t dh[4], dm[4];
+          QL_IMMA0("s8", dh, acc_init, e0, e1, o0, o1, xv.x, xv.y);
+          QL_IMMA0("u8", dm, acc_init, e0, e1, o0, o1, xv.z, xv.w);
+          float t[4];  // T = 256 D_hi + D_mid
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            t[q] = fmaf(__int_as_float(dh[q]) - GEMV_ACC0_F, 256.f, __int_as_float(dm[q]) - GEMV_ACC0_F);
+          if constexpr (FMT == FMT_INT4) {
+            const uint32_t gw0g = gw0[gg >> 1], gw1g = gw1[gg >> 1];
+            const int bsc = 2 * (gg & 1);
+            const float S0 = fmaf(byte_magic(gw0g, bsc), ss0, nss0), Z0 = fmaf(byte_magic(gw0g, bsc + 1), zs0, nzs0);
+            const float S1 = fmaf(byte_magic(gw1g, bsc), ss1, nss1), Z1 = fmaf(byte_magic(gw1g, bsc + 1), zs1, nzs1);
+            acc[0] = fmaf(S0 * gax, fmaf(Z0, Ga.y, t[0]), acc[0]);
+            acc[1] = fmaf(S0 * gbx, fmaf(Z0, Gb.y, t[1]), acc[1]);
+            acc[2] = fmaf(S1 * gax, fmaf(Z1, Ga.y, t[2]), acc[2]);
+            acc[3] = fmaf(S1 * gbx, fmaf(Z1, Gb.y, t[3]), acc[3]);
+          } else {
+            // slice gg lies in affine group gg * 32 / G of the super-block; its word holds (s, b) bf16
+            const uint32_t gw0g = gw0[gg * 32 / G], gw1g = gw1[gg * 32 / G];
+            const float s0 = bf16_bits_to_f32(gw0g) * SF, b0 = bf16_bits_to_f32(gw0g >> 16);
+            const float s1 = bf16_bits_to_f32(gw1g) * SF, b1 = bf16_bits_to_f32(gw1g >> 16);
+            // b 2^-a X = -b G_x G_y
+            acc[0] = fmaf(s0 * gax, t[0], fmaf(-b0 * gax, Ga.y, acc[0]));
+            acc[1] = fmaf(s0 * gbx, t[1], fmaf(-b0 * gbx, Gb.y, acc[1]));
+            acc[2] = fmaf(s1 * gax, t[2], fmaf(-b1 * gax, Ga.y, acc[2]));
+            acc[3] = fmaf(s1 * gbx, t[3], fmaf(-b1 * gbx, Gb.y, acc[3]));
+          }
+        }
         __syncwarp();
         if (lane == 0) mbar_arrive(bar_empty(s));
       }
     }
     // publish: rows n0, n1 x tokens 2c, 2c + 1
     const int tk0 = 2 * c, tk1 = 2 * c + 1;
+    if (__any_sync(0xffffffffu, (x24s & 1u) != 0u) && ok) {  // rare
+      const float4 lb = gemv_mt_low_bytes<FMT, BITS, G>(p.codes, p.gmeta, c0, c1, st0, st1, p.ws.flags, p.ws.gsum,
+                                                        xlg, p.K, M, sb0, nsb);
+      acc[0] += lb.x;
+      acc[1] += lb.y;
+      acc[2] += lb.z;
+      acc[3] += lb.w;
+    }
     if (ok) {
       if (P == 1) {
         if (n0 < p.N) {
@@ -979,6 +1133,20 @@ __global__ void __launch_bounds__(GEMV_MT_THREADS, GEMV_MT_CTAS_PER_SM)
       }
     }
   }
+}
+
+// The kernels: the same body under the register budget of each format (see gemv_mt_ctas_per_sm).
+__global__ void __launch_bounds__(GEMV_MT_THREADS, GEMV_MT_CTAS_PER_SM)
+    gemv_mt_int4_kernel(const __grid_constant__ CUtensorMap map_codes, const __grid_constant__ CUtensorMap map_gmeta,
+                        GemvMtParams p) {
+  gemv_mt_body<FMT_INT4, 4, 32>(map_codes, map_gmeta, p);
+}
+
+template <int BITS, int G>
+__global__ void __maxnreg__(GEMV_MT_AFFINE_NREG)
+    gemv_mt_affine_kernel(const __grid_constant__ CUtensorMap map_codes, const __grid_constant__ CUtensorMap map_gmeta,
+                          GemvMtParams p) {
+  gemv_mt_body<FMT_AFFINE, BITS, G>(map_codes, map_gmeta, p);
 }
 
 }  // namespace ql

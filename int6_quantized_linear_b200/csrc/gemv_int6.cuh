@@ -21,12 +21,14 @@
 // super-block whose 16-bit form would lose too much (as in the int4 kernels),
 // 24-bit (max |x_int| in [2^22, 2^23): exact for every bf16 element within 2^15
 // of the group's largest magnitude), split into a signed high and unsigned
-// middle and low bytes, one MMA each (the low byte only for 24-bit); per (row,
-// group) the sums are exact below 2^19, so the accumulators start at the bits of
-// 1.5 * 2^23 and read back with one subtraction:
-//     T = 65536 D_hi + 256 D_mid + D_lo = 4 * 2^u * sum_k q_k x_int_k,
-//     y += S (2^-a / (4 * 2^u)) T,   u = 0 (24-bit) or 8 (16-bit)
-// with S = code * step (exact in fp32).
+// middle and low bytes, one MMA each; per (row, group) the sums are exact below
+// 2^19, so the accumulators start at the bits of 1.5 * 2^23 and read back with
+// one subtraction.  The streaming loop runs the high and middle bytes:
+//     T = 256 D_hi + D_mid,   y += S G T
+// with S = code * step (exact in fp32) and G = 2^-a / 4 for 16-bit x (the whole
+// product).  For 24-bit x, G = 2^8 * 2^-a / 4 carries the 24-bit marker
+// (mark_24bit) and an out-of-line pass after the loop adds S G 2^-8 D_lo for
+// the marked super-blocks (gemv_int6_low_bytes).
 //
 // A CTA is a producer warp and four consumer warps on 64 weight rows and a
 // range of super-blocks.  A stage holds the codes box (64 rows x 208 bytes: the
@@ -82,23 +84,24 @@ QL_DEVI void int6p_a_words(uint32_t l0, uint32_t l1, uint32_t h, uint32_t (&a)[4
 }
 
 // x preparation: one thread per (token, 16-element group), so a half-warp holds one token's 16 groups
-// of a super-block (16- or 24-bit as in the int4 kernels; the flag byte [sb][m] says which).  Entry
+// of a super-block (16- or 24-bit as in the int4 kernels; flag byte [sb][m] and the scale's marker say which).  Entry
 // (sb, m, set, j, gi) of the x words
 // is the B pairs of k-step j for group 8 set + gi: (hi, 0, mid, 0) for gi < 4 (its lane feeds b0),
 // (0, hi, 0, mid) for gi >= 4 (b1), and (lo, 0) or (0, lo) in the low-byte region that follows the
-// K/256 * M * 1024 bytes of the first; the group scale 2^-a / 4 goes to gscale[sb][m][16].
+// K/256 * M * 1024 bytes of the first (24-bit x only); the group scale goes to gscale[sb][m][16].
 // Also zeroes the first n_counters row-group counters.
 template <bool PLANAR>
 __global__ void __launch_bounds__(256) gemv_xprep_int6_kernel(const __nv_bfloat16 *x, int64_t M, int64_t K,
                                                               int64_t n_counters, GemvWorkspace ws) {
   pdl_launch_dependents();  // the streaming kernel may start fetching weights now
-  pdl_wait();               // x (and this workspace) may belong to the kernel launched before this one
   const int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-  if (t < n_counters) ws.counters[t] = 0;
   const int64_t ng = K / 16;
   const bool live = t < M * ng;  // every lane takes part in the ballot below
   const int64_t m = live ? t / ng : 0, gg = live ? t - m * ng : 0;
   const uint4 *src = reinterpret_cast<const uint4 *>(x + m * K + 16 * gg);
+  if (live) prefetch_l2(src);
+  pdl_wait();               // x (and this workspace) may belong to the kernel launched before this one
+  if (t < n_counters) ws.counters[t] = 0;
   uint4 v0 = make_uint4(0u, 0u, 0u, 0u), v1 = v0;
   if (live) {
     v0 = __ldg(src);
@@ -147,13 +150,15 @@ __global__ void __launch_bounds__(256) gemv_xprep_int6_kernel(const __nv_bfloat1
       const int v = xi[int6_kperm<PLANAR>(j, b)];
       hi |= ((uint32_t)(v >> hs) & 0xffu) << (8 * b);
       mid |= ((uint32_t)(v >> (hs - 8)) & 0xffu) << (8 * b);
-      lo |= (sb24 ? ((uint32_t)v & 0xffu) : 0u) << (8 * b);
+      lo |= ((uint32_t)v & 0xffu) << (8 * b);
     }
     dst[8 * j] = gi < 4 ? make_uint4(hi, 0u, mid, 0u) : make_uint4(0u, hi, 0u, mid);
-    dst8[8 * j] = gi < 4 ? make_uint2(lo, 0u) : make_uint2(0u, lo);
+    if (sb24) dst8[8 * j] = gi < 4 ? make_uint2(lo, 0u) : make_uint2(0u, lo);
   }
-  // the group scale 2^-a / (4 * 2^u), u = 0 (24-bit) or 8 (16-bit): T below is 4 * 2^u * sum q x_int
-  reinterpret_cast<float *>(ws.gsum)[(sb * M + m) * 16 + gl] = exp2i(-a) * (sb24 ? 0.25f : 0.25f / 256.f);
+  // the group scale 2^-a / 4, times 2^8 for 24-bit x (whose T = 256 D_hi + D_mid is then 2^-8 of
+  // 4 sum q x_int, less the low byte's 2^-8 D_lo) and then carrying the 24-bit marker (mark_24bit)
+  const float gsc = exp2i(-a) * (sb24 ? 64.f : 0.25f);
+  reinterpret_cast<float *>(ws.gsum)[(sb * M + m) * 16 + gl] = sb24 ? mark_24bit(gsc) : gsc;
   if (gl == 0) ws.flags[sb * 16 + m] = sb24 ? 1 : 0;
 }
 
@@ -174,16 +179,14 @@ constexpr int GEMV6_CTAS_PER_SM = 3;
 constexpr int GEMV6_CODE_ROW = 208;  // bytes per row in a stage: 192 of the super-block + 16 of the next
 
 // Stage layout for up to TM tokens: codes [64][208], scale codes [64][16], group scales [TM][16] f32,
-// (hi, mid) x words [TM][2 sets][4 k-steps][8 groups][16 B] and the 24-bit flags [16 B] (a 24-bit
-// super-block's lo x words are read from global memory).  The ring is as deep (4, 3 or 2 stages) as
-// three CTAs per SM allow.
+// (hi, mid) x words [TM][2 sets][4 k-steps][8 groups][16 B] (a 24-bit super-block's lo x words are
+// read from global memory).  The ring is as deep (4, 3 or 2 stages) as three CTAs per SM allow.
 template <int TM>
 struct Int6Layout {
   static constexpr int ST_SC = 64 * GEMV6_CODE_ROW;
   static constexpr int ST_G = ST_SC + 64 * 16;
   static constexpr int ST_X = ST_G + TM * 64;
-  static constexpr int ST_FL = ST_X + TM * 1024;  // 16 B: a byte per token, non-zero when its x is 24-bit
-  static constexpr int STAGE = (ST_FL + 16 + 127) / 128 * 128;
+  static constexpr int STAGE = (ST_X + TM * 1024 + 127) / 128 * 128;
   static constexpr int EXTRA = 16 + 2 * 4 * 8 + 16 + 128;  // zero slot, barriers, flags, alignment
   static constexpr int RING = GEMV6_CTAS_PER_SM * (4 * STAGE + EXTRA + 1024) <= 233472   ? 4
                             : GEMV6_CTAS_PER_SM * (3 * STAGE + EXTRA + 1024) <= 233472 ? 3
@@ -192,6 +195,7 @@ struct Int6Layout {
 };
 
 struct Gemv6Params {
+  const uint8_t *codes, *sc;  // [N][3K/4], [N][K/16]: read directly only by the 24-bit tail
   const uint16_t *steps;      // fp16 [N][K/256]
   const __nv_bfloat16 *bias;  // [N] or NULL
   int64_t N, K;
@@ -200,6 +204,86 @@ struct Gemv6Params {
   GemvWorkspace ws;
   __nv_bfloat16 *y;
 };
+
+// The low bytes of 24-bit x for one consumer warp of the int6 kernel: S G 2^-8 D_lo per (row, token,
+// 16-weight group) of every super-block of the range [sb0, sb0 + nsb) in which some token's x is
+// 24-bit, the weights read again from global memory (rows c0, c1; rows past N read row N - 1 and their
+// sums are never stored).  Flagged super-blocks are rare, so this runs out of line and leaves the
+// streaming loop's registers alone.  Returns the sums to add per (token, row r0 | r1).
+template <int TM>
+struct Int6LowBytes {
+  float v[TM][2];
+};
+
+template <int TM, bool PLANAR>
+__device__ __noinline__ Int6LowBytes<TM> gemv_int6_low_bytes(const uint8_t *codes, const uint8_t *sc, int64_t c0,
+                                                             int64_t c1, const uint16_t *st0, const uint16_t *st1,
+                                                             const uint8_t *flags, const float *gscale,
+                                                             const uint2 *xlg, int64_t K, int M, int sb0, int nsb) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
+  const bool on = (g & 3) == c;  // lane (g, c) feeds x for group g of a set
+  const uint64_t fmask = M >= 8 ? ~0ull : ((1ull << (8 * M)) - 1);  // the flag bytes of tokens < M
+  const int32_t acc_init[4] = {GEMV_ACC0, GEMV_ACC0, GEMV_ACC0, GEMV_ACC0};
+  const uint8_t *q0 = codes + c0 * (K / 256) * 192, *q1 = codes + c1 * (K / 256) * 192;
+  const uint8_t *s0p = sc + c0 * (K / 16), *s1p = sc + c1 * (K / 16);
+  const int bo = 8 * ((2 * c) & 3);
+  Int6LowBytes<TM> out;
+#pragma unroll
+  for (int m = 0; m < TM; ++m) out.v[m][0] = out.v[m][1] = 0.f;
+  for (int i = 0; i < nsb; ++i) {
+    const int64_t sb = sb0 + i;
+    const uint2 fw = __ldg(reinterpret_cast<const uint2 *>(flags + sb * 16));
+    const uint64_t f24 = ((uint64_t)fw.y << 32 | fw.x) & fmask;
+    if (f24 == 0) continue;  // the same for the whole warp
+    const float p0 = f16_bits_to_f32(__ldg(st0 + i)), p1 = f16_bits_to_f32(__ldg(st1 + i));
+    const uint8_t *b0 = q0 + sb * 192, *b1 = q1 + sb * 192;
+    const float *gsc = gscale + sb * M * 16;
+    const uint2 *xls = xlg + sb * M * 64;
+#pragma unroll 1
+    for (int set = 0; set < 2; ++set) {
+      uint32_t A00[4], A01[4], A10[4], A11[4];  // as in the streaming loop, from the rows in global memory
+      const int gl = 8 * set + c;
+      if constexpr (PLANAR) {
+        const uint2 l00 = __ldg(reinterpret_cast<const uint2 *>(b0 + 8 * gl)), l01 = __ldg(reinterpret_cast<const uint2 *>(b0 + 8 * gl + 32));
+        const uint2 l10 = __ldg(reinterpret_cast<const uint2 *>(b1 + 8 * gl)), l11 = __ldg(reinterpret_cast<const uint2 *>(b1 + 8 * gl + 32));
+        int6p_a_words(l00.x, l00.y, __ldg(reinterpret_cast<const uint32_t *>(b0 + 128 + 4 * gl)), A00);
+        int6p_a_words(l01.x, l01.y, __ldg(reinterpret_cast<const uint32_t *>(b0 + 144 + 4 * gl)), A01);
+        int6p_a_words(l10.x, l10.y, __ldg(reinterpret_cast<const uint32_t *>(b1 + 128 + 4 * gl)), A10);
+        int6p_a_words(l11.x, l11.y, __ldg(reinterpret_cast<const uint32_t *>(b1 + 144 + 4 * gl)), A11);
+      } else {
+        const uint32_t *w0 = reinterpret_cast<const uint32_t *>(b0 + 12 * gl);
+        const uint32_t *w1 = reinterpret_cast<const uint32_t *>(b1 + 12 * gl);
+        int6_a_words(__ldg(w0), __ldg(w0 + 1), __ldg(w0 + 2), A00);
+        int6_a_words(__ldg(w0 + 12), __ldg(w0 + 13), __ldg(w0 + 14), A01);
+        int6_a_words(__ldg(w1), __ldg(w1 + 1), __ldg(w1 + 2), A10);
+        int6_a_words(__ldg(w1 + 12), __ldg(w1 + 13), __ldg(w1 + 14), A11);
+      }
+      const uint32_t sw0 = __ldg(reinterpret_cast<const uint32_t *>(s0p + sb * 16 + 8 * set + 4 * (c >> 1)));
+      const uint32_t sw1 = __ldg(reinterpret_cast<const uint32_t *>(s1p + sb * 16 + 8 * set + 4 * (c >> 1)));
+      const float S00 = __fmul_rn((float)(int8_t)(sw0 >> bo), p0), S01 = __fmul_rn((float)(int8_t)(sw0 >> (bo + 8)), p0);
+      const float S10 = __fmul_rn((float)(int8_t)(sw1 >> bo), p1), S11 = __fmul_rn((float)(int8_t)(sw1 >> (bo + 8)), p1);
+#pragma unroll
+      for (int m = 0; m < TM; ++m) {
+        if (m < M && ((f24 >> (8 * m)) & 0xffu) != 0) {  // the same for the warp
+          int32_t dl[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint2 xl = on ? __ldg(xls + ((m * 2 + set) * 4 + j) * 8 + g) : make_uint2(0u, 0u);
+            if (j == 0) QL_IMMA6_0("u8", dl, acc_init, A00[0], A10[0], A01[0], A11[0], xl.x, xl.y);
+            else QL_IMMA6("u8", dl, A00[j], A10[j], A01[j], A11[j], xl.x, xl.y);
+          }
+          const float2 G = __ldg(reinterpret_cast<const float2 *>(gsc + m * 16 + 8 * set + 2 * c));
+          const float gx = unmark(G.x) * (1.f / 256.f), gy = unmark(G.y) * (1.f / 256.f);
+          out.v[m][0] = fmaf(S00 * gx, __int_as_float(dl[0]) - GEMV_ACC0_F, out.v[m][0]);
+          out.v[m][0] = fmaf(S01 * gy, __int_as_float(dl[1]) - GEMV_ACC0_F, out.v[m][0]);
+          out.v[m][1] = fmaf(S10 * gx, __int_as_float(dl[2]) - GEMV_ACC0_F, out.v[m][1]);
+          out.v[m][1] = fmaf(S11 * gy, __int_as_float(dl[3]) - GEMV_ACC0_F, out.v[m][1]);
+        }
+      }
+    }
+  }
+  return out;
+}
 
 template <int TM, bool PLANAR>
 __global__ void __launch_bounds__(GEMV6_THREADS, GEMV6_CTAS_PER_SM)
@@ -233,6 +317,12 @@ __global__ void __launch_bounds__(GEMV6_THREADS, GEMV6_CTAS_PER_SM)
     flags[1] = 0;
     fence_mbar_init();
   }
+  // the group scales of tokens M..TM-1 in every stage: never written by the copies, read (and their
+  // sums dropped) for odd M; zero, so they carry no 24-bit marker
+  if (threadIdx.x < (TM - M) * 16) {
+#pragma unroll
+    for (int s = 0; s < RING; ++s) reinterpret_cast<uint32_t *>(smem + s * L::STAGE + L::ST_G + M * 64)[threadIdx.x] = 0u;
+  }
   __syncthreads();
   pdl_launch_dependents();  // the next call's preparation pass waits for this grid before touching anything
 
@@ -240,7 +330,7 @@ __global__ void __launch_bounds__(GEMV6_THREADS, GEMV6_CTAS_PER_SM)
     if (lane == 0) {
       tma_prefetch_desc(&map_codes);
       tma_prefetch_desc(&map_sc);
-      const uint32_t tx = (uint32_t)L::ST_G + (uint32_t)M * (64 + 1024) + 16;
+      const uint32_t tx = (uint32_t)L::ST_G + (uint32_t)M * (64 + 1024);
       const float *gscale = reinterpret_cast<const float *>(p.ws.gsum);
       auto issue_w = [&](int i, int s) {
         const uint32_t st = sbase + s * L::STAGE;
@@ -253,10 +343,9 @@ __global__ void __launch_bounds__(GEMV6_THREADS, GEMV6_CTAS_PER_SM)
         const int64_t sb = sb0 + i;
         bulk_load(st + L::ST_G, gscale + sb * M * 16, (uint32_t)M * 64, bar_full(s));
         bulk_load(st + L::ST_X, p.ws.xq + sb * M * 64, (uint32_t)M * 1024, bar_full(s));
-        bulk_load(st + L::ST_FL, p.ws.flags + sb * 16, 16, bar_full(s));
       };
-      const bool hold = copies_withheld();
-      const int pre = hold ? 0 : (nsb < RING ? nsb : RING);
+      const int nis = copies_withheld() ? 0 : nsb;  // super-blocks whose copies are started
+      const int pre = nis < RING ? nis : RING;
       for (int i = 0; i < pre; ++i) issue_w(i, i);  // weights need no x
       pdl_wait();
       for (int i = 0; i < pre; ++i) issue_x(i, i);
@@ -264,7 +353,7 @@ __global__ void __launch_bounds__(GEMV6_THREADS, GEMV6_CTAS_PER_SM)
       uint32_t ph = 0;
       bool ok = true;
       int i = pre;
-      for (; i < nsb && !hold; ++i) {  // unit i reuses the stage of unit i - RING
+      for (; i < nis; ++i) {  // unit i reuses the stage of unit i - RING
         if (!mbar_wait_bounded(bar_empty(s), ph, abort_flag)) {
           ok = false;
           break;
@@ -309,6 +398,7 @@ __global__ void __launch_bounds__(GEMV6_THREADS, GEMV6_CTAS_PER_SM)
     float acc[TM][2];  // (token) x (row r0 | r1)
 #pragma unroll
     for (int m = 0; m < TM; ++m) acc[m][0] = acc[m][1] = 0.f;
+    uint32_t x24s = 0u;  // bit 0: some super-block's group scale carries the 24-bit marker
     bool ok = true;
     for (int base = 0; base < nsb && ok; base += RING) {
       const uint32_t par = (uint32_t)((base / RING) & 1);
@@ -326,12 +416,6 @@ __global__ void __launch_bounds__(GEMV6_THREADS, GEMV6_CTAS_PER_SM)
           break;
         }
         const uint32_t stg = sbase + s * L::STAGE;
-        bool x24;  // some token's x of this super-block is 24-bit: the low-byte MMA runs (the same for the warp)
-        {
-          const uint2 fw = lds64(stg + L::ST_FL);
-          const uint64_t f = ((uint64_t)fw.y << 32 | fw.x) & (M >= 8 ? ~0ull : ((1ull << (8 * M)) - 1));
-          x24 = f != 0;
-        }
         const float stp0 = f16_bits_to_f32(sr0[s]), stp1 = f16_bits_to_f32(sr1[s]);
         // scale codes of the D columns: groups 8 set + 2c, 8 set + 2c + 1 of rows r0, r1
         const uint32_t scw00 = lds32(stg + L::ST_SC + r0 * 16 + 4 * (c >> 1));
@@ -347,85 +431,82 @@ __global__ void __launch_bounds__(GEMV6_THREADS, GEMV6_CTAS_PER_SM)
           S[0][1][h] = __fmul_rn((float)(int8_t)(scw10 >> (bo + 8 * h)), stp1);
           S[1][1][h] = __fmul_rn((float)(int8_t)(scw11 >> (bo + 8 * h)), stp1);
         }
-        const int64_t sbw = (int64_t)(sb0 + i) * M * 64;  // the super-block's lo x words, in uint2
-        auto sets = [&](auto x24c) {  // the stage's two 8-group sets: two bytes of x, or three for 24-bit x
-          constexpr bool X24 = decltype(x24c)::value;
-  #pragma unroll
-          for (int set = 0; set < 2; ++set) {
-            // A: groups 8 set + c (slots 4c ..) and 8 set + c + 4 (slots 16 + 4c ..) of rows r0, r1
-            uint32_t A00[4], A01[4], A10[4], A11[4];  // [row][group half]
-            if constexpr (PLANAR) {  // group gg: low plane bytes 8 gg .., high plane bytes 128 + 4 gg ..
-              const uint32_t gl = 8 * set + c;
-              const uint32_t a0 = stg + r0 * GEMV6_CODE_ROW, a1 = stg + r1 * GEMV6_CODE_ROW;
-              const uint2 l00 = lds64(a0 + 8 * gl), l01 = lds64(a0 + 8 * gl + 32);
-              const uint2 l10 = lds64(a1 + 8 * gl), l11 = lds64(a1 + 8 * gl + 32);
-              int6p_a_words(l00.x, l00.y, lds32(a0 + 128 + 4 * gl), A00);
-              int6p_a_words(l01.x, l01.y, lds32(a0 + 144 + 4 * gl), A01);
-              int6p_a_words(l10.x, l10.y, lds32(a1 + 128 + 4 * gl), A10);
-              int6p_a_words(l11.x, l11.y, lds32(a1 + 144 + 4 * gl), A11);
-            } else {
-              const uint32_t o = stg + 12 * (8 * set + c);
-              const uint32_t a0 = o + r0 * GEMV6_CODE_ROW, a1 = o + r1 * GEMV6_CODE_ROW;
-              int6_a_words(lds32(a0), lds32(a0 + 4), lds32(a0 + 8), A00);
-              int6_a_words(lds32(a0 + 48), lds32(a0 + 52), lds32(a0 + 56), A01);
-              int6_a_words(lds32(a1), lds32(a1 + 4), lds32(a1 + 8), A10);
-              int6_a_words(lds32(a1 + 48), lds32(a1 + 52), lds32(a1 + 56), A11);
-            }
-            // up to four tokens at a time: eight independent accumulator chains (hi / lo) per k-step
-  #pragma unroll
-            for (int m0 = 0; m0 < TM; m0 += MP) {
-              if (m0 < M) {
-                int32_t dh[MP][4], dm[MP][4], dl[MP][4];
-  #pragma unroll
-                for (int mm = 0; mm < MP; ++mm)
-  #pragma unroll
-                  for (int q = 0; q < 4; ++q) dl[mm][q] = GEMV_ACC0;
-  #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-  #pragma unroll
-                  for (int mm = 0; mm < MP; ++mm) {
-                    const int m = m0 + mm;  // a token past M (odd M) reads stale stage words; its sums are never stored
-                    const uint32_t xrow = stg + L::ST_X + ((m * 2 + set) * 4 + j) * 128 + 16 * g;
-                    const uint4 xv = lds128(on ? xrow : zero_a);
-                    if (j == 0) {
-                      QL_IMMA6_0("s8", dh[mm], acc_init, A00[0], A10[0], A01[0], A11[0], xv.x, xv.y);
-                      QL_IMMA6_0("u8", dm[mm], acc_init, A00[0], A10[0], A01[0], A11[0], xv.z, xv.w);
-                    } else {
-                      QL_IMMA6("s8", dh[mm], A00[j], A10[j], A01[j], A11[j], xv.x, xv.y);
-                      QL_IMMA6("u8", dm[mm], A00[j], A10[j], A01[j], A11[j], xv.z, xv.w);
-                    }
-                    if constexpr (X24) {  // the low byte of 24-bit x, from global memory (L2); feeding lanes only
-                      const uint2 xl = (on && m < M) ? __ldg(xlg + sbw + ((m * 2 + set) * 4 + j) * 8 + g)
-                                                     : make_uint2(0u, 0u);
-                      QL_IMMA6("u8", dl[mm], A00[j], A10[j], A01[j], A11[j], xl.x, xl.y);
-                    }
-                  }
-                }
-  #pragma unroll
+        // A operand of set `set`: groups 8 set + c (slots 4c ..) and 8 set + c + 4 (slots 16 + 4c ..) of
+        // rows r0, r1, as [row][group half]
+        auto a_words = [&](int set, uint32_t (&A00)[4], uint32_t (&A01)[4], uint32_t (&A10)[4], uint32_t (&A11)[4]) {
+          if constexpr (PLANAR) {  // group gg: low plane bytes 8 gg .., high plane bytes 128 + 4 gg ..
+            const uint32_t gl = 8 * set + c;
+            const uint32_t a0 = stg + r0 * GEMV6_CODE_ROW, a1 = stg + r1 * GEMV6_CODE_ROW;
+            const uint2 l00 = lds64(a0 + 8 * gl), l01 = lds64(a0 + 8 * gl + 32);
+            const uint2 l10 = lds64(a1 + 8 * gl), l11 = lds64(a1 + 8 * gl + 32);
+            int6p_a_words(l00.x, l00.y, lds32(a0 + 128 + 4 * gl), A00);
+            int6p_a_words(l01.x, l01.y, lds32(a0 + 144 + 4 * gl), A01);
+            int6p_a_words(l10.x, l10.y, lds32(a1 + 128 + 4 * gl), A10);
+            int6p_a_words(l11.x, l11.y, lds32(a1 + 144 + 4 * gl), A11);
+          } else {
+            const uint32_t o = stg + 12 * (8 * set + c);
+            const uint32_t a0 = o + r0 * GEMV6_CODE_ROW, a1 = o + r1 * GEMV6_CODE_ROW;
+            int6_a_words(lds32(a0), lds32(a0 + 4), lds32(a0 + 8), A00);
+            int6_a_words(lds32(a0 + 48), lds32(a0 + 52), lds32(a0 + 56), A01);
+            int6_a_words(lds32(a1), lds32(a1 + 4), lds32(a1 + 8), A10);
+            int6_a_words(lds32(a1 + 48), lds32(a1 + 52), lds32(a1 + 56), A11);
+          }
+        };
+#pragma unroll
+        for (int set = 0; set < 2; ++set) {
+          uint32_t A00[4], A01[4], A10[4], A11[4];
+          a_words(set, A00, A01, A10, A11);
+          // up to four tokens at a time: eight independent accumulator chains (hi / mid) per k-step
+#pragma unroll
+          for (int m0 = 0; m0 < TM; m0 += MP) {
+            if (m0 < M) {
+              int32_t dh[MP][4], dm[MP][4];
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+#pragma unroll
                 for (int mm = 0; mm < MP; ++mm) {
-                  const int m = m0 + mm;
-                  // D[q]: q = 0 (r0, group 8 set + 2c), 1 (r0, + 1), 2 (r1, 2c), 3 (r1, + 1)
-                  const float2 G = lds64f(stg + L::ST_G + (m * 16 + 8 * set + 2 * c) * 4);
-                  float t[4];  // T = 65536 D_hi + 256 D_mid + D_lo
-  #pragma unroll
-                  for (int q = 0; q < 4; ++q) {
-                    t[q] = fmaf(__int_as_float(dh[mm][q]) - GEMV_ACC0_F, 256.f, __int_as_float(dm[mm][q]) - GEMV_ACC0_F);
-                    if constexpr (X24) t[q] = fmaf(t[q], 256.f, __int_as_float(dl[mm][q]) - GEMV_ACC0_F);
-                    else t[q] *= 256.f;
+                  const int m = m0 + mm;  // a token past M (odd M) reads stale stage words; its sums are never stored
+                  const uint32_t xrow = stg + L::ST_X + ((m * 2 + set) * 4 + j) * 128 + 16 * g;
+                  const uint4 xv = lds128(on ? xrow : zero_a);
+                  if (j == 0) {
+                    QL_IMMA6_0("s8", dh[mm], acc_init, A00[0], A10[0], A01[0], A11[0], xv.x, xv.y);
+                    QL_IMMA6_0("u8", dm[mm], acc_init, A00[0], A10[0], A01[0], A11[0], xv.z, xv.w);
+                  } else {
+                    QL_IMMA6("s8", dh[mm], A00[j], A10[j], A01[j], A11[j], xv.x, xv.y);
+                    QL_IMMA6("u8", dm[mm], A00[j], A10[j], A01[j], A11[j], xv.z, xv.w);
                   }
-                  acc[m][0] = fmaf(S[set][0][0] * G.x, t[0], acc[m][0]);
-                  acc[m][0] = fmaf(S[set][0][1] * G.y, t[1], acc[m][0]);
-                  acc[m][1] = fmaf(S[set][1][0] * G.x, t[2], acc[m][1]);
-                  acc[m][1] = fmaf(S[set][1][1] * G.y, t[3], acc[m][1]);
                 }
+              }
+#pragma unroll
+              for (int mm = 0; mm < MP; ++mm) {
+                const int m = m0 + mm;
+                // D[q]: q = 0 (r0, group 8 set + 2c), 1 (r0, + 1), 2 (r1, 2c), 3 (r1, + 1)
+                const float2 G = lds64f(stg + L::ST_G + (m * 16 + 8 * set + 2 * c) * 4);
+                if (set == 0) x24s |= __float_as_uint(G.x);  // zero for tokens past M
+                float t[4];  // T = 256 D_hi + D_mid
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                  t[q] = fmaf(__int_as_float(dh[mm][q]) - GEMV_ACC0_F, 256.f, __int_as_float(dm[mm][q]) - GEMV_ACC0_F);
+                acc[m][0] = fmaf(S[set][0][0] * G.x, t[0], acc[m][0]);
+                acc[m][0] = fmaf(S[set][0][1] * G.y, t[1], acc[m][0]);
+                acc[m][1] = fmaf(S[set][1][0] * G.x, t[2], acc[m][1]);
+                acc[m][1] = fmaf(S[set][1][1] * G.y, t[3], acc[m][1]);
               }
             }
           }
-        };
-        if (x24) sets(std::true_type{});
-        else sets(std::false_type{});
+        }
         __syncwarp();
         if (lane == 0) mbar_arrive(bar_empty(s));
+      }
+    }
+    if (__any_sync(0xffffffffu, (x24s & 1u) != 0u) && ok) {  // rare
+      const Int6LowBytes<TM> lb = gemv_int6_low_bytes<TM, PLANAR>(p.codes, p.sc, c0, c1, st0, st1, p.ws.flags,
+                                                                 reinterpret_cast<const float *>(p.ws.gsum), xlg,
+                                                                 p.K, M, sb0, nsb);
+#pragma unroll
+      for (int m = 0; m < TM; ++m) {
+        acc[m][0] += lb.v[m][0];
+        acc[m][1] += lb.v[m][1];
       }
     }
     // the four lanes of a row hold its groups 2c, 2c + 1 of each set: sum them

@@ -231,13 +231,15 @@ ql_status launch_gemv_mt(const ql_desc *d, const ql_packed_const *w, const __nv_
     if (cudaLaunchKernelEx(&pc, gemv_xprep_mt_kernel, xb, M, K, TG, ws) != cudaSuccess) return cuda_failed();
   }
   GemvMtParams p;
+  p.codes = static_cast<const uint8_t *>(w->codes);
+  p.gmeta = static_cast<const uint8_t *>(w->gmeta);
   p.steps = static_cast<const uint8_t *>(w->steps);
   p.bias = bb;
   p.N = N;
   p.K = K;
   p.M = (int)M;
   // split K over P CTAs per 64-row group while the row groups alone leave a wave unfilled
-  int64_t P = std::max<int64_t>(1, std::min<int64_t>(NS, (int64_t)sms * GEMV_MT_CTAS_PER_SM / TG));
+  int64_t P = std::max<int64_t>(1, std::min<int64_t>(NS, (int64_t)sms * gemv_mt_ctas_per_sm<FMT>() / TG));
   P = std::min<int64_t>(P, std::max<int64_t>(1, GEMV_MT_MAX_CTAS / TG));
   if (P > 1 && TG * P > GEMV_MT_MAX_CTAS) return QL_ERR_RANGE;  // partial sums only exist for P > 1
   p.P = (int)P;
@@ -251,7 +253,10 @@ ql_status launch_gemv_mt(const ql_desc *d, const ql_packed_const *w, const __nv_
       !encode_2d(&mg, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->gmeta, meta_row, (uint64_t)N, meta_row, L::META_ROW, 64,
                  CU_TENSOR_MAP_SWIZZLE_NONE))
     return cuda_failed();
-  auto kern = gemv_mt_kernel<FMT, BITS, G>;
+  auto kern = [] {
+    if constexpr (FMT == FMT_INT4) return gemv_mt_int4_kernel;
+    else return gemv_mt_affine_kernel<BITS, G>;
+  }();
   static thread_local int configured_dev = -1;  // per instantiation and thread
   int dev = 0;
   cudaGetDevice(&dev);
@@ -298,6 +303,8 @@ ql_status launch_gemv_int6(const ql_desc *d, const ql_packed_const *w, const __n
       return cuda_failed();
   }
   Gemv6Params p;
+  p.codes = static_cast<const uint8_t *>(w->codes);
+  p.sc = static_cast<const uint8_t *>(w->gmeta);
   p.steps = static_cast<const uint16_t *>(w->steps);
   p.bias = bb;
   p.N = N;
@@ -380,6 +387,8 @@ ql_status launch_gemv(const ql_desc *d, const ql_packed_const *w, const void *x,
           return cuda_failed();
       }
       GemvTcParams p;
+      p.codes = static_cast<const uint8_t *>(w->codes);
+      p.gmeta = static_cast<const uint8_t *>(w->gmeta);
       p.steps = static_cast<const uint8_t *>(w->steps);
       p.bias = bb;
       p.N = d->N;
@@ -787,12 +796,9 @@ ql_status qlinear_quantize_meta(const ql_desc *d, const float *scale, const floa
   return launched();
 }
 
-ql_status qlinear_set_wait_limit(int64_t cycles, int32_t withhold_copies) {
-  const long long v = cycles > 0 ? (long long)cycles : QL_WAIT_LIMIT_CYCLES;
-  const int h = withhold_copies ? 1 : 0;
-  if (cudaMemcpyToSymbol(g_ql_wait_limit, &v, sizeof v) != cudaSuccess ||
-      cudaMemcpyToSymbol(g_ql_withhold, &h, sizeof h) != cudaSuccess)
-    return cuda_failed();
+ql_status qlinear_set_withhold_copies(int32_t on) {
+  const int h = on ? 1 : 0;
+  if (cudaMemcpyToSymbol(g_ql_withhold, &h, sizeof h) != cudaSuccess) return cuda_failed();
   return QL_OK;
 }
 
