@@ -39,8 +39,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM bytes per GEMV launch from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum),
 # valid only while the GEMV source is unchanged (hash of csrc/gemv.cuh at capture time).
-NCU_TRAFFIC = {"gemv_src_sha256": "ae072c352b994a98ad5c91b47f7f268d7cab37c4c3f7e62bffbb3aed4b0a0f9c",
-               "bytes_per_launch": 83054464}  # mean over the two decode layers
+NCU_TRAFFIC = {"gemv_src_sha256": "b294c01463628313d5d4a869b847dc5dcf4046f6a1201c3396eed4cc0e6426d0",
+               "bytes_per_launch": 83361664}  # mean over the two decode layers
 
 
 def parse_args(argv=None):
