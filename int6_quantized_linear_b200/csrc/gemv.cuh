@@ -111,6 +111,46 @@ __global__ void __launch_bounds__(256) gemv_simple_kernel(WeightPtrs p, int64_t 
 
 constexpr int GEMV_MT_MAX_CTAS = 4096;  // bound on the CTAs of one multi-token launch (sizes its partial sums)
 
+// The split of K over parts (warps of the M = 1 kernel, CTAs of the others): units -- 16-row tiles or
+// 64-row groups -- 0 .. extra - 1 take P + 1 parts and the rest P, so that units x parts can match
+// the resident slots exactly and no SM idles while the others stream.  Part w of the grid belongs to
+// unit `unit`, is its part `part` of `pu`, and the unit's parts start at grid index `first`.
+struct SplitK {
+  int P, extra;
+  __host__ __device__ int64_t total(int64_t units) const { return units * P + extra; }
+  // 32-bit arithmetic: a grid has fewer than 2^31 parts
+  __host__ __device__ void locate(int w, int64_t &unit, int &part, int &pu, int64_t &first) const {
+    const int big = extra * (P + 1);
+    int u, f;
+    if (w < big) {
+      u = w / (P + 1);
+      pu = P + 1;
+      f = u * pu;
+    } else {
+      const int q = (w - big) / P;
+      u = extra + q;
+      pu = P;
+      f = big + q * P;
+    }
+    part = w - f;
+    unit = u;
+    first = f;
+  }
+};
+
+// P = slots / units parts per unit (at least 1, at most NS, the super-blocks of K).  With fill, when
+// the units alone nearly fill the slots (P = 1), the leftover slots take the second halves of as many
+// units (measured: the int4 multi-token and int6 kernels at 432 row groups of 444 slots gain 3-4 %);
+// when K is already split, or without fill, the parts stay even (uneven parts measured slower there:
+// the unsplit CTAs remain the critical path and the split adds its partial sums).
+inline SplitK split_k(int64_t units, int64_t slots, int64_t NS, bool fill) {
+  SplitK s;
+  const int64_t P = std::max<int64_t>(1, std::min<int64_t>(NS, slots / units));
+  s.P = (int)P;
+  s.extra = fill && P == 1 && NS > 1 ? (int)std::max<int64_t>(0, std::min<int64_t>(units, slots - units)) : 0;
+  return s;
+}
+
 // M = 1 x block per super-block: 8 x (G_x, G_y) (64 B) and the (hi, mid) x words (1 KB) -- the part
 // a stage copies -- then the lo x words (512 B), written and read only for a 24-bit super-block
 constexpr int GEMV_XBLOB = 1600, GEMV_XCOPY = 1088, GEMV_XB_Q = 64, GEMV_XB_L = 1088;
@@ -351,7 +391,7 @@ struct GemvTcParams {
   const uint8_t *steps;
   const __nv_bfloat16 *bias;  // [N] or NULL
   int64_t N, K;
-  int parts;  // warps splitting K for one tile (1 .. K/256); warp w of the grid takes part w % parts of tile w / parts
+  SplitK split;  // of K over the warps of the grid, per 16-row tile
   GemvWorkspace ws;
   __nv_bfloat16 *y;
 };
@@ -426,13 +466,12 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS, GEMV_CTAS_PER_SM)
   uint64_t *bars = reinterpret_cast<uint64_t *>(zero_blk + GEMV_ZERO_BYTES);
   __shared__ int abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int P = p.parts;
   const int64_t n_tiles = (p.N + 15) / 16;
-  const int64_t wid = (int64_t)blockIdx.x * GEMV_WARPS + warp;
-  const int64_t tile = wid / P;
-  const int part = (int)(wid - tile * P);
+  int64_t tile, first;
+  int part, P;  // this warp is part `part` of the P splitting its tile's K
+  p.split.locate((int)blockIdx.x * GEMV_WARPS + warp, tile, part, P, first);
   const int g = lane >> 2, c = lane & 3;
-  const bool active = tile < n_tiles;
+  const bool active = tile < n_tiles;  // warps past the split's total have none
   const int NS = (int)(p.K / 256);
   const int sb0 = active ? part * NS / P : 0, nsb = active ? (part + 1) * NS / P - sb0 : 0;
   const uint32_t ring = smem_u32(smem + warp * GEMV_RING * GEMV_STAGE_BYTES);
@@ -610,7 +649,7 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS, GEMV_CTAS_PER_SM)
   }
   // K split over warps of (possibly) different CTAs: publish this part's sums; the warp that
   // finishes the tile last adds the P parts in part order, so the result does not depend on timing
-  float *part_sums = p.ws.partial + tile * P * 16;
+  float *part_sums = p.ws.partial + first * 16;
   {  // lane r < 16 stores the sum of tile row r (held by lane 4g with pg(g) = r mod 8)
     const int rr = lane & 15, prow = rr & 7;
     const int src = 4 * (((prow & 3) << 1) | (prow >> 2));
@@ -774,7 +813,7 @@ struct GemvMtParams {
   const __nv_bfloat16 *bias;  // [N] or NULL
   int64_t N, K;
   int M;  // 1 .. 8 tokens (int4: 2 .. 8)
-  int P;  // CTAs per 64-row group (K split)
+  SplitK split;  // of K over the CTAs of the grid, per 64-row group
   GemvWorkspace ws;
   __nv_bfloat16 *y;
 };
@@ -879,10 +918,11 @@ __device__ __forceinline__ void gemv_mt_body(const CUtensorMap &map_codes, const
   auto bar_full = [&](int s) { return smem_u32(bars + s); };
   auto bar_empty = [&](int s) { return smem_u32(bars + RING + s); };
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int P = p.P, M = p.M;
+  const int M = p.M;
   const int NS = (int)(p.K / 256);
-  const int64_t rg = blockIdx.x / P;  // 64-row group
-  const int part = (int)(blockIdx.x - rg * P);
+  int64_t rg, first;  // 64-row group, index of its first part
+  int part, P;        // this CTA is part `part` of the P splitting the group's K
+  p.split.locate((int)blockIdx.x, rg, part, P, first);
   const int sb0 = part * NS / P, nsb = (part + 1) * NS / P - sb0;
   if (threadIdx.x == 0) {
     for (int s = 0; s < RING; ++s) {
@@ -1123,7 +1163,7 @@ __device__ __forceinline__ void gemv_mt_body(const CUtensorMap &map_codes, const
     if (threadIdx.x == 0 && !*abort_flag) flags[1] = atomic_add_acq_rel_gpu(p.ws.counters + rg, 1) == P - 1;
     __syncthreads();  // thread 0's acquire precedes the reads of the other parts
     if (flags[1] && warp < GEMV_MT_WARPS) {
-      const float *base = p.ws.partial + (int64_t)rg * P * M * 64;
+      const float *base = p.ws.partial + first * M * 64;
       for (int e = threadIdx.x; e < M * 64; e += GEMV_MT_WARPS * 32) {
         const int tk = e >> 6, r = e & 63;
         float sum = 0.f;

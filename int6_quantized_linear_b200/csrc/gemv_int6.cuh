@@ -200,7 +200,7 @@ struct Gemv6Params {
   const __nv_bfloat16 *bias;  // [N] or NULL
   int64_t N, K;
   int M;  // 1 .. TM tokens
-  int P;  // CTAs per 64-row group (K split)
+  SplitK split;  // of K over the CTAs of the grid, per 64-row group
   GemvWorkspace ws;
   __nv_bfloat16 *y;
 };
@@ -302,10 +302,11 @@ __global__ void __launch_bounds__(GEMV6_THREADS, GEMV6_CTAS_PER_SM)
   auto bar_full = [&](int s) { return smem_u32(bars + s); };
   auto bar_empty = [&](int s) { return smem_u32(bars + RING + s); };
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int P = p.P, M = p.M;
+  const int M = p.M;
   const int NS = (int)(p.K / 256);
-  const int64_t rg = blockIdx.x / P;  // 64-row group
-  const int part = (int)(blockIdx.x - rg * P);
+  int64_t rg, first;  // 64-row group, index of its first part
+  int part, P;        // this CTA is part `part` of the P splitting the group's K
+  p.split.locate((int)blockIdx.x, rg, part, P, first);
   const int sb0 = part * NS / P, nsb = (part + 1) * NS / P - sb0;
   if (threadIdx.x < 4) reinterpret_cast<uint32_t *>(zero16)[threadIdx.x] = 0u;
   if (threadIdx.x == 0) {
@@ -539,7 +540,7 @@ __global__ void __launch_bounds__(GEMV6_THREADS, GEMV6_CTAS_PER_SM)
     if (threadIdx.x == 0 && !*abort_flag) flags[1] = atomic_add_acq_rel_gpu(p.ws.counters + rg, 1) == P - 1;
     __syncthreads();  // thread 0's acquire precedes the reads of the other parts
     if (flags[1] && warp < GEMV6_WARPS) {
-      const float *base = p.ws.partial + (int64_t)rg * P * M * 64;
+      const float *base = p.ws.partial + first * M * 64;
       for (int e = threadIdx.x; e < M * 64; e += GEMV6_WARPS * 32) {
         const int tk = e >> 6, r = e & 63;
         float sum = 0.f;

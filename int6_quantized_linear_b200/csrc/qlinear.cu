@@ -238,11 +238,10 @@ ql_status launch_gemv_mt(const ql_desc *d, const ql_packed_const *w, const __nv_
   p.N = N;
   p.K = K;
   p.M = (int)M;
-  // split K over P CTAs per 64-row group while the row groups alone leave a wave unfilled
-  int64_t P = std::max<int64_t>(1, std::min<int64_t>(NS, (int64_t)sms * gemv_mt_ctas_per_sm<FMT>() / TG));
-  P = std::min<int64_t>(P, std::max<int64_t>(1, GEMV_MT_MAX_CTAS / TG));
-  if (P > 1 && TG * P > GEMV_MT_MAX_CTAS) return QL_ERR_RANGE;  // partial sums only exist for P > 1
-  p.P = (int)P;
+  // split K over the CTAs of a 64-row group so that the groups fill one wave of resident CTAs
+  p.split = split_k(TG, (int64_t)sms * gemv_mt_ctas_per_sm<FMT>(), NS, FMT == FMT_INT4);
+  const int64_t ctas = p.split.total(TG);
+  if (p.split.P + (p.split.extra > 0) > 1 && ctas > GEMV_MT_MAX_CTAS) return QL_ERR_RANGE;  // partial sums' room
   p.ws = ws;
   p.y = yb;
   const uint64_t code_row = FMT == FMT_INT4 ? (uint64_t)K / 2 : (uint64_t)K * BITS / 8;
@@ -266,7 +265,7 @@ ql_status launch_gemv_mt(const ql_desc *d, const ql_packed_const *w, const __nv_
     configured_dev = dev;
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(TG * P));
+  cfg.gridDim = dim3((unsigned)ctas);
   cfg.blockDim = dim3(GEMV_MT_THREADS);
   cfg.dynamicSmemBytes = L::SMEM;
   cfg.stream = st;
@@ -283,22 +282,23 @@ ql_status launch_gemv_int6(const ql_desc *d, const ql_packed_const *w, const __n
   using L = Int6Layout<TM>;
   const int64_t N = d->N, K = d->K, NS = K / 256, TG = (N + 63) / 64;
   const GemvWorkspace ws = gemv_workspace_carve(workspace, M, N, K);
-  // split K over P CTAs per 64-row group while the row groups alone leave a wave unfilled
-  int64_t P = std::max<int64_t>(1, std::min<int64_t>(NS, (int64_t)sms * GEMV6_CTAS_PER_SM / TG));
-  P = std::min<int64_t>(P, std::max<int64_t>(1, GEMV_MT_MAX_CTAS / TG));
-  if (P > 1 && TG * P > GEMV_MT_MAX_CTAS) return QL_ERR_RANGE;  // partial sums only exist for P > 1
+  // split K over the CTAs of a 64-row group so that the groups fill one wave of resident CTAs
+  const SplitK split = split_k(TG, (int64_t)sms * GEMV6_CTAS_PER_SM, NS, true);
+  const int64_t ctas = split.total(TG);
+  const bool splits = split.P + (split.extra > 0) > 1;  // some group's K is split
+  if (splits && ctas > GEMV_MT_MAX_CTAS) return QL_ERR_RANGE;  // partial sums' room
   cudaLaunchAttribute pa[1];
   pa[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   pa[0].val.programmaticStreamSerializationAllowed = 1;
   {
-    const int64_t threads = std::max<int64_t>(M * (K / 16), P > 1 ? TG : 0);
+    const int64_t threads = std::max<int64_t>(M * (K / 16), splits ? TG : 0);
     cudaLaunchConfig_t pc = {};
     pc.gridDim = dim3((unsigned)((threads + 255) / 256));
     pc.blockDim = dim3(256);
     pc.stream = st;
     pc.attrs = pa;
     pc.numAttrs = 1;
-    if (cudaLaunchKernelEx(&pc, gemv_xprep_int6_kernel<PLANAR>, xb, M, K, P > 1 ? TG : (int64_t)0, ws) !=
+    if (cudaLaunchKernelEx(&pc, gemv_xprep_int6_kernel<PLANAR>, xb, M, K, splits ? TG : (int64_t)0, ws) !=
         cudaSuccess)
       return cuda_failed();
   }
@@ -310,7 +310,7 @@ ql_status launch_gemv_int6(const ql_desc *d, const ql_packed_const *w, const __n
   p.N = N;
   p.K = K;
   p.M = (int)M;
-  p.P = (int)P;
+  p.split = split;
   p.ws = ws;
   p.y = yb;
   const uint64_t code_row = (uint64_t)K * 3 / 4, sc_row = (uint64_t)K / 16;
@@ -330,7 +330,7 @@ ql_status launch_gemv_int6(const ql_desc *d, const ql_packed_const *w, const __n
     configured_dev = dev;
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(TG * P));
+  cfg.gridDim = dim3((unsigned)ctas);
   cfg.blockDim = dim3(GEMV6_THREADS);
   cfg.dynamicSmemBytes = L::SMEM;
   cfg.stream = st;
@@ -366,12 +366,13 @@ ql_status launch_gemv(const ql_desc *d, const ql_packed_const *w, const void *x,
       const GemvWorkspace ws = gemv_workspace_carve(workspace, M, d->N, d->K);
       const int64_t ng = M * (d->K / 32);
       const int64_t NS = d->K / 256, n_tiles = (d->N + 15) / 16;
-      // split K over P warps per 16-row tile while the tiles alone leave the resident warp slots
-      // unfilled; the parts' sums go through the workspace (at most GEMV_MT_MAX_CTAS * 64 floats)
-      const int64_t warp_slots = (int64_t)sms * GEMV_CTAS_PER_SM * GEMV_WARPS;
-      int64_t P = std::max<int64_t>(1, std::min<int64_t>(NS, warp_slots / n_tiles));
-      P = std::min<int64_t>(P, std::max<int64_t>(1, (int64_t)GEMV_MT_MAX_CTAS * 64 / 16 / n_tiles));
-      const int64_t n_counters = P > 1 ? n_tiles : 0;
+      // split K over the warps of a 16-row tile so that the tiles fill the resident warp slots; the
+      // parts' sums go through the workspace (16 floats a warp: at most the slots' 16 * 1776 of its
+      // GEMV_MT_MAX_CTAS * 64)
+      const SplitK split = split_k(n_tiles, (int64_t)sms * GEMV_CTAS_PER_SM * GEMV_WARPS, NS, false);
+      const bool splits = split.P + (split.extra > 0) > 1;
+      if (splits && split.total(n_tiles) * 16 > (int64_t)GEMV_MT_MAX_CTAS * 64) return QL_ERR_RANGE;
+      const int64_t n_counters = splits ? n_tiles : 0;
       {  // programmatic dependent of whatever precedes it on the stream (it waits before reading x)
         const int64_t threads = std::max<int64_t>(4 * ng, n_counters);  // four lanes per group
         cudaLaunchConfig_t pc = {};
@@ -402,7 +403,7 @@ ql_status launch_gemv(const ql_desc *d, const ql_packed_const *w, const void *x,
           !encode_2d(&mg, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->gmeta, (uint64_t)d->K / 16, (uint64_t)d->N,
                      (uint64_t)d->K / 16, 16, 16, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cuda_failed();
-      p.parts = (int)P;
+      p.split = split;
       static thread_local int configured_dev = -1;
       int dev = 0;
       cudaGetDevice(&dev);
@@ -413,7 +414,7 @@ ql_status launch_gemv(const ql_desc *d, const ql_packed_const *w, const void *x,
         configured_dev = dev;
       }
       cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3((unsigned)((n_tiles * P + GEMV_WARPS - 1) / GEMV_WARPS));
+      cfg.gridDim = dim3((unsigned)((split.total(n_tiles) + GEMV_WARPS - 1) / GEMV_WARPS));
       cfg.blockDim = dim3(32 * GEMV_WARPS);
       cfg.dynamicSmemBytes = gemv_smem_bytes();
       cfg.stream = st;
