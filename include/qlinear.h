@@ -248,9 +248,16 @@ ql_status qlinear_gemv_workspace_bytes(const ql_desc *desc, int64_t M, size_t *b
  *    int4 at M >= 2 and affine use the tokens as MMA columns.  K may be split
  *    over warps or CTAs, the parts added in a fixed order through the
  *    workspace.
+ *  - Affine with group 32 or 64 and K % 256 == 0 at 9 <= M <= 32: two
+ *    launches, fp16 tensor cores.  A pass writes x as fp16 with one
+ *    power-of-two scale per token (qlinear_gemm's first pass); the streaming
+ *    kernel dequantises each weight once to fp16 (q * s' + b', one rounding,
+ *    with (s, b) scaled per row by a power of two from the row's group
+ *    words) and multiplies it with mma.sync m16n8k16 against two or four
+ *    8-token column tiles, fp32 accumulation over K, both scales undone at
+ *    the end.
  *  - Affine with other groups, or K % 256 != 0, at M < 8: one launch, exact
- *    binary32 weights, fp32 FMA.
- *  - Affine at M >= 9 (M >= 8 on the path above): runs as qlinear_gemm.
+ *    binary32 weights, fp32 FMA; from M = 8: runs as qlinear_gemm.
  * ExecuTorch page above, "Quant schema update" (the int4 / int6 formats)
  * and the review's "Things done well" (the decode kernel's per-super-block
  * step word and full-warp trip counts).

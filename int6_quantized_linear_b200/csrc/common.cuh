@@ -34,6 +34,14 @@ __device__ unsigned int g_ql_status;
 __constant__ int g_ql_withhold;
 QL_DEVI bool copies_withheld() { return g_ql_withhold != 0; }
 
+// Programmatic dependent launch: let the next grid on the stream start, and wait for the previous one
+// (all of its memory operations complete and visible) before touching what it may have written.
+QL_DEVI void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+QL_DEVI void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Bring a line into L2 ahead of a dependent read: L2 is where the previous kernel's stores land, so a
+// load after griddepcontrol.wait still sees them, only sooner.
+QL_DEVI void prefetch_l2(const void *p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
+
 QL_DEVI uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

@@ -79,10 +79,22 @@ QL_DEVI int scale_exponent(float amax, int top) {
 // chunk the elements are stored in the order k = 0,4,1,5,2,6,3,7 (pairs (0,4) (1,5) (2,6) (3,7)):
 // the weight operand is written in the same order, which is the order a single bit operation
 // pulls nibble pairs out of a code word (the MMA's sum over k does not depend on it).
+// DEP: launched as a programmatic dependent (of whatever precedes it on the stream) by the fp16 GEMV,
+// whose streaming kernel is in turn its dependent: the pass lets that kernel start, waits for its own
+// predecessor before reading x, and clears the first n_counters K-split counters.
+template <bool DEP = false>
 __global__ void __launch_bounds__(256) x_to_f16_kernel(const __nv_bfloat16 *x, int64_t M, int64_t K,
-                                                        GemmWorkspace ws) {
+                                                        GemmWorkspace ws, int *counters = nullptr,
+                                                        int64_t n_counters = 0) {
   const int lane = threadIdx.x & 31;
-  const int64_t m = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+  const int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  const int64_t m = t >> 5;
+  if constexpr (DEP) {
+    pdl_launch_dependents();
+    if (m < M) prefetch_l2(x + m * K + 8 * lane);
+    pdl_wait();
+    if (t < n_counters) counters[t] = 0;
+  }
   if (m >= M) return;
   const uint4 *row = reinterpret_cast<const uint4 *>(x + m * K);
   const int64_t nv = K / 8;  // 16-byte vectors

@@ -193,11 +193,6 @@ QL_DEVI int atomic_add_acq_rel_gpu(int *addr, int v) {
   return old;
 }
 
-QL_DEVI void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-QL_DEVI void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-// Bring a line into L2 ahead of a dependent read: L2 is where the previous kernel's stores land, so a
-// load after griddepcontrol.wait still sees them, only sooner.
-QL_DEVI void prefetch_l2(const void *p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
 
 // The 24-bit marker: the lowest mantissa bit of a group's x scale G_x.  For 16-bit x, G_x is a power of
 // two (that bit is 0); for 24-bit x it is a normal power of two with the bit set, which changes it by

@@ -9,6 +9,7 @@
 #include "gemm_sm100.cuh"
 #include "gemv.cuh"
 #include "gemv_int6.cuh"
+#include "gemv_f16.cuh"
 #include "pack_dequant.cuh"
 
 using namespace ql;
@@ -142,7 +143,7 @@ ql_status launch_gemm_tt(const ql_desc *d, const ql_packed_const *w, const void 
   const uint64_t row_bytes = (uint64_t)K * code_bits(FMT, BITS) / 8;
   const GemmWorkspace ws = gemm_workspace_carve(workspace, M, N, K);
   // pass 1: scaled fp16 activations; pass 2: per-row weight scales
-  x_to_f16_kernel<<<(int)((M * 32 + 255) / 256), 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(x), M, K, ws);
+  x_to_f16_kernel<false><<<(int)((M * 32 + 255) / 256), 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(x), M, K, ws);
   w_scale_kernel<FMT, BITS><<<(int)(((int64_t)padded_rows(N) * 32 + 255) / 256), 256, 0, st>>>(
       static_cast<const uint8_t *>(w->gmeta), static_cast<const uint8_t *>(w->steps), N, K, d->group, ws);
   CUtensorMap mx, mc;
@@ -186,16 +187,15 @@ ql_status launch_gemm(const ql_desc *d, const ql_packed_const *w, const void *x,
   return launch_gemm_tt<FMT, BITS, gemm::BM>(d, w, x, M, bias, y, workspace, st, sms);
 }
 
-// Which GEMV calls run on the tensor-core GEMM (measured faster there on the benchmark layers:
-// affine M=32 70-74 us vs 537-551 us on the CUDA-core kernel): affine from M = 9 when a multi-token
-// tensor-core GEMV exists for it (group 32 / 64, K a multiple of 256), else from M = 8.  int4 and int6
-// have tensor-core GEMVs over their whole GEMV range (M <= 8).
+// Affine layers the tensor-core GEMVs serve: group 32 or 64, K a multiple of 256 (the integer
+// multi-token kernel up to 8 tokens, the fp16 kernel from 9 to 32).
+inline bool affine_tc(const ql_desc *d) { return (d->group == 32 || d->group == 64) && d->K % 256 == 0; }
+
+// Which GEMV calls run on the tensor-core GEMM: affine with other groups from M = 8 (measured faster
+// there than on the CUDA-core kernel: M=32 70-74 us vs 537-551 us).  int4 and int6 have tensor-core
+// GEMVs over their whole GEMV range (M <= 8).
 inline bool gemv_runs_on_gemm(const ql_desc *d, int64_t M) {
-  if (d->fmt == QL_AFFINE_U32) {  // 2-, 4- and 8-bit affine with group 32 / 64: multi-token kernel up to M = 8
-    const bool mt = (d->group == 32 || d->group == 64) && d->K % 256 == 0;
-    return M >= (mt ? 9 : 8);
-  }
-  return false;
+  return d->fmt == QL_AFFINE_U32 && !affine_tc(d) && M >= 8;
 }
 
 inline size_t gemv_call_workspace_bytes(const ql_desc *d, int64_t M) {
@@ -340,6 +340,75 @@ ql_status launch_gemv_int6(const ql_desc *d, const ql_packed_const *w, const __n
   return launched();
 }
 
+// fp16 tensor-core GEMV for affine at 9..32 tokens (NT column tiles of 8): the x pass (fp16, one
+// exponent per token, programmatic dependent of what precedes it), then the streaming kernel as its
+// dependent.  x16 and the token exponents sit at the start of the workspace (the GEMM's layout), the
+// partial sums and counters of a K split where the GEMV layout has them (past 7 M K bytes).
+template <int BITS, int G, int NT>
+ql_status launch_gemv_f16(const ql_desc *d, const ql_packed_const *w, const __nv_bfloat16 *xb, int64_t M,
+                          const __nv_bfloat16 *bb, __nv_bfloat16 *yb, void *workspace, cudaStream_t st, int sms) {
+  using L = F16Layout<BITS, G, NT>;
+  const int64_t N = d->N, K = d->K, NS = K / 256, TG = (N + 63) / 64;
+  const GemmWorkspace gw = gemm_workspace_carve(workspace, M, N, K);
+  const GemvWorkspace vw = gemv_workspace_carve(workspace, M, N, K);
+  const SplitK split = split_k(TG, (int64_t)sms * L::CTAS, NS, false);
+  const int64_t ctas = split.total(TG);
+  const bool splits = split.P > 1;
+  if (splits && ctas > GEMV_MT_MAX_CTAS) return QL_ERR_RANGE;  // partial sums' room
+  cudaLaunchAttribute pa[1];
+  pa[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pa[0].val.programmaticStreamSerializationAllowed = 1;
+  {
+    const int64_t n_counters = splits ? TG : 0;
+    const int64_t threads = std::max<int64_t>(M * 32, n_counters);  // a warp per token row
+    cudaLaunchConfig_t pc = {};
+    pc.gridDim = dim3((unsigned)((threads + 255) / 256));
+    pc.blockDim = dim3(256);
+    pc.stream = st;
+    pc.attrs = pa;
+    pc.numAttrs = 1;
+    if (cudaLaunchKernelEx(&pc, x_to_f16_kernel<true>, xb, M, K, gw, vw.counters, n_counters) != cudaSuccess)
+      return cuda_failed();
+  }
+  GemvF16Params p;
+  p.gmeta = static_cast<const uint8_t *>(w->gmeta);
+  p.bias = bb;
+  p.xexp = gw.xexp;
+  p.N = N;
+  p.K = K;
+  p.M = (int)M;
+  p.split = split;
+  p.ws = vw;
+  p.y = yb;
+  const uint64_t code_row = (uint64_t)K * BITS / 8, meta_row = (uint64_t)K / G * 4;
+  CUtensorMap mc, mg, mx;  // codes: 64 rows x CODE_BOX bytes, swizzled; group words: 64 x META_ROW; x: 8 NT x 32 halves
+  if (!encode_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->codes, code_row, (uint64_t)N, code_row, L::CODE_BOX, 64,
+                 L::CODE_BOX == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !encode_2d(&mg, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->gmeta, meta_row, (uint64_t)N, meta_row, L::META_ROW, 64,
+                 CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !encode_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, gw.x16, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, 32,
+                 (uint32_t)L::XROWS, CU_TENSOR_MAP_SWIZZLE_64B))
+    return cuda_failed();
+  auto kern = gemv_f16_kernel<BITS, G, NT>;
+  static thread_local int configured_dev = -1;  // per instantiation and thread
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (configured_dev != dev) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM) != cudaSuccess)
+      return cuda_failed();
+    configured_dev = dev;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)ctas);
+  cfg.blockDim = dim3(GEMV_MT_THREADS);
+  cfg.dynamicSmemBytes = L::SMEM;
+  cfg.stream = st;
+  cfg.attrs = pa;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, mc, mg, mx, p) != cudaSuccess) return cuda_failed();
+  return launched();
+}
+
 template <int FMT, int BITS>
 ql_status launch_gemv(const ql_desc *d, const ql_packed_const *w, const void *x, int64_t M, const void *bias,
                       void *y, void *workspace, cudaStream_t st, int sms) {
@@ -358,8 +427,17 @@ ql_status launch_gemv(const ql_desc *d, const ql_packed_const *w, const void *x,
     return launch_gemv_int6<8, PL>(d, w, xb, M, bb, yb, workspace, st, sms);
   }
   if constexpr (FMT == FMT_AFFINE) {  // bits 2, 4, 8
-    if (d->K % 256 == 0 && d->group == 64) return launch_gemv_mt<FMT_AFFINE, BITS, 64>(d, w, xb, M, bb, yb, workspace, st, sms);
-    if (d->K % 256 == 0 && d->group == 32) return launch_gemv_mt<FMT_AFFINE, BITS, 32>(d, w, xb, M, bb, yb, workspace, st, sms);
+    if (affine_tc(d) && M <= 8) {
+      if (d->group == 64) return launch_gemv_mt<FMT_AFFINE, BITS, 64>(d, w, xb, M, bb, yb, workspace, st, sms);
+      return launch_gemv_mt<FMT_AFFINE, BITS, 32>(d, w, xb, M, bb, yb, workspace, st, sms);
+    }
+    if (affine_tc(d)) {  // 9..32 tokens
+      if (d->group == 64)
+        return M <= 16 ? launch_gemv_f16<BITS, 64, 2>(d, w, xb, M, bb, yb, workspace, st, sms)
+                       : launch_gemv_f16<BITS, 64, 4>(d, w, xb, M, bb, yb, workspace, st, sms);
+      return M <= 16 ? launch_gemv_f16<BITS, 32, 2>(d, w, xb, M, bb, yb, workspace, st, sms)
+                     : launch_gemv_f16<BITS, 32, 4>(d, w, xb, M, bb, yb, workspace, st, sms);
+    }
   }
   if constexpr (FMT == FMT_INT4) {
     if (M == 1) {  // tensor-core path: preparation pass, then the streaming kernel as its dependent

@@ -140,8 +140,8 @@ def test_edge_pack_unpack_dequant_bitexact(cuda, fmt, bits, group):
 
 
 def _gemv_token_counts(fmt, group):
-    if fmt == "affine":  # multi-token kernel (group 32 / 64) or CUDA cores (group 128) up to 7-8 tokens,
-        return (1, 7, 8, 12, 32)  # the tcgen05 GEMM from there
+    if fmt == "affine":  # group 32 / 64: integer multi-token kernel to 8 tokens, the fp16 tensor-core
+        return (1, 7, 8, 9, 12, 16, 31, 32)  # GEMV from 9; group 128: CUDA cores to 7, the tcgen05 GEMM from 8
     return (1, 2, 5, 7, 8)
 
 

@@ -164,6 +164,31 @@ def test_gemv_affine2_multi_token(cuda, bits, group, N, K):
         assert np.array_equal(y, run_gemv(L, xd, M))
 
 
+@pytest.mark.parametrize("bits,group", [(2, 64), (4, 64), (8, 64), (2, 32), (4, 32), (8, 32)])
+@pytest.mark.parametrize("N,K", [(200, 1536), (64, 256), (1000, 4096)])
+def test_gemv_affine_f16_token_counts(cuda, bits, group, N, K):
+    """Affine at 9..32 tokens on the fp16 tensor-core GEMV (two or four 8-token column tiles, K split
+    over CTAs for the small layers, ragged N): every token count on its own layer checked against the
+    oracle; repeated runs give identical bits; the bias variant adds bias[n]."""
+    L = Layer("affine", N, K, seed=17 * N + K + bits, bits=bits, group=group)
+    w_ref = L.oracle_w()
+    bias_b = synth.activations(N + 3 * K, 1, N)[0]
+    xb32, _ = x_dev(K, 32, seed=300 + bits)
+    for M in (9, 10, 15, 16, 17, 23, 24, 31, 32):
+        xb = xb32[:M]
+        xd = dev(xb)
+        y = run_gemv(L, xd, M)
+        y_ref = OC.matmul_f64(xb, w_ref)
+        assert_close(y, y_ref, f"affine{bits} g{group} f16 gemv N={N} K={K} M={M}")
+        assert np.array_equal(y, run_gemv(L, xd, M))
+        if M in (9, 32):
+            yb = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+            ql.qlinear_gemv_bias(L.desc, *L.packed(), xd, M, dev(bias_b).view(torch.bfloat16), yb)
+            assert ql.qlinear_sync_status() == ql.QL_OK
+            assert_close(host(yb.view(torch.int16), np.uint16), y_ref + bf16_to_f64(bias_b)[None, :],
+                         f"affine{bits} g{group} f16 gemv+bias M={M}")
+
+
 @pytest.mark.parametrize("fmt", ["int6", "int6p"])
 @pytest.mark.parametrize("N,K", [(200, 1536), (64, 256), (1000, 5120)])
 def test_gemv_int6_every_token_count(cuda, fmt, N, K):
