@@ -54,6 +54,12 @@ def parse_args(argv=None):
     ap.add_argument("--no-other-configs", action="store_true")
     ap.add_argument("--load-window", type=float, default=1.5,
                     help="seconds of extra steps run after the timed region so the clock sampler sees load")
+    ap.add_argument("--case", default=None,
+                    help="profiling aid: pack one workload layer (synth.WORKLOADS name), run --case-calls "
+                         "qlinear_gemv (or --case-gemm: qlinear_gemm) calls at --case-m tokens, print one line")
+    ap.add_argument("--case-m", type=int, default=1)
+    ap.add_argument("--case-calls", type=int, default=3)
+    ap.add_argument("--case-gemm", action="store_true")
     return ap.parse_args(argv)
 
 
@@ -739,8 +745,39 @@ def run_reference(args):
     }
 
 
+def run_case(args):
+    """A few eager calls of one workload layer, for a profiler's launch list or capture (the
+    commands in profiles/): no timing, no JSON contract line."""
+    import torch
+
+    import int6_quantized_linear_b200 as ql
+    from int6_quantized_linear_b200 import synth
+
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    wl = synth.WORKLOADS[args.case]
+    d, packed, _ = packed_layer(wl, device)
+    M = args.case_m
+    x = torch.from_numpy(wl.x(M).view("int16")).to(device).view(torch.bfloat16)
+    y = torch.empty((M, wl.N), dtype=torch.bfloat16, device=device)
+    if args.case_gemm:
+        ws = ql.alloc_gemm_workspace(d, M, device)
+        for _ in range(args.case_calls):
+            ql.qlinear_gemm(d, *packed, x, M, y, ws)
+    else:
+        ws = ql.alloc_gemv_workspace(d, M, device)
+        for _ in range(args.case_calls):
+            ql.qlinear_gemv(d, *packed, x, M, y, ws)
+    status = ql.qlinear_sync_status()
+    print(f"case {args.case} M={M} calls={args.case_calls} status={ql.status_string(status)}")
+    return None
+
+
 def main(argv=None):
     args = parse_args(argv)
+    if args.case:
+        run_case(args)
+        return
     line = run_reference(args) if args.impl == "reference" else run_native(args)
     if line is not None:
         print(json.dumps(line), flush=True)
