@@ -39,8 +39,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM bytes per GEMV launch from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum),
 # valid only while the GEMV source is unchanged (hash of csrc/gemv.cuh at capture time).
-NCU_TRAFFIC = {"gemv_src_sha256": "b294c01463628313d5d4a869b847dc5dcf4046f6a1201c3396eed4cc0e6426d0",
-               "bytes_per_launch": 83361664}  # mean over the two decode layers
+NCU_TRAFFIC = {"gemv_src_sha256": "5851b5cb8872c942c39e8b2aa4402a168f73f18aff8127599745241a6825d466",
+               "bytes_per_launch": 83032576}  # mean over the two decode layers
 
 
 def parse_args(argv=None):
