@@ -75,57 +75,90 @@ QL_DEVI int scale_exponent(float amax, int top) {
   return s < -126 ? -126 : (s > 126 ? 126 : s);
 }
 
-// One warp per token row: find max|x|, then write the scaled fp16 row.  Within every 8-element
-// chunk the elements are stored in the order k = 0,4,1,5,2,6,3,7 (pairs (0,4) (1,5) (2,6) (3,7)):
-// the weight operand is written in the same order, which is the order a single bit operation
-// pulls nibble pairs out of a code word (the MMA's sum over k does not depend on it).
+// One CTA of 256 threads per token row: find max|x|, then write the scaled fp16 row.  Within every
+// 8-element chunk the elements are stored in the order k = 0,4,1,5,2,6,3,7 (pairs (0,4) (1,5) (2,6)
+// (3,7)): the weight operand is written in the same order, which is the order a single bit operation
+// pulls nibble pairs out of a code word (the MMA's sum over k does not depend on it).  Rows of up to
+// X2F16_REGS * 256 16-byte vectors are read once and kept in registers; longer rows are read again for
+// the conversion.
 // DEP: launched as a programmatic dependent (of whatever precedes it on the stream) by the fp16 GEMV,
 // whose streaming kernel is in turn its dependent: the pass lets that kernel start, waits for its own
-// predecessor before reading x, and clears the first n_counters K-split counters.
+// predecessor before reading x, and clears the first n_counters K-split counters (the grid has at
+// least n_counters threads).
+constexpr int X2F16_THREADS = 256, X2F16_REGS = 4;
+
+QL_DEVI uint4 x_chunk_to_f16(uint4 v, float sc) {
+  const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+  uint32_t o[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {  // pair j = (x[j], x[j + 4]): u[j / 2] holds x[j & ~1], x[j | 1]
+    const uint32_t a = u[j >> 1], b = u[2 + (j >> 1)];
+    const float lo = (j & 1) ? __uint_as_float(a & 0xffff0000u) : __uint_as_float(a << 16);
+    const float hi = (j & 1) ? __uint_as_float(b & 0xffff0000u) : __uint_as_float(b << 16);
+    const __half2 h = __floats2half2_rn(lo * sc, hi * sc);
+    o[j] = *reinterpret_cast<const uint32_t *>(&h);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+QL_DEVI float chunk_amax(uint4 v, float amax) {
+  const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(u[j] << 16)), fabsf(__uint_as_float(u[j] & 0xffff0000u))));
+  return amax;
+}
+
 template <bool DEP = false>
-__global__ void __launch_bounds__(256) x_to_f16_kernel(const __nv_bfloat16 *x, int64_t M, int64_t K,
-                                                        GemmWorkspace ws, int *counters = nullptr,
-                                                        int64_t n_counters = 0) {
-  const int lane = threadIdx.x & 31;
-  const int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-  const int64_t m = t >> 5;
+__global__ void __launch_bounds__(X2F16_THREADS) x_to_f16_kernel(const __nv_bfloat16 *x, int64_t M, int64_t K,
+                                                                 GemmWorkspace ws, int *counters = nullptr,
+                                                                 int64_t n_counters = 0) {
+  __shared__ float red[X2F16_THREADS / 32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t m = blockIdx.x;
+  const int64_t nv = K / 8;  // 16-byte vectors of the row
+  const uint4 *row = reinterpret_cast<const uint4 *>(x + m * K);
   if constexpr (DEP) {
     pdl_launch_dependents();
-    if (m < M) prefetch_l2(x + m * K + 8 * lane);
+    if (m < M && tid < nv) prefetch_l2(row + tid);
     pdl_wait();
+    const int64_t t = m * X2F16_THREADS + tid;
     if (t < n_counters) counters[t] = 0;
   }
-  if (m >= M) return;
-  const uint4 *row = reinterpret_cast<const uint4 *>(x + m * K);
-  const int64_t nv = K / 8;  // 16-byte vectors
+  if (m >= M) return;  // whole CTAs leave together
+  const bool in_regs = nv <= (int64_t)X2F16_REGS * X2F16_THREADS;
+  uint4 v[X2F16_REGS];
   float amax = 0.f;
-  for (int64_t i = lane; i < nv; i += 32) {
-    const uint4 v = __ldg(row + i);
-    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+  if (in_regs) {
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
-      amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(u[j] << 16)), fabsf(__uint_as_float(u[j] & 0xffff0000u))));
+    for (int r = 0; r < X2F16_REGS; ++r) {
+      const int64_t i = tid + (int64_t)r * X2F16_THREADS;
+      v[r] = i < nv ? __ldg(row + i) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int r = 0; r < X2F16_REGS; ++r) amax = chunk_amax(v[r], amax);
+  } else {
+    for (int64_t i = tid; i < nv; i += X2F16_THREADS) amax = chunk_amax(__ldg(row + i), amax);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if (lane == 0) red[warp] = amax;
+  __syncthreads();
+#pragma unroll
+  for (int w = 0; w < X2F16_THREADS / 32; ++w) amax = fmaxf(amax, red[w]);
   const int a = scale_exponent(amax, 15);
   const float sc = exp2i(a);
   uint4 *out = reinterpret_cast<uint4 *>(ws.x16 + m * K);
-  for (int64_t i = lane; i < nv; i += 32) {
-    const uint4 v = __ldg(row + i);
-    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
-    uint32_t o[4];
+  if (in_regs) {
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {  // pair j = (x[j], x[j + 4]): u[j / 2] holds x[j & ~1], x[j | 1]
-      const uint32_t a = u[j >> 1], b = u[2 + (j >> 1)];
-      const float lo = (j & 1) ? __uint_as_float(a & 0xffff0000u) : __uint_as_float(a << 16);
-      const float hi = (j & 1) ? __uint_as_float(b & 0xffff0000u) : __uint_as_float(b << 16);
-      const __half2 h = __floats2half2_rn(lo * sc, hi * sc);
-      o[j] = *reinterpret_cast<const uint32_t *>(&h);
+    for (int r = 0; r < X2F16_REGS; ++r) {
+      const int64_t i = tid + (int64_t)r * X2F16_THREADS;
+      if (i < nv) out[i] = x_chunk_to_f16(v[r], sc);
     }
-    out[i] = make_uint4(o[0], o[1], o[2], o[3]);
+  } else {
+    for (int64_t i = tid; i < nv; i += X2F16_THREADS) out[i] = x_chunk_to_f16(__ldg(row + i), sc);
   }
-  if (lane == 0) ws.xexp[m] = -a;
+  if (tid == 0) ws.xexp[m] = -a;
 }
 
 // One warp per weight row: bound max|w| from the metadata (lanes stride over the groups, then a

@@ -143,7 +143,7 @@ ql_status launch_gemm_tt(const ql_desc *d, const ql_packed_const *w, const void 
   const uint64_t row_bytes = (uint64_t)K * code_bits(FMT, BITS) / 8;
   const GemmWorkspace ws = gemm_workspace_carve(workspace, M, N, K);
   // pass 1: scaled fp16 activations; pass 2: per-row weight scales
-  x_to_f16_kernel<false><<<(int)((M * 32 + 255) / 256), 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(x), M, K, ws);
+  x_to_f16_kernel<false><<<(unsigned)M, X2F16_THREADS, 0, st>>>(static_cast<const __nv_bfloat16 *>(x), M, K, ws);
   w_scale_kernel<FMT, BITS><<<(int)(((int64_t)padded_rows(N) * 32 + 255) / 256), 256, 0, st>>>(
       static_cast<const uint8_t *>(w->gmeta), static_cast<const uint8_t *>(w->steps), N, K, d->group, ws);
   CUtensorMap mx, mc;
@@ -360,10 +360,10 @@ ql_status launch_gemv_f16(const ql_desc *d, const ql_packed_const *w, const __nv
   pa[0].val.programmaticStreamSerializationAllowed = 1;
   {
     const int64_t n_counters = splits ? TG : 0;
-    const int64_t threads = std::max<int64_t>(M * 32, n_counters);  // a warp per token row
+    const int64_t blocks = std::max<int64_t>(M, (n_counters + X2F16_THREADS - 1) / X2F16_THREADS);  // a CTA per token row
     cudaLaunchConfig_t pc = {};
-    pc.gridDim = dim3((unsigned)((threads + 255) / 256));
-    pc.blockDim = dim3(256);
+    pc.gridDim = dim3((unsigned)blocks);
+    pc.blockDim = dim3(X2F16_THREADS);
     pc.stream = st;
     pc.attrs = pa;
     pc.numAttrs = 1;

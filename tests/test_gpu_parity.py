@@ -189,6 +189,23 @@ def test_gemv_affine_f16_token_counts(cuda, bits, group, N, K):
                          f"affine{bits} g{group} f16 gemv+bias M={M}")
 
 
+@pytest.mark.parametrize("bits,group", [(4, 64), (2, 32), (8, 64)])
+@pytest.mark.parametrize("N,K", [(37900, 512), (3000, 2304)])
+def test_gemv_affine_f16_unit_ranges(cuda, bits, group, N, K):
+    """The fp16 GEMV on larger layers: K = 512 with far more 64-row groups than CTA slots and a ragged
+    last group, K = 2304 with its K split over CTAs; every output checked against the oracle, bits
+    repeatable."""
+    L = Layer("affine", N, K, seed=19 * N + K + bits, bits=bits, group=group)
+    w_ref = L.oracle_w()
+    xb32, _ = x_dev(K, 32, seed=400 + bits)
+    for M in (9, 32):
+        xb = xb32[:M]
+        xd = dev(xb)
+        y = run_gemv(L, xd, M)
+        assert_close(y, OC.matmul_f64(xb, w_ref), f"affine{bits} g{group} f16 gemv N={N} K={K} M={M}")
+        assert np.array_equal(y, run_gemv(L, xd, M))
+
+
 @pytest.mark.parametrize("fmt", ["int6", "int6p"])
 @pytest.mark.parametrize("N,K", [(200, 1536), (64, 256), (1000, 5120)])
 def test_gemv_int6_every_token_count(cuda, fmt, N, K):
