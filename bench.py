@@ -240,8 +240,14 @@ def gemv_step(layers, i: int, ql):
         ql.qlinear_gemv(L["desc"], c, g, s, L["x"], 1, L["y"], L["ws"])
 
 
-# qlinear_gemv at int4, M=1 launches two kernels: the x-preparation kernel and the GEMV kernel
-KERNELS_PER_GEMV = 2
+def gemv_m1_launches(K: int, N: int, sms: int) -> int:
+    """Kernels one qlinear_gemv call at int4, M=1 launches: the streaming kernel, plus the kernel that
+    adds the parts when K is split (the launcher's rule: the 4-tile CTA groups fill 3 CTAs per SM, at
+    most K/256 parts, and at least enough parts that each holds 22 super-blocks of x)."""
+    NS, groups = K // 256, -(-(-(-N // 16)) // 4)
+    P = max(1, min(NS, sms * 3 // groups))
+    P = max(P, -(-NS // 22))
+    return 1 + (P > 1)
 
 
 def _ev():
@@ -355,6 +361,7 @@ def run_native(args):
 
     if rank != 0:
         return None
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
     line = {
         "metric": METRIC,
         "value": round(value_bps / 1e9, 2),
@@ -377,7 +384,7 @@ def run_native(args):
         "gemm_m2048": gemm,
         "other_configs": others,
         "e2e": e2e,
-        "gpu_launches": args.steps * len(layers) * KERNELS_PER_GEMV,
+        "gpu_launches": args.steps * sum(gemv_m1_launches(L["K"], L["N"], sms) for L in layers),
         "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
         "clock_samples": clocks["samples"],
     }

@@ -229,15 +229,20 @@ ql_status qlinear_gemv_workspace_bytes(const ql_desc *desc, int64_t M, size_t *b
  * fp32 scales and accumulation, one nearest-even rounding to bf16 at the end.
  * 1 <= M <= 8 for int4 / int6; 1 <= M <= 32 for affine.
  *  - Tensor-core path (int4 and int6 at every M; affine with group 32 or 64
- *    and K % 256 == 0 at M <= 8): two launches.  A short pass turns each x
- *    group (32 elements; 16 for int6) into fixed point, x_int = rint(x *
+ *    and K % 256 == 0 at M <= 8): two launches (int4 at M = 1: one, plus a
+ *    short kernel that adds the parts when K is split).  Each x
+ *    group (32 elements; 16 for int6) is turned into fixed point, x_int = rint(x *
  *    2^a): 16-bit (the group's max |x| scaled into [2^14, 2^15): exact for
  *    every bf16 element within 2^7 of the group's largest magnitude), or
  *    24-bit (max in [2^22, 2^23): exact within 2^15) for every group of a
  *    super-block (per token) in which some group's 16-bit rounding error
  *    exceeds 2^-12 of its mass outside its largest element; split into high,
  *    middle and (24-bit) low bytes in the order the tensor-core fragments
- *    read them, with the group's scale (and sum); then the streaming kernel
+ *    read them, with the group's scale (and sum) -- by a short pass, or, for
+ *    int4 at M = 1, by each CTA of the streaming kernel for its part of K,
+ *    into shared memory (K split into parts of at most 22 super-blocks,
+ *    16 partial sums a part and 16 rows within the workspace's 4*4096*64
+ *    bytes; QL_ERR_RANGE beyond); then the streaming kernel
  *    multiplies the codes (as u8 or s8 bytes: 16q for nibbles, 4q for int6,
  *    q for 2- and 8-bit fields) by those bytes on the integer tensor core
  *    (mma.sync m16n8k32, exact s32 sums, one MMA per byte: high and middle
@@ -265,8 +270,8 @@ ql_status qlinear_gemv_workspace_bytes(const ql_desc *desc, int64_t M, size_t *b
  * caller-owned, overwritten; calls sharing one workspace must not overlap on
  * the GPU.  Consecutive tensor-core calls on one stream chain by
  * programmatic dependent launch: a call's weight stream may start while the
- * previous kernel on the stream drains, and its preparation pass waits for
- * that kernel before it reads x or writes the workspace.
+ * previous kernel on the stream drains, and its first kernel waits for that
+ * kernel before it reads x or writes the workspace.
  * Errors: QL_ERR_NULL, QL_ERR_SHAPE (also: workspace too small),
  * QL_ERR_ALIGN, QL_ERR_RANGE, QL_ERR_UNSUPPORTED, QL_ERR_CUDA. */
 ql_status qlinear_gemv(const ql_desc *desc, const ql_packed_const *w,

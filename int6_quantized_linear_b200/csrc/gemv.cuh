@@ -156,12 +156,11 @@ inline SplitK split_k(int64_t units, int64_t slots, int64_t NS, bool fill) {
 constexpr int GEMV_XBLOB = 1600, GEMV_XCOPY = 1088, GEMV_XB_Q = 64, GEMV_XB_L = 1088;
 
 struct GemvWorkspace {
-  uint4 *xq;        // int4 M = 1: [K/256 super-blocks] blocks of GEMV_XBLOB bytes (gemv_xprep_kernel)
-                    // int4 M > 1 / affine: [K/32 groups][M tokens][4][16 B] (hi, mid) B-operand words, then
+  uint4 *xq;        // int4 M > 1 / affine: [K/32 groups][M tokens][4][16 B] (hi, mid) B-operand words, then
                     //   [K/32][M][4][8 B] lo words (gemv_xprep_mt_kernel); int6: see gemv_xprep_int6_kernel
   float2 *gsum;     // M > 1: [K/32][M]: (G_x, G_y); int6: per 16-element group scales
-  float *partial;   // M = 1: [16-row tile][part][16 rows]; M > 1: [CTA][M][64 rows]: sums of one K range
-  int *counters;    // parts finished so far: M = 1 per 16-row tile, M > 1 per 64-row group
+  float *partial;   // [CTA][M][64 rows]: sums of one K range
+  int *counters;    // parts finished so far, per 64-row group
   uint8_t *flags;   // [K/256][16]: byte m non-zero when token m's x of that super-block is 24-bit
 };
 
@@ -214,87 +213,75 @@ QL_DEVI bool group_needs_24bit(float err, float mass, float amax_scaled) {
   return err > (mass - amax_scaled) * (1.f / 4096.f);
 }
 
-// x preparation for the int4 M = 1 kernel: four lanes per 32-element group (lane c holds k = 8c ..
-// 8c + 7), so one warp holds one super-block's eight groups.  Fixed-point conversion with the
-// group's max and sum by shuffles, 16-bit unless some group of the super-block needs 24 bits (then
-// the whole super-block is 24-bit and flagged), byte split in fragment order.  Chunk (j, kind) of
-// group grp is what its feeding lane loads: the high-byte and middle-byte words of
-// k = 8j + kind + {0, 2, 4, 6}, each paired with a zero word so that one 16-byte load gives the B
-// pairs of two MMAs -- (x, 0) for groups 0-3 (their lanes feed b0), (0, x) for groups 4-7 (b1) --
-// and the low-byte word paired the same way (8 bytes).  Lane c writes the chunks (j = c, kind = 0 / 1).
-// It also zeroes the first n_counters tile counters of the K split.
-__global__ void __launch_bounds__(256) gemv_xprep_kernel(const __nv_bfloat16 *x, int64_t M, int64_t K,
-                                                         int64_t n_counters, GemvWorkspace ws) {
-  pdl_launch_dependents();  // the streaming kernel may start fetching weights now
-  const int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-  const int64_t ng = K / 32;
-  const int64_t gi = t >> 2;  // over M * ng groups
-  const int c = (int)(t & 3);
-  const bool live = gi < M * ng;  // every lane takes part in the shuffles
-  if (live) prefetch_l2(reinterpret_cast<const uint4 *>(x) + 4 * gi + c);
-  pdl_wait();               // x (and this workspace) may belong to the kernel launched before this one
-  if (t < n_counters) ws.counters[t] = 0;
-  uint4 v = make_uint4(0u, 0u, 0u, 0u);
-  if (live) v = __ldg(reinterpret_cast<const uint4 *>(x) + 4 * gi + c);  // 8 bf16 = 16 bytes
-  const uint32_t u[4] = {v.x, v.y, v.z, v.w};
-  float xs[8];
+// x conversion for the int4 M = 1 kernel, one lane per 32-element group, eight lanes per super-block:
+// fixed point with the group's max and sum, 16-bit unless some group of the super-block needs 24 bits
+// (then the whole super-block is 24-bit), byte split in fragment order into the super-block's block
+// blk (shared memory, GEMV_XBLOB bytes): the eight groups' (G_x, G_y), then chunk (j, kind) of group
+// grp at [j][kind][grp] of the (hi, mid) region -- the high-byte and middle-byte words of
+// k = 8j + kind + {0, 2, 4, 6}, each paired with a zero word so that one 16-byte load gives the B pairs
+// of two MMAs: (x, 0) for groups 0-3 (their lanes feed b0), (0, x) for groups 4-7 (b1) -- and, for
+// 24-bit x only, the low-byte word paired the same way (8 bytes) in the lo region.  v: the group's 32
+// bf16; live: the lane holds a group (every lane takes part in the vote).  Returns whether the
+// super-block is 24-bit.
+QL_DEVI bool gemv_m1_convert_group(const uint4 (&v)[4], bool live, int grp, uint8_t *blk) {
+  const int lane = threadIdx.x & 31;
+  float xs[32];
   float amax = 0.f;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    xs[2 * i] = bf16_bits_to_f32(u[i]);
-    xs[2 * i + 1] = bf16_bits_to_f32(u[i] >> 16);
-    amax = fmaxf(amax, fmaxf(fabsf(xs[2 * i]), fabsf(xs[2 * i + 1])));
+  for (int q = 0; q < 4; ++q) {
+    const uint32_t u[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      xs[8 * q + 2 * i] = bf16_bits_to_f32(u[i]);
+      xs[8 * q + 2 * i + 1] = bf16_bits_to_f32(u[i] >> 16);
+    }
   }
-  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+#pragma unroll
+  for (int k = 0; k < 32; ++k) amax = fmaxf(amax, fabsf(xs[k]));
   const int a16 = scale_exponent(amax, 14);  // max |x_int| < 2^15
   const float s16 = exp2i(a16);
   float err = 0.f, mass = 0.f;
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
+  for (int k = 0; k < 32; ++k) {
     const float sv = xs[k] * s16;
     err += fabsf(sv - rintf(sv));
     mass += fabsf(sv);
   }
-  const bool wide = group_needs_24bit(err, mass, amax * s16);
-  const bool sb24 = __any_sync(0xffffffffu, wide && live);  // the warp holds one super-block
-  const int a = sb24 ? scale_exponent(amax, 22) : a16;     // 24-bit: max |x_int| < 2^23
+  // 16-bit fixed point loses too much when the summed rounding error is above 2^-12 of the group's mass
+  // outside its largest element (all in units of 2^-a16)
+  const bool wide = live && err > (mass - amax * s16) * (1.f / 4096.f);
+  const bool sb24 = ((__ballot_sync(0xffffffffu, wide) >> (lane & ~7)) & 0xffu) != 0u;  // the super-block's 8 lanes
+  const int a = sb24 ? scale_exponent(amax, 22) : a16;  // 24-bit: max |x_int| < 2^23
   const float sc = exp2i(a);
-  int xi[8];
+  if (!live) return sb24;
+  int xi[32];
   int sum = 0;  // |sum| < 32 * 2^23
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
+  for (int k = 0; k < 32; ++k) {
     xi[k] = __float2int_rn(xs[k] * sc);
     sum += xi[k];
   }
-  sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-  sum += __shfl_xor_sync(0xffffffffu, sum, 2);
-  if (!live) return;
-  // group gi = (m, super-block sb, group-in-block grp): per (m, sb) one block of GEMV_XBLOB bytes,
-  // the eight groups' (G_x, G_y), then chunk (j, kind) at [j][kind][grp] of the (hi, mid) region
-  // and, for 24-bit x only, of the lo region
-  const int64_t grp = gi & 7, msb = gi >> 3;
-  uint8_t *blk = reinterpret_cast<uint8_t *>(ws.xq) + msb * GEMV_XBLOB;
   const int hs = sb24 ? 16 : 8;  // the value's top byte: bits 16.. (24-bit) or 8.. (16-bit, lo = 0)
 #pragma unroll
-  for (int kind = 0; kind < 2; ++kind) {
-    uint32_t hi = 0, mid = 0, lo = 0;
+  for (int j = 0; j < 4; ++j)
 #pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      const int val = xi[2 * b + kind];
-      hi |= ((uint32_t)(val >> hs) & 0xffu) << (8 * b);
-      mid |= ((uint32_t)(val >> (hs - 8)) & 0xffu) << (8 * b);
-      lo |= ((uint32_t)val & 0xffu) << (8 * b);
+    for (int kind = 0; kind < 2; ++kind) {
+      uint32_t hi = 0, mid = 0, lo = 0;
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const int val = xi[8 * j + 2 * b + kind];
+        hi |= ((uint32_t)(val >> hs) & 0xffu) << (8 * b);
+        mid |= ((uint32_t)(val >> (hs - 8)) & 0xffu) << (8 * b);
+        lo |= ((uint32_t)val & 0xffu) << (8 * b);
+      }
+      const int ch = 8 * (2 * j + kind) + grp;  // chunk (j, kind) of group grp
+      reinterpret_cast<uint4 *>(blk + GEMV_XB_Q)[ch] = grp < 4 ? make_uint4(hi, 0u, mid, 0u) : make_uint4(0u, hi, 0u, mid);
+      if (sb24) reinterpret_cast<uint2 *>(blk + GEMV_XB_L)[ch] = grp < 4 ? make_uint2(lo, 0u) : make_uint2(0u, lo);
     }
-    const int ch = 8 * (2 * c + kind) + (int)grp;  // chunk (j = c, kind) of group grp
-    reinterpret_cast<uint4 *>(blk + GEMV_XB_Q)[ch] = grp < 4 ? make_uint4(hi, 0u, mid, 0u) : make_uint4(0u, hi, 0u, mid);
-    if (sb24) reinterpret_cast<uint2 *>(blk + GEMV_XB_L)[ch] = grp < 4 ? make_uint2(lo, 0u) : make_uint2(0u, lo);
-  }
-  if (c == 0) {  // (G_x, G_y) = (2^-a / 16, -16 X) scaled by (2^v, 2^-v), v = 8 (24-bit) or 0 (16-bit)
-    const float v = sb24 ? 256.f : 1.f, vi = sb24 ? 1.f / 256.f : 1.f, gx = exp2i(-a) * 0.0625f * v;
-    reinterpret_cast<float2 *>(blk)[grp] = make_float2(sb24 ? mark_24bit(gx) : gx, -16.f * (float)sum * vi);
-  }
-  if ((t & 31) == 0) ws.flags[msb * 16] = sb24 ? 1 : 0;  // M = 1: msb is the super-block
+  // (G_x, G_y) = (2^-a / 16, -16 X) scaled by (2^v, 2^-v), v = 8 (24-bit) or 0 (16-bit)
+  const float vs = sb24 ? 256.f : 1.f, vi = sb24 ? 1.f / 256.f : 1.f, gx = exp2i(-a) * 0.0625f * vs;
+  reinterpret_cast<float2 *>(blk)[grp] = make_float2(sb24 ? mark_24bit(gx) : gx, -16.f * (float)sum * vi);
+  return sb24;
 }
 
 // A byte of a metadata word as a float: 2^23 + b, to be fused into an FMA with -2^23 * step.
@@ -370,48 +357,51 @@ constexpr float GEMV_ACC0_F = 12582912.f;
 
 constexpr int GEMV_RING = 4;   // super-blocks in flight per warp
 constexpr int GEMV_CTAS_PER_SM = 3;
-constexpr int GEMV_WARPS = 4;  // warps per CTA: GEMV_WARPS / parts tiles, each split over `parts` warps
-// one stage = one super-block of a 16-row tile: codes (16 rows x 128 B, 128-byte swizzle), the
-// tile's group words [16 rows][16 B], then the first GEMV_XCOPY bytes of the super-block's x block:
-// 8 x (G_x, G_y) and its (hi, mid) x pairs [4 j][2 kinds][8 groups][16 B]
-constexpr int GEMV_ST_CODES = 0, GEMV_ST_GMETA = 2048, GEMV_ST_GSUM = 2304, GEMV_ST_X = 2304 + GEMV_XB_Q;
-constexpr int GEMV_STAGE_BYTES = 4096;      // multiple of 1024 (the swizzle atom)
-constexpr uint32_t GEMV_STAGE_TX = 2048 + 256 + GEMV_XCOPY;
-static_assert(GEMV_ST_GSUM + GEMV_XCOPY <= GEMV_STAGE_BYTES && GEMV_XB_Q + 1024 == GEMV_XCOPY &&
-              GEMV_XB_L + 512 == GEMV_XBLOB && GEMV_XBLOB % 16 == 0, "stage layout");
+constexpr int GEMV_WARPS = 4;     // warps per CTA: four 16-row tiles over the same part of K
+constexpr int GEMV_XSB_MAX = 22;  // super-blocks of x a CTA converts and keeps: its part of K
+// a stage of a warp's ring = one super-block of a 16-row tile: its codes (16 rows x 128 B, 128-byte
+// swizzle) in the codes ring, its group words [16 rows][16 B] in the group-word ring
+constexpr int GEMV_CODES_BYTES = GEMV_WARPS * GEMV_RING * 2048;  // 1024-aligned stages
+constexpr int GEMV_GMETA_BYTES = GEMV_WARPS * GEMV_RING * 256;
+constexpr uint32_t GEMV_STAGE_TX = 2048 + 256;
+static_assert(GEMV_XB_Q + 1024 == GEMV_XCOPY && GEMV_XB_L + 512 == GEMV_XBLOB && GEMV_XBLOB % 16 == 0, "x block");
 constexpr int GEMV_ZERO_BYTES = 1024;       // zero x chunks at a 128-byte stride, for lanes that feed no x
 
 struct GemvTcParams {
   const uint8_t *codes, *gmeta;  // [N][K/2], [N][K/16]: read directly only by the 24-bit tail
   const uint8_t *steps;
   const __nv_bfloat16 *bias;  // [N] or NULL
+  const __nv_bfloat16 *x;     // [K]
   int64_t N, K;
-  SplitK split;  // of K over the warps of the grid, per 16-row tile
-  GemvWorkspace ws;
+  int P;           // parts of K: CTA b takes part b % P of tiles 4 (b / P) .. + 3
+  float *partial;  // P > 1: [tile][part][16 rows], added by gemv_m1_sum_parts
   __nv_bfloat16 *y;
 };
 
-// dynamic shared memory: [warp][stage] (1024-aligned), zero block, mbarriers
+// dynamic shared memory: codes rings (1024-aligned), group-word rings, the CTA's x blocks and their
+// 24-bit flags, zero block, mbarriers
 inline constexpr int gemv_smem_bytes() {
-  return GEMV_WARPS * GEMV_RING * GEMV_STAGE_BYTES + GEMV_ZERO_BYTES + GEMV_WARPS * GEMV_RING * 8 + 1024;
+  return GEMV_CODES_BYTES + GEMV_GMETA_BYTES + GEMV_XSB_MAX * GEMV_XBLOB + 32 + GEMV_ZERO_BYTES +
+         GEMV_WARPS * GEMV_RING * 8 + 1024;
 }
+static_assert(GEMV_CTAS_PER_SM * (gemv_smem_bytes() + 1024) <= 233472, "three CTAs an SM");
 
 // The low bytes of 24-bit x for one warp of the M = 1 kernel: S G_x 2^-8 D_lo per (row, group) of every
 // flagged super-block of its range, the weights read again from global memory (q0, q1: the code rows of
-// rows r0, r1 at the range's first super-block; m0, m1: their group words; st0, st1: their step words;
-// fl: the range's flags).  Flagged super-blocks are rare, so this runs out of line and leaves the
-// streaming loop's registers alone.  Returns the sums to add for rows r0 and r1 (the lane's groups 2c,
-// 2c + 1).
+// rows r0, r1 at the range's first super-block; m0, m1: their group words; st0, st1: their step words)
+// and x from the CTA's blocks in shared memory (xs: the first block; fl: the blocks' 24-bit flags).
+// Flagged super-blocks are rare, so this runs out of line and leaves the streaming loop's registers
+// alone.  Returns the sums to add for rows r0 and r1 (the lane's groups 2c, 2c + 1).
 __device__ __noinline__ float2 gemv_m1_low_bytes(const uint8_t *q0, const uint8_t *q1, const uint8_t *m0,
                                                  const uint8_t *m1, const uint32_t *st0, const uint32_t *st1,
-                                                 const uint8_t *xb_sb, const uint8_t *fl, int nsb) {
+                                                 const uint8_t *xs, const uint8_t *fl, int nsb) {
   const int lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
   const bool on0 = (g == c), feed = on0 || (g == c + 4);
-  const uint2 *xlg = reinterpret_cast<const uint2 *>(xb_sb + GEMV_XB_L) + (on0 ? c : c + 4);
+  const uint2 *xlg = reinterpret_cast<const uint2 *>(xs + GEMV_XB_L) + (on0 ? c : c + 4);
   const int32_t acc_init[4] = {GEMV_ACC0, GEMV_ACC0, GEMV_ACC0, GEMV_ACC0};
   float a0 = 0.f, a1 = 0.f;
   for (int i = 0; i < nsb; ++i) {
-    if (__ldg(fl + (int64_t)i * 16) == 0) continue;  // the same for the whole warp
+    if (fl[i] == 0) continue;  // the same for the whole warp
     const uint4 *c0 = reinterpret_cast<const uint4 *>(q0 + (int64_t)i * 128);
     const uint4 *c1 = reinterpret_cast<const uint4 *>(q1 + (int64_t)i * 128);
     const uint4 v00 = __ldg(c0 + c), v01 = __ldg(c0 + c + 4), v10 = __ldg(c1 + c), v11 = __ldg(c1 + c + 4);
@@ -421,8 +411,8 @@ __device__ __noinline__ float2 gemv_m1_low_bytes(const uint8_t *q0, const uint8_
     int32_t dl[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const uint2 le = feed ? __ldg(lg + 16 * j) : make_uint2(0u, 0u);      // even k
-      const uint2 lo = feed ? __ldg(lg + 16 * j + 8) : make_uint2(0u, 0u);  // odd k
+      const uint2 le = feed ? lg[16 * j] : make_uint2(0u, 0u);      // even k
+      const uint2 lo = feed ? lg[16 * j + 8] : make_uint2(0u, 0u);  // odd k
       const uint32_t h00 = u00[j] & 0xF0F0F0F0u, h10 = u10[j] & 0xF0F0F0F0u;
       const uint32_t h01 = u01[j] & 0xF0F0F0F0u, h11 = u11[j] & 0xF0F0F0F0u;
       const uint32_t e00 = (u00[j] << 4) & 0xF0F0F0F0u, e10 = (u10[j] << 4) & 0xF0F0F0F0u;
@@ -432,7 +422,7 @@ __device__ __noinline__ float2 gemv_m1_low_bytes(const uint8_t *q0, const uint8_
       QL_IMMA("u8", dl, e00, e10, e01, e11, le.x, le.y);
     }
     // (G_x, G_y) of groups 2c, 2c + 1; S = sc * ss per row and group
-    const float4 G = __ldg(reinterpret_cast<const float4 *>(xb_sb + (int64_t)i * GEMV_XBLOB) + c);
+    const float4 G = reinterpret_cast<const float4 *>(xs + (int64_t)i * GEMV_XBLOB)[c];
     const uint32_t cm0 = __ldg(reinterpret_cast<const uint32_t *>(m0 + (int64_t)i * 16) + c);
     const uint32_t cm1 = __ldg(reinterpret_cast<const uint32_t *>(m1 + (int64_t)i * 16) + c);
     const float ss0 = f16_bits_to_f32(__ldg(st0 + i)), ss1 = f16_bits_to_f32(__ldg(st1 + i));
@@ -445,31 +435,40 @@ __device__ __noinline__ float2 gemv_m1_low_bytes(const uint8_t *q0, const uint8_
   return make_float2(a0, a1);
 }
 
-// Everything a super-block needs except its step words arrives by one stage of a per-warp ring:
-// the codes box (TMA, 128-byte swizzle: 16-byte chunk j of row r at chunk j ^ (r & 7)), the group
-// words box (TMA) and the x bytes and group sums (bulk copies), all completing on the stage's
-// mbarrier.  MMA row g (and g + 8) reads tile row pg = (g >> 1) | ((g & 1) << 2), so the two rows of
-// one 8-lane shared-load phase differ in bit 2 and their chunks never share banks.  The loop runs
-// RING super-blocks per turn so every shared-memory offset is a constant; step words come through
-// the L1 cache RING - 1 super-blocks ahead.
+// One CTA = four 16-row tiles over the same part of K.  After the grid it depends on has finished,
+// its warps convert the part's x (GEMV_XSB_MAX super-blocks at most) into shared memory once for all
+// four tiles -- no separate pass, no hand-over between kernels -- while the first stages of the weights,
+// started before that wait, are in flight.  The weights of a super-block arrive by one stage of a
+// per-warp ring: the codes box (TMA, 128-byte swizzle: 16-byte chunk j of row r at chunk j ^ (r & 7))
+// and the group words box (TMA), both completing on the stage's mbarrier.  MMA row g (and g + 8) reads
+// tile row pg = (g >> 1) | ((g & 1) << 2), so the two rows of one 8-lane shared-load phase differ in
+// bit 2 and their chunks never share banks.  The loop runs RING super-blocks per turn so every
+// shared-memory offset inside a stage is a constant; step words come through the L1 cache RING - 1
+// super-blocks ahead.  With K split (P > 1), each part's row sums go to the workspace and a small
+// dependent kernel adds them in part order, so the result does not depend on timing.
 __global__ void __launch_bounds__(32 * GEMV_WARPS, GEMV_CTAS_PER_SM)
     gemv_int4_m1_tc_kernel(const __grid_constant__ CUtensorMap map_codes,
                            const __grid_constant__ CUtensorMap map_gmeta, GemvTcParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t *zero_blk = smem + GEMV_WARPS * GEMV_RING * GEMV_STAGE_BYTES;
+  uint8_t *gm_ring = smem + GEMV_CODES_BYTES;
+  uint8_t *xblk = gm_ring + GEMV_GMETA_BYTES;               // [GEMV_XSB_MAX][GEMV_XBLOB]
+  uint8_t *xflag = xblk + GEMV_XSB_MAX * GEMV_XBLOB;        // [GEMV_XSB_MAX]
+  uint8_t *zero_blk = xflag + 32;
   uint64_t *bars = reinterpret_cast<uint64_t *>(zero_blk + GEMV_ZERO_BYTES);
   __shared__ int abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t n_tiles = (p.N + 15) / 16;
-  int64_t tile, first;
-  int part, P;  // this warp is part `part` of the P splitting its tile's K
-  p.split.locate((int)blockIdx.x * GEMV_WARPS + warp, tile, part, P, first);
+  const int P = p.P;
+  const int part = (int)(blockIdx.x % (unsigned)P);
+  const int64_t tile = (int64_t)(blockIdx.x / (unsigned)P) * GEMV_WARPS + warp;
   const int g = lane >> 2, c = lane & 3;
-  const bool active = tile < n_tiles;  // warps past the split's total have none
+  const bool active = tile < n_tiles;  // warps past the last tile stream nothing
   const int NS = (int)(p.K / 256);
-  const int sb0 = active ? part * NS / P : 0, nsb = active ? (part + 1) * NS / P - sb0 : 0;
-  const uint32_t ring = smem_u32(smem + warp * GEMV_RING * GEMV_STAGE_BYTES);
+  const int sb0 = part * NS / P, nsb = (part + 1) * NS / P - sb0;  // the CTA's part of K
+  const int nsw = active ? nsb : 0;                                // super-blocks this warp streams
+  const uint32_t cring = smem_u32(smem + warp * GEMV_RING * 2048);
+  const uint32_t gring = smem_u32(gm_ring + warp * GEMV_RING * 256);
   const uint32_t bar0 = smem_u32(bars + warp * GEMV_RING);
   if (threadIdx.x == 0) abort_flag = 0;
   for (int t = threadIdx.x; t < GEMV_ZERO_BYTES / 16; t += blockDim.x)
@@ -479,22 +478,17 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS, GEMV_CTAS_PER_SM)
     fence_mbar_init();
   }
   __syncthreads();
-  // the next call's preparation pass may be scheduled as this grid's CTAs retire; it waits for this
-  // grid to finish before touching x or the workspace
+  // the next call's kernel may be scheduled as this grid's CTAs retire; it waits for this grid to
+  // finish before it reads x
   pdl_launch_dependents();
-  const uint8_t *xb_sb = reinterpret_cast<const uint8_t *>(p.ws.xq) + (int64_t)sb0 * GEMV_XBLOB;  // M = 1
-  // stage s of super-block i: weights (codes, group words) need no x; x and sums come after pdl_wait
+  // stage s of super-block i: weights only (codes, group words), independent of x
   auto issue_w = [&](int i, int s) {
-    const uint32_t st = ring + s * GEMV_STAGE_BYTES, bar = bar0 + 8 * s;
+    const uint32_t bar = bar0 + 8 * s;
     mbar_arrive_expect_tx(bar, GEMV_STAGE_TX);
-    tma_load_2d(st + GEMV_ST_CODES, &map_codes, bar, (sb0 + i) * 128, (int32_t)(tile * 16));
-    tma_load_2d(st + GEMV_ST_GMETA, &map_gmeta, bar, (sb0 + i) * 16, (int32_t)(tile * 16));
+    tma_load_2d(cring + s * 2048, &map_codes, bar, (sb0 + i) * 128, (int32_t)(tile * 16));
+    tma_load_2d(gring + s * 256, &map_gmeta, bar, (sb0 + i) * 16, (int32_t)(tile * 16));
   };
-  auto issue_x = [&](int i, int s) {
-    const uint32_t st = ring + s * GEMV_STAGE_BYTES, bar = bar0 + 8 * s;
-    bulk_load(st + GEMV_ST_GSUM, xb_sb + (int64_t)i * GEMV_XBLOB, GEMV_XCOPY, bar);  // sums, then x
-  };
-  const int nis = copies_withheld() ? 0 : nsb;  // super-blocks whose copies this warp starts
+  const int nis = copies_withheld() ? 0 : nsw;  // super-blocks whose copies this warp starts
   const int pre = nis < GEMV_RING - 1 ? nis : GEMV_RING - 1;
   int issued = pre;  // super-blocks whose stage copies were started (lane 0's count is the one used)
   if (lane == 0) {
@@ -518,34 +512,54 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS, GEMV_CTAS_PER_SM)
       sr1[s] = __ldg(st1 + s);
     }
   }
-  pdl_wait();  // x bytes and group sums are ready from here on
-  if (lane == 0)
-    for (int i = 0; i < pre; ++i) issue_x(i, i);
+  // x of the part: thread t of pass k converts group 128 k + t (super-block (128 k + t) / 8)
+  constexpr int XPASS = (8 * GEMV_XSB_MAX + 32 * GEMV_WARPS - 1) / (32 * GEMV_WARPS);
+  const uint4 *xg = reinterpret_cast<const uint4 *>(p.x + (int64_t)sb0 * 256);
+#pragma unroll
+  for (int k = 0; k < XPASS; ++k) {
+    const int q = 32 * GEMV_WARPS * k + (int)threadIdx.x;
+    if (q < 8 * nsb) prefetch_l2(xg + 4 * q);
+  }
+  pdl_wait();  // x may be the output of the kernel launched before this one
+  {
+    uint4 xv[XPASS][4];
+#pragma unroll
+    for (int k = 0; k < XPASS; ++k) {
+      const int q = 32 * GEMV_WARPS * k + (int)threadIdx.x;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) xv[k][e] = q < 8 * nsb ? __ldg(xg + 4 * q + e) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int k = 0; k < XPASS; ++k) {
+      const int q = 32 * GEMV_WARPS * k + (int)threadIdx.x, i = q >> 3;
+      const bool live = q < 8 * nsb;
+      const bool sb24 = gemv_m1_convert_group(xv[k], live, q & 7, xblk + (live ? i : 0) * GEMV_XBLOB);
+      if (live && (q & 7) == 0) xflag[i] = sb24 ? 1 : 0;
+    }
+  }
+  __syncthreads();  // the part's x blocks are complete
 
   // per-lane shared-memory addresses (offsets inside a stage are added as constants)
   const bool on0 = (g == c), on1 = (g == c + 4);
-  const uint32_t zero_a = smem_u32(zero_blk);
-  uint32_t xa[GEMV_RING];  // this lane's B pairs of MMA step (j, kind): (hi, mid) at xa + 128 (2 j + kind)
-#pragma unroll
-  for (int s = 0; s < GEMV_RING; ++s) {
-    xa[s] = on0 ? ring + s * GEMV_STAGE_BYTES + GEMV_ST_X + 16 * c
-          : on1 ? ring + s * GEMV_STAGE_BYTES + GEMV_ST_X + 16 * (c + 4) : zero_a;
-  }
-  const uint32_t a00 = ring + pg * 128 + ((c ^ pg) << 4), a01 = ring + pg * 128 + (((c + 4) ^ pg) << 4);
+  const uint32_t xs0 = smem_u32(xblk);
+  const uint32_t xa0 = on0 ? xs0 + GEMV_XB_Q + 16 * c : on1 ? xs0 + GEMV_XB_Q + 16 * (c + 4) : smem_u32(zero_blk);
+  const uint32_t xstep = (on0 || on1) ? GEMV_XBLOB : 0u;  // lanes that feed no x read the zero block
+  const uint32_t a00 = cring + pg * 128 + ((c ^ pg) << 4), a01 = cring + pg * 128 + (((c + 4) ^ pg) << 4);
   const uint32_t a10 = a00 + 1024, a11 = a01 + 1024;  // row pg + 8: same swizzle phase, next atom
-  const uint32_t ag = ring + GEMV_ST_GSUM + 16 * c;
-  const uint32_t am = ring + GEMV_ST_GMETA + pg * 16 + 4 * c;
+  const uint32_t am = gring + pg * 16 + 4 * c;
+  const uint32_t ag = xs0 + 16 * c;
 
   const int32_t acc_init[4] = {GEMV_ACC0, GEMV_ACC0, GEMV_ACC0, GEMV_ACC0};
   float acc0 = 0.f, acc1 = 0.f;
   uint32_t x24s = 0u;  // bit 0: some super-block's G_x carries the 24-bit marker
   bool ok = true;
-  for (int base = 0; base < nsb && ok; base += GEMV_RING) {
+  for (int base = 0; base < nsw && ok; base += GEMV_RING) {
     const uint32_t par = (uint32_t)((base / GEMV_RING) & 1);
+    const uint32_t xt = xa0 + (uint32_t)base * xstep, gt = ag + (uint32_t)base * GEMV_XBLOB;
 #pragma unroll
     for (int s = 0; s < GEMV_RING; ++s) {
       const int i = base + s;
-      if (i >= nsb) break;
+      if (i >= nsw) break;
       // refill the stage released by the previous super-block with super-block i + RING - 1
       const int nx = i + GEMV_RING - 1;
       const int sn = (s + GEMV_RING - 1) % GEMV_RING;
@@ -553,7 +567,6 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS, GEMV_CTAS_PER_SM)
       if (nx < nis) {
         if (lane == 0) {
           issue_w(nx, sn);
-          issue_x(nx, sn);
           issued = nx + 1;
         }
         sr0[sn] = __ldg(st0 + nx);
@@ -563,18 +576,19 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS, GEMV_CTAS_PER_SM)
         ok = false;
         break;
       }
-      const uint32_t so = s * GEMV_STAGE_BYTES;
+      const uint32_t so = s * 2048, sg = s * 256;
       const uint4 w00 = lds128(a00 + so), w10 = lds128(a10 + so);  // (r0 | r1, group c)
       const uint4 w01 = lds128(a01 + so), w11 = lds128(a11 + so);  // (r0 | r1, group c+4)
-      const float4 G = lds128f(ag + so);                           // (G_x, G_y) of groups 2c, 2c+1
-      const uint32_t cm0 = lds32(am + so), cm1 = lds32(am + so + 128);
+      const float4 G = lds128f(gt + s * GEMV_XBLOB);               // (G_x, G_y) of groups 2c, 2c+1
+      const uint32_t cm0 = lds32(am + sg), cm1 = lds32(am + sg + 128);
+      const uint32_t xi = xt + (uint32_t)s * xstep;
       const uint32_t ww00[4] = {w00.x, w00.y, w00.z, w00.w}, ww01[4] = {w01.x, w01.y, w01.z, w01.w};
       const uint32_t ww10[4] = {w10.x, w10.y, w10.z, w10.w}, ww11[4] = {w11.x, w11.y, w11.z, w11.w};
       // D[q]: q = 0 (r0, group 2c), 1 (r0, 2c+1), 2 (r1, 2c), 3 (r1, 2c+1); T = 256 D_hi + D_mid
       int32_t dh[4], dm[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const uint4 xe = lds128(xa[s] + 256 * j), xo = lds128(xa[s] + 256 * j + 128);  // even k, odd k
+        const uint4 xe = lds128(xi + 256 * j), xo = lds128(xi + 256 * j + 128);  // even k, odd k
         const uint32_t h00 = ww00[j] & 0xF0F0F0F0u, h10 = ww10[j] & 0xF0F0F0F0u;  // odd k, x16
         const uint32_t h01 = ww01[j] & 0xF0F0F0F0u, h11 = ww11[j] & 0xF0F0F0F0u;
         if (j == 0) {
@@ -623,8 +637,7 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS, GEMV_CTAS_PER_SM)
     const float2 lb = gemv_m1_low_bytes(p.codes + r0 * (p.K / 2) + (int64_t)sb0 * 128,
                                         p.codes + r1 * (p.K / 2) + (int64_t)sb0 * 128,
                                         p.gmeta + r0 * (p.K / 16) + (int64_t)sb0 * 16,
-                                        p.gmeta + r1 * (p.K / 16) + (int64_t)sb0 * 16, st0, st1, xb_sb,
-                                        p.ws.flags + (int64_t)sb0 * 16, nsb);
+                                        p.gmeta + r1 * (p.K / 16) + (int64_t)sb0 * 16, st0, st1, xblk, xflag, nsw);
     acc0 += lb.x;
     acc1 += lb.y;
   }
@@ -633,36 +646,37 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS, GEMV_CTAS_PER_SM)
   acc0 += __shfl_xor_sync(0xffffffffu, acc0, 2);
   acc1 += __shfl_xor_sync(0xffffffffu, acc1, 1);
   acc1 += __shfl_xor_sync(0xffffffffu, acc1, 2);
-  if (!active) return;
   if (P == 1) {
-    if (c == 0) {
+    if (active && ok && c == 0) {
       const int64_t ra = tile * 16 + pg, rb = ra + 8;
       if (ra < p.N) p.y[ra] = __float2bfloat16_rn(acc0 + bias_at(p.bias, ra));
       if (rb < p.N) p.y[rb] = __float2bfloat16_rn(acc1 + bias_at(p.bias, rb));
     }
     return;
   }
-  // K split over warps of (possibly) different CTAs: publish this part's sums; the warp that
-  // finishes the tile last adds the P parts in part order, so the result does not depend on timing
-  float *part_sums = p.ws.partial + first * 16;
+  // K split: this part's sums of the tile's rows go to the workspace; gemv_m1_sum_parts, the dependent
+  // launch after this grid, adds the P parts in part order
+  if (!active) return;
   {  // lane r < 16 stores the sum of tile row r (held by lane 4g with pg(g) = r mod 8)
     const int rr = lane & 15, prow = rr & 7;
     const int src = 4 * (((prow & 3) << 1) | (prow >> 2));
     const float v0 = __shfl_sync(0xffffffffu, acc0, src), v1 = __shfl_sync(0xffffffffu, acc1, src);
-    if (lane < 16) part_sums[part * 16 + rr] = rr < 8 ? v0 : v1;
+    if (lane < 16) p.partial[(tile * P + part) * 16 + rr] = rr < 8 ? v0 : v1;
   }
-  __syncwarp();  // the stores above precede lane 0's release
-  int last = 0;
-  if (lane == 0) last = atomic_add_acq_rel_gpu(p.ws.counters + tile, 1) == P - 1;
-  last = __shfl_sync(0xffffffffu, last, 0);
-  if (!last) return;
-  __syncwarp();  // lane 0's acquire precedes every lane's reads of the other parts
-  if (lane < 16) {
-    float sum = 0.f;
-    for (int q = 0; q < P; ++q) sum += __ldcg(part_sums + q * 16 + lane);
-    const int64_t r = tile * 16 + lane;
-    if (r < p.N) p.y[r] = __float2bfloat16_rn(sum + bias_at(p.bias, r));
-  }
+}
+
+// The parts of a K split of the M = 1 kernel, added in part order: one thread per output row.  Launched
+// as a programmatic dependent of that kernel (it lets the next kernel start, then waits for the parts).
+__global__ void __launch_bounds__(256) gemv_m1_sum_parts(const float *partial, int P, int64_t N,
+                                                         const __nv_bfloat16 *bias, __nv_bfloat16 *y) {
+  pdl_launch_dependents();
+  const int64_t r = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  pdl_wait();
+  if (r >= N) return;
+  const float *src = partial + (r >> 4) * P * 16 + (r & 15);
+  float sum = 0.f;
+  for (int q = 0; q < P; ++q) sum += src[q * 16];
+  y[r] = __float2bfloat16_rn(sum + bias_at(bias, r));
 }
 
 

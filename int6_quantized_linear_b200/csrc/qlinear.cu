@@ -440,39 +440,24 @@ ql_status launch_gemv(const ql_desc *d, const ql_packed_const *w, const void *x,
     }
   }
   if constexpr (FMT == FMT_INT4) {
-    if (M == 1) {  // tensor-core path: preparation pass, then the streaming kernel as its dependent
+    if (M == 1) {  // each CTA converts its part of x, then streams four 16-row tiles over it (+ the parts' sum)
+      const int64_t NS = d->K / 256, n_tiles = (d->N + 15) / 16, groups = (n_tiles + GEMV_WARPS - 1) / GEMV_WARPS;
+      // split K so that the tile groups fill the resident CTA slots, and so that each part's x fits the
+      // CTA's blocks; the parts' sums go through the workspace (16 floats a tile and part)
+      int64_t P = std::max<int64_t>(1, std::min<int64_t>(NS, (int64_t)sms * GEMV_CTAS_PER_SM / groups));
+      P = std::max<int64_t>(P, (NS + GEMV_XSB_MAX - 1) / GEMV_XSB_MAX);
+      if (P > 1 && groups * GEMV_WARPS * P * 16 > (int64_t)GEMV_MT_MAX_CTAS * 64) return QL_ERR_RANGE;
       const GemvWorkspace ws = gemv_workspace_carve(workspace, M, d->N, d->K);
-      const int64_t ng = M * (d->K / 32);
-      const int64_t NS = d->K / 256, n_tiles = (d->N + 15) / 16;
-      // split K over the warps of a 16-row tile so that the tiles fill the resident warp slots; the
-      // parts' sums go through the workspace (16 floats a warp: at most the slots' 16 * 1776 of its
-      // GEMV_MT_MAX_CTAS * 64)
-      const SplitK split = split_k(n_tiles, (int64_t)sms * GEMV_CTAS_PER_SM * GEMV_WARPS, NS, false);
-      const bool splits = split.P + (split.extra > 0) > 1;
-      if (splits && split.total(n_tiles) * 16 > (int64_t)GEMV_MT_MAX_CTAS * 64) return QL_ERR_RANGE;
-      const int64_t n_counters = splits ? n_tiles : 0;
-      {  // programmatic dependent of whatever precedes it on the stream (it waits before reading x)
-        const int64_t threads = std::max<int64_t>(4 * ng, n_counters);  // four lanes per group
-        cudaLaunchConfig_t pc = {};
-        pc.gridDim = dim3((unsigned)((threads + 255) / 256));
-        pc.blockDim = dim3(256);
-        pc.stream = st;
-        cudaLaunchAttribute pa[1];
-        pa[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        pa[0].val.programmaticStreamSerializationAllowed = 1;
-        pc.attrs = pa;
-        pc.numAttrs = 1;
-        if (cudaLaunchKernelEx(&pc, gemv_xprep_kernel, xb, M, (int64_t)d->K, n_counters, ws) != cudaSuccess)
-          return cuda_failed();
-      }
       GemvTcParams p;
       p.codes = static_cast<const uint8_t *>(w->codes);
       p.gmeta = static_cast<const uint8_t *>(w->gmeta);
       p.steps = static_cast<const uint8_t *>(w->steps);
       p.bias = bb;
+      p.x = xb;
       p.N = d->N;
       p.K = d->K;
-      p.ws = ws;
+      p.P = (int)P;
+      p.partial = ws.partial;
       p.y = yb;
       CUtensorMap mc, mg;  // codes as [N][K/2] bytes, boxes of 16 rows x 128 bytes, 128-byte swizzle;
                            // group words as [N][K/16] bytes, boxes of 16 rows x 16 bytes
@@ -481,7 +466,6 @@ ql_status launch_gemv(const ql_desc *d, const ql_packed_const *w, const void *x,
           !encode_2d(&mg, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->gmeta, (uint64_t)d->K / 16, (uint64_t)d->N,
                      (uint64_t)d->K / 16, 16, 16, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cuda_failed();
-      p.split = split;
       static thread_local int configured_dev = -1;
       int dev = 0;
       cudaGetDevice(&dev);
@@ -492,16 +476,27 @@ ql_status launch_gemv(const ql_desc *d, const ql_packed_const *w, const void *x,
         configured_dev = dev;
       }
       cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3((unsigned)((split.total(n_tiles) + GEMV_WARPS - 1) / GEMV_WARPS));
+      cfg.gridDim = dim3((unsigned)(groups * P));
       cfg.blockDim = dim3(32 * GEMV_WARPS);
       cfg.dynamicSmemBytes = gemv_smem_bytes();
       cfg.stream = st;
       cudaLaunchAttribute attr[1];
-      attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // programmatic dependent of whatever precedes it
       attr[0].val.programmaticStreamSerializationAllowed = 1;
       cfg.attrs = attr;
       cfg.numAttrs = 1;
       if (cudaLaunchKernelEx(&cfg, gemv_int4_m1_tc_kernel, mc, mg, p) != cudaSuccess) return cuda_failed();
+      if (P > 1) {  // the parts' sums, added by the kernel that depends on this one
+        cudaLaunchConfig_t rc = {};
+        rc.gridDim = dim3((unsigned)((d->N + 255) / 256));
+        rc.blockDim = dim3(256);
+        rc.stream = st;
+        rc.attrs = attr;
+        rc.numAttrs = 1;
+        if (cudaLaunchKernelEx(&rc, gemv_m1_sum_parts, (const float *)ws.partial, (int)P, (int64_t)d->N, bb, yb) !=
+            cudaSuccess)
+          return cuda_failed();
+      }
       return launched();
     }
   }
