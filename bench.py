@@ -39,8 +39,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM bytes per GEMV launch from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum),
 # valid only while the GEMV source is unchanged (hash of csrc/gemv.cuh at capture time).
-NCU_TRAFFIC = {"gemv_src_sha256": "5851b5cb8872c942c39e8b2aa4402a168f73f18aff8127599745241a6825d466",
-               "bytes_per_launch": 83032576}  # mean over the two decode layers
+NCU_TRAFFIC = {"gemv_src_sha256": "e7ad75c8117363d2807c221a4c7e589273cc8b5edeba74ddf0e814efe6303860",
+               "bytes_per_launch": 83041280}  # mean over the two decode layers
 
 
 def parse_args(argv=None):
@@ -256,7 +256,9 @@ def _ev():
 
 
 def capture(fn, device):
-    """Record fn()'s launches into a CUDA graph (replayed on the current stream)."""
+    """Record fn()'s launches into a CUDA graph (replayed on the current stream) and upload it to the
+    device: the first launch of an executable graph otherwise uploads it first, a one-time cost
+    (measured about 120 us for the 20-step decode graph) that belongs to no step."""
     import torch
     side = torch.cuda.Stream(device)
     side.wait_stream(torch.cuda.current_stream(device))
@@ -264,12 +266,18 @@ def capture(fn, device):
     with torch.cuda.graph(g, stream=side):
         fn()
     torch.cuda.current_stream(device).wait_stream(side)
+    import cuda.bindings.runtime as cudart
+    err, = cudart.cudaGraphUpload(g.raw_cuda_graph_exec(), torch.cuda.current_stream(device).cuda_stream)
+    if err != cudart.cudaError_t.cudaSuccess:
+        raise RuntimeError(f"cudaGraphUpload: {err}")
+    torch.cuda.synchronize(device)
     return g
 
 
-def per_launch_us(layers, ql, device, calls=30):
-    """Mean device time of one qlinear_gemv call per layer: a graph of `calls` calls over the
-    rotating copies, replayed twice between CUDA events on the launching stream."""
+def per_launch_us(layers, ql, device, calls=30, reps=5):
+    """Device time of one qlinear_gemv call per layer: a graph of `calls` calls over the rotating
+    copies, replayed `reps` times, each replay between CUDA events on the launching stream; the
+    median replay's time per call."""
     import torch
     out = []
     for L in layers:
@@ -280,13 +288,15 @@ def per_launch_us(layers, ql, device, calls=30):
         gr = capture(body, device)
         gr.replay()
         torch.cuda.synchronize(device)
-        a, b = _ev(), _ev()
-        a.record()
-        gr.replay()
-        gr.replay()
-        b.record()
-        torch.cuda.synchronize(device)
-        out.append(a.elapsed_time(b) * 1e3 / (2 * calls))
+        times = []
+        for _ in range(reps):
+            a, b = _ev(), _ev()
+            a.record()
+            gr.replay()
+            b.record()
+            torch.cuda.synchronize(device)
+            times.append(a.elapsed_time(b) * 1e3 / calls)
+        out.append(sorted(times)[reps // 2])
         del gr
     return out
 
