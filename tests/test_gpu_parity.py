@@ -107,6 +107,21 @@ def test_gemv_full_size_sampled(cuda, name):
         assert_close(y[:, rows], y_ref, f"gemv {name} M={M}")
 
 
+@pytest.mark.parametrize("N,K", [(14400, 6144), (16384, 11520), (5000, 256)])
+def test_gemv_int4_m1_part_sizes(cuda, N, K):
+    """int4 at M=1 where the parts of K are set by how much x a CTA holds (at most 22 super-blocks):
+    K = 6144 and 11520 with enough rows to fill every CTA slot unsplit still split K in two and
+    three parts; K = 256 is a single super-block.  Sampled rows (all of them for the last case)
+    checked against the oracle, bits repeatable."""
+    L = Layer("int4", N, K, seed=N + K)
+    rows = _sampled_rows(N, 384, N) if N * K > 4_000_000 else np.arange(N)
+    w_ref = L.oracle_w(rows)
+    xb, xd = x_dev(K, 1, seed=K + 5)
+    y = run_gemv(L, xd, 1)
+    assert_close(y[:, rows], OC.matmul_f64(xb, w_ref), f"int4 M=1 N={N} K={K}")
+    assert np.array_equal(y, run_gemv(L, xd, 1))
+
+
 @pytest.mark.parametrize("M", [512, 2048, 8192])
 def test_gemm_full_size_sampled(cuda, M):
     wl = synth.WORKLOADS["int4_gemm_k5120_n27648"]
