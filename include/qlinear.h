@@ -229,8 +229,9 @@ ql_status qlinear_gemv_workspace_bytes(const ql_desc *desc, int64_t M, size_t *b
  * fp32 scales and accumulation, one nearest-even rounding to bf16 at the end.
  * 1 <= M <= 8 for int4 / int6; 1 <= M <= 32 for affine.
  *  - Tensor-core path (int4 and int6 at every M; affine with group 32 or 64
- *    and K % 256 == 0 at M <= 8): two launches (int4 at M = 1: one, plus a
- *    short kernel that adds the parts when K is split).  Each x
+ *    and K % 256 == 0 at M <= 8): two launches (int4 and 4-bit affine at
+ *    M = 1: one, plus a short kernel that adds the parts when K is split).
+ *    Each x
  *    group (32 elements; 16 for int6) is turned into fixed point, x_int = rint(x *
  *    2^a): 16-bit (the group's max |x| scaled into [2^14, 2^15): exact for
  *    every bf16 element within 2^7 of the group's largest magnitude), or
@@ -239,7 +240,8 @@ ql_status qlinear_gemv_workspace_bytes(const ql_desc *desc, int64_t M, size_t *b
  *    exceeds 2^-12 of its mass outside its largest element; split into high,
  *    middle and (24-bit) low bytes in the order the tensor-core fragments
  *    read them, with the group's scale (and sum) -- by a short pass, or, for
- *    int4 at M = 1, by each CTA of the streaming kernel for its part of K,
+ *    int4 and 4-bit affine (group 32 / 64) at M = 1, by each CTA of the
+ *    streaming kernel for its part of K,
  *    into shared memory (K split into parts of at most 22 super-blocks,
  *    16 partial sums a part and 16 rows within the workspace's 4*4096*64
  *    bytes; QL_ERR_RANGE beyond); then the streaming kernel
@@ -248,9 +250,10 @@ ql_status qlinear_gemv_workspace_bytes(const ql_desc *desc, int64_t M, size_t *b
  *    (mma.sync m16n8k32, exact s32 sums, one MMA per byte: high and middle
  *    in the streaming loop, the low bytes of 24-bit super-blocks in a pass
  *    after it that reads their weights again) and applies scale (and zero
- *    or bias) once per (row, group[, token]) in fp32.  int4 at M =
- *    1 and int6 use a diagonal x operand (one MMA column per weight group);
- *    int4 at M >= 2 and affine use the tokens as MMA columns.  K may be split
+ *    or bias) once per (row, group[, token]) in fp32.  int4 and 4-bit
+ *    affine at M = 1 and int6 use a diagonal x operand (one MMA column per
+ *    weight group); int4 at M >= 2 and the other affine calls use the tokens
+ *    as MMA columns.  K may be split
  *    over warps or CTAs, the parts added in a fixed order through the
  *    workspace.
  *  - Affine with group 32 or 64 and K % 256 == 0 at 9 <= M <= 32: two

@@ -111,8 +111,8 @@ __global__ void __launch_bounds__(256) gemv_simple_kernel(WeightPtrs p, int64_t 
 
 constexpr int GEMV_MT_MAX_CTAS = 4096;  // bound on the CTAs of one multi-token launch (sizes its partial sums)
 
-// The split of K over parts (warps of the M = 1 kernel, CTAs of the others): units -- 16-row tiles or
-// 64-row groups -- 0 .. extra - 1 take P + 1 parts and the rest P, so that units x parts can match
+// The split of K over the CTAs of the multi-token and int6 GEMVs: units -- 64-row groups -- 0 .. extra - 1
+// take P + 1 parts and the rest P, so that units x parts can match
 // the resident slots exactly and no SM idles while the others stream.  Part w of the grid belongs to
 // unit `unit`, is its part `part` of `pu`, and the unit's parts start at grid index `first`.
 struct SplitK {
@@ -358,43 +358,51 @@ constexpr float GEMV_ACC0_F = 12582912.f;
 constexpr int GEMV_RING = 4;   // super-blocks in flight per warp
 constexpr int GEMV_CTAS_PER_SM = 3;
 constexpr int GEMV_WARPS = 4;     // warps per CTA: four 16-row tiles over the same part of K
-constexpr int GEMV_XSB_MAX = 22;  // super-blocks of x a CTA converts and keeps: its part of K
 // a stage of a warp's ring = one super-block of a 16-row tile: its codes (16 rows x 128 B, 128-byte
-// swizzle) in the codes ring, its group words [16 rows][16 B] in the group-word ring
-constexpr int GEMV_CODES_BYTES = GEMV_WARPS * GEMV_RING * 2048;  // 1024-aligned stages
-constexpr int GEMV_GMETA_BYTES = GEMV_WARPS * GEMV_RING * 256;
-constexpr uint32_t GEMV_STAGE_TX = 2048 + 256;
+// swizzle) in the codes ring, its group words in the group-word ring: int4 16 B a row (u16 sc | zc per
+// group; the step words come through L1), 4-bit affine 4 (256 / G) B a row ((s, b) bf16 per group)
 static_assert(GEMV_XB_Q + 1024 == GEMV_XCOPY && GEMV_XB_L + 512 == GEMV_XBLOB && GEMV_XBLOB % 16 == 0, "x block");
-constexpr int GEMV_ZERO_BYTES = 1024;       // zero x chunks at a 128-byte stride, for lanes that feed no x
+constexpr int GEMV_ZERO_BYTES = 1024;  // zero x chunks at a 128-byte stride, for lanes that feed no x
+
+template <int FMT, int G>
+struct M1Layout {
+  static constexpr int GM_ROW = FMT == FMT_INT4 ? 16 : 4 * (256 / G);
+  static constexpr int GM_STAGE = 16 * GM_ROW;
+  static constexpr int XSB_MAX = GM_ROW > 16 ? 20 : 22;  // super-blocks of x a CTA converts and keeps
+  static constexpr int CODES_BYTES = GEMV_WARPS * GEMV_RING * 2048;  // 1024-aligned stages
+  static constexpr int GMETA_BYTES = GEMV_WARPS * GEMV_RING * GM_STAGE;
+  static constexpr uint32_t STAGE_TX = 2048 + GM_STAGE;
+  // dynamic shared memory: codes rings, group-word rings, the CTA's x blocks and their 24-bit flags,
+  // zero block, mbarriers
+  static constexpr int SMEM = CODES_BYTES + GMETA_BYTES + XSB_MAX * GEMV_XBLOB + 32 + GEMV_ZERO_BYTES +
+                              GEMV_WARPS * GEMV_RING * 8 + 1024;
+  static_assert(GEMV_CTAS_PER_SM * (SMEM + 1024) <= 233472, "three CTAs an SM");
+};
 
 struct GemvTcParams {
-  const uint8_t *codes, *gmeta;  // [N][K/2], [N][K/16]: read directly only by the 24-bit tail
-  const uint8_t *steps;
-  const __nv_bfloat16 *bias;  // [N] or NULL
-  const __nv_bfloat16 *x;     // [K]
+  const uint8_t *codes, *gmeta;  // [N][K/2], group words [N][K/16] (int4) or [N][4K/G]: read directly only
+                                 // by the 24-bit tail
+  const uint8_t *steps;          // int4: [N][K/256] step words
+  const __nv_bfloat16 *bias;     // [N] or NULL
+  const __nv_bfloat16 *x;        // [K]
   int64_t N, K;
   int P;           // parts of K: CTA b takes part b % P of tiles 4 (b / P) .. + 3
   float *partial;  // P > 1: [tile][part][16 rows], added by gemv_m1_sum_parts
   __nv_bfloat16 *y;
 };
 
-// dynamic shared memory: codes rings (1024-aligned), group-word rings, the CTA's x blocks and their
-// 24-bit flags, zero block, mbarriers
-inline constexpr int gemv_smem_bytes() {
-  return GEMV_CODES_BYTES + GEMV_GMETA_BYTES + GEMV_XSB_MAX * GEMV_XBLOB + 32 + GEMV_ZERO_BYTES +
-         GEMV_WARPS * GEMV_RING * 8 + 1024;
-}
-static_assert(GEMV_CTAS_PER_SM * (gemv_smem_bytes() + 1024) <= 233472, "three CTAs an SM");
-
-// The low bytes of 24-bit x for one warp of the M = 1 kernel: S G_x 2^-8 D_lo per (row, group) of every
-// flagged super-block of its range, the weights read again from global memory (q0, q1: the code rows of
-// rows r0, r1 at the range's first super-block; m0, m1: their group words; st0, st1: their step words)
-// and x from the CTA's blocks in shared memory (xs: the first block; fl: the blocks' 24-bit flags).
-// Flagged super-blocks are rare, so this runs out of line and leaves the streaming loop's registers
-// alone.  Returns the sums to add for rows r0 and r1 (the lane's groups 2c, 2c + 1).
+// The low bytes of 24-bit x for one warp of the M = 1 kernel: S G_x 2^-8 D_lo per (row, 32-k slice) of
+// every flagged super-block of its range (S = sc ss for int4, the group's s for affine), the weights read
+// again from global memory (q0, q1: the code rows of rows r0, r1 at the range's first super-block;
+// m0, m1: their group words; st0, st1: int4 step words) and x from the CTA's blocks in shared memory
+// (xs: the first block; fl: the blocks' 24-bit flags).  Flagged super-blocks are rare, so this runs out
+// of line and leaves the streaming loop's registers alone.  Returns the sums to add for rows r0 and r1
+// (the lane's slices 2c, 2c + 1).
+template <int FMT, int G>
 __device__ __noinline__ float2 gemv_m1_low_bytes(const uint8_t *q0, const uint8_t *q1, const uint8_t *m0,
                                                  const uint8_t *m1, const uint32_t *st0, const uint32_t *st1,
                                                  const uint8_t *xs, const uint8_t *fl, int nsb) {
+  constexpr int GM_ROW = M1Layout<FMT, G>::GM_ROW;
   const int lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
   const bool on0 = (g == c), feed = on0 || (g == c + 4);
   const uint2 *xlg = reinterpret_cast<const uint2 *>(xs + GEMV_XB_L) + (on0 ? c : c + 4);
@@ -422,15 +430,29 @@ __device__ __noinline__ float2 gemv_m1_low_bytes(const uint8_t *q0, const uint8_
       QL_IMMA("u8", dl, e00, e10, e01, e11, le.x, le.y);
     }
     // (G_x, G_y) of groups 2c, 2c + 1; S = sc * ss per row and group
-    const float4 G = reinterpret_cast<const float4 *>(xs + (int64_t)i * GEMV_XBLOB)[c];
-    const uint32_t cm0 = __ldg(reinterpret_cast<const uint32_t *>(m0 + (int64_t)i * 16) + c);
-    const uint32_t cm1 = __ldg(reinterpret_cast<const uint32_t *>(m1 + (int64_t)i * 16) + c);
-    const float ss0 = f16_bits_to_f32(__ldg(st0 + i)), ss1 = f16_bits_to_f32(__ldg(st1 + i));
-    const float gx0 = unmark(G.x) * (1.f / 256.f), gx1 = unmark(G.z) * (1.f / 256.f);
-    a0 = fmaf(fmaf(byte_magic(cm0, 0), ss0, -8388608.f * ss0) * gx0, __int_as_float(dl[0]) - GEMV_ACC0_F, a0);
-    a0 = fmaf(fmaf(byte_magic(cm0, 2), ss0, -8388608.f * ss0) * gx1, __int_as_float(dl[1]) - GEMV_ACC0_F, a0);
-    a1 = fmaf(fmaf(byte_magic(cm1, 0), ss1, -8388608.f * ss1) * gx0, __int_as_float(dl[2]) - GEMV_ACC0_F, a1);
-    a1 = fmaf(fmaf(byte_magic(cm1, 2), ss1, -8388608.f * ss1) * gx1, __int_as_float(dl[3]) - GEMV_ACC0_F, a1);
+    const float4 Gx = reinterpret_cast<const float4 *>(xs + (int64_t)i * GEMV_XBLOB)[c];
+    const float gx0 = unmark(Gx.x) * (1.f / 256.f), gx1 = unmark(Gx.z) * (1.f / 256.f);
+    float s0a, s0b, s1a, s1b;  // the scales of slices 2c, 2c + 1 for rows r0, r1
+    if constexpr (FMT == FMT_INT4) {
+      const uint32_t cm0 = __ldg(reinterpret_cast<const uint32_t *>(m0 + (int64_t)i * GM_ROW) + c);
+      const uint32_t cm1 = __ldg(reinterpret_cast<const uint32_t *>(m1 + (int64_t)i * GM_ROW) + c);
+      const float ss0 = f16_bits_to_f32(__ldg(st0 + i)), ss1 = f16_bits_to_f32(__ldg(st1 + i));
+      s0a = fmaf(byte_magic(cm0, 0), ss0, -8388608.f * ss0);
+      s0b = fmaf(byte_magic(cm0, 2), ss0, -8388608.f * ss0);
+      s1a = fmaf(byte_magic(cm1, 0), ss1, -8388608.f * ss1);
+      s1b = fmaf(byte_magic(cm1, 2), ss1, -8388608.f * ss1);
+    } else {  // slice 2c + h lies in group (2c + h) * 32 / G
+      const uint32_t *w0 = reinterpret_cast<const uint32_t *>(m0 + (int64_t)i * GM_ROW);
+      const uint32_t *w1 = reinterpret_cast<const uint32_t *>(m1 + (int64_t)i * GM_ROW);
+      s0a = bf16_bits_to_f32(__ldg(w0 + 2 * c * 32 / G));
+      s0b = bf16_bits_to_f32(__ldg(w0 + (2 * c + 1) * 32 / G));
+      s1a = bf16_bits_to_f32(__ldg(w1 + 2 * c * 32 / G));
+      s1b = bf16_bits_to_f32(__ldg(w1 + (2 * c + 1) * 32 / G));
+    }
+    a0 = fmaf(s0a * gx0, __int_as_float(dl[0]) - GEMV_ACC0_F, a0);
+    a0 = fmaf(s0b * gx1, __int_as_float(dl[1]) - GEMV_ACC0_F, a0);
+    a1 = fmaf(s1a * gx0, __int_as_float(dl[2]) - GEMV_ACC0_F, a1);
+    a1 = fmaf(s1b * gx1, __int_as_float(dl[3]) - GEMV_ACC0_F, a1);
   }
   return make_float2(a0, a1);
 }
@@ -446,14 +468,16 @@ __device__ __noinline__ float2 gemv_m1_low_bytes(const uint8_t *q0, const uint8_
 // shared-memory offset inside a stage is a constant; step words come through the L1 cache RING - 1
 // super-blocks ahead.  With K split (P > 1), each part's row sums go to the workspace and a small
 // dependent kernel adds them in part order, so the result does not depend on timing.
-__global__ void __launch_bounds__(32 * GEMV_WARPS, GEMV_CTAS_PER_SM)
-    gemv_int4_m1_tc_kernel(const __grid_constant__ CUtensorMap map_codes,
-                           const __grid_constant__ CUtensorMap map_gmeta, GemvTcParams p) {
+template <int FMT, int G>
+__device__ __forceinline__ void gemv_m1_body(const CUtensorMap &map_codes, const CUtensorMap &map_gmeta,
+                                             const GemvTcParams &p) {
+  using L = M1Layout<FMT, G>;
+  constexpr int GM_ROW = L::GM_ROW;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t *gm_ring = smem + GEMV_CODES_BYTES;
-  uint8_t *xblk = gm_ring + GEMV_GMETA_BYTES;               // [GEMV_XSB_MAX][GEMV_XBLOB]
-  uint8_t *xflag = xblk + GEMV_XSB_MAX * GEMV_XBLOB;        // [GEMV_XSB_MAX]
+  uint8_t *gm_ring = smem + L::CODES_BYTES;
+  uint8_t *xblk = gm_ring + L::GMETA_BYTES;                 // [XSB_MAX][GEMV_XBLOB]
+  uint8_t *xflag = xblk + L::XSB_MAX * GEMV_XBLOB;          // [XSB_MAX]
   uint8_t *zero_blk = xflag + 32;
   uint64_t *bars = reinterpret_cast<uint64_t *>(zero_blk + GEMV_ZERO_BYTES);
   __shared__ int abort_flag;
@@ -468,7 +492,7 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS, GEMV_CTAS_PER_SM)
   const int sb0 = part * NS / P, nsb = (part + 1) * NS / P - sb0;  // the CTA's part of K
   const int nsw = active ? nsb : 0;                                // super-blocks this warp streams
   const uint32_t cring = smem_u32(smem + warp * GEMV_RING * 2048);
-  const uint32_t gring = smem_u32(gm_ring + warp * GEMV_RING * 256);
+  const uint32_t gring = smem_u32(gm_ring + warp * GEMV_RING * L::GM_STAGE);
   const uint32_t bar0 = smem_u32(bars + warp * GEMV_RING);
   if (threadIdx.x == 0) abort_flag = 0;
   for (int t = threadIdx.x; t < GEMV_ZERO_BYTES / 16; t += blockDim.x)
@@ -484,9 +508,9 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS, GEMV_CTAS_PER_SM)
   // stage s of super-block i: weights only (codes, group words), independent of x
   auto issue_w = [&](int i, int s) {
     const uint32_t bar = bar0 + 8 * s;
-    mbar_arrive_expect_tx(bar, GEMV_STAGE_TX);
+    mbar_arrive_expect_tx(bar, L::STAGE_TX);
     tma_load_2d(cring + s * 2048, &map_codes, bar, (sb0 + i) * 128, (int32_t)(tile * 16));
-    tma_load_2d(gring + s * 256, &map_gmeta, bar, (sb0 + i) * 16, (int32_t)(tile * 16));
+    tma_load_2d(gring + s * L::GM_STAGE, &map_gmeta, bar, (sb0 + i) * GM_ROW, (int32_t)(tile * 16));
   };
   const int nis = copies_withheld() ? 0 : nsw;  // super-blocks whose copies this warp starts
   const int pre = nis < GEMV_RING - 1 ? nis : GEMV_RING - 1;
@@ -502,18 +526,18 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS, GEMV_CTAS_PER_SM)
   if (r1 >= p.N) r1 = p.N - 1;
   const uint32_t *st0 = reinterpret_cast<const uint32_t *>(p.steps) + r0 * NS + sb0;
   const uint32_t *st1 = reinterpret_cast<const uint32_t *>(p.steps) + r1 * NS + sb0;
-  uint32_t sr0[GEMV_RING], sr1[GEMV_RING];  // step words of the next RING - 1 super-blocks, by stage
+  uint32_t sr0[GEMV_RING], sr1[GEMV_RING];  // int4 step words of the next RING - 1 super-blocks, by stage
 #pragma unroll
   for (int s = 0; s < GEMV_RING; ++s) {
     sr0[s] = 0u;
     sr1[s] = 0u;
-    if (s < pre) {
+    if (FMT == FMT_INT4 && s < pre) {
       sr0[s] = __ldg(st0 + s);
       sr1[s] = __ldg(st1 + s);
     }
   }
   // x of the part: thread t of pass k converts group 128 k + t (super-block (128 k + t) / 8)
-  constexpr int XPASS = (8 * GEMV_XSB_MAX + 32 * GEMV_WARPS - 1) / (32 * GEMV_WARPS);
+  constexpr int XPASS = (8 * L::XSB_MAX + 32 * GEMV_WARPS - 1) / (32 * GEMV_WARPS);
   const uint4 *xg = reinterpret_cast<const uint4 *>(p.x + (int64_t)sb0 * 256);
 #pragma unroll
   for (int k = 0; k < XPASS; ++k) {
@@ -546,7 +570,8 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS, GEMV_CTAS_PER_SM)
   const uint32_t xstep = (on0 || on1) ? GEMV_XBLOB : 0u;  // lanes that feed no x read the zero block
   const uint32_t a00 = cring + pg * 128 + ((c ^ pg) << 4), a01 = cring + pg * 128 + (((c + 4) ^ pg) << 4);
   const uint32_t a10 = a00 + 1024, a11 = a01 + 1024;  // row pg + 8: same swizzle phase, next atom
-  const uint32_t am = gring + pg * 16 + 4 * c;
+  // group words of the lane's slices 2c, 2c + 1: int4 the u16 pair at 4c; affine group (2c) * 32 / G
+  const uint32_t am = gring + pg * GM_ROW + (FMT == FMT_INT4 ? 4 * c : 4 * (2 * c * 32 / G));
   const uint32_t ag = xs0 + 16 * c;
 
   const int32_t acc_init[4] = {GEMV_ACC0, GEMV_ACC0, GEMV_ACC0, GEMV_ACC0};
@@ -569,18 +594,28 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS, GEMV_CTAS_PER_SM)
           issue_w(nx, sn);
           issued = nx + 1;
         }
-        sr0[sn] = __ldg(st0 + nx);
-        sr1[sn] = __ldg(st1 + nx);
+        if constexpr (FMT == FMT_INT4) {
+          sr0[sn] = __ldg(st0 + nx);
+          sr1[sn] = __ldg(st1 + nx);
+        }
       }
       if (!mbar_wait_suspend(bar0 + 8 * s, par, &abort_flag)) {
         ok = false;
         break;
       }
-      const uint32_t so = s * 2048, sg = s * 256;
+      const uint32_t so = s * 2048, sg = s * L::GM_STAGE;
       const uint4 w00 = lds128(a00 + so), w10 = lds128(a10 + so);  // (r0 | r1, group c)
       const uint4 w01 = lds128(a01 + so), w11 = lds128(a11 + so);  // (r0 | r1, group c+4)
-      const float4 G = lds128f(gt + s * GEMV_XBLOB);               // (G_x, G_y) of groups 2c, 2c+1
-      const uint32_t cm0 = lds32(am + sg), cm1 = lds32(am + sg + 128);
+      const float4 Gx = lds128f(gt + s * GEMV_XBLOB);              // (G_x, G_y) of groups 2c, 2c+1
+      // group words of rows r0, r1 (row r1 = pg + 8): int4 one word; affine group 64 one, group 32 two
+      uint32_t cm0, cm1, cn0 = 0u, cn1 = 0u;
+      if constexpr (FMT == FMT_INT4 || G == 64) {
+        cm0 = lds32(am + sg);
+        cm1 = lds32(am + sg + 8 * GM_ROW);
+      } else {
+        const uint2 u0 = lds64(am + sg), u1 = lds64(am + sg + 8 * GM_ROW);
+        cm0 = u0.x, cn0 = u0.y, cm1 = u1.x, cn1 = u1.y;
+      }
       const uint32_t xi = xt + (uint32_t)s * xstep;
       const uint32_t ww00[4] = {w00.x, w00.y, w00.z, w00.w}, ww01[4] = {w01.x, w01.y, w01.z, w01.w};
       const uint32_t ww10[4] = {w10.x, w10.y, w10.z, w10.w}, ww11[4] = {w11.x, w11.y, w11.z, w11.w};
@@ -607,21 +642,31 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS, GEMV_CTAS_PER_SM)
 #pragma unroll
       for (int q = 0; q < 4; ++q)
         t[q] = fmaf(__int_as_float(dh[q]) - GEMV_ACC0_F, 256.f, __int_as_float(dm[q]) - GEMV_ACC0_F);
-      // S = sc * ss and Z = zc * zs, each one FMA from the byte placed in the mantissa of 2^23
-      const uint32_t cs0 = sr0[s], cs1 = sr1[s];
-      const float ss0 = f16_bits_to_f32(cs0), zs0 = f16_bits_to_f32(cs0 >> 16);
-      const float ss1 = f16_bits_to_f32(cs1), zs1 = f16_bits_to_f32(cs1 >> 16);
-      const float nss0 = -8388608.f * ss0, nzs0 = -8388608.f * zs0;
-      const float nss1 = -8388608.f * ss1, nzs1 = -8388608.f * zs1;
-      x24s |= __float_as_uint(G.x);
-      const float S00 = fmaf(byte_magic(cm0, 0), ss0, nss0) * G.x, Z00 = fmaf(byte_magic(cm0, 1), zs0, nzs0);
-      const float S01 = fmaf(byte_magic(cm0, 2), ss0, nss0) * G.z, Z01 = fmaf(byte_magic(cm0, 3), zs0, nzs0);
-      const float S10 = fmaf(byte_magic(cm1, 0), ss1, nss1) * G.x, Z10 = fmaf(byte_magic(cm1, 1), zs1, nzs1);
-      const float S11 = fmaf(byte_magic(cm1, 2), ss1, nss1) * G.z, Z11 = fmaf(byte_magic(cm1, 3), zs1, nzs1);
-      acc0 = fmaf(S00, fmaf(Z00, G.y, t[0]), acc0);
-      acc0 = fmaf(S01, fmaf(Z01, G.w, t[1]), acc0);
-      acc1 = fmaf(S10, fmaf(Z10, G.y, t[2]), acc1);
-      acc1 = fmaf(S11, fmaf(Z11, G.w, t[3]), acc1);
+      x24s |= __float_as_uint(Gx.x);
+      if constexpr (FMT == FMT_INT4) {
+        // S = sc * ss and Z = zc * zs, each one FMA from the byte placed in the mantissa of 2^23
+        const uint32_t cs0 = sr0[s], cs1 = sr1[s];
+        const float ss0 = f16_bits_to_f32(cs0), zs0 = f16_bits_to_f32(cs0 >> 16);
+        const float ss1 = f16_bits_to_f32(cs1), zs1 = f16_bits_to_f32(cs1 >> 16);
+        const float nss0 = -8388608.f * ss0, nzs0 = -8388608.f * zs0;
+        const float nss1 = -8388608.f * ss1, nzs1 = -8388608.f * zs1;
+        const float S00 = fmaf(byte_magic(cm0, 0), ss0, nss0) * Gx.x, Z00 = fmaf(byte_magic(cm0, 1), zs0, nzs0);
+        const float S01 = fmaf(byte_magic(cm0, 2), ss0, nss0) * Gx.z, Z01 = fmaf(byte_magic(cm0, 3), zs0, nzs0);
+        const float S10 = fmaf(byte_magic(cm1, 0), ss1, nss1) * Gx.x, Z10 = fmaf(byte_magic(cm1, 1), zs1, nzs1);
+        const float S11 = fmaf(byte_magic(cm1, 2), ss1, nss1) * Gx.z, Z11 = fmaf(byte_magic(cm1, 3), zs1, nzs1);
+        acc0 = fmaf(S00, fmaf(Z00, Gx.y, t[0]), acc0);
+        acc0 = fmaf(S01, fmaf(Z01, Gx.w, t[1]), acc0);
+        acc1 = fmaf(S10, fmaf(Z10, Gx.y, t[2]), acc1);
+        acc1 = fmaf(S11, fmaf(Z11, Gx.w, t[3]), acc1);
+      } else {  // w = q s + b: s G_x T + b 2^-a X, with b 2^-a X = -b G_x G_y
+        const uint32_t wa0 = cm0, wb0 = G == 64 ? cm0 : cn0, wa1 = cm1, wb1 = G == 64 ? cm1 : cn1;
+        const float ga0 = bf16_bits_to_f32(wa0) * Gx.x, gb0 = bf16_bits_to_f32(wb0) * Gx.z;
+        const float ga1 = bf16_bits_to_f32(wa1) * Gx.x, gb1 = bf16_bits_to_f32(wb1) * Gx.z;
+        acc0 = fmaf(ga0, t[0], fmaf(-bf16_bits_to_f32(wa0 >> 16) * Gx.x, Gx.y, acc0));
+        acc0 = fmaf(gb0, t[1], fmaf(-bf16_bits_to_f32(wb0 >> 16) * Gx.z, Gx.w, acc0));
+        acc1 = fmaf(ga1, t[2], fmaf(-bf16_bits_to_f32(wa1 >> 16) * Gx.x, Gx.y, acc1));
+        acc1 = fmaf(gb1, t[3], fmaf(-bf16_bits_to_f32(wb1 >> 16) * Gx.z, Gx.w, acc1));
+      }
     }
   }
   if (!ok && lane == 0) {  // a wait gave up: let this warp's copies in flight land first
@@ -634,10 +679,12 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS, GEMV_CTAS_PER_SM)
     }
   }
   if (__any_sync(0xffffffffu, (x24s & 1u) != 0u) && ok) {  // rare
-    const float2 lb = gemv_m1_low_bytes(p.codes + r0 * (p.K / 2) + (int64_t)sb0 * 128,
-                                        p.codes + r1 * (p.K / 2) + (int64_t)sb0 * 128,
-                                        p.gmeta + r0 * (p.K / 16) + (int64_t)sb0 * 16,
-                                        p.gmeta + r1 * (p.K / 16) + (int64_t)sb0 * 16, st0, st1, xblk, xflag, nsw);
+    const int64_t gm_stride = p.K / 256 * GM_ROW;  // group-word bytes a row
+    const float2 lb = gemv_m1_low_bytes<FMT, G>(p.codes + r0 * (p.K / 2) + (int64_t)sb0 * 128,
+                                                p.codes + r1 * (p.K / 2) + (int64_t)sb0 * 128,
+                                                p.gmeta + r0 * gm_stride + (int64_t)sb0 * GM_ROW,
+                                                p.gmeta + r1 * gm_stride + (int64_t)sb0 * GM_ROW, st0, st1, xblk,
+                                                xflag, nsw);
     acc0 += lb.x;
     acc1 += lb.y;
   }
@@ -677,6 +724,21 @@ __global__ void __launch_bounds__(256) gemv_m1_sum_parts(const float *partial, i
   float sum = 0.f;
   for (int q = 0; q < P; ++q) sum += src[q * 16];
   y[r] = __float2bfloat16_rn(sum + bias_at(bias, r));
+}
+
+// int4 (nested superscale) at M = 1
+__global__ void __launch_bounds__(32 * GEMV_WARPS, GEMV_CTAS_PER_SM)
+    gemv_int4_m1_tc_kernel(const __grid_constant__ CUtensorMap map_codes,
+                           const __grid_constant__ CUtensorMap map_gmeta, GemvTcParams p) {
+  gemv_m1_body<FMT_INT4, 32>(map_codes, map_gmeta, p);
+}
+
+// 4-bit affine (group G = 32 or 64) at M = 1: the same nibble layout, (s, b) per group
+template <int G>
+__global__ void __launch_bounds__(32 * GEMV_WARPS, GEMV_CTAS_PER_SM)
+    gemv_affine4_m1_tc_kernel(const __grid_constant__ CUtensorMap map_codes,
+                              const __grid_constant__ CUtensorMap map_gmeta, GemvTcParams p) {
+  gemv_m1_body<FMT_AFFINE, G>(map_codes, map_gmeta, p);
 }
 
 

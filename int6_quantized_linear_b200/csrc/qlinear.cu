@@ -409,6 +409,73 @@ ql_status launch_gemv_f16(const ql_desc *d, const ql_packed_const *w, const __nv
   return launched();
 }
 
+// M = 1 on the diagonal-x kernel (int4, or 4-bit affine with group 32 / 64): each CTA converts its part
+// of x, then streams four 16-row tiles over it (+ the kernel that adds the parts when K is split)
+template <int FMT, int G>
+ql_status launch_gemv_m1(const ql_desc *d, const ql_packed_const *w, const __nv_bfloat16 *xb,
+                         const __nv_bfloat16 *bb, __nv_bfloat16 *yb, void *workspace, cudaStream_t st, int sms) {
+  using L = M1Layout<FMT, G>;
+  const int64_t M = 1;
+  const int64_t NS = d->K / 256, n_tiles = (d->N + 15) / 16, groups = (n_tiles + GEMV_WARPS - 1) / GEMV_WARPS;
+  // split K so that the tile groups fill the resident CTA slots, and so that each part's x fits the
+  // CTA's blocks; the parts' sums go through the workspace (16 floats a tile and part)
+  int64_t P = std::max<int64_t>(1, std::min<int64_t>(NS, (int64_t)sms * GEMV_CTAS_PER_SM / groups));
+  P = std::max<int64_t>(P, (NS + L::XSB_MAX - 1) / L::XSB_MAX);
+  if (P > 1 && groups * GEMV_WARPS * P * 16 > (int64_t)GEMV_MT_MAX_CTAS * 64) return QL_ERR_RANGE;
+  const GemvWorkspace ws = gemv_workspace_carve(workspace, M, d->N, d->K);
+  GemvTcParams p;
+  p.codes = static_cast<const uint8_t *>(w->codes);
+  p.gmeta = static_cast<const uint8_t *>(w->gmeta);
+  p.steps = static_cast<const uint8_t *>(w->steps);
+  p.bias = bb;
+  p.x = xb;
+  p.N = d->N;
+  p.K = d->K;
+  p.P = (int)P;
+  p.partial = ws.partial;
+  p.y = yb;
+  const uint64_t gm_row = (uint64_t)NS * L::GM_ROW;  // group-word bytes a row
+  CUtensorMap mc, mg;  // codes as [N][K/2] bytes, boxes of 16 rows x 128 bytes, 128-byte swizzle;
+                       // group words as [N][gm_row] bytes, boxes of 16 rows x GM_ROW bytes
+  if (!encode_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->codes, (uint64_t)d->K / 2, (uint64_t)d->N,
+                 (uint64_t)d->K / 2, 128, 16, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_2d(&mg, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->gmeta, gm_row, (uint64_t)d->N, gm_row, L::GM_ROW, 16,
+                 CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cuda_failed();
+  auto kern = FMT == FMT_INT4 ? gemv_int4_m1_tc_kernel : gemv_affine4_m1_tc_kernel<G>;
+  static thread_local int configured_dev = -1;  // per instantiation and thread
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (configured_dev != dev) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM) != cudaSuccess)
+      return cuda_failed();
+    configured_dev = dev;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(groups * P));
+  cfg.blockDim = dim3(32 * GEMV_WARPS);
+  cfg.dynamicSmemBytes = L::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // programmatic dependent of whatever precedes it
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, mc, mg, p) != cudaSuccess) return cuda_failed();
+  if (P > 1) {  // the parts' sums, added by the kernel that depends on this one
+    cudaLaunchConfig_t rc = {};
+    rc.gridDim = dim3((unsigned)((d->N + 255) / 256));
+    rc.blockDim = dim3(256);
+    rc.stream = st;
+    rc.attrs = attr;
+    rc.numAttrs = 1;
+    if (cudaLaunchKernelEx(&rc, gemv_m1_sum_parts, (const float *)ws.partial, (int)P, (int64_t)d->N, bb, yb) !=
+        cudaSuccess)
+      return cuda_failed();
+  }
+  return launched();
+}
+
 template <int FMT, int BITS>
 ql_status launch_gemv(const ql_desc *d, const ql_packed_const *w, const void *x, int64_t M, const void *bias,
                       void *y, void *workspace, cudaStream_t st, int sms) {
@@ -427,6 +494,11 @@ ql_status launch_gemv(const ql_desc *d, const ql_packed_const *w, const void *x,
     return launch_gemv_int6<8, PL>(d, w, xb, M, bb, yb, workspace, st, sms);
   }
   if constexpr (FMT == FMT_AFFINE) {  // bits 2, 4, 8
+    if constexpr (BITS == 4) {  // one token: the diagonal-x kernel of int4 (the same nibble layout)
+      if (affine_tc(d) && M == 1)
+        return d->group == 64 ? launch_gemv_m1<FMT_AFFINE, 64>(d, w, xb, bb, yb, workspace, st, sms)
+                              : launch_gemv_m1<FMT_AFFINE, 32>(d, w, xb, bb, yb, workspace, st, sms);
+    }
     if (affine_tc(d) && M <= 8) {
       if (d->group == 64) return launch_gemv_mt<FMT_AFFINE, BITS, 64>(d, w, xb, M, bb, yb, workspace, st, sms);
       return launch_gemv_mt<FMT_AFFINE, BITS, 32>(d, w, xb, M, bb, yb, workspace, st, sms);
@@ -440,65 +512,7 @@ ql_status launch_gemv(const ql_desc *d, const ql_packed_const *w, const void *x,
     }
   }
   if constexpr (FMT == FMT_INT4) {
-    if (M == 1) {  // each CTA converts its part of x, then streams four 16-row tiles over it (+ the parts' sum)
-      const int64_t NS = d->K / 256, n_tiles = (d->N + 15) / 16, groups = (n_tiles + GEMV_WARPS - 1) / GEMV_WARPS;
-      // split K so that the tile groups fill the resident CTA slots, and so that each part's x fits the
-      // CTA's blocks; the parts' sums go through the workspace (16 floats a tile and part)
-      int64_t P = std::max<int64_t>(1, std::min<int64_t>(NS, (int64_t)sms * GEMV_CTAS_PER_SM / groups));
-      P = std::max<int64_t>(P, (NS + GEMV_XSB_MAX - 1) / GEMV_XSB_MAX);
-      if (P > 1 && groups * GEMV_WARPS * P * 16 > (int64_t)GEMV_MT_MAX_CTAS * 64) return QL_ERR_RANGE;
-      const GemvWorkspace ws = gemv_workspace_carve(workspace, M, d->N, d->K);
-      GemvTcParams p;
-      p.codes = static_cast<const uint8_t *>(w->codes);
-      p.gmeta = static_cast<const uint8_t *>(w->gmeta);
-      p.steps = static_cast<const uint8_t *>(w->steps);
-      p.bias = bb;
-      p.x = xb;
-      p.N = d->N;
-      p.K = d->K;
-      p.P = (int)P;
-      p.partial = ws.partial;
-      p.y = yb;
-      CUtensorMap mc, mg;  // codes as [N][K/2] bytes, boxes of 16 rows x 128 bytes, 128-byte swizzle;
-                           // group words as [N][K/16] bytes, boxes of 16 rows x 16 bytes
-      if (!encode_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->codes, (uint64_t)d->K / 2, (uint64_t)d->N,
-                     (uint64_t)d->K / 2, 128, 16, CU_TENSOR_MAP_SWIZZLE_128B) ||
-          !encode_2d(&mg, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->gmeta, (uint64_t)d->K / 16, (uint64_t)d->N,
-                     (uint64_t)d->K / 16, 16, 16, CU_TENSOR_MAP_SWIZZLE_NONE))
-        return cuda_failed();
-      static thread_local int configured_dev = -1;
-      int dev = 0;
-      cudaGetDevice(&dev);
-      if (configured_dev != dev) {
-        if (cudaFuncSetAttribute(gemv_int4_m1_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 gemv_smem_bytes()) != cudaSuccess)
-          return cuda_failed();
-        configured_dev = dev;
-      }
-      cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3((unsigned)(groups * P));
-      cfg.blockDim = dim3(32 * GEMV_WARPS);
-      cfg.dynamicSmemBytes = gemv_smem_bytes();
-      cfg.stream = st;
-      cudaLaunchAttribute attr[1];
-      attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // programmatic dependent of whatever precedes it
-      attr[0].val.programmaticStreamSerializationAllowed = 1;
-      cfg.attrs = attr;
-      cfg.numAttrs = 1;
-      if (cudaLaunchKernelEx(&cfg, gemv_int4_m1_tc_kernel, mc, mg, p) != cudaSuccess) return cuda_failed();
-      if (P > 1) {  // the parts' sums, added by the kernel that depends on this one
-        cudaLaunchConfig_t rc = {};
-        rc.gridDim = dim3((unsigned)((d->N + 255) / 256));
-        rc.blockDim = dim3(256);
-        rc.stream = st;
-        rc.attrs = attr;
-        rc.numAttrs = 1;
-        if (cudaLaunchKernelEx(&rc, gemv_m1_sum_parts, (const float *)ws.partial, (int)P, (int64_t)d->N, bb, yb) !=
-            cudaSuccess)
-          return cuda_failed();
-      }
-      return launched();
-    }
+    if (M == 1) return launch_gemv_m1<FMT_INT4, 32>(d, w, xb, bb, yb, workspace, st, sms);
   }
   if constexpr (FMT == FMT_AFFINE) {  // groups without the multi-token kernel, M < 8: CUDA cores
     const WeightPtrs p = make_ptrs(d, w);
