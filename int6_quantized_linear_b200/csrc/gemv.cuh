@@ -374,9 +374,13 @@ struct M1Layout {
   static constexpr uint32_t STAGE_TX = 2048 + GM_STAGE;
   // dynamic shared memory: codes rings, group-word rings, the CTA's x blocks and their 24-bit flags,
   // zero block, mbarriers
-  static constexpr int SMEM = CODES_BYTES + GMETA_BYTES + XSB_MAX * GEMV_XBLOB + 32 + GEMV_ZERO_BYTES +
+  static constexpr int USED = CODES_BYTES + GMETA_BYTES + XSB_MAX * GEMV_XBLOB + 32 + GEMV_ZERO_BYTES +
                               GEMV_WARPS * GEMV_RING * 8 + 1024;
-  static_assert(GEMV_CTAS_PER_SM * (SMEM + 1024) <= 233472, "three CTAs an SM");
+  static_assert(GEMV_CTAS_PER_SM * (USED + 1024) <= 233472, "three CTAs an SM");
+  // affine: a request that keeps a third CTA off an SM, so a layer with half as many tile groups as
+  // slots spreads over two thirds of the SMs instead of being packed onto half of them
+  static constexpr int FLOOR = 233472 / 3;
+  static constexpr int SMEM = FMT == FMT_AFFINE && USED < FLOOR ? FLOOR : USED;
 };
 
 struct GemvTcParams {
