@@ -39,8 +39,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM bytes per GEMV launch from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum),
 # valid only while the GEMV source is unchanged (hash of csrc/gemv.cuh at capture time).
-NCU_TRAFFIC = {"gemv_src_sha256": "e7ad75c8117363d2807c221a4c7e589273cc8b5edeba74ddf0e814efe6303860",
-               "bytes_per_launch": 83041280}  # mean over the two decode layers
+NCU_TRAFFIC = {"gemv_src_sha256": "9a89b43b1360763d86ba986f5d5168a904d4fab0fc6658b1c92017349d3c049b",
+               "bytes_per_launch": 83152640}  # mean over the two decode layers
 
 
 def parse_args(argv=None):
