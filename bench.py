@@ -634,11 +634,15 @@ def run_e2e(args, layers, device, step_bytes):
     h2d = sum(x.numel() * 2 for x in xh)
     d2h = sum(y.numel() * 2 for y in yh)
 
-    def step(i):
-        for L, xhost, yhost in zip(layers, xh, yh):
-            c, g, s = L["reps"][i % len(L["reps"])]
+    stream = torch.cuda.current_stream(device)
+
+    def step(i):  # the step's inputs in, its layers back to back (chained on the stream), its results out
+        for L, xhost in zip(layers, xh):
             L["x"].copy_(xhost, non_blocking=True)
-            ql.qlinear_gemv(L["desc"], c, g, s, L["x"], 1, L["y"], L["ws"])
+        for L in layers:
+            c, g, s = L["reps"][i % len(L["reps"])]
+            ql.qlinear_gemv(L["desc"], c, g, s, L["x"], 1, L["y"], L["ws"], stream)
+        for L, yhost in zip(layers, yh):
             yhost.copy_(L["y"], non_blocking=True)
 
     for i in range(args.warmup):

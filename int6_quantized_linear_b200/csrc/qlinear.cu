@@ -123,16 +123,48 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
+// A tensor map is a pure function of these arguments, so the last few encodings are kept per host
+// thread and reused: a decode loop calls the same layers with the same buffers over and over, and the
+// encoding is host time on every call's critical path.
+struct TmapKey {
+  const void *base;
+  uint64_t inner, outer, row_bytes;
+  uint32_t box_inner, box_outer;
+  int dt, sw;
+  bool operator==(const TmapKey &o) const {
+    return base == o.base && inner == o.inner && outer == o.outer && row_bytes == o.row_bytes &&
+           box_inner == o.box_inner && box_outer == o.box_outer && dt == o.dt && sw == o.sw;
+  }
+};
+
 bool encode_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64_t inner, uint64_t outer,
                uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
+  constexpr int kEntries = 32;
+  struct Entry {
+    TmapKey key;
+    CUtensorMap map;
+    bool valid;
+  };
+  static thread_local Entry cache[kEntries] = {};
+  static thread_local int next = 0;
+  const TmapKey key{base, inner, outer, row_bytes, box_inner, box_outer, (int)dt, (int)sw};
+  for (int i = 0; i < kEntries; ++i)
+    if (cache[i].valid && cache[i].key == key) {
+      *map = cache[i].map;
+      return true;
+    }
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {inner, outer};
   cuuint64_t strides[1] = {row_bytes};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
-  return fn(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  if (fn(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  cache[next] = Entry{key, *map, true};
+  next = (next + 1) % kEntries;
+  return true;
 }
 
 template <int FMT, int BITS, int TT>
