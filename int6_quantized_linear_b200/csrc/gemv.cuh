@@ -261,19 +261,20 @@ QL_DEVI bool gemv_m1_convert_group(const uint4 (&v)[4], bool live, int grp, uint
     xi[k] = __float2int_rn(xs[k] * sc);
     sum += xi[k];
   }
-  const int hs = sb24 ? 16 : 8;  // the value's top byte: bits 16.. (24-bit) or 8.. (16-bit, lo = 0)
+  // byte b of a word = the chosen byte of value b: the value's top byte is byte 2 (24-bit) or byte 1
+  // (16-bit, no low byte), its middle byte the one below; gathered by byte permutes
+  const uint32_t th = sb24 ? 2u : 1u, sel_hi = th | ((4u + th) << 4), sel_mid = (th - 1u) | ((3u + th) << 4);
+  auto gather = [](int v0, int v1, int v2, int v3, uint32_t sel) {
+    return __byte_perm(__byte_perm((uint32_t)v0, (uint32_t)v1, sel), __byte_perm((uint32_t)v2, (uint32_t)v3, sel),
+                       0x5410u);
+  };
 #pragma unroll
   for (int j = 0; j < 4; ++j)
 #pragma unroll
     for (int kind = 0; kind < 2; ++kind) {
-      uint32_t hi = 0, mid = 0, lo = 0;
-#pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        const int val = xi[8 * j + 2 * b + kind];
-        hi |= ((uint32_t)(val >> hs) & 0xffu) << (8 * b);
-        mid |= ((uint32_t)(val >> (hs - 8)) & 0xffu) << (8 * b);
-        lo |= ((uint32_t)val & 0xffu) << (8 * b);
-      }
+      const int *v = xi + 8 * j + kind;  // values k = 8j + kind + {0, 2, 4, 6}
+      const uint32_t hi = gather(v[0], v[2], v[4], v[6], sel_hi), mid = gather(v[0], v[2], v[4], v[6], sel_mid);
+      const uint32_t lo = sb24 ? gather(v[0], v[2], v[4], v[6], 0x40u) : 0u;
       const int ch = 8 * (2 * j + kind) + grp;  // chunk (j, kind) of group grp
       reinterpret_cast<uint4 *>(blk + GEMV_XB_Q)[ch] = grp < 4 ? make_uint4(hi, 0u, mid, 0u) : make_uint4(0u, hi, 0u, mid);
       if (sb24) reinterpret_cast<uint2 *>(blk + GEMV_XB_L)[ch] = grp < 4 ? make_uint2(lo, 0u) : make_uint2(0u, lo);
