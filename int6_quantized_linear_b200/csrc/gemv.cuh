@@ -213,22 +213,25 @@ QL_DEVI bool group_needs_24bit(float err, float mass, float amax_scaled) {
   return err > (mass - amax_scaled) * (1.f / 4096.f);
 }
 
-// x conversion for the int4 M = 1 kernel, one lane per 32-element group, eight lanes per super-block:
-// fixed point with the group's max and sum, 16-bit unless some group of the super-block needs 24 bits
-// (then the whole super-block is 24-bit), byte split in fragment order into the super-block's block
-// blk (shared memory, GEMV_XBLOB bytes): the eight groups' (G_x, G_y), then chunk (j, kind) of group
-// grp at [j][kind][grp] of the (hi, mid) region -- the high-byte and middle-byte words of
-// k = 8j + kind + {0, 2, 4, 6}, each paired with a zero word so that one 16-byte load gives the B pairs
-// of two MMAs: (x, 0) for groups 0-3 (their lanes feed b0), (0, x) for groups 4-7 (b1) -- and, for
-// 24-bit x only, the low-byte word paired the same way (8 bytes) in the lo region.  v: the group's 32
-// bf16; live: the lane holds a group (every lane takes part in the vote).  Returns whether the
+// x conversion for the int4 M = 1 kernel, NP lanes per 32-element group (1, 2 or 4; lane part p holds
+// k = p 32/NP .. (p + 1) 32/NP - 1), 8 NP lanes per super-block: fixed point with the group's max and sum
+// (combined over its lanes by shuffles), 16-bit unless some group of the super-block needs 24 bits (then
+// the whole super-block is 24-bit), byte split in fragment order into the super-block's block blk
+// (shared memory, GEMV_XBLOB bytes): the eight groups' (G_x, G_y), then chunk (j, kind) of group grp at
+// [j][kind][grp] of the (hi, mid) region -- the high-byte and middle-byte words of k = 8j + kind +
+// {0, 2, 4, 6}, each paired with a zero word so that one 16-byte load gives the B pairs of two MMAs:
+// (x, 0) for groups 0-3 (their lanes feed b0), (0, x) for groups 4-7 (b1) -- and, for 24-bit x only,
+// the low-byte word paired the same way (8 bytes) in the lo region.  v: the lane's 32/NP bf16; live: the
+// lane holds a group (every lane takes part in the shuffles and the vote).  Returns whether the
 // super-block is 24-bit.
-QL_DEVI bool gemv_m1_convert_group(const uint4 (&v)[4], bool live, int grp, uint8_t *blk) {
+template <int NP>
+QL_DEVI bool gemv_m1_convert_group(const uint4 (&v)[4], bool live, int grp, int part, uint8_t *blk) {
+  constexpr int EL = 32 / NP;  // elements a lane
   const int lane = threadIdx.x & 31;
-  float xs[32];
+  float xs[EL];
   float amax = 0.f;
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
+  for (int q = 0; q < EL / 8; ++q) {
     const uint32_t u[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -237,30 +240,40 @@ QL_DEVI bool gemv_m1_convert_group(const uint4 (&v)[4], bool live, int grp, uint
     }
   }
 #pragma unroll
-  for (int k = 0; k < 32; ++k) amax = fmaxf(amax, fabsf(xs[k]));
+  for (int k = 0; k < EL; ++k) amax = fmaxf(amax, fabsf(xs[k]));
+#pragma unroll
+  for (int o = 1; o < NP; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
   const int a16 = scale_exponent(amax, 14);  // max |x_int| < 2^15
   const float s16 = exp2i(a16);
   float err = 0.f, mass = 0.f;
 #pragma unroll
-  for (int k = 0; k < 32; ++k) {
+  for (int k = 0; k < EL; ++k) {
     const float sv = xs[k] * s16;
     err += fabsf(sv - rintf(sv));
     mass += fabsf(sv);
   }
+#pragma unroll
+  for (int o = 1; o < NP; o <<= 1) {
+    err += __shfl_xor_sync(0xffffffffu, err, o);
+    mass += __shfl_xor_sync(0xffffffffu, mass, o);
+  }
   // 16-bit fixed point loses too much when the summed rounding error is above 2^-12 of the group's mass
   // outside its largest element (all in units of 2^-a16)
   const bool wide = live && err > (mass - amax * s16) * (1.f / 4096.f);
-  const bool sb24 = ((__ballot_sync(0xffffffffu, wide) >> (lane & ~7)) & 0xffu) != 0u;  // the super-block's 8 lanes
+  constexpr uint32_t SEG = 8 * NP == 32 ? 0xffffffffu : (1u << (8 * NP)) - 1u;  // the super-block's lanes
+  const bool sb24 = ((__ballot_sync(0xffffffffu, wide) >> (lane & ~(8 * NP - 1))) & SEG) != 0u;
   const int a = sb24 ? scale_exponent(amax, 22) : a16;  // 24-bit: max |x_int| < 2^23
   const float sc = exp2i(a);
-  if (!live) return sb24;
-  int xi[32];
+  int xi[EL];
   int sum = 0;  // |sum| < 32 * 2^23
 #pragma unroll
-  for (int k = 0; k < 32; ++k) {
+  for (int k = 0; k < EL; ++k) {
     xi[k] = __float2int_rn(xs[k] * sc);
     sum += xi[k];
   }
+#pragma unroll
+  for (int o = 1; o < NP; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if (!live) return sb24;
   // byte b of a word = the chosen byte of value b: the value's top byte is byte 2 (24-bit) or byte 1
   // (16-bit, no low byte), its middle byte the one below; gathered by byte permutes
   const uint32_t th = sb24 ? 2u : 1u, sel_hi = th | ((4u + th) << 4), sel_mid = (th - 1u) | ((3u + th) << 4);
@@ -269,19 +282,21 @@ QL_DEVI bool gemv_m1_convert_group(const uint4 (&v)[4], bool live, int grp, uint
                        0x5410u);
   };
 #pragma unroll
-  for (int j = 0; j < 4; ++j)
+  for (int jj = 0; jj < EL / 8; ++jj)
 #pragma unroll
     for (int kind = 0; kind < 2; ++kind) {
-      const int *v = xi + 8 * j + kind;  // values k = 8j + kind + {0, 2, 4, 6}
-      const uint32_t hi = gather(v[0], v[2], v[4], v[6], sel_hi), mid = gather(v[0], v[2], v[4], v[6], sel_mid);
-      const uint32_t lo = sb24 ? gather(v[0], v[2], v[4], v[6], 0x40u) : 0u;
+      const int j = part * (EL / 8) + jj;
+      const int *vv = xi + 8 * jj + kind;  // values k = 8j + kind + {0, 2, 4, 6}
+      const uint32_t hi = gather(vv[0], vv[2], vv[4], vv[6], sel_hi), mid = gather(vv[0], vv[2], vv[4], vv[6], sel_mid);
+      const uint32_t lo = sb24 ? gather(vv[0], vv[2], vv[4], vv[6], 0x40u) : 0u;
       const int ch = 8 * (2 * j + kind) + grp;  // chunk (j, kind) of group grp
       reinterpret_cast<uint4 *>(blk + GEMV_XB_Q)[ch] = grp < 4 ? make_uint4(hi, 0u, mid, 0u) : make_uint4(0u, hi, 0u, mid);
       if (sb24) reinterpret_cast<uint2 *>(blk + GEMV_XB_L)[ch] = grp < 4 ? make_uint2(lo, 0u) : make_uint2(0u, lo);
     }
-  // (G_x, G_y) = (2^-a / 16, -16 X) scaled by (2^v, 2^-v), v = 8 (24-bit) or 0 (16-bit)
-  const float vs = sb24 ? 256.f : 1.f, vi = sb24 ? 1.f / 256.f : 1.f, gx = exp2i(-a) * 0.0625f * vs;
-  reinterpret_cast<float2 *>(blk)[grp] = make_float2(sb24 ? mark_24bit(gx) : gx, -16.f * (float)sum * vi);
+  if (part == 0) {  // (G_x, G_y) = (2^-a / 16, -16 X) scaled by (2^v, 2^-v), v = 8 (24-bit) or 0 (16-bit)
+    const float vs = sb24 ? 256.f : 1.f, vi = sb24 ? 1.f / 256.f : 1.f, gx = exp2i(-a) * 0.0625f * vs;
+    reinterpret_cast<float2 *>(blk)[grp] = make_float2(sb24 ? mark_24bit(gx) : gx, -16.f * (float)sum * vi);
+  }
   return sb24;
 }
 
@@ -541,29 +556,37 @@ __device__ __forceinline__ void gemv_m1_body(const CUtensorMap &map_codes, const
       sr1[s] = __ldg(st1 + s);
     }
   }
-  // x of the part: thread t of pass k converts group 128 k + t (super-block (128 k + t) / 8)
-  constexpr int XPASS = (8 * L::XSB_MAX + 32 * GEMV_WARPS - 1) / (32 * GEMV_WARPS);
+  // x of the part: its first 128 groups one a thread, the rest (at most 8 * XSB_MAX - 128) two or four
+  // lanes a group, so that the second pass is as short as the first allows
+  static_assert(8 * L::XSB_MAX <= 2 * 32 * GEMV_WARPS, "two passes");
+  const int ng = 8 * nsb, rest = ng - 32 * GEMV_WARPS;
+  const int np = rest <= 0 ? 0 : rest <= 8 * GEMV_WARPS ? 4 : rest <= 16 * GEMV_WARPS ? 2 : 1;  // lanes a group
   const uint4 *xg = reinterpret_cast<const uint4 *>(p.x + (int64_t)sb0 * 256);
-#pragma unroll
-  for (int k = 0; k < XPASS; ++k) {
-    const int q = 32 * GEMV_WARPS * k + (int)threadIdx.x;
-    if (q < 8 * nsb) prefetch_l2(xg + 4 * q);
-  }
+  const int q1 = (int)threadIdx.x;                                          // pass 1: group q1
+  const int q2 = 32 * GEMV_WARPS + (np ? (int)threadIdx.x / np : 0);        // pass 2: group q2,
+  const int part2 = np ? (int)threadIdx.x % np : 0, per2 = np ? 4 / np : 0;  // part part2 of it
+  if (q1 < ng) prefetch_l2(xg + 4 * q1);
+  if (np && q2 < ng) prefetch_l2(xg + 4 * q2);
   pdl_wait();  // x may be the output of the kernel launched before this one
   {
-    uint4 xv[XPASS][4];
+    uint4 v1[4], v2[4];  // both passes' loads in flight before either converts
 #pragma unroll
-    for (int k = 0; k < XPASS; ++k) {
-      const int q = 32 * GEMV_WARPS * k + (int)threadIdx.x;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) xv[k][e] = q < 8 * nsb ? __ldg(xg + 4 * q + e) : make_uint4(0u, 0u, 0u, 0u);
+    for (int e = 0; e < 4; ++e) {
+      v1[e] = q1 < ng ? __ldg(xg + 4 * q1 + e) : make_uint4(0u, 0u, 0u, 0u);
+      v2[e] = np && q2 < ng && e < per2 ? __ldg(xg + 4 * q2 + part2 * per2 + e) : make_uint4(0u, 0u, 0u, 0u);
     }
-#pragma unroll
-    for (int k = 0; k < XPASS; ++k) {
-      const int q = 32 * GEMV_WARPS * k + (int)threadIdx.x, i = q >> 3;
-      const bool live = q < 8 * nsb;
-      const bool sb24 = gemv_m1_convert_group(xv[k], live, q & 7, xblk + (live ? i : 0) * GEMV_XBLOB);
-      if (live && (q & 7) == 0) xflag[i] = sb24 ? 1 : 0;
+    {
+      const bool live = q1 < ng;
+      const bool sb24 = gemv_m1_convert_group<1>(v1, live, q1 & 7, 0, xblk + (live ? q1 >> 3 : 0) * GEMV_XBLOB);
+      if (live && (q1 & 7) == 0) xflag[q1 >> 3] = sb24 ? 1 : 0;
+    }
+    if (np) {  // the same for the whole CTA
+      const bool live = q2 < ng;
+      uint8_t *blk = xblk + (live ? q2 >> 3 : 0) * GEMV_XBLOB;
+      const bool sb24 = np == 4   ? gemv_m1_convert_group<4>(v2, live, q2 & 7, part2, blk)
+                        : np == 2 ? gemv_m1_convert_group<2>(v2, live, q2 & 7, part2, blk)
+                                  : gemv_m1_convert_group<1>(v2, live, q2 & 7, part2, blk);
+      if (live && (q2 & 7) == 0 && part2 == 0) xflag[q2 >> 3] = sb24 ? 1 : 0;
     }
   }
   __syncthreads();  // the part's x blocks are complete
