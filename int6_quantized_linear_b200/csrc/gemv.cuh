@@ -100,13 +100,13 @@ __global__ void __launch_bounds__(256) gemv_simple_kernel(WeightPtrs p, int64_t 
 // x, T is 2^-8 of 16 sum_k q_k x_int_k less the low bytes' share, so (G_x, G_y)
 // = (2^8 * 2^-a_g / 16, -16 X_g / 2^8), G_x carries the 24-bit marker
 // (mark_24bit), and after the loop an out-of-line pass adds S G_x 2^-8 D_lo for
-// the marked super-blocks, reading their weights again (gemv_m1_low_bytes).  A
-// short preparation pass writes the x bytes in the order the fragments read
-// them, (G_x, G_y) per group and a 24-bit flag per super-block; the streaming
-// kernel is launched as a programmatic dependent of that pass and starts
-// fetching weights before it has finished (griddepcontrol.wait guards the
-// first read of x).  Lanes that hold no x for an MMA read a zero block, so no
-// per-MMA selects are needed.
+// the marked super-blocks, reading their weights again (gemv_m1_low_bytes).
+// Each CTA (four tiles over one part of K) converts its part of x itself into
+// shared memory -- the x bytes in the order the fragments read them, (G_x, G_y)
+// per group and a 24-bit flag per super-block -- after its weight copies have
+// started and griddepcontrol.wait has let the previous kernel on the stream
+// finish.  Lanes that hold no x for an MMA read a zero block, so no per-MMA
+// selects are needed.
 // ===========================================================================
 
 constexpr int GEMV_MT_MAX_CTAS = 4096;  // bound on the CTAs of one multi-token launch (sizes its partial sums)
@@ -151,8 +151,8 @@ inline SplitK split_k(int64_t units, int64_t slots, int64_t NS, bool fill) {
   return s;
 }
 
-// M = 1 x block per super-block: 8 x (G_x, G_y) (64 B) and the (hi, mid) x words (1 KB) -- the part
-// a stage copies -- then the lo x words (512 B), written and read only for a 24-bit super-block
+// M = 1 x block per super-block (in the CTA's shared memory): 8 x (G_x, G_y) (64 B) and the (hi, mid)
+// x words (1 KB), then the lo x words (512 B), written and read only for a 24-bit super-block
 constexpr int GEMV_XBLOB = 1600, GEMV_XCOPY = 1088, GEMV_XB_Q = 64, GEMV_XB_L = 1088;
 
 struct GemvWorkspace {
