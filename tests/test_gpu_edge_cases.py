@@ -140,15 +140,17 @@ def test_edge_pack_unpack_dequant_bitexact(cuda, fmt, bits, group):
 
 
 def _gemv_token_counts(fmt, group):
-    if fmt == "affine":  # group 32 / 64: integer multi-token kernel to 8 tokens, the fp16 tensor-core
-        return (1, 7, 8, 9, 12, 16, 31, 32)  # GEMV from 9; group 128: CUDA cores to 7, the tcgen05 GEMM from 8
+    if fmt == "affine":  # group 32 / 64: the diagonal kernel at one token (4-bit), the integer multi-token
+        return (1, 7, 8, 9, 12, 16, 31, 32)  # kernel to 8 tokens, the fp16 tensor-core GEMV from 9; group
+                                             # 128: CUDA cores to 7, the tcgen05 GEMM from 8
     return (1, 2, 5, 7, 8)
 
 
 @pytest.mark.parametrize("fmt,bits,group", CASES, ids=CASE_IDS)
 def test_edge_gemv(cuda, fmt, bits, group):
     """qlinear_gemv on edge weights and edge activations: every activation kind alone at M = 1
-    (int4's diagonal kernel), and the kinds side by side at the larger token counts."""
+    (the diagonal kernel for int4 and 4-bit affine), and the kinds side by side at the larger token
+    counts."""
     L, cats, names = edge_layer(fmt, N_SMALL, K_SMALL, bits, group, seed=5)
     w_ref = L.oracle_w()
     bad = []
