@@ -218,7 +218,8 @@ ql_status qlinear_quantize_meta(const ql_desc *desc, const float *scale, const f
  * bytes per element plus the zero padding of the diagonal operands) in the
  * order the tensor-core fragments read it, 8*M*K/32 for the per-group x
  * scales and sums,
- * 4*4096*64*M for the partial sums of a K split, 4*ceil(N/16) for its
+ * 4*max(4096*64*M, 64*ceil(N/64)*ceil(K/5120)) for the partial sums of a
+ * K split, 4*ceil(N/16) for its
  * counters and 16*K/256 for the per-super-block precision flags, each part
  * rounded up to 256 bytes; for affine calls that run on
  * the GEMM (below) at least qlinear_gemm_workspace_bytes().
@@ -242,9 +243,8 @@ ql_status qlinear_gemv_workspace_bytes(const ql_desc *desc, int64_t M, size_t *b
  *    read them, with the group's scale (and sum) -- by a short pass, or, for
  *    int4 and 4-bit affine (group 32 / 64) at M = 1, by each CTA of the
  *    streaming kernel for its part of K,
- *    into shared memory (K split into parts of at most 22 super-blocks,
- *    16 partial sums a part and 16 rows within the workspace's 4*4096*64
- *    bytes; QL_ERR_RANGE beyond); then the streaming kernel
+ *    into shared memory (K split into parts of at most 22 super-blocks, their
+ *    partial sums in the workspace); then the streaming kernel
  *    multiplies the codes (as u8 or s8 bytes: 16q for nibbles, 4q for int6,
  *    q for 2- and 8-bit fields) by those bytes on the integer tensor core
  *    (mma.sync m16n8k32, exact s32 sums, one MMA per byte: high and middle

@@ -164,9 +164,17 @@ struct GemvWorkspace {
   uint8_t *flags;   // [K/256][16]: byte m non-zero when token m's x of that super-block is 24-bit
 };
 
+// floats of partial sums: the multi-token and int6 kernels' bound, or the M = 1 kernel's when a wide
+// layer splits K only so that each part's x fits a CTA (64 sums a CTA, parts of at least 20 super-blocks)
+inline size_t gemv_partial_floats(int64_t M, int64_t N, int64_t K) {
+  const size_t mt = (size_t)GEMV_MT_MAX_CTAS * 64 * M;
+  const size_t m1 = (size_t)64 * ((N + 63) / 64) * ((K / 256 + 19) / 20);
+  return mt > m1 ? mt : m1;
+}
+
 inline size_t gemv_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   return align256((size_t)M * K * 7) + align256((size_t)M * (K / 32) * 8) +
-         align256((size_t)GEMV_MT_MAX_CTAS * 64 * M * 4) + align256((size_t)((N + 15) / 16) * 4) +
+         align256(gemv_partial_floats(M, N, K) * 4) + align256((size_t)((N + 15) / 16) * 4) +
          align256((size_t)(K / 256) * 16);
 }
 
@@ -178,7 +186,7 @@ inline GemvWorkspace gemv_workspace_carve(void *base, int64_t M, int64_t N, int6
   w.gsum = reinterpret_cast<float2 *>(p);
   p += align256((size_t)M * (K / 32) * 8);
   w.partial = reinterpret_cast<float *>(p);
-  p += align256((size_t)GEMV_MT_MAX_CTAS * 64 * M * 4);
+  p += align256(gemv_partial_floats(M, N, K) * 4);
   w.counters = reinterpret_cast<int *>(p);
   p += align256((size_t)((N + 15) / 16) * 4);
   w.flags = p;

@@ -453,7 +453,7 @@ ql_status launch_gemv_m1(const ql_desc *d, const ql_packed_const *w, const __nv_
   // CTA's blocks; the parts' sums go through the workspace (16 floats a tile and part)
   int64_t P = std::max<int64_t>(1, std::min<int64_t>(NS, (int64_t)sms * GEMV_CTAS_PER_SM / groups));
   P = std::max<int64_t>(P, (NS + L::XSB_MAX - 1) / L::XSB_MAX);
-  if (P > 1 && groups * GEMV_WARPS * P * 16 > (int64_t)GEMV_MT_MAX_CTAS * 64) return QL_ERR_RANGE;
+  if (P > 1 && groups * GEMV_WARPS * P * 16 > (int64_t)gemv_partial_floats(M, d->N, d->K)) return QL_ERR_RANGE;
   const GemvWorkspace ws = gemv_workspace_carve(workspace, M, d->N, d->K);
   GemvTcParams p;
   p.codes = static_cast<const uint8_t *>(w->codes);

@@ -121,13 +121,15 @@ def _a256(n):
 
 @pytest.mark.parametrize("fmt,bits,group,N,K,M", [("int4", 0, 0, 300, 512, 1), ("int4", 0, 0, 27648, 5120, 8),
                                                   ("int6", 0, 0, 5120, 5120, 1), ("int6", 0, 0, 1000, 768, 8),
-                                                  ("affine", 2, 64, 14336, 4096, 8), ("affine", 4, 128, 64, 256, 3)])
+                                                  ("affine", 2, 64, 14336, 4096, 8), ("affine", 4, 128, 64, 256, 3),
+                                                  ("int4", 0, 0, 131072, 16384, 1)])
 def test_gemv_workspace_formula(lib, fmt, bits, group, N, K, M):
     """The GEMV workspace size is the documented sum: x words (three bytes of 24-bit fixed point per
     element, laid out for the tensor-core fragments), per-group scales and sums, the partial sums of a K
-    split, one counter per 16 rows, a 16-byte flag record per super-block, each part rounded up to 256
-    bytes."""
-    want = (_a256(7 * M * K) + _a256(8 * M * (K // 32)) + _a256(4 * 4096 * 64 * M) + _a256(4 * ((N + 15) // 16))
+    split (for a wide layer at M=1 enough for its parts of at most 20 super-blocks), one counter per 16
+    rows, a 16-byte flag record per super-block, each part rounded up to 256 bytes."""
+    partial = max(4096 * 64 * M, 64 * -(-N // 64) * -(-(K // 256) // 20))  # floats
+    want = (_a256(7 * M * K) + _a256(8 * M * (K // 32)) + _a256(4 * partial) + _a256(4 * ((N + 15) // 16))
             + _a256(16 * (K // 256)))
     assert ql.qlinear_gemv_workspace_bytes(ql.Desc(fmt, N, K, bits, group), M) == want
 
