@@ -2,25 +2,38 @@
 //
 //   y[M][N] = x[M][K] . W^T,  x bf16, W quantized, y bf16, fp32 accumulation
 //
-// Persistent kernel, one CTA per SM, tiles of BM=256 tokens x BN=128 weight
-// rows, K streamed in BK=64 steps through a 3- or 4-deep shared-memory ring.
-// Each k-step is two MMAs of M=128 (the two token halves) against the same
-// dequantised weight tile, so every weight is dequantised once per 256 tokens.
+// Persistent kernel, one CTA per SM, tiles of BN=128 weight rows x TT tokens,
+// K streamed in BK=64 steps through a shared-memory ring of x and code tiles.
+// Two forms:
+//   TT = 256 (prefill): the dequantised weight tile never touches shared
+//     memory.  The dequantisers write it into tensor memory (TMEM), where one
+//     MMA of M = 128 (weight rows, A read from TMEM) x N = 256 (tokens, B = the
+//     x tile in shared memory) per 16-k slice consumes it.  Shared memory then
+//     carries only the x tile (written once by TMA, read once by the tensor
+//     core) and the packed codes, which is what bounds this form: a
+//     shared-memory weight tile would add its store, and a second token half
+//     would read it again, roughly doubling the bytes shared memory moves per
+//     MMA.  The accumulator (128 lanes x 256 columns) and a ring of A stages
+//     (32 columns each) share the 512 TMEM columns, so there is one
+//     accumulator and the epilogue of a tile runs between two tiles' MMAs.
+//   TT = 32 (small batches): the dequantised tile goes to shared memory in the
+//     canonical K-major 128-byte-swizzled layout as the A operand (M = 128),
+//     against a 32-token x tile as B (N = 32), with two accumulators.
 // Warp roles:
-//   warp 0      TMA producer: scaled fp16 x tile (256 x 64, 128-byte
+//   warp 0      TMA producer: scaled fp16 x tile (TT x 64, 128-byte
 //               swizzle) and the packed code tile (128 rows x BK codes)
-//   warp 1      TMEM allocator; lane 0 issues tcgen05.mma (M=128, N=128,
-//               K=16, f16 x f16 -> f32), two per 16-k slice, into one of two
-//               TMEM accumulator pairs
+//   warp 1      TMEM allocator; lane 0 issues tcgen05.mma (f16 x f16 -> f32)
 //   warps 2-3   (int4) copy each stage's group and step words into a
 //               metadata ring, MSTAGES ahead
-//   warps 4-7   epilogue: tcgen05.ld the accumulators (warp w reads TMEM
-//               lanes 32*(w%4).. of both halves), undo the two power-of-two
-//               scales (exponents added first), round to bf16, store y
-//   warps 8-15  dequantisers, one tile row and 32 weights each per stage:
-//               packed codes + metadata -> weight times 2^b_n -> fp16, written
-//               in the canonical K-major 128-byte-swizzled layout the MMA reads
-//               as its B operand
+//   warps 4-7   epilogue: tcgen05.ld the accumulator (warp w reads TMEM lanes
+//               32*(w%4).., one weight row per lane), undo the two
+//               power-of-two scales (exponents added first), round to bf16,
+//               store y
+//   warps 8-15  dequantisers: packed codes + metadata -> weight times 2^b_n
+//               -> fp16.  TT = 256: warps 8-11 fill even stages and 12-15 odd
+//               ones, one whole 64-weight tile row per thread, into the TMEM
+//               lanes of the warp's quarter.  TT = 32: one tile row and 32
+//               weights per thread and stage, into shared memory.
 // The operands are fp16 rather than bf16 because rounding every weight to
 // bf16 costs ~1% of rms(y); fp16 costs ~0.1% (see gemm_prep.cuh for the
 // scaling that keeps fp32 range).  Loop state advances by counters: no
@@ -34,7 +47,7 @@
 namespace ql {
 namespace gemm {
 
-constexpr int BM = 256;  // tokens per tile: two MMA halves of 128
+constexpr int BM = 256;  // tokens per tile of the prefill form (the MMA's N)
 constexpr int BN = 128;  // weight rows per tile
 constexpr int BK = 64;
 constexpr int NUM_DEQ_WARPS = 8;
@@ -57,17 +70,23 @@ __host__ __device__ constexpr int code_bits(int fmt, int bits) {
 __host__ __device__ constexpr int p_row_bytes(int fmt, int bits) { return BK * code_bits(fmt, bits) / 8; }
 __host__ __device__ constexpr int p_bytes(int fmt, int bits) { return BN * p_row_bytes(fmt, bits); }
 
-// TT is the token tile: BM = 256 (two M = 128 MMAs per 16-k slice with the x tile as A, the weight
-// tile as B, N = 128) or TT_SWAP = 32 for small batches (one M = 128, N = 32 MMA per slice with the
-// weight tile as A and the x tile as B), whose accumulators are 32 TMEM columns.
+// TT is the token tile: BM = 256 (one M = 128, N = 256 MMA per 16-k slice, the weight tile as A in
+// TMEM, the x tile as B) or TT_SWAP = 32 for small batches (one M = 128, N = 32 MMA per slice, the
+// weight tile as A in shared memory), whose two accumulators are 32 TMEM columns each.
 __host__ __device__ constexpr int a_bytes(int tt) { return tt * BK * 2; }  // the fp16 x tile
-__host__ __device__ constexpr uint32_t tmem_cols(int tt) { return tt == BM ? 512u : 64u; }  // two accumulators
+__host__ __device__ constexpr int b_bytes(int tt) { return tt == BM ? 0 : B_BYTES; }  // weight tile in smem
+__host__ __device__ constexpr uint32_t tmem_cols(int tt) { return tt == BM ? 512u : 64u; }
+constexpr uint32_t TA_ACOL0 = BM;       // TT = 256: A stage s at TMEM columns 256 + 32 s
+constexpr uint32_t TA_ACOLS = BK / 2;   // 64 fp16 per row = 32 columns
+constexpr int STAGES_MAX_TA = 6;
 
-// Stages of the ring: as many as fit, up to four (six for the small x tile of the swapped form).
-// int4 adds the metadata ring [MSTAGES][BN rows][8 bytes] and its barriers.
+// Stages of the ring: as many as fit, up to six (TT = 256: six A stages of 32 columns fit beside the
+// 256-column accumulator).  int4 adds the metadata ring [MSTAGES][BN rows][8 bytes] and its barriers.
 constexpr int NUM_BARS_PER_STAGE = 3;  // tma_full, b_full, empty
 constexpr int NUM_BARS_FIXED = 5;      // acc_full[2], acc_empty[2], final
-__host__ __device__ constexpr int stage_bytes(int fmt, int bits, int tt) { return a_bytes(tt) + B_BYTES + p_bytes(fmt, bits); }
+__host__ __device__ constexpr int stage_bytes(int fmt, int bits, int tt) {
+  return a_bytes(tt) + b_bytes(tt) + p_bytes(fmt, bits);
+}
 __host__ __device__ constexpr int meta_bytes(int fmt) { return fmt == FMT_INT4 ? MSTAGES * META_STAGE_BYTES : 0; }
 __host__ __device__ constexpr int meta_bars(int fmt) { return fmt == FMT_INT4 ? 2 * MSTAGES : 0; }
 __host__ __device__ constexpr int smem_need(int fmt, int bits, int tt, int st) {
@@ -75,18 +94,18 @@ __host__ __device__ constexpr int smem_need(int fmt, int bits, int tt, int st) {
          (NUM_BARS_PER_STAGE * st + NUM_BARS_FIXED + meta_bars(fmt)) * 8 + 16 + 1024;
 }
 __host__ __device__ constexpr int stages(int fmt, int bits, int tt) {
-  return (tt != BM && smem_need(fmt, bits, tt, 6) <= SMEM_LIMIT) ? 6
-       : (tt != BM && smem_need(fmt, bits, tt, 5) <= SMEM_LIMIT) ? 5
+  return smem_need(fmt, bits, tt, 6) <= SMEM_LIMIT ? 6
+       : smem_need(fmt, bits, tt, 5) <= SMEM_LIMIT ? 5
        : smem_need(fmt, bits, tt, 4) <= SMEM_LIMIT ? 4 : 3;
 }
 
 // byte offsets inside the dynamic shared memory (base aligned to 1024)
 __host__ __device__ constexpr int off_a(int tt, int s) { return s * a_bytes(tt); }
 __host__ __device__ constexpr int off_b(int fmt, int bits, int tt, int s) {
-  return stages(fmt, bits, tt) * a_bytes(tt) + s * B_BYTES;
+  return stages(fmt, bits, tt) * a_bytes(tt) + s * b_bytes(tt);
 }
 __host__ __device__ constexpr int off_p(int fmt, int bits, int tt, int s) {
-  return stages(fmt, bits, tt) * (a_bytes(tt) + B_BYTES) + s * p_bytes(fmt, bits);
+  return stages(fmt, bits, tt) * (a_bytes(tt) + b_bytes(tt)) + s * p_bytes(fmt, bits);
 }
 __host__ __device__ constexpr int off_meta(int fmt, int bits, int tt, int s) {
   return stages(fmt, bits, tt) * stage_bytes(fmt, bits, tt) + s * META_STAGE_BYTES;
@@ -166,11 +185,110 @@ QL_DEVI void smem_decode32(const uint8_t *src, const uint8_t *src_hi, uint32_t g
   }
 }
 
+// Words of one 32-weight chunk's codes, read from shared memory (int4, affine): code_bits words.
+template <int FMT, int BITS>
+QL_DEVI void load_code_words(const uint8_t *src, uint32_t (&cw)[code_bits(FMT, BITS)]) {
+  if constexpr (code_bits(FMT, BITS) == 2) {
+    const uint2 v = *reinterpret_cast<const uint2 *>(src);
+    cw[0] = v.x;
+    cw[1] = v.y;
+  } else {
+#pragma unroll
+    for (int t = 0; t < code_bits(FMT, BITS) / 4; ++t) {
+      const uint4 v = reinterpret_cast<const uint4 *>(src)[t];
+      cw[4 * t] = v.x; cw[4 * t + 1] = v.y; cw[4 * t + 2] = v.z; cw[4 * t + 3] = v.w;
+    }
+  }
+}
+
+// One 32-weight chunk of a tile row -> 16 words of fp16 pairs, each weight times 2^b_n (sc is the
+// row's 2^b_n).  Word 4 q + e holds weights (8 q + e, 8 q + e + 4): the k order of the x tile, whose
+// 16-byte chunks hold k = 0,4,1,5,2,6,3,7 of their 8 values.  int4 and affine take the chunk's code
+// words `cw`; int6 (and int6 planar, with its high-plane bytes at `src_hi`) decode from `src`.
+template <int FMT, int BITS>
+QL_DEVI void chunk_to_f16(const uint32_t (&cw)[code_bits(FMT, BITS)], const uint8_t *src, const uint8_t *src_hi,
+                          uint32_t gm, uint32_t st, float sc, uint32_t (&o)[16]) {
+  if constexpr (FMT == FMT_INT4) {
+    // packed-half arithmetic: q as 1024+q / 64+q from one bit operation, then
+    // w * 2^b_n = q * S' - Z * S' in fp16 with S' = S * 2^b_n; the codes sc, zc become floats
+    // by placing the byte in the mantissa of 2^23 and subtracting 2^23 (exact)
+    const float scf = __uint_as_float(0x4B000000u | (gm & 0xffu)) - 8388608.f;
+    const float zcf = __uint_as_float(0x4B000000u | ((gm >> 8) & 0xffu)) - 8388608.f;
+    const float S = __fmul_rn(scf, f16_bits_to_f32(st)) * sc;
+    const float ZS = __fmul_rn(zcf, f16_bits_to_f32(st >> 16)) * S;
+    const __half2 s2 = __float2half2_rn(S), nz2 = __float2half2_rn(-ZS);
+    const __half2 m1024 = __float2half2_rn(1024.f), m64 = __float2half2_rn(64.f);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint32_t wd = cw[q], w8 = wd >> 8;
+      uint32_t pr[4];
+      pr[0] = (wd & 0x000F000Fu) | 0x64006400u;  // (1024 + n0, 1024 + n4)
+      pr[1] = (wd & 0x00F000F0u) | 0x54005400u;  // (64 + n1, 64 + n5)
+      pr[2] = (w8 & 0x000F000Fu) | 0x64006400u;  // (1024 + n2, 1024 + n6)
+      pr[3] = (w8 & 0x00F000F0u) | 0x54005400u;  // (64 + n3, 64 + n7)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const __half2 qv = __hsub2(*reinterpret_cast<const __half2 *>(&pr[e]), (e & 1) ? m64 : m1024);
+        const __half2 wv = __hfma2(qv, s2, nz2);
+        o[4 * q + e] = *reinterpret_cast<const uint32_t *>(&wv);
+      }
+    }
+  } else if constexpr (FMT == FMT_AFFINE) {
+    // packed-half arithmetic: the codes become 1024 + q halves by bit operations (q exact after
+    // one subtraction), then w * 2^b_n = q * s' + b' in one fused multiply-add with s' = s * 2^b_n
+    // and b' = b * 2^b_n, which are exact in fp16 (bf16 values scaled into fp16's range), so each
+    // weight is rounded once
+    const __half2 s2 = __float2half2_rn(bf16_bits_to_f32(gm) * sc);
+    const __half2 b2 = __float2half2_rn(bf16_bits_to_f32(gm >> 16) * sc);
+    const __half2 m1024 = __float2half2_rn(1024.f);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {  // output words 4q..: weights 8q .. 8q+7 of the chunk, as (k, k+4) pairs
+      uint32_t pr[4];
+      if constexpr (BITS == 4) {
+        const uint32_t wd = cw[q], w8 = wd >> 8;
+        pr[0] = (wd & 0x000F000Fu) | 0x64006400u;  // (1024 + n0, 1024 + n4)
+        pr[1] = ((wd >> 4) & 0x000F000Fu) | 0x64006400u;
+        pr[2] = (w8 & 0x000F000Fu) | 0x64006400u;
+        pr[3] = ((w8 >> 4) & 0x000F000Fu) | 0x64006400u;
+      } else if constexpr (BITS == 8) {
+        const uint32_t w0 = cw[2 * q], w1 = cw[2 * q + 1];  // k 0..3, k 4..7
+        const uint32_t t0 = __byte_perm(w0, w1, 0x5140), t1 = __byte_perm(w0, w1, 0x7362);  // (0 4 1 5) (2 6 3 7)
+        pr[0] = __byte_perm(t0, 0x64646464u, 0x4140);
+        pr[1] = __byte_perm(t0, 0x64646464u, 0x4342);
+        pr[2] = __byte_perm(t1, 0x64646464u, 0x4140);
+        pr[3] = __byte_perm(t1, 0x64646464u, 0x4342);
+      } else {  // 2-bit: codes 8q .. 8q+7 are bits 16 (q & 1) .. of word q / 2
+        const uint32_t wd = cw[q >> 1] >> (16 * (q & 1));
+        const uint32_t u = __byte_perm(wd, 0u, 0x4140);  // codes 0-3 in byte 0, codes 4-7 in byte 2
+#pragma unroll
+        for (int e = 0; e < 4; ++e) pr[e] = ((u >> (2 * e)) & 0x00030003u) | 0x64006400u;
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const __half2 qv = __hsub2(*reinterpret_cast<const __half2 *>(&pr[e]), m1024);
+        const __half2 wv = __hfma2(qv, s2, b2);
+        o[4 * q + e] = *reinterpret_cast<const uint32_t *>(&wv);
+      }
+    }
+  } else {
+    float w[32];
+    smem_decode32<FMT, BITS>(src, src_hi, gm, st, w);
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[4 * q + e] = pack_f16x2(w[8 * q + e] * sc, w[8 * q + e + 4] * sc);
+  }
+}
+
 template <int FMT, int BITS, int TT>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_codes,
                 Params p) {
-  constexpr bool SWAP = TT != BM;
+  constexpr bool SWAP = TT != BM;  // else the weight tile is the MMA's A operand in TMEM
+  constexpr int NACC = SWAP ? 2 : 1;  // accumulators in TMEM
+  // dequantising warps per stage: TT = 256 alternates stages between two groups of four
+  constexpr int DEQ_PER_STAGE = SWAP ? NUM_DEQ_WARPS : NUM_DEQ_WARPS / 2;
+  static_assert(SWAP || TA_ACOL0 + STAGES_MAX_TA * TA_ACOLS <= 512, "A ring beside the accumulator");
   constexpr int PROW = p_row_bytes(FMT, BITS);
   constexpr int STAGES = stages(FMT, BITS, TT);
   constexpr uint32_t STAGE_TX = a_bytes(TT) + p_bytes(FMT, BITS);
@@ -230,7 +348,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(bar_tma_full(s), 1);
-      mbar_init(bar_b_full(s), NUM_DEQ_WARPS);
+      mbar_init(bar_b_full(s), DEQ_PER_STAGE);
       mbar_init(bar_empty(s), 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -241,7 +359,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if constexpr (FMT == FMT_INT4) {
       for (int s = 0; s < MSTAGES; ++s) {
         mbar_init(bar_meta_full(s), NUM_META_WARPS * 32);  // one cp.async arrival per copying thread
-        mbar_init(bar_meta_empty(s), NUM_DEQ_WARPS);
+        mbar_init(bar_meta_empty(s), DEQ_PER_STAGE);
       }
     }
     *abort_flag = 0;
@@ -299,38 +417,35 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else if (warp == WARP_MMA) {
     if (lane == 0) {
-      constexpr uint32_t idesc = SWAP ? umma_idesc_f16_f32(BN, TT) : umma_idesc_f16_f32(128, BN);
+      // D[weight row][token] += W tile (A, M = 128) x x tile (B, N = TT)
+      constexpr uint32_t idesc = umma_idesc_f16_f32(BN, TT);
       int64_t tcount = 0;
       int s = 0;
       uint32_t ph = 0;
       bool ok = true, issued = false;
       for (int64_t tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++tcount) {
-        const int a = (int)(tcount & 1);
-        const uint32_t ause = (uint32_t)(tcount >> 1);
+        const int a = (int)(tcount % NACC);
+        const uint32_t ause = (uint32_t)(tcount / NACC);
         if (!mbar_wait_bounded(bar_acc_empty(a), (ause & 1) ^ 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        // accumulator a: columns a * 2 * BN .. (two token halves of BN columns) or, swapped, a * TT ..
-        const uint32_t d_tmem = tmem_base + (uint32_t)(SWAP ? a * TT : a * 2 * BN);
+        const uint32_t d_tmem = tmem_base + (uint32_t)(a * TT);  // accumulator a: columns a * TT ..
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait_bounded(bar_tma_full(s), ph, abort_flag) || !mbar_wait_bounded(bar_b_full(s), ph, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint64_t wdesc = umma_desc_k_sw128(sbase + off_b(FMT, BITS, TT, s));
-          if constexpr (SWAP) {  // D[weight row][token] += W tile (A, M = 128) x x tile (B, N = TT)
-            const uint64_t xdesc = umma_desc_k_sw128(sbase + off_a(TT, s));
+          const uint64_t xdesc = umma_desc_k_sw128(sbase + off_a(TT, s));
+          if constexpr (SWAP) {
+            const uint64_t wdesc = umma_desc_k_sw128(sbase + off_b(FMT, BITS, TT, s));
 #pragma unroll
             for (int kk = 0; kk < BK / 16; ++kk)  // advance 16 fp16 = 32 bytes = 2 descriptor units
               umma_f16(d_tmem, wdesc + 2 * kk, xdesc + 2 * kk, idesc, (kb | kk) != 0);
           } else {
+            const uint32_t a_tmem = tmem_base + TA_ACOL0 + (uint32_t)s * TA_ACOLS;  // lanes 0..127
 #pragma unroll
-            for (int hm = 0; hm < 2; ++hm) {  // token half: rows 128*hm.. of the x tile (16 KB in)
-              const uint64_t adesc = umma_desc_k_sw128(sbase + off_a(TT, s) + hm * (a_bytes(TT) / 2));
-#pragma unroll
-              for (int kk = 0; kk < BK / 16; ++kk)  // advance 16 fp16 = 32 bytes = 2 descriptor units
-                umma_f16(d_tmem + (uint32_t)(hm * BN), adesc + 2 * kk, wdesc + 2 * kk, idesc, (kb | kk) != 0);
-            }
+            for (int kk = 0; kk < BK / 16; ++kk)  // 16 fp16 = 8 TMEM columns; 32 bytes = 2 descriptor units
+              umma_f16_tmem_a(d_tmem, a_tmem + 8 * kk, xdesc + 2 * kk, idesc, (kb | kk) != 0);
           }
           umma_commit(bar_empty(s));
           issued = true;
@@ -373,89 +488,67 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       cp_async_wait_all();  // no copy may land after the CTA is gone
     }
   } else if (warp >= WARP_EPI0 && warp < WARP_EPI0 + 4) {
+    // lane = weight row n of the tile (TMEM lane 32 e + lane); its TT columns = the tile's tokens
     const int e = warp - WARP_EPI0;  // TMEM lane quarter
     int64_t tcount = 0;
-    const bool vec_ok = (p.N % 8) == 0;
     for (int64_t tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tcount) {
       const int64_t n_tile = tile / m_tiles, m_tile = tile - n_tile * m_tiles;
-      const int a = (int)(tcount & 1);
-      const uint32_t ause = (uint32_t)(tcount >> 1);
+      const int a = (int)(tcount % NACC);
+      const uint32_t ause = (uint32_t)(tcount / NACC);
       if (!mbar_wait_bounded(bar_acc_full(a), ause & 1, abort_flag)) break;
       tc_fence_after();
-      if constexpr (SWAP) {
-        // lane = weight row n of the tile (TMEM lane 32 e + lane), its TT columns = the tile's tokens
-        uint32_t r[32];
-        static_assert(TT == 32, "one 32-column TMEM load per row");
-        tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(32 * e) << 16) + (uint32_t)(a * TT), r);
+      const int64_t n = n_tile * BN + 32 * e + lane;
+      const int we = n < p.N ? p.ws.wexp[n] : 0;
+      const float bn = (p.bias && n < p.N) ? __bfloat162float(p.bias[n]) : 0.f;
+      // two neighbouring rows n, n + 1 of one token share a 4-byte store when every row of the warp
+      // exists and N is even (the row pair then starts on a 4-byte boundary)
+      const bool pairs = (p.N % 2) == 0 && n_tile * BN + 32 * e + 32 <= p.N;
+#pragma unroll 1
+      for (int c = 0; c < TT / 16; ++c) {  // 16 tokens at a time
+        uint32_t r[16];
+        tmem_ld_32x32b_x16(tmem_base + ((uint32_t)(32 * e) << 16) + (uint32_t)(a * TT + 16 * c), r);
         tmem_ld_wait();
-        const int64_t n = n_tile * BN + 32 * e + lane, m0 = m_tile * TT;
-        const int we = n < p.N ? p.ws.wexp[n] : 0;
-        const float bn = (p.bias && n < p.N) ? __bfloat162float(p.bias[n]) : 0.f;
-        const int xe_lane = m0 + lane < p.M ? p.ws.xexp[m0 + lane] : 0;
+        if (c == TT / 16 - 1) {  // the accumulator is in registers: the next tile's MMAs may start
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar_acc_empty(a));
+        }
+        const int64_t m0 = m_tile * TT + 16 * c;
+        const int xe_lane = m0 + (lane & 15) < p.M ? p.ws.xexp[m0 + (lane & 15)] : 0;
 #pragma unroll
-        for (int t = 0; t < TT; ++t) {  // y = D * 2^-(a_m + b_n) (exponents added first), + bias, one rounding
+        for (int t = 0; t < 16; ++t) {  // y = D * 2^-(a_m + b_n) (exponents added first), + bias, one rounding
           const int xe = __shfl_sync(0xffffffffu, xe_lane, t);
-          const float v = mul_pow2(__uint_as_float(r[t]), xe + we) + bn;
-          if (m0 + t < p.M && n < p.N) p.y[(m0 + t) * p.N + n] = __float2bfloat16_rn(v);
+          r[t] = __float_as_uint(mul_pow2(__uint_as_float(r[t]), xe + we) + bn);
         }
-      } else {
-#pragma unroll 1
-      for (int hm = 0; hm < 2; ++hm) {
-        const int64_t m = m_tile * BM + 128 * hm + 32 * e + lane;
-        const int xe = m < p.M ? p.ws.xexp[m] : 0;
-#pragma unroll 1
-        for (int cchunk = 0; cchunk < BN / 32; ++cchunk) {
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(32 * e) << 16) + (uint32_t)(a * 2 * BN + hm * BN + 32 * cchunk),
-                             r);
-          tmem_ld_wait();
-          const int64_t n0 = n_tile * BN + 32 * cchunk;
-          {  // y = D * 2^-(a_m + b_n): the two exponents are added first, then D is scaled exactly
-            const int4 *we = reinterpret_cast<const int4 *>(p.ws.wexp + n0);
+        if (pairs) {
+          // even lane: tokens 2t of rows n, n+1; odd lane: tokens 2t+1 of rows n-1, n
+          const int odd = lane & 1;
+          __nv_bfloat16 *dst = p.y + (m0 + odd) * p.N + (n - odd);
+          const int64_t rows_left = p.M - m0 - odd;
 #pragma unroll
-            for (int t = 0; t < 8; ++t) {
-              const int4 v = we[t];
-              r[4 * t + 0] = __float_as_uint(mul_pow2(__uint_as_float(r[4 * t + 0]), xe + v.x));
-              r[4 * t + 1] = __float_as_uint(mul_pow2(__uint_as_float(r[4 * t + 1]), xe + v.y));
-              r[4 * t + 2] = __float_as_uint(mul_pow2(__uint_as_float(r[4 * t + 2]), xe + v.z));
-              r[4 * t + 3] = __float_as_uint(mul_pow2(__uint_as_float(r[4 * t + 3]), xe + v.w));
-            }
+          for (int t = 0; t < 8; ++t) {  // (token 2t, token 2t+1) of row n as bf16, in place
+            r[t] = pack_bf16x2(__uint_as_float(r[2 * t]), __uint_as_float(r[2 * t + 1]));
           }
-          if (p.bias) {  // + bias[n], still in fp32 (fully unrolled: r stays in registers)
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (n0 + i < p.N) r[i] = __float_as_uint(__uint_as_float(r[i]) + __bfloat162float(p.bias[n0 + i]));
+          for (int t = 0; t < 8; ++t) {
+            const uint32_t other = __shfl_xor_sync(0xffffffffu, r[t], 1);  // the same tokens of row n^1
+            const uint32_t pr = odd ? __byte_perm(other, r[t], 0x7632) : __byte_perm(r[t], other, 0x5410);
+            if (2 * t < rows_left) *reinterpret_cast<uint32_t *>(dst) = pr;
+            dst += 2 * p.N;
           }
-          if (m < p.M) {
-            __nv_bfloat16 *dst = p.y + m * p.N + n0;
-            if (vec_ok && n0 + 32 <= p.N) {
+        } else {
 #pragma unroll
-              for (int t = 0; t < 4; ++t) {
-                uint4 v;
-                v.x = pack_bf16x2(__uint_as_float(r[8 * t + 0]), __uint_as_float(r[8 * t + 1]));
-                v.y = pack_bf16x2(__uint_as_float(r[8 * t + 2]), __uint_as_float(r[8 * t + 3]));
-                v.z = pack_bf16x2(__uint_as_float(r[8 * t + 4]), __uint_as_float(r[8 * t + 5]));
-                v.w = pack_bf16x2(__uint_as_float(r[8 * t + 6]), __uint_as_float(r[8 * t + 7]));
-                reinterpret_cast<uint4 *>(dst)[t] = v;
-              }
-            } else {
-#pragma unroll
-              for (int i = 0; i < 32; ++i)
-                if (n0 + i < p.N) dst[i] = __float2bfloat16_rn(__uint_as_float(r[i]));
-            }
-          }
+          for (int t = 0; t < 16; ++t)
+            if (m0 + t < p.M && n < p.N) p.y[(m0 + t) * p.N + n] = __float2bfloat16_rn(__uint_as_float(r[t]));
         }
       }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_acc_empty(a));
     }
   } else if (warp >= WARP_DEQ0) {
+    auto row_scale = [&](int64_t n) { return n < p.N ? p.ws.wsc[n] : 0.f; };
+    if constexpr (SWAP) {
     const int t = threadIdx.x - WARP_DEQ0 * 32;  // 0..255
     const int h = t & 1;                          // which 32-weight half of the 64-k stage
     const int r = t >> 1;                         // the tile row this thread fills
-    auto row_scale = [&](int64_t n) { return n < p.N ? p.ws.wsc[n] : 0.f; };
     Cursor nxt = cursor0();  // the stage after the current one
     advance(nxt);
     int s = 0, ms = 0;
@@ -488,96 +581,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       if (!mbar_wait_bounded(bar_tma_full(s), ph, abort_flag)) break;
       const uint8_t *src = smem + off_p(FMT, BITS, TT, s) + r * PROW + h * (PROW / 2);
+      const uint8_t *src_hi = nullptr;
+      if constexpr (FMT == FMT_INT6P) {  // boxes [2 low halves][BN rows][16 B], then [BN rows][16 B] high
+        src = smem + off_p(FMT, BITS, TT, s) + h * 16 * BN + r * 16;
+        src_hi = smem + off_p(FMT, BITS, TT, s) + 32 * BN + r * 16 + 8 * h;
+      }
+      uint32_t cw[code_bits(FMT, BITS)];
+      if constexpr (FMT == FMT_INT4 || FMT == FMT_AFFINE) load_code_words<FMT, BITS>(src, cw);
+      uint32_t o[16];
+      chunk_to_f16<FMT, BITS>(cw, src, src_hi, gm, st, sc, o);
       uint8_t *dst_row = row + off_b(FMT, BITS, TT, s);
-      // each 16-byte chunk holds k = 0,4,1,5,2,6,3,7 of its 8 weights (the order of the x tile)
-      if constexpr (FMT == FMT_INT4) {
-        // packed-half arithmetic: q as 1024+q / 64+q from one bit operation, then
-        // w * 2^b_n = q * S' - Z * S' in fp16 with S' = S * 2^b_n; the codes sc, zc become floats
-        // by placing the byte in the mantissa of 2^23 and subtracting 2^23 (exact)
-        const float scf = __uint_as_float(0x4B000000u | (gm & 0xffu)) - 8388608.f;
-        const float zcf = __uint_as_float(0x4B000000u | ((gm >> 8) & 0xffu)) - 8388608.f;
-        const float S = __fmul_rn(scf, f16_bits_to_f32(st)) * sc;
-        const float ZS = __fmul_rn(zcf, f16_bits_to_f32(st >> 16)) * S;
-        const __half2 s2 = __float2half2_rn(S), nz2 = __float2half2_rn(-ZS);
-        const __half2 m1024 = __float2half2_rn(1024.f), m64 = __float2half2_rn(64.f);
-        const uint4 cv = *reinterpret_cast<const uint4 *>(src);
-        const uint32_t cw[4] = {cv.x, cv.y, cv.z, cv.w};
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint32_t wd = cw[q], w8 = wd >> 8;
-          uint32_t pr[4];
-          pr[0] = (wd & 0x000F000Fu) | 0x64006400u;  // (1024 + n0, 1024 + n4)
-          pr[1] = (wd & 0x00F000F0u) | 0x54005400u;  // (64 + n1, 64 + n5)
-          pr[2] = (w8 & 0x000F000Fu) | 0x64006400u;  // (1024 + n2, 1024 + n6)
-          pr[3] = (w8 & 0x00F000F0u) | 0x54005400u;  // (64 + n3, 64 + n7)
-          uint32_t o[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const __half2 qv = __hsub2(*reinterpret_cast<const __half2 *>(&pr[e]), (e & 1) ? m64 : m1024);
-            const __half2 wv = __hfma2(qv, s2, nz2);
-            o[e] = *reinterpret_cast<const uint32_t *>(&wv);
-          }
-          const int j = 4 * h + q;  // logical 16-byte chunk of the 128-byte row
-          *reinterpret_cast<uint4 *>(dst_row + ((j ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-        }
-      } else if constexpr (FMT == FMT_AFFINE) {
-        // packed-half arithmetic: the codes become 1024 + q halves by bit operations (q exact after
-        // one subtraction), then w * 2^b_n = q * s' + b' in one fused multiply-add with s' = s * 2^b_n
-        // and b' = b * 2^b_n, which are exact in fp16 (bf16 values scaled into fp16's range), so each
-        // weight is rounded once
-        const __half2 s2 = __float2half2_rn(bf16_bits_to_f32(gm) * sc);
-        const __half2 b2 = __float2half2_rn(bf16_bits_to_f32(gm >> 16) * sc);
-        const __half2 m1024 = __float2half2_rn(1024.f);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {  // output chunk q: weights 8q .. 8q+7 of the thread's 32, as (k, k+4) pairs
-          uint32_t pr[4];
-          if constexpr (BITS == 4) {
-            const uint32_t wd = reinterpret_cast<const uint32_t *>(src)[q], w8 = wd >> 8;
-            pr[0] = (wd & 0x000F000Fu) | 0x64006400u;  // (1024 + n0, 1024 + n4)
-            pr[1] = ((wd >> 4) & 0x000F000Fu) | 0x64006400u;
-            pr[2] = (w8 & 0x000F000Fu) | 0x64006400u;
-            pr[3] = ((w8 >> 4) & 0x000F000Fu) | 0x64006400u;
-          } else if constexpr (BITS == 8) {
-            const uint32_t w0 = reinterpret_cast<const uint32_t *>(src)[2 * q];      // k 0..3
-            const uint32_t w1 = reinterpret_cast<const uint32_t *>(src)[2 * q + 1];  // k 4..7
-            const uint32_t t0 = __byte_perm(w0, w1, 0x5140), t1 = __byte_perm(w0, w1, 0x7362);  // (0 4 1 5) (2 6 3 7)
-            pr[0] = __byte_perm(t0, 0x64646464u, 0x4140);
-            pr[1] = __byte_perm(t0, 0x64646464u, 0x4342);
-            pr[2] = __byte_perm(t1, 0x64646464u, 0x4140);
-            pr[3] = __byte_perm(t1, 0x64646464u, 0x4342);
-          } else {  // 2-bit: codes 8q .. 8q+7 are bits 16 (q & 1) .. of word q / 2
-            const uint32_t wd = reinterpret_cast<const uint32_t *>(src)[q >> 1] >> (16 * (q & 1));
-            const uint32_t u = __byte_perm(wd, 0u, 0x4140);  // codes 0-3 in byte 0, codes 4-7 in byte 2
-#pragma unroll
-            for (int e = 0; e < 4; ++e) pr[e] = ((u >> (2 * e)) & 0x00030003u) | 0x64006400u;
-          }
-          uint32_t o[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const __half2 qv = __hsub2(*reinterpret_cast<const __half2 *>(&pr[e]), m1024);
-            const __half2 wv = __hfma2(qv, s2, b2);
-            o[e] = *reinterpret_cast<const uint32_t *>(&wv);
-          }
-          const int j = 4 * h + q;  // logical 16-byte chunk of the 128-byte row
-          *reinterpret_cast<uint4 *>(dst_row + ((j ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-        }
-      } else {
-        float w[32];
-        if constexpr (FMT == FMT_INT6P)  // boxes [2 low halves][BN rows][16 B], then [BN rows][16 B] high
-          smem_decode32<FMT, BITS>(smem + off_p(FMT, BITS, TT, s) + h * 16 * BN + r * 16,
-                                   smem + off_p(FMT, BITS, TT, s) + 32 * BN + r * 16 + 8 * h, gm, st, w);
-        else
-          smem_decode32<FMT, BITS>(src, nullptr, gm, st, w);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int j = 4 * h + q;  // logical 16-byte chunk of the 128-byte row
-          uint4 v;
-          v.x = pack_f16x2(w[8 * q + 0] * sc, w[8 * q + 4] * sc);
-          v.y = pack_f16x2(w[8 * q + 1] * sc, w[8 * q + 5] * sc);
-          v.z = pack_f16x2(w[8 * q + 2] * sc, w[8 * q + 6] * sc);
-          v.w = pack_f16x2(w[8 * q + 3] * sc, w[8 * q + 7] * sc);
-          *reinterpret_cast<uint4 *>(dst_row + ((j ^ (r & 7)) << 4)) = v;
-        }
+      for (int q = 0; q < 4; ++q) {
+        const int j = 4 * h + q;  // logical 16-byte chunk of the 128-byte row
+        *reinterpret_cast<uint4 *>(dst_row + ((j ^ (r & 7)) << 4)) = make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
       }
       fence_proxy_async_smem();
       __syncwarp();
@@ -586,6 +603,111 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       gm = ngm;
       st = nst;
       sc = nsc;
+    }
+    } else {
+      // Stages alternate between warps 8-11 (even) and 12-15 (odd).  A thread fills one whole tile
+      // row (64 weights, both 32-weight chunks) of its stage into TMEM lane r = its warp's lane
+      // quarter + lane, columns TA_ACOL0 + 32 s ..: the A operand of that stage's MMAs.
+      const int wd = warp - WARP_DEQ0;     // 0..7
+      const int g = wd >> 2;               // stages it = g, g + 2, ...
+      const int r = 32 * (wd & 3) + lane;  // tile row
+      const uint32_t t_row = tmem_base + ((uint32_t)(32 * (wd & 3)) << 16) + TA_ACOL0;
+      auto step2 = [](int &slot, uint32_t &phase, int depth) {
+        slot += 2;
+        if (slot >= depth) {
+          slot -= depth;
+          phase ^= 1u;
+        }
+      };
+      Cursor cur = cursor0();
+      if (g) advance(cur);
+      int s = g, ms = g;
+      uint32_t ph = 0, phm = 0;
+      uint32_t gm[2] = {0, 0}, st[2] = {0, 0};
+      float sc = 0.f;
+      if (g < total_it) {
+        if constexpr (FMT != FMT_INT4) {
+          load_meta<FMT>(p, cur.n_tile * BN + r, (int64_t)cur.kb * 2, gm[0], st[0]);
+          load_meta<FMT>(p, cur.n_tile * BN + r, (int64_t)cur.kb * 2 + 1, gm[1], st[1]);
+        }
+        sc = row_scale(cur.n_tile * BN + r);
+      }
+      for (int64_t it = g; it < total_it; it += 2) {
+        Cursor nx = cur;  // this group's next stage
+        advance(nx);
+        advance(nx);
+        uint32_t ngm[2] = {0, 0}, nst[2] = {0, 0};
+        float nsc = sc;
+        if (it + 2 < total_it) {  // its metadata (int6, affine) and row scale, loaded ahead
+          const int64_t n = nx.n_tile * BN + r;
+          if constexpr (FMT != FMT_INT4) {
+            load_meta<FMT>(p, n, (int64_t)nx.kb * 2, ngm[0], nst[0]);
+            load_meta<FMT>(p, n, (int64_t)nx.kb * 2 + 1, ngm[1], nst[1]);
+          }
+          if (nx.n_tile != cur.n_tile) nsc = row_scale(n);
+        }
+        if constexpr (FMT == FMT_INT4) {  // this stage's group and step words, from the metadata ring
+          if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar_meta_full(ms), phm, abort_flag))) break;
+          const uint2 mv = *reinterpret_cast<const uint2 *>(smem + off_meta(FMT, BITS, TT, ms) + r * 8);
+          gm[0] = mv.x & 0xffffu;
+          gm[1] = mv.x >> 16;
+          st[0] = st[1] = mv.y;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar_meta_empty(ms));
+          step2(ms, phm, MSTAGES);
+        }
+        // the codes have landed, and the MMAs that last read this A stage have completed (they
+        // released the stage before TMA refilled it)
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar_tma_full(s), ph, abort_flag))) break;
+        tc_fence_after();
+        const uint8_t *prow = smem + off_p(FMT, BITS, TT, s) + r * PROW;
+        uint32_t o[32];
+        if constexpr (PROW == 32 && (FMT == FMT_INT4 || FMT == FMT_AFFINE)) {
+          // the row's two 16-byte chunks, read in the order (h ^ bit 2 of r) so that the 32 lanes'
+          // first reads cover all 32 banks in four wavefronts (rows are 32 bytes apart)
+          const int sw = (r >> 2) & 1;
+          const uint4 va = reinterpret_cast<const uint4 *>(prow)[sw];
+          const uint4 vb = reinterpret_cast<const uint4 *>(prow)[sw ^ 1];
+          const uint4 c0 = sw ? vb : va, c1 = sw ? va : vb;
+          const uint32_t cw0[4] = {c0.x, c0.y, c0.z, c0.w}, cw1[4] = {c1.x, c1.y, c1.z, c1.w};
+          uint32_t o0[16], o1[16];
+          chunk_to_f16<FMT, BITS>(cw0, nullptr, nullptr, gm[0], st[0], sc, o0);
+          chunk_to_f16<FMT, BITS>(cw1, nullptr, nullptr, gm[1], st[1], sc, o1);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            o[i] = o0[i];
+            o[16 + i] = o1[i];
+          }
+        } else {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const uint8_t *src = prow + h * (PROW / 2);
+            const uint8_t *src_hi = nullptr;
+            if constexpr (FMT == FMT_INT6P) {
+              src = smem + off_p(FMT, BITS, TT, s) + h * 16 * BN + r * 16;
+              src_hi = smem + off_p(FMT, BITS, TT, s) + 32 * BN + r * 16 + 8 * h;
+            }
+            uint32_t cw[code_bits(FMT, BITS)];
+            if constexpr (FMT == FMT_INT4 || FMT == FMT_AFFINE) load_code_words<FMT, BITS>(src, cw);
+            uint32_t oh[16];
+            chunk_to_f16<FMT, BITS>(cw, src, src_hi, gm[h], st[h], sc, oh);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) o[16 * h + i] = oh[i];
+          }
+        }
+        tmem_st_32x32b_x32(t_row + (uint32_t)s * TA_ACOLS, o);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_b_full(s));
+        step2(s, ph, STAGES);
+        cur = nx;
+        sc = nsc;
+        gm[0] = ngm[0];
+        gm[1] = ngm[1];
+        st[0] = nst[0];
+        st[1] = nst[1];
+      }
     }
   }
 
