@@ -39,8 +39,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM bytes per GEMV launch from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum),
 # valid only while the GEMV source is unchanged (hash of csrc/gemv.cuh at capture time).
-NCU_TRAFFIC = {"gemv_src_sha256": "b76e9422f26698306dcff9da9dd4dccb16430113d0cc20bc5e5390e8ac0408b1",
-               "bytes_per_launch": 83321088}  # mean over the two decode layers
+NCU_TRAFFIC = {"gemv_src_sha256": "e96a8dbc0350f04aaba0ef5fcaa3db81b517d0102074e935a68b0e258c1b5f39",
+               "bytes_per_launch": 83039104}  # mean over the two decode layers
 
 
 def parse_args(argv=None):

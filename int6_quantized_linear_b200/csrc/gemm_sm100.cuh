@@ -89,8 +89,10 @@ __host__ __device__ constexpr int stage_bytes(int fmt, int bits, int tt) {
 }
 __host__ __device__ constexpr int meta_bytes(int fmt) { return fmt == FMT_INT4 ? MSTAGES * META_STAGE_BYTES : 0; }
 __host__ __device__ constexpr int meta_bars(int fmt) { return fmt == FMT_INT4 ? 2 * MSTAGES : 0; }
+// each epilogue warp's copy of the tile's token scale exponents, one signed byte per token
+__host__ __device__ constexpr int xe_bytes(int tt) { return 4 * tt; }
 __host__ __device__ constexpr int smem_need(int fmt, int bits, int tt, int st) {
-  return st * stage_bytes(fmt, bits, tt) + meta_bytes(fmt) +
+  return st * stage_bytes(fmt, bits, tt) + meta_bytes(fmt) + xe_bytes(tt) +
          (NUM_BARS_PER_STAGE * st + NUM_BARS_FIXED + meta_bars(fmt)) * 8 + 16 + 1024;
 }
 __host__ __device__ constexpr int stages(int fmt, int bits, int tt) {
@@ -110,9 +112,10 @@ __host__ __device__ constexpr int off_p(int fmt, int bits, int tt, int s) {
 __host__ __device__ constexpr int off_meta(int fmt, int bits, int tt, int s) {
   return stages(fmt, bits, tt) * stage_bytes(fmt, bits, tt) + s * META_STAGE_BYTES;
 }
-__host__ __device__ constexpr int off_bar(int fmt, int bits, int tt) {
+__host__ __device__ constexpr int off_xe(int fmt, int bits, int tt) {
   return stages(fmt, bits, tt) * stage_bytes(fmt, bits, tt) + meta_bytes(fmt);
 }
+__host__ __device__ constexpr int off_bar(int fmt, int bits, int tt) { return off_xe(fmt, bits, tt) + xe_bytes(tt); }
 // barriers: tma_full[S], b_full[S], empty[S], acc_full[2], acc_empty[2], final, (int4) meta_full[MS],
 // meta_empty[MS]; then the tmem base and the abort flag
 __host__ __device__ constexpr int smem_bytes(int fmt, int bits, int tt) {
@@ -495,14 +498,36 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int64_t n_tile = tile / m_tiles, m_tile = tile - n_tile * m_tiles;
       const int a = (int)(tcount % NACC);
       const uint32_t ause = (uint32_t)(tcount / NACC);
-      if (!mbar_wait_bounded(bar_acc_full(a), ause & 1, abort_flag)) break;
-      tc_fence_after();
+      // the tile's scale exponents and bias, loaded while its MMAs run: lane l holds the exponents of
+      // tokens l, l + 32, .. (a load per column chunk would put an L2 round trip between the chunks)
       const int64_t n = n_tile * BN + 32 * e + lane;
       const int we = n < p.N ? p.ws.wexp[n] : 0;
       const float bn = (p.bias && n < p.N) ? __bfloat162float(p.bias[n]) : 0.f;
-      // two neighbouring rows n, n + 1 of one token share a 4-byte store when every row of the warp
-      // exists and N is even (the row pair then starts on a 4-byte boundary)
-      const bool pairs = (p.N % 2) == 0 && n_tile * BN + 32 * e + 32 <= p.N;
+      // (each exponent lies in [-126, 126], so one signed byte holds it: a chunk's 16 are one broadcast
+      // 16-byte load from this warp's own copy, which no other warp touches)
+      int8_t *xe_s = reinterpret_cast<int8_t *>(smem + off_xe(FMT, BITS, TT)) + TT * e;
+      int xe_lo = 1 << 20, xe_hi = -(1 << 20);
+      __syncwarp();  // every lane is done with the previous tile's copy
+#pragma unroll
+      for (int j = 0; j < TT / 32; ++j) {
+        const int64_t m = m_tile * TT + 32 * j + lane;
+        const int xe = m < p.M ? p.ws.xexp[m] : 0;
+        xe_s[32 * j + lane] = (int8_t)xe;
+        xe_lo = min(xe_lo, xe);
+        xe_hi = max(xe_hi, xe);
+      }
+      __syncwarp();
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        xe_lo = min(xe_lo, __shfl_xor_sync(0xffffffffu, xe_lo, o));
+        xe_hi = max(xe_hi, __shfl_xor_sync(0xffffffffu, xe_hi, o));
+      }
+      // every exponent sum of the warp's rows and the tile's tokens is that of a normal float: then
+      // D * 2^e is one multiplication by 2^e built from its bits, the same single rounding as mul_pow2
+      const bool one_mul = __all_sync(0xffffffffu, xe_lo + we >= -126 && xe_hi + we <= 127);
+      const int w_bits = we * (1 << 23) + 0x3F800000;  // bits of 2^(xe + we) = xe * 2^23 + w_bits
+      if (!mbar_wait_bounded(bar_acc_full(a), ause & 1, abort_flag)) break;
+      tc_fence_after();
 #pragma unroll 1
       for (int c = 0; c < TT / 16; ++c) {  // 16 tokens at a time
         uint32_t r[16];
@@ -514,32 +539,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (lane == 0) mbar_arrive(bar_acc_empty(a));
         }
         const int64_t m0 = m_tile * TT + 16 * c;
-        const int xe_lane = m0 + (lane & 15) < p.M ? p.ws.xexp[m0 + (lane & 15)] : 0;
+        const uint4 xv = *reinterpret_cast<const uint4 *>(xe_s + 16 * c);  // tokens 16c .. 16c + 15
+        const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+        // y = D * 2^-(a_m + b_n) (exponents added first), + bias, one rounding
+        if (one_mul) {
 #pragma unroll
-        for (int t = 0; t < 16; ++t) {  // y = D * 2^-(a_m + b_n) (exponents added first), + bias, one rounding
-          const int xe = __shfl_sync(0xffffffffu, xe_lane, t);
-          r[t] = __float_as_uint(mul_pow2(__uint_as_float(r[t]), xe + we) + bn);
-        }
-        if (pairs) {
-          // even lane: tokens 2t of rows n, n+1; odd lane: tokens 2t+1 of rows n-1, n
-          const int odd = lane & 1;
-          __nv_bfloat16 *dst = p.y + (m0 + odd) * p.N + (n - odd);
-          const int64_t rows_left = p.M - m0 - odd;
-#pragma unroll
-          for (int t = 0; t < 8; ++t) {  // (token 2t, token 2t+1) of row n as bf16, in place
-            r[t] = pack_bf16x2(__uint_as_float(r[2 * t]), __uint_as_float(r[2 * t + 1]));
-          }
-#pragma unroll
-          for (int t = 0; t < 8; ++t) {
-            const uint32_t other = __shfl_xor_sync(0xffffffffu, r[t], 1);  // the same tokens of row n^1
-            const uint32_t pr = odd ? __byte_perm(other, r[t], 0x7632) : __byte_perm(r[t], other, 0x5410);
-            if (2 * t < rows_left) *reinterpret_cast<uint32_t *>(dst) = pr;
-            dst += 2 * p.N;
+          for (int t = 0; t < 16; ++t) {
+            const int xe = (int)(int8_t)(xw[t >> 2] >> (8 * (t & 3)));
+            r[t] = __float_as_uint(__fmul_rn(__uint_as_float(r[t]), __int_as_float(xe * (1 << 23) + w_bits)) + bn);
           }
         } else {
 #pragma unroll
-          for (int t = 0; t < 16; ++t)
-            if (m0 + t < p.M && n < p.N) p.y[(m0 + t) * p.N + n] = __float2bfloat16_rn(__uint_as_float(r[t]));
+          for (int t = 0; t < 16; ++t) {
+            const int xe = (int)(int8_t)(xw[t >> 2] >> (8 * (t & 3)));
+            r[t] = __float_as_uint(mul_pow2(__uint_as_float(r[t]), xe + we) + bn);
+          }
+        }
+        if (n < p.N) {  // token t of row n: the warp's 32 rows are 64 contiguous bytes of y's row m0 + t
+          __nv_bfloat16 *dst = p.y + m0 * p.N + n;
+          const int64_t rows_left = p.M - m0;
+#pragma unroll
+          for (int t = 0; t < 16; ++t) {
+            if (t < rows_left) *dst = __float2bfloat16_rn(__uint_as_float(r[t]));
+            dst += p.N;
+          }
         }
       }
     }
