@@ -123,6 +123,13 @@ QL_DEVI void cp_async4(uint32_t dst, const void *src, bool valid) {
                "r"(valid ? 4 : 0)
                : "memory");
 }
+// 16-byte asynchronous copy global -> shared (both addresses 16-byte aligned); with valid == false the
+// 16 bytes are zero-filled and src is not read.
+QL_DEVI void cp_async16(uint32_t dst, const void *src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(reinterpret_cast<uint64_t>(src)),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
 // The mbarrier receives one arrival once every cp.async this thread issued before has landed
 // (counted in the barrier's expected arrivals).
 QL_DEVI void cp_async_arrive_noinc(uint32_t bar) {

@@ -23,8 +23,8 @@
 //   warp 0      TMA producer: scaled fp16 x tile (TT x 64, 128-byte
 //               swizzle) and the packed code tile (128 rows x BK codes)
 //   warp 1      TMEM allocator; lane 0 issues tcgen05.mma (f16 x f16 -> f32)
-//   warps 2-3   (int4) copy each stage's group and step words into a
-//               metadata ring, MSTAGES ahead
+//   warps 2-3   (int4) copy each super-block's group and step words into a
+//               metadata ring, MSLOTS super-blocks ahead
 //   warps 4-7   epilogue: tcgen05.ld the accumulator (warp w reads TMEM lanes
 //               32*(w%4).., one weight row per lane), undo the two
 //               power-of-two scales (exponents added first), round to bf16,
@@ -60,8 +60,12 @@ constexpr int WARP_DEQ0 = 8;
 constexpr int NUM_THREADS = (WARP_DEQ0 + NUM_DEQ_WARPS) * 32;
 constexpr int B_BYTES = BN * BK * 2;  // 16 KB: the dequantised weight tile
 constexpr int TT_SWAP = 32;           // token tile of the swapped form (weights as the M = 128 operand)
-constexpr int MSTAGES = 8;            // metadata ring depth (int4)
-constexpr int META_STAGE_BYTES = BN * 8;  // per tile row: the stage's two group words (u32), its step word
+// int4 metadata ring: one slot per 256-weight super-block (four k-stages): [BN rows][16 bytes] of group
+// words (the u32 of stage kb holds its two 32-weight groups), then [BN rows][4 bytes] of step words.
+// Whole super-blocks make a row's copy one 16-byte and one 4-byte cp.async, against two 4-byte copies a
+// stage, each from another row's line (int4 K is a multiple of 256, so no super-block straddles tiles).
+constexpr int MSLOTS = 3;
+constexpr int META_SLOT_BYTES = BN * 16 + BN * 4;
 constexpr int SMEM_LIMIT = 232448;        // dynamic shared memory a CTA may use
 
 __host__ __device__ constexpr int code_bits(int fmt, int bits) {
@@ -81,14 +85,14 @@ constexpr uint32_t TA_ACOLS = BK / 2;   // 64 fp16 per row = 32 columns
 constexpr int STAGES_MAX_TA = 6;
 
 // Stages of the ring: as many as fit, up to six (TT = 256: six A stages of 32 columns fit beside the
-// 256-column accumulator).  int4 adds the metadata ring [MSTAGES][BN rows][8 bytes] and its barriers.
+// 256-column accumulator).  int4 adds the metadata ring [MSLOTS][META_SLOT_BYTES] and its barriers.
 constexpr int NUM_BARS_PER_STAGE = 3;  // tma_full, b_full, empty
 constexpr int NUM_BARS_FIXED = 5;      // acc_full[2], acc_empty[2], final
 __host__ __device__ constexpr int stage_bytes(int fmt, int bits, int tt) {
   return a_bytes(tt) + b_bytes(tt) + p_bytes(fmt, bits);
 }
-__host__ __device__ constexpr int meta_bytes(int fmt) { return fmt == FMT_INT4 ? MSTAGES * META_STAGE_BYTES : 0; }
-__host__ __device__ constexpr int meta_bars(int fmt) { return fmt == FMT_INT4 ? 2 * MSTAGES : 0; }
+__host__ __device__ constexpr int meta_bytes(int fmt) { return fmt == FMT_INT4 ? MSLOTS * META_SLOT_BYTES : 0; }
+__host__ __device__ constexpr int meta_bars(int fmt) { return fmt == FMT_INT4 ? 2 * MSLOTS : 0; }
 // each epilogue warp's copy of the tile's token scale exponents, one signed byte per token
 __host__ __device__ constexpr int xe_bytes(int tt) { return 4 * tt; }
 __host__ __device__ constexpr int smem_need(int fmt, int bits, int tt, int st) {
@@ -110,7 +114,7 @@ __host__ __device__ constexpr int off_p(int fmt, int bits, int tt, int s) {
   return stages(fmt, bits, tt) * (a_bytes(tt) + b_bytes(tt)) + s * p_bytes(fmt, bits);
 }
 __host__ __device__ constexpr int off_meta(int fmt, int bits, int tt, int s) {
-  return stages(fmt, bits, tt) * stage_bytes(fmt, bits, tt) + s * META_STAGE_BYTES;
+  return stages(fmt, bits, tt) * stage_bytes(fmt, bits, tt) + s * META_SLOT_BYTES;
 }
 __host__ __device__ constexpr int off_xe(int fmt, int bits, int tt) {
   return stages(fmt, bits, tt) * stage_bytes(fmt, bits, tt) + meta_bytes(fmt);
@@ -310,7 +314,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   auto bar_acc_empty = [&](int a) { return smem_u32(bars + 3 * STAGES + 2 + a); };
   const uint32_t bar_final = smem_u32(bars + 3 * STAGES + 4);
   auto bar_meta_full = [&](int s) { return smem_u32(bars + 3 * STAGES + 5 + s); };
-  auto bar_meta_empty = [&](int s) { return smem_u32(bars + 3 * STAGES + 5 + MSTAGES + s); };
+  auto bar_meta_empty = [&](int s) { return smem_u32(bars + 3 * STAGES + 5 + MSLOTS + s); };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t m_tiles = (p.M + TT - 1) / TT, n_tiles = (p.N + BN - 1) / BN;
@@ -360,9 +364,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     mbar_init(bar_final, 1);
     if constexpr (FMT == FMT_INT4) {
-      for (int s = 0; s < MSTAGES; ++s) {
+      for (int s = 0; s < MSLOTS; ++s) {
         mbar_init(bar_meta_full(s), NUM_META_WARPS * 32);  // one cp.async arrival per copying thread
-        mbar_init(bar_meta_empty(s), DEQ_PER_STAGE);
+        mbar_init(bar_meta_empty(s), NUM_DEQ_WARPS);        // every dequantising warp, once a super-block
       }
     }
     *abort_flag = 0;
@@ -466,13 +470,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else if (warp >= WARP_META0 && warp < WARP_META0 + NUM_META_WARPS) {
     if constexpr (FMT == FMT_INT4) {
-      // for every stage, each tile row's group words (u32 holding the stage's two 32-weight groups)
-      // and its super-block step word, up to MSTAGES stages ahead of the dequantisers
+      // for every super-block, each tile row's 16 bytes of group words and its step word, up to
+      // MSLOTS super-blocks ahead of the dequantisers
       const int t = threadIdx.x - WARP_META0 * 32;  // 0..63: rows t and t + 64
       int ms = 0;
       uint32_t phm = 0;
       Cursor cur = cursor0();
-      for (int64_t it = 0; it < total_it; ++it) {
+      for (int64_t it = 0; it < total_it; it += 4) {
         if (!mbar_wait_bounded(bar_meta_empty(ms), phm ^ 1u, abort_flag)) break;
         const uint32_t dst = sbase + off_meta(FMT, BITS, TT, ms);
 #pragma unroll
@@ -481,12 +485,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const int64_t n = cur.n_tile * BN + r;
           const bool valid = n < p.N;
           const int64_t nn = valid ? n : p.N - 1;
-          cp_async4(dst + r * 8, p.gmeta + nn * (p.K / 16) + 4 * cur.kb, valid);
-          cp_async4(dst + r * 8 + 4, p.steps + 4 * (nn * (p.K / 256) + cur.kb / 4), valid);
+          cp_async16(dst + r * 16, p.gmeta + nn * (p.K / 16) + 16 * (cur.kb >> 2), valid);
+          cp_async4(dst + BN * 16 + r * 4, p.steps + 4 * (nn * (p.K / 256) + (cur.kb >> 2)), valid);
         }
         cp_async_arrive_noinc(bar_meta_full(ms));
-        step_ring(ms, phm, MSTAGES);
-        advance(cur);
+        step_ring(ms, phm, MSLOTS);
+        for (int j = 0; j < 4; ++j) advance(cur);
       }
       cp_async_wait_all();  // no copy may land after the CTA is gone
     }
@@ -594,13 +598,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       advance(nxt);
       if constexpr (FMT == FMT_INT4) {  // this stage's group and step words, from the metadata ring
-        if (!mbar_wait_bounded(bar_meta_full(ms), phm, abort_flag)) break;
-        const uint2 mv = *reinterpret_cast<const uint2 *>(smem + off_meta(FMT, BITS, TT, ms) + r * 8);
-        gm = (mv.x >> (16 * h)) & 0xffffu;
-        st = mv.y;
-        __syncwarp();
-        if ((t & 31) == 0) mbar_arrive(bar_meta_empty(ms));
-        step_ring(ms, phm, MSTAGES);
+        const int q = (int)(it & 3);      // stage of the super-block
+        if (q == 0 && !mbar_wait_bounded(bar_meta_full(ms), phm, abort_flag)) break;
+        const uint8_t *slot = smem + off_meta(FMT, BITS, TT, ms);
+        gm = (*reinterpret_cast<const uint32_t *>(slot + r * 16 + 4 * q) >> (16 * h)) & 0xffffu;
+        st = *reinterpret_cast<const uint32_t *>(slot + BN * 16 + r * 4);
+        if (q == 3) {  // the super-block's last stage: release the slot
+          __syncwarp();
+          if ((t & 31) == 0) mbar_arrive(bar_meta_empty(ms));
+          step_ring(ms, phm, MSLOTS);
+        }
       }
       if (!mbar_wait_bounded(bar_tma_full(s), ph, abort_flag)) break;
       const uint8_t *src = smem + off_p(FMT, BITS, TT, s) + r * PROW + h * (PROW / 2);
@@ -644,7 +651,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       };
       Cursor cur = cursor0();
       if (g) advance(cur);
-      int s = g, ms = g;
+      int s = g, ms = 0;  // both groups visit every super-block's slot
       uint32_t ph = 0, phm = 0;
       uint32_t gm[2] = {0, 0}, st[2] = {0, 0};
       float sc = 0.f;
@@ -670,14 +677,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (nx.n_tile != cur.n_tile) nsc = row_scale(n);
         }
         if constexpr (FMT == FMT_INT4) {  // this stage's group and step words, from the metadata ring
-          if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar_meta_full(ms), phm, abort_flag))) break;
-          const uint2 mv = *reinterpret_cast<const uint2 *>(smem + off_meta(FMT, BITS, TT, ms) + r * 8);
-          gm[0] = mv.x & 0xffffu;
-          gm[1] = mv.x >> 16;
-          st[0] = st[1] = mv.y;
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar_meta_empty(ms));
-          step2(ms, phm, MSTAGES);
+          const int q = (int)(it & 3);  // stage of the super-block: this group sees q = g and g + 2
+          if (q == g && !__all_sync(0xffffffffu, mbar_wait_bounded(bar_meta_full(ms), phm, abort_flag))) break;
+          const uint8_t *slot = smem + off_meta(FMT, BITS, TT, ms);
+          const uint32_t w = *reinterpret_cast<const uint32_t *>(slot + r * 16 + 4 * q);
+          gm[0] = w & 0xffffu;
+          gm[1] = w >> 16;
+          st[0] = st[1] = *reinterpret_cast<const uint32_t *>(slot + BN * 16 + r * 4);
+          if (q == g + 2) {  // this group's last stage of the super-block: release the slot
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_meta_empty(ms));
+            step_ring(ms, phm, MSLOTS);
+          }
         }
         // the codes have landed, and the MMAs that last read this A stage have completed (they
         // released the stage before TMA refilled it)
