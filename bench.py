@@ -629,21 +629,27 @@ def run_e2e(args, layers, device, step_bytes):
 
     import int6_quantized_linear_b200 as ql
 
-    xh = [L["x"].cpu().pin_memory() for L in layers]
-    yh = [torch.empty(L["y"].shape, dtype=torch.bfloat16).pin_memory() for L in layers]
-    h2d = sum(x.numel() * 2 for x in xh)
-    d2h = sum(y.numel() * 2 for y in yh)
+    # the step's inputs (both layers' x) in one pinned host buffer and one device buffer, its results
+    # likewise: one copy each way per step; every layer's slice starts on a 16-byte boundary
+    xs, ys = [L["x"].reshape(-1) for L in layers], [L["y"].reshape(-1) for L in layers]
+    assert all(t.numel() % 8 == 0 for t in xs + ys)
+    xh = torch.cat([t.cpu() for t in xs]).pin_memory()
+    yh = torch.empty(sum(t.numel() for t in ys), dtype=torch.bfloat16).pin_memory()
+    xd = torch.empty(xh.numel(), dtype=torch.bfloat16, device=device)
+    yd = torch.empty(yh.numel(), dtype=torch.bfloat16, device=device)
+    xv = list(torch.split(xd, [t.numel() for t in xs]))
+    yv = list(torch.split(yd, [t.numel() for t in ys]))
+    h2d = xh.numel() * 2
+    d2h = yh.numel() * 2
 
     stream = torch.cuda.current_stream(device)
 
     def step(i):  # the step's inputs in, its layers back to back (chained on the stream), its results out
-        for L, xhost in zip(layers, xh):
-            L["x"].copy_(xhost, non_blocking=True)
-        for L in layers:
+        xd.copy_(xh, non_blocking=True)
+        for L, x, y in zip(layers, xv, yv):
             c, g, s = L["reps"][i % len(L["reps"])]
-            ql.qlinear_gemv(L["desc"], c, g, s, L["x"], 1, L["y"], L["ws"], stream)
-        for L, yhost in zip(layers, yh):
-            yhost.copy_(L["y"], non_blocking=True)
+            ql.qlinear_gemv(L["desc"], c, g, s, x, 1, y, L["ws"], stream)
+        yh.copy_(yd, non_blocking=True)
 
     for i in range(args.warmup):
         step(i)
