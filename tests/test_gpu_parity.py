@@ -135,6 +135,25 @@ def test_gemm_full_size_sampled(cuda, M):
     assert_close(y[np.ix_(toks, rows)], y_ref, f"gemm full M={M}")
 
 
+@pytest.mark.parametrize("fmt,bits,group", [("int4", 0, 0), ("int6", 0, 0), ("affine", 4, 64)])
+@pytest.mark.parametrize("M", [24, 600])
+def test_gemm_ragged_multi_tile(cuda, fmt, bits, group, M):
+    """Several tiles per CTA in both GEMM forms, with a ragged last row tile (N = 20000 = 156 x 128 +
+    32): M = 24 runs the 32-token form (157 tiles, so some CTAs use both accumulators in turn), M = 600
+    the 256-token form (3 x 157 tiles, the last token tile 88 tokens: the accumulator is handed from
+    tile to tile).  Sampled rows (the last 40 included) and tokens against the oracle; a second call
+    must give the same bits."""
+    N, K = 20000, 1024
+    L = Layer(fmt, N, K, seed=7 * M + K, bits=bits, group=group)
+    rows = np.unique(np.concatenate([_sampled_rows(N, 160, M), np.arange(N - 40, N)]))
+    w_ref = L.oracle_w(rows)
+    xb, xd = x_dev(K, M, seed=M + 11)
+    y = run_gemm(L, xd, M)
+    toks = _sampled_rows(M, 48, M + 3)
+    assert_close(y[np.ix_(toks, rows)], OC.matmul_f64(xb[toks], w_ref), f"gemm {fmt} N={N} K={K} M={M}")
+    assert np.array_equal(y, run_gemm(L, xd, M))
+
+
 def test_gemm_error_budget(cuda):
     """fp16 operands with per-row power-of-two scales: the only rounding beyond fp32 accumulation is
     one 11-bit rounding per weight, so the error stays far inside the gate (bf16 weights would use ~100%)."""
