@@ -4,21 +4,20 @@
 //
 // Persistent kernel, one CTA per SM, tiles of BN=128 weight rows x TT tokens,
 // K streamed in BK=64 steps through a shared-memory ring of x and code tiles.
-// Two forms:
-//   TT = 256 (prefill): the dequantised weight tile never touches shared
-//     memory.  The dequantisers write it into tensor memory (TMEM), where one
-//     MMA of M = 128 (weight rows, A read from TMEM) x N = 256 (tokens, B = the
-//     x tile in shared memory) per 16-k slice consumes it.  Shared memory then
-//     carries only the x tile (written once by TMA, read once by the tensor
-//     core) and the packed codes, which is what bounds this form: a
-//     shared-memory weight tile would add its store, and a second token half
-//     would read it again, roughly doubling the bytes shared memory moves per
-//     MMA.  The accumulator (128 lanes x 256 columns) and a ring of A stages
-//     (32 columns each) share the 512 TMEM columns, so there is one
-//     accumulator and the epilogue of a tile runs between two tiles' MMAs.
-//   TT = 32 (small batches): the dequantised tile goes to shared memory in the
-//     canonical K-major 128-byte-swizzled layout as the A operand (M = 128),
-//     against a 32-token x tile as B (N = 32), with two accumulators.
+// The dequantised weight tile never touches shared memory: the dequantisers
+// write it into tensor memory (TMEM), where the MMAs of M = 128 (weight rows,
+// A read from TMEM) x N = TT (tokens, B = the x tile in shared memory) consume
+// it.  Shared memory then carries only the x tile (written once by TMA, read
+// once by the tensor core) and the packed codes, which is what bounds the
+// 256-token form: a shared-memory weight tile would add its store, and a second
+// token half would read it again, roughly doubling the bytes shared memory
+// moves per MMA.  Two token tiles:
+//   TT = 256 (prefill): one M = 128, N = 256 MMA per 16-k slice.  The
+//     accumulator (128 lanes x 256 columns) and a ring of A stages (32 columns
+//     each) share the 512 TMEM columns, so there is one accumulator and the
+//     epilogue of a tile runs between two tiles' MMAs.
+//   TT = 32 (up to 32 tokens): one M = 128, N = 32 MMA per slice, two 32-column
+//     accumulators (an epilogue overlaps the next tile), the A ring beside them.
 // Warp roles:
 //   warp 0      TMA producer: scaled fp16 x tile (TT x 64, 128-byte
 //               swizzle) and the packed code tile (128 rows x BK codes)
@@ -30,10 +29,9 @@
 //               power-of-two scales (exponents added first), round to bf16,
 //               store y
 //   warps 8-15  dequantisers: packed codes + metadata -> weight times 2^b_n
-//               -> fp16.  TT = 256: warps 8-11 fill even stages and 12-15 odd
-//               ones, one whole 64-weight tile row per thread, into the TMEM
-//               lanes of the warp's quarter.  TT = 32: one tile row and 32
-//               weights per thread and stage, into shared memory.
+//               -> fp16.  Warps 8-11 fill even stages and 12-15 odd ones, one
+//               whole 64-weight tile row per thread, into the TMEM lanes of the
+//               warp's quarter.
 // The operands are fp16 rather than bf16 because rounding every weight to
 // bf16 costs ~1% of rms(y); fp16 costs ~0.1% (see gemm_prep.cuh for the
 // scaling that keeps fp32 range).  Loop state advances by counters: no
@@ -58,8 +56,7 @@ constexpr int NUM_META_WARPS = 2;
 constexpr int WARP_EPI0 = 4;
 constexpr int WARP_DEQ0 = 8;
 constexpr int NUM_THREADS = (WARP_DEQ0 + NUM_DEQ_WARPS) * 32;
-constexpr int B_BYTES = BN * BK * 2;  // 16 KB: the dequantised weight tile
-constexpr int TT_SWAP = 32;           // token tile of the swapped form (weights as the M = 128 operand)
+constexpr int TT_SMALL = 32;          // token tile for up to 32 tokens
 // int4 metadata ring: one slot per 256-weight super-block (four k-stages): [BN rows][16 bytes] of group
 // words (the u32 of stage kb holds its two 32-weight groups), then [BN rows][4 bytes] of step words.
 // Whole super-blocks make a row's copy one 16-byte and one 4-byte cp.async, against two 4-byte copies a
@@ -74,14 +71,13 @@ __host__ __device__ constexpr int code_bits(int fmt, int bits) {
 __host__ __device__ constexpr int p_row_bytes(int fmt, int bits) { return BK * code_bits(fmt, bits) / 8; }
 __host__ __device__ constexpr int p_bytes(int fmt, int bits) { return BN * p_row_bytes(fmt, bits); }
 
-// TT is the token tile: BM = 256 (one M = 128, N = 256 MMA per 16-k slice, the weight tile as A in
-// TMEM, the x tile as B) or TT_SWAP = 32 for small batches (one M = 128, N = 32 MMA per slice, the
-// weight tile as A in shared memory), whose two accumulators are 32 TMEM columns each.
+// TT is the token tile: BM = 256 (one accumulator of 256 columns) or TT_SMALL = 32 (two of 32); the
+// A ring of the dequantised weight tiles follows the accumulators in TMEM.
 __host__ __device__ constexpr int a_bytes(int tt) { return tt * BK * 2; }  // the fp16 x tile
-__host__ __device__ constexpr int b_bytes(int tt) { return tt == BM ? 0 : B_BYTES; }  // weight tile in smem
-__host__ __device__ constexpr uint32_t tmem_cols(int tt) { return tt == BM ? 512u : 64u; }
-constexpr uint32_t TA_ACOL0 = BM;       // TT = 256: A stage s at TMEM columns 256 + 32 s
-constexpr uint32_t TA_ACOLS = BK / 2;   // 64 fp16 per row = 32 columns
+__host__ __device__ constexpr uint32_t tmem_cols(int tt) { return tt == BM ? 512u : 256u; }
+__host__ __device__ constexpr int num_acc(int tt) { return tt == BM ? 1 : 2; }
+__host__ __device__ constexpr uint32_t ta_acol0(int tt) { return (uint32_t)(num_acc(tt) * tt); }
+constexpr uint32_t TA_ACOLS = BK / 2;   // an A stage: 64 fp16 per row = 32 columns
 constexpr int STAGES_MAX_TA = 6;
 
 // Stages of the ring: as many as fit, up to six (TT = 256: six A stages of 32 columns fit beside the
@@ -89,7 +85,7 @@ constexpr int STAGES_MAX_TA = 6;
 constexpr int NUM_BARS_PER_STAGE = 3;  // tma_full, b_full, empty
 constexpr int NUM_BARS_FIXED = 5;      // acc_full[2], acc_empty[2], final
 __host__ __device__ constexpr int stage_bytes(int fmt, int bits, int tt) {
-  return a_bytes(tt) + b_bytes(tt) + p_bytes(fmt, bits);
+  return a_bytes(tt) + p_bytes(fmt, bits);
 }
 __host__ __device__ constexpr int meta_bytes(int fmt) { return fmt == FMT_INT4 ? MSLOTS * META_SLOT_BYTES : 0; }
 __host__ __device__ constexpr int meta_bars(int fmt) { return fmt == FMT_INT4 ? 2 * MSLOTS : 0; }
@@ -107,11 +103,8 @@ __host__ __device__ constexpr int stages(int fmt, int bits, int tt) {
 
 // byte offsets inside the dynamic shared memory (base aligned to 1024)
 __host__ __device__ constexpr int off_a(int tt, int s) { return s * a_bytes(tt); }
-__host__ __device__ constexpr int off_b(int fmt, int bits, int tt, int s) {
-  return stages(fmt, bits, tt) * a_bytes(tt) + s * b_bytes(tt);
-}
 __host__ __device__ constexpr int off_p(int fmt, int bits, int tt, int s) {
-  return stages(fmt, bits, tt) * (a_bytes(tt) + b_bytes(tt)) + s * p_bytes(fmt, bits);
+  return stages(fmt, bits, tt) * a_bytes(tt) + s * p_bytes(fmt, bits);
 }
 __host__ __device__ constexpr int off_meta(int fmt, int bits, int tt, int s) {
   return stages(fmt, bits, tt) * stage_bytes(fmt, bits, tt) + s * META_SLOT_BYTES;
@@ -291,15 +284,16 @@ template <int FMT, int BITS, int TT>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_codes,
                 Params p) {
-  constexpr bool SWAP = TT != BM;  // else the weight tile is the MMA's A operand in TMEM
-  constexpr int NACC = SWAP ? 2 : 1;  // accumulators in TMEM
+  constexpr int NACC = num_acc(TT);  // accumulators in TMEM
+  constexpr uint32_t A_COL0 = ta_acol0(TT);
   // dequantising warps per stage: TT = 256 alternates stages between two groups of four
-  constexpr int DEQ_PER_STAGE = SWAP ? NUM_DEQ_WARPS : NUM_DEQ_WARPS / 2;
-  static_assert(SWAP || TA_ACOL0 + STAGES_MAX_TA * TA_ACOLS <= 512, "A ring beside the accumulator");
+  constexpr int DEQ_PER_STAGE = NUM_DEQ_WARPS / 2;
+
   constexpr int PROW = p_row_bytes(FMT, BITS);
   constexpr int STAGES = stages(FMT, BITS, TT);
   constexpr uint32_t STAGE_TX = a_bytes(TT) + p_bytes(FMT, BITS);
   constexpr uint32_t TMEM_COLS = tmem_cols(TT);
+  static_assert(A_COL0 + STAGES * TA_ACOLS <= TMEM_COLS, "A ring beside the accumulators");
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -443,17 +437,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           tc_fence_after();
           const uint64_t xdesc = umma_desc_k_sw128(sbase + off_a(TT, s));
-          if constexpr (SWAP) {
-            const uint64_t wdesc = umma_desc_k_sw128(sbase + off_b(FMT, BITS, TT, s));
+          const uint32_t a_tmem = tmem_base + A_COL0 + (uint32_t)s * TA_ACOLS;  // lanes 0..127
 #pragma unroll
-            for (int kk = 0; kk < BK / 16; ++kk)  // advance 16 fp16 = 32 bytes = 2 descriptor units
-              umma_f16(d_tmem, wdesc + 2 * kk, xdesc + 2 * kk, idesc, (kb | kk) != 0);
-          } else {
-            const uint32_t a_tmem = tmem_base + TA_ACOL0 + (uint32_t)s * TA_ACOLS;  // lanes 0..127
-#pragma unroll
-            for (int kk = 0; kk < BK / 16; ++kk)  // 16 fp16 = 8 TMEM columns; 32 bytes = 2 descriptor units
-              umma_f16_tmem_a(d_tmem, a_tmem + 8 * kk, xdesc + 2 * kk, idesc, (kb | kk) != 0);
-          }
+          for (int kk = 0; kk < BK / 16; ++kk)  // 16 fp16 = 8 TMEM columns; 32 bytes = 2 descriptor units
+            umma_f16_tmem_a(d_tmem, a_tmem + 8 * kk, xdesc + 2 * kk, idesc, (kb | kk) != 0);
           umma_commit(bar_empty(s));
           issued = true;
           step_ring(s, ph, STAGES);
@@ -572,176 +559,112 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else if (warp >= WARP_DEQ0) {
     auto row_scale = [&](int64_t n) { return n < p.N ? p.ws.wsc[n] : 0.f; };
-    if constexpr (SWAP) {
-    const int t = threadIdx.x - WARP_DEQ0 * 32;  // 0..255
-    const int h = t & 1;                          // which 32-weight half of the 64-k stage
-    const int r = t >> 1;                         // the tile row this thread fills
-    Cursor nxt = cursor0();  // the stage after the current one
-    advance(nxt);
-    int s = 0, ms = 0;
-    uint32_t ph = 0, phm = 0;
-    uint32_t gm = 0, st = 0;
-    float sc = 0.f;
-    if (total_it > 0) {
-      const int64_t n_tile = cursor0().n_tile;
-      if constexpr (FMT != FMT_INT4) load_meta<FMT>(p, n_tile * BN + r, h, gm, st);
-      sc = row_scale(n_tile * BN + r);
-    }
-    uint8_t *row = smem + (r >> 3) * 1024 + (r & 7) * 128;  // + off_b(stage)
-    for (int64_t it = 0; it < total_it; ++it) {
-      uint32_t ngm = 0, nst = 0;
-      float nsc = sc;
-      if (it + 1 < total_it) {  // the next stage's metadata (int6, affine) and row scale
-        const int64_t n = nxt.n_tile * BN + r;
-        if constexpr (FMT != FMT_INT4) load_meta<FMT>(p, n, (int64_t)nxt.kb * (BK / 32) + h, ngm, nst);
-        if (nxt.kb == 0) nsc = row_scale(n);
+    // Stages alternate between warps 8-11 (even) and 12-15 (odd).  A thread fills one whole tile
+    // row (64 weights, both 32-weight chunks) of its stage into TMEM lane r = its warp's lane
+    // quarter + lane, columns A_COL0 + 32 s ..: the A operand of that stage's MMAs.
+    const int wd = warp - WARP_DEQ0;     // 0..7
+    const int g = wd >> 2;               // stages it = g, g + 2, ...
+    const int r = 32 * (wd & 3) + lane;  // tile row
+    const uint32_t t_row = tmem_base + ((uint32_t)(32 * (wd & 3)) << 16) + A_COL0;
+    auto step2 = [](int &slot, uint32_t &phase, int depth) {
+      slot += 2;
+      if (slot >= depth) {
+        slot -= depth;
+        phase ^= 1u;
       }
-      advance(nxt);
+    };
+    Cursor cur = cursor0();
+    if (g) advance(cur);
+    int s = g, ms = 0;  // both groups visit every super-block's slot
+    uint32_t ph = 0, phm = 0;
+    uint32_t gm[2] = {0, 0}, st[2] = {0, 0};
+    float sc = 0.f;
+    if (g < total_it) {
+      if constexpr (FMT != FMT_INT4) {
+        load_meta<FMT>(p, cur.n_tile * BN + r, (int64_t)cur.kb * 2, gm[0], st[0]);
+        load_meta<FMT>(p, cur.n_tile * BN + r, (int64_t)cur.kb * 2 + 1, gm[1], st[1]);
+      }
+      sc = row_scale(cur.n_tile * BN + r);
+    }
+    for (int64_t it = g; it < total_it; it += 2) {
+      Cursor nx = cur;  // this group's next stage
+      advance(nx);
+      advance(nx);
+      uint32_t ngm[2] = {0, 0}, nst[2] = {0, 0};
+      float nsc = sc;
+      if (it + 2 < total_it) {  // its metadata (int6, affine) and row scale, loaded ahead
+        const int64_t n = nx.n_tile * BN + r;
+        if constexpr (FMT != FMT_INT4) {
+          load_meta<FMT>(p, n, (int64_t)nx.kb * 2, ngm[0], nst[0]);
+          load_meta<FMT>(p, n, (int64_t)nx.kb * 2 + 1, ngm[1], nst[1]);
+        }
+        if (nx.n_tile != cur.n_tile) nsc = row_scale(n);
+      }
       if constexpr (FMT == FMT_INT4) {  // this stage's group and step words, from the metadata ring
-        const int q = (int)(it & 3);      // stage of the super-block
-        if (q == 0 && !mbar_wait_bounded(bar_meta_full(ms), phm, abort_flag)) break;
+        const int q = (int)(it & 3);  // stage of the super-block: this group sees q = g and g + 2
+        if (q == g && !__all_sync(0xffffffffu, mbar_wait_bounded(bar_meta_full(ms), phm, abort_flag))) break;
         const uint8_t *slot = smem + off_meta(FMT, BITS, TT, ms);
-        gm = (*reinterpret_cast<const uint32_t *>(slot + r * 16 + 4 * q) >> (16 * h)) & 0xffffu;
-        st = *reinterpret_cast<const uint32_t *>(slot + BN * 16 + r * 4);
-        if (q == 3) {  // the super-block's last stage: release the slot
+        const uint32_t w = *reinterpret_cast<const uint32_t *>(slot + r * 16 + 4 * q);
+        gm[0] = w & 0xffffu;
+        gm[1] = w >> 16;
+        st[0] = st[1] = *reinterpret_cast<const uint32_t *>(slot + BN * 16 + r * 4);
+        if (q == g + 2) {  // this group's last stage of the super-block: release the slot
           __syncwarp();
-          if ((t & 31) == 0) mbar_arrive(bar_meta_empty(ms));
+          if (lane == 0) mbar_arrive(bar_meta_empty(ms));
           step_ring(ms, phm, MSLOTS);
         }
       }
-      if (!mbar_wait_bounded(bar_tma_full(s), ph, abort_flag)) break;
-      const uint8_t *src = smem + off_p(FMT, BITS, TT, s) + r * PROW + h * (PROW / 2);
-      const uint8_t *src_hi = nullptr;
-      if constexpr (FMT == FMT_INT6P) {  // boxes [2 low halves][BN rows][16 B], then [BN rows][16 B] high
-        src = smem + off_p(FMT, BITS, TT, s) + h * 16 * BN + r * 16;
-        src_hi = smem + off_p(FMT, BITS, TT, s) + 32 * BN + r * 16 + 8 * h;
-      }
-      uint32_t cw[code_bits(FMT, BITS)];
-      if constexpr (FMT == FMT_INT4 || FMT == FMT_AFFINE) load_code_words<FMT, BITS>(src, cw);
-      uint32_t o[16];
-      chunk_to_f16<FMT, BITS>(cw, src, src_hi, gm, st, sc, o);
-      uint8_t *dst_row = row + off_b(FMT, BITS, TT, s);
+      // the codes have landed, and the MMAs that last read this A stage have completed (they
+      // released the stage before TMA refilled it)
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar_tma_full(s), ph, abort_flag))) break;
+      tc_fence_after();
+      const uint8_t *prow = smem + off_p(FMT, BITS, TT, s) + r * PROW;
+      uint32_t o[32];
+      if constexpr (PROW == 32 && (FMT == FMT_INT4 || FMT == FMT_AFFINE)) {
+        // the row's two 16-byte chunks, read in the order (h ^ bit 2 of r) so that the 32 lanes'
+        // first reads cover all 32 banks in four wavefronts (rows are 32 bytes apart)
+        const int sw = (r >> 2) & 1;
+        const uint4 va = reinterpret_cast<const uint4 *>(prow)[sw];
+        const uint4 vb = reinterpret_cast<const uint4 *>(prow)[sw ^ 1];
+        const uint4 c0 = sw ? vb : va, c1 = sw ? va : vb;
+        const uint32_t cw0[4] = {c0.x, c0.y, c0.z, c0.w}, cw1[4] = {c1.x, c1.y, c1.z, c1.w};
+        uint32_t o0[16], o1[16];
+        chunk_to_f16<FMT, BITS>(cw0, nullptr, nullptr, gm[0], st[0], sc, o0);
+        chunk_to_f16<FMT, BITS>(cw1, nullptr, nullptr, gm[1], st[1], sc, o1);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int j = 4 * h + q;  // logical 16-byte chunk of the 128-byte row
-        *reinterpret_cast<uint4 *>(dst_row + ((j ^ (r & 7)) << 4)) = make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+        for (int i = 0; i < 16; ++i) {
+          o[i] = o0[i];
+          o[16 + i] = o1[i];
+        }
+      } else {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint8_t *src = prow + h * (PROW / 2);
+          const uint8_t *src_hi = nullptr;
+          if constexpr (FMT == FMT_INT6P) {
+            src = smem + off_p(FMT, BITS, TT, s) + h * 16 * BN + r * 16;
+            src_hi = smem + off_p(FMT, BITS, TT, s) + 32 * BN + r * 16 + 8 * h;
+          }
+          uint32_t cw[code_bits(FMT, BITS)];
+          if constexpr (FMT == FMT_INT4 || FMT == FMT_AFFINE) load_code_words<FMT, BITS>(src, cw);
+          uint32_t oh[16];
+          chunk_to_f16<FMT, BITS>(cw, src, src_hi, gm[h], st[h], sc, oh);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) o[16 * h + i] = oh[i];
+        }
       }
-      fence_proxy_async_smem();
+      tmem_st_32x32b_x32(t_row + (uint32_t)s * TA_ACOLS, o);
+      tmem_st_wait();
+      tc_fence_before();
       __syncwarp();
-      if ((t & 31) == 0) mbar_arrive(bar_b_full(s));
-      step_ring(s, ph, STAGES);
-      gm = ngm;
-      st = nst;
+      if (lane == 0) mbar_arrive(bar_b_full(s));
+      step2(s, ph, STAGES);
+      cur = nx;
       sc = nsc;
-    }
-    } else {
-      // Stages alternate between warps 8-11 (even) and 12-15 (odd).  A thread fills one whole tile
-      // row (64 weights, both 32-weight chunks) of its stage into TMEM lane r = its warp's lane
-      // quarter + lane, columns TA_ACOL0 + 32 s ..: the A operand of that stage's MMAs.
-      const int wd = warp - WARP_DEQ0;     // 0..7
-      const int g = wd >> 2;               // stages it = g, g + 2, ...
-      const int r = 32 * (wd & 3) + lane;  // tile row
-      const uint32_t t_row = tmem_base + ((uint32_t)(32 * (wd & 3)) << 16) + TA_ACOL0;
-      auto step2 = [](int &slot, uint32_t &phase, int depth) {
-        slot += 2;
-        if (slot >= depth) {
-          slot -= depth;
-          phase ^= 1u;
-        }
-      };
-      Cursor cur = cursor0();
-      if (g) advance(cur);
-      int s = g, ms = 0;  // both groups visit every super-block's slot
-      uint32_t ph = 0, phm = 0;
-      uint32_t gm[2] = {0, 0}, st[2] = {0, 0};
-      float sc = 0.f;
-      if (g < total_it) {
-        if constexpr (FMT != FMT_INT4) {
-          load_meta<FMT>(p, cur.n_tile * BN + r, (int64_t)cur.kb * 2, gm[0], st[0]);
-          load_meta<FMT>(p, cur.n_tile * BN + r, (int64_t)cur.kb * 2 + 1, gm[1], st[1]);
-        }
-        sc = row_scale(cur.n_tile * BN + r);
-      }
-      for (int64_t it = g; it < total_it; it += 2) {
-        Cursor nx = cur;  // this group's next stage
-        advance(nx);
-        advance(nx);
-        uint32_t ngm[2] = {0, 0}, nst[2] = {0, 0};
-        float nsc = sc;
-        if (it + 2 < total_it) {  // its metadata (int6, affine) and row scale, loaded ahead
-          const int64_t n = nx.n_tile * BN + r;
-          if constexpr (FMT != FMT_INT4) {
-            load_meta<FMT>(p, n, (int64_t)nx.kb * 2, ngm[0], nst[0]);
-            load_meta<FMT>(p, n, (int64_t)nx.kb * 2 + 1, ngm[1], nst[1]);
-          }
-          if (nx.n_tile != cur.n_tile) nsc = row_scale(n);
-        }
-        if constexpr (FMT == FMT_INT4) {  // this stage's group and step words, from the metadata ring
-          const int q = (int)(it & 3);  // stage of the super-block: this group sees q = g and g + 2
-          if (q == g && !__all_sync(0xffffffffu, mbar_wait_bounded(bar_meta_full(ms), phm, abort_flag))) break;
-          const uint8_t *slot = smem + off_meta(FMT, BITS, TT, ms);
-          const uint32_t w = *reinterpret_cast<const uint32_t *>(slot + r * 16 + 4 * q);
-          gm[0] = w & 0xffffu;
-          gm[1] = w >> 16;
-          st[0] = st[1] = *reinterpret_cast<const uint32_t *>(slot + BN * 16 + r * 4);
-          if (q == g + 2) {  // this group's last stage of the super-block: release the slot
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar_meta_empty(ms));
-            step_ring(ms, phm, MSLOTS);
-          }
-        }
-        // the codes have landed, and the MMAs that last read this A stage have completed (they
-        // released the stage before TMA refilled it)
-        if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar_tma_full(s), ph, abort_flag))) break;
-        tc_fence_after();
-        const uint8_t *prow = smem + off_p(FMT, BITS, TT, s) + r * PROW;
-        uint32_t o[32];
-        if constexpr (PROW == 32 && (FMT == FMT_INT4 || FMT == FMT_AFFINE)) {
-          // the row's two 16-byte chunks, read in the order (h ^ bit 2 of r) so that the 32 lanes'
-          // first reads cover all 32 banks in four wavefronts (rows are 32 bytes apart)
-          const int sw = (r >> 2) & 1;
-          const uint4 va = reinterpret_cast<const uint4 *>(prow)[sw];
-          const uint4 vb = reinterpret_cast<const uint4 *>(prow)[sw ^ 1];
-          const uint4 c0 = sw ? vb : va, c1 = sw ? va : vb;
-          const uint32_t cw0[4] = {c0.x, c0.y, c0.z, c0.w}, cw1[4] = {c1.x, c1.y, c1.z, c1.w};
-          uint32_t o0[16], o1[16];
-          chunk_to_f16<FMT, BITS>(cw0, nullptr, nullptr, gm[0], st[0], sc, o0);
-          chunk_to_f16<FMT, BITS>(cw1, nullptr, nullptr, gm[1], st[1], sc, o1);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            o[i] = o0[i];
-            o[16 + i] = o1[i];
-          }
-        } else {
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const uint8_t *src = prow + h * (PROW / 2);
-            const uint8_t *src_hi = nullptr;
-            if constexpr (FMT == FMT_INT6P) {
-              src = smem + off_p(FMT, BITS, TT, s) + h * 16 * BN + r * 16;
-              src_hi = smem + off_p(FMT, BITS, TT, s) + 32 * BN + r * 16 + 8 * h;
-            }
-            uint32_t cw[code_bits(FMT, BITS)];
-            if constexpr (FMT == FMT_INT4 || FMT == FMT_AFFINE) load_code_words<FMT, BITS>(src, cw);
-            uint32_t oh[16];
-            chunk_to_f16<FMT, BITS>(cw, src, src_hi, gm[h], st[h], sc, oh);
-#pragma unroll
-            for (int i = 0; i < 16; ++i) o[16 * h + i] = oh[i];
-          }
-        }
-        tmem_st_32x32b_x32(t_row + (uint32_t)s * TA_ACOLS, o);
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar_b_full(s));
-        step2(s, ph, STAGES);
-        cur = nx;
-        sc = nsc;
-        gm[0] = ngm[0];
-        gm[1] = ngm[1];
-        st[0] = nst[0];
-        st[1] = nst[1];
-      }
+      gm[0] = ngm[0];
+      gm[1] = ngm[1];
+      st[0] = nst[0];
+      st[1] = nst[1];
     }
   }
 

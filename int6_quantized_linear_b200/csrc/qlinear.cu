@@ -210,12 +210,12 @@ ql_status launch_gemm_tt(const ql_desc *d, const ql_packed_const *w, const void 
   return launched();
 }
 
-// Up to 32 tokens: the swapped form (weights as the M = 128 operand, the tokens as N = 32), so no MMA
-// runs on padding rows; from 33 tokens: tiles of 256 tokens x 128 weight rows.
+// Up to 32 tokens: tiles of 32 tokens (MMA N = 32), so no MMA runs on padding tokens; from 33 tokens:
+// tiles of 256 tokens.  Both take 128 weight rows as the MMA's M = 128 operand.
 template <int FMT, int BITS>
 ql_status launch_gemm(const ql_desc *d, const ql_packed_const *w, const void *x, int64_t M, const void *bias,
                       void *y, void *workspace, cudaStream_t st, int sms) {
-  if (M <= gemm::TT_SWAP) return launch_gemm_tt<FMT, BITS, gemm::TT_SWAP>(d, w, x, M, bias, y, workspace, st, sms);
+  if (M <= gemm::TT_SMALL) return launch_gemm_tt<FMT, BITS, gemm::TT_SMALL>(d, w, x, M, bias, y, workspace, st, sms);
   return launch_gemm_tt<FMT, BITS, gemm::BM>(d, w, x, M, bias, y, workspace, st, sms);
 }
 
