@@ -206,7 +206,7 @@ ql_status launch_gemm_tt(const ql_desc *d, const ql_packed_const *w, const void 
   }
   const int64_t tiles = ((M + TT - 1) / TT) * ((N + BN - 1) / BN);
   const int grid = (int)(tiles < sms ? tiles : sms);
-  kern<<<grid, NUM_THREADS, smem, st>>>(mx, mc, p);
+  kern<<<grid, num_threads(TT), smem, st>>>(mx, mc, p);
   return launched();
 }
 
