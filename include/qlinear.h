@@ -306,8 +306,9 @@ ql_status qlinear_gemm_workspace_bytes(const ql_desc *desc, int64_t M, size_t *b
  * the row's max |x| in [2^15, 2^16) and stored as fp16 in the workspace
  * (exact for every value within 2^29 of the row maximum); (2) each weight
  * row gets a power of two 2^b_n from a metadata bound on its max |w|;
- * (3) the persistent GEMM (tiles of 256 tokens x 128 weight rows) dequantises
- * each weight once per tile into fp16 -- int4 as q * S' - Z * S' in packed
+ * (3) the persistent GEMM (tiles of 128 weight rows x 256 tokens, or x 32
+ * tokens up to M = 32) dequantises each weight once per tile into fp16, into
+ * tensor memory as the MMA's A operand -- int4 as q * S' - Z * S' in packed
  * halves with S' = S * 2^b_n, int6 / affine as the exact binary32 value times
  * 2^b_n rounded once -- contracts with fp32 accumulation in tensor memory,
  * and stores RN_bf16(acc * 2^-a_m * 2^-b_n).  fp16 operands rather than
