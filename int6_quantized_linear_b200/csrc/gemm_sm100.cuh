@@ -422,39 +422,56 @@ __global__ void __launch_bounds__(num_threads(TT), 1)
     }
   } else if (warp == WARP_MMA) {
     if (lane == 0) {
-      // D[weight row][token] += W tile (A, M = 128) x x tile (B, N = TT)
+      // D[weight row][token] += W tile (A, M = 128) x x tile (B, N = TT).  This one thread sets the
+      // kernel's pace, so its loop is unrolled over the ring's slots: slot j's x-tile descriptor
+      // and A columns are compile-time offsets from slot 0's, and the phase flips once a ring cycle.
       constexpr uint32_t idesc = umma_idesc_f16_f32(BN, TT);
-      int64_t tcount = 0;
-      int s = 0;
-      uint32_t ph = 0;
+      constexpr uint32_t XDESC_STEP = (uint32_t)(a_bytes(TT) >> 4);  // descriptor address units
+      const uint64_t xdesc0 = umma_desc_k_sw128(sbase + off_a(TT, 0));
+      const uint32_t a_tmem0 = tmem_base + A_COL0;
+      int64_t tcount = 0, tile = blockIdx.x;
+      int kb = 0;  // stage within the current tile
+      uint32_t ph = 0, d_tmem = tmem_base;
       bool ok = true, issued = false;
-      for (int64_t tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++tcount) {
+      // start a tile: its accumulator must have been drained (bounded wait)
+      auto begin_tile = [&]() {
         const int a = (int)(tcount % NACC);
         const uint32_t ause = (uint32_t)(tcount / NACC);
-        if (!mbar_wait_bounded(bar_acc_empty(a), (ause & 1) ^ 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait_bounded(bar_acc_empty(a), (ause & 1) ^ 1, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + (uint32_t)(a * TT);  // accumulator a: columns a * TT ..
-        for (int kb = 0; kb < num_kb; ++kb) {
-          // b_full alone: its arrivals come from dequantisers that waited for this stage's tma_full, so
-          // the x tile has landed before the MMAs read it (and a copy that never lands ends their
-          // wait, and so this one, by the abort flag).  One wait a stage fewer on this warp's path,
-          // which sets the pace (3.6 %).
-          if (!mbar_wait_bounded(bar_b_full(s), ph, abort_flag)) {
+        d_tmem = tmem_base + (uint32_t)(a * TT);  // accumulator a: columns a * TT ..
+        return true;
+      };
+      if (tile < num_tiles) ok = begin_tile();
+      while (ok && tile < num_tiles) {
+#pragma unroll
+        for (int j = 0; j < STAGES; ++j) {
+          if (!ok || tile >= num_tiles) break;
+          // b_full alone: its arrivals come from dequantisers that waited for this stage's tma_full,
+          // so the x tile has landed before the MMAs read it (and a copy that never lands ends their
+          // wait, and so this one, by the abort flag)
+          if (!mbar_wait_bounded(bar_b_full(j), ph, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint64_t xdesc = umma_desc_k_sw128(sbase + off_a(TT, s));
-          const uint32_t a_tmem = tmem_base + A_COL0 + (uint32_t)s * TA_ACOLS;  // lanes 0..127
+          const uint64_t xdesc = xdesc0 + (uint64_t)(j * XDESC_STEP);
+          const uint32_t a_tmem = a_tmem0 + (uint32_t)(j * TA_ACOLS);  // lanes 0..127
+          // 16 fp16 = 8 TMEM columns; 32 bytes = 2 descriptor units
+          umma_f16_tmem_a(d_tmem, a_tmem, xdesc, idesc, kb != 0);
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk)  // 16 fp16 = 8 TMEM columns; 32 bytes = 2 descriptor units
-            umma_f16_tmem_a(d_tmem, a_tmem + 8 * kk, xdesc + 2 * kk, idesc, (kb | kk) != 0);
-          umma_commit(bar_empty(s));
+          for (int kk = 1; kk < BK / 16; ++kk) umma_f16_tmem_a(d_tmem, a_tmem + 8 * kk, xdesc + 2 * kk, idesc, 1u);
+          umma_commit(bar_empty(j));
           issued = true;
-          step_ring(s, ph, STAGES);
+          if (++kb == num_kb) {  // the tile's last stage
+            kb = 0;
+            umma_commit(bar_acc_full((int)(tcount % NACC)));
+            tile += gridDim.x;
+            ++tcount;
+            if (tile < num_tiles) ok = begin_tile();
+          }
         }
-        if (!ok) break;
-        umma_commit(bar_acc_full(a));
+        ph ^= 1u;
       }
       if (issued) {  // all MMAs retired before teardown
         umma_commit(bar_final);
