@@ -8,10 +8,11 @@
 // write it into tensor memory (TMEM), where the MMAs of M = 128 (weight rows,
 // A read from TMEM) x N = TT (tokens, B = the x tile in shared memory) consume
 // it.  Shared memory then carries only the x tile (written once by TMA, read
-// once by the tensor core) and the packed codes, which is what bounds the
-// 256-token form: a shared-memory weight tile would add its store, and a second
-// token half would read it again, roughly doubling the bytes shared memory
-// moves per MMA.  Two token tiles:
+// once by the tensor core) and the packed codes: a shared-memory weight tile
+// would add its store, and a second token half would read it again, roughly
+// doubling the bytes shared memory moves per MMA.  Within a tile the pace is
+// set by the one thread that issues the MMAs (its per-stage waits, commits and
+// bookkeeping).  Two token tiles:
 //   TT = 256 (prefill): one M = 128, N = 256 MMA per 16-k slice.  The
 //     accumulator (128 lanes x 256 columns) and a ring of A stages (32 columns
 //     each) share the 512 TMEM columns, so there is one accumulator and the
@@ -28,10 +29,11 @@
 //               32*(w%4).., one weight row per lane), undo the two
 //               power-of-two scales (exponents added first), round to bf16,
 //               store y
-//   warps 8-15  dequantisers: packed codes + metadata -> weight times 2^b_n
-//               -> fp16.  Warps 8-11 fill even stages and 12-15 odd ones, one
-//               whole 64-weight tile row per thread, into the TMEM lanes of the
-//               warp's quarter.
+//   warps 8..    dequantisers: packed codes + metadata -> weight times 2^b_n
+//               -> fp16, one whole 64-weight tile row per thread, into the
+//               TMEM lanes of the warp's quarter.  Groups of four warps take
+//               the stages in turn: two groups (warps 8-15) at TT = 256, four
+//               (warps 8-23) at TT = 32.
 // The operands are fp16 rather than bf16 because rounding every weight to
 // bf16 costs ~1% of rms(y); fp16 costs ~0.1% (see gemm_prep.cuh for the
 // scaling that keeps fp32 range).  Loop state advances by counters: no
@@ -50,13 +52,13 @@ constexpr int BN = 128;  // weight rows per tile
 constexpr int BK = 64;
 constexpr int WARP_TMA = 0;
 constexpr int WARP_MMA = 1;
-constexpr int WARP_META0 = 2;    // int4: two warps copy each stage's group and step words ahead
+constexpr int WARP_META0 = 2;    // int4: two warps copy each super-block's group and step words ahead
 constexpr int NUM_META_WARPS = 2;
 constexpr int WARP_EPI0 = 4;
 constexpr int WARP_DEQ0 = 8;
 // dequantising warps: groups of four (one per TMEM lane quarter) take turns on the stages; the
 // 32-token form, whose MMAs are short, has four groups, the 256-token form two (its register budget)
-__host__ __device__ constexpr int deq_warps(int tt) { return tt == 256 ? 8 : 16; }
+__host__ __device__ constexpr int deq_warps(int tt) { return tt == BM ? 8 : 16; }
 __host__ __device__ constexpr int num_threads(int tt) { return (WARP_DEQ0 + deq_warps(tt)) * 32; }
 constexpr int TT_SMALL = 32;          // token tile for up to 32 tokens
 // int4 metadata ring: one slot per 256-weight super-block (four k-stages): [BN rows][16 bytes] of group
@@ -80,7 +82,6 @@ __host__ __device__ constexpr uint32_t tmem_cols(int tt) { return tt == BM ? 512
 __host__ __device__ constexpr int num_acc(int tt) { return tt == BM ? 1 : 2; }
 __host__ __device__ constexpr uint32_t ta_acol0(int tt) { return (uint32_t)(num_acc(tt) * tt); }
 constexpr uint32_t TA_ACOLS = BK / 2;   // an A stage: 64 fp16 per row = 32 columns
-constexpr int STAGES_MAX_TA = 6;
 
 // Stages of the ring: as many as fit, up to six (TT = 256: six A stages of 32 columns fit beside the
 // 256-column accumulator).  int4 adds the metadata ring [MSLOTS][META_SLOT_BYTES] and its barriers.
