@@ -298,6 +298,7 @@ __global__ void __launch_bounds__(num_threads(TT), 1)
   constexpr int STAGES = stages(FMT, BITS, TT);
   constexpr uint32_t STAGE_TX = a_bytes(TT) + p_bytes(FMT, BITS);
   constexpr uint32_t TMEM_COLS = tmem_cols(TT);
+  static_assert(NG < STAGES, "a group's step through the ring crosses its end at most once");
   static_assert(A_COL0 + STAGES * TA_ACOLS <= TMEM_COLS, "A ring beside the accumulators");
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
