@@ -118,6 +118,7 @@ __global__ void __launch_bounds__(X2F16_THREADS) x_to_f16_kernel(const __nv_bflo
   const int64_t m = blockIdx.x;
   const int64_t nv = K / 8;  // 16-byte vectors of the row
   const uint4 *row = reinterpret_cast<const uint4 *>(x + m * K);
+  if constexpr (!DEP) pdl_launch_dependents();  // the GEMM's weight-scale pass needs nothing from here
   if constexpr (DEP) {
     pdl_launch_dependents();
     if (m < M && tid < nv) prefetch_l2(row + tid);
@@ -165,11 +166,8 @@ __global__ void __launch_bounds__(X2F16_THREADS) x_to_f16_kernel(const __nv_bflo
 // max-reduction), pick b_n.  The grid covers the rows up to N rounded to 256: rows past N get
 // scale 0 and exponent 0, so the padded columns of a tile are defined (and never stored).
 template <int FMT, int BITS>
-__global__ void __launch_bounds__(256) w_scale_kernel(const uint8_t *gmeta, const uint8_t *steps, int64_t N,
-                                                       int64_t K, int G, GemmWorkspace ws) {
-  const int lane = threadIdx.x & 31;
-  const int64_t n = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
-  if (n >= (int64_t)padded_rows(N)) return;  // whole warps leave together
+__device__ __forceinline__ void w_scale_row(const uint8_t *gmeta, const uint8_t *steps, int64_t N, int64_t K,
+                                            int G, GemmWorkspace ws, int64_t n, int lane) {
   if (n >= N) {
     if (lane == 0) {
       ws.wsc[n] = 0.f;
@@ -212,6 +210,19 @@ __global__ void __launch_bounds__(256) w_scale_kernel(const uint8_t *gmeta, cons
     ws.wsc[n] = exp2i(e);
     ws.wexp[n] = -e;
   }
+}
+
+// Launched as a programmatic dependent of the GEMM's x pass: it reads only the weights' metadata, so it
+// runs alongside that pass, and waits for it before exiting -- the GEMM, a programmatic dependent of
+// this kernel, then finds both passes' results complete.
+template <int FMT, int BITS>
+__global__ void __launch_bounds__(256) w_scale_kernel(const uint8_t *gmeta, const uint8_t *steps, int64_t N,
+                                                       int64_t K, int G, GemmWorkspace ws) {
+  pdl_launch_dependents();
+  const int lane = threadIdx.x & 31;
+  const int64_t n = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+  if (n < (int64_t)padded_rows(N)) w_scale_row<FMT, BITS>(gmeta, steps, N, K, G, ws, n, lane);
+  pdl_wait();
 }
 
 }  // namespace ql

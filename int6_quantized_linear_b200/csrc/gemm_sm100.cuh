@@ -380,6 +380,9 @@ __global__ void __launch_bounds__(num_threads(TT), 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  // launched as a programmatic dependent of the weight-scale pass (which waits for the x pass): the
+  // set-up above overlapped them; the workspace they write is read only from here on
+  pdl_wait();
 
   if (warp == WARP_TMA) {
     if (lane == 0) {

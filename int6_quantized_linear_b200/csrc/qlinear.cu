@@ -175,9 +175,24 @@ ql_status launch_gemm_tt(const ql_desc *d, const ql_packed_const *w, const void 
   const uint64_t row_bytes = (uint64_t)K * code_bits(FMT, BITS) / 8;
   const GemmWorkspace ws = gemm_workspace_carve(workspace, M, N, K);
   // pass 1: scaled fp16 activations; pass 2: per-row weight scales
+  // the weight-scale pass and the GEMM are programmatic dependents: each starts while the kernel before
+  // it drains (the scale pass needs nothing from the x pass and waits for it only before exiting; the
+  // GEMM waits after its set-up)
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
   x_to_f16_kernel<false><<<(unsigned)M, X2F16_THREADS, 0, st>>>(static_cast<const __nv_bfloat16 *>(x), M, K, ws);
-  w_scale_kernel<FMT, BITS><<<(int)(((int64_t)padded_rows(N) * 32 + 255) / 256), 256, 0, st>>>(
-      static_cast<const uint8_t *>(w->gmeta), static_cast<const uint8_t *>(w->steps), N, K, d->group, ws);
+  {
+    cudaLaunchConfig_t wc = {};
+    wc.gridDim = dim3((unsigned)(((int64_t)padded_rows(N) * 32 + 255) / 256));
+    wc.blockDim = dim3(256);
+    wc.stream = st;
+    wc.attrs = pdl;
+    wc.numAttrs = 1;
+    if (cudaLaunchKernelEx(&wc, w_scale_kernel<FMT, BITS>, static_cast<const uint8_t *>(w->gmeta),
+                           static_cast<const uint8_t *>(w->steps), N, K, d->group, ws) != cudaSuccess)
+      return cuda_failed();
+  }
   CUtensorMap mx, mc;
   if (!encode_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws.x16, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, BK, TT,
                  CU_TENSOR_MAP_SWIZZLE_128B))
@@ -206,7 +221,14 @@ ql_status launch_gemm_tt(const ql_desc *d, const ql_packed_const *w, const void 
   }
   const int64_t tiles = ((M + TT - 1) / TT) * ((N + BN - 1) / BN);
   const int grid = (int)(tiles < sms ? tiles : sms);
-  kern<<<grid, num_threads(TT), smem, st>>>(mx, mc, p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(num_threads(TT));
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, mx, mc, p) != cudaSuccess) return cuda_failed();
   return launched();
 }
 
