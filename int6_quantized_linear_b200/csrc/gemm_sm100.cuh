@@ -56,10 +56,12 @@ constexpr int WARP_META0 = 2;    // int4: two warps copy each super-block's grou
 constexpr int NUM_META_WARPS = 2;
 constexpr int WARP_EPI0 = 4;
 constexpr int WARP_DEQ0 = 8;
-// dequantising warps: groups of four (one per TMEM lane quarter) take turns on the stages; the
-// 32-token form, whose MMAs are short, has four groups, the 256-token form two (its register budget)
-__host__ __device__ constexpr int deq_warps(int tt) { return tt == BM ? 8 : 16; }
-__host__ __device__ constexpr int num_threads(int tt) { return (WARP_DEQ0 + deq_warps(tt)) * 32; }
+// dequantising warps: groups of four (one per TMEM lane quarter) take turns on the stages.  CPS is the
+// CTAs resident per SM.  The 32-token form, whose MMAs are short and whose pace is its stage chain, has
+// four groups at one CTA an SM, or two at two CTAs an SM (a layer with more 128-row tiles than SMs
+// then runs every tile at once); the 256-token form has two (its register budget).
+__host__ __device__ constexpr int deq_warps(int tt, int cps = 1) { return tt == BM || cps == 2 ? 8 : 16; }
+__host__ __device__ constexpr int num_threads(int tt, int cps = 1) { return (WARP_DEQ0 + deq_warps(tt, cps)) * 32; }
 constexpr int TT_SMALL = 32;          // token tile for up to 32 tokens
 // int4 metadata ring: one slot per 256-weight super-block (four k-stages): [BN rows][16 bytes] of group
 // words (the u32 of stage kb holds its two 32-weight groups), then [BN rows][4 bytes] of step words.
@@ -283,14 +285,15 @@ QL_DEVI void chunk_to_f16(const uint32_t (&cw)[code_bits(FMT, BITS)], const uint
   }
 }
 
-template <int FMT, int BITS, int TT>
-__global__ void __launch_bounds__(num_threads(TT), 1)
+template <int FMT, int BITS, int TT, int CPS = 1>
+__global__ void __launch_bounds__(num_threads(TT, CPS), CPS)
     gemm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_codes,
                 Params p) {
   constexpr int NACC = num_acc(TT);  // accumulators in TMEM
   constexpr uint32_t A_COL0 = ta_acol0(TT);
   // dequantising warps per stage: TT = 256 alternates stages between two groups of four
-  constexpr int DEQ_WARPS = deq_warps(TT), NG = DEQ_WARPS / 4;  // dequantiser groups
+  static_assert(CPS == 1 || (CPS == 2 && TT != BM), "two CTAs an SM: the 32-token form only");
+  constexpr int DEQ_WARPS = deq_warps(TT, CPS), NG = DEQ_WARPS / 4;  // dequantiser groups
   constexpr int DEQ_PER_STAGE = 4;                                   // one group fills a stage
   static_assert(NG >= 1 && 4 % NG == 0, "groups take whole turns within a super-block");
 

@@ -167,7 +167,7 @@ bool encode_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint6
   return true;
 }
 
-template <int FMT, int BITS, int TT>
+template <int FMT, int BITS, int TT, int CPS = 1>
 ql_status launch_gemm_tt(const ql_desc *d, const ql_packed_const *w, const void *x, int64_t M, const void *bias,
                          void *y, void *workspace, cudaStream_t st, int sms) {
   using namespace ql::gemm;
@@ -210,7 +210,7 @@ ql_status launch_gemm_tt(const ql_desc *d, const ql_packed_const *w, const void 
   p.y = static_cast<__nv_bfloat16 *>(y);
   p.ws = ws;
   const int smem = smem_bytes(FMT, BITS, TT);
-  auto kern = gemm_kernel<FMT, BITS, TT>;
+  auto kern = gemm_kernel<FMT, BITS, TT, CPS>;
   static thread_local int configured_dev = -1;  // per (kernel instantiation, thread)
   int dev = 0;
   cudaGetDevice(&dev);
@@ -220,10 +220,11 @@ ql_status launch_gemm_tt(const ql_desc *d, const ql_packed_const *w, const void 
     configured_dev = dev;
   }
   const int64_t tiles = ((M + TT - 1) / TT) * ((N + BN - 1) / BN);
-  const int grid = (int)(tiles < sms ? tiles : sms);
+  const int slots = CPS * sms;
+  const int grid = (int)(tiles < slots ? tiles : slots);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid);
-  cfg.blockDim = dim3(num_threads(TT));
+  cfg.blockDim = dim3(num_threads(TT, CPS));
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cfg.attrs = pdl;
@@ -232,12 +233,18 @@ ql_status launch_gemm_tt(const ql_desc *d, const ql_packed_const *w, const void 
   return launched();
 }
 
-// Up to 32 tokens: tiles of 32 tokens (MMA N = 32), so no MMA runs on padding tokens; from 33 tokens:
-// tiles of 256 tokens.  Both take 128 weight rows as the MMA's M = 128 operand.
+// Up to 32 tokens: tiles of 32 tokens (MMA N = 32), so no MMA runs on padding tokens -- two CTAs an SM
+// when the layer has more 128-row tiles than SMs (every tile then runs at once instead of some SMs
+// taking two in turn); from 33 tokens: tiles of 256 tokens.  Both take 128 weight rows as the MMA's
+// M = 128 operand.
 template <int FMT, int BITS>
 ql_status launch_gemm(const ql_desc *d, const ql_packed_const *w, const void *x, int64_t M, const void *bias,
                       void *y, void *workspace, cudaStream_t st, int sms) {
-  if (M <= gemm::TT_SMALL) return launch_gemm_tt<FMT, BITS, gemm::TT_SMALL>(d, w, x, M, bias, y, workspace, st, sms);
+  if (M <= gemm::TT_SMALL) {
+    if ((d->N + gemm::BN - 1) / gemm::BN > sms)
+      return launch_gemm_tt<FMT, BITS, gemm::TT_SMALL, 2>(d, w, x, M, bias, y, workspace, st, sms);
+    return launch_gemm_tt<FMT, BITS, gemm::TT_SMALL>(d, w, x, M, bias, y, workspace, st, sms);
+  }
   return launch_gemm_tt<FMT, BITS, gemm::BM>(d, w, x, M, bias, y, workspace, st, sms);
 }
 
